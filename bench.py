@@ -1,0 +1,480 @@
+#!/usr/bin/env python
+"""Benchmark of the 4-bit MoE expert-layer numerics on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one pass of the whole hot path over one batch: routing, NVFP4
+quantisation of tokens and expert weights, NVFP4 dispatch, the two NVFP4
+grouped GEMMs with SwiGLU and combine, then the backward: MXFP8 quantisation of
+the gradients, stochastic requantisation of the saved weights and activations,
+MXFP8 dgrad and wgrad grouped GEMMs, SwiGLU backward and un-permute.  The
+workload is the 384-expert layer (top-8 of 32768 tokens, d_model 4096, d_ff
+1024, Zipf(1.2) loads with 8 empty experts, Student-t(3) activations), synthetic
+and seeded.  The step's working set (~40 GB) is far larger than L2, so no
+flush is needed between steps.
+
+Multi-GPU: one process per GPU; every rank runs its own replica of the step on
+its own tokens (no collective on the data path: weak scaling).  Times are the
+max over ranks of CUDA-event device time.
+
+`value` is the NVFP4 grouped-GEMM throughput (both forward GEMMs, flops over
+true routed rows) in TFLOP/s, measured inside the timed steps.  The line also
+carries the per-stage breakdown, the quantiser bandwidth on the 16384x4096
+quantiser stream, the roofline of the dominant kernel, clocks, the end-to-end
+number through host buffers, and the CPU oracle baseline.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "moe_layer"
+QUANT_WORKLOAD = "quant_stream"
+METRIC = "NVFP4 grouped expert GEMM TFLOPS (% of B200 FP4 peak); quantiser GB/s (% HBM)"
+UNIT = "TFLOP/s"
+NOMINAL_NVFP4_TFLOPS = 9000.0
+NOMINAL_MXFP8_TFLOPS = 4500.0
+NOMINAL_HBM_GBS = 8000.0
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sus=d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                    src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+# --------------------------------------------------------------------------
+# clocks sampled during the timed region
+# --------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(f[1]), smax=float(f[2]), power=float(f[3]),
+                                 hw=f[5], hwt=f[6], swt=f[7], pcap=f[8]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no nvidia-smi samples"], "samples": 0}
+        loaded = [r for r in rows if r["power"] > 300] or rows
+        reasons = set()
+        for r in loaded:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"), ("swt", "sw_thermal_slowdown"),
+                              ("pcap", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in loaded), "sm_max_mhz": max(r["smax"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(loaded)}
+
+
+# --------------------------------------------------------------------------
+# distributed plumbing
+# --------------------------------------------------------------------------
+def dist_setup(n_gpus):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+        pg = dist
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return rank, world, local, pg
+
+
+def barrier(pg):
+    if pg is not None:
+        pg.barrier()
+
+
+def max_over_ranks(pg, values, device):
+    """Element-wise max of a list of floats over ranks."""
+    if pg is None:
+        return list(values)
+    import torch
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return t.tolist()
+
+
+def sum_over_ranks(pg, values, device):
+    if pg is None:
+        return list(values)
+    import torch
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.SUM)
+    return t.tolist()
+
+
+# --------------------------------------------------------------------------
+# algorithmic work per stage (bytes read+written once, flops over true rows)
+# --------------------------------------------------------------------------
+def stage_work(c, counts, M_pad):
+    T, k, E, D, F = c["T"], c["k"], c["E"], c["D"], c["F"]
+    N1 = 2 * F if c["gated"] else F
+    R = T * k                                       # true routed rows
+    nv = lambda rows, cols: rows * cols * (0.5 + 1 / 16) + rows * 4          # NVFP4 bytes (+ outer)
+    mx = lambda rows, cols: rows * cols * (1 + 1 / 32)                       # MXFP8 bytes
+    f_g1 = 2 * R * N1 * D
+    f_g2 = 2 * R * D * F
+    w = {
+        # name: (kind, work)  kind: "tensor4" / "tensor8" flops, "hbm" bytes
+        "quant_x": ("hbm", T * D * 2 + nv(T, D)),
+        "gather": ("hbm", 2 * nv(R, D)),
+        "quant_w": ("hbm", E * N1 * D * 2 + nv(E * N1, D) + E * D * F * 2 + nv(E * D, F)),
+        "gemm1": ("tensor4", f_g1),
+        "swiglu": ("hbm", R * N1 * 2 + R * F * 2),
+        "quant_a": ("hbm", R * F * 2 + nv(R, F)),
+        "gemm2": ("tensor4", f_g2),
+        "combine": ("hbm", R * D * 2 + T * D * 2),
+        "dispatch_grad": ("hbm", T * D * 2 + R * D * 2),
+        "quant_dy2": ("hbm", R * D * 2 + 2 * mx(R, D)),
+        "requant_w2": ("hbm", nv(E * D, F) + mx(E * D, F)),
+        "dgrad2": ("tensor8", 2 * R * F * D),
+        "requant_a": ("hbm", nv(R, F) + mx(R, F)),
+        "wgrad2": ("tensor8", 2 * R * D * F),
+        "swiglu_bwd": ("hbm", R * N1 * 2 + R * F * 2 + R * N1 * 2),
+        "quant_dh1": ("hbm", R * N1 * 2 + 2 * mx(R, N1)),
+        "requant_w1": ("hbm", nv(E * N1, D) + mx(E * N1, D)),
+        "dgrad1": ("tensor8", 2 * R * D * N1),
+        "requant_x": ("hbm", nv(R, D) + mx(R, D)),
+        "wgrad1": ("tensor8", 2 * R * N1 * D),
+        "unpermute": ("hbm", R * D * 2 + T * D * 2),
+    }
+    return w
+
+
+# launches of this library's kernels per step (ExpertLayer call sequence):
+# route 4, quant_x 1, gather 1, quant_w 2x3, gemm1 1, swiglu 1, quant_a 1,
+# gemm2 1, combine 1, then 13 single-kernel backward stages
+LAUNCHES_PER_STEP = 4 + 1 + 1 + 6 + 1 + 1 + 1 + 1 + 1 + 13
+
+
+def run_ours(args):
+    import torch
+    from fp8_moe_numerics_b200 import api, workloads
+    from fp8_moe_numerics_b200.layer import ExpertLayer
+
+    rank, world, local, pg = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    peaks = load_peaks()
+    c = workloads.CONFIGS[WORKLOAD]
+    # each rank draws its own tokens (weak scaling); weights are shared seeds
+    inp = workloads.layer_inputs(WORKLOAD, device=dev)
+    if rank:
+        g = torch.Generator(device=dev)
+        g.manual_seed(c["seed"] + 17 * rank)
+        inp["x"] = workloads.activations(c["T"], c["D"], c["x_dist"], c["seed"] + 1 + 1000 * rank, dev)
+    topk = inp["topk"].to(dev)
+    counts = torch.bincount(inp["topk"].reshape(-1).long(), minlength=c["E"]).tolist()
+    M_pad = sum((x + 127) // 128 * 128 for x in counts)
+    layer = ExpertLayer(inp["x"], topk, inp["w_comb"].to(dev), inp["w1"], inp["w2"], inp["dout"], gated=c["gated"],
+                        seed=1234)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        layer.step()
+    api.sync_status()
+    torch.cuda.synchronize()
+
+    # ---------------------------------------------------------------- timed
+    layer.reset_marks()
+    barrier(pg)
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(args.steps):
+            layer.step(record=True)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier(pg)
+    api.sync_status()
+    total_ms = t0.elapsed_time(t1)
+    stages = layer.stage_times_ms()
+    work = stage_work(c, counts, M_pad)
+    names = list(work)
+    stage_ms = [stages.get(n, 0.0) for n in names]
+    maxed = max_over_ranks(pg, [total_ms] + stage_ms, dev)
+    total_ms, stage_ms = maxed[0], dict(zip(names, maxed[1:]))
+    K = args.steps
+    gemm_flops = (work["gemm1"][1] + work["gemm2"][1]) * K
+    nvfp4_ms = stage_ms["gemm1"] + stage_ms["gemm2"]
+    value = world * gemm_flops / (nvfp4_ms * 1e-3) / 1e12
+
+    # roofline of the dominant kernel
+    dom = max(names, key=lambda n: stage_ms[n])
+    kind, wk = work[dom]
+    per_launch_ms = stage_ms[dom] / K
+    if kind == "hbm":
+        achieved = wk / (per_launch_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm"], 4), "traffic": None, "kernel": dom,
+                "peak_source": peaks["src"] + " copy bandwidth"}
+    else:
+        ratio = 4 if kind == "tensor4" else 2
+        peak = peaks["bf16_sus"] * ratio
+        achieved = wk / (per_launch_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4), "traffic": None, "kernel": dom,
+                "peak_source": f"{peaks['src']} sustained bf16 x {ratio} (nominal dense ratio)"}
+    breakdown = {}
+    for n in names:
+        kind, wk = work[n]
+        t = stage_ms[n] / K
+        if kind == "hbm":
+            breakdown[n] = {"ms": round(t, 4), "GB/s": round(wk / (t * 1e-3) / 1e9, 1) if t > 0 else None,
+                            "frac_hbm": round(wk / (t * 1e-3) / 1e9 / peaks["hbm"], 3) if t > 0 else None}
+        else:
+            ratio = 4 if kind == "tensor4" else 2
+            tf = wk / (t * 1e-3) / 1e12 if t > 0 else None
+            breakdown[n] = {"ms": round(t, 4), "TFLOP/s": round(tf, 1) if tf else None,
+                            "frac_nominal": round(tf / (NOMINAL_NVFP4_TFLOPS if ratio == 4 else NOMINAL_MXFP8_TFLOPS), 3)
+                            if tf else None,
+                            "frac_measured": round(tf / (peaks["bf16_sus"] * ratio), 3) if tf else None}
+
+    quant = quantiser_stream(dev, peaks) if rank == 0 else None
+
+    # ---------------------------------------------------------------- e2e
+    e2e = e2e_leg(layer, inp, dev, args, gemm_flops / K, pg, world)
+
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(total_ms / K, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "nvfp4/mxfp8 (fp32 accumulate), bf16 i/o", "data": "synthetic",
+        "config": {"workload": f"{WORKLOAD}: 384 experts, top-8 of 32768 tokens (262144 routed rows, "
+                               f"{M_pad} padded), d_model 4096, d_ff 1024 SwiGLU, Zipf(1.2) loads with 8 empty "
+                               "experts, t(3) activations; NVFP4 forward + MXFP8-SR backward",
+                   "parallelism": f"replicas x{world} (one per GPU, no data-path collective)",
+                   "l2": "per-step working set ~40 GB >> 126 MB L2 (no flush needed)",
+                   "seed": c["seed"], "sr_rbits": 8},
+        "nvfp4_gemm": {"tflops": round(value / world, 1), "frac_of_9pf_nominal": round(value / world / NOMINAL_NVFP4_TFLOPS, 4),
+                       "frac_of_measured": round(value / world / (peaks["bf16_sus"] * 4), 4),
+                       "peak_measured_basis": f"{peaks['src']} bf16 sustained {peaks['bf16_sus']} x4"},
+        "stages": breakdown,
+        "quantiser": quant,
+        "roofline": roof,
+        "clocks": clk.summary(),
+        "e2e": e2e,
+        "gpu_launches": LAUNCHES_PER_STEP * K,
+        "impl": "ours",
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(inp, layer, seconds=args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.destroy_process_group()
+
+
+def quantiser_stream(dev, peaks, reps: int = 20):
+    """NVFP4 quantise + MXFP8 stochastic requantise-transpose of the
+    16384x4096 Student-t(4) stream; L2 flushed before every launch."""
+    import torch
+    from fp8_moe_numerics_b200 import api, workloads
+    c = workloads.CONFIGS[QUANT_WORKLOAD]
+    rows, cols = c["rows"], c["cols"]
+    x = workloads.activations(rows, cols, c["x_dist"], c["seed"], dev)
+    q = api.nvfp4_quantize(x, 1, api.MX_SF_MMA)
+    t = api.mxfp8_requant_transpose_sr(*q, rows, cols, 1, api.MX_SF_MMA, None, c["sr_seed"], 0, 8, api.MX_SF_MMA)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    res = {}
+    for name, fn, nbytes in (
+            ("nvfp4_quantize", lambda: api.nvfp4_quantize(x, 1, api.MX_SF_MMA, out=q),
+             rows * cols * 2 + rows * cols * (0.5 + 1 / 16) + rows * 4),
+            ("mxfp8_requant_transpose_sr", lambda: api.mxfp8_requant_transpose_sr(
+                *q, rows, cols, 1, api.MX_SF_MMA, None, c["sr_seed"], 0, 8, api.MX_SF_MMA, out=t),
+             rows * cols * (0.5 + 1 / 16) + rows * 4 + rows * cols * (1 + 1 / 32))):
+        for _ in range(3):
+            fn()
+        ms = []
+        for _ in range(reps):
+            flush.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ms.append(a.elapsed_time(b))
+        med = statistics.median(ms)
+        gbs = nbytes / (med * 1e-3) / 1e9
+        res[name] = {"us": round(med * 1e3, 2), "GB/s": round(gbs, 1), "frac_hbm_measured": round(gbs / peaks["hbm"], 3),
+                     "frac_hbm_8tbs": round(gbs / NOMINAL_HBM_GBS, 3), "bytes": int(nbytes)}
+    res["workload"] = "quant_stream: bf16 16384x4096 Student-t(4) x 10^U(-3,3) per row; L2 flushed per launch"
+    return res
+
+
+def e2e_leg(layer, inp, dev, args, flops_per_step, pg, world):
+    """Same metric through the public API with host buffers: every step copies
+    its inputs (tokens, routing, combine weights, upstream gradient) from
+    pinned host memory and reads the layer output and input gradient back."""
+    import torch
+    hx = inp["x"].cpu().pin_memory()
+    htopk = inp["topk"].cpu().pin_memory()
+    hw = inp["w_comb"].cpu().pin_memory()
+    hd = inp["dout"].cpu().pin_memory()
+    hout = torch.empty(layer.out.shape, dtype=layer.out.dtype).pin_memory()
+    hdx = torch.empty(layer.dx.shape, dtype=layer.dx.dtype).pin_memory()
+    h2d = hx.numel() * 2 + htopk.numel() * 4 + hw.numel() * 4 + hd.numel() * 2
+    d2h = hout.numel() * 2 + hdx.numel() * 2
+
+    def one():
+        layer.x.copy_(hx, non_blocking=True)
+        layer.topk.copy_(htopk, non_blocking=True)
+        layer.w_comb.copy_(hw, non_blocking=True)
+        layer.dout.copy_(hd, non_blocking=True)
+        layer.step()
+        hout.copy_(layer.out, non_blocking=True)
+        hdx.copy_(layer.dx, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    barrier(pg)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    n = max(1, min(args.steps, 5))
+    a.record()
+    for _ in range(n):
+        one()
+    b.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(pg, [a.elapsed_time(b) / n], dev)[0]
+    return {"value": round(world * flops_per_step / (ms * 1e-3) / 1e12, 1), "unit": UNIT,
+            "ms_per_step": round(ms, 3), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "note": "NVFP4 GEMM flops per step / whole step time including pinned-host copies"}
+
+
+def cpu_baseline(inp, layer, seconds: float = 15.0):
+    """The oracle, as it stands, on the host cores: NVFP4-quantise a sample of
+    token rows and expert-weight rows and run the fp64 grouped GEMM of those
+    rows against one expert's W1 tile, until ~`seconds` of CPU work."""
+    import numpy as np
+    import oracle
+    x = inp["x"][:256].cpu().view(np.int16) if False else inp["x"][:256].cpu().view(__import__("torch").int16).numpy().view(np.uint16)
+    w = inp["w1"][0, :256].cpu().view(__import__("torch").int16).numpy().view(np.uint16)
+    D = x.shape[1]
+    N = w.shape[0]
+    flops = 0
+    t0 = time.perf_counter()
+    it = 0
+    while time.perf_counter() - t0 < seconds or it == 0:
+        a = oracle.nvfp4_quantize(x)
+        b = oracle.nvfp4_quantize(w, group_rows=N)
+        seg = np.array([0, x.shape[0]], np.int64)
+        oracle.grouped_gemm_nvfp4(*a, *b, seg, N)
+        flops += 2 * x.shape[0] * N * D
+        it += 1
+    dt = time.perf_counter() - t0
+    return {"value": round(flops / dt / 1e12, 6), "unit": UNIT, "cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"{it} x (NVFP4 quantise 256x{D} tokens + 256x{D} rows of W1[0], fp64 GEMM 256x{N}x{D})",
+            "seconds": round(dt, 2)}
+
+
+def run_reference(args):
+    """Reference arm: the CPU oracle timed on the host cores (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    import numpy as np
+    import torch
+    import oracle
+    from fp8_moe_numerics_b200 import workloads
+    c = workloads.CONFIGS[WORKLOAD]
+    D, F = c["D"], c["F"]
+    x = workloads.activations(256, D, c["x_dist"], c["seed"] + 1).view(torch.int16).numpy().view(np.uint16)
+    w = workloads.weights(1, 2 * F, D, c["w_std"], c["seed"] + 2)[0, :256].view(torch.int16).numpy().view(np.uint16)
+    seg = np.array([0, 256], np.int64)
+    per = 2 * 256 * 256 * D
+
+    def step():
+        a = oracle.nvfp4_quantize(x)
+        b = oracle.nvfp4_quantize(w, group_rows=256)
+        oracle.grouped_gemm_nvfp4(*a, *b, seg, 256)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    v = per * args.steps / dt / 1e12
+    line = {"metric": METRIC, "value": round(v, 6), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic",
+            "config": {"workload": f"{WORKLOAD} (bounded sample: 256 token rows x 256 W1 rows, d_model {D})"},
+            "impl": "reference",
+            "cpu_baseline": {"value": round(v, 6), "unit": UNIT, "cores": os.cpu_count(), "kind": "oracle",
+                             "sample": "per step: NVFP4-quantise 256x4096 tokens and 256x4096 W1 rows, fp64 GEMM"},
+            "e2e": {"value": round(v, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

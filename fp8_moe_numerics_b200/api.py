@@ -1,0 +1,198 @@
+"""Python binding of the mxmoe C ABI (include/mxmoe.h).
+
+Argument marshalling only: each function allocates its outputs with torch on
+the inputs' CUDA device, passes raw device pointers and the current CUDA
+stream to the library, and raises MxError on a non-MX_OK status.  Every
+computation happens in the library's sm_100a kernels.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib as L
+from ._lib import (MX_GEMM_DGRAD, MX_GEMM_WGRAD, MX_OUT_BF16, MX_OUT_F32, MX_ROUND_RNE, MX_ROUND_SR,
+                   MX_SF_MMA, MX_SF_ROWMAJOR, MxError)
+
+__all__ = [
+    "MX_SF_ROWMAJOR", "MX_SF_MMA", "MX_ROUND_RNE", "MX_ROUND_SR", "MX_GEMM_DGRAD", "MX_GEMM_WGRAD", "MxError",
+    "sf_bytes", "sync_status", "nvfp4_quantize", "mxfp8_requant_transpose_sr", "mxfp8_quantize",
+    "grouped_gemm_nvfp4", "grouped_gemm_mxfp8", "moe_route", "nvfp4_gather_rows", "swiglu_fwd", "swiglu_bwd",
+    "moe_combine", "moe_dispatch_grad",
+]
+
+
+def _p(t) -> ctypes.c_void_p:
+    if t is None:
+        return ctypes.c_void_p(0)
+    if not t.is_cuda:
+        raise ValueError("mxmoe operates on CUDA tensors")
+    if not t.is_contiguous():
+        raise ValueError("mxmoe expects contiguous tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _s() -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _u8(n: int, dev) -> torch.Tensor:
+    return torch.empty(int(n), dtype=torch.uint8, device=dev)
+
+
+def sf_bytes(rows: int, cols: int, block: int, layout: int) -> int:
+    n = L.lib().mx_sf_bytes(rows, cols, block, layout)
+    if n == 0 and rows * cols > 0:
+        raise ValueError(f"scale shape {rows}x{cols}/{block} not allowed for layout {layout}")
+    return n
+
+
+def sync_status(stream=None) -> None:
+    s = ctypes.c_void_p((stream or torch.cuda.current_stream()).cuda_stream)
+    st = L.lib().mx_sync_status(s)
+    if st != L.MX_OK:
+        raise MxError("mx_sync_status", st, L.lib().mx_last_cuda_error())
+
+
+def nvfp4_quantize(x: torch.Tensor, group_rows: int = 1, sf_layout: int = MX_SF_MMA, out=None):
+    """bf16 [rows, cols] -> (codes u8 [rows, cols/2], sf u8, outer f32 [rows/group_rows])."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2
+    rows, cols = x.shape
+    dev = x.device
+    if out is None:
+        out = (torch.empty(rows, cols // 2, dtype=torch.uint8, device=dev),
+               _u8(sf_bytes(rows, cols, 16, sf_layout), dev),
+               torch.empty(rows // group_rows, dtype=torch.float32, device=dev))
+    codes, sf, outer = out
+    L.call("nvfp4_quantize", _p(x), rows, cols, group_rows, _p(codes), _p(sf), _p(outer), sf_layout, _s())
+    return codes, sf, outer
+
+
+def mxfp8_requant_transpose_sr(codes, sf, outer, rows: int, cols: int, group_rows: int = 1,
+                               in_sf_layout: int = MX_SF_MMA, rows_valid=None, seed: int = 0, stream_id: int = 0,
+                               rbits: int = 8, out_sf_layout: int = MX_SF_MMA, out=None):
+    """Saved NVFP4 [rows, cols] -> MXFP8 [cols, rows] codes and E8M0 scales."""
+    dev = codes.device
+    if out is None:
+        out = (torch.empty(cols, rows, dtype=torch.uint8, device=dev), _u8(sf_bytes(cols, rows, 32, out_sf_layout), dev))
+    oc, oe = out
+    L.call("mxfp8_requant_transpose_sr", _p(codes), _p(sf), _p(outer), rows, cols, group_rows, in_sf_layout,
+           _p(rows_valid), ctypes.c_uint64(seed), ctypes.c_uint64(stream_id), rbits, _p(oc), _p(oe),
+           out_sf_layout, _s())
+    return oc, oe
+
+
+def mxfp8_quantize(x: torch.Tensor, row: bool = True, col: bool = True, rounding: int = MX_ROUND_RNE,
+                   seed: int = 0, stream_id: int = 0, rbits: int = 8, rows_valid=None,
+                   sf_layout: int = MX_SF_MMA, out=None):
+    """bf16 [rows, cols] -> (row codes [rows, cols], row E8M0, col codes [cols, rows], col E8M0);
+    the forms not requested are None."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2
+    rows, cols = x.shape
+    dev = x.device
+    if out is None:
+        out = (torch.empty(rows, cols, dtype=torch.uint8, device=dev) if row else None,
+               _u8(sf_bytes(rows, cols, 32, sf_layout), dev) if row else None,
+               torch.empty(cols, rows, dtype=torch.uint8, device=dev) if col else None,
+               _u8(sf_bytes(cols, rows, 32, sf_layout), dev) if col else None)
+    rc, re, cc, ce = out
+    L.call("mxfp8_quantize", _p(x), rows, cols, rounding, ctypes.c_uint64(seed), ctypes.c_uint64(stream_id), rbits,
+           _p(rows_valid), _p(rc), _p(re), _p(cc), _p(ce), sf_layout, _s())
+    return rc, re, cc, ce
+
+
+def _out_code(dtype) -> int:
+    if dtype == torch.float32:
+        return MX_OUT_F32
+    if dtype == torch.bfloat16:
+        return MX_OUT_BF16
+    raise ValueError(dtype)
+
+
+def grouped_gemm_nvfp4(a, b, seg: torch.Tensor, E: int, N: int, K: int, out_dtype=torch.bfloat16, out=None):
+    """a = (codes [M_cap, K/2], sf, outer [M_cap]); b = (codes [E*N, K/2], sf, outer [E]).
+    Returns out [M_cap, N]; rows >= seg[E] are not written."""
+    M_cap = a[0].shape[0]
+    if out is None:
+        out = torch.empty(M_cap, N, dtype=out_dtype, device=a[0].device)
+    L.call("grouped_gemm_nvfp4", _p(a[0]), _p(a[1]), _p(a[2]), _p(b[0]), _p(b[1]), _p(b[2]), _p(seg), E, M_cap, N,
+           K, _p(out), _out_code(out.dtype), _s())
+    return out
+
+
+def grouped_gemm_mxfp8(mode: int, a_codes, a_e8m0, b_codes, b_e8m0, seg: torch.Tensor, E: int, M_cap: int, N: int,
+                       K: int, out_dtype=torch.bfloat16, out=None):
+    """DGRAD: A [M_cap, K], B [N, E*K] -> out [M_cap, N].
+    WGRAD: A [N, M_cap], B [K, M_cap] -> out [E, N, K]."""
+    if out is None:
+        shape = (M_cap, N) if mode == MX_GEMM_DGRAD else (E, N, K)
+        out = torch.empty(*shape, dtype=out_dtype, device=a_codes.device)
+    L.call("grouped_gemm_mxfp8", mode, _p(a_codes), _p(a_e8m0), _p(b_codes), _p(b_e8m0), _p(seg), E, M_cap, N, K,
+           _p(out), _out_code(out.dtype), _s())
+    return out
+
+
+def max_routed_rows(T: int, k: int, E: int) -> int:
+    cap = T * k + 127 * E
+    return (cap + 127) // 128 * 128
+
+
+def moe_route(topk: torch.Tensor, E: int, M_cap: int | None = None, out=None):
+    """topk int32 [T, k] -> (seg int64 [E+1], src int32 [M_cap], pos int32 [T, k])."""
+    T, k = topk.shape
+    dev = topk.device
+    if M_cap is None:
+        M_cap = max_routed_rows(T, k, E)
+    ws_bytes = L.lib().mx_route_workspace_bytes(T, E)
+    if out is None:
+        out = (torch.empty(E + 1, dtype=torch.int64, device=dev), torch.empty(M_cap, dtype=torch.int32, device=dev),
+               torch.empty(T, k, dtype=torch.int32, device=dev), _u8(max(ws_bytes, 16), dev))
+    seg, src, pos, ws = out
+    L.call("moe_route", _p(topk), T, k, E, M_cap, _p(seg), _p(src), _p(pos), _p(ws), ws.numel(), _s())
+    return seg, src, pos
+
+
+def nvfp4_gather_rows(codes, sf_rowmajor, outer, src: torch.Tensor, k: int, cols: int, out=None):
+    M_cap = src.shape[0]
+    dev = codes.device
+    if out is None:
+        out = (torch.empty(M_cap, cols // 2, dtype=torch.uint8, device=dev), _u8(sf_bytes(M_cap, cols, 16, MX_SF_MMA), dev),
+               torch.empty(M_cap, dtype=torch.float32, device=dev))
+    oc, osf, oo = out
+    L.call("nvfp4_gather_rows", _p(codes), _p(sf_rowmajor), _p(outer), _p(src), k, M_cap, cols, _p(oc), _p(osf),
+           _p(oo), _s())
+    return oc, osf, oo
+
+
+def swiglu_fwd(h: torch.Tensor, F: int, gated: bool = True, rows_valid=None, out=None):
+    rows = h.shape[0]
+    if out is None:
+        out = torch.empty(rows, F, dtype=torch.bfloat16, device=h.device)
+    L.call("swiglu_fwd", _p(h), rows, F, int(gated), _p(rows_valid), _p(out), _s())
+    return out
+
+
+def swiglu_bwd(h: torch.Tensor, da: torch.Tensor, F: int, gated: bool = True, rows_valid=None, out=None):
+    rows = h.shape[0]
+    if out is None:
+        out = torch.empty_like(h)
+    L.call("swiglu_bwd", _p(h), _p(da), rows, F, int(gated), _p(rows_valid), _p(out), _s())
+    return out
+
+
+def moe_combine(y: torch.Tensor, pos: torch.Tensor, w, D: int, out=None):
+    T, k = pos.shape
+    if out is None:
+        out = torch.empty(T, D, dtype=torch.bfloat16, device=y.device)
+    L.call("moe_combine", _p(y), _p(pos), _p(w), T, k, D, _p(out), _s())
+    return out
+
+
+def moe_dispatch_grad(dout: torch.Tensor, src: torch.Tensor, w, k: int, out=None):
+    M_cap = src.shape[0]
+    D = dout.shape[1]
+    if out is None:
+        out = torch.empty(M_cap, D, dtype=torch.bfloat16, device=dout.device)
+    L.call("moe_dispatch_grad", _p(dout), _p(src), _p(w), k, M_cap, D, _p(out), _s())
+    return out

@@ -1,0 +1,53 @@
+// abi.cu -- status handling and size helpers of the mxmoe C ABI.
+#include "mx_common.cuh"
+
+namespace {
+thread_local int g_last_cuda_error = 0;
+constexpr int kMaxDevices = 64;
+int g_device_ok[kMaxDevices] = {0};   // 0 unknown, 1 sm_100, -1 other
+}  // namespace
+
+int mx_set_cuda_error(cudaError_t e) {
+    g_last_cuda_error = (int)e;
+    return MX_ECUDA;
+}
+
+int mx_launch_status(void) {
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? MX_OK : mx_set_cuda_error(e);
+}
+
+int mx_check_device(void) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return mx_set_cuda_error(e);
+    if (dev >= 0 && dev < kMaxDevices && g_device_ok[dev]) return g_device_ok[dev] > 0 ? MX_OK : MX_EUNSUPPORTED;
+    int major = 0, minor = 0;
+    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess)
+        return mx_set_cuda_error(e);
+    const bool ok = major == 10 && minor == 0;
+    if (dev >= 0 && dev < kMaxDevices) g_device_ok[dev] = ok ? 1 : -1;
+    return ok ? MX_OK : MX_EUNSUPPORTED;
+}
+
+extern "C" int mx_version(void) { return 1; }
+
+extern "C" int mx_last_cuda_error(void) { return g_last_cuda_error; }
+
+extern "C" size_t mx_sf_bytes(int64_t rows, int64_t cols, int block, int sf_layout) {
+    if (rows < 0 || cols <= 0 || (block != 16 && block != 32) || cols % block) return 0;
+    const int64_t S = cols / block;
+    if (sf_layout == MX_SF_ROWMAJOR) return (size_t)(rows * S);
+    if (sf_layout == MX_SF_MMA) {
+        if (rows % 128 || S % 4) return 0;
+        return (size_t)(rows * S);                  // atoms tile the array exactly
+    }
+    return 0;
+}
+
+extern "C" size_t mx_route_workspace_bytes(int64_t T, int64_t E) {
+    if (T < 0 || E <= 0) return 0;
+    const int64_t chunks = (T + 255) / 256;
+    return (size_t)((chunks * E + E) * sizeof(int32_t));
+}

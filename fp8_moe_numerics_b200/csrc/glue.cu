@@ -1,0 +1,316 @@
+// glue.cu -- expert-layer glue around the quantisers and GEMMs: routing
+// permutation, NVFP4 dispatch gather, SiLU / SwiGLU, combine and its gradient.
+//
+// [ai-primer] "Inkling 2 Small uses four-bit training...", §Quantized NVLink and
+// BBBK: tokens travel to their routed experts in NVFP4 and the backward pass
+// reuses the quantised forward activations -- here the per-token NVFP4 rows are
+// quantised once and gathered into expert-major order.
+#include "mx_common.cuh"
+
+namespace {
+
+constexpr int kChunk = 256;   // tokens per routing chunk
+
+// Per-chunk expert histogram: hist[c][e].
+__global__ void route_count_kernel(const int32_t* __restrict__ topk, int64_t T, int64_t k, int64_t E,
+                                   int32_t* __restrict__ hist) {
+    extern __shared__ int32_t h[];
+    for (int64_t e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
+    __syncthreads();
+    const int64_t t = (int64_t)blockIdx.x * kChunk + threadIdx.x;
+    if (t < T)
+        for (int64_t j = 0; j < k; ++j) atomicAdd(&h[topk[t * k + j]], 1);
+    __syncthreads();
+    for (int64_t e = threadIdx.x; e < E; e += blockDim.x) hist[(int64_t)blockIdx.x * E + e] = h[e];
+}
+
+// Totals, 128-padded exclusive scan into seg_offsets, and per-(chunk, expert)
+// base rows written back over hist.
+__global__ void route_scan_kernel(int32_t* __restrict__ hist, int32_t* __restrict__ counts, int64_t nchunks,
+                                  int64_t E, int64_t* __restrict__ seg) {
+    extern __shared__ int64_t start[];   // [E + 1]
+    for (int64_t e = threadIdx.x; e < E; e += blockDim.x) {
+        int64_t c = 0;
+        for (int64_t ch = 0; ch < nchunks; ++ch) c += hist[ch * E + e];
+        counts[e] = (int32_t)c;
+        start[e + 1] = (c + 127) / 128 * 128;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        start[0] = 0;
+        for (int64_t e = 0; e < E; ++e) start[e + 1] += start[e];
+    }
+    __syncthreads();
+    for (int64_t e = threadIdx.x; e <= E; e += blockDim.x) seg[e] = start[e];
+    for (int64_t e = threadIdx.x; e < E; e += blockDim.x) {
+        int64_t run = start[e];
+        for (int64_t ch = 0; ch < nchunks; ++ch) {
+            const int32_t c = hist[ch * E + e];
+            hist[ch * E + e] = (int32_t)run;
+            run += c;
+        }
+    }
+}
+
+// One warp per chunk: rows handed out in token order.  For each group of 32
+// tokens a shared bitmask per expert marks the lanes that chose it; a lane's
+// rank is the number of lower lanes in that mask.
+__global__ void route_scatter_kernel(const int32_t* __restrict__ topk, int64_t T, int64_t k, int64_t E,
+                                     const int32_t* __restrict__ base, int32_t* __restrict__ src,
+                                     int32_t* __restrict__ pos) {
+    extern __shared__ uint32_t sm[];
+    uint32_t* mask = sm;                                   // [E]
+    int32_t* run = reinterpret_cast<int32_t*>(sm + E);     // [E]
+    const int lane = threadIdx.x;
+    for (int64_t e = lane; e < E; e += 32) { mask[e] = 0; run[e] = base[(int64_t)blockIdx.x * E + e]; }
+    __syncwarp();
+    const uint32_t below = (1u << lane) - 1u;
+    for (int gi = 0; gi < kChunk / 32; ++gi) {
+        const int64_t t = (int64_t)blockIdx.x * kChunk + gi * 32 + lane;
+        const bool act = t < T;
+        if (act)
+            for (int64_t j = 0; j < k; ++j) atomicOr(&mask[topk[t * k + j]], 1u << lane);
+        __syncwarp();
+        if (act)
+            for (int64_t j = 0; j < k; ++j) {
+                const int32_t e = topk[t * k + j];
+                const int32_t p = run[e] + __popc(mask[e] & below);
+                pos[t * k + j] = p;
+                src[p] = (int32_t)(t * k + j);
+            }
+        __syncwarp();
+        if (act)
+            for (int64_t j = 0; j < k; ++j) {
+                const int32_t e = topk[t * k + j];
+                const uint32_t m = mask[e];
+                if ((m & below) == 0) { run[e] += __popc(m); mask[e] = 0; }
+            }
+        __syncwarp();
+    }
+}
+
+// src = -1 on each expert's padding rows and on rows >= seg[E].
+__global__ void route_pad_kernel(const int64_t* __restrict__ seg, const int32_t* __restrict__ counts, int64_t E,
+                                 int64_t M_cap, int32_t* __restrict__ src) {
+    const int64_t e = blockIdx.x;
+    int64_t a, b;
+    if (e < E) { a = seg[e] + counts[e]; b = seg[e + 1]; }
+    else { a = seg[E]; b = M_cap; }
+    for (int64_t p = a + threadIdx.x; p < b; p += blockDim.x) src[p] = -1;
+}
+
+// One warp per output row.
+__global__ void gather_rows_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sf,
+                                   const float* __restrict__ outer, const int32_t* __restrict__ src, int64_t k,
+                                   int64_t M_cap, int64_t cols, uint8_t* __restrict__ out_codes,
+                                   uint8_t* __restrict__ out_sf, float* __restrict__ out_outer) {
+    const int lane = threadIdx.x & 31;
+    const int64_t p = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (p >= M_cap) return;
+    const int32_t sidx = src[p];
+    const int64_t t = sidx < 0 ? -1 : sidx / k;
+    const int64_t n16 = cols / 32;                         // uint4 of codes per row
+    const uint4* ci = reinterpret_cast<const uint4*>(codes + (t < 0 ? 0 : t) * (cols / 2));
+    uint4* co = reinterpret_cast<uint4*>(out_codes + p * (cols / 2));
+    for (int64_t i = lane; i < n16; i += 32) co[i] = t < 0 ? make_uint4(0, 0, 0, 0) : __ldg(ci + i);
+    const int64_t S = cols / 16;
+    for (int64_t a = lane; a < S / 4; a += 32) {
+        const uint32_t v = t < 0 ? 0u : __ldg(reinterpret_cast<const uint32_t*>(sf + t * S) + a);
+        *reinterpret_cast<uint32_t*>(out_sf + sf_offset_mma(p, 4 * a, S)) = v;
+    }
+    if (lane == 0) out_outer[p] = t < 0 ? 0.0f : outer[t];
+}
+
+__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
+__device__ __forceinline__ float dsilu_f(float g) {
+    const float s = 1.0f / (1.0f + expf(-g));
+    return s * (1.0f + g * (1.0f - s));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// 8 outputs per thread.
+__global__ void swiglu_fwd_kernel(const uint16_t* __restrict__ h, int64_t rows, int64_t F, int gated,
+                                  const int64_t* rows_valid, uint16_t* __restrict__ a) {
+    const int64_t nv = F / 8;
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= rows * nv) return;
+    const int64_t r = i / nv, c = (i % nv) * 8;
+    uint4 o = make_uint4(0, 0, 0, 0);
+    if (r < load_rows_valid(rows_valid, rows)) {
+        const int64_t hw = gated ? 2 * F : F;
+        const uint4 gv = *reinterpret_cast<const uint4*>(h + r * hw + c);
+        const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+        uint32_t uw[4] = {0x3f803f80u, 0x3f803f80u, 0x3f803f80u, 0x3f803f80u};   // bf16 1.0
+        if (gated) {
+            const uint4 uv = *reinterpret_cast<const uint4*>(h + r * hw + F + c);
+            uw[0] = uv.x; uw[1] = uv.y; uw[2] = uv.z; uw[3] = uv.w;
+        }
+        uint32_t ow[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            ow[j] = pack_bf16x2(silu_f(bf16_lo(gw[j])) * bf16_lo(uw[j]), silu_f(bf16_hi(gw[j])) * bf16_hi(uw[j]));
+        o = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+    }
+    *reinterpret_cast<uint4*>(a + r * F + c) = o;
+}
+
+__global__ void swiglu_bwd_kernel(const uint16_t* __restrict__ h, const uint16_t* __restrict__ da, int64_t rows,
+                                  int64_t F, int gated, const int64_t* rows_valid, uint16_t* __restrict__ dh) {
+    const int64_t nv = F / 8;
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= rows * nv) return;
+    const int64_t r = i / nv, c = (i % nv) * 8;
+    const int64_t hw = gated ? 2 * F : F;
+    uint4 og = make_uint4(0, 0, 0, 0), ou = make_uint4(0, 0, 0, 0);
+    if (r < load_rows_valid(rows_valid, rows)) {
+        const uint4 gv = *reinterpret_cast<const uint4*>(h + r * hw + c);
+        const uint4 dv = *reinterpret_cast<const uint4*>(da + r * F + c);
+        const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w}, dw[4] = {dv.x, dv.y, dv.z, dv.w};
+        uint32_t uw[4] = {0x3f803f80u, 0x3f803f80u, 0x3f803f80u, 0x3f803f80u};
+        if (gated) {
+            const uint4 uv = *reinterpret_cast<const uint4*>(h + r * hw + F + c);
+            uw[0] = uv.x; uw[1] = uv.y; uw[2] = uv.z; uw[3] = uv.w;
+        }
+        uint32_t wg[4], wu[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float g0 = bf16_lo(gw[j]), g1 = bf16_hi(gw[j]);
+            const float d0 = bf16_lo(dw[j]), d1 = bf16_hi(dw[j]);
+            const float u0 = bf16_lo(uw[j]), u1 = bf16_hi(uw[j]);
+            wg[j] = pack_bf16x2(d0 * u0 * dsilu_f(g0), d1 * u1 * dsilu_f(g1));
+            wu[j] = pack_bf16x2(d0 * silu_f(g0), d1 * silu_f(g1));
+        }
+        og = make_uint4(wg[0], wg[1], wg[2], wg[3]);
+        ou = make_uint4(wu[0], wu[1], wu[2], wu[3]);
+    }
+    *reinterpret_cast<uint4*>(dh + r * hw + c) = og;
+    if (gated) *reinterpret_cast<uint4*>(dh + r * hw + F + c) = ou;
+}
+
+// One block per token; 8 bf16 per thread per step.
+__global__ void combine_kernel(const uint16_t* __restrict__ y, const int32_t* __restrict__ pos,
+                               const float* __restrict__ w, int64_t k, int64_t D, uint16_t* __restrict__ out) {
+    const int64_t t = blockIdx.x;
+    for (int64_t c = threadIdx.x * 8; c < D; c += blockDim.x * 8) {
+        float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        for (int64_t j = 0; j < k; ++j) {
+            const float wj = w ? w[t * k + j] : 1.0f;
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(y + (int64_t)pos[t * k + j] * D + c));
+            const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                acc[2 * q] += wj * bf16_lo(vw[q]);
+                acc[2 * q + 1] += wj * bf16_hi(vw[q]);
+            }
+        }
+        *reinterpret_cast<uint4*>(out + t * D + c) = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                                                                pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+    }
+}
+
+// One block per row of the expert-major buffer.
+__global__ void dispatch_grad_kernel(const uint16_t* __restrict__ dout, const int32_t* __restrict__ src,
+                                     const float* __restrict__ w, int64_t k, int64_t D, uint16_t* __restrict__ dy) {
+    const int64_t p = blockIdx.x;
+    const int32_t s = src[p];
+    const float wj = s < 0 ? 0.0f : (w ? w[s] : 1.0f);
+    const int64_t t = s < 0 ? 0 : s / k;
+    for (int64_t c = threadIdx.x * 8; c < D; c += blockDim.x * 8) {
+        uint4 o = make_uint4(0, 0, 0, 0);
+        if (s >= 0) {
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(dout + t * D + c));
+            o = make_uint4(pack_bf16x2(wj * bf16_lo(v.x), wj * bf16_hi(v.x)), pack_bf16x2(wj * bf16_lo(v.y), wj * bf16_hi(v.y)),
+                           pack_bf16x2(wj * bf16_lo(v.z), wj * bf16_hi(v.z)), pack_bf16x2(wj * bf16_lo(v.w), wj * bf16_hi(v.w)));
+        }
+        *reinterpret_cast<uint4*>(dy + p * D + c) = o;
+    }
+}
+
+}  // namespace
+
+extern "C" int moe_route(const int32_t* topk, int64_t T, int64_t k, int64_t E, int64_t M_cap, int64_t* seg_offsets,
+                         int32_t* src, int32_t* pos, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+    if (!topk || !seg_offsets || !src || !pos || T < 0 || k <= 0 || k > 32 || E <= 0 || M_cap < 0 || M_cap % 128)
+        return MX_EINVAL;
+    const int64_t need_rows = (T * k + 127 * E + 127) / 128 * 128;
+    if (M_cap < need_rows || !workspace || workspace_bytes < mx_route_workspace_bytes(T, E)) return MX_EINVAL;
+    if (T * k >= (int64_t)1 << 31 || E * 8 > 48 * 1024) return MX_EINVAL;
+    if (int st = mx_check_device()) return st;
+    const int64_t nchunks = (T + kChunk - 1) / kChunk;
+    int32_t* hist = static_cast<int32_t*>(workspace);
+    int32_t* counts = hist + nchunks * E;
+    if (nchunks > 0) {
+        route_count_kernel<<<(unsigned)nchunks, kChunk, E * sizeof(int32_t), stream>>>(topk, T, k, E, hist);
+    }
+    route_scan_kernel<<<1, 1024, (E + 1) * sizeof(int64_t), stream>>>(hist, counts, nchunks, E, seg_offsets);
+    if (nchunks > 0)
+        route_scatter_kernel<<<(unsigned)nchunks, 32, 2 * E * sizeof(uint32_t), stream>>>(topk, T, k, E, hist, src, pos);
+    route_pad_kernel<<<(unsigned)(E + 1), 256, 0, stream>>>(seg_offsets, counts, E, M_cap, src);
+    return mx_launch_status();
+}
+
+extern "C" int nvfp4_gather_rows(const uint8_t* codes, const uint8_t* sf, const float* outer, const int32_t* src,
+                                 int64_t k, int64_t M_cap, int64_t cols, uint8_t* out_codes, uint8_t* out_sf,
+                                 float* out_outer, cudaStream_t stream) {
+    if (!codes || !sf || !outer || !src || !out_codes || !out_sf || !out_outer || k <= 0 || M_cap < 0 ||
+        M_cap % 128 || cols <= 0 || cols % 64 || !mx_aligned(codes, 16) || !mx_aligned(out_codes, 16) ||
+        !mx_aligned(sf, 4) || !mx_aligned(out_sf, 4))
+        return MX_EINVAL;
+    if (int st = mx_check_device()) return st;
+    if (M_cap == 0) return MX_OK;
+    gather_rows_kernel<<<(unsigned)((M_cap + 7) / 8), 256, 0, stream>>>(codes, sf, outer, src, k, M_cap, cols,
+                                                                       out_codes, out_sf, out_outer);
+    return mx_launch_status();
+}
+
+extern "C" int swiglu_fwd(const void* h, int64_t rows, int64_t F, int gated, const int64_t* rows_valid, void* a,
+                          cudaStream_t stream) {
+    if (!h || !a || rows < 0 || F <= 0 || F % 8 || !mx_aligned(h, 16) || !mx_aligned(a, 16)) return MX_EINVAL;
+    if (int st = mx_check_device()) return st;
+    const int64_t n = rows * (F / 8);
+    if (n == 0) return MX_OK;
+    swiglu_fwd_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(static_cast<const uint16_t*>(h), rows, F,
+                                                                        gated, rows_valid, static_cast<uint16_t*>(a));
+    return mx_launch_status();
+}
+
+extern "C" int swiglu_bwd(const void* h, const void* da, int64_t rows, int64_t F, int gated, const int64_t* rows_valid,
+                          void* dh, cudaStream_t stream) {
+    if (!h || !da || !dh || rows < 0 || F <= 0 || F % 8 || !mx_aligned(h, 16) || !mx_aligned(da, 16) ||
+        !mx_aligned(dh, 16))
+        return MX_EINVAL;
+    if (int st = mx_check_device()) return st;
+    const int64_t n = rows * (F / 8);
+    if (n == 0) return MX_OK;
+    swiglu_bwd_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(
+        static_cast<const uint16_t*>(h), static_cast<const uint16_t*>(da), rows, F, gated, rows_valid,
+        static_cast<uint16_t*>(dh));
+    return mx_launch_status();
+}
+
+extern "C" int moe_combine(const void* y, const int32_t* pos, const float* w, int64_t T, int64_t k, int64_t D,
+                           void* out, cudaStream_t stream) {
+    if (!y || !pos || !out || T < 0 || k <= 0 || D <= 0 || D % 8 || !mx_aligned(y, 16) || !mx_aligned(out, 16))
+        return MX_EINVAL;
+    if (int st = mx_check_device()) return st;
+    if (T == 0) return MX_OK;
+    combine_kernel<<<(unsigned)T, 128, 0, stream>>>(static_cast<const uint16_t*>(y), pos, w, k, D,
+                                                    static_cast<uint16_t*>(out));
+    return mx_launch_status();
+}
+
+extern "C" int moe_dispatch_grad(const void* dout, const int32_t* src, const float* w, int64_t k, int64_t M_cap,
+                                 int64_t D, void* dy, cudaStream_t stream) {
+    if (!dout || !src || !dy || k <= 0 || M_cap < 0 || D <= 0 || D % 8 || !mx_aligned(dout, 16) ||
+        !mx_aligned(dy, 16))
+        return MX_EINVAL;
+    if (int st = mx_check_device()) return st;
+    if (M_cap == 0) return MX_OK;
+    dispatch_grad_kernel<<<(unsigned)M_cap, 128, 0, stream>>>(static_cast<const uint16_t*>(dout), src, w, k, D,
+                                                              static_cast<uint16_t*>(dy));
+    return mx_launch_status();
+}

@@ -1,0 +1,175 @@
+// mx_common.cuh -- device helpers shared by the mxmoe kernels (sm_100a).
+//
+// Number formats ([ai-primer] "Inkling 2 Small uses four-bit training...",
+// §Block scales and per-token activations): NVFP4 = E2M1 values with one E4M3
+// scale per 16 values and an FP32 outer scale; MXFP8 = E4M3 values with one
+// E8M0 scale per 32 values.  Conversions use the PTX `cvt` instructions
+// (round-to-nearest-even, saturating to the largest finite value); the
+// stochastic rounding and the E8M0 exponent are exact integer arithmetic on
+// the fp32 bit patterns.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "../../include/mxmoe.h"
+
+// ---------------------------------------------------------------------------
+// Host-side status helpers (defined in abi.cu)
+// ---------------------------------------------------------------------------
+int mx_set_cuda_error(cudaError_t e);   // records e, returns MX_ECUDA
+int mx_check_device(void);              // MX_OK on sm_100, else MX_EUNSUPPORTED / MX_ECUDA
+int mx_launch_status(void);             // cudaGetLastError -> MX_OK / MX_ECUDA
+
+static inline bool mx_aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// ---------------------------------------------------------------------------
+// Scale-factor layouts
+// ---------------------------------------------------------------------------
+// MMA layout: 512-byte atoms of 128 rows x 4 scale columns; atom index
+// (r/128)*(S/4) + s/4, byte (r%32)*16 + ((r%128)/32)*4 + s%4 inside it.
+__host__ __device__ __forceinline__ int64_t sf_offset_mma(int64_t r, int64_t s, int64_t S) {
+    return (((r >> 7) * (S >> 2) + (s >> 2)) << 9) + ((r & 31) << 4) + (((r >> 5) & 3) << 2) + (s & 3);
+}
+__host__ __device__ __forceinline__ int64_t sf_offset(int64_t r, int64_t s, int64_t S, int layout) {
+    return layout == MX_SF_MMA ? sf_offset_mma(r, s, S) : r * S + s;
+}
+
+// ---------------------------------------------------------------------------
+// Element conversions (PTX cvt, sm_100a)
+// ---------------------------------------------------------------------------
+// Two fp32 -> one byte of two E2M1 codes; `lo` lands in the low nibble.
+__device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
+    uint32_t out;
+    asm("{\n\t.reg .b8 b;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b, %2, %1;\n\t"
+        "cvt.u32.u8 %0, b;\n\t}"
+        : "=r"(out) : "f"(lo), "f"(hi));
+    return out;
+}
+
+// Two fp32 -> two E4M3 codes in a 16-bit value; `lo` in the low byte.
+__device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
+    uint16_t out;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %2, %1;" : "=h"(out) : "f"(lo), "f"(hi));
+    return out;
+}
+
+// One E4M3 code -> fp32 (exact).
+__device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
+    uint32_t h2;
+    uint16_t in = (uint16_t)((code & 0xff) * 0x0101u);   // same code in both lanes
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
+    return __half2float(__ushort_as_half((unsigned short)(h2 & 0xffff)));
+}
+
+// Byte of two E2M1 codes -> two halves (exact).
+__device__ __forceinline__ __half2 e2m1x2_to_h2(uint32_t byte) {
+    uint32_t h2;
+    asm("{\n\t.reg .b8 b;\n\t"
+        "cvt.u8.u32 b, %1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b;\n\t}"
+        : "=r"(h2) : "r"(byte));
+    return *reinterpret_cast<__half2*>(&h2);
+}
+
+// E4M3 code -> half (exact: E4M3 is a subset of fp16).
+__device__ __forceinline__ __half e4m3_to_h(uint32_t code) {
+    uint32_t h2;
+    uint16_t in = (uint16_t)((code & 0xff) * 0x0101u);   // same code in both lanes
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
+    return __ushort_as_half((unsigned short)(h2 & 0xffff));
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// ---------------------------------------------------------------------------
+// MXFP8 block exponent: smallest e with amax <= 448 * 2^e, clamped to
+// [-127, 127]; -127 for amax == 0.  448 = 1.75 * 2^8, so for a normal
+// amax = 1.f * 2^E the answer is E-8 when 1.f <= 1.75, else E-7.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int e8m0_exponent(float amax) {
+    uint32_t b = __float_as_uint(amax) & 0x7fffffffu;
+    int eb = (int)(b >> 23);
+    if (eb == 0) return -127;                    // zero or fp32-subnormal: E <= -127
+    int E = eb - 127;
+    int e = ((b & 0x7fffffu) <= 0x600000u) ? E - 8 : E - 7;
+    return e < -127 ? -127 : (e > 127 ? 127 : e);
+}
+
+// 2^-e as an fp32 (e in [-127, 127]); 2^-127 is the subnormal 0x00200000.
+__device__ __forceinline__ float exp2_neg(int e) {
+    int k = 127 - e;                             // biased exponent of 2^-e
+    return k >= 1 ? __uint_as_float((uint32_t)k << 23) : __uint_as_float(0x00200000u);
+}
+
+// ---------------------------------------------------------------------------
+// Stochastic rounding of y = xh * 2^-e onto the E4M3 grid, exactly.
+// xh is any finite fp32.  With y = M * 2^p (M the 24-bit significand), the
+// quantum is 2^Q, Q = max(floor(log2 y) - 3, -9); the sh = Q - p bits of M
+// below the quantum are dropped and the value rounds up iff
+// u < floor(rem * 2^R / 2^sh).  The E4M3 code of units * 2^Q is
+// (Q + 9) * 8 + units for every Q >= -9 (codes are monotone in magnitude, so a
+// carry into the next binade is the next code).  Caller guarantees |y| <= 448.
+// ---------------------------------------------------------------------------
+template <int R>
+__device__ __forceinline__ uint32_t e4m3_sr_code(float xh, int e, uint32_t u) {
+    uint32_t bits = __float_as_uint(xh);
+    uint32_t sign = (bits >> 24) & 0x80u;
+    uint32_t mag = bits & 0x7fffffffu;
+    if (mag == 0) return sign;
+    uint32_t eb = mag >> 23;
+    uint32_t M = eb ? ((mag & 0x7fffffu) | 0x800000u) : mag;
+    int p = (eb ? (int)eb - 150 : -149) - e;     // exponent of M's unit bit in y
+    int fl = p + (31 - __clz(M));                // floor(log2 y)
+    int Q = fl - 3 < -9 ? -9 : fl - 3;
+    int sh = Q - p;
+    uint32_t units;
+    if (sh <= 0) {
+        units = M << (-sh);                      // on the grid already
+    } else {
+        uint32_t lo = sh >= 32 ? 0u : (M >> sh);
+        uint64_t rem = sh >= 32 ? (uint64_t)M : (uint64_t)(M & ((1u << sh) - 1u));
+        uint64_t thr = sh >= 64 ? 0ull : ((rem << R) >> sh);
+        units = lo + ((uint64_t)u < thr ? 1u : 0u);
+    }
+    return sign | (uint32_t)((Q + 9) * 8 + (int)units);
+}
+
+// ---------------------------------------------------------------------------
+// Philox4x32-10 (Salmon, Moraes, Dror, Shaw, SC'11): ten rounds of the
+// multiply / cross / key-add network; the key advances by the Weyl constants
+// between rounds.  counter = (g lo, g hi, stream lo, stream hi),
+// key = (seed lo, seed hi).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint4 philox4x32_10(uint64_t g, uint64_t stream, uint64_t seed) {
+    uint32_t c0 = (uint32_t)g, c1 = (uint32_t)(g >> 32), c2 = (uint32_t)stream, c3 = (uint32_t)(stream >> 32);
+    uint32_t k0 = (uint32_t)seed, k1 = (uint32_t)(seed >> 32);
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+        uint32_t hi0 = __umulhi(0xD2511F53u, c0), lo0 = 0xD2511F53u * c0;
+        uint32_t hi1 = __umulhi(0xCD9E8D57u, c2), lo1 = 0xCD9E8D57u * c2;
+        uint32_t n0 = hi1 ^ c1 ^ k0, n2 = hi0 ^ c3 ^ k1;
+        c0 = n0; c1 = lo1; c2 = n2; c3 = lo0;
+        k0 += 0x9E3779B9u; k1 += 0xBB67AE85u;
+    }
+    return make_uint4(c0, c1, c2, c3);
+}
+
+// R-bit random integer j (0 <= j < 128/R) of a Philox block.
+template <int R>
+__device__ __forceinline__ uint32_t philox_field(const uint4& w, int j) {
+    const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+    if (R == 32) return words[j];
+    int bit = j * R;
+    return (words[bit >> 5] >> (bit & 31)) & ((1u << (R & 31)) - 1u);
+}
+
+__device__ __forceinline__ int64_t load_rows_valid(const int64_t* rows_valid, int64_t rows) {
+    if (!rows_valid) return rows;
+    int64_t v = *rows_valid;
+    return v < rows ? v : rows;
+}

@@ -1,0 +1,424 @@
+// quant.cu -- NVFP4 quantiser, MXFP8 quantiser and the NVFP4 -> MXFP8
+// stochastic requantisation across a transpose (sm_100a).
+//
+// All three are HBM streams: 128-bit coalesced loads and stores, amax by
+// packed-integer max and warp shuffles, every rounding decision taken by a PTX
+// cvt or by exact integer arithmetic (see mx_common.cuh).
+#include "mx_common.cuh"
+
+namespace {
+
+constexpr int kWarpsPerBlock = 8;
+
+// Max of |bf16| over the 8 elements of a uint4, as the bf16 magnitude bits
+// (integer order equals numeric order for non-NaN magnitudes).
+__device__ __forceinline__ uint32_t absmax8_bf16(const uint4& v) {
+    uint32_t m = __vmaxu2(v.x & 0x7fff7fffu, v.y & 0x7fff7fffu);
+    m = __vmaxu2(m, v.z & 0x7fff7fffu);
+    m = __vmaxu2(m, v.w & 0x7fff7fffu);
+    return max(m & 0xffffu, m >> 16);
+}
+
+__device__ __forceinline__ uint32_t warp_max_u32(uint32_t v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+// Quantise one 16-element block (two uint4 of bf16) with outer scale s > 0.
+// Returns the E4M3 scale code; writes 8 bytes of packed E2M1 codes.
+__device__ __forceinline__ uint32_t nvfp4_block(const uint4& a, const uint4& b, float s, uint2& packed) {
+    uint32_t ab_bits = max(absmax8_bf16(a), absmax8_bf16(b));
+    float ab = __uint_as_float(ab_bits << 16);
+    float t = __fmul_rn(6.0f, s);
+    float d = __fdiv_rn(ab, t);
+    uint32_t sc = cvt_e4m3x2(d, 0.0f) & 0xffu;
+    if (sc == 0) { packed = make_uint2(0u, 0u); return 0u; }
+    float inv = __frcp_rn(__fmul_rn(e4m3_to_f32(sc), s));
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    uint32_t out[2] = {0u, 0u};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        uint32_t byte = cvt_e2m1x2(__fmul_rn(bf16_lo(w[i]), inv), __fmul_rn(bf16_hi(w[i]), inv));
+        out[i >> 2] |= byte << ((i & 3) * 8);
+    }
+    packed = make_uint2(out[0], out[1]);
+    return sc;
+}
+
+// One warp per row; lane l handles 16-element blocks l, l+32, ...  Rows of up
+// to 32*16*kNB elements stay in registers; longer rows are read twice.
+// GROUP: the outer scale is per group of rows and `outer` already holds the
+// group's amax bits (written by nvfp4_group_amax_kernel).
+template <int kNB, bool kGroup, int kLayout>
+__global__ void __launch_bounds__(kWarpsPerBlock * 32)
+nvfp4_quant_rows_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t group_rows,
+                        uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, float* __restrict__ outer) {
+    const int lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
+    if (row >= rows) return;
+    const int64_t nblk = cols >> 4;
+    const uint4* xr = reinterpret_cast<const uint4*>(x + row * cols);
+
+    uint4 va[kNB], vb[kNB];
+    uint32_t amax_bits = 0;
+    const bool resident = nblk <= 32 * kNB;
+#pragma unroll
+    for (int i = 0; i < kNB; ++i) {
+        int64_t blk = lane + 32 * i;
+        if (resident && blk < nblk) {
+            va[i] = __ldcs(xr + 2 * blk);
+            vb[i] = __ldcs(xr + 2 * blk + 1);
+            amax_bits = max(amax_bits, max(absmax8_bf16(va[i]), absmax8_bf16(vb[i])));
+        }
+    }
+    if (!resident) {
+        for (int64_t blk = lane; blk < nblk; blk += 32)
+            amax_bits = max(amax_bits, max(absmax8_bf16(xr[2 * blk]), absmax8_bf16(xr[2 * blk + 1])));
+    }
+
+    float s;
+    if (kGroup) {
+        s = __fdiv_rn(__uint_as_float(__float_as_uint(outer[row / group_rows])), 2688.0f);
+    } else {
+        amax_bits = warp_max_u32(amax_bits);
+        s = __fdiv_rn(__uint_as_float(amax_bits << 16), 2688.0f);
+        if (lane == 0) outer[row] = s;
+    }
+
+    uint8_t* crow = codes + row * (cols >> 1);
+    auto emit = [&](int64_t blk, const uint4& a, const uint4& b) {
+        uint2 packed = make_uint2(0u, 0u);
+        uint32_t sc = 0;
+        if (s > 0.0f) sc = nvfp4_block(a, b, s, packed);
+        *reinterpret_cast<uint2*>(crow + blk * 8) = packed;
+        sf[sf_offset(row, blk, nblk, kLayout)] = (uint8_t)sc;
+    };
+    if (resident) {
+#pragma unroll
+        for (int i = 0; i < kNB; ++i) {
+            const int64_t blk = lane + 32 * i;
+            if (blk < nblk) emit(blk, va[i], vb[i]);
+        }
+    } else {
+        for (int64_t blk = lane; blk < nblk; blk += 32) emit(blk, xr[2 * blk], xr[2 * blk + 1]);
+    }
+}
+
+// amax over each group of rows, as fp32 bits, atomically max-ed into outer[g]
+// (pre-zeroed).  Grid-stride over 16-element blocks.
+__global__ void nvfp4_group_amax_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols,
+                                        int64_t group_rows, float* __restrict__ outer) {
+    const int64_t nblk_row = cols >> 4;
+    const int64_t total = rows * nblk_row;
+    const uint4* xv = reinterpret_cast<const uint4*>(x);
+    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    // consecutive threads take consecutive blocks; a warp's blocks usually
+    // share a group, so reduce inside the warp before the atomic
+    for (int64_t base = i - threadIdx.x % 32; base < total; base += stride) {
+        int64_t blk = base + (threadIdx.x % 32);
+        uint32_t m = 0;
+        int64_t g = -1;
+        if (blk < total) {
+            m = max(absmax8_bf16(__ldcs(xv + 2 * blk)), absmax8_bf16(__ldcs(xv + 2 * blk + 1)));
+            g = (blk / nblk_row) / group_rows;
+        }
+        int64_t g0 = __shfl_sync(0xffffffffu, g, 0);
+        bool same = __all_sync(0xffffffffu, g == g0 || g < 0);
+        if (same) {
+            m = warp_max_u32(m);
+            if ((threadIdx.x % 32) == 0 && g0 >= 0)
+                atomicMax(reinterpret_cast<unsigned int*>(outer) + g0, m << 16);
+        } else if (g >= 0) {
+            atomicMax(reinterpret_cast<unsigned int*>(outer) + g, m << 16);
+        }
+    }
+}
+
+__global__ void nvfp4_group_finish_kernel(float* outer, int64_t ngroups) {
+    int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (g < ngroups) outer[g] = __fdiv_rn(outer[g], 2688.0f);
+}
+
+// ---------------------------------------------------------------------------
+// Transpose tile: 128 rows x 64 columns of the input.  Phase 1 loads the tile
+// (bf16, or NVFP4 dequantised to fp32) -- thread t owns row t/2, columns
+// 32*(t%2) .. +31 -- and stores fp32 values transposed into shared memory
+// T[c][r] (128 words per row c, the r index XOR-swizzled by 16*(c/32) so both
+// column halves hit disjoint banks).  Phase 2: thread (c, g) takes output row
+// c, elements r = 16g .. 16g+15 (8 threads cover the tile's 128 r of row c);
+// lane pairs (g, g^1) form one 32-element MXFP8 block.
+// ---------------------------------------------------------------------------
+constexpr int kTR = 128, kTC = 64, kTileThreads = 256;
+
+__device__ __forceinline__ int tsw(int c, int r) { return c * kTR + (r ^ ((c >> 5) << 4)); }
+
+// Phase 2: from smem T to MXFP8 codes of the transposed output.
+// kSR: stochastic rounding with kR random bits, else RNE.
+template <bool kSR, int kR, int kLayout>
+__device__ __forceinline__ void tile_emit_transposed(const float* T, int64_t rows, int64_t cols, int64_t r0, int64_t c0,
+                                                     uint64_t seed, uint64_t stream_id,
+                                                     uint8_t* __restrict__ out_codes, uint8_t* __restrict__ out_e8m0) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int g = lane & 7;
+    const int64_t S = rows >> 5;                        // output scales per output row
+#pragma unroll 1
+    for (int it = 0; it < 2; ++it) {
+        const int c = it * 32 + warp * 4 + (lane >> 3);
+        float v[16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int pj = (j + (g >> 1)) & 3;         // bank-conflict-free chunk order
+            const float4 q = *reinterpret_cast<const float4*>(T + tsw(c, 16 * g + 4 * pj));
+            v[4 * pj + 0] = q.x; v[4 * pj + 1] = q.y; v[4 * pj + 2] = q.z; v[4 * pj + 3] = q.w;
+        }
+        uint32_t m = 0;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) m = max(m, __float_as_uint(v[i]) & 0x7fffffffu);
+        m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
+        const int e = e8m0_exponent(__uint_as_float(m));
+        const int64_t cg = c0 + c;
+        const int64_t rr = r0 + 16 * g;
+        uint32_t w[4];
+        if (kSR) {
+            const int64_t L0 = cg * rows + rr;          // output element index
+            constexpr int kPer = 128 / kR;              // elements per Philox block
+#pragma unroll
+            for (int blk = 0; blk < 16 / kPer + (16 % kPer ? 1 : 0); ++blk) {
+                const uint4 rnd = philox4x32_10((uint64_t)(L0 / kPer) + blk, stream_id, seed);
+#pragma unroll
+                for (int jj = 0; jj < kPer && blk * kPer + jj < 16; ++jj) {
+                    const int i = blk * kPer + jj;
+                    const uint32_t code = e4m3_sr_code<kR>(v[i], e, philox_field<kR>(rnd, jj));
+                    if ((i & 3) == 0) w[i >> 2] = code; else w[i >> 2] |= code << (8 * (i & 3));
+                }
+            }
+        } else {
+            const float sc = exp2_neg(e);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                w[i] = cvt_e4m3x2(__fmul_rn(v[4 * i], sc), __fmul_rn(v[4 * i + 1], sc)) |
+                       (cvt_e4m3x2(__fmul_rn(v[4 * i + 2], sc), __fmul_rn(v[4 * i + 3], sc)) << 16);
+        }
+        *reinterpret_cast<uint4*>(out_codes + cg * rows + rr) = make_uint4(w[0], w[1], w[2], w[3]);
+        if ((g & 1) == 0) out_e8m0[sf_offset(cg, rr >> 5, S, kLayout)] = (uint8_t)(e + 127);
+    }
+}
+
+// MXFP8 quantisation of bf16 [rows, cols]: row-wise blocks (phase 1, straight
+// from registers) and/or the transposed column-wise form (phase 2).
+template <bool kRow, bool kCol, bool kSR, int kR, int kLayout>
+__global__ void __launch_bounds__(kTileThreads)
+mxfp8_tile_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, const int64_t* rows_valid,
+                  uint64_t seed, uint64_t stream_row, uint64_t stream_col,
+                  uint8_t* __restrict__ row_codes, uint8_t* __restrict__ row_e8m0,
+                  uint8_t* __restrict__ col_codes, uint8_t* __restrict__ col_e8m0) {
+    __shared__ __align__(16) float T[kCol ? kTC * kTR : 4];
+    const int64_t c0 = (int64_t)blockIdx.x * kTC, r0 = (int64_t)blockIdx.y * kTR;
+    if (r0 >= load_rows_valid(rows_valid, rows)) return;
+    const int t = threadIdx.x;
+    const int rl = t >> 1, h = t & 1;
+    const int64_t r = r0 + rl;
+    const uint4* src = reinterpret_cast<const uint4*>(x + r * cols + c0 + 32 * h);
+    uint4 q[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) q[i] = __ldcs(src + i);
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t w[4] = {q[i].x, q[i].y, q[i].z, q[i].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) { v[8 * i + 2 * j] = bf16_lo(w[j]); v[8 * i + 2 * j + 1] = bf16_hi(w[j]); }
+    }
+    if (kRow) {
+        uint32_t m = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) m = max(m, absmax8_bf16(q[i]));
+        const int e = e8m0_exponent(__uint_as_float(m << 16));
+        uint32_t w[8];
+        const int64_t L0 = r * cols + c0 + 32 * h;
+        if (kSR) {
+            constexpr int kPer = 128 / kR;
+#pragma unroll
+            for (int blk = 0; blk < 32 / kPer; ++blk) {
+                const uint4 rnd = philox4x32_10((uint64_t)(L0 / kPer) + blk, stream_row, seed);
+#pragma unroll
+                for (int jj = 0; jj < kPer; ++jj) {
+                    const int i = blk * kPer + jj;
+                    const uint32_t code = e4m3_sr_code<kR>(v[i], e, philox_field<kR>(rnd, jj));
+                    if ((i & 3) == 0) w[i >> 2] = code; else w[i >> 2] |= code << (8 * (i & 3));
+                }
+            }
+        } else {
+            const float sc = exp2_neg(e);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                w[i] = cvt_e4m3x2(__fmul_rn(v[4 * i], sc), __fmul_rn(v[4 * i + 1], sc)) |
+                       (cvt_e4m3x2(__fmul_rn(v[4 * i + 2], sc), __fmul_rn(v[4 * i + 3], sc)) << 16);
+        }
+        uint4* dst = reinterpret_cast<uint4*>(row_codes + L0);
+        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        row_e8m0[sf_offset(r, (c0 >> 5) + h, cols >> 5, kLayout)] = (uint8_t)(e + 127);
+    }
+    if (kCol) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) T[tsw(32 * h + i, rl)] = v[i];
+        __syncthreads();
+        tile_emit_transposed<kSR, kR, kLayout>(T, rows, cols, r0, c0, seed, stream_col, col_codes, col_e8m0);
+    }
+}
+
+// NVFP4 [rows, cols] -> dequantise -> transpose -> MXFP8 with SR.
+template <int kR, int kInLayout, int kOutLayout>
+__global__ void __launch_bounds__(kTileThreads)
+requant_tile_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sf, const float* __restrict__ outer,
+                    int64_t rows, int64_t cols, int64_t group_rows, const int64_t* rows_valid,
+                    uint64_t seed, uint64_t stream_id, uint8_t* __restrict__ out_codes, uint8_t* __restrict__ out_e8m0) {
+    __shared__ __align__(16) float T[kTC * kTR];
+    const int64_t c0 = (int64_t)blockIdx.x * kTC, r0 = (int64_t)blockIdx.y * kTR;
+    if (r0 >= load_rows_valid(rows_valid, rows)) return;
+    const int t = threadIdx.x;
+    const int rl = t >> 1, h = t & 1;
+    const int64_t r = r0 + rl;
+    const uint4 q = __ldcs(reinterpret_cast<const uint4*>(codes + r * (cols >> 1) + (c0 >> 1) + 16 * h));
+    const int64_t S = cols >> 4;
+    const int64_t s0 = (c0 >> 4) + 2 * h;
+    const uint32_t sc0 = sf[sf_offset(r, s0, S, kInLayout)];
+    const uint32_t sc1 = sf[sf_offset(r, s0 + 1, S, kInLayout)];
+    const float so = outer[r / group_rows];
+    const __half2 f0 = __half2half2(e4m3_to_h(sc0)), f1 = __half2half2(e4m3_to_h(sc1));
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {                     // byte i = elements 2i, 2i+1
+        const uint32_t byte = (w[i >> 2] >> (8 * (i & 3))) & 0xffu;
+        const __half2 p = __hmul2(e2m1x2_to_h2(byte), i < 8 ? f0 : f1);   // exact
+        const float2 pf = __half22float2(p);
+        T[tsw(32 * h + 2 * i, rl)] = __fmul_rn(pf.x, so);
+        T[tsw(32 * h + 2 * i + 1, rl)] = __fmul_rn(pf.y, so);
+    }
+    __syncthreads();
+    tile_emit_transposed<true, kR, kOutLayout>(T, rows, cols, r0, c0, seed, stream_id, out_codes, out_e8m0);
+}
+
+template <typename F>
+int dispatch_layout(int layout, F&& f) {
+    if (layout == MX_SF_MMA) return f(std::integral_constant<int, MX_SF_MMA>());
+    return f(std::integral_constant<int, MX_SF_ROWMAJOR>());
+}
+
+}  // namespace
+
+// ===========================================================================
+// C ABI
+// ===========================================================================
+
+extern "C" int nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t group_rows, uint8_t* codes,
+                              uint8_t* sf, float* outer, int sf_layout, cudaStream_t stream) {
+    if (!x || !codes || !sf || !outer || rows < 0 || cols <= 0 || cols % 16 || group_rows <= 0 ||
+        rows % group_rows || !mx_aligned(x, 16) || !mx_aligned(codes, 16))
+        return MX_EINVAL;
+    if (sf_layout != MX_SF_ROWMAJOR && sf_layout != MX_SF_MMA) return MX_EINVAL;
+    if (sf_layout == MX_SF_MMA && (rows % 128 || cols % 64)) return MX_EINVAL;
+    if (int st = mx_check_device()) return st;
+    if (rows == 0) return MX_OK;
+    const uint16_t* xb = static_cast<const uint16_t*>(x);
+    const int64_t ngroups = rows / group_rows;
+    const int64_t nblk_row = cols / 16;
+    const dim3 block(kWarpsPerBlock * 32);
+    const dim3 grid((unsigned)((rows + kWarpsPerBlock - 1) / kWarpsPerBlock));
+    return dispatch_layout(sf_layout, [&](auto L) {
+        constexpr int kL = decltype(L)::value;
+        if (group_rows == 1) {
+            if (nblk_row <= 32 * 2)
+                nvfp4_quant_rows_kernel<2, false, kL><<<grid, block, 0, stream>>>(xb, rows, cols, 1, codes, sf, outer);
+            else
+                nvfp4_quant_rows_kernel<8, false, kL><<<grid, block, 0, stream>>>(xb, rows, cols, 1, codes, sf, outer);
+        } else {
+            if (cudaMemsetAsync(outer, 0, sizeof(float) * ngroups, stream) != cudaSuccess) return mx_launch_status();
+            const int64_t total = rows * nblk_row;
+            const unsigned g = (unsigned)std::min<int64_t>((total + 255) / 256, 148 * 16);
+            nvfp4_group_amax_kernel<<<g, 256, 0, stream>>>(xb, rows, cols, group_rows, outer);
+            if (nblk_row <= 32 * 2)
+                nvfp4_quant_rows_kernel<2, true, kL><<<grid, block, 0, stream>>>(xb, rows, cols, group_rows, codes, sf, outer);
+            else
+                nvfp4_quant_rows_kernel<8, true, kL><<<grid, block, 0, stream>>>(xb, rows, cols, group_rows, codes, sf, outer);
+            nvfp4_group_finish_kernel<<<(unsigned)((ngroups + 255) / 256), 256, 0, stream>>>(outer, ngroups);
+        }
+        return mx_launch_status();
+    });
+}
+
+extern "C" int mxfp8_quantize(const void* x, int64_t rows, int64_t cols, int rounding, uint64_t seed,
+                              uint64_t stream_id, int rbits, const int64_t* rows_valid,
+                              uint8_t* row_codes, uint8_t* row_e8m0, uint8_t* col_codes, uint8_t* col_e8m0,
+                              int sf_layout, cudaStream_t stream) {
+    const bool do_row = row_codes != nullptr, do_col = col_codes != nullptr;
+    if (!x || rows < 0 || cols <= 0 || rows % kTR || cols % 128 || !mx_aligned(x, 16)) return MX_EINVAL;
+    if (!do_row && !do_col) return MX_EINVAL;
+    if ((do_row && (!row_e8m0 || !mx_aligned(row_codes, 16))) || (do_col && (!col_e8m0 || !mx_aligned(col_codes, 16))))
+        return MX_EINVAL;
+    if (rounding != MX_ROUND_RNE && rounding != MX_ROUND_SR) return MX_EINVAL;
+    if (rounding == MX_ROUND_SR && rbits != 8 && rbits != 16 && rbits != 32) return MX_EINVAL;
+    if (sf_layout != MX_SF_ROWMAJOR && sf_layout != MX_SF_MMA) return MX_EINVAL;
+    if (int st = mx_check_device()) return st;
+    if (rows == 0) return MX_OK;
+    const dim3 grid((unsigned)(cols / kTC), (unsigned)(rows / kTR));
+    const uint64_t s_row = stream_id, s_col = do_row ? stream_id + 1 : stream_id;
+    const uint16_t* xb = static_cast<const uint16_t*>(x);
+    return dispatch_layout(sf_layout, [&](auto L) {
+        constexpr int kL = decltype(L)::value;
+        auto launch = [&](auto kRowC, auto kColC) {
+            constexpr bool kRow = decltype(kRowC)::value, kCol = decltype(kColC)::value;
+            if (rounding == MX_ROUND_RNE)
+                mxfp8_tile_kernel<kRow, kCol, false, 8, kL><<<grid, kTileThreads, 0, stream>>>(
+                    xb, rows, cols, rows_valid, seed, s_row, s_col, row_codes, row_e8m0, col_codes, col_e8m0);
+            else if (rbits == 8)
+                mxfp8_tile_kernel<kRow, kCol, true, 8, kL><<<grid, kTileThreads, 0, stream>>>(
+                    xb, rows, cols, rows_valid, seed, s_row, s_col, row_codes, row_e8m0, col_codes, col_e8m0);
+            else if (rbits == 16)
+                mxfp8_tile_kernel<kRow, kCol, true, 16, kL><<<grid, kTileThreads, 0, stream>>>(
+                    xb, rows, cols, rows_valid, seed, s_row, s_col, row_codes, row_e8m0, col_codes, col_e8m0);
+            else
+                mxfp8_tile_kernel<kRow, kCol, true, 32, kL><<<grid, kTileThreads, 0, stream>>>(
+                    xb, rows, cols, rows_valid, seed, s_row, s_col, row_codes, row_e8m0, col_codes, col_e8m0);
+        };
+        if (do_row && do_col) launch(std::true_type(), std::true_type());
+        else if (do_row) launch(std::true_type(), std::false_type());
+        else launch(std::false_type(), std::true_type());
+        return mx_launch_status();
+    });
+}
+
+extern "C" int mxfp8_requant_transpose_sr(const uint8_t* codes, const uint8_t* sf, const float* outer,
+                                          int64_t rows, int64_t cols, int64_t group_rows, int in_sf_layout,
+                                          const int64_t* rows_valid, uint64_t seed, uint64_t stream_id, int rbits,
+                                          uint8_t* out_codes, uint8_t* out_e8m0, int out_sf_layout,
+                                          cudaStream_t stream) {
+    if (!codes || !sf || !outer || !out_codes || !out_e8m0 || rows < 0 || cols <= 0 || rows % kTR || cols % kTC ||
+        group_rows <= 0 || rows % group_rows || !mx_aligned(codes, 16) || !mx_aligned(out_codes, 16))
+        return MX_EINVAL;
+    if (rbits != 8 && rbits != 16 && rbits != 32) return MX_EINVAL;
+    for (int l : {in_sf_layout, out_sf_layout})
+        if (l != MX_SF_ROWMAJOR && l != MX_SF_MMA) return MX_EINVAL;
+    if (out_sf_layout == MX_SF_MMA && (cols % 128 || rows % 128)) return MX_EINVAL;
+    if (int st = mx_check_device()) return st;
+    if (rows == 0) return MX_OK;
+    const dim3 grid((unsigned)(cols / kTC), (unsigned)(rows / kTR));
+    return dispatch_layout(in_sf_layout, [&](auto Li) {
+        return dispatch_layout(out_sf_layout, [&](auto Lo) {
+            constexpr int kLi = decltype(Li)::value, kLo = decltype(Lo)::value;
+            if (rbits == 8)
+                requant_tile_kernel<8, kLi, kLo><<<grid, kTileThreads, 0, stream>>>(
+                    codes, sf, outer, rows, cols, group_rows, rows_valid, seed, stream_id, out_codes, out_e8m0);
+            else if (rbits == 16)
+                requant_tile_kernel<16, kLi, kLo><<<grid, kTileThreads, 0, stream>>>(
+                    codes, sf, outer, rows, cols, group_rows, rows_valid, seed, stream_id, out_codes, out_e8m0);
+            else
+                requant_tile_kernel<32, kLi, kLo><<<grid, kTileThreads, 0, stream>>>(
+                    codes, sf, outer, rows, cols, group_rows, rows_valid, seed, stream_id, out_codes, out_e8m0);
+            return mx_launch_status();
+        });
+    });
+}

@@ -1,0 +1,172 @@
+"""One expert layer's numerics, forward and backward, as a chain of C-ABI calls.
+
+This is the whole hot path in order ([ai-primer] "Inkling 2 Small uses
+four-bit training...", §NVFP4 forward, MXFP8 backward and §Stochastic rounding
+across transposes):
+
+  forward   route -> NVFP4 quantise tokens (per-token outer scale) -> gather
+            into expert order -> NVFP4 quantise W1, W2 (per-expert outer
+            scale) -> grouped NVFP4 GEMM1 -> SwiGLU -> NVFP4 quantise ->
+            grouped NVFP4 GEMM2 -> combine
+  backward  combine gradient -> MXFP8 quantise dY2 (row- and column-wise) ->
+            requantise W2 and the saved activations (dequantise, transpose,
+            MXFP8 with stochastic rounding) -> MXFP8 dgrad / wgrad GEMMs ->
+            SwiGLU backward -> same for W1 and the saved tokens -> un-permute
+
+All buffers are allocated once; `forward()` / `backward()` only enqueue
+kernels on the current stream (no host synchronisation, no allocation), so a
+step can be timed or captured.  Python here only sequences calls.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import api
+from .api import MX_GEMM_DGRAD, MX_GEMM_WGRAD, MX_ROUND_RNE, MX_SF_MMA, MX_SF_ROWMAJOR
+
+
+def nvfp4_gemm_flops(counts, N: int, K: int) -> int:
+    """2 * sum_e m_e * N * K over true (unpadded) rows."""
+    return 2 * int(sum(int(c) for c in counts)) * N * K
+
+
+class ExpertLayer:
+    """Buffers and call sequence of one MoE expert layer.
+
+    x [T, D] bf16, topk [T, k] int32, w_comb [T, k] f32, w1 [E, 2F or F, D]
+    bf16, w2 [E, D, F] bf16, dout [T, D] bf16, all on one CUDA device.
+    `wgrad_dtype` is the dtype of dW1 / dW2 (bf16 or fp32).
+    """
+
+    def __init__(self, x, topk, w_comb, w1, w2, dout, gated: bool = True, seed: int = 0,
+                 wgrad_dtype=torch.bfloat16, out_dtype=torch.bfloat16, rbits: int = 8):
+        dev = x.device
+        self.dev = dev
+        self.T, self.D = x.shape
+        self.k = topk.shape[1]
+        self.E, self.N1, _ = w1.shape
+        self.F = w2.shape[2]
+        self.gated = gated
+        assert self.N1 == (2 * self.F if gated else self.F)
+        self.seed, self.rbits = seed, rbits
+        self.x, self.topk, self.w_comb, self.w1, self.w2, self.dout = x, topk, w_comb, w1, w2, dout
+        T, D, k, E, F, N1 = self.T, D, self.k, self.E, self.F, self.N1
+        self.M_cap = M = api.max_routed_rows(T, k, E)
+        e = lambda *s, dt=torch.uint8: torch.empty(*s, dtype=dt, device=dev)
+        sfb = api.sf_bytes
+        # routing
+        self.seg = e(E + 1, dt=torch.int64)
+        self.src = e(M, dt=torch.int32)
+        self.pos = e(T, k, dt=torch.int32)
+        self.route_ws = e(max(16, api.L.lib().mx_route_workspace_bytes(T, E)))
+        self.rows_valid = self.seg[E:E + 1]
+        # forward
+        self.xq = (e(T, D // 2), e(sfb(T, D, 16, MX_SF_ROWMAJOR)), e(T, dt=torch.float32))
+        self.xp = (e(M, D // 2), e(sfb(M, D, 16, MX_SF_MMA)), e(M, dt=torch.float32))
+        self.w1q = (e(E * N1, D // 2), e(sfb(E * N1, D, 16, MX_SF_MMA)), e(E, dt=torch.float32))
+        self.w2q = (e(E * D, F // 2), e(sfb(E * D, F, 16, MX_SF_MMA)), e(E, dt=torch.float32))
+        self.h1 = e(M, N1, dt=out_dtype)
+        self.a = e(M, F, dt=torch.bfloat16)
+        self.aq = (e(M, F // 2), e(sfb(M, F, 16, MX_SF_MMA)), e(M, dt=torch.float32))
+        self.y2 = e(M, D, dt=out_dtype)
+        self.out = e(T, D, dt=torch.bfloat16)
+        # backward
+        self.dy2 = e(M, D, dt=torch.bfloat16)
+        self.dy2q = (e(M, D), e(sfb(M, D, 32, MX_SF_MMA)), e(D, M), e(sfb(D, M, 32, MX_SF_MMA)))
+        self.w2t = (e(F, E * D), e(sfb(F, E * D, 32, MX_SF_MMA)))
+        self.da = e(M, F, dt=torch.bfloat16)
+        self.at = (e(F, M), e(sfb(F, M, 32, MX_SF_MMA)))
+        self.dw2 = e(E, D, F, dt=wgrad_dtype)
+        self.dh1 = e(M, N1, dt=torch.bfloat16)
+        self.dh1q = (e(M, N1), e(sfb(M, N1, 32, MX_SF_MMA)), e(N1, M), e(sfb(N1, M, 32, MX_SF_MMA)))
+        self.w1t = (e(D, E * N1), e(sfb(D, E * N1, 32, MX_SF_MMA)))
+        self.dxp = e(M, D, dt=torch.bfloat16)
+        self.xt = (e(D, M), e(sfb(D, M, 32, MX_SF_MMA)))
+        self.dw1 = e(E, N1, D, dt=wgrad_dtype)
+        self.dx = e(T, D, dt=torch.bfloat16)
+        self.marks = []
+
+    # ------------------------------------------------------------------ timing
+    def _mark(self, name: str, record: bool):
+        if record:
+            ev = torch.cuda.Event(enable_timing=True)
+            ev.record()
+            self.marks.append((name, ev))
+
+    def reset_marks(self):
+        self.marks = []
+
+    # ----------------------------------------------------------------- forward
+    def forward(self, record: bool = False):
+        T, D, k, E, F, N1, M = self.T, self.D, self.k, self.E, self.F, self.N1, self.M_cap
+        self._mark("start", record)
+        api.moe_route(self.topk, E, M, out=(self.seg, self.src, self.pos, self.route_ws))
+        self._mark("route", record)
+        api.nvfp4_quantize(self.x, 1, MX_SF_ROWMAJOR, out=self.xq)
+        self._mark("quant_x", record)
+        api.nvfp4_gather_rows(*self.xq, self.src, k, D, out=self.xp)
+        self._mark("gather", record)
+        api.nvfp4_quantize(self.w1.view(E * N1, D), N1, MX_SF_MMA, out=self.w1q)
+        api.nvfp4_quantize(self.w2.view(E * D, F), D, MX_SF_MMA, out=self.w2q)
+        self._mark("quant_w", record)
+        api.grouped_gemm_nvfp4(self.xp, self.w1q, self.seg, E, N1, D, out=self.h1)
+        self._mark("gemm1", record)
+        api.swiglu_fwd(self.h1, F, self.gated, self.rows_valid, out=self.a)
+        self._mark("swiglu", record)
+        api.nvfp4_quantize(self.a, 1, MX_SF_MMA, out=self.aq)
+        self._mark("quant_a", record)
+        api.grouped_gemm_nvfp4(self.aq, self.w2q, self.seg, E, D, F, out=self.y2)
+        self._mark("gemm2", record)
+        api.moe_combine(self.y2, self.pos, self.w_comb, D, out=self.out)
+        self._mark("combine", record)
+        return self.out
+
+    # ---------------------------------------------------------------- backward
+    def backward(self, record: bool = False):
+        T, D, k, E, F, N1, M = self.T, self.D, self.k, self.E, self.F, self.N1, self.M_cap
+        s, R = self.seed, self.rbits
+        self._mark("bwd_start", record)
+        api.moe_dispatch_grad(self.dout, self.src, self.w_comb, k, out=self.dy2)
+        self._mark("dispatch_grad", record)
+        api.mxfp8_quantize(self.dy2, rows_valid=self.rows_valid, rounding=MX_ROUND_RNE, out=self.dy2q)
+        self._mark("quant_dy2", record)
+        api.mxfp8_requant_transpose_sr(*self.w2q, E * D, F, D, MX_SF_MMA, None, s, 1, R, out=self.w2t)
+        self._mark("requant_w2", record)
+        api.grouped_gemm_mxfp8(MX_GEMM_DGRAD, self.dy2q[0], self.dy2q[1], *self.w2t, self.seg, E, M, F, D, out=self.da)
+        self._mark("dgrad2", record)
+        api.mxfp8_requant_transpose_sr(*self.aq, M, F, 1, MX_SF_MMA, self.rows_valid, s, 2, R, out=self.at)
+        self._mark("requant_a", record)
+        api.grouped_gemm_mxfp8(MX_GEMM_WGRAD, self.dy2q[2], self.dy2q[3], *self.at, self.seg, E, M, D, F, out=self.dw2)
+        self._mark("wgrad2", record)
+        api.swiglu_bwd(self.h1, self.da, F, self.gated, self.rows_valid, out=self.dh1)
+        self._mark("swiglu_bwd", record)
+        api.mxfp8_quantize(self.dh1, rows_valid=self.rows_valid, rounding=MX_ROUND_RNE, out=self.dh1q)
+        self._mark("quant_dh1", record)
+        api.mxfp8_requant_transpose_sr(*self.w1q, E * N1, D, N1, MX_SF_MMA, None, s, 3, R, out=self.w1t)
+        self._mark("requant_w1", record)
+        api.grouped_gemm_mxfp8(MX_GEMM_DGRAD, self.dh1q[0], self.dh1q[1], *self.w1t, self.seg, E, M, D, N1,
+                               out=self.dxp)
+        self._mark("dgrad1", record)
+        api.mxfp8_requant_transpose_sr(*self.xp, M, D, 1, MX_SF_MMA, self.rows_valid, s, 4, R, out=self.xt)
+        self._mark("requant_x", record)
+        api.grouped_gemm_mxfp8(MX_GEMM_WGRAD, self.dh1q[2], self.dh1q[3], *self.xt, self.seg, E, M, N1, D,
+                               out=self.dw1)
+        self._mark("wgrad1", record)
+        api.moe_combine(self.dxp, self.pos, None, D, out=self.dx)
+        self._mark("unpermute", record)
+        return self.dx, self.dw1, self.dw2
+
+    def step(self, record: bool = False):
+        self.forward(record)
+        return self.backward(record)
+
+    def stage_times_ms(self) -> dict:
+        """Device time (ms) of each stage, summed over the recorded steps: the
+        interval between a mark and the one before it is charged to the later
+        mark's name (call after synchronising)."""
+        out = {}
+        for (_, a), (name, b) in zip(self.marks, self.marks[1:]):
+            if name in ("start",):
+                continue
+            out[name] = out.get(name, 0.0) + a.elapsed_time(b)
+        return out

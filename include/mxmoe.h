@@ -1,0 +1,247 @@
+/*
+ * mxmoe.h -- C ABI of the B200 (sm_100a) library for 4-bit mixture-of-experts
+ * training numerics: NVFP4 forward expert GEMMs, and MXFP8 backward GEMMs fed by
+ * a dequantise -> transpose -> stochastic-rounding requantisation of the saved
+ * NVFP4 tensors.
+ *
+ * The method is the one reported for Thinking Machines' "End-to-End 4-Bit
+ * Training" (Inkling 2 Small).  Citations name the web page and its section:
+ *   [ai-primer] "Inkling 2 Small uses four-bit training, Thinking Machines
+ *               reports 8% and 20% savings" (ai-primer.com)
+ *   [hermes]    "Thinking Machines' Inkling 2 Small Trains a 594B Model in 68
+ *               Hours" (hermes-ai.net)
+ *
+ * Conventions for every entry point
+ *   - Pointers marked "device" are CUDA device pointers owned by the caller;
+ *     the library allocates no memory and keeps no pointer after returning.
+ *   - Work is enqueued asynchronously on `stream`; outputs are valid after the
+ *     stream is synchronised.  Nothing is synchronised inside a call.
+ *   - Return value: MX_OK, or MX_EINVAL (bad argument; checked on the host
+ *     before any launch, nothing is written), MX_ECUDA (launch failure;
+ *     mx_last_cuda_error() gives the cudaError_t), MX_EUNSUPPORTED (device is
+ *     not sm_100 or a mode that is not built).  Device-side bounded waits that
+ *     expire are reported later by mx_sync_status() as MX_ETIMEOUT.
+ *   - bf16 tensors are row-major, 2 bytes per element.
+ *   - NVFP4 tensor [rows, cols]: codes u8 [rows, cols/2] (E2M1, element 2j in
+ *     the low nibble of byte j), E4M3 block scales (one per 16 consecutive
+ *     elements of a row), fp32 outer scales (one per group of `group_rows`
+ *     rows: 1 = per token, N = per expert matrix of N rows).
+ *   - MXFP8 tensor [rows, cols]: codes u8 [rows, cols] (E4M3), E8M0 block
+ *     scales (one per 32 consecutive elements of a row; value 2^(byte-127)).
+ *   - Scale layouts (`sf_layout`):
+ *       MX_SF_ROWMAJOR: scale (r, s) at byte r*S + s, S = cols/block.
+ *       MX_SF_MMA: the tcgen05 block-scaled MMA layout.  Rows come in groups
+ *         of 128 and scale columns in groups of 4; each (row group, column
+ *         group) is a 512-byte atom stored at atom index
+ *         (r/128)*(S/4) + s/4, and (r, s) sits at byte
+ *         (r%32)*16 + ((r%128)/32)*4 + s%4 of its atom.  Needs rows % 128 == 0
+ *         and S % 4 == 0.
+ *   - Expert-major row buffers: `seg_offsets` (device, int64 [E+1]) gives the
+ *     first row of each expert; every segment length is a multiple of 128
+ *     (empty experts have length 0); seg_offsets[E] = M_pad <= M_cap, the
+ *     allocated row count.  Rows in [M_pad, M_cap) belong to no expert.
+ */
+#ifndef MXMOE_H
+#define MXMOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define MX_API __attribute__((visibility("default")))
+#else
+#define MX_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum { MX_OK = 0, MX_EINVAL = 1, MX_ECUDA = 2, MX_ETIMEOUT = 3, MX_EUNSUPPORTED = 4 };
+enum { MX_SF_ROWMAJOR = 0, MX_SF_MMA = 1 };
+enum { MX_OUT_F32 = 0, MX_OUT_BF16 = 1 };
+enum { MX_ROUND_RNE = 0, MX_ROUND_SR = 1 };
+enum { MX_GEMM_DGRAD = 0, MX_GEMM_WGRAD = 1 };
+
+/* Library version, for the bindings' sanity check. */
+MX_API int mx_version(void);
+
+/* cudaError_t of the last MX_ECUDA returned on this host thread. */
+MX_API int mx_last_cuda_error(void);
+
+/* Synchronises `stream`, then returns and clears the device status word of
+ * the current device: MX_ETIMEOUT if a bounded wait inside a GEMM kernel
+ * expired since the last call (that kernel's output is then undefined),
+ * MX_ECUDA if the synchronisation failed, else MX_OK. */
+MX_API int mx_sync_status(cudaStream_t stream);
+
+/* Bytes of a scale array of `rows` x `cols` elements with one scale per
+ * `block` (16 or 32) elements in `sf_layout`; 0 if the shape is not allowed
+ * for that layout. */
+MX_API size_t mx_sf_bytes(int64_t rows, int64_t cols, int block, int sf_layout);
+
+/* --------------------------------------------------------------------------
+ * nvfp4_quantize -- bf16 [rows, cols] -> NVFP4.
+ * [ai-primer §Block scales and per-token activations]: E2M1 values, one E4M3
+ * scale per 16-value block, an FP32 outer scale per token (activations,
+ * group_rows = 1) or per expert (weights [E*N, K], group_rows = N).
+ * Per group: s = amax/2688 (2688 = 6*448, s = 0 for an all-zero group); per
+ * block: sf = E4M3_rne_satfinite(amax_block / (6*s)); codes =
+ * E2M1_rne_satfinite(x * (1/(sf*s))), all zero when sf == 0.  Every step is
+ * one IEEE fp32 round-to-nearest operation.
+ *   x      device bf16 [rows, cols]
+ *   codes  device u8 [rows, cols/2];  sf device u8 mx_sf_bytes(rows,cols,16,sf_layout)
+ *   outer  device f32 [rows/group_rows]
+ * Requires cols % 16 == 0 (cols % 64 == 0 and rows % 128 == 0 for MX_SF_MMA),
+ * rows % group_rows == 0, 16-byte aligned x and codes.
+ * ------------------------------------------------------------------------ */
+MX_API int nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t group_rows,
+                   uint8_t* codes, uint8_t* sf, float* outer, int sf_layout, cudaStream_t stream);
+
+/* --------------------------------------------------------------------------
+ * mxfp8_requant_transpose_sr -- saved NVFP4 [rows, cols] -> MXFP8 transpose.
+ * [ai-primer §Stochastic rounding across transposes]: dequantise the saved
+ * tensor, transpose in higher precision, re-quantise to MXFP8 with stochastic
+ * rounding so represented values are preserved in expectation.
+ * Dequantised value: (q*sf)*s in fp32.  Output out[c][r] ([cols, rows]) with
+ * one E8M0 scale per 32 consecutive r: e = smallest integer with
+ * amax <= 448*2^e (clamped to [-127,127], -127 for a zero block); element
+ * y = x*2^-e rounded onto the E4M3 grid stochastically: with the quantum q of
+ * y's binade, round up iff u < floor(frac(y/q) * 2^rbits), u the rbits-bit
+ * random integer of output element L = c*rows + r.
+ * Random stream: Philox4x32-10 (Salmon et al., SC'11), key = (seed lo, seed
+ * hi), counter = (g lo, g hi, stream_id lo, stream_id hi) with
+ * g = L / (128/rbits); element L takes bits [j*rbits mod 32, +rbits) of word
+ * floor(j*rbits/32), j = L mod (128/rbits).
+ * Expert segments start at multiples of 32 rows, so each expert's transposed
+ * block is a column range [seg_e, seg_e+1) of the output.
+ *   codes/sf/outer  device NVFP4 input (sf in in_sf_layout), outer per
+ *                   group_rows rows (1 for activations, N for a weight stack)
+ *   out_codes       device u8 [cols, rows]
+ *   out_e8m0        device u8 mx_sf_bytes(cols, rows, 32, out_sf_layout)
+ *   rows_valid      device int64 or NULL: only r < *rows_valid are read and
+ *                   written (an expert-major buffer passes &seg_offsets[E])
+ * Requires rows % 128 == 0, cols % 64 == 0, rbits in {8, 16, 32}.
+ * ------------------------------------------------------------------------ */
+MX_API int mxfp8_requant_transpose_sr(const uint8_t* codes, const uint8_t* sf, const float* outer,
+                               int64_t rows, int64_t cols, int64_t group_rows, int in_sf_layout,
+                               const int64_t* rows_valid, uint64_t seed, uint64_t stream_id, int rbits,
+                               uint8_t* out_codes, uint8_t* out_e8m0, int out_sf_layout, cudaStream_t stream);
+
+/* --------------------------------------------------------------------------
+ * mxfp8_quantize -- bf16 [rows, cols] -> MXFP8, row-wise and/or column-wise.
+ * [ai-primer §NVFP4 forward, MXFP8 backward]: gradients are computed with
+ * MXFP8 matrix multiplications.  Same E8M0 rule as above; rounding
+ * MX_ROUND_RNE (E4M3 round-to-nearest-even) or MX_ROUND_SR (the stochastic
+ * rule and stream above, L = index in the output written).
+ *   row_codes [rows, cols], row_e8m0 (rows x cols, block 32): blocks along rows
+ *   col_codes [cols, rows], col_e8m0 (cols x rows, block 32): the transpose,
+ *     blocks along the original columns' length (tokens)
+ * Either output pair may be NULL (not produced).  With both and SR, the
+ * column-wise form uses stream_id + 1.  rows_valid as above.
+ * Requires rows % 128 == 0, cols % 128 == 0.
+ * ------------------------------------------------------------------------ */
+MX_API int mxfp8_quantize(const void* x, int64_t rows, int64_t cols, int rounding, uint64_t seed,
+                   uint64_t stream_id, int rbits, const int64_t* rows_valid,
+                   uint8_t* row_codes, uint8_t* row_e8m0, uint8_t* col_codes, uint8_t* col_e8m0,
+                   int sf_layout, cudaStream_t stream);
+
+/* --------------------------------------------------------------------------
+ * grouped_gemm_nvfp4 -- forward expert GEMM on tcgen05 block-scaled MMA.
+ * [ai-primer §NVFP4 forward, MXFP8 backward]: forward expert-layer matmuls in
+ * NVFP4 with a dedicated kernel.
+ * For rows r of expert e (seg_offsets[e] <= r < seg_offsets[e+1]):
+ *   out[r, n] = a_outer[r] * b_outer[e] * sum_k (qa*sfa)[r,k] * (qb*sfb)[e*N+n,k]
+ * accumulated in fp32; bf16 output is the round-to-nearest of the fp32 value.
+ *   A: NVFP4 [M_cap, K], sf MX_SF_MMA, outer per row
+ *   B: NVFP4 [E*N, K] (expert weight stack), sf MX_SF_MMA, outer per expert
+ *   out: [M_cap, N] f32 or bf16 (out_dtype); rows >= seg_offsets[E] untouched
+ * Requires K % 256 == 0, N % 128 == 0, M_cap % 128 == 0, 1 <= E.
+ * ------------------------------------------------------------------------ */
+MX_API int grouped_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_outer,
+                       const uint8_t* b_codes, const uint8_t* b_sf, const float* b_outer,
+                       const int64_t* seg_offsets, int64_t E, int64_t M_cap, int64_t N, int64_t K,
+                       void* out, int out_dtype, cudaStream_t stream);
+
+/* --------------------------------------------------------------------------
+ * grouped_gemm_mxfp8 -- backward expert GEMMs on tcgen05 block-scaled MMA.
+ * [ai-primer §Stochastic rounding across transposes]: gradients come from
+ * MXFP8 matrix multiplications of the re-quantised tensors.
+ * MX_GEMM_DGRAD (input gradient), contraction length K (the forward N):
+ *   A: MXFP8 [M_cap, K] (row-wise gradient), B: MXFP8 [N, E*K] (the
+ *   transposed weight stack; expert e = columns [e*K, (e+1)*K)),
+ *   out[r, n] = sum_k A[r,k] * B[n, e*K+k] for rows r of expert e; out [M_cap, N];
+ *   rows >= seg_offsets[E] untouched.
+ * MX_GEMM_WGRAD (weight gradient), contraction over each expert's tokens:
+ *   A: MXFP8 [N, M_cap], B: MXFP8 [K, M_cap] (column-wise forms),
+ *   out[e, n, k] = sum over t in segment e of A[n,t] * B[k,t]; out [E, N, K];
+ *   an empty expert gets zeros.
+ * All scales MX_SF_MMA.  Requires K % 128 == 0 and N % 128 == 0 (DGRAD);
+ * N % 128 == 0, K % 128 == 0, M_cap % 128 == 0 (WGRAD).
+ * ------------------------------------------------------------------------ */
+MX_API int grouped_gemm_mxfp8(int mode, const uint8_t* a_codes, const uint8_t* a_e8m0,
+                       const uint8_t* b_codes, const uint8_t* b_e8m0,
+                       const int64_t* seg_offsets, int64_t E, int64_t M_cap, int64_t N, int64_t K,
+                       void* out, int out_dtype, cudaStream_t stream);
+
+/* --------------------------------------------------------------------------
+ * Expert-layer glue (routing permutation, NVFP4 dispatch, SwiGLU, combine).
+ * [ai-primer §Quantized NVLink and BBBK]: tokens travel to their experts in
+ * NVFP4 and the backward pass reuses the quantised forward activations;
+ * [hermes §594B weights, 17B at work]: each token uses 8 of 384 experts.
+ * ------------------------------------------------------------------------ */
+
+/* Scratch bytes moe_route needs for T tokens and E experts. */
+MX_API size_t mx_route_workspace_bytes(int64_t T, int64_t E);
+
+/* moe_route -- top-k expert ids -> expert-major row order.
+ *   topk       device int32 [T, k], distinct ids in [0, E) per token
+ *   seg_offsets device int64 [E+1] out: segment starts, each segment padded
+ *              to a multiple of 128 rows
+ *   src        device int32 [M_cap] out: t*k + j of the assignment stored at
+ *              that row, -1 for padding rows and rows >= seg_offsets[E]
+ *   pos        device int32 [T, k] out: row of assignment (t, j)
+ *   workspace  device, mx_route_workspace_bytes(T, E) bytes of scratch
+ * Rows of one expert are in increasing token order.  M_cap must be at least
+ * T*k + 127*E rounded up to 128. */
+MX_API int moe_route(const int32_t* topk, int64_t T, int64_t k, int64_t E, int64_t M_cap,
+              int64_t* seg_offsets, int32_t* src, int32_t* pos,
+              void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* nvfp4_gather_rows -- dispatch per-token NVFP4 rows into expert-major order:
+ * row p of the output is row src[p]/k of the input (zeros when src[p] < 0).
+ * Input sf MX_SF_ROWMAJOR, output sf MX_SF_MMA.  Writes all M_cap rows.
+ * Requires cols % 64 == 0, M_cap % 128 == 0. */
+MX_API int nvfp4_gather_rows(const uint8_t* codes, const uint8_t* sf, const float* outer,
+                      const int32_t* src, int64_t k, int64_t M_cap, int64_t cols,
+                      uint8_t* out_codes, uint8_t* out_sf, float* out_outer, cudaStream_t stream);
+
+/* swiglu_fwd -- a = silu(g)*u (gated: g = h[:, :F], u = h[:, F:]) or
+ * a = silu(h) (not gated), fp32 math, bf16 round-to-nearest output.
+ *   h device bf16 [rows, 2F or F];  a device bf16 [rows, F]
+ * Rows >= *rows_valid (when rows_valid != NULL) are written as zero. */
+MX_API int swiglu_fwd(const void* h, int64_t rows, int64_t F, int gated, const int64_t* rows_valid,
+               void* a, cudaStream_t stream);
+
+/* swiglu_bwd -- dh from h and da (analytic derivative of swiglu_fwd). */
+MX_API int swiglu_bwd(const void* h, const void* da, int64_t rows, int64_t F, int gated,
+               const int64_t* rows_valid, void* dh, cudaStream_t stream);
+
+/* moe_combine -- out[t] = sum_j w[t,j] * y[pos[t,j]], fp32 accumulation,
+ * bf16 output.  y device bf16 [*, D], pos int32 [T, k], w f32 [T, k] (NULL:
+ * all weights 1). */
+MX_API int moe_combine(const void* y, const int32_t* pos, const float* w, int64_t T, int64_t k, int64_t D,
+                void* out, cudaStream_t stream);
+
+/* moe_dispatch_grad -- gradient of moe_combine w.r.t. y:
+ * dy[p] = w[src[p]] * dout[src[p]/k] (bf16), zero rows where src[p] < 0.
+ * Writes all M_cap rows. */
+MX_API int moe_dispatch_grad(const void* dout, const int32_t* src, const float* w, int64_t k,
+                      int64_t M_cap, int64_t D, void* dy, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MXMOE_H */

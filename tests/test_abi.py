@@ -1,0 +1,63 @@
+"""The C-ABI library loads and exports every symbol include/mxmoe.h declares,
+and rejects invalid arguments on the host before any launch (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "mxmoe.h")).read()
+    return re.findall(r"^MX_API\s+(?:int|size_t)\s+([a-z0-9_]+)\(", src, flags=re.M)
+
+
+@pytest.fixture(scope="module")
+def mx():
+    from fp8_moe_numerics_b200 import build, _lib
+    build.build()
+    return _lib.lib()
+
+
+def test_every_declared_symbol_is_exported(mx):
+    names = _declared()
+    assert len(names) >= 16
+    for n in names:
+        assert hasattr(mx, n), n
+    from fp8_moe_numerics_b200._lib import SIGNATURES
+    assert set(SIGNATURES) == set(names)
+
+
+def test_sizes_and_version(mx):
+    assert mx.mx_version() == 1
+    assert mx.mx_sf_bytes(256, 4096, 16, 1) == 256 * 256
+    assert mx.mx_sf_bytes(100, 4096, 16, 1) == 0          # MMA layout needs rows % 128
+    assert mx.mx_sf_bytes(100, 4096, 16, 0) == 100 * 256
+    assert mx.mx_sf_bytes(128, 96, 32, 1) == 0            # 3 scale columns: not a multiple of 4
+    assert mx.mx_route_workspace_bytes(32768, 384) == (128 * 384 + 384) * 4
+
+
+def test_invalid_arguments_are_rejected_before_launch(mx):
+    buf = (ctypes.c_uint8 * 4096)()
+    p = ctypes.cast(buf, ctypes.c_void_p)
+    null = ctypes.c_void_p(0)
+    EINVAL = 1
+    # null input
+    assert mx.nvfp4_quantize(null, 16, 64, 1, p, p, p, 0, null) == EINVAL
+    # cols not a multiple of 16
+    assert mx.nvfp4_quantize(p, 16, 40, 1, p, p, p, 0, null) == EINVAL
+    # MMA layout with rows % 128 != 0
+    assert mx.nvfp4_quantize(p, 16, 64, 1, p, p, p, 1, null) == EINVAL
+    # misaligned input pointer
+    assert mx.nvfp4_quantize(ctypes.c_void_p(ctypes.addressof(buf) + 1), 16, 64, 1, p, p, p, 0, null) == EINVAL
+    # bad rbits
+    assert mx.mxfp8_requant_transpose_sr(p, p, p, 128, 64, 1, 0, null, 0, 0, 7, p, p, 0, null) == EINVAL
+    # K not a multiple of 256 for the NVFP4 GEMM
+    assert mx.grouped_gemm_nvfp4(p, p, p, p, p, p, p, 1, 128, 256, 128, p, 0, null) == EINVAL
+    # unknown GEMM mode
+    assert mx.grouped_gemm_mxfp8(5, p, p, p, p, p, 1, 128, 128, 128, p, 0, null) == EINVAL
+    # routing capacity too small
+    assert mx.moe_route(p, 16, 2, 4, 128, p, p, p, p, 4096, null) == EINVAL

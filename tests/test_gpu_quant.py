@@ -1,0 +1,267 @@
+"""GPU parity of the quantisers, the stochastic requantisation and the glue
+kernels against the CPU oracle, through the C ABI.
+
+Bar: bit-exact codes, scales, outer scales, permutations; SwiGLU / combine
+within one bf16 rounding (the oracle computes them in fp64).  All inputs are
+seeded and synthetic; every expected value comes from the oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from fp8_moe_numerics_b200 import api, workloads
+from tests.layouts import mma_to_rowmajor, rowmajor_to_mma
+
+pytestmark = pytest.mark.gpu
+
+
+def to_dev_bf16(u16: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(u16).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def to_np_u16(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+def np_(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().numpy()
+
+
+def heavy_rows(rows, cols, seed, nu=4, spread=3.0):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_t(nu, (rows, cols)) * 10.0 ** rng.uniform(-spread, spread, (rows, 1))
+    return oracle.f32_to_bf16(x.astype(np.float32))
+
+
+def crafted_rows():
+    """Rows whose blocks land exactly on E2M1 and E4M3 rounding ties, zero
+    blocks, zero rows, negative zeros and saturating values."""
+    rows = []
+    ties_e2m1 = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 6.0], np.float64)
+    # outer scale 1 (row max 2688); a block with max 1536 gets sf = 256 exactly,
+    # so x/(sf*s) = x/256 is exact and elements 256*tie are exact ties
+    r = np.zeros(256, np.float64)
+    r[0] = 2688.0
+    blk = np.concatenate([ties_e2m1, -ties_e2m1]) * 256.0
+    blk[7] = 1536.0
+    r[16:32] = blk
+    r[32:48] = -blk
+    # E4M3 ties on the block scale: block max 6 * midpoint, s = 1
+    e4 = np.abs(np.arange(0x7F, dtype=np.uint8).view(__import__("ml_dtypes").float8_e4m3fn).astype(np.float64))
+    mids = (e4[1:] + e4[:-1]) / 2
+    for i, m in enumerate(mids[[0, 5, 20, 60, 100, 120]]):
+        r[64 + 16 * i] = 6.0 * m
+    r[200:216] = -0.0
+    rows.append(r)
+    rows.append(np.zeros(256))
+    rr = np.zeros(256); rr[5] = -1e-30; rr[6] = 3e-39; rows.append(rr)   # tiny / subnormal-range values
+    return oracle.f32_to_bf16(np.array(rows, np.float32))
+
+
+# ---------------------------------------------------------------------------
+# NVFP4 quantiser
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("rows,cols", [(256, 4096), (128, 1024), (384, 256), (7, 48), (130, 3072)])
+def test_nvfp4_quantize_per_token_bit_exact(cuda, rows, cols):
+    x = heavy_rows(rows, cols, seed=rows + cols)
+    codes, sf, outer = oracle.nvfp4_quantize(x)
+    xd = to_dev_bf16(x)
+    gc, gsf, go = api.nvfp4_quantize(xd, sf_layout=api.MX_SF_ROWMAJOR)
+    torch.cuda.synchronize()
+    assert np.array_equal(np_(gc), codes)
+    assert np.array_equal(np_(gsf).reshape(rows, cols // 16), sf)
+    assert np.array_equal(np_(go).view(np.uint32), outer.view(np.uint32))
+    if rows % 128 == 0 and cols % 64 == 0:
+        gc2, gsf2, go2 = api.nvfp4_quantize(xd, sf_layout=api.MX_SF_MMA)
+        assert np.array_equal(np_(gc2), codes)
+        assert np.array_equal(mma_to_rowmajor(np_(gsf2), rows, cols // 16), sf)
+
+
+def test_nvfp4_quantize_crafted_ties_and_zeros(cuda):
+    x = crafted_rows()
+    codes, sf, outer = oracle.nvfp4_quantize(x)
+    gc, gsf, go = api.nvfp4_quantize(to_dev_bf16(x), sf_layout=api.MX_SF_ROWMAJOR)
+    assert np.array_equal(np_(gc), codes)
+    assert np.array_equal(np_(gsf).reshape(sf.shape), sf)
+    assert np.array_equal(np_(go).view(np.uint32), outer.view(np.uint32))
+
+
+@pytest.mark.parametrize("E,N,K", [(4, 128, 256), (3, 256, 512), (2, 128, 4096)])
+def test_nvfp4_quantize_per_expert_bit_exact(cuda, E, N, K):
+    w = workloads.weights(E, N, K, 0.02, seed=E * N + K)
+    wn = w.reshape(E * N, K).view(torch.int16).numpy().view(np.uint16)
+    codes, sf, outer = oracle.nvfp4_quantize(wn, group_rows=N)
+    gc, gsf, go = api.nvfp4_quantize(w.reshape(E * N, K).cuda(), group_rows=N, sf_layout=api.MX_SF_MMA)
+    assert np.array_equal(np_(gc), codes)
+    assert np.array_equal(mma_to_rowmajor(np_(gsf), E * N, K // 16), sf)
+    assert np.array_equal(np_(go).view(np.uint32), outer.view(np.uint32))
+
+
+# ---------------------------------------------------------------------------
+# MXFP8 quantiser
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("rounding", [api.MX_ROUND_RNE, api.MX_ROUND_SR])
+@pytest.mark.parametrize("rows,cols", [(128, 128), (256, 384), (512, 1024)])
+def test_mxfp8_quantize_rows_and_cols_bit_exact(cuda, rows, cols, rounding):
+    x = heavy_rows(rows, cols, seed=3 * rows + cols, spread=6.0)
+    sr = rounding == api.MX_ROUND_SR
+    seed, stream = 0xDEADBEEF12345, 7
+    rc, re = oracle.mxfp8_quantize_rows(x, sr=sr, seed=seed, stream=stream, R=8)
+    cc, ce = oracle.mxfp8_quantize_cols(x, sr=sr, seed=seed, stream=stream + 1, R=8)
+    for layout in (api.MX_SF_ROWMAJOR, api.MX_SF_MMA):
+        g = api.mxfp8_quantize(to_dev_bf16(x), rounding=rounding, seed=seed, stream_id=stream, rbits=8,
+                               sf_layout=layout)
+        assert np.array_equal(np_(g[0]), rc)
+        assert np.array_equal(np_(g[2]), cc)
+        if layout == api.MX_SF_ROWMAJOR:
+            assert np.array_equal(np_(g[1]).reshape(re.shape), re)
+            assert np.array_equal(np_(g[3]).reshape(ce.shape), ce)
+        else:
+            assert np.array_equal(mma_to_rowmajor(np_(g[1]), rows, cols // 32), re)
+            assert np.array_equal(mma_to_rowmajor(np_(g[3]), cols, rows // 32), ce)
+
+
+def test_mxfp8_quantize_column_only_and_rows_valid(cuda):
+    rows, cols = 384, 256
+    x = heavy_rows(rows, cols, seed=11)
+    cc, ce = oracle.mxfp8_quantize_cols(x[:256])
+    valid = torch.tensor([256], dtype=torch.int64, device="cuda")
+    out = (None, None, torch.full((cols, rows), 0xAB, dtype=torch.uint8, device="cuda"),
+           torch.full((cols * rows // 32,), 0xAB, dtype=torch.uint8, device="cuda"))
+    g = api.mxfp8_quantize(to_dev_bf16(x), row=False, col=True, rows_valid=valid, sf_layout=api.MX_SF_ROWMAJOR,
+                           out=out)
+    gc = np_(g[2])
+    assert np.array_equal(gc[:, :256], cc)
+    assert np.all(gc[:, 256:] == 0xAB)              # rows beyond rows_valid untouched
+
+
+# ---------------------------------------------------------------------------
+# Requantisation across the transpose
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("R", [8, 16, 32])
+@pytest.mark.parametrize("rows,cols", [(128, 64), (256, 512), (512, 4096)])
+def test_requant_transpose_sr_bit_exact(cuda, rows, cols, R):
+    x = heavy_rows(rows, cols, seed=rows * 7 + cols + R)
+    codes, sf, outer = oracle.nvfp4_quantize(x)
+    seed, stream = 0x0123456789ABCDEF, 0xFEDCBA98
+    oc, oe = oracle.mxfp8_requant_transpose_sr(codes, sf, outer, 1, seed, stream, R)
+    dc = torch.from_numpy(codes).cuda()
+    do = torch.from_numpy(outer).cuda()
+    for lin in (api.MX_SF_ROWMAJOR, api.MX_SF_MMA):
+        if lin == api.MX_SF_MMA and (rows % 128 or cols % 64):
+            continue
+        dsf = torch.from_numpy(sf.reshape(-1).copy() if lin == api.MX_SF_ROWMAJOR else rowmajor_to_mma(sf)).cuda()
+        for lout in (api.MX_SF_ROWMAJOR, api.MX_SF_MMA):
+            if lout == api.MX_SF_MMA and cols % 128:
+                continue
+            gc, ge = api.mxfp8_requant_transpose_sr(dc, dsf, do, rows, cols, 1, lin, None, seed, stream, R, lout)
+            assert np.array_equal(np_(gc), oc)
+            ge = np_(ge)
+            got_e = ge.reshape(oe.shape) if lout == api.MX_SF_ROWMAJOR else mma_to_rowmajor(ge, cols, rows // 32)
+            assert np.array_equal(got_e, oe)
+
+
+def test_requant_weights_per_expert_outer(cuda):
+    E, N, K = 3, 128, 256
+    w = workloads.weights(E, N, K, 0.02, seed=5).reshape(E * N, K).view(torch.int16).numpy().view(np.uint16)
+    codes, sf, outer = oracle.nvfp4_quantize(w, group_rows=N)
+    oc, oe = oracle.mxfp8_requant_transpose_sr(codes, sf, outer, N, 3, 4, 8)
+    gc, ge = api.mxfp8_requant_transpose_sr(torch.from_numpy(codes).cuda(), torch.from_numpy(rowmajor_to_mma(sf)).cuda(),
+                                            torch.from_numpy(outer).cuda(), E * N, K, N, api.MX_SF_MMA, None, 3, 4, 8,
+                                            api.MX_SF_MMA)
+    assert np.array_equal(np_(gc), oc)
+    assert np.array_equal(mma_to_rowmajor(np_(ge), K, E * N // 32), oe)
+
+
+def test_requant_crafted_values(cuda):
+    # the crafted row (ties, zeros, -0) repeated with power-of-two row scales
+    base = oracle.bf16_to_f32(crafted_rows()[0:1, :128]).astype(np.float64)
+    x = oracle.f32_to_bf16((np.repeat(base, 128, 0) * 2.0 ** (np.arange(128) % 7 - 3)[:, None]).astype(np.float32))
+    codes, sf, outer = oracle.nvfp4_quantize(x)
+    oc, oe = oracle.mxfp8_requant_transpose_sr(codes, sf, outer, 1, 9, 9, 8)
+    gc, ge = api.mxfp8_requant_transpose_sr(torch.from_numpy(codes).cuda(), torch.from_numpy(sf.reshape(-1).copy()).cuda(),
+                                            torch.from_numpy(outer).cuda(), 128, 128, 1, api.MX_SF_ROWMAJOR, None, 9, 9, 8,
+                                            api.MX_SF_ROWMAJOR)
+    assert np.array_equal(np_(gc), oc)
+    assert np.array_equal(np_(ge).reshape(oe.shape), oe)
+
+
+# ---------------------------------------------------------------------------
+# Glue
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("T,k,E,kind,n_empty", [(256, 2, 4, "uniform", 0), (1000, 8, 64, "zipf", 3),
+                                                (3000, 8, 384, "zipf", 8), (5, 3, 7, "uniform", 0)])
+def test_route_gather_bit_exact(cuda, T, k, E, kind, n_empty):
+    ids = workloads.routing(T, k, E, kind, 1.2, n_empty, seed=T + E)
+    seg, src, pos = oracle.route(ids.numpy(), E)
+    M_cap = api.max_routed_rows(T, k, E)
+    gseg, gsrc, gpos = api.moe_route(ids.cuda(), E, M_cap)
+    gseg, gsrc, gpos = np_(gseg), np_(gsrc), np_(gpos)
+    assert np.array_equal(gseg, seg)
+    assert np.array_equal(gpos, pos)
+    Mp = int(seg[-1])
+    # the ABI stores the assignment index t*k + j; the oracle stores the token
+    flat = np.full(Mp, -1, np.int64)
+    flat[pos.reshape(-1)] = np.arange(T * k)
+    assert np.array_equal(gsrc[:Mp], flat)
+    assert np.all(gsrc[Mp:] == -1)
+    assert np.array_equal(np.where(flat >= 0, flat // k, -1), src)
+    # NVFP4 dispatch: gather the per-token rows
+    D = 256
+    x = heavy_rows(T, D, seed=T)
+    codes, sf, outer = oracle.nvfp4_quantize(x)
+    oc, osf, oo = oracle.gather_nvfp4_rows(codes, sf, outer, src)
+    gc, gsf, go = api.nvfp4_gather_rows(torch.from_numpy(codes).cuda(), torch.from_numpy(sf.reshape(-1).copy()).cuda(),
+                                        torch.from_numpy(outer).cuda(), torch.from_numpy(gsrc).cuda(), k, D)
+    gc, gsf, go = np_(gc), np_(gsf), np_(go)
+    assert np.array_equal(gc[:Mp], oc)
+    assert np.array_equal(mma_to_rowmajor(gsf, M_cap, D // 16)[:Mp], osf)
+    assert np.array_equal(go[:Mp].view(np.uint32), oo.view(np.uint32))
+    assert np.all(gc[Mp:] == 0) and np.all(go[Mp:] == 0)
+
+
+def _ulp_close(got_u16, ref_u16):
+    g = oracle.bf16_to_f32(got_u16).astype(np.float64)
+    r = oracle.bf16_to_f32(ref_u16).astype(np.float64)
+    tol = np.maximum(np.abs(r), 1e-30) * 2.0 ** -7
+    return np.all(np.abs(g - r) <= tol)
+
+
+@pytest.mark.parametrize("gated", [True, False])
+def test_swiglu_fwd_bwd_within_one_rounding(cuda, gated):
+    rows, F = 256, 512
+    rng = np.random.default_rng(3)
+    h = oracle.f32_to_bf16((rng.standard_normal((rows, 2 * F if gated else F)) * 3).astype(np.float32))
+    da = oracle.f32_to_bf16(rng.standard_normal((rows, F)).astype(np.float32))
+    a = oracle.swiglu_fwd(h, gated)
+    dh = oracle.swiglu_bwd(h, da, gated)
+    valid = torch.tensor([128], dtype=torch.int64, device="cuda")
+    ga = to_np_u16(api.swiglu_fwd(to_dev_bf16(h), F, gated, rows_valid=valid))
+    gdh = to_np_u16(api.swiglu_bwd(to_dev_bf16(h), to_dev_bf16(da), F, gated, rows_valid=valid))
+    assert _ulp_close(ga[:128], a[:128]) and np.all(ga[128:] == 0)
+    assert _ulp_close(gdh[:128], dh[:128]) and np.all(gdh[128:] == 0)
+
+
+def test_combine_and_dispatch_grad(cuda):
+    T, k, E, D = 300, 4, 16, 256
+    ids = workloads.routing(T, k, E, "zipf", 1.1, 0, seed=2)
+    seg, src, pos = oracle.route(ids.numpy(), E)
+    M = int(seg[-1])
+    rng = np.random.default_rng(4)
+    y = oracle.f32_to_bf16(rng.standard_normal((M, D)).astype(np.float32))
+    w = np.full((T, k), 1.0 / k, np.float32)
+    ref = oracle.combine(y, pos, w)
+    got = to_np_u16(api.moe_combine(to_dev_bf16(y), torch.from_numpy(pos).cuda(), torch.from_numpy(w).cuda(), D))
+    assert _ulp_close(got, ref)
+    dout = oracle.f32_to_bf16(rng.standard_normal((T, D)).astype(np.float32))
+    ref_dy = oracle.dispatch_grad(dout, pos, w, M)
+    M_cap = api.max_routed_rows(T, k, E)
+    _, gsrc, _ = api.moe_route(ids.cuda(), E, M_cap)
+    gdy = to_np_u16(api.moe_dispatch_grad(to_dev_bf16(dout), gsrc, torch.from_numpy(w).cuda(), k))
+    assert np.array_equal(gdy[:M], ref_dy)
+    assert np.all(gdy[M:] == 0)
