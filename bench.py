@@ -169,6 +169,7 @@ def stage_work(c, counts, M_pad):
     f_g2 = 2 * R * D * F
     w = {
         # name: (kind, work)  kind: "tensor4" / "tensor8" flops, "hbm" bytes
+        "route": ("hbm", T * k * 4 * 2 + (T * k + 127 * E) * 4),
         "quant_x": ("hbm", T * D * 2 + nv(T, D)),
         "gather": ("hbm", 2 * nv(R, D)),
         "quant_w": ("hbm", E * N1 * D * 2 + nv(E * N1, D) + E * D * F * 2 + nv(E * D, F)),
@@ -212,8 +213,6 @@ def run_ours(args):
     # each rank draws its own tokens (weak scaling); weights are shared seeds
     inp = workloads.layer_inputs(WORKLOAD, device=dev)
     if rank:
-        g = torch.Generator(device=dev)
-        g.manual_seed(c["seed"] + 17 * rank)
         inp["x"] = workloads.activations(c["T"], c["D"], c["x_dist"], c["seed"] + 1 + 1000 * rank, dev)
     topk = inp["topk"].to(dev)
     counts = torch.bincount(inp["topk"].reshape(-1).long(), minlength=c["E"]).tolist()
@@ -401,8 +400,9 @@ def cpu_baseline(inp, layer, seconds: float = 15.0):
     rows against one expert's W1 tile, until ~`seconds` of CPU work."""
     import numpy as np
     import oracle
-    x = inp["x"][:256].cpu().view(np.int16) if False else inp["x"][:256].cpu().view(__import__("torch").int16).numpy().view(np.uint16)
-    w = inp["w1"][0, :256].cpu().view(__import__("torch").int16).numpy().view(np.uint16)
+    import torch
+    x = inp["x"][:256].cpu().view(torch.int16).numpy().view(np.uint16)
+    w = inp["w1"][0, :256].cpu().view(torch.int16).numpy().view(np.uint16)
     D = x.shape[1]
     N = w.shape[0]
     flops = 0

@@ -50,7 +50,7 @@ class ExpertLayer:
         assert self.N1 == (2 * self.F if gated else self.F)
         self.seed, self.rbits = seed, rbits
         self.x, self.topk, self.w_comb, self.w1, self.w2, self.dout = x, topk, w_comb, w1, w2, dout
-        T, D, k, E, F, N1 = self.T, D, self.k, self.E, self.F, self.N1
+        T, D, k, E, F, N1 = self.T, self.D, self.k, self.E, self.F, self.N1
         self.M_cap = M = api.max_routed_rows(T, k, E)
         e = lambda *s, dt=torch.uint8: torch.empty(*s, dtype=dt, device=dev)
         sfb = api.sf_bytes

@@ -1,0 +1,50 @@
+"""Host-side check of the expert-layer call sequence (no GPU).
+
+ExpertLayer is run on CPU tensors with the binding's pointer check relaxed:
+every call reaches the real C library, whose argument validation runs on the
+host before the device check.  Valid arguments therefore return MX_ECUDA (no
+CUDA device here), invalid ones MX_EINVAL -- so each call's shapes, strides,
+alignment and sizes are checked against the ABI contract.
+"""
+import ctypes
+
+import pytest
+import torch
+
+from fp8_moe_numerics_b200 import _lib, api, workloads
+from fp8_moe_numerics_b200.layer import ExpertLayer
+
+
+@pytest.fixture
+def host_calls(monkeypatch):
+    from fp8_moe_numerics_b200 import build
+    build.build()
+    calls = []
+
+    def p(t):
+        return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+    def call(name, *args):
+        st = getattr(_lib.lib(), name)(*args)
+        calls.append((name, st))
+        assert st != _lib.MX_EINVAL, f"{name} rejected its arguments"
+
+    monkeypatch.setattr(api, "_p", p)
+    monkeypatch.setattr(api, "_s", lambda: ctypes.c_void_p(0))
+    monkeypatch.setattr(_lib, "call", call)
+    monkeypatch.setattr(api.L, "call", call)
+    return calls
+
+
+@pytest.mark.parametrize("name", ["tiny_layer"])
+def test_layer_sequence_passes_host_validation(host_calls, name):
+    inp = workloads.layer_inputs(name, device="cpu")
+    c = inp["cfg"]
+    L = ExpertLayer(inp["x"], inp["topk"], inp["w_comb"], inp["w1"], inp["w2"], inp["dout"], gated=c["gated"])
+    L.step()
+    names = [n for n, _ in host_calls]
+    assert names[0] == "moe_route" and names[-1] == "moe_combine"
+    assert names.count("grouped_gemm_nvfp4") == 2 and names.count("grouped_gemm_mxfp8") == 4
+    assert names.count("mxfp8_requant_transpose_sr") == 4
+    assert len(names) == 23
+    assert all(st == _lib.MX_ECUDA for _, st in host_calls)   # valid, and no device here
