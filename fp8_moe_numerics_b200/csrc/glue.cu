@@ -7,6 +7,8 @@
 // quantised once and gathered into expert-major order.
 #include "mx_common.cuh"
 
+#include <mutex>
+
 namespace {
 
 constexpr int kChunk = 256;   // tokens per routing chunk
@@ -313,4 +315,58 @@ extern "C" int moe_dispatch_grad(const void* dout, const int32_t* src, const flo
     dispatch_grad_kernel<<<(unsigned)M_cap, 128, 0, stream>>>(static_cast<const uint16_t*>(dout), src, w, k, D,
                                                               static_cast<uint16_t*>(dy));
     return mx_launch_status();
+}
+
+// ===========================================================================
+// moe_route_static -- moe_route for callers that cannot allocate device memory
+// ===========================================================================
+// Some callers cannot hand this library a scratch buffer: code running inside
+// a custom allocator or memory-pool callback, or an embedding runtime that owns
+// every device allocation and forbids new ones.  For them the routing scratch
+// (per-chunk expert histograms and per-expert counts) lives in this fixed
+// array, part of the library's device image: every GPU that loads the library
+// holds these bytes until the process exits.
+//
+// Every word of the scratch that a call reads is written earlier in the same
+// call, so nothing has to be cleared between calls.  Calls share the array:
+// two calls that may run at the same time on the GPU (different streams, or
+// different host threads, without ordering between them) race on it and give
+// undefined results.
+namespace {
+
+constexpr size_t kRouteStaticScratchBytes = size_t(1) << 20;   // 1 MiB
+static __device__ __align__(256) int32_t g_route_scratch[kRouteStaticScratchBytes / sizeof(int32_t)];
+
+std::mutex g_route_scratch_mutex;
+void* g_route_scratch_ptr[64] = {nullptr};
+
+// Device address of the scratch array on the current device, looked up once
+// per device (the array's host-side name is not a device address).
+int route_scratch_address(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return mx_set_cuda_error(e);
+    if (dev < 0 || dev >= 64) return MX_EUNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_route_scratch_mutex);
+    if (!g_route_scratch_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_route_scratch);
+        if (e != cudaSuccess || !p) return mx_set_cuda_error(e != cudaSuccess ? e : cudaErrorInvalidSymbol);
+        g_route_scratch_ptr[dev] = p;
+    }
+    *out = g_route_scratch_ptr[dev];
+    return MX_OK;
+}
+
+}  // namespace
+
+extern "C" int moe_route_static(const int32_t* topk, int64_t T, int64_t k, int64_t E, int64_t M_cap,
+                                int64_t* seg_offsets, int32_t* src, int32_t* pos, cudaStream_t stream) {
+    if (!topk || !seg_offsets || !src || !pos || T < 0 || k <= 0 || k > 32 || E <= 0 || M_cap < 0 || M_cap % 128)
+        return MX_EINVAL;
+    if (mx_route_workspace_bytes(T, E) > kRouteStaticScratchBytes) return MX_EINVAL;   // beyond the fixed scratch
+    if (int st = mx_check_device()) return st;
+    void* scratch = nullptr;
+    if (int st = route_scratch_address(&scratch)) return st;
+    return moe_route(topk, T, k, E, M_cap, seg_offsets, src, pos, scratch, kRouteStaticScratchBytes, stream);
 }

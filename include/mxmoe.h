@@ -209,6 +209,22 @@ MX_API int moe_route(const int32_t* topk, int64_t T, int64_t k, int64_t E, int64
               int64_t* seg_offsets, int32_t* src, int32_t* pos,
               void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* moe_route_static -- moe_route without a caller-provided workspace.
+ * The pages describe nothing like this; it exists for callers that cannot
+ * allocate device memory for scratch (for example code running inside an
+ * allocator or memory-pool callback, or a host runtime that owns every device
+ * allocation).  The scratch is a fixed 1 MiB array inside the library's device
+ * image, held by every GPU that loads the library until the process exits.
+ * Arguments and outputs are those of moe_route.  Returns MX_EINVAL when
+ * mx_route_workspace_bytes(T, E) exceeds 1 MiB.  Allocates nothing and frees
+ * nothing.  The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * Every call uses the same array, and each call writes every scratch word it
+ * reads, so no clearing is needed; calls that can overlap on the GPU (other
+ * streams, other host threads) race on the array and give undefined results. */
+MX_API int moe_route_static(const int32_t* topk, int64_t T, int64_t k, int64_t E, int64_t M_cap,
+                            int64_t* seg_offsets, int32_t* src, int32_t* pos, cudaStream_t stream);
+
 /* nvfp4_gather_rows -- dispatch per-token NVFP4 rows into expert-major order:
  * row p of the output is row src[p]/k of the input (zeros when src[p] < 0).
  * Input sf MX_SF_ROWMAJOR, output sf MX_SF_MMA.  Writes all M_cap rows.
