@@ -71,7 +71,7 @@ def nvfp4_quantize(x: torch.Tensor, group_rows: int = 1, sf_layout: int = MX_SF_
 
 def mxfp8_requant_transpose_sr(codes, sf, outer, rows: int, cols: int, group_rows: int = 1,
                                in_sf_layout: int = MX_SF_MMA, rows_valid=None, seed: int = 0, stream_id: int = 0,
-                               rbits: int = 8, out_sf_layout: int = MX_SF_MMA, out=None):
+                               rbits: int = 16, out_sf_layout: int = MX_SF_MMA, out=None):
     """Saved NVFP4 [rows, cols] -> MXFP8 [cols, rows] codes and E8M0 scales."""
     dev = codes.device
     if out is None:
@@ -84,7 +84,7 @@ def mxfp8_requant_transpose_sr(codes, sf, outer, rows: int, cols: int, group_row
 
 
 def mxfp8_quantize(x: torch.Tensor, row: bool = True, col: bool = True, rounding: int = MX_ROUND_RNE,
-                   seed: int = 0, stream_id: int = 0, rbits: int = 8, rows_valid=None,
+                   seed: int = 0, stream_id: int = 0, rbits: int = 16, rows_valid=None,
                    sf_layout: int = MX_SF_MMA, out=None):
     """bf16 [rows, cols] -> (row codes [rows, cols], row E8M0, col codes [cols, rows], col E8M0);
     the forms not requested are None."""

@@ -114,29 +114,88 @@ __device__ __forceinline__ float exp2_neg(int e) {
 // u < floor(rem * 2^R / 2^sh).  The E4M3 code of units * 2^Q is
 // (Q + 9) * 8 + units for every Q >= -9 (codes are monotone in magnitude, so a
 // carry into the next binade is the next code).  Caller guarantees |y| <= 448.
+//
+// Fast path: xh normal and y >= 2^-6 (E4M3 normal range) means sh = 20, so
+// the code is the top 11 magnitude bits of xh re-biased, plus the carry
+// decided by the top R of the 20 dropped bits.  `sr_block` precomputes the
+// per-block constants.
 // ---------------------------------------------------------------------------
+struct SrBlock {
+    int lo_eb;        // smallest fp32 biased exponent taking the fast path
+    uint32_t off;     // (e + 120) << 3
+    int e;
+};
+
+__device__ __forceinline__ SrBlock sr_block(int e) {
+    SrBlock b;
+    b.lo_eb = max(1, e + 121);
+    b.off = (uint32_t)(e + 120) << 3;
+    b.e = e;
+    return b;
+}
+
 template <int R>
-__device__ __forceinline__ uint32_t e4m3_sr_code(float xh, int e, uint32_t u) {
-    uint32_t bits = __float_as_uint(xh);
-    uint32_t sign = (bits >> 24) & 0x80u;
-    uint32_t mag = bits & 0x7fffffffu;
-    if (mag == 0) return sign;
-    uint32_t eb = mag >> 23;
-    uint32_t M = eb ? ((mag & 0x7fffffu) | 0x800000u) : mag;
-    int p = (eb ? (int)eb - 150 : -149) - e;     // exponent of M's unit bit in y
-    int fl = p + (31 - __clz(M));                // floor(log2 y)
-    int Q = fl - 3 < -9 ? -9 : fl - 3;
-    int sh = Q - p;
+__device__ __noinline__ uint32_t e4m3_sr_general(uint32_t mag, int e, uint32_t u) {
+    if (mag == 0) return 0u;
+    const uint32_t eb = mag >> 23;
+    const uint32_t M = eb ? ((mag & 0x7fffffu) | 0x800000u) : mag;
+    const int p = (eb ? (int)eb - 150 : -149) - e;     // exponent of M's unit bit in y
+    const int fl = p + (31 - __clz(M));                // floor(log2 y)
+    const int Q = fl - 3 < -9 ? -9 : fl - 3;
+    const int sh = Q - p;                              // >= -3
     uint32_t units;
     if (sh <= 0) {
-        units = M << (-sh);                      // on the grid already
+        units = M << (-sh);                            // on the grid already
     } else {
-        uint32_t lo = sh >= 32 ? 0u : (M >> sh);
-        uint64_t rem = sh >= 32 ? (uint64_t)M : (uint64_t)(M & ((1u << sh) - 1u));
-        uint64_t thr = sh >= 64 ? 0ull : ((rem << R) >> sh);
-        units = lo + ((uint64_t)u < thr ? 1u : 0u);
+        const uint32_t lo = sh >= 32 ? 0u : (M >> sh);
+        const uint32_t rem = sh >= 32 ? M : (M & ((1u << sh) - 1u));
+        uint32_t thr;
+        if (sh >= R) {
+            const int d = sh - R;
+            thr = d >= 32 ? 0u : (rem >> d);
+        } else {
+            thr = rem << (R - sh);                     // rem < 2^sh, so < 2^R
+        }
+        units = lo + (u < thr ? 1u : 0u);
     }
-    return sign | (uint32_t)((Q + 9) * 8 + (int)units);
+    return (uint32_t)((Q + 9) * 8 + (int)units);
+}
+
+template <int R>
+__device__ __forceinline__ uint32_t e4m3_sr_code(float xh, const SrBlock& b, uint32_t u) {
+    const uint32_t bits = __float_as_uint(xh);
+    const uint32_t sign = (bits >> 24) & 0x80u;
+    const uint32_t mag = bits & 0x7fffffffu;
+    const uint32_t rem = mag & 0xfffffu;
+    const uint32_t thr = R <= 20 ? (rem >> (20 - R)) : (rem << (R - 20));
+    uint32_t code = (mag >> 20) - b.off + (u < thr ? 1u : 0u);
+    if ((int)(mag >> 23) < b.lo_eb) code = e4m3_sr_general<R>(mag, b.e, u);
+    return sign | code;
+}
+
+template <int R>
+__device__ __forceinline__ uint32_t e4m3_sr_code(float xh, int e, uint32_t u) {
+    return e4m3_sr_code<R>(xh, sr_block(e), u);
+}
+
+// ---------------------------------------------------------------------------
+// Hardware stochastic rounding (sm_100a cvt.rs) of two values onto E4M3.
+// cvt.rs.satfinite.e4m3x4.f32 d, {a, b, c, f}, rbits puts f's code in byte 0
+// and b's in byte 2; f adds rbits[15:0] and b adds rbits[31:16] as 16 random
+// bits just below the kept E4M3 bits and truncates (the carry rounds up).  With
+// u the 16-bit value of the stream, feeding 0xFFFF - u rounds up exactly when
+// u < floor(frac * 2^16): the rule of e4m3_sr_code<16>, in one instruction
+// (established by comparing the instruction with the oracle on a B200).  The
+// a and c lanes are not used: their random bits are not independent of b's
+// and f's.  y_lo / y_hi must be |y| <= 448; the result packs lo in bits 0-7
+// and hi in bits 8-15.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t cvt_rs16_e4m3_pair(float y_lo, float y_hi, uint32_t u_lo, uint32_t u_hi) {
+    const uint32_t rbits = ~((u_hi << 16) | (u_lo & 0xffffu));
+    uint32_t d;
+    asm("cvt.rs.satfinite.e4m3x4.f32 %0, {%1, %2, %3, %4}, %5;"
+        : "=r"(d) : "f"(0.0f), "f"(y_hi), "f"(0.0f), "f"(y_lo), "r"(rbits));
+    return (d & 0xffu) | ((d >> 8) & 0xff00u);
 }
 
 // ---------------------------------------------------------------------------
@@ -147,14 +206,14 @@ __device__ __forceinline__ uint32_t e4m3_sr_code(float xh, int e, uint32_t u) {
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint4 philox4x32_10(uint64_t g, uint64_t stream, uint64_t seed) {
     uint32_t c0 = (uint32_t)g, c1 = (uint32_t)(g >> 32), c2 = (uint32_t)stream, c3 = (uint32_t)(stream >> 32);
-    uint32_t k0 = (uint32_t)seed, k1 = (uint32_t)(seed >> 32);
+    const uint32_t k0 = (uint32_t)seed, k1 = (uint32_t)(seed >> 32);
 #pragma unroll
     for (int r = 0; r < 10; ++r) {
-        uint32_t hi0 = __umulhi(0xD2511F53u, c0), lo0 = 0xD2511F53u * c0;
-        uint32_t hi1 = __umulhi(0xCD9E8D57u, c2), lo1 = 0xCD9E8D57u * c2;
-        uint32_t n0 = hi1 ^ c1 ^ k0, n2 = hi0 ^ c3 ^ k1;
-        c0 = n0; c1 = lo1; c2 = n2; c3 = lo0;
-        k0 += 0x9E3779B9u; k1 += 0xBB67AE85u;
+        const uint64_t p0 = (uint64_t)0xD2511F53u * c0;         // one 32x32->64 multiply each
+        const uint64_t p1 = (uint64_t)0xCD9E8D57u * c2;
+        const uint32_t n0 = (uint32_t)(p1 >> 32) ^ c1 ^ (k0 + (uint32_t)r * 0x9E3779B9u);
+        const uint32_t n2 = (uint32_t)(p0 >> 32) ^ c3 ^ (k1 + (uint32_t)r * 0xBB67AE85u);
+        c0 = n0; c1 = (uint32_t)p1; c2 = n2; c3 = (uint32_t)p0;
     }
     return make_uint4(c0, c1, c2, c3);
 }

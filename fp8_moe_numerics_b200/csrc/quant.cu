@@ -106,34 +106,40 @@ nvfp4_quant_rows_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t co
 }
 
 // amax over each group of rows, as fp32 bits, atomically max-ed into outer[g]
-// (pre-zeroed).  Grid-stride over 16-element blocks.
-__global__ void nvfp4_group_amax_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols,
-                                        int64_t group_rows, float* __restrict__ outer) {
-    const int64_t nblk_row = cols >> 4;
-    const int64_t total = rows * nblk_row;
-    const uint4* xv = reinterpret_cast<const uint4*>(x);
-    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    // consecutive threads take consecutive blocks; a warp's blocks usually
-    // share a group, so reduce inside the warp before the atomic
-    for (int64_t base = i - threadIdx.x % 32; base < total; base += stride) {
-        int64_t blk = base + (threadIdx.x % 32);
-        uint32_t m = 0;
-        int64_t g = -1;
-        if (blk < total) {
-            m = max(absmax8_bf16(__ldcs(xv + 2 * blk)), absmax8_bf16(__ldcs(xv + 2 * blk + 1)));
-            g = (blk / nblk_row) / group_rows;
+// (pre-zeroed).  blockIdx.y = group, blockIdx.x = chunk of the group's
+// contiguous elements; each thread keeps four 16-byte loads in flight and the
+// block issues one atomic.
+constexpr int kAmaxThreads = 256, kAmaxUnroll = 4;
+
+__global__ void __launch_bounds__(kAmaxThreads)
+nvfp4_group_amax_kernel(const uint16_t* __restrict__ x, int64_t ngroups, int64_t group_vec, int64_t chunk_vec,
+                        float* __restrict__ outer) {
+  __shared__ uint32_t wm[kAmaxThreads / 32];
+  for (int64_t g = blockIdx.y; g < ngroups; g += gridDim.y) {
+    const uint4* xv = reinterpret_cast<const uint4*>(x) + g * group_vec;
+    const int64_t v0 = (int64_t)blockIdx.x * chunk_vec;
+    const int64_t v1 = min(group_vec, v0 + chunk_vec);
+    uint32_t m = 0;
+    for (int64_t v = v0 + threadIdx.x; v < v1; v += kAmaxThreads * kAmaxUnroll) {
+        uint4 q[kAmaxUnroll];
+#pragma unroll
+        for (int u = 0; u < kAmaxUnroll; ++u) {
+            const int64_t idx = v + (int64_t)u * kAmaxThreads;
+            q[u] = idx < v1 ? __ldcs(xv + idx) : make_uint4(0, 0, 0, 0);
         }
-        int64_t g0 = __shfl_sync(0xffffffffu, g, 0);
-        bool same = __all_sync(0xffffffffu, g == g0 || g < 0);
-        if (same) {
-            m = warp_max_u32(m);
-            if ((threadIdx.x % 32) == 0 && g0 >= 0)
-                atomicMax(reinterpret_cast<unsigned int*>(outer) + g0, m << 16);
-        } else if (g >= 0) {
-            atomicMax(reinterpret_cast<unsigned int*>(outer) + g, m << 16);
-        }
+#pragma unroll
+        for (int u = 0; u < kAmaxUnroll; ++u) m = max(m, absmax8_bf16(q[u]));
     }
+    m = warp_max_u32(m);
+    if ((threadIdx.x & 31) == 0) wm[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t b = 0;
+        for (int w = 0; w < kAmaxThreads / 32; ++w) b = max(b, wm[w]);
+        atomicMax(reinterpret_cast<unsigned int*>(outer) + g, b << 16);
+    }
+    __syncthreads();
+  }
 }
 
 __global__ void nvfp4_group_finish_kernel(float* outer, int64_t ngroups) {
@@ -145,14 +151,20 @@ __global__ void nvfp4_group_finish_kernel(float* outer, int64_t ngroups) {
 // Transpose tile: 128 rows x 64 columns of the input.  Phase 1 loads the tile
 // (bf16, or NVFP4 dequantised to fp32) -- thread t owns row t/2, columns
 // 32*(t%2) .. +31 -- and stores fp32 values transposed into shared memory
-// T[c][r] (128 words per row c, the r index XOR-swizzled by 16*(c/32) so both
-// column halves hit disjoint banks).  Phase 2: thread (c, g) takes output row
-// c, elements r = 16g .. 16g+15 (8 threads cover the tile's 128 r of row c);
-// lane pairs (g, g^1) form one 32-element MXFP8 block.
+// T[c][r] (128 words per row c).  Phase 2: thread (c, g) takes output row c,
+// elements r = 16g .. 16g+15 as four 16-byte chunks (8 threads cover the
+// tile's 128 r of row c); lane pairs (g, g^1) form one 32-element MXFP8 block.
+// Swizzle: the 16-byte chunk j of group g sits at chunk j ^ ((g/2)%4), and
+// columns c >= 32 flip r's bit 4, so phase-1 scalar stores (16 rows x 2
+// column halves per warp) and phase-2 16-byte loads (8 groups of one row per
+// quarter warp) are both free of bank conflicts.
 // ---------------------------------------------------------------------------
 constexpr int kTR = 128, kTC = 64, kTileThreads = 256;
 
-__device__ __forceinline__ int tsw(int c, int r) { return c * kTR + (r ^ ((c >> 5) << 4)); }
+__device__ __forceinline__ int tsw(int c, int r) {
+    const int rs = (r & ~12) | ((((r >> 2) & 3) ^ ((r >> 5) & 3)) << 2);
+    return c * kTR + (rs ^ ((c >> 5) << 4));
+}
 
 // Phase 2: from smem T to MXFP8 codes of the transposed output.
 // kSR: stochastic rounding with kR random bits, else RNE.
@@ -169,19 +181,35 @@ __device__ __forceinline__ void tile_emit_transposed(const float* T, int64_t row
         float v[16];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const int pj = (j + (g >> 1)) & 3;         // bank-conflict-free chunk order
-            const float4 q = *reinterpret_cast<const float4*>(T + tsw(c, 16 * g + 4 * pj));
-            v[4 * pj + 0] = q.x; v[4 * pj + 1] = q.y; v[4 * pj + 2] = q.z; v[4 * pj + 3] = q.w;
+            const float4 q = *reinterpret_cast<const float4*>(T + tsw(c, 16 * g + 4 * j));
+            v[4 * j + 0] = q.x; v[4 * j + 1] = q.y; v[4 * j + 2] = q.z; v[4 * j + 3] = q.w;
         }
-        uint32_t m = 0;
+        float mf = 0.0f;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) m = max(m, __float_as_uint(v[i]) & 0x7fffffffu);
-        m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
-        const int e = e8m0_exponent(__uint_as_float(m));
+        for (int i = 0; i < 16; ++i) mf = fmaxf(mf, fabsf(v[i]));
+        mf = fmaxf(mf, __shfl_xor_sync(0xffffffffu, mf, 1));
+        const int e = e8m0_exponent(mf);
+        const SrBlock sb = sr_block(e);
         const int64_t cg = c0 + c;
         const int64_t rr = r0 + 16 * g;
         uint32_t w[4];
-        if (kSR) {
+        if (kSR && kR == 16) {
+            // hardware stochastic rounding, two elements per instruction
+            const int64_t L0 = cg * rows + rr;          // output element index
+            const float sc = exp2_neg(e);
+#pragma unroll
+            for (int blk = 0; blk < 2; ++blk) {
+                const uint4 rnd = philox4x32_10((uint64_t)(L0 / 8) + blk, stream_id, seed);
+                const uint32_t wd[4] = {rnd.x, rnd.y, rnd.z, rnd.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int i = blk * 8 + 2 * q;     // elements i, i+1 use word q's halves
+                    const uint32_t pr = cvt_rs16_e4m3_pair(__fmul_rn(v[i], sc), __fmul_rn(v[i + 1], sc),
+                                                           wd[q] & 0xffffu, wd[q] >> 16);
+                    if ((q & 1) == 0) w[blk * 2 + (q >> 1)] = pr; else w[blk * 2 + (q >> 1)] |= pr << 16;
+                }
+            }
+        } else if (kSR) {
             const int64_t L0 = cg * rows + rr;          // output element index
             constexpr int kPer = 128 / kR;              // elements per Philox block
 #pragma unroll
@@ -190,7 +218,7 @@ __device__ __forceinline__ void tile_emit_transposed(const float* T, int64_t row
 #pragma unroll
                 for (int jj = 0; jj < kPer && blk * kPer + jj < 16; ++jj) {
                     const int i = blk * kPer + jj;
-                    const uint32_t code = e4m3_sr_code<kR>(v[i], e, philox_field<kR>(rnd, jj));
+                    const uint32_t code = e4m3_sr_code<kR>(v[i], sb, philox_field<kR>(rnd, jj));
                     if ((i & 3) == 0) w[i >> 2] = code; else w[i >> 2] |= code << (8 * (i & 3));
                 }
             }
@@ -238,7 +266,21 @@ mxfp8_tile_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, co
         const int e = e8m0_exponent(__uint_as_float(m << 16));
         uint32_t w[8];
         const int64_t L0 = r * cols + c0 + 32 * h;
-        if (kSR) {
+        if (kSR && kR == 16) {
+            const float sc = exp2_neg(e);
+#pragma unroll
+            for (int blk = 0; blk < 4; ++blk) {
+                const uint4 rnd = philox4x32_10((uint64_t)(L0 / 8) + blk, stream_row, seed);
+                const uint32_t wd[4] = {rnd.x, rnd.y, rnd.z, rnd.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int i = blk * 8 + 2 * q;
+                    const uint32_t pr = cvt_rs16_e4m3_pair(__fmul_rn(v[i], sc), __fmul_rn(v[i + 1], sc),
+                                                           wd[q] & 0xffffu, wd[q] >> 16);
+                    if ((q & 1) == 0) w[blk * 2 + (q >> 1)] = pr; else w[blk * 2 + (q >> 1)] |= pr << 16;
+                }
+            }
+        } else if (kSR) {
             constexpr int kPer = 128 / kR;
 #pragma unroll
             for (int blk = 0; blk < 32 / kPer; ++blk) {
@@ -272,7 +314,7 @@ mxfp8_tile_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, co
 
 // NVFP4 [rows, cols] -> dequantise -> transpose -> MXFP8 with SR.
 template <int kR, int kInLayout, int kOutLayout>
-__global__ void __launch_bounds__(kTileThreads)
+__global__ void __launch_bounds__(kTileThreads, 4)
 requant_tile_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sf, const float* __restrict__ outer,
                     int64_t rows, int64_t cols, int64_t group_rows, const int64_t* rows_valid,
                     uint64_t seed, uint64_t stream_id, uint8_t* __restrict__ out_codes, uint8_t* __restrict__ out_e8m0) {
@@ -287,7 +329,8 @@ requant_tile_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict
     const int64_t s0 = (c0 >> 4) + 2 * h;
     const uint32_t sc0 = sf[sf_offset(r, s0, S, kInLayout)];
     const uint32_t sc1 = sf[sf_offset(r, s0 + 1, S, kInLayout)];
-    const float so = outer[r / group_rows];
+    // group_rows is 1 or a multiple of 128, so a tile's rows share one group
+    const float so = outer[group_rows == 1 ? r : (int64_t)((uint32_t)r0 / (uint32_t)group_rows)];
     const __half2 f0 = __half2half2(e4m3_to_h(sc0)), f1 = __half2half2(e4m3_to_h(sc1));
     const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
@@ -337,9 +380,10 @@ extern "C" int nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t
                 nvfp4_quant_rows_kernel<8, false, kL><<<grid, block, 0, stream>>>(xb, rows, cols, 1, codes, sf, outer);
         } else {
             if (cudaMemsetAsync(outer, 0, sizeof(float) * ngroups, stream) != cudaSuccess) return mx_launch_status();
-            const int64_t total = rows * nblk_row;
-            const unsigned g = (unsigned)std::min<int64_t>((total + 255) / 256, 148 * 16);
-            nvfp4_group_amax_kernel<<<g, 256, 0, stream>>>(xb, rows, cols, group_rows, outer);
+            const int64_t group_vec = group_rows * cols / 8;          // 16-byte vectors per group
+            const int64_t chunk_vec = 16384;                            // 256 KiB per block
+            const dim3 ag((unsigned)((group_vec + chunk_vec - 1) / chunk_vec), (unsigned)std::min<int64_t>(ngroups, 65535));
+            nvfp4_group_amax_kernel<<<ag, kAmaxThreads, 0, stream>>>(xb, ngroups, group_vec, chunk_vec, outer);
             if (nblk_row <= 32 * 2)
                 nvfp4_quant_rows_kernel<2, true, kL><<<grid, block, 0, stream>>>(xb, rows, cols, group_rows, codes, sf, outer);
             else
@@ -403,6 +447,8 @@ extern "C" int mxfp8_requant_transpose_sr(const uint8_t* codes, const uint8_t* s
     for (int l : {in_sf_layout, out_sf_layout})
         if (l != MX_SF_ROWMAJOR && l != MX_SF_MMA) return MX_EINVAL;
     if (out_sf_layout == MX_SF_MMA && (cols % 128 || rows % 128)) return MX_EINVAL;
+    if (group_rows != 1 && group_rows % kTR) return MX_EINVAL;
+    if (rows >= ((int64_t)1 << 31)) return MX_EINVAL;
     if (int st = mx_check_device()) return st;
     if (rows == 0) return MX_OK;
     const dim3 grid((unsigned)(cols / kTC), (unsigned)(rows / kTR));

@@ -39,7 +39,7 @@ class ExpertLayer:
     """
 
     def __init__(self, x, topk, w_comb, w1, w2, dout, gated: bool = True, seed: int = 0,
-                 wgrad_dtype=torch.bfloat16, out_dtype=torch.bfloat16, rbits: int = 8):
+                 wgrad_dtype=torch.bfloat16, out_dtype=torch.bfloat16, rbits: int = 16):
         dev = x.device
         self.dev = dev
         self.T, self.D = x.shape

@@ -122,7 +122,8 @@ MX_API int nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t gro
  *   out_e8m0        device u8 mx_sf_bytes(cols, rows, 32, out_sf_layout)
  *   rows_valid      device int64 or NULL: only r < *rows_valid are read and
  *                   written (an expert-major buffer passes &seg_offsets[E])
- * Requires rows % 128 == 0, cols % 64 == 0, rbits in {8, 16, 32}.
+ * Requires rows % 128 == 0, cols % 64 == 0, rbits in {8, 16, 32}, group_rows 1
+ * or a multiple of 128, rows < 2^31.
  * ------------------------------------------------------------------------ */
 MX_API int mxfp8_requant_transpose_sr(const uint8_t* codes, const uint8_t* sf, const float* outer,
                                int64_t rows, int64_t cols, int64_t group_rows, int in_sf_layout,

@@ -131,6 +131,11 @@ def test_grouped_gemm_mxfp8_dgrad(cuda, E, Nout, Kc, counts):
     got = out.cpu().numpy()
     assert np.all(np.isnan(got[M_pad:]))
     assert rel_fro(got[:M_pad].astype(np.float64), ref) <= TOL_FRO
+    outb = api.grouped_gemm_mxfp8(api.MX_GEMM_DGRAD, dev(pad_rows(ac, M_cap)), dev(rowmajor_to_mma(pad_rows(ae, M_cap))),
+                                  dev(bc), dev(rowmajor_to_mma(be)), dev(seg), E, M_cap, Nout, Kc,
+                                  out_dtype=torch.bfloat16)
+    gb = outb.float().cpu().numpy()[:M_pad].astype(np.float64)
+    assert np.all(np.abs(gb - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-4 * np.abs(ref).max())
 
 
 @pytest.mark.parametrize("E,Nw,Kw,counts", [(3, 256, 256, [128, 0, 300]), (2, 128, 384, [60, 200]),
@@ -154,3 +159,7 @@ def test_grouped_gemm_mxfp8_wgrad(cuda, E, Nw, Kw, counts):
         if seg[e + 1] == seg[e]:
             assert np.all(got[e] == 0)                    # empty expert -> zeros
     assert rel_fro(got, ref) <= TOL_FRO
+    outb = api.grouped_gemm_mxfp8(api.MX_GEMM_WGRAD, dev(ac), dev(rowmajor_to_mma(ae)), dev(bc), dev(rowmajor_to_mma(be)),
+                                  dev(seg), E, M_cap, Nw, Kw, out_dtype=torch.bfloat16)
+    gb = outb.float().cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(gb - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-4 * np.abs(ref).max())

@@ -69,16 +69,16 @@ def test_tiny_layer_forward_backward_against_oracle(cuda):
     dy2 = oracle.dispatch_grad(dout, pos, w, Mp)
     dy2_r = oracle.mxfp8_quantize_rows(dy2)
     dy2_c = oracle.mxfp8_quantize_cols(pad(dy2, M))
-    w2t = oracle.mxfp8_requant_transpose_sr(*w2q, D, seed, 1, 8)
+    w2t = oracle.mxfp8_requant_transpose_sr(*w2q, D, seed, 1, 16)
     da = oracle.f64_to_bf16(oracle.grouped_gemm_mxfp8_dgrad(*dy2_r, *w2t, seg))
-    at = oracle.mxfp8_requant_transpose_sr(pad(aq[0], M), pad(aq[1], M), pad(aq[2], M), 1, seed, 2, 8)
+    at = oracle.mxfp8_requant_transpose_sr(pad(aq[0], M), pad(aq[1], M), pad(aq[2], M), 1, seed, 2, 16)
     dw2 = oracle.grouped_gemm_mxfp8_wgrad(*dy2_c, *at, seg)
     dh1 = oracle.swiglu_bwd(h1, da, gated=False)
     dh1_r = oracle.mxfp8_quantize_rows(dh1)
     dh1_c = oracle.mxfp8_quantize_cols(pad(dh1, M))
-    w1t = oracle.mxfp8_requant_transpose_sr(*w1q, F, seed, 3, 8)
+    w1t = oracle.mxfp8_requant_transpose_sr(*w1q, F, seed, 3, 16)
     dxp = oracle.f64_to_bf16(oracle.grouped_gemm_mxfp8_dgrad(*dh1_r, *w1t, seg))
-    xt = oracle.mxfp8_requant_transpose_sr(pad(xp[0], M), pad(xp[1], M), pad(xp[2], M), 1, seed, 4, 8)
+    xt = oracle.mxfp8_requant_transpose_sr(pad(xp[0], M), pad(xp[1], M), pad(xp[2], M), 1, seed, 4, 16)
     dw1 = oracle.grouped_gemm_mxfp8_wgrad(*dh1_c, *xt, seg)
     dx = oracle.combine(dxp, pos, np.ones_like(w))
 

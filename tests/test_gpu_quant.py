@@ -103,16 +103,17 @@ def test_nvfp4_quantize_per_expert_bit_exact(cuda, E, N, K):
 # MXFP8 quantiser
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("rounding", [api.MX_ROUND_RNE, api.MX_ROUND_SR])
+@pytest.mark.parametrize("rounding,R", [(api.MX_ROUND_RNE, 8), (api.MX_ROUND_SR, 8), (api.MX_ROUND_SR, 16),
+                                        (api.MX_ROUND_SR, 32)])
 @pytest.mark.parametrize("rows,cols", [(128, 128), (256, 384), (512, 1024)])
-def test_mxfp8_quantize_rows_and_cols_bit_exact(cuda, rows, cols, rounding):
+def test_mxfp8_quantize_rows_and_cols_bit_exact(cuda, rows, cols, rounding, R):
     x = heavy_rows(rows, cols, seed=3 * rows + cols, spread=6.0)
     sr = rounding == api.MX_ROUND_SR
     seed, stream = 0xDEADBEEF12345, 7
-    rc, re = oracle.mxfp8_quantize_rows(x, sr=sr, seed=seed, stream=stream, R=8)
-    cc, ce = oracle.mxfp8_quantize_cols(x, sr=sr, seed=seed, stream=stream + 1, R=8)
+    rc, re = oracle.mxfp8_quantize_rows(x, sr=sr, seed=seed, stream=stream, R=R)
+    cc, ce = oracle.mxfp8_quantize_cols(x, sr=sr, seed=seed, stream=stream + 1, R=R)
     for layout in (api.MX_SF_ROWMAJOR, api.MX_SF_MMA):
-        g = api.mxfp8_quantize(to_dev_bf16(x), rounding=rounding, seed=seed, stream_id=stream, rbits=8,
+        g = api.mxfp8_quantize(to_dev_bf16(x), rounding=rounding, seed=seed, stream_id=stream, rbits=R,
                                sf_layout=layout)
         assert np.array_equal(np_(g[0]), rc)
         assert np.array_equal(np_(g[2]), cc)
@@ -163,6 +164,21 @@ def test_requant_transpose_sr_bit_exact(cuda, rows, cols, R):
             ge = np_(ge)
             got_e = ge.reshape(oe.shape) if lout == api.MX_SF_ROWMAJOR else mma_to_rowmajor(ge, cols, rows // 32)
             assert np.array_equal(got_e, oe)
+
+
+@pytest.mark.parametrize("R", [8, 16, 32])
+def test_requant_extreme_dynamic_range(cuda, R):
+    # per-row scales over 24 decades: inside one 32-row block most values sit
+    # far below E4M3's normal range (and many below its smallest subnormal),
+    # exercising every branch of the stochastic rounding down to fp32 subnormals
+    x = heavy_rows(256, 128, seed=77 + R, spread=12.0)
+    codes, sf, outer = oracle.nvfp4_quantize(x)
+    oc, oe = oracle.mxfp8_requant_transpose_sr(codes, sf, outer, 1, 11, 12, R)
+    gc, ge = api.mxfp8_requant_transpose_sr(torch.from_numpy(codes).cuda(), torch.from_numpy(sf.reshape(-1).copy()).cuda(),
+                                            torch.from_numpy(outer).cuda(), 256, 128, 1, api.MX_SF_ROWMAJOR, None, 11, 12,
+                                            R, api.MX_SF_ROWMAJOR)
+    assert np.array_equal(np_(gc), oc)
+    assert np.array_equal(np_(ge).reshape(oe.shape), oe)
 
 
 def test_requant_weights_per_expert_outer(cuda):
