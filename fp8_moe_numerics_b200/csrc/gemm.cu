@@ -118,22 +118,73 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                  : "memory");
 }
 
-__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                 :: "r"(smem_u32(dst_smem)), "r"(ncols) : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+// Operand tile of a CTA pair: lands in this CTA's shared memory, its bytes
+// are counted on the leader CTA's mbarrier (a shared::cluster address).
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+                 " [%0], [%1, {%2, %3}], [%4];"
+                 :: "r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar_cluster)
+                 : "memory");
 }
 
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// shared::cluster address of the variable at the same offset in CTA `rank` of this cluster.
+__device__ __forceinline__ uint32_t map_to_rank(const void* p, uint32_t rank) {
+    uint32_t a;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(p)), "r"(rank));
+    return a;
+}
+
+// Arrive on a barrier of another CTA of the cluster.  CTA-scope release: what
+// the arrival publishes is TMEM state, already ordered by tcgen05.wait and
+// tcgen05.fence; a cluster-scope release would add a memory fence per call.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" :: "r"(bar_cluster) : "memory");
+}
+
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+template <bool kPair>
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+    if (kPair) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+                     :: "r"(smem_u32(dst_smem)), "r"(ncols) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    } else {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     :: "r"(smem_u32(dst_smem)), "r"(ncols) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+}
+
+template <bool kPair>
 __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(taddr), "r"(ncols) : "memory");
+    if (kPair)
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" :: "r"(taddr), "r"(ncols) : "memory");
+    else
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(taddr), "r"(ncols) : "memory");
 }
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
+// Arrive on `bar` once every MMA issued so far has completed.  A pair's
+// leader signals the barrier at the same offset in both CTAs.
+template <bool kPair>
 __device__ __forceinline__ void tc_commit(uint64_t* bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
-                 :: "r"(smem_u32(bar)) : "memory");
+    if (kPair)
+        asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+                     :: "r"(smem_u32(bar)), "h"((uint16_t)0x3) : "memory");
+    else
+        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                     :: "r"(smem_u32(bar)) : "memory");
 }
 
 // Shared-memory matrix descriptor (tcgen05): start address >> 4 in bits
@@ -152,32 +203,37 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint
 
 // K-major operand, 128-byte swizzle: 8-row groups 1024 bytes apart.
 __device__ __forceinline__ uint64_t operand_desc(uint32_t saddr) { return smem_desc(saddr, 16, 1024, 2); }
-// Instruction descriptor of a block-scaled MMA with M = 128, N = n, K-major
+// Instruction descriptor of a block-scaled MMA with M = m, N = n, K-major
 // A and B: formats in bits [7,10) and [10,13), N>>3 in [17,23), scale format
 // in bit 23 (0 = UE4M3, 1 = UE8M0), M>>4 in [24,29), scale-factor byte ids of
 // A in [29,31) and of B in [4,6).
-__device__ __forceinline__ uint32_t idesc_block_scaled(uint32_t fmt, uint32_t scale_fmt, int n, uint32_t sfa_id,
+__device__ __forceinline__ uint32_t idesc_block_scaled(uint32_t fmt, uint32_t scale_fmt, int m, int n, uint32_t sfa_id,
                                                        uint32_t sfb_id) {
     return (sfb_id << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)(n >> 3) << 17) | (scale_fmt << 23) |
-           ((uint32_t)(kBM >> 4) << 24) | (sfa_id << 29);
+           ((uint32_t)(m >> 4) << 24) | (sfa_id << 29);
 }
 
-template <int kKind>
+// One block-scaled MMA.  kPair: issued by the leader of a CTA pair, M = 256
+// with 128 rows of A and half of B's rows in each CTA's shared memory, each
+// CTA's accumulator and scale factors in its own TMEM.
+template <int kKind, bool kPair>
 __device__ __forceinline__ void mma_block_scaled(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                                  uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+#define MX_MMA_ASM(GROUP, KIND)                                                                                  \
+    asm volatile("{\n\t.reg .pred p;\n\t"                                                                      \
+                 "setp.ne.b32 p, %4, 0;\n\t"                                                                     \
+                 "tcgen05.mma.cta_group::" GROUP ".kind::" KIND " [%0], %1, %2, %3, [%5], [%6], p;\n\t}"          \
+                 :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem),             \
+                    "r"(sfb_tmem)                                                                                 \
+                 : "memory")
     if (kKind == kKindNVFP4) {
-        asm volatile("{\n\t.reg .pred p;\n\t"
-                     "setp.ne.b32 p, %4, 0;\n\t"
-                     "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
-                     :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
-                     : "memory");
+        if (kPair) MX_MMA_ASM("2", "mxf4nvf4.block_scale.block16");
+        else MX_MMA_ASM("1", "mxf4nvf4.block_scale.block16");
     } else {
-        asm volatile("{\n\t.reg .pred p;\n\t"
-                     "setp.ne.b32 p, %4, 0;\n\t"
-                     "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
-                     :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
-                     : "memory");
+        if (kPair) MX_MMA_ASM("2", "mxf8f6f4.block_scale.block32");
+        else MX_MMA_ASM("1", "mxf8f6f4.block_scale.block32");
     }
+#undef MX_MMA_ASM
 }
 
 // 32 columns of fp32 for this thread's TMEM lane, waited for inside the asm.
@@ -199,17 +255,28 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, float* v) {
 // ---------------------------------------------------------------------------
 // Tile scheduling shared by all roles
 // ---------------------------------------------------------------------------
+// A work item is one output tile.  Single-CTA items are 128 rows x kBN
+// columns.  Pair items are 256 rows x kBN columns: CTA rank r of the pair owns
+// rows [128 r, 128 r + 128) of the tile and loads half of B's kBN rows.  In
+// ROWS mode expert e holds ceil(tiles_e / 2) row pairs (segments are padded
+// to 128 rows, not 256); each CTA scans these counts into a shared-memory
+// prefix at start-up, so items form a dense list.  When an expert's tile
+// count is odd its last pair has no second half: CTA 1 then recomputes CTA
+// 0's rows (valid memory, no special case in the pipeline) and stores nothing.
+constexpr int kMaxPairExperts = 768;    // prefix capacity (shared memory)
 struct Tile {
+    bool valid;         // false: a hole in the item list, no work
+    bool store;         // false: this CTA's half lies outside the expert
     int64_t e;          // expert
-    int64_t row0;       // first output row (ROWS: token row; WGRAD: row of out viewed as [E*N, K])
+    int64_t row0;       // first output row of this CTA (ROWS: token row; WGRAD: row of out viewed as [E*N, K])
     int64_t col0;       // first output column
-    int64_t a_y;        // A tile row coordinate
-    int64_t b_y;        // B tile row coordinate
+    int64_t a_y;        // A tile row coordinate (this CTA's 128 rows)
+    int64_t b_y;        // B tile row coordinate (this CTA's share of the kBN rows)
     int64_t k0_bytes;   // first K byte of the contraction (A and B x coordinate base)
     int64_t b_x0;       // B x coordinate base (DGRAD: e*K)
     int64_t k_tiles;    // stages of 128 K-bytes
     int64_t sfa_atom0;  // first SFA atom of the tile's first stage
-    int64_t sfb_atom0;  // first SFB atom (row group 0)
+    int64_t sfb_atom0;  // first SFB atom (row group 0 of the kBN columns)
 };
 
 __device__ __forceinline__ int64_t find_expert(const int64_t* seg, int64_t E, int64_t row) {
@@ -221,80 +288,138 @@ __device__ __forceinline__ int64_t find_expert(const int64_t* seg, int64_t E, in
     return lo;
 }
 
-template <int kKind, int kMode, int kBN>
-__device__ __forceinline__ int64_t total_tiles(const GemmArgs& p) {
-    if (kMode == kModeRows) return (__ldg(p.seg + p.E) / kBM) * (p.N / kBN);
-    return p.E * (p.N / kBM) * (p.K / kBN);
+template <int kMode, int kBN, bool kPair>
+__device__ __forceinline__ int64_t total_tiles(const GemmArgs& p, const int32_t* pfx) {
+    if (kMode == kModeRows)
+        return (kPair ? (int64_t)pfx[p.E] : __ldg(p.seg + p.E) / kBM) * (p.N / kBN);
+    return p.E * (p.N / (kPair ? 2 * kBM : kBM)) * (p.K / kBN);
 }
 
-template <int kKind, int kMode, int kBN>
-__device__ __forceinline__ Tile make_tile(const GemmArgs& p, int64_t idx) {
+// Pair ROWS mode: pfx[e] = row pairs of experts 0..e-1 (pfx[E] = all pairs).
+__device__ __forceinline__ void build_pair_prefix(const GemmArgs& p, int32_t* pfx) {
+    for (int64_t e = threadIdx.x; e < p.E; e += blockDim.x) {
+        const int64_t tiles = (__ldg(p.seg + e + 1) - __ldg(p.seg + e)) / kBM;
+        pfx[e + 1] = (int32_t)((tiles + 1) / 2);
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        int32_t carry = 0;
+        for (int64_t b = 0; b < p.E; b += 32) {
+            const int64_t e = b + lane;
+            int32_t v = e < p.E ? pfx[e + 1] : 0;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int32_t u = __shfl_up_sync(0xffffffffu, v, o);
+                if (lane >= o) v += u;
+            }
+            if (e < p.E) pfx[e + 1] = carry + v;
+            carry += __shfl_sync(0xffffffffu, v, 31);
+        }
+        if (lane == 0) pfx[0] = 0;
+    }
+    __syncthreads();
+}
+
+template <int kKind, int kMode, int kBN, bool kPair>
+__device__ __forceinline__ Tile make_tile(const GemmArgs& p, int64_t idx, uint32_t rank, const int32_t* pfx) {
     Tile t;
-    const int64_t spg = kKind == kKindNVFP4 ? 4 : 1;   // scale atoms per stage per 128-row group
+    t.valid = true;
+    t.store = true;
+    const int64_t half = kPair ? (int64_t)rank * kBM : 0;      // this CTA's row offset inside a pair item
+    const int64_t b_half = kPair ? (int64_t)rank * (kBN / 2) : 0;
     if (kMode == kModeRows) {
         const int64_t n_tiles = p.N / kBN;
         const int64_t mt = idx / n_tiles, nt = idx % n_tiles;
-        t.row0 = mt * kBM;
+        int64_t base, a_row;
+        if (kPair) {
+            int lo = 0, hi = (int)p.E;                   // last expert with pfx[e] <= mt
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if (pfx[mid] <= mt) lo = mid; else hi = mid;
+            }
+            t.e = lo;
+            base = __ldg(p.seg + t.e) + (mt - pfx[t.e]) * (2 * kBM);
+            t.store = rank == 0 || base + kBM < __ldg(p.seg + t.e + 1);
+            a_row = t.store ? base + half : base;
+        } else {
+            base = mt * kBM;
+            t.e = find_expert(p.seg, p.E, base);
+            a_row = base;
+        }
+        t.row0 = base + half;
         t.col0 = nt * kBN;
-        t.e = find_expert(p.seg, p.E, t.row0);
         const int64_t kbytes = kKind == kKindNVFP4 ? p.K / 2 : p.K;
         t.k_tiles = kbytes / kStageBytesK;
         t.k0_bytes = 0;
-        t.a_y = t.row0;
-        t.sfa_atom0 = mt * p.sfa_groups;
+        t.a_y = a_row;
+        t.sfa_atom0 = (a_row / kBM) * p.sfa_groups;
         if (kKind == kKindNVFP4) {                      // B = weight stack [E*N, K]
-            t.b_y = t.e * p.N + t.col0;
+            const int64_t b_first = t.e * p.N + t.col0;
+            t.b_y = b_first + b_half;
             t.b_x0 = 0;
-            t.sfb_atom0 = (t.b_y / kBM) * p.sfb_groups;
+            t.sfb_atom0 = (b_first / kBM) * p.sfb_groups;
         } else {                                        // DGRAD: B = [N, E*K]
-            t.b_y = t.col0;
+            t.b_y = t.col0 + b_half;
             t.b_x0 = t.e * p.K;
-            t.sfb_atom0 = (t.b_y / kBM) * p.sfb_groups + t.e * p.K / 128;
+            t.sfb_atom0 = (t.col0 / kBM) * p.sfb_groups + t.e * p.K / 128;
         }
-        (void)spg;
     } else {                                            // WGRAD: out [E, N, K]
-        const int64_t nt_n = p.N / kBM, nt_k = p.K / kBN;
+        const int64_t rows = kPair ? 2 * kBM : kBM;
+        const int64_t nt_n = p.N / rows, nt_k = p.K / kBN;
         t.e = idx / (nt_n * nt_k);
         const int64_t rem = idx % (nt_n * nt_k);
         const int64_t tn = rem / nt_k, tk = rem % nt_k;
         const int64_t s0 = __ldg(p.seg + t.e), s1 = __ldg(p.seg + t.e + 1);
-        t.row0 = t.e * p.N + tn * kBM;
+        t.a_y = tn * rows + half;
+        t.row0 = t.e * p.N + t.a_y;
         t.col0 = tk * kBN;
         t.k_tiles = (s1 - s0) / kStageBytesK;
         t.k0_bytes = s0;
         t.b_x0 = 0;
-        t.a_y = tn * kBM;
-        t.b_y = tk * kBN;
+        t.b_y = t.col0 + b_half;
         t.sfa_atom0 = t.a_y / kBM * p.sfa_groups + s0 / 128;
-        t.sfb_atom0 = t.b_y / kBM * p.sfb_groups + s0 / 128;
+        t.sfb_atom0 = t.col0 / kBM * p.sfb_groups + s0 / 128;
     }
     return t;
 }
 
-template <int kKind, int kBN>
+// Shared-memory and TMEM budget of one CTA.  A stage holds 128 K-bytes of A
+// (128 rows), of B (kBN rows, or kBN/2 for a pair) and the stage's scale
+// atoms: SFA for this CTA's 128 rows and SFB for all kBN columns (each CTA of
+// a pair keeps a full copy: the MMA reads B's scales from every CTA's TMEM).
+constexpr int kSmemLimit = 227 * 1024;
+template <int kKind, int kBN, bool kPair>
 struct Smem {
     static constexpr int kA = kBM * kStageBytesK;                       // 16 KB
-    static constexpr int kB = kBN * kStageBytesK;                       // 16 / 32 KB
+    static constexpr int kB = (kPair ? kBN / 2 : kBN) * kStageBytesK;
     static constexpr int kAtomsA = kKind == kKindNVFP4 ? 4 : 1;         // scale atoms per stage, 128-row group
     static constexpr int kAtomsB = kAtomsA * (kBN / 128);
     static constexpr int kSfa = kAtomsA * 512;
     static constexpr int kSfb = kAtomsB * 512;
-    static constexpr int kStageTx = kA + kB + kSfa + kSfb;             // bytes the TMA engine delivers per stage
-    static constexpr int kStage = (kStageTx + 1023) / 1024 * 1024;      // stage stride: keeps every SW128 tile 1024-aligned
+    static constexpr int kAbTx = kA + kB;                               // operand bytes per stage and CTA
+    static constexpr int kSfTx = kSfa + kSfb;
+    static constexpr int kStage = (kAbTx + kSfTx + 1023) / 1024 * 1024;  // stride keeps every SW128 tile 1024-aligned
     static constexpr int kStaging = 8 * 4096;                           // epilogue: one 64x32 bf16 box per warp
-    static constexpr int kStages = (kStage * 6 + kStaging <= 220 * 1024) ? 6
-                                 : (kStage * 4 + kStaging <= 220 * 1024) ? 4 : 3;
-    static constexpr int kStagingOff = kStages * kStage;
-    static_assert(kStage % 1024 == 0 && kStagingOff % 1024 == 0, "128-byte swizzle needs 1024-byte aligned tiles");
-    static constexpr int kBarOff = kStagingOff + kStaging;
-    static constexpr int kBytes = kBarOff + 512 + 1024;                  // + barriers + alignment slack
-    // TMEM: accumulator buffer(s), then one scale region per stage
     static constexpr int kSfaCols = 4 * kAtomsA;
     static constexpr int kSfbCols = 4 * kAtomsB;
     static constexpr int kSfRegion = kSfaCols + kSfbCols;
+    static constexpr int kPfxBytes = kPair ? 4 * (kMaxPairExperts + 4) : 0;
+    static constexpr int kFixed = kStaging + 512 + kPfxBytes + 1024;    // + barriers + prefix + alignment slack
+    static constexpr int fit(int s) {
+        return (s * kStage + kFixed <= kSmemLimit && kBN + s * kSfRegion <= kTmemCols) ? s : 0;
+    }
+    static constexpr int kStages = fit(6) ? 6 : fit(5) ? 5 : fit(4) ? 4 : fit(3) ? 3 : 2;
+    static constexpr int kStagingOff = kStages * kStage;
+    static_assert(kStage % 1024 == 0 && kStagingOff % 1024 == 0, "128-byte swizzle needs 1024-byte aligned tiles");
+    static constexpr int kBarOff = kStagingOff + kStaging;
+    static constexpr int kPfxOff = kBarOff + 512;
+    static constexpr int kBytes = kPfxOff + kPfxBytes + 1024;
+    // TMEM: accumulator buffer(s), then one scale region per stage
     static constexpr int kAccBufs = (2 * kBN + kStages * kSfRegion <= kTmemCols) ? 2 : 1;
     static constexpr int kSfCol = kAccBufs * kBN;
     static_assert(kSfCol + kStages * kSfRegion <= kTmemCols, "TMEM budget");
+    static_assert(kBytes <= kSmemLimit, "shared memory budget");
 };
 
 __device__ __forceinline__ void tmem_st_32x32b_x4(uint32_t taddr, const uint4& v) {
@@ -302,47 +427,61 @@ __device__ __forceinline__ void tmem_st_32x32b_x4(uint32_t taddr, const uint4& v
                  :: "r"(taddr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
 }
 
-template <int kKind, int kMode, int kBN, bool kOutBF16>
+// Bounded wait for phase `parity` of a local barrier against a shared deadline
+// (used only while draining at exit).
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, unsigned long long t0) {
+    while (!mbar_try_wait(bar, parity) && globaltimer() - t0 < kWaitLimitNs) {}
+}
+
+template <int kKind, int kMode, int kBN, bool kOutBF16, bool kPair>
 __global__ void __launch_bounds__(kThreads, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmOut, const GemmArgs p) {
-    using L = Smem<kKind, kBN>;
+    using L = Smem<kKind, kBN, kPair>;
     constexpr int kStages = L::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);   // operands landed
-    uint64_t* sf_full = full + kStages;                                 // scales written to TMEM
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);   // operands landed (pair: leader's counts both CTAs)
+    uint64_t* sf_full = full + kStages;                                 // scales written to TMEM (pair: both CTAs)
     uint64_t* empty = sf_full + kStages;                                // stage consumed by the MMAs
-    uint64_t* acc_full = empty + kStages;        // [2]: accumulator buffer b ready
-    uint64_t* acc_empty = acc_full + 2;          // [2]: accumulator buffer b drained
+    uint64_t* sf_landed = empty + kStages;                              // pair: this CTA's scale atoms landed
+    uint64_t* acc_full = sf_landed + kStages;    // [2]: accumulator buffer b ready
+    uint64_t* acc_empty = acc_full + 2;          // [2]: accumulator buffer b drained (pair: both CTAs)
     uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t total = total_tiles<kKind, kMode, kBN>(p);
-    if ((int64_t)blockIdx.x >= total) return;
+    const uint32_t rank = kPair ? cluster_ctarank() : 0u;
+    const int64_t first = kPair ? (int64_t)(blockIdx.x >> 1) : (int64_t)blockIdx.x;
+    const int64_t stride = kPair ? (int64_t)(gridDim.x >> 1) : (int64_t)gridDim.x;
+    int32_t* pfx = reinterpret_cast<int32_t*>(smem + L::kPfxOff);
+    if (kPair && kMode == kModeRows) build_pair_prefix(p, pfx);
+    const int64_t total = total_tiles<kMode, kBN, kPair>(p, pfx);
+    if (first >= total) return;                                         // uniform across a pair
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&sf_full[s], 4);
+            mbar_init(&sf_full[s], kPair ? 8 : 4);
             mbar_init(&empty[s], 1);
+            mbar_init(&sf_landed[s], 1);
         }
-        for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], 8); }
+        for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], kPair ? 16 : 8); }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
         asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
         if (kOutBF16) asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(&tmOut)) : "memory");
     }
-    if (warp == 1) tmem_alloc(tmem_base_slot, kTmemCols);
+    if (kPair) cluster_sync();                  // the peer's barriers exist before anything arrives on them
+    if (warp == 1) tmem_alloc<kPair>(tmem_base_slot, kTmemCols);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_base_slot;
 
     if (warp == 0) {
-        // ------------------------------------------------------------ TMA producer (A, B)
+        // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
@@ -350,45 +489,68 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             bool issued[kStages];
             for (int s = 0; s < kStages; ++s) { issued[s] = false; issued_phase[s] = 0; }
             bool ok = true;
-            for (int64_t idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
-                const Tile t = make_tile<kKind, kMode, kBN>(p, idx);
+            for (int64_t idx = first; idx < total && ok; idx += stride) {
+                const Tile t = make_tile<kKind, kMode, kBN, kPair>(p, idx, rank, pfx);
+                if (!t.valid) continue;
                 for (int64_t kt = 0; kt < t.k_tiles; ++kt) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
                     uint8_t* sa = smem + stage * L::kStage;
                     uint8_t* sb = sa + L::kA;
                     uint8_t* ssfa = sb + L::kB;
                     uint8_t* ssfb = ssfa + L::kSfa;
-                    mbar_expect_tx(&full[stage], (uint32_t)L::kStageTx);
                     const int kx = (int)(t.k0_bytes + kt * kStageBytesK);
-                    tma_load_2d(sa, &tmA, &full[stage], kx, (int)t.a_y);
-                    tma_load_2d(sb, &tmB, &full[stage], (int)t.b_x0 + kx, (int)t.b_y);
-                    bulk_load(ssfa, p.sfa + (t.sfa_atom0 + kt * L::kAtomsA) * 512, L::kSfa, &full[stage]);
+                    uint64_t* sf_bar = &full[stage];
+                    if (kPair) {
+                        // A and B count on the leader's barrier (it expects both CTAs' bytes);
+                        // the scale atoms on this CTA's own barrier for its scale movers.
+                        const uint32_t lead_full = map_to_rank(&full[stage], 0);
+                        if (rank == 0) mbar_expect_tx(&full[stage], (uint32_t)(2 * L::kAbTx));
+                        tma_load_2d_pair(sa, &tmA, lead_full, kx, (int)t.a_y);
+                        tma_load_2d_pair(sb, &tmB, lead_full, (int)t.b_x0 + kx, (int)t.b_y);
+                        sf_bar = &sf_landed[stage];
+                        mbar_expect_tx(sf_bar, (uint32_t)L::kSfTx);
+                    } else {
+                        mbar_expect_tx(&full[stage], (uint32_t)(L::kAbTx + L::kSfTx));
+                        tma_load_2d(sa, &tmA, &full[stage], kx, (int)t.a_y);
+                        tma_load_2d(sb, &tmB, &full[stage], (int)t.b_x0 + kx, (int)t.b_y);
+                    }
+                    bulk_load(ssfa, p.sfa + (t.sfa_atom0 + kt * L::kAtomsA) * 512, L::kSfa, sf_bar);
 #pragma unroll
                     for (int h = 0; h < kBN / 128; ++h)
                         bulk_load(ssfb + h * L::kAtomsA * 512, p.sfb + (t.sfb_atom0 + h * p.sfb_groups + kt * L::kAtomsA) * 512,
-                                  L::kAtomsA * 512, &full[stage]);
+                                  L::kAtomsA * 512, sf_bar);
                     issued[stage] = true;
                     issued_phase[stage] = phase;
                     if (++stage == kStages) { stage = 0; phase ^= 1u; }
                 }
             }
-            // drain: every issued copy has landed before shared memory is released
+            // drain: every copy this CTA issued has landed before its shared
+            // memory is released (a pair's operand bytes are counted on the
+            // leader; once the MMAs consumed a stage, its copies had landed)
+            const unsigned long long t0 = globaltimer();
             for (int s = 0; s < kStages; ++s)
                 if (issued[s]) {
-                    const unsigned long long t0 = globaltimer();
-                    while (!mbar_try_wait(&full[s], issued_phase[s]) && globaltimer() - t0 < kWaitLimitNs) {}
+                    if (kPair) {
+                        drain_wait(&sf_landed[s], issued_phase[s], t0);
+                        if (rank == 0) drain_wait(&full[s], issued_phase[s], t0);
+                        else drain_wait(&empty[s], issued_phase[s], t0);
+                    } else {
+                        drain_wait(&full[s], issued_phase[s], t0);
+                    }
                 }
         }
     } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        // ------------------------------------------------------------ MMA issuer (a pair's leader only)
+        if (lane == 0 && rank == 0) {
             constexpr uint32_t kFmt = kKind == kKindNVFP4 ? 1u : 0u;      // E2M1 / E4M3
             constexpr uint32_t kScaleFmt = kKind == kKindNVFP4 ? 0u : 1u; // UE4M3 / UE8M0
+            constexpr int kM = kPair ? 2 * kBM : kBM;
             int stage = 0, buf = 0;
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
-            for (int64_t idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
-                const Tile t = make_tile<kKind, kMode, kBN>(p, idx);
+            for (int64_t idx = first; idx < total && ok; idx += stride) {
+                const Tile t = make_tile<kKind, kMode, kBN, kPair>(p, idx, rank, pfx);
+                if (!t.valid) continue;
                 if (!mbar_wait(&acc_empty[buf], acc_phase ^ 1u, abort_flag)) break;
                 tc_fence_after();
                 const uint32_t acc = tmem + (uint32_t)(buf * kBN);
@@ -409,20 +571,20 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                         if (kKind == kKindNVFP4) {
                             sfa_t = sfa + 4 * j;
                             sfb_t = sfb + (kBN / 32) * j;
-                            id = idesc_block_scaled(kFmt, kScaleFmt, kBN, 0, 0);
+                            id = idesc_block_scaled(kFmt, kScaleFmt, kM, kBN, 0, 0);
                         } else {
                             sfa_t = sfa | ((uint32_t)j << 30);
                             sfb_t = sfb | ((uint32_t)j << 30);
-                            id = idesc_block_scaled(kFmt, kScaleFmt, kBN, (uint32_t)j, (uint32_t)j);
+                            id = idesc_block_scaled(kFmt, kScaleFmt, kM, kBN, (uint32_t)j, (uint32_t)j);
                         }
-                        mma_block_scaled<kKind>(acc, operand_desc(a0 + 32 * j), operand_desc(b0 + 32 * j), id,
-                                                sfa_t, sfb_t, (kt > 0 || j > 0) ? 1u : 0u);
+                        mma_block_scaled<kKind, kPair>(acc, operand_desc(a0 + 32 * j), operand_desc(b0 + 32 * j), id,
+                                                       sfa_t, sfb_t, (kt > 0 || j > 0) ? 1u : 0u);
                     }
-                    tc_commit(&empty[stage]);
+                    tc_commit<kPair>(&empty[stage]);
                     if (++stage == kStages) { stage = 0; phase ^= 1u; }
                 }
                 if (!ok) break;
-                tc_commit(&acc_full[buf]);
+                tc_commit<kPair>(&acc_full[buf]);
                 if (++buf == L::kAccBufs) { buf = 0; acc_phase ^= 1u; }
             }
         }
@@ -434,15 +596,17 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         // l+96 of the 128-row group), the replicated layout the block-scaled
         // MMA reads in every quarter.  tcgen05.st from registers does not
         // occupy the tensor pipe (tcgen05.cp would, ~24 cycles per atom).
+        // In a pair each CTA fills its own TMEM and reports to the leader.
         const int q = warp & 3;
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
-        for (int64_t idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
-            const Tile t = make_tile<kKind, kMode, kBN>(p, idx);
+        for (int64_t idx = first; idx < total && ok; idx += stride) {
+            const Tile t = make_tile<kKind, kMode, kBN, kPair>(p, idx, rank, pfx);
+            if (!t.valid) continue;
             for (int64_t kt = 0; kt < t.k_tiles; ++kt) {
-                if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+                if (!mbar_wait(kPair ? &sf_landed[stage] : &full[stage], phase, abort_flag)) { ok = false; break; }
                 const uint8_t* ssfa = smem + stage * L::kStage + L::kA + L::kB;
                 const uint8_t* ssfb = ssfa + L::kSfa;
                 uint4 va[L::kAtomsA], vb[L::kAtomsB];
@@ -463,7 +627,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&sf_full[stage]);
+                if (lane == 0) {
+                    if (kPair) mbar_arrive_cluster(map_to_rank(&sf_full[stage], 0));
+                    else mbar_arrive(&sf_full[stage]);
+                }
                 if (++stage == kStages) { stage = 0; phase ^= 1u; }
             }
         }
@@ -474,119 +641,137 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         // output: each 32-column chunk is scaled and packed as it arrives, the
         // accumulator is released after the last chunk, and the stores overlap
         // the next tile's main loop.  fp32 output stores chunk by chunk and
-        // releases the accumulator afterwards.
+        // releases the accumulator afterwards.  A pair's CTAs each drain their
+        // own 128 rows and both report to the leader.
         constexpr int kCols = kBN / 2;
         const int q = warp & 3;
         const int half = (warp - 8) >> 2;
         const int r = q * 32 + lane;
         const int cb = half * kCols;
+        const uint32_t acc_empty_lead[2] = {kPair ? map_to_rank(&acc_empty[0], 0) : 0u,
+                                            kPair ? map_to_rank(&acc_empty[1], 0) : 0u};
         uint32_t acc_phase = 0;
         int buf = 0;
-        for (int64_t idx = blockIdx.x; idx < total; idx += gridDim.x) {
-            const Tile t = make_tile<kKind, kMode, kBN>(p, idx);
+        for (int64_t idx = first; idx < total; idx += stride) {
+            const Tile t = make_tile<kKind, kMode, kBN, kPair>(p, idx, rank, pfx);
+            if (!t.valid) continue;
             if (!mbar_wait(&acc_full[buf], acc_phase, abort_flag)) break;
             tc_fence_after();
-            float scale = 1.0f;
-            if (kKind == kKindNVFP4) scale = __ldg(p.a_outer + t.row0 + r) * __ldg(p.b_outer + t.e);
-            const int64_t orow = t.row0 + r;
-            const uint32_t taddr = tmem + (uint32_t)(buf * kBN) + ((uint32_t)(q * 32) << 16) + cb;
-            if (kOutBF16) {
-                // 32 rows x kCols bf16 per warp, written by TMA tensor stores of
-                // 64-column boxes staged in this warp's 4 KB of shared memory
-                // (128-byte swizzle: 16-byte chunk c of row r at c ^ (r % 8)).
-                uint8_t* stg = smem + L::kStagingOff + (warp - 8) * 4096;
-                const uint32_t srow = smem_u32(stg) + (uint32_t)lane * 128u;
-                const int ox = (int)(t.col0 + cb), oy = (int)(t.row0 + q * 32);
-                if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");   // previous tile's box
-                __syncwarp();
-                uint32_t pk[kCols > 64 ? kCols / 2 - 32 : 1];  // columns 64.. held until the staging buffer frees
-#pragma unroll
-                for (int c = 0; c < kCols; c += 32) {
-                    float v[32];
-                    if (t.k_tiles > 0) tmem_ld_32x32b_x32(taddr + c, v);
-                    else {
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) v[i] = 0.0f;
-                    }
-                    uint32_t w[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        __nv_bfloat162 b = __floats2bfloat162_rn(v[2 * i] * scale, v[2 * i + 1] * scale);
-                        w[i] = *reinterpret_cast<uint32_t*>(&b);
-                    }
-                    if (c < 64) {
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const uint32_t chunk = (uint32_t)((c / 8 + i) ^ (lane & 7));
-                            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
-                                         :: "r"(srow + chunk * 16u), "r"(w[4 * i]), "r"(w[4 * i + 1]), "r"(w[4 * i + 2]),
-                                            "r"(w[4 * i + 3]) : "memory");
-                        }
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) pk[(c - 64) / 2 + i] = w[i];
-                    }
-                }
+            auto release = [&]() {
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&acc_empty[buf]);
-                // box 0 (columns 0..63 of this warp's block)
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                __syncwarp();
                 if (lane == 0) {
-                    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];"
-                                 :: "l"(reinterpret_cast<uint64_t>(&tmOut)), "r"(ox), "r"(oy), "r"(smem_u32(stg)) : "memory");
-                    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-                    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+                    if (kPair) mbar_arrive_cluster(acc_empty_lead[buf]);
+                    else mbar_arrive(&acc_empty[buf]);
                 }
-                __syncwarp();
-                if (kCols > 64) {
-                    // box 1 (columns 64..127) from registers
+            };
+            if (!t.store) {
+                release();
+            } else {
+                float scale = 1.0f;
+                if (kKind == kKindNVFP4) scale = __ldg(p.a_outer + t.row0 + r) * __ldg(p.b_outer + t.e);
+                const int64_t orow = t.row0 + r;
+                const uint32_t taddr = tmem + (uint32_t)(buf * kBN) + ((uint32_t)(q * 32) << 16) + cb;
+                if (kOutBF16) {
+                    // 32 rows x kCols bf16 per warp, written by TMA tensor stores of
+                    // 64-column boxes staged in this warp's 4 KB of shared memory
+                    // (128-byte swizzle: 16-byte chunk c of row r at c ^ (r % 8)).
+                    uint8_t* stg = smem + L::kStagingOff + (warp - 8) * 4096;
+                    const uint32_t srow = smem_u32(stg) + (uint32_t)lane * 128u;
+                    const int ox = (int)(t.col0 + cb), oy = (int)(t.row0 + q * 32);
+                    if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");   // previous tile's box
+                    __syncwarp();
+                    uint32_t pk[kCols > 64 ? kCols / 2 - 32 : 1];  // columns 64.. held until the staging buffer frees
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const uint32_t chunk = (uint32_t)(i ^ (lane & 7));
-                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
-                                     :: "r"(srow + chunk * 16u), "r"(pk[4 * i]), "r"(pk[4 * i + 1]), "r"(pk[4 * i + 2]),
-                                        "r"(pk[4 * i + 3]) : "memory");
+                    for (int c = 0; c < kCols; c += 32) {
+                        float v[32];
+                        if (t.k_tiles > 0) tmem_ld_32x32b_x32(taddr + c, v);
+                        else {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+                        }
+                        uint32_t w[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            __nv_bfloat162 b = __floats2bfloat162_rn(v[2 * i] * scale, v[2 * i + 1] * scale);
+                            w[i] = *reinterpret_cast<uint32_t*>(&b);
+                        }
+                        if (c < 64) {
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const uint32_t chunk = (uint32_t)((c / 8 + i) ^ (lane & 7));
+                                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                                             :: "r"(srow + chunk * 16u), "r"(w[4 * i]), "r"(w[4 * i + 1]),
+                                                "r"(w[4 * i + 2]), "r"(w[4 * i + 3]) : "memory");
+                            }
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) pk[(c - 64) / 2 + i] = w[i];
+                        }
                     }
+                    release();
+                    // box 0 (columns 0..63 of this warp's block)
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                     __syncwarp();
                     if (lane == 0) {
                         asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];"
-                                     :: "l"(reinterpret_cast<uint64_t>(&tmOut)), "r"(ox + 64), "r"(oy), "r"(smem_u32(stg)) : "memory");
+                                     :: "l"(reinterpret_cast<uint64_t>(&tmOut)), "r"(ox), "r"(oy), "r"(smem_u32(stg))
+                                     : "memory");
                         asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                        asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
                     }
-                }
-            } else {
-                float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow * p.ldo + t.col0 + cb);
+                    __syncwarp();
+                    if (kCols > 64) {
+                        // box 1 (columns 64..127) from registers
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const uint32_t chunk = (uint32_t)(i ^ (lane & 7));
+                            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                                         :: "r"(srow + chunk * 16u), "r"(pk[4 * i]), "r"(pk[4 * i + 1]),
+                                            "r"(pk[4 * i + 2]), "r"(pk[4 * i + 3]) : "memory");
+                        }
+                        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                        __syncwarp();
+                        if (lane == 0) {
+                            asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];"
+                                         :: "l"(reinterpret_cast<uint64_t>(&tmOut)), "r"(ox + 64), "r"(oy),
+                                            "r"(smem_u32(stg)) : "memory");
+                            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                        }
+                    }
+                } else {
+                    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow * p.ldo + t.col0 + cb);
 #pragma unroll 1
-                for (int c = 0; c < kCols; c += 32) {
-                    float v[32];
-                    if (t.k_tiles > 0) tmem_ld_32x32b_x32(taddr + c, v);
-                    else {
+                    for (int c = 0; c < kCols; c += 32) {
+                        float v[32];
+                        if (t.k_tiles > 0) tmem_ld_32x32b_x32(taddr + c, v);
+                        else {
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+                            for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+                        }
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            dst[c / 4 + i] = make_float4(v[4 * i] * scale, v[4 * i + 1] * scale, v[4 * i + 2] * scale,
+                                                         v[4 * i + 3] * scale);
                     }
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        dst[c / 4 + i] = make_float4(v[4 * i] * scale, v[4 * i + 1] * scale, v[4 * i + 2] * scale,
-                                                     v[4 * i + 3] * scale);
+                    release();
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&acc_empty[buf]);
             }
             if (++buf == L::kAccBufs) { buf = 0; acc_phase ^= 1u; }
         }
         if (kOutBF16 && lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
     }
 
+    // Teardown: every MMA has completed (the epilogue saw each accumulator's
+    // commit) and every TMEM read is done before the columns are freed; a
+    // pair frees its joint allocation only once both CTAs are here.
     tc_fence_before();
     __syncthreads();
+    if (kPair) cluster_sync();
     if (warp == 1) {
         __syncwarp();
         tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
+        tmem_dealloc<kPair>(tmem, kTmemCols);
     }
 }
 
@@ -644,37 +829,69 @@ int num_sms() {
     return n;
 }
 
-template <int kKind, int kMode, int kBN, bool kOutBF16>
-int launch(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mo, const GemmArgs& args, int64_t max_tiles,
+// Largest grid of co-resident CTA pairs for one pair kernel on this device.
+template <typename Kern>
+int max_pairs(Kern kern, const cudaLaunchConfig_t& cfg) {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+    if (cached[dev] > 0) return cached[dev];
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess || clusters <= 0) {
+        (void)cudaGetLastError();
+        clusters = num_sms() / 2;
+    }
+    cached[dev] = clusters;
+    return clusters;
+}
+
+template <int kKind, int kMode, int kBN, bool kOutBF16, bool kPair>
+int launch(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mo, const GemmArgs& args, int64_t items,
            cudaStream_t stream) {
-    using L = Smem<kKind, kBN>;
-    auto kern = grouped_gemm_kernel<kKind, kMode, kBN, kOutBF16>;
+    using L = Smem<kKind, kBN, kPair>;
+    auto kern = grouped_gemm_kernel<kKind, kMode, kBN, kOutBF16, kPair>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes) != cudaSuccess)
         return mx_launch_status();
-    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(max_tiles, num_sms()));
-    kern<<<(unsigned)grid, kThreads, L::kBytes, stream>>>(ma, mb, mo, args);
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = L::kBytes;
+    cfg.stream = stream;
+    int64_t slots = num_sms();
+    if (kPair) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        cfg.gridDim = dim3(2);
+        slots = max_pairs(kern, cfg);
+    }
+    const int64_t n = std::max<int64_t>(1, std::min<int64_t>(items, slots));
+    cfg.gridDim = dim3((unsigned)(kPair ? 2 * n : n));
+    if (cudaLaunchKernelEx(&cfg, kern, ma, mb, mo, args) != cudaSuccess) return mx_launch_status();
     return mx_launch_status();
 }
 
-// Tile width: 256 columns (one accumulator) whenever the output width allows
-// it; 128 columns (two accumulators) otherwise.  Measured on B200, the wide
-// tile is faster even for short K loops: it halves the A traffic per flop.
+// CTA pairs with 256 x 256 output tiles wherever the shape allows (measured
+// on B200: halving each CTA's B traffic per flop and the deeper pipeline it
+// buys lift the tensor pipe's duty cycle); otherwise single CTAs with 128 x
+// 128 tiles and two accumulators.
 template <int kKind, int kMode>
-int dispatch(int64_t out_cols, int64_t out_rows, int64_t k_stages, int out_dtype, const CUtensorMap& ma256,
-             const CUtensorMap& mb256, const CUtensorMap& ma128, const CUtensorMap& mb128, const GemmArgs& args,
-             int64_t tiles128, cudaStream_t stream) {
+int dispatch(bool pair, int64_t out_rows, int64_t out_cols, int out_dtype, const CUtensorMap& ma,
+             const CUtensorMap& mb, const GemmArgs& args, int64_t items_pair, int64_t items_single,
+             cudaStream_t stream) {
     CUtensorMap mo;
     memset(&mo, 0, sizeof(mo));
-    if (out_dtype == MX_OUT_BF16)
-        if (int st = make_out_map(&mo, args.out, out_rows, out_cols)) return st;
-    (void)k_stages;
-    const bool wide = out_cols % 256 == 0;
     const bool bf16 = out_dtype == MX_OUT_BF16;
-    if (wide)
-        return bf16 ? launch<kKind, kMode, 256, true>(ma256, mb256, mo, args, tiles128 / 2, stream)
-                    : launch<kKind, kMode, 256, false>(ma256, mb256, mo, args, tiles128 / 2, stream);
-    return bf16 ? launch<kKind, kMode, 128, true>(ma128, mb128, mo, args, tiles128, stream)
-                : launch<kKind, kMode, 128, false>(ma128, mb128, mo, args, tiles128, stream);
+    if (bf16)
+        if (int st = make_out_map(&mo, args.out, out_rows, out_cols)) return st;
+    if (pair)
+        return bf16 ? launch<kKind, kMode, 256, true, true>(ma, mb, mo, args, items_pair, stream)
+                    : launch<kKind, kMode, 256, false, true>(ma, mb, mo, args, items_pair, stream);
+    return bf16 ? launch<kKind, kMode, 128, true, false>(ma, mb, mo, args, items_single, stream)
+                : launch<kKind, kMode, 128, false, false>(ma, mb, mo, args, items_single, stream);
 }
 
 }  // namespace
@@ -703,16 +920,14 @@ extern "C" int grouped_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_sf, c
     if (M_cap >= (int64_t)1 << 31 || E * N >= (int64_t)1 << 31 || K / 2 >= (int64_t)1 << 31) return MX_EINVAL;
     if (int st = mx_check_device()) return st;
     if (M_cap == 0) return MX_OK;
-    CUtensorMap ma, mb, mb2;
+    CUtensorMap ma, mb;
     if (int st = make_map(&ma, a_codes, M_cap, K / 2, kBM)) return st;
     if (int st = make_map(&mb, b_codes, E * N, K / 2, 128)) return st;
-    if (N % 256 == 0)
-        if (int st = make_map(&mb2, b_codes, E * N, K / 2, 256)) return st;
     GemmArgs a{};
     a.sfa = a_sf; a.sfb = b_sf; a.a_outer = a_outer; a.b_outer = b_outer; a.seg = seg_offsets; a.out = out;
     a.E = E; a.M_cap = M_cap; a.N = N; a.K = K;
     a.sfa_groups = K / 64; a.sfb_groups = K / 64; a.ldo = N;
-    return dispatch<kKindNVFP4, kModeRows>(N, M_cap, K / 2 / kStageBytesK, out_dtype, ma, mb2, ma, mb, a,
+    return dispatch<kKindNVFP4, kModeRows>(N % 256 == 0 && E <= kMaxPairExperts, M_cap, N, out_dtype, ma, mb, a, (M_cap / kBM) * (N / 256),
                                            (M_cap / kBM) * (N / 128), stream);
 }
 
@@ -736,22 +951,18 @@ extern "C" int grouped_gemm_mxfp8(int mode, const uint8_t* a_codes, const uint8_
     a.E = E; a.M_cap = M_cap; a.N = N; a.K = K;
     if (mode == MX_GEMM_DGRAD) {
         // A [M_cap, K], B [N, E*K]; out [M_cap, N]
-        CUtensorMap mb2;
         if (int st = make_map(&ma, a_codes, M_cap, K, kBM)) return st;
         if (int st = make_map(&mb, b_codes, N, E * K, 128)) return st;
-        if (N % 256 == 0)
-            if (int st = make_map(&mb2, b_codes, N, E * K, 256)) return st;
         a.sfa_groups = K / 128; a.sfb_groups = E * K / 128; a.ldo = N;
-        return dispatch<kKindMXFP8, kModeRows>(N, M_cap, K / kStageBytesK, out_dtype, ma, mb2, ma, mb, a,
-                                               (M_cap / kBM) * (N / 128), stream);
+        return dispatch<kKindMXFP8, kModeRows>(N % 256 == 0 && E <= kMaxPairExperts, M_cap, N, out_dtype, ma, mb, a,
+                                               (M_cap / kBM) * (N / 256), (M_cap / kBM) * (N / 128), stream);
     }
     // WGRAD: A [N, M_cap], B [K, M_cap]; out [E, N, K]
     if (M_cap == 0) return MX_EINVAL;
-    CUtensorMap mb2;
     if (int st = make_map(&ma, a_codes, N, M_cap, kBM)) return st;
     if (int st = make_map(&mb, b_codes, K, M_cap, 128)) return st;
-    if (K % 256 == 0)
-        if (int st = make_map(&mb2, b_codes, K, M_cap, 256)) return st;
     a.sfa_groups = M_cap / 128; a.sfb_groups = M_cap / 128; a.ldo = K;
-    return dispatch<kKindMXFP8, kModeWgrad>(K, E * N, 0, out_dtype, ma, mb2, ma, mb, a, E * (N / kBM) * (K / 128), stream);
+    const bool pair = N % 256 == 0 && K % 256 == 0;
+    return dispatch<kKindMXFP8, kModeWgrad>(pair, E * N, K, out_dtype, ma, mb, a, E * (N / 256) * (K / 256),
+                                            E * (N / 128) * (K / 128), stream);
 }
