@@ -236,20 +236,28 @@ __device__ __forceinline__ void mma_block_scaled(uint32_t d_tmem, uint64_t a_des
 #undef MX_MMA_ASM
 }
 
-// 32 columns of fp32 for this thread's TMEM lane, waited for inside the asm.
-__device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, float* v) {
-    uint32_t r[32];
+// Two 32-column loads in flight at once, waited for inside the same asm so no
+// use of the registers can be scheduled before the wait.
+__device__ __forceinline__ void tmem_ld2_32x32b_x32(uint32_t taddr0, uint32_t taddr1, float* v0, float* v1) {
+    uint32_t a[32], b[32];
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 "
                  "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-                 "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
+                 "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%64];\n\t"
+                 "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+                 "{%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+                 "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%65];\n\t"
                  "tcgen05.wait::ld.sync.aligned;"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-                   "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-                   "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-                   "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-                 : "r"(taddr) : "memory");
+                 : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]), "=r"(a[4]), "=r"(a[5]), "=r"(a[6]), "=r"(a[7]),
+                   "=r"(a[8]), "=r"(a[9]), "=r"(a[10]), "=r"(a[11]), "=r"(a[12]), "=r"(a[13]), "=r"(a[14]), "=r"(a[15]),
+                   "=r"(a[16]), "=r"(a[17]), "=r"(a[18]), "=r"(a[19]), "=r"(a[20]), "=r"(a[21]), "=r"(a[22]), "=r"(a[23]),
+                   "=r"(a[24]), "=r"(a[25]), "=r"(a[26]), "=r"(a[27]), "=r"(a[28]), "=r"(a[29]), "=r"(a[30]), "=r"(a[31]),
+                   "=r"(b[0]), "=r"(b[1]), "=r"(b[2]), "=r"(b[3]), "=r"(b[4]), "=r"(b[5]), "=r"(b[6]), "=r"(b[7]),
+                   "=r"(b[8]), "=r"(b[9]), "=r"(b[10]), "=r"(b[11]), "=r"(b[12]), "=r"(b[13]), "=r"(b[14]), "=r"(b[15]),
+                   "=r"(b[16]), "=r"(b[17]), "=r"(b[18]), "=r"(b[19]), "=r"(b[20]), "=r"(b[21]), "=r"(b[22]), "=r"(b[23]),
+                   "=r"(b[24]), "=r"(b[25]), "=r"(b[26]), "=r"(b[27]), "=r"(b[28]), "=r"(b[29]), "=r"(b[30]), "=r"(b[31])
+                 : "r"(taddr0), "r"(taddr1) : "memory");
 #pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+    for (int i = 0; i < 32; ++i) { v0[i] = __uint_as_float(a[i]); v1[i] = __uint_as_float(b[i]); }
 }
 
 // ---------------------------------------------------------------------------
@@ -265,7 +273,6 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, float* v) {
 // 0's rows (valid memory, no special case in the pipeline) and stores nothing.
 constexpr int kMaxPairExperts = 768;    // prefix capacity (shared memory)
 struct Tile {
-    bool valid;         // false: a hole in the item list, no work
     bool store;         // false: this CTA's half lies outside the expert
     int64_t e;          // expert
     int64_t row0;       // first output row of this CTA (ROWS: token row; WGRAD: row of out viewed as [E*N, K])
@@ -324,7 +331,6 @@ __device__ __forceinline__ void build_pair_prefix(const GemmArgs& p, int32_t* pf
 template <int kKind, int kMode, int kBN, bool kPair>
 __device__ __forceinline__ Tile make_tile(const GemmArgs& p, int64_t idx, uint32_t rank, const int32_t* pfx) {
     Tile t;
-    t.valid = true;
     t.store = true;
     const int64_t half = kPair ? (int64_t)rank * kBM : 0;      // this CTA's row offset inside a pair item
     const int64_t b_half = kPair ? (int64_t)rank * (kBN / 2) : 0;
@@ -388,6 +394,14 @@ __device__ __forceinline__ Tile make_tile(const GemmArgs& p, int64_t idx, uint32
 // (128 rows), of B (kBN rows, or kBN/2 for a pair) and the stage's scale
 // atoms: SFA for this CTA's 128 rows and SFB for all kBN columns (each CTA of
 // a pair keeps a full copy: the MMA reads B's scales from every CTA's TMEM).
+//
+// TMEM (512 columns): two accumulator buffers of kBN columns at 0 and
+// kAccStride, then a ring of kSfSlots scale regions.  When 2 kBN columns do
+// not fit beside the scales the buffers overlap in kOvChunks 32-column chunks:
+// the epilogue drains those first and releases them, so the next tile's MMAs
+// wait for a fraction of the drain instead of all of it.  NVFP4 pairs keep
+// only two scale regions (a ring released by MMA commits, decoupled from the
+// shared-memory stages) to make that overlap small.
 constexpr int kSmemLimit = 227 * 1024;
 template <int kKind, int kBN, bool kPair>
 struct Smem {
@@ -400,14 +414,14 @@ struct Smem {
     static constexpr int kAbTx = kA + kB;                               // operand bytes per stage and CTA
     static constexpr int kSfTx = kSfa + kSfb;
     static constexpr int kStage = (kAbTx + kSfTx + 1023) / 1024 * 1024;  // stride keeps every SW128 tile 1024-aligned
-    static constexpr int kStaging = 8 * 4096;                           // epilogue: one 64x32 bf16 box per warp
+    static constexpr int kStaging = 8 * 4096;                           // epilogue: 4 KB of store boxes per warp
     static constexpr int kSfaCols = 4 * kAtomsA;
     static constexpr int kSfbCols = 4 * kAtomsB;
     static constexpr int kSfRegion = kSfaCols + kSfbCols;
     static constexpr int kPfxBytes = kPair ? 4 * (kMaxPairExperts + 4) : 0;
     static constexpr int kFixed = kStaging + 512 + kPfxBytes + 1024;    // + barriers + prefix + alignment slack
     static constexpr int fit(int s) {
-        return (s * kStage + kFixed <= kSmemLimit && kBN + s * kSfRegion <= kTmemCols) ? s : 0;
+        return s * kStage + kFixed <= kSmemLimit ? s : 0;
     }
     static constexpr int kStages = fit(6) ? 6 : fit(5) ? 5 : fit(4) ? 4 : fit(3) ? 3 : 2;
     static constexpr int kStagingOff = kStages * kStage;
@@ -415,11 +429,16 @@ struct Smem {
     static constexpr int kBarOff = kStagingOff + kStaging;
     static constexpr int kPfxOff = kBarOff + 512;
     static constexpr int kBytes = kPfxOff + kPfxBytes + 1024;
-    // TMEM: accumulator buffer(s), then one scale region per stage
-    static constexpr int kAccBufs = (2 * kBN + kStages * kSfRegion <= kTmemCols) ? 2 : 1;
-    static constexpr int kSfCol = kAccBufs * kBN;
-    static_assert(kSfCol + kStages * kSfRegion <= kTmemCols, "TMEM budget");
     static_assert(kBytes <= kSmemLimit, "shared memory budget");
+    // TMEM
+    static constexpr int kSfSlots = (kPair && kKind == kKindNVFP4) ? 2 : kStages;
+    static constexpr int kSfCols = kSfSlots * kSfRegion;
+    static constexpr int kAccStride = (kTmemCols - kBN - kSfCols) / 32 * 32 < kBN
+                                    ? (kTmemCols - kBN - kSfCols) / 32 * 32 : kBN;
+    static constexpr int kOvChunks = (kBN - kAccStride) / 32;           // chunks shared by the two buffers
+    static constexpr int kSfCol = kAccStride + kBN;
+    static_assert(kSfCol + kSfCols <= kTmemCols && kAccStride > 0, "TMEM budget");
+    static_assert(kOvChunks <= 4, "shared chunks must fall in the epilogue's first load group");
 };
 
 __device__ __forceinline__ void tmem_st_32x32b_x4(uint32_t taddr, const uint4& v) {
@@ -439,15 +458,18 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     const __grid_constant__ CUtensorMap tmOut, const GemmArgs p) {
     using L = Smem<kKind, kBN, kPair>;
     constexpr int kStages = L::kStages;
+    constexpr int kSlots = L::kSfSlots;
+    constexpr bool kSfRing = kSlots < kStages;                          // scale regions released by MMA commits
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);   // operands landed (pair: leader's counts both CTAs)
-    uint64_t* sf_full = full + kStages;                                 // scales written to TMEM (pair: both CTAs)
-    uint64_t* empty = sf_full + kStages;                                // stage consumed by the MMAs
+    uint64_t* empty = full + kStages;                                   // stage consumed by the MMAs
     uint64_t* sf_landed = empty + kStages;                              // pair: this CTA's scale atoms landed
-    uint64_t* acc_full = sf_landed + kStages;    // [2]: accumulator buffer b ready
-    uint64_t* acc_empty = acc_full + 2;          // [2]: accumulator buffer b drained (pair: both CTAs)
-    uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+    uint64_t* sf_full = sf_landed + kStages;                            // [kSlots] scales in TMEM (pair: both CTAs)
+    uint64_t* sf_free = sf_full + kSlots;                               // [kSlots] scale region read by the MMAs
+    uint64_t* acc_full = sf_free + kSlots;       // [2]: accumulator buffer b ready
+    uint64_t* acc_free = acc_full + 2;           // [2]: see the epilogue (pair: both CTAs report)
+    uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(acc_free + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -462,16 +484,19 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&sf_full[s], kPair ? 8 : 4);
             mbar_init(&empty[s], 1);
             mbar_init(&sf_landed[s], 1);
         }
-        for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], kPair ? 16 : 8); }
+        for (int s = 0; s < kSlots; ++s) {
+            mbar_init(&sf_full[s], kPair ? 8 : 4);
+            mbar_init(&sf_free[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_free[b], kPair ? 16 : 8); }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
         asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
-        if (kOutBF16) asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(&tmOut)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(&tmOut)) : "memory");
     }
     if (kPair) cluster_sync();                  // the peer's barriers exist before anything arrives on them
     if (warp == 1) tmem_alloc<kPair>(tmem_base_slot, kTmemCols);
@@ -491,7 +516,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             bool ok = true;
             for (int64_t idx = first; idx < total && ok; idx += stride) {
                 const Tile t = make_tile<kKind, kMode, kBN, kPair>(p, idx, rank, pfx);
-                if (!t.valid) continue;
                 for (int64_t kt = 0; kt < t.k_tiles; ++kt) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
                     uint8_t* sa = smem + stage * L::kStage;
@@ -541,28 +565,34 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer (a pair's leader only)
+        // Tile i accumulates into buffer i & 1.  With disjoint buffers it
+        // waits until tile i-2 left its buffer; with overlapping buffers until
+        // tile i-1's shared chunks were drained (which implies the former).
         if (lane == 0 && rank == 0) {
             constexpr uint32_t kFmt = kKind == kKindNVFP4 ? 1u : 0u;      // E2M1 / E4M3
             constexpr uint32_t kScaleFmt = kKind == kKindNVFP4 ? 0u : 1u; // UE4M3 / UE8M0
             constexpr int kM = kPair ? 2 * kBM : kBM;
-            int stage = 0, buf = 0;
-            uint32_t phase = 0, acc_phase = 0;
+            int stage = 0, slot = 0;
+            uint32_t phase = 0, sphase = 0, it = 0;
             bool ok = true;
             for (int64_t idx = first; idx < total && ok; idx += stride) {
                 const Tile t = make_tile<kKind, kMode, kBN, kPair>(p, idx, rank, pfx);
-                if (!t.valid) continue;
-                if (!mbar_wait(&acc_empty[buf], acc_phase ^ 1u, abort_flag)) break;
+                if (L::kOvChunks > 0) {
+                    if (it > 0 && !mbar_wait(&acc_free[(it - 1) & 1], ((it - 1) >> 1) & 1u, abort_flag)) break;
+                } else {
+                    if (!mbar_wait(&acc_free[it & 1], ((it >> 1) & 1u) ^ 1u, abort_flag)) break;
+                }
                 tc_fence_after();
-                const uint32_t acc = tmem + (uint32_t)(buf * kBN);
+                const uint32_t acc = tmem + (uint32_t)((it & 1) * L::kAccStride);
                 for (int64_t kt = 0; kt < t.k_tiles; ++kt) {
-                    if (!mbar_wait(&full[stage], phase, abort_flag) || !mbar_wait(&sf_full[stage], phase, abort_flag)) {
+                    if (!mbar_wait(&full[stage], phase, abort_flag) || !mbar_wait(&sf_full[slot], sphase, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const uint8_t* sa = smem + stage * L::kStage;
                     const uint8_t* sb = sa + L::kA;
-                    const uint32_t sfa = tmem + L::kSfCol + stage * L::kSfRegion;
+                    const uint32_t sfa = tmem + L::kSfCol + slot * L::kSfRegion;
                     const uint32_t sfb = sfa + L::kSfaCols;
                     const uint32_t a0 = smem_u32(sa), b0 = smem_u32(sb);
 #pragma unroll
@@ -581,11 +611,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                                                        sfa_t, sfb_t, (kt > 0 || j > 0) ? 1u : 0u);
                     }
                     tc_commit<kPair>(&empty[stage]);
+                    if (kSfRing) tc_commit<kPair>(&sf_free[slot]);
                     if (++stage == kStages) { stage = 0; phase ^= 1u; }
+                    if (++slot == kSlots) { slot = 0; sphase ^= 1u; }
                 }
                 if (!ok) break;
-                tc_commit<kPair>(&acc_full[buf]);
-                if (++buf == L::kAccBufs) { buf = 0; acc_phase ^= 1u; }
+                tc_commit<kPair>(&acc_full[it & 1]);
+                ++it;
             }
         }
     } else if (warp >= 4 && warp < 8) {
@@ -599,12 +631,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         // In a pair each CTA fills its own TMEM and reports to the leader.
         const int q = warp & 3;
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-        int stage = 0;
-        uint32_t phase = 0;
+        int stage = 0, slot = 0;
+        uint32_t phase = 0, sphase = 0;
         bool ok = true;
         for (int64_t idx = first; idx < total && ok; idx += stride) {
             const Tile t = make_tile<kKind, kMode, kBN, kPair>(p, idx, rank, pfx);
-            if (!t.valid) continue;
             for (int64_t kt = 0; kt < t.k_tiles; ++kt) {
                 if (!mbar_wait(kPair ? &sf_landed[stage] : &full[stage], phase, abort_flag)) { ok = false; break; }
                 const uint8_t* ssfa = smem + stage * L::kStage + L::kA + L::kB;
@@ -614,8 +645,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 for (int j = 0; j < L::kAtomsA; ++j) va[j] = reinterpret_cast<const uint4*>(ssfa + j * 512)[lane];
 #pragma unroll
                 for (int j = 0; j < L::kAtomsB; ++j) vb[j] = reinterpret_cast<const uint4*>(ssfb + j * 512)[lane];
+                if (kSfRing && !mbar_wait(&sf_free[slot], sphase ^ 1u, abort_flag)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t sfa = tmem + lane_base + L::kSfCol + stage * L::kSfRegion;
+                const uint32_t sfa = tmem + lane_base + L::kSfCol + slot * L::kSfRegion;
                 const uint32_t sfb = sfa + L::kSfaCols;
 #pragma unroll
                 for (int j = 0; j < L::kAtomsA; ++j) tmem_st_32x32b_x4(sfa + 4 * j, va[j]);
@@ -628,41 +660,45 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) {
-                    if (kPair) mbar_arrive_cluster(map_to_rank(&sf_full[stage], 0));
-                    else mbar_arrive(&sf_full[stage]);
+                    if (kPair) mbar_arrive_cluster(map_to_rank(&sf_full[slot], 0));
+                    else mbar_arrive(&sf_full[slot]);
                 }
                 if (++stage == kStages) { stage = 0; phase ^= 1u; }
+                if (++slot == kSlots) { slot = 0; sphase ^= 1u; }
             }
         }
     } else if (warp >= 8) {
         // ------------------------------------------------------------ epilogue
-        // Eight warps: warp w reads TMEM lane quarter w%4 (the hardware lets a
-        // warp touch only its own 32 lanes) and column half (w-8)/4.  bf16
-        // output: each 32-column chunk is scaled and packed as it arrives, the
-        // accumulator is released after the last chunk, and the stores overlap
-        // the next tile's main loop.  fp32 output stores chunk by chunk and
-        // releases the accumulator afterwards.  A pair's CTAs each drain their
-        // own 128 rows and both report to the leader.
-        constexpr int kCols = kBN / 2;
+        // Eight warps: warp w reads TMEM lane quarter w%4 (a warp may touch
+        // only its own 32 lanes) and every other 32-column chunk of the tile
+        // (parity (w-8)/4), in a drain order that puts the chunks shared with
+        // the other accumulator buffer first.  Chunks are loaded two at a
+        // time; after the first pair (which holds every shared chunk) the warp
+        // reports on acc_free, then converts, stages each chunk as one 32x32
+        // box in shared memory and writes it with a TMA tensor store.  bf16
+        // boxes (64-byte rows, 64-byte swizzle) alternate between two 2 KB
+        // buffers; fp32 boxes (128-byte rows, 128-byte swizzle) use one 4 KB
+        // buffer.  A pair's CTAs each drain their own 128 rows.
+        constexpr int kChunks = kBN / 32;
+        constexpr int kOv = L::kOvChunks;
         const int q = warp & 3;
-        const int half = (warp - 8) >> 2;
+        const int h = (warp - 8) >> 2;
         const int r = q * 32 + lane;
-        const int cb = half * kCols;
-        const uint32_t acc_empty_lead[2] = {kPair ? map_to_rank(&acc_empty[0], 0) : 0u,
-                                            kPair ? map_to_rank(&acc_empty[1], 0) : 0u};
-        uint32_t acc_phase = 0;
-        int buf = 0;
+        uint8_t* stg = smem + L::kStagingOff + (warp - 8) * 4096;
+        const uint32_t acc_free_lead[2] = {kPair ? map_to_rank(&acc_free[0], 0) : 0u,
+                                           kPair ? map_to_rank(&acc_free[1], 0) : 0u};
+        uint32_t it = 0, nbox = 0;
         for (int64_t idx = first; idx < total; idx += stride) {
             const Tile t = make_tile<kKind, kMode, kBN, kPair>(p, idx, rank, pfx);
-            if (!t.valid) continue;
-            if (!mbar_wait(&acc_full[buf], acc_phase, abort_flag)) break;
+            const int b = (int)(it & 1);
+            if (!mbar_wait(&acc_full[b], (it >> 1) & 1u, abort_flag)) break;
             tc_fence_after();
             auto release = [&]() {
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) {
-                    if (kPair) mbar_arrive_cluster(acc_empty_lead[buf]);
-                    else mbar_arrive(&acc_empty[buf]);
+                    if (kPair) mbar_arrive_cluster(acc_free_lead[b]);
+                    else mbar_arrive(&acc_free[b]);
                 }
             };
             if (!t.store) {
@@ -670,96 +706,75 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             } else {
                 float scale = 1.0f;
                 if (kKind == kKindNVFP4) scale = __ldg(p.a_outer + t.row0 + r) * __ldg(p.b_outer + t.e);
-                const int64_t orow = t.row0 + r;
-                const uint32_t taddr = tmem + (uint32_t)(buf * kBN) + ((uint32_t)(q * 32) << 16) + cb;
-                if (kOutBF16) {
-                    // 32 rows x kCols bf16 per warp, written by TMA tensor stores of
-                    // 64-column boxes staged in this warp's 4 KB of shared memory
-                    // (128-byte swizzle: 16-byte chunk c of row r at c ^ (r % 8)).
-                    uint8_t* stg = smem + L::kStagingOff + (warp - 8) * 4096;
-                    const uint32_t srow = smem_u32(stg) + (uint32_t)lane * 128u;
-                    const int ox = (int)(t.col0 + cb), oy = (int)(t.row0 + q * 32);
-                    if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");   // previous tile's box
-                    __syncwarp();
-                    uint32_t pk[kCols > 64 ? kCols / 2 - 32 : 1];  // columns 64.. held until the staging buffer frees
+                const uint32_t tbase = tmem + (uint32_t)(b * L::kAccStride) + ((uint32_t)(q * 32) << 16);
+                const int oy = (int)(t.row0 + q * 32);
 #pragma unroll
-                    for (int c = 0; c < kCols; c += 32) {
-                        float v[32];
-                        if (t.k_tiles > 0) tmem_ld_32x32b_x32(taddr + c, v);
-                        else {
+                for (int g = 0; g < kChunks / 4; ++g) {
+                    int col[2];
 #pragma unroll
-                            for (int i = 0; i < 32; ++i) v[i] = 0.0f;
-                        }
-                        uint32_t w[16];
+                    for (int u = 0; u < 2; ++u) {
+                        const int j = h + 4 * g + 2 * u;                // drain position
+                        col[u] = 32 * (b == 0 ? (j < kOv ? kChunks - kOv + j : j - kOv) : j);
+                    }
+                    float v[2][32];
+                    if (t.k_tiles > 0) {
+                        tmem_ld2_32x32b_x32(tbase + (uint32_t)col[0], tbase + (uint32_t)col[1], v[0], v[1]);
+                    } else {
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            __nv_bfloat162 b = __floats2bfloat162_rn(v[2 * i] * scale, v[2 * i + 1] * scale);
-                            w[i] = *reinterpret_cast<uint32_t*>(&b);
-                        }
-                        if (c < 64) {
+                        for (int u = 0; u < 2; ++u)
 #pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                const uint32_t chunk = (uint32_t)((c / 8 + i) ^ (lane & 7));
+                            for (int i = 0; i < 32; ++i) v[u][i] = 0.0f;
+                    }
+                    if (g == (kOv > 0 ? 0 : kChunks / 4 - 1)) release();
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        uint8_t* box;
+                        if (kOutBF16) {
+                            box = stg + (nbox & 1u) * 2048;
+                            if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+                            __syncwarp();
+                            const uint32_t row = smem_u32(box) + (uint32_t)lane * 64u;
+#pragma unroll
+                            for (int c = 0; c < 4; ++c) {
+                                uint32_t w[4];
+#pragma unroll
+                                for (int i = 0; i < 4; ++i) {
+                                    __nv_bfloat162 bb = __floats2bfloat162_rn(v[u][8 * c + 2 * i] * scale,
+                                                                              v[u][8 * c + 2 * i + 1] * scale);
+                                    w[i] = *reinterpret_cast<uint32_t*>(&bb);
+                                }
+                                const uint32_t sw = (uint32_t)(c ^ ((lane >> 1) & 3));
                                 asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
-                                             :: "r"(srow + chunk * 16u), "r"(w[4 * i]), "r"(w[4 * i + 1]),
-                                                "r"(w[4 * i + 2]), "r"(w[4 * i + 3]) : "memory");
+                                             :: "r"(row + sw * 16u), "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]) : "memory");
                             }
                         } else {
+                            box = stg;
+                            if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+                            __syncwarp();
+                            const uint32_t row = smem_u32(box) + (uint32_t)lane * 128u;
 #pragma unroll
-                            for (int i = 0; i < 16; ++i) pk[(c - 64) / 2 + i] = w[i];
-                        }
-                    }
-                    release();
-                    // box 0 (columns 0..63 of this warp's block)
-                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                    __syncwarp();
-                    if (lane == 0) {
-                        asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];"
-                                     :: "l"(reinterpret_cast<uint64_t>(&tmOut)), "r"(ox), "r"(oy), "r"(smem_u32(stg))
-                                     : "memory");
-                        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-                        asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-                    }
-                    __syncwarp();
-                    if (kCols > 64) {
-                        // box 1 (columns 64..127) from registers
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const uint32_t chunk = (uint32_t)(i ^ (lane & 7));
-                            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
-                                         :: "r"(srow + chunk * 16u), "r"(pk[4 * i]), "r"(pk[4 * i + 1]),
-                                            "r"(pk[4 * i + 2]), "r"(pk[4 * i + 3]) : "memory");
+                            for (int c = 0; c < 8; ++c) {
+                                const uint32_t sw = (uint32_t)(c ^ (lane & 7));
+                                asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};"
+                                             :: "r"(row + sw * 16u), "f"(v[u][4 * c] * scale), "f"(v[u][4 * c + 1] * scale),
+                                                "f"(v[u][4 * c + 2] * scale), "f"(v[u][4 * c + 3] * scale) : "memory");
+                            }
                         }
                         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                         __syncwarp();
                         if (lane == 0) {
                             asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];"
-                                         :: "l"(reinterpret_cast<uint64_t>(&tmOut)), "r"(ox + 64), "r"(oy),
-                                            "r"(smem_u32(stg)) : "memory");
+                                         :: "l"(reinterpret_cast<uint64_t>(&tmOut)), "r"((int)t.col0 + col[u]), "r"(oy),
+                                            "r"(smem_u32(box)) : "memory");
                             asm volatile("cp.async.bulk.commit_group;" ::: "memory");
                         }
+                        ++nbox;
                     }
-                } else {
-                    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow * p.ldo + t.col0 + cb);
-#pragma unroll 1
-                    for (int c = 0; c < kCols; c += 32) {
-                        float v[32];
-                        if (t.k_tiles > 0) tmem_ld_32x32b_x32(taddr + c, v);
-                        else {
-#pragma unroll
-                            for (int i = 0; i < 32; ++i) v[i] = 0.0f;
-                        }
-#pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            dst[c / 4 + i] = make_float4(v[4 * i] * scale, v[4 * i + 1] * scale, v[4 * i + 2] * scale,
-                                                         v[4 * i + 3] * scale);
-                    }
-                    release();
                 }
             }
-            if (++buf == L::kAccBufs) { buf = 0; acc_phase ^= 1u; }
+            ++it;
         }
-        if (kOutBF16 && lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+        if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
     }
 
     // Teardown: every MMA has completed (the epilogue saw each accumulator's
@@ -809,16 +824,20 @@ int make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t inner, int 
     return r == CUDA_SUCCESS ? MX_OK : MX_EINVAL;
 }
 
-// bf16 output [rows, cols] (row stride cols), box 64 x 32, 128-byte swizzle.
-int make_out_map(CUtensorMap* m, void* base, int64_t rows, int64_t cols) {
+// Output [rows, cols] (row stride cols), box 32 x 32: bf16 with 64-byte rows
+// and 64-byte swizzle, fp32 with 128-byte rows and 128-byte swizzle.
+int make_out_map(CUtensorMap* m, void* base, int64_t rows, int64_t cols, bool bf16) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return MX_EUNSUPPORTED;
+    const cuuint64_t esize = bf16 ? 2 : 4;
     const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-    const cuuint32_t box[2] = {64, 32};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols * esize};
+    const cuuint32_t box[2] = {32, 32};
     const cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r = fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    bf16 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? MX_OK : MX_EINVAL;
 }
 
@@ -883,10 +902,8 @@ int dispatch(bool pair, int64_t out_rows, int64_t out_cols, int out_dtype, const
              const CUtensorMap& mb, const GemmArgs& args, int64_t items_pair, int64_t items_single,
              cudaStream_t stream) {
     CUtensorMap mo;
-    memset(&mo, 0, sizeof(mo));
     const bool bf16 = out_dtype == MX_OUT_BF16;
-    if (bf16)
-        if (int st = make_out_map(&mo, args.out, out_rows, out_cols)) return st;
+    if (int st = make_out_map(&mo, args.out, out_rows, out_cols, bf16)) return st;
     if (pair)
         return bf16 ? launch<kKind, kMode, 256, true, true>(ma, mb, mo, args, items_pair, stream)
                     : launch<kKind, kMode, 256, false, true>(ma, mb, mo, args, items_pair, stream);

@@ -179,7 +179,7 @@ __device__ __forceinline__ uint32_t e4m3_sr_code(float xh, int e, uint32_t u) {
 }
 
 // ---------------------------------------------------------------------------
-// Hardware stochastic rounding (sm_100a cvt.rs) of two values onto E4M3.
+// Hardware stochastic rounding (sm_100a cvt.rs) onto E4M3.
 // cvt.rs.satfinite.e4m3x4.f32 d, {a, b, c, f}, rbits puts f's code in byte 0
 // and b's in byte 2; f adds rbits[15:0] and b adds rbits[31:16] as 16 random
 // bits just below the kept E4M3 bits and truncates (the carry rounds up).  With
@@ -187,15 +187,20 @@ __device__ __forceinline__ uint32_t e4m3_sr_code(float xh, int e, uint32_t u) {
 // u < floor(frac * 2^16): the rule of e4m3_sr_code<16>, in one instruction
 // (established by comparing the instruction with the oracle on a B200).  The
 // a and c lanes are not used: their random bits are not independent of b's
-// and f's.  y_lo / y_hi must be |y| <= 448; the result packs lo in bits 0-7
-// and hi in bits 8-15.
+// and f's.  Inputs must be |y| <= 448.
+//
+// Four consecutive elements: y0, y1 take the low and high halves of random
+// word u01, y2, y3 those of u23; the codes are packed
+// y0 | y1 << 8 | y2 << 16 | y3 << 24 by one byte permute.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t cvt_rs16_e4m3_pair(float y_lo, float y_hi, uint32_t u_lo, uint32_t u_hi) {
-    const uint32_t rbits = ~((u_hi << 16) | (u_lo & 0xffffu));
-    uint32_t d;
+__device__ __forceinline__ uint32_t cvt_rs16_e4m3_quad(float y0, float y1, float y2, float y3, uint32_t u01,
+                                                       uint32_t u23) {
+    uint32_t d0, d1;
     asm("cvt.rs.satfinite.e4m3x4.f32 %0, {%1, %2, %3, %4}, %5;"
-        : "=r"(d) : "f"(0.0f), "f"(y_hi), "f"(0.0f), "f"(y_lo), "r"(rbits));
-    return (d & 0xffu) | ((d >> 8) & 0xff00u);
+        : "=r"(d0) : "f"(0.0f), "f"(y1), "f"(0.0f), "f"(y0), "r"(~u01));
+    asm("cvt.rs.satfinite.e4m3x4.f32 %0, {%1, %2, %3, %4}, %5;"
+        : "=r"(d1) : "f"(0.0f), "f"(y3), "f"(0.0f), "f"(y2), "r"(~u23));
+    return __byte_perm(d0, d1, 0x6420);
 }
 
 // ---------------------------------------------------------------------------

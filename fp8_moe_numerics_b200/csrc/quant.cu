@@ -8,8 +8,6 @@
 
 namespace {
 
-constexpr int kWarpsPerBlock = 8;
-
 // Max of |bf16| over the 8 elements of a uint4, as the bf16 magnitude bits
 // (integer order equals numeric order for non-NaN magnitudes).
 __device__ __forceinline__ uint32_t absmax8_bf16(const uint4& v) {
@@ -36,72 +34,106 @@ __device__ __forceinline__ uint32_t nvfp4_block(const uint4& a, const uint4& b, 
     if (sc == 0) { packed = make_uint2(0u, 0u); return 0u; }
     float inv = __frcp_rn(__fmul_rn(e4m3_to_f32(sc), s));
     const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-    uint32_t out[2] = {0u, 0u};
+    uint32_t byte[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        uint32_t byte = cvt_e2m1x2(__fmul_rn(bf16_lo(w[i]), inv), __fmul_rn(bf16_hi(w[i]), inv));
-        out[i >> 2] |= byte << ((i & 3) * 8);
-    }
-    packed = make_uint2(out[0], out[1]);
+    for (int i = 0; i < 8; ++i) byte[i] = cvt_e2m1x2(__fmul_rn(bf16_lo(w[i]), inv), __fmul_rn(bf16_hi(w[i]), inv));
+    // bytes -> words with byte permutes (byte 1 of a code byte is zero)
+    packed = make_uint2(__byte_perm(__byte_perm(byte[0], byte[1], 0x1140), __byte_perm(byte[2], byte[3], 0x1140), 0x5410),
+                        __byte_perm(__byte_perm(byte[4], byte[5], 0x1140), __byte_perm(byte[6], byte[7], 0x1140), 0x5410));
     return sc;
 }
 
-// One warp per row; lane l handles 16-element blocks l, l+32, ...  Rows of up
-// to 32*16*kNB elements stay in registers; longer rows are read twice.
+// kTPR threads per row (a power of two, 16..256), 256 / kTPR rows per block.
+// Thread j of a row handles the 16-element blocks j, j + kTPR, ... (kNB of
+// them held in registers when the row fits, so each warp's loads cover
+// contiguous bytes); longer rows are read twice.  The row amax is reduced by
+// warp shuffles and, across the row's warps, through shared memory.  Scale
+// bytes of four consecutive blocks are merged by shuffles into one 32-bit
+// store when the row has a multiple of four blocks (`word_sf`).
 // GROUP: the outer scale is per group of rows and `outer` already holds the
 // group's amax bits (written by nvfp4_group_amax_kernel).
-template <int kNB, bool kGroup, int kLayout>
-__global__ void __launch_bounds__(kWarpsPerBlock * 32)
+constexpr int kRowThreads = 256;
+
+template <int kTPR, int kNB, bool kGroup, int kLayout>
+__global__ void __launch_bounds__(kRowThreads, kNB <= 4 ? 4 : 2)
 nvfp4_quant_rows_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t group_rows,
-                        uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, float* __restrict__ outer) {
+                        bool word_sf, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, float* __restrict__ outer) {
+    constexpr int kRPB = kRowThreads / kTPR;
+    __shared__ uint32_t wmax[kRowThreads / 32];
     const int lane = threadIdx.x & 31;
-    const int64_t row = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
-    if (row >= rows) return;
+    const int j = threadIdx.x % kTPR;
+    const int64_t row = (int64_t)blockIdx.x * kRPB + threadIdx.x / kTPR;
+    const bool active = row < rows;
     const int64_t nblk = cols >> 4;
-    const uint4* xr = reinterpret_cast<const uint4*>(x + row * cols);
+    const uint4* xr = reinterpret_cast<const uint4*>(x + (active ? row : 0) * cols);
 
     uint4 va[kNB], vb[kNB];
     uint32_t amax_bits = 0;
-    const bool resident = nblk <= 32 * kNB;
+    const bool resident = nblk <= (int64_t)kTPR * kNB;
 #pragma unroll
     for (int i = 0; i < kNB; ++i) {
-        int64_t blk = lane + 32 * i;
-        if (resident && blk < nblk) {
+        const int64_t blk = j + (int64_t)kTPR * i;
+        va[i] = make_uint4(0, 0, 0, 0);
+        vb[i] = va[i];
+        if (active && resident && blk < nblk) {
             va[i] = __ldcs(xr + 2 * blk);
             vb[i] = __ldcs(xr + 2 * blk + 1);
-            amax_bits = max(amax_bits, max(absmax8_bf16(va[i]), absmax8_bf16(vb[i])));
         }
     }
-    if (!resident) {
-        for (int64_t blk = lane; blk < nblk; blk += 32)
+#pragma unroll
+    for (int i = 0; i < kNB; ++i) amax_bits = max(amax_bits, max(absmax8_bf16(va[i]), absmax8_bf16(vb[i])));
+    if (active && !resident) {
+        for (int64_t blk = j; blk < nblk; blk += kTPR)
             amax_bits = max(amax_bits, max(absmax8_bf16(xr[2 * blk]), absmax8_bf16(xr[2 * blk + 1])));
     }
 
     float s;
     if (kGroup) {
-        s = __fdiv_rn(__uint_as_float(__float_as_uint(outer[row / group_rows])), 2688.0f);
+        const int64_t g = rows < ((int64_t)1 << 32) ? (int64_t)((uint32_t)row / (uint32_t)group_rows) : row / group_rows;
+        s = active ? __fdiv_rn(outer[g], 2688.0f) : 0.0f;
     } else {
-        amax_bits = warp_max_u32(amax_bits);
+        if (kTPR >= 32) {
+            amax_bits = warp_max_u32(amax_bits);
+        } else {                                          // rows of kTPR lanes inside a warp
+#pragma unroll
+            for (int o = kTPR / 2; o > 0; o >>= 1) amax_bits = max(amax_bits, __shfl_xor_sync(0xffffffffu, amax_bits, o));
+        }
+        if (kTPR > 32) {
+            if (lane == 0) wmax[threadIdx.x >> 5] = amax_bits;
+            __syncthreads();
+            const int w0 = (threadIdx.x / kTPR) * (kTPR / 32);
+#pragma unroll
+            for (int w = 0; w < kTPR / 32; ++w) amax_bits = max(amax_bits, wmax[w0 + w]);
+        }
         s = __fdiv_rn(__uint_as_float(amax_bits << 16), 2688.0f);
-        if (lane == 0) outer[row] = s;
+        if (active && j == 0) outer[row] = s;
     }
 
-    uint8_t* crow = codes + row * (cols >> 1);
+    uint8_t* crow = codes + (active ? row : 0) * (cols >> 1);
     auto emit = [&](int64_t blk, const uint4& a, const uint4& b) {
         uint2 packed = make_uint2(0u, 0u);
         uint32_t sc = 0;
-        if (s > 0.0f) sc = nvfp4_block(a, b, s, packed);
-        *reinterpret_cast<uint2*>(crow + blk * 8) = packed;
-        sf[sf_offset(row, blk, nblk, kLayout)] = (uint8_t)sc;
+        const bool live = active && blk < nblk;
+        if (live && s > 0.0f) sc = nvfp4_block(a, b, s, packed);
+        if (live) *reinterpret_cast<uint2*>(crow + blk * 8) = packed;
+        if (word_sf) {                                   // blocks 4m..4m+3 sit in lanes 4m'..4m'+3
+            uint32_t w = sc << (8 * (lane & 3));
+            w |= __shfl_xor_sync(0xffffffffu, w, 1);
+            w |= __shfl_xor_sync(0xffffffffu, w, 2);
+            if (live && (lane & 3) == 0) *reinterpret_cast<uint32_t*>(sf + sf_offset(row, blk, nblk, kLayout)) = w;
+        } else if (live) {
+            sf[sf_offset(row, blk, nblk, kLayout)] = (uint8_t)sc;
+        }
     };
     if (resident) {
 #pragma unroll
-        for (int i = 0; i < kNB; ++i) {
-            const int64_t blk = lane + 32 * i;
-            if (blk < nblk) emit(blk, va[i], vb[i]);
-        }
+        for (int i = 0; i < kNB; ++i) emit(j + (int64_t)kTPR * i, va[i], vb[i]);
     } else {
-        for (int64_t blk = lane; blk < nblk; blk += 32) emit(blk, xr[2 * blk], xr[2 * blk + 1]);
+        const int64_t nb_pad = (nblk + kTPR - 1) / kTPR * kTPR;   // every lane runs every shuffle
+        for (int64_t blk = j; blk < nb_pad; blk += kTPR) {
+            const bool in = active && blk < nblk;
+            emit(blk, in ? xr[2 * blk] : make_uint4(0, 0, 0, 0), in ? xr[2 * blk + 1] : make_uint4(0, 0, 0, 0));
+        }
     }
 }
 
@@ -202,11 +234,11 @@ __device__ __forceinline__ void tile_emit_transposed(const float* T, int64_t row
                 const uint4 rnd = philox4x32_10((uint64_t)(L0 / 8) + blk, stream_id, seed);
                 const uint32_t wd[4] = {rnd.x, rnd.y, rnd.z, rnd.w};
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int i = blk * 8 + 2 * q;     // elements i, i+1 use word q's halves
-                    const uint32_t pr = cvt_rs16_e4m3_pair(__fmul_rn(v[i], sc), __fmul_rn(v[i + 1], sc),
-                                                           wd[q] & 0xffffu, wd[q] >> 16);
-                    if ((q & 1) == 0) w[blk * 2 + (q >> 1)] = pr; else w[blk * 2 + (q >> 1)] |= pr << 16;
+                for (int q = 0; q < 4; q += 2) {       // elements i..i+3 use words q, q+1
+                    const int i = blk * 8 + 2 * q;
+                    w[blk * 2 + (q >> 1)] = cvt_rs16_e4m3_quad(__fmul_rn(v[i], sc), __fmul_rn(v[i + 1], sc),
+                                                               __fmul_rn(v[i + 2], sc), __fmul_rn(v[i + 3], sc),
+                                                               wd[q], wd[q + 1]);
                 }
             }
         } else if (kSR) {
@@ -273,11 +305,11 @@ mxfp8_tile_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, co
                 const uint4 rnd = philox4x32_10((uint64_t)(L0 / 8) + blk, stream_row, seed);
                 const uint32_t wd[4] = {rnd.x, rnd.y, rnd.z, rnd.w};
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
+                for (int q = 0; q < 4; q += 2) {
                     const int i = blk * 8 + 2 * q;
-                    const uint32_t pr = cvt_rs16_e4m3_pair(__fmul_rn(v[i], sc), __fmul_rn(v[i + 1], sc),
-                                                           wd[q] & 0xffffu, wd[q] >> 16);
-                    if ((q & 1) == 0) w[blk * 2 + (q >> 1)] = pr; else w[blk * 2 + (q >> 1)] |= pr << 16;
+                    w[blk * 2 + (q >> 1)] = cvt_rs16_e4m3_quad(__fmul_rn(v[i], sc), __fmul_rn(v[i + 1], sc),
+                                                               __fmul_rn(v[i + 2], sc), __fmul_rn(v[i + 3], sc),
+                                                               wd[q], wd[q + 1]);
                 }
             }
         } else if (kSR) {
@@ -369,25 +401,35 @@ extern "C" int nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t
     const uint16_t* xb = static_cast<const uint16_t*>(x);
     const int64_t ngroups = rows / group_rows;
     const int64_t nblk_row = cols / 16;
-    const dim3 block(kWarpsPerBlock * 32);
-    const dim3 grid((unsigned)((rows + kWarpsPerBlock - 1) / kWarpsPerBlock));
+    // word-sized scale stores need four blocks per row and 4-byte aligned rows
+    const bool word_sf = nblk_row % 4 == 0 && mx_aligned(sf, 4);
     return dispatch_layout(sf_layout, [&](auto L) {
         constexpr int kL = decltype(L)::value;
+        auto run = [&](auto kGroupC) {
+            constexpr bool kG = decltype(kGroupC)::value;
+            auto go = [&](auto kern, int tpr) {
+                const int64_t rpb = kRowThreads / tpr;
+                kern<<<(unsigned)((rows + rpb - 1) / rpb), kRowThreads, 0, stream>>>(xb, rows, cols, group_rows, word_sf,
+                                                                                       codes, sf, outer);
+            };
+            // four 16-element blocks (128 bytes) per thread in flight, 4 CTAs per SM:
+            // 128 KB of loads outstanding per SM covers HBM latency under load
+            if (nblk_row <= 64) go(nvfp4_quant_rows_kernel<16, 4, kG, kL>, 16);
+            else if (nblk_row <= 128) go(nvfp4_quant_rows_kernel<32, 4, kG, kL>, 32);
+            else if (nblk_row <= 256) go(nvfp4_quant_rows_kernel<64, 4, kG, kL>, 64);
+            else if (nblk_row <= 512) go(nvfp4_quant_rows_kernel<128, 4, kG, kL>, 128);
+            else if (nblk_row <= 1024) go(nvfp4_quant_rows_kernel<256, 4, kG, kL>, 256);
+            else go(nvfp4_quant_rows_kernel<256, 8, kG, kL>, 256);
+        };
         if (group_rows == 1) {
-            if (nblk_row <= 32 * 2)
-                nvfp4_quant_rows_kernel<2, false, kL><<<grid, block, 0, stream>>>(xb, rows, cols, 1, codes, sf, outer);
-            else
-                nvfp4_quant_rows_kernel<8, false, kL><<<grid, block, 0, stream>>>(xb, rows, cols, 1, codes, sf, outer);
+            run(std::false_type());
         } else {
             if (cudaMemsetAsync(outer, 0, sizeof(float) * ngroups, stream) != cudaSuccess) return mx_launch_status();
             const int64_t group_vec = group_rows * cols / 8;          // 16-byte vectors per group
             const int64_t chunk_vec = 16384;                            // 256 KiB per block
             const dim3 ag((unsigned)((group_vec + chunk_vec - 1) / chunk_vec), (unsigned)std::min<int64_t>(ngroups, 65535));
             nvfp4_group_amax_kernel<<<ag, kAmaxThreads, 0, stream>>>(xb, ngroups, group_vec, chunk_vec, outer);
-            if (nblk_row <= 32 * 2)
-                nvfp4_quant_rows_kernel<2, true, kL><<<grid, block, 0, stream>>>(xb, rows, cols, group_rows, codes, sf, outer);
-            else
-                nvfp4_quant_rows_kernel<8, true, kL><<<grid, block, 0, stream>>>(xb, rows, cols, group_rows, codes, sf, outer);
+            run(std::true_type());
             nvfp4_group_finish_kernel<<<(unsigned)((ngroups + 255) / 256), 256, 0, stream>>>(outer, ngroups);
         }
         return mx_launch_status();

@@ -63,7 +63,8 @@ def crafted_rows():
 # NVFP4 quantiser
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("rows,cols", [(256, 4096), (128, 1024), (384, 256), (7, 48), (130, 3072)])
+@pytest.mark.parametrize("rows,cols", [(256, 4096), (128, 1024), (384, 256), (7, 48), (130, 3072),
+                                       (16, 8192), (3, 12304), (5, 16400), (4, 40960)])
 def test_nvfp4_quantize_per_token_bit_exact(cuda, rows, cols):
     x = heavy_rows(rows, cols, seed=rows + cols)
     codes, sf, outer = oracle.nvfp4_quantize(x)
