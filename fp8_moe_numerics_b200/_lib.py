@@ -29,6 +29,7 @@ SZ = ctypes.c_size_t
 SIGNATURES = {
     "mx_version": (I32, []),
     "mx_last_cuda_error": (I32, []),
+    "mx_kernel_launches": (ctypes.c_ulonglong, []),
     "mx_sync_status": (I32, [P]),
     "mx_sf_bytes": (SZ, [I64, I64, I32, I32]),
     "nvfp4_quantize": (I32, [P, I64, I64, I64, P, P, P, I32, P]),
@@ -43,7 +44,7 @@ SIGNATURES = {
     "swiglu_fwd": (I32, [P, I64, I64, I32, P, P, P]),
     "swiglu_bwd": (I32, [P, P, I64, I64, I32, P, P, P]),
     "moe_combine": (I32, [P, P, P, I64, I64, I64, P, P]),
-    "moe_dispatch_grad": (I32, [P, P, P, I64, I64, I64, P, P]),
+    "moe_dispatch_grad": (I32, [P, P, P, P, I64, I64, I64, I64, P, P]),
 }
 
 _lib = None

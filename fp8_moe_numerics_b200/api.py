@@ -189,10 +189,12 @@ def moe_combine(y: torch.Tensor, pos: torch.Tensor, w, D: int, out=None):
     return out
 
 
-def moe_dispatch_grad(dout: torch.Tensor, src: torch.Tensor, w, k: int, out=None):
+def moe_dispatch_grad(dout: torch.Tensor, src: torch.Tensor, pos: torch.Tensor, w, out=None):
+    """dout bf16 [T, D], src [M_cap], pos [T, k] from moe_route -> dy bf16 [M_cap, D]."""
     M_cap = src.shape[0]
+    T, k = pos.shape
     D = dout.shape[1]
     if out is None:
         out = torch.empty(M_cap, D, dtype=torch.bfloat16, device=dout.device)
-    L.call("moe_dispatch_grad", _p(dout), _p(src), _p(w), k, M_cap, D, _p(out), _s())
+    L.call("moe_dispatch_grad", _p(dout), _p(src), _p(pos), _p(w), T, k, M_cap, D, _p(out), _s())
     return out

@@ -1,6 +1,8 @@
 // abi.cu -- status handling and size helpers of the mxmoe C ABI.
 #include "mx_common.cuh"
 
+#include <atomic>
+
 namespace {
 thread_local int g_last_cuda_error = 0;
 constexpr int kMaxDevices = 64;
@@ -11,6 +13,14 @@ int mx_set_cuda_error(cudaError_t e) {
     g_last_cuda_error = (int)e;
     return MX_ECUDA;
 }
+
+namespace {
+std::atomic<unsigned long long> g_kernel_launches{0};
+}  // namespace
+
+void mx_count_launch(void) { g_kernel_launches.fetch_add(1, std::memory_order_relaxed); }
+
+extern "C" unsigned long long mx_kernel_launches(void) { return g_kernel_launches.load(std::memory_order_relaxed); }
 
 int mx_launch_status(void) {
     cudaError_t e = cudaGetLastError();

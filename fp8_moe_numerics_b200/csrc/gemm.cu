@@ -890,6 +890,7 @@ int launch(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mo, 
     const int64_t n = std::max<int64_t>(1, std::min<int64_t>(items, slots));
     cfg.gridDim = dim3((unsigned)(kPair ? 2 * n : n));
     if (cudaLaunchKernelEx(&cfg, kern, ma, mb, mo, args) != cudaSuccess) return mx_launch_status();
+    mx_count_launch();
     return mx_launch_status();
 }
 

@@ -214,21 +214,44 @@ __global__ void combine_kernel(const uint16_t* __restrict__ y, const int32_t* __
     }
 }
 
-// One block per row of the expert-major buffer.
-__global__ void dispatch_grad_kernel(const uint16_t* __restrict__ dout, const int32_t* __restrict__ src,
-                                     const float* __restrict__ w, int64_t k, int64_t D, uint16_t* __restrict__ dy) {
-    const int64_t p = blockIdx.x;
-    const int32_t s = src[p];
-    const float wj = s < 0 ? 0.0f : (w ? w[s] : 1.0f);
-    const int64_t t = s < 0 ? 0 : s / k;
-    for (int64_t c = threadIdx.x * 8; c < D; c += blockDim.x * 8) {
-        uint4 o = make_uint4(0, 0, 0, 0);
-        if (s >= 0) {
-            const uint4 v = __ldg(reinterpret_cast<const uint4*>(dout + t * D + c));
-            o = make_uint4(pack_bf16x2(wj * bf16_lo(v.x), wj * bf16_hi(v.x)), pack_bf16x2(wj * bf16_lo(v.y), wj * bf16_hi(v.y)),
-                           pack_bf16x2(wj * bf16_lo(v.z), wj * bf16_hi(v.z)), pack_bf16x2(wj * bf16_lo(v.w), wj * bf16_hi(v.w)));
+// Blocks [0, T): token t's row of dout is read once (streaming) and written,
+// scaled by w[t, j], to its k rows pos[t, j].  Blocks from T on: 32 rows of
+// the buffer each, a warp per row, writing zeros to the rows with src < 0
+// (expert padding and the tail past the last segment).
+constexpr int kDispatchThreads = 128;
+
+__global__ void __launch_bounds__(kDispatchThreads)
+dispatch_grad_kernel(const uint16_t* __restrict__ dout, const int32_t* __restrict__ src, const int32_t* __restrict__ pos,
+                     const float* __restrict__ w, int64_t T, int64_t k, int64_t M_cap, int64_t D,
+                     uint16_t* __restrict__ dy) {
+    __shared__ int32_t sp[32];
+    __shared__ float sw[32];
+    const int64_t b = blockIdx.x;
+    if (b < T) {
+        if (threadIdx.x < k) {
+            sp[threadIdx.x] = pos[b * k + threadIdx.x];
+            sw[threadIdx.x] = w ? w[b * k + threadIdx.x] : 1.0f;
         }
-        *reinterpret_cast<uint4*>(dy + p * D + c) = o;
+        __syncthreads();
+        for (int64_t c = threadIdx.x * 8; c < D; c += kDispatchThreads * 8) {
+            const uint4 v = __ldcs(reinterpret_cast<const uint4*>(dout + b * D + c));
+            for (int64_t j = 0; j < k; ++j) {
+                const float wj = sw[j];
+                const uint4 o = make_uint4(pack_bf16x2(wj * bf16_lo(v.x), wj * bf16_hi(v.x)),
+                                           pack_bf16x2(wj * bf16_lo(v.y), wj * bf16_hi(v.y)),
+                                           pack_bf16x2(wj * bf16_lo(v.z), wj * bf16_hi(v.z)),
+                                           pack_bf16x2(wj * bf16_lo(v.w), wj * bf16_hi(v.w)));
+                *reinterpret_cast<uint4*>(dy + (int64_t)sp[j] * D + c) = o;
+            }
+        }
+    } else {
+        const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+        for (int i = 0; i < 8; ++i) {
+            const int64_t p = (b - T) * 32 + warp * 8 + i;
+            if (p >= M_cap || src[p] >= 0) continue;
+            for (int64_t c = lane * 8; c < D; c += 32 * 8)
+                *reinterpret_cast<uint4*>(dy + p * D + c) = make_uint4(0, 0, 0, 0);
+        }
     }
 }
 
@@ -247,11 +270,16 @@ extern "C" int moe_route(const int32_t* topk, int64_t T, int64_t k, int64_t E, i
     int32_t* counts = hist + nchunks * E;
     if (nchunks > 0) {
         route_count_kernel<<<(unsigned)nchunks, kChunk, E * sizeof(int32_t), stream>>>(topk, T, k, E, hist);
+        mx_count_launch();
     }
     route_scan_kernel<<<1, 1024, (E + 1) * sizeof(int64_t), stream>>>(hist, counts, nchunks, E, seg_offsets);
-    if (nchunks > 0)
+    mx_count_launch();
+    if (nchunks > 0) {
         route_scatter_kernel<<<(unsigned)nchunks, 32, 2 * E * sizeof(uint32_t), stream>>>(topk, T, k, E, hist, src, pos);
+        mx_count_launch();
+    }
     route_pad_kernel<<<(unsigned)(E + 1), 256, 0, stream>>>(seg_offsets, counts, E, M_cap, src);
+    mx_count_launch();
     return mx_launch_status();
 }
 
@@ -266,6 +294,7 @@ extern "C" int nvfp4_gather_rows(const uint8_t* codes, const uint8_t* sf, const 
     if (M_cap == 0) return MX_OK;
     gather_rows_kernel<<<(unsigned)((M_cap + 7) / 8), 256, 0, stream>>>(codes, sf, outer, src, k, M_cap, cols,
                                                                        out_codes, out_sf, out_outer);
+    mx_count_launch();
     return mx_launch_status();
 }
 
@@ -277,6 +306,7 @@ extern "C" int swiglu_fwd(const void* h, int64_t rows, int64_t F, int gated, con
     if (n == 0) return MX_OK;
     swiglu_fwd_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(static_cast<const uint16_t*>(h), rows, F,
                                                                         gated, rows_valid, static_cast<uint16_t*>(a));
+    mx_count_launch();
     return mx_launch_status();
 }
 
@@ -291,6 +321,7 @@ extern "C" int swiglu_bwd(const void* h, const void* da, int64_t rows, int64_t F
     swiglu_bwd_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(
         static_cast<const uint16_t*>(h), static_cast<const uint16_t*>(da), rows, F, gated, rows_valid,
         static_cast<uint16_t*>(dh));
+    mx_count_launch();
     return mx_launch_status();
 }
 
@@ -302,18 +333,21 @@ extern "C" int moe_combine(const void* y, const int32_t* pos, const float* w, in
     if (T == 0) return MX_OK;
     combine_kernel<<<(unsigned)T, 128, 0, stream>>>(static_cast<const uint16_t*>(y), pos, w, k, D,
                                                     static_cast<uint16_t*>(out));
+    mx_count_launch();
     return mx_launch_status();
 }
 
-extern "C" int moe_dispatch_grad(const void* dout, const int32_t* src, const float* w, int64_t k, int64_t M_cap,
-                                 int64_t D, void* dy, cudaStream_t stream) {
-    if (!dout || !src || !dy || k <= 0 || M_cap < 0 || D <= 0 || D % 8 || !mx_aligned(dout, 16) ||
-        !mx_aligned(dy, 16))
+extern "C" int moe_dispatch_grad(const void* dout, const int32_t* src, const int32_t* pos, const float* w, int64_t T,
+                                 int64_t k, int64_t M_cap, int64_t D, void* dy, cudaStream_t stream) {
+    if (!dout || !src || !pos || !dy || T < 0 || k <= 0 || k > 32 || M_cap < 0 || D <= 0 || D % 8 ||
+        !mx_aligned(dout, 16) || !mx_aligned(dy, 16))
         return MX_EINVAL;
     if (int st = mx_check_device()) return st;
     if (M_cap == 0) return MX_OK;
-    dispatch_grad_kernel<<<(unsigned)M_cap, 128, 0, stream>>>(static_cast<const uint16_t*>(dout), src, w, k, D,
-                                                              static_cast<uint16_t*>(dy));
+    const int64_t blocks = T + (M_cap + 31) / 32;
+    dispatch_grad_kernel<<<(unsigned)blocks, kDispatchThreads, 0, stream>>>(
+        static_cast<const uint16_t*>(dout), src, pos, w, T, k, M_cap, D, static_cast<uint16_t*>(dy));
+    mx_count_launch();
     return mx_launch_status();
 }
 

@@ -22,6 +22,7 @@
 int mx_set_cuda_error(cudaError_t e);   // records e, returns MX_ECUDA
 int mx_check_device(void);              // MX_OK on sm_100, else MX_EUNSUPPORTED / MX_ECUDA
 int mx_launch_status(void);             // cudaGetLastError -> MX_OK / MX_ECUDA
+void mx_count_launch(void);             // one more kernel launched by this library (mx_kernel_launches)
 
 static inline bool mx_aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 

@@ -54,16 +54,17 @@ __device__ __forceinline__ uint32_t nvfp4_block(const uint4& a, const uint4& b, 
 // group's amax bits (written by nvfp4_group_amax_kernel).
 constexpr int kRowThreads = 256;
 
+// Rows [block * 256/kTPR, +256/kTPR) of x, those below row_end.
 template <int kTPR, int kNB, bool kGroup, int kLayout>
-__global__ void __launch_bounds__(kRowThreads, kNB <= 4 ? 4 : 2)
-nvfp4_quant_rows_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t group_rows,
-                        bool word_sf, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, float* __restrict__ outer) {
+__device__ __forceinline__ void quant_rows_block(const uint16_t* __restrict__ x, int64_t rows, int64_t row_end,
+                                                 int64_t cols, int64_t group_rows, bool word_sf,
+                                                 uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
+                                                 float* __restrict__ outer, int64_t block, uint32_t* wmax) {
     constexpr int kRPB = kRowThreads / kTPR;
-    __shared__ uint32_t wmax[kRowThreads / 32];
     const int lane = threadIdx.x & 31;
     const int j = threadIdx.x % kTPR;
-    const int64_t row = (int64_t)blockIdx.x * kRPB + threadIdx.x / kTPR;
-    const bool active = row < rows;
+    const int64_t row = block * kRPB + threadIdx.x / kTPR;
+    const bool active = row < row_end;
     const int64_t nblk = cols >> 4;
     const uint4* xr = reinterpret_cast<const uint4*>(x + (active ? row : 0) * cols);
 
@@ -137,20 +138,25 @@ nvfp4_quant_rows_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t co
     }
 }
 
+template <int kTPR, int kNB, bool kGroup, int kLayout>
+__global__ void __launch_bounds__(kRowThreads, kNB <= 4 ? 4 : 2)
+nvfp4_quant_rows_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t group_rows,
+                        bool word_sf, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, float* __restrict__ outer) {
+    __shared__ uint32_t wmax[kRowThreads / 32];
+    quant_rows_block<kTPR, kNB, kGroup, kLayout>(x, rows, rows, cols, group_rows, word_sf, codes, sf, outer,
+                                                 (int64_t)blockIdx.x, wmax);
+}
+
 // amax over each group of rows, as fp32 bits, atomically max-ed into outer[g]
 // (pre-zeroed).  blockIdx.y = group, blockIdx.x = chunk of the group's
 // contiguous elements; each thread keeps four 16-byte loads in flight and the
 // block issues one atomic.
 constexpr int kAmaxThreads = 256, kAmaxUnroll = 4;
 
-__global__ void __launch_bounds__(kAmaxThreads)
-nvfp4_group_amax_kernel(const uint16_t* __restrict__ x, int64_t ngroups, int64_t group_vec, int64_t chunk_vec,
-                        float* __restrict__ outer) {
-  __shared__ uint32_t wm[kAmaxThreads / 32];
-  for (int64_t g = blockIdx.y; g < ngroups; g += gridDim.y) {
+// One chunk [v0, v1) of group g's 16-byte vectors (streaming loads).
+__device__ __forceinline__ void group_amax_chunk(const uint16_t* __restrict__ x, int64_t g, int64_t group_vec,
+                                                 int64_t v0, int64_t v1, float* __restrict__ outer, uint32_t* wm) {
     const uint4* xv = reinterpret_cast<const uint4*>(x) + g * group_vec;
-    const int64_t v0 = (int64_t)blockIdx.x * chunk_vec;
-    const int64_t v1 = min(group_vec, v0 + chunk_vec);
     uint32_t m = 0;
     for (int64_t v = v0 + threadIdx.x; v < v1; v += kAmaxThreads * kAmaxUnroll) {
         uint4 q[kAmaxUnroll];
@@ -171,7 +177,16 @@ nvfp4_group_amax_kernel(const uint16_t* __restrict__ x, int64_t ngroups, int64_t
         atomicMax(reinterpret_cast<unsigned int*>(outer) + g, b << 16);
     }
     __syncthreads();
-  }
+}
+
+__global__ void __launch_bounds__(kAmaxThreads)
+nvfp4_group_amax_kernel(const uint16_t* __restrict__ x, int64_t ngroups, int64_t group_vec, int64_t chunk_vec,
+                        float* __restrict__ outer) {
+    __shared__ uint32_t wm[kAmaxThreads / 32];
+    for (int64_t g = blockIdx.y; g < ngroups; g += gridDim.y) {
+        const int64_t v0 = (int64_t)blockIdx.x * chunk_vec;
+        group_amax_chunk(x, g, group_vec, v0, min(group_vec, v0 + chunk_vec), outer, wm);
+    }
 }
 
 __global__ void nvfp4_group_finish_kernel(float* outer, int64_t ngroups) {
@@ -267,82 +282,98 @@ __device__ __forceinline__ void tile_emit_transposed(const float* T, int64_t row
 }
 
 // MXFP8 quantisation of bf16 [rows, cols]: row-wise blocks (phase 1, straight
-// from registers) and/or the transposed column-wise form (phase 2).
+// from registers) and/or the transposed column-wise form (phase 2).  Blocks
+// loop over 128x64 tiles (column tiles fastest) and load the next tile's
+// values into registers before the current tile's transposed phase.
 template <bool kRow, bool kCol, bool kSR, int kR, int kLayout>
-__global__ void __launch_bounds__(kTileThreads)
+__global__ void __launch_bounds__(kTileThreads, 4)
 mxfp8_tile_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, const int64_t* rows_valid,
                   uint64_t seed, uint64_t stream_row, uint64_t stream_col,
                   uint8_t* __restrict__ row_codes, uint8_t* __restrict__ row_e8m0,
                   uint8_t* __restrict__ col_codes, uint8_t* __restrict__ col_e8m0) {
     __shared__ __align__(16) float T[kCol ? kTC * kTR : 4];
-    const int64_t c0 = (int64_t)blockIdx.x * kTC, r0 = (int64_t)blockIdx.y * kTR;
-    if (r0 >= load_rows_valid(rows_valid, rows)) return;
+    const int64_t tiles_c = cols / kTC;
+    const int64_t ntiles = tiles_c * ((load_rows_valid(rows_valid, rows) + kTR - 1) / kTR);
+    int64_t tile = blockIdx.x;
+    if (tile >= ntiles) return;
     const int t = threadIdx.x;
     const int rl = t >> 1, h = t & 1;
-    const int64_t r = r0 + rl;
-    const uint4* src = reinterpret_cast<const uint4*>(x + r * cols + c0 + 32 * h);
     uint4 q[4];
+    auto fetch = [&](int64_t tl) {
+        const int64_t c0 = (tl % tiles_c) * kTC, r = (tl / tiles_c) * kTR + rl;
+        const uint4* src = reinterpret_cast<const uint4*>(x + r * cols + c0 + 32 * h);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) q[i] = __ldcs(src + i);
-    float v[32];
+        for (int i = 0; i < 4; ++i) q[i] = __ldcs(src + i);
+    };
+    fetch(tile);
+    for (; tile < ntiles; tile += gridDim.x) {
+        const int64_t c0 = (tile % tiles_c) * kTC, r0 = (tile / tiles_c) * kTR;
+        const int64_t r = r0 + rl;
+        float v[32];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const uint32_t w[4] = {q[i].x, q[i].y, q[i].z, q[i].w};
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t w[4] = {q[i].x, q[i].y, q[i].z, q[i].w};
 #pragma unroll
-        for (int j = 0; j < 4; ++j) { v[8 * i + 2 * j] = bf16_lo(w[j]); v[8 * i + 2 * j + 1] = bf16_hi(w[j]); }
-    }
-    if (kRow) {
-        uint32_t m = 0;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) m = max(m, absmax8_bf16(q[i]));
-        const int e = e8m0_exponent(__uint_as_float(m << 16));
-        uint32_t w[8];
-        const int64_t L0 = r * cols + c0 + 32 * h;
-        if (kSR && kR == 16) {
-            const float sc = exp2_neg(e);
-#pragma unroll
-            for (int blk = 0; blk < 4; ++blk) {
-                const uint4 rnd = philox4x32_10((uint64_t)(L0 / 8) + blk, stream_row, seed);
-                const uint32_t wd[4] = {rnd.x, rnd.y, rnd.z, rnd.w};
-#pragma unroll
-                for (int q = 0; q < 4; q += 2) {
-                    const int i = blk * 8 + 2 * q;
-                    w[blk * 2 + (q >> 1)] = cvt_rs16_e4m3_quad(__fmul_rn(v[i], sc), __fmul_rn(v[i + 1], sc),
-                                                               __fmul_rn(v[i + 2], sc), __fmul_rn(v[i + 3], sc),
-                                                               wd[q], wd[q + 1]);
-                }
-            }
-        } else if (kSR) {
-            constexpr int kPer = 128 / kR;
-#pragma unroll
-            for (int blk = 0; blk < 32 / kPer; ++blk) {
-                const uint4 rnd = philox4x32_10((uint64_t)(L0 / kPer) + blk, stream_row, seed);
-#pragma unroll
-                for (int jj = 0; jj < kPer; ++jj) {
-                    const int i = blk * kPer + jj;
-                    const uint32_t code = e4m3_sr_code<kR>(v[i], e, philox_field<kR>(rnd, jj));
-                    if ((i & 3) == 0) w[i >> 2] = code; else w[i >> 2] |= code << (8 * (i & 3));
-                }
-            }
-        } else {
-            const float sc = exp2_neg(e);
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-                w[i] = cvt_e4m3x2(__fmul_rn(v[4 * i], sc), __fmul_rn(v[4 * i + 1], sc)) |
-                       (cvt_e4m3x2(__fmul_rn(v[4 * i + 2], sc), __fmul_rn(v[4 * i + 3], sc)) << 16);
+            for (int j = 0; j < 4; ++j) { v[8 * i + 2 * j] = bf16_lo(w[j]); v[8 * i + 2 * j + 1] = bf16_hi(w[j]); }
         }
-        uint4* dst = reinterpret_cast<uint4*>(row_codes + L0);
-        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-        row_e8m0[sf_offset(r, (c0 >> 5) + h, cols >> 5, kLayout)] = (uint8_t)(e + 127);
-    }
-    if (kCol) {
+        if (kRow) {
+            uint32_t m = 0;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) T[tsw(32 * h + i, rl)] = v[i];
-        __syncthreads();
-        tile_emit_transposed<kSR, kR, kLayout>(T, rows, cols, r0, c0, seed, stream_col, col_codes, col_e8m0);
+            for (int i = 0; i < 4; ++i) m = max(m, absmax8_bf16(q[i]));
+            const int e = e8m0_exponent(__uint_as_float(m << 16));
+            uint32_t w[8];
+            const int64_t L0 = r * cols + c0 + 32 * h;
+            if (kSR && kR == 16) {
+                const float sc = exp2_neg(e);
+#pragma unroll
+                for (int blk = 0; blk < 4; ++blk) {
+                    const uint4 rnd = philox4x32_10((uint64_t)(L0 / 8) + blk, stream_row, seed);
+                    const uint32_t wd[4] = {rnd.x, rnd.y, rnd.z, rnd.w};
+#pragma unroll
+                    for (int q = 0; q < 4; q += 2) {
+                        const int i = blk * 8 + 2 * q;
+                        w[blk * 2 + (q >> 1)] = cvt_rs16_e4m3_quad(__fmul_rn(v[i], sc), __fmul_rn(v[i + 1], sc),
+                                                                   __fmul_rn(v[i + 2], sc), __fmul_rn(v[i + 3], sc),
+                                                                   wd[q], wd[q + 1]);
+                    }
+                }
+            } else if (kSR) {
+                constexpr int kPer = 128 / kR;
+#pragma unroll
+                for (int blk = 0; blk < 32 / kPer; ++blk) {
+                    const uint4 rnd = philox4x32_10((uint64_t)(L0 / kPer) + blk, stream_row, seed);
+#pragma unroll
+                    for (int jj = 0; jj < kPer; ++jj) {
+                        const int i = blk * kPer + jj;
+                        const uint32_t code = e4m3_sr_code<kR>(v[i], e, philox_field<kR>(rnd, jj));
+                        if ((i & 3) == 0) w[i >> 2] = code; else w[i >> 2] |= code << (8 * (i & 3));
+                    }
+                }
+            } else {
+                const float sc = exp2_neg(e);
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    w[i] = cvt_e4m3x2(__fmul_rn(v[4 * i], sc), __fmul_rn(v[4 * i + 1], sc)) |
+                           (cvt_e4m3x2(__fmul_rn(v[4 * i + 2], sc), __fmul_rn(v[4 * i + 3], sc)) << 16);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(row_codes + L0);
+            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+            dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+            row_e8m0[sf_offset(r, (c0 >> 5) + h, cols >> 5, kLayout)] = (uint8_t)(e + 127);
+        }
+        if (kCol) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) T[tsw(32 * h + i, rl)] = v[i];
+            __syncthreads();
+            if (tile + gridDim.x < ntiles) fetch(tile + gridDim.x);
+            tile_emit_transposed<kSR, kR, kLayout>(T, rows, cols, r0, c0, seed, stream_col, col_codes, col_e8m0);
+            __syncthreads();                               // T is rewritten by the next tile
+        } else if (tile + gridDim.x < ntiles) {
+            fetch(tile + gridDim.x);
+        }
     }
 }
+
 
 // NVFP4 [rows, cols] -> dequantise -> transpose -> MXFP8 with SR.
 template <int kR, int kInLayout, int kOutLayout>
@@ -411,6 +442,7 @@ extern "C" int nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t
                 const int64_t rpb = kRowThreads / tpr;
                 kern<<<(unsigned)((rows + rpb - 1) / rpb), kRowThreads, 0, stream>>>(xb, rows, cols, group_rows, word_sf,
                                                                                        codes, sf, outer);
+                mx_count_launch();
             };
             // four 16-element blocks (128 bytes) per thread in flight, 4 CTAs per SM:
             // 128 KB of loads outstanding per SM covers HBM latency under load
@@ -429,8 +461,10 @@ extern "C" int nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t
             const int64_t chunk_vec = 16384;                            // 256 KiB per block
             const dim3 ag((unsigned)((group_vec + chunk_vec - 1) / chunk_vec), (unsigned)std::min<int64_t>(ngroups, 65535));
             nvfp4_group_amax_kernel<<<ag, kAmaxThreads, 0, stream>>>(xb, ngroups, group_vec, chunk_vec, outer);
+            mx_count_launch();
             run(std::true_type());
             nvfp4_group_finish_kernel<<<(unsigned)((ngroups + 255) / 256), 256, 0, stream>>>(outer, ngroups);
+            mx_count_launch();
         }
         return mx_launch_status();
     });
@@ -450,7 +484,9 @@ extern "C" int mxfp8_quantize(const void* x, int64_t rows, int64_t cols, int rou
     if (sf_layout != MX_SF_ROWMAJOR && sf_layout != MX_SF_MMA) return MX_EINVAL;
     if (int st = mx_check_device()) return st;
     if (rows == 0) return MX_OK;
-    const dim3 grid((unsigned)(cols / kTC), (unsigned)(rows / kTR));
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const dim3 grid((unsigned)std::min<int64_t>((cols / kTC) * (rows / kTR), (int64_t)sms * 4));
     const uint64_t s_row = stream_id, s_col = do_row ? stream_id + 1 : stream_id;
     const uint16_t* xb = static_cast<const uint16_t*>(x);
     return dispatch_layout(sf_layout, [&](auto L) {
@@ -469,6 +505,7 @@ extern "C" int mxfp8_quantize(const void* x, int64_t rows, int64_t cols, int rou
             else
                 mxfp8_tile_kernel<kRow, kCol, true, 32, kL><<<grid, kTileThreads, 0, stream>>>(
                     xb, rows, cols, rows_valid, seed, s_row, s_col, row_codes, row_e8m0, col_codes, col_e8m0);
+            mx_count_launch();
         };
         if (do_row && do_col) launch(std::true_type(), std::true_type());
         else if (do_row) launch(std::true_type(), std::false_type());
@@ -493,6 +530,9 @@ extern "C" int mxfp8_requant_transpose_sr(const uint8_t* codes, const uint8_t* s
     if (rows >= ((int64_t)1 << 31)) return MX_EINVAL;
     if (int st = mx_check_device()) return st;
     if (rows == 0) return MX_OK;
+    // one 128x64 tile per block: short independent blocks drift apart, so one
+    // block's loads overlap another's rounding arithmetic (measured faster on
+    // B200 than persistent blocks, which move through the phases in step)
     const dim3 grid((unsigned)(cols / kTC), (unsigned)(rows / kTR));
     return dispatch_layout(in_sf_layout, [&](auto Li) {
         return dispatch_layout(out_sf_layout, [&](auto Lo) {
@@ -506,6 +546,7 @@ extern "C" int mxfp8_requant_transpose_sr(const uint8_t* codes, const uint8_t* s
             else
                 requant_tile_kernel<32, kLi, kLo><<<grid, kTileThreads, 0, stream>>>(
                     codes, sf, outer, rows, cols, group_rows, rows_valid, seed, stream_id, out_codes, out_e8m0);
+            mx_count_launch();
             return mx_launch_status();
         });
     });

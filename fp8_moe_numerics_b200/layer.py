@@ -126,7 +126,7 @@ class ExpertLayer:
         T, D, k, E, F, N1, M = self.T, self.D, self.k, self.E, self.F, self.N1, self.M_cap
         s, R = self.seed, self.rbits
         self._mark("bwd_start", record)
-        api.moe_dispatch_grad(self.dout, self.src, self.w_comb, k, out=self.dy2)
+        api.moe_dispatch_grad(self.dout, self.src, self.pos, self.w_comb, out=self.dy2)
         self._mark("dispatch_grad", record)
         api.mxfp8_quantize(self.dy2, rows_valid=self.rows_valid, rounding=MX_ROUND_RNE, out=self.dy2q)
         self._mark("quant_dy2", record)

@@ -70,6 +70,10 @@ MX_API int mx_version(void);
 /* cudaError_t of the last MX_ECUDA returned on this host thread. */
 MX_API int mx_last_cuda_error(void);
 
+/* Kernels this library has launched in this process so far (all threads,
+ * all devices), for accounting by callers; the pages have no counterpart. */
+MX_API unsigned long long mx_kernel_launches(void);
+
 /* Synchronises `stream`, then returns and clears the device status word of
  * the current device: MX_ETIMEOUT if a bounded wait inside a GEMM kernel
  * expired since the last call (that kernel's output is then undefined),
@@ -253,9 +257,13 @@ MX_API int moe_combine(const void* y, const int32_t* pos, const float* w, int64_
 
 /* moe_dispatch_grad -- gradient of moe_combine w.r.t. y:
  * dy[p] = w[src[p]] * dout[src[p]/k] (bf16), zero rows where src[p] < 0.
- * Writes all M_cap rows. */
-MX_API int moe_dispatch_grad(const void* dout, const int32_t* src, const float* w, int64_t k,
-                      int64_t M_cap, int64_t D, void* dy, cudaStream_t stream);
+ * dout bf16 [T, D]; src int32 [M_cap] and pos int32 [T, k] as written by
+ * moe_route (pos[t*k + j] is the row of token t's j-th copy, so
+ * src[pos[i]] == i); w fp32 [T, k] or NULL (all ones); dy bf16 [M_cap, D].
+ * Writes all M_cap rows, reading each token's row of dout once.  dout and dy
+ * 16-byte aligned, D a multiple of 8; else MX_EINVAL. */
+MX_API int moe_dispatch_grad(const void* dout, const int32_t* src, const int32_t* pos, const float* w, int64_t T,
+                             int64_t k, int64_t M_cap, int64_t D, void* dy, cudaStream_t stream);
 
 #ifdef __cplusplus
 }

@@ -12,7 +12,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 def _declared():
     src = open(os.path.join(ROOT, "include", "mxmoe.h")).read()
-    return re.findall(r"^MX_API\s+(?:int|size_t)\s+([a-z0-9_]+)\(", src, flags=re.M)
+    return re.findall(r"^MX_API\s+(?:int|size_t|unsigned long long)\s+([a-z0-9_]+)\(", src, flags=re.M)
 
 
 @pytest.fixture(scope="module")
@@ -29,6 +29,14 @@ def test_every_declared_symbol_is_exported(mx):
         assert hasattr(mx, n), n
     from fp8_moe_numerics_b200._lib import SIGNATURES
     assert set(SIGNATURES) == set(names)
+
+
+def test_launch_counter_ignores_rejected_calls(mx):
+    before = mx.mx_kernel_launches()
+    assert isinstance(before, int) and before >= 0
+    # rejected on the host: no kernel is launched
+    assert mx.nvfp4_quantize(None, 16, 64, 1, None, None, None, 1, None) == 1
+    assert mx.mx_kernel_launches() == before
 
 
 def test_sizes_and_version(mx):

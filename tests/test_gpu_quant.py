@@ -100,6 +100,19 @@ def test_nvfp4_quantize_per_expert_bit_exact(cuda, E, N, K):
     assert np.array_equal(np_(go).view(np.uint32), outer.view(np.uint32))
 
 
+def test_nvfp4_quantize_per_expert_unaligned_groups(cuda):
+    # 3 experts of 2046 x 4096 (16.8 MB each): expert boundaries fall inside a
+    # block of rows of the quantiser, with row-major scales
+    E, N, K = 3, 2046, 4096
+    w = workloads.weights(E, N, K, 0.02, seed=77)
+    wn = w.reshape(E * N, K).view(torch.int16).numpy().view(np.uint16)
+    codes, sf, outer = oracle.nvfp4_quantize(wn, group_rows=N)
+    gc, gsf, go = api.nvfp4_quantize(w.reshape(E * N, K).cuda(), group_rows=N, sf_layout=api.MX_SF_ROWMAJOR)
+    assert np.array_equal(np_(gc), codes)
+    assert np.array_equal(np_(gsf).reshape(sf.shape), sf)
+    assert np.array_equal(np_(go).view(np.uint32), outer.view(np.uint32))
+
+
 # ---------------------------------------------------------------------------
 # MXFP8 quantiser
 # ---------------------------------------------------------------------------
@@ -276,9 +289,12 @@ def test_combine_and_dispatch_grad(cuda):
     got = to_np_u16(api.moe_combine(to_dev_bf16(y), torch.from_numpy(pos).cuda(), torch.from_numpy(w).cuda(), D))
     assert _ulp_close(got, ref)
     dout = oracle.f32_to_bf16(rng.standard_normal((T, D)).astype(np.float32))
-    ref_dy = oracle.dispatch_grad(dout, pos, w, M)
     M_cap = api.max_routed_rows(T, k, E)
-    _, gsrc, _ = api.moe_route(ids.cuda(), E, M_cap)
-    gdy = to_np_u16(api.moe_dispatch_grad(to_dev_bf16(dout), gsrc, torch.from_numpy(w).cuda(), k))
-    assert np.array_equal(gdy[:M], ref_dy)
-    assert np.all(gdy[M:] == 0)
+    _, gsrc, gpos = api.moe_route(ids.cuda(), E, M_cap)
+    # non-uniform weights and the all-ones (NULL) form; padding rows and the tail are zero
+    wr = rng.uniform(0.1, 1.0, (T, k)).astype(np.float32)
+    for wv, wd in ((wr, torch.from_numpy(wr).cuda()), (np.ones((T, k), np.float32), None)):
+        ref_dy = oracle.dispatch_grad(dout, pos, wv, M)
+        gdy = to_np_u16(api.moe_dispatch_grad(to_dev_bf16(dout), gsrc, gpos, wd))
+        assert np.array_equal(gdy[:M], ref_dy)
+        assert np.all(gdy[M:] == 0)
