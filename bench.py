@@ -43,6 +43,13 @@ UNIT = "TFLOP/s"
 NOMINAL_NVFP4_TFLOPS = 9000.0
 NOMINAL_MXFP8_TFLOPS = 4500.0
 NOMINAL_HBM_GBS = 8000.0
+SM_MAX_MHZ = 1965.0                   # clocks.max.sm of this machine's B200s
+# stages that issue more than one kernel (routing: 4; per-expert NVFP4 weights: amax, quantise, finish)
+MULTI_LAUNCH_STAGES = ("route", "quant_w")
+# mxfp8_requant_transpose_sr (R = 16) per element, from one ncu capture of `bench.py --kernel requant_w`
+# (64 experts x 2048 x 4096, output 0.55 GB > L2): warp-instructions executed and DRAM bytes (read + write)
+REQUANT_WARP_INST_PER_ELEM = 0.8232
+REQUANT_DRAM_BYTES_PER_ELEM = 1.6217
 
 
 def load_peaks():
@@ -180,15 +187,15 @@ def stage_work(c, counts, M_pad):
         "combine": ("hbm", R * D * 2 + T * D * 2),
         "dispatch_grad": ("hbm", T * D * 2 + R * D * 2),
         "quant_dy2": ("hbm", R * D * 2 + 2 * mx(R, D)),
-        "requant_w2": ("hbm", nv(E * D, F) + mx(E * D, F)),
+        "requant_w2": ("alu", (nv(E * D, F) + mx(E * D, F), (E * D) * (F))),
         "dgrad2": ("tensor8", 2 * R * F * D),
-        "requant_a": ("hbm", nv(R, F) + mx(R, F)),
+        "requant_a": ("alu", (nv(R, F) + mx(R, F), (R) * (F))),
         "wgrad2": ("tensor8", 2 * R * D * F),
         "swiglu_bwd": ("hbm", R * N1 * 2 + R * F * 2 + R * N1 * 2),
         "quant_dh1": ("hbm", R * N1 * 2 + 2 * mx(R, N1)),
-        "requant_w1": ("hbm", nv(E * N1, D) + mx(E * N1, D)),
+        "requant_w1": ("alu", (nv(E * N1, D) + mx(E * N1, D), (E * N1) * (D))),
         "dgrad1": ("tensor8", 2 * R * D * N1),
-        "requant_x": ("hbm", nv(R, D) + mx(R, D)),
+        "requant_x": ("alu", (nv(R, D) + mx(R, D), (R) * (D))),
         "wgrad1": ("tensor8", 2 * R * N1 * D),
         "unpermute": ("hbm", R * D * 2 + T * D * 2),
     }
@@ -249,11 +256,23 @@ def run_ours(args):
     nvfp4_ms = stage_ms["gemm1"] + stage_ms["gemm2"]
     value = world * gemm_flops / (nvfp4_ms * 1e-3) / 1e12
 
-    # roofline of the dominant kernel
-    dom = max(names, key=lambda n: stage_ms[n])
+    # roofline of the dominant kernel: the longest stage that is one launch
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    issue_peak = sms * 4 * SM_MAX_MHZ * 1e6 / 1e9           # warp-instructions per ns = G/s
+    dom = max((n for n in names if n not in MULTI_LAUNCH_STAGES), key=lambda n: stage_ms[n])
     kind, wk = work[dom]
     per_launch_ms = stage_ms[dom] / K
-    if kind == "hbm":
+    if kind == "alu":
+        nbytes, elems = wk
+        achieved = REQUANT_WARP_INST_PER_ELEM * elems / (per_launch_ms * 1e-3) / 1e9
+        roof = {"bound": "alu", "achieved": round(achieved, 1), "peak": round(issue_peak, 1), "unit": "Ginst/s",
+                "frac": round(achieved / issue_peak, 4),
+                "traffic": round(REQUANT_DRAM_BYTES_PER_ELEM * elems) if REQUANT_DRAM_BYTES_PER_ELEM else None,
+                "kernel": dom,
+                "peak_source": f"{sms} SMs x 4 warp schedulers x {SM_MAX_MHZ} MHz (one warp-instruction each per "
+                               "clock); instructions per element from ncu smsp__inst_executed",
+                "hbm_frac": round(nbytes / (per_launch_ms * 1e-3) / 1e9 / peaks["hbm"], 4)}
+    elif kind == "hbm":
         achieved = wk / (per_launch_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm"], "unit": "GB/s",
                 "frac": round(achieved / peaks["hbm"], 4), "traffic": None, "kernel": dom,
@@ -269,7 +288,13 @@ def run_ours(args):
     for n in names:
         kind, wk = work[n]
         t = stage_ms[n] / K
-        if kind == "hbm":
+        if kind == "alu":
+            nbytes, elems = wk
+            breakdown[n] = {"ms": round(t, 4), "GB/s": round(nbytes / (t * 1e-3) / 1e9, 1) if t > 0 else None,
+                            "frac_hbm": round(nbytes / (t * 1e-3) / 1e9 / peaks["hbm"], 3) if t > 0 else None,
+                            "frac_issue": round(REQUANT_WARP_INST_PER_ELEM * elems / (t * 1e-3) / 1e9 / issue_peak, 3)
+                            if t > 0 else None}
+        elif kind == "hbm":
             breakdown[n] = {"ms": round(t, 4), "GB/s": round(wk / (t * 1e-3) / 1e9, 1) if t > 0 else None,
                             "frac_hbm": round(wk / (t * 1e-3) / 1e9 / peaks["hbm"], 3) if t > 0 else None}
         else:
@@ -419,6 +444,71 @@ def cpu_baseline(inp, layer, seconds: float = 15.0):
             "seconds": round(dt, 2)}
 
 
+# --------------------------------------------------------------------------
+# single-kernel cases for ncu captures (small enough to profile, outputs
+# larger than L2 where DRAM traffic is read off)
+# --------------------------------------------------------------------------
+KERNEL_CASES = ("gemm_nvfp4", "gemm_mxfp8_dgrad", "gemm_mxfp8_wgrad", "requant", "requant_w", "nvfp4_quantize",
+                "mxfp8_quantize")
+
+
+def run_kernel(args):
+    import torch
+    from fp8_moe_numerics_b200 import api, workloads
+    dev = torch.device("cuda")
+    which = args.kernel
+    if which.startswith("gemm"):
+        # 64 experts, top-8 of 4096 tokens (Zipf 1.2), d_model 4096, d_ff 1024 (gated)
+        E, T, k, D, F = 64, 4096, 8, 4096, 1024
+        ids = workloads.routing(T, k, E, "zipf", 1.2, 0, 7).to(dev)
+        seg, src, pos = api.moe_route(ids, E)
+        M = src.shape[0]
+        x = workloads.activations(T, D, "t3", 1, dev)
+        xq = api.nvfp4_quantize(x, 1, api.MX_SF_ROWMAJOR)
+        xp = api.nvfp4_gather_rows(*xq, src, k, D)
+        w1 = workloads.weights(E, 2 * F, D, 0.02, 2, dev).view(E * 2 * F, D)
+        w1q = api.nvfp4_quantize(w1, 2 * F, api.MX_SF_MMA)
+        if which == "gemm_nvfp4":
+            run = lambda: api.grouped_gemm_nvfp4(xp, w1q, seg, E, 2 * F, D)
+        else:
+            dh = workloads.gradient(M, 2 * F, 1e-3, 3, dev)
+            q = api.mxfp8_quantize(dh)
+            if which == "gemm_mxfp8_dgrad":
+                w1t = api.mxfp8_requant_transpose_sr(*w1q, E * 2 * F, D, 2 * F, seed=1, stream_id=1)
+                run = lambda: api.grouped_gemm_mxfp8(api.MX_GEMM_DGRAD, q[0], q[1], *w1t, seg, E, M, D, 2 * F)
+            else:
+                xt = api.mxfp8_requant_transpose_sr(*xp, M, D, 1, rows_valid=seg[E:E + 1], seed=1, stream_id=2)
+                run = lambda: api.grouped_gemm_mxfp8(api.MX_GEMM_WGRAD, q[2], q[3], *xt, seg, E, M, 2 * F, D)
+    elif which in ("requant", "nvfp4_quantize"):
+        c = workloads.CONFIGS[QUANT_WORKLOAD]
+        x = workloads.activations(c["rows"], c["cols"], c["x_dist"], c["seed"], dev)
+        q = api.nvfp4_quantize(x)
+        if which == "requant":
+            run = lambda: api.mxfp8_requant_transpose_sr(*q, c["rows"], c["cols"], seed=c["sr_seed"])
+        else:
+            run = lambda: api.nvfp4_quantize(x, out=q)
+    elif which == "requant_w":
+        # 64 experts of 2048 x 4096 weights, per-expert outer scales (output 0.55 GB > L2)
+        E, N, K = 64, 2048, 4096
+        w = workloads.weights(E, N, K, 0.02, 2, dev).view(E * N, K)
+        q = api.nvfp4_quantize(w, N)
+        run = lambda: api.mxfp8_requant_transpose_sr(*q, E * N, K, N, seed=1, stream_id=3)
+    else:                                               # mxfp8_quantize, row + column forms, RNE
+        x = workloads.gradient(65536, 4096, 1.0, 5, dev)
+        run = lambda: api.mxfp8_quantize(x)
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize()
+    api.sync_status()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    run()
+    e1.record()
+    torch.cuda.synchronize()
+    api.sync_status()
+    print(json.dumps({"kernel": which, "ms": round(e0.elapsed_time(e1), 4)}), flush=True)
+
+
 def run_reference(args):
     """Reference arm: the CPU oracle timed on the host cores (rank 0 only)."""
     rank = int(os.environ.get("RANK", "0"))
@@ -467,8 +557,12 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel", choices=KERNEL_CASES, default=None,
+                    help="run one kernel on a small case (warm-up, then one launch) for profiling")
     args = ap.parse_args()
-    if args.impl == "reference":
+    if args.kernel:
+        run_kernel(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)
