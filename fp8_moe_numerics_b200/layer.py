@@ -96,6 +96,21 @@ class ExpertLayer:
     def reset_marks(self):
         self.marks = []
 
+    # ------------------------------------------------------------------ I/O
+    IO = ("x", "topk", "w_comb", "dout", "out", "dx")
+
+    def io(self) -> dict:
+        """The per-step inputs (x, topk, w_comb, dout) and outputs (out, dx)."""
+        return {n: getattr(self, n) for n in self.IO}
+
+    def bind_io(self, bufs: dict) -> None:
+        """Point the next steps at other device tensors of the same shapes for
+        the per-step inputs and outputs (weights and intermediates stay)."""
+        for n in self.IO:
+            t = bufs[n]
+            assert t.shape == getattr(self, n).shape and t.dtype == getattr(self, n).dtype, n
+            setattr(self, n, t)
+
     # ----------------------------------------------------------------- forward
     def forward(self, record: bool = False):
         T, D, k, E, F, N1, M = self.T, self.D, self.k, self.E, self.F, self.N1, self.M_cap
@@ -170,3 +185,51 @@ class ExpertLayer:
                 continue
             out[name] = out.get(name, 0.0) + a.elapsed_time(b)
         return out
+
+
+def host_stream_steps(layer: ExpertLayer, host_in: dict, host_out: dict, steps: int) -> None:
+    """Run `steps` layer steps whose inputs come from pinned host memory and
+    whose outputs go back to it, every step copying its own inputs and results.
+
+    host_in holds pinned x, topk, w_comb, dout; host_out pinned out, dx.  Two
+    device buffer sets alternate between steps; a host-to-device stream fills
+    step i+1's inputs and a device-to-host stream drains step i-1's outputs
+    while step i's kernels run on the current stream (the copy engines work
+    beside the SMs).  Everything is enqueued; the caller synchronises.
+    """
+    cs = torch.cuda.current_stream()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    up.wait_stream(cs)                                     # earlier work on the buffers comes first
+    own = layer.io()
+    sets = [own, {n: torch.empty_like(t) for n, t in own.items()}]
+    for t in list(own.values()) + list(sets[1].values()):
+        t.record_stream(up)                                # used beside the allocating stream
+        t.record_stream(down)
+    in_ready = [torch.cuda.Event() for _ in range(2)]
+    in_free = [torch.cuda.Event() for _ in range(2)]
+    out_ready = [torch.cuda.Event() for _ in range(2)]
+    out_free = [torch.cuda.Event() for _ in range(2)]
+    for i in range(steps):
+        b = i % 2
+        buf = sets[b]
+        with torch.cuda.stream(up):
+            if i >= 2:
+                up.wait_event(in_free[b])                  # step i-2 has read this set
+            for n in ("x", "topk", "w_comb", "dout"):
+                buf[n].copy_(host_in[n], non_blocking=True)
+            in_ready[b].record(up)
+        cs.wait_event(in_ready[b])
+        if i >= 2:
+            cs.wait_event(out_free[b])                     # step i-2's results are on the host
+        layer.bind_io(buf)
+        layer.step()
+        in_free[b].record(cs)
+        out_ready[b].record(cs)
+        with torch.cuda.stream(down):
+            down.wait_event(out_ready[b])
+            for n in ("out", "dx"):
+                host_out[n].copy_(buf[n], non_blocking=True)
+            out_free[b].record(down)
+    cs.wait_stream(down)
+    layer.bind_io(own)
+

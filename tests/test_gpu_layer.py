@@ -107,3 +107,22 @@ def test_tiny_layer_forward_backward_against_oracle(cuda):
     for got, ref in ((f64(u16(L.out)), f64(out)), (f64(u16(L.da)[:Mp]), f64(da)), (g(L.dw2).astype(np.float64), dw2),
                      (f64(u16(L.dxp)[:Mp]), f64(dxp)), (g(L.dw1).astype(np.float64), dw1), (f64(u16(L.dx)), f64(dx))):
         assert rel(got, ref) < 2e-2
+
+
+def test_host_stream_steps_matches_plain_step(cuda):
+    # three steps with inputs from pinned host memory and outputs read back,
+    # neighbouring steps' copies overlapping: the same bytes as one plain step
+    from fp8_moe_numerics_b200.layer import host_stream_steps
+    inp = workloads.layer_inputs("tiny_layer", device="cpu")
+    L = ExpertLayer(inp["x"].cuda(), inp["topk"].cuda(), inp["w_comb"].cuda(), inp["w1"].cuda(), inp["w2"].cuda(),
+                    inp["dout"].cuda(), gated=False, seed=5)
+    own = {n: t.data_ptr() for n, t in L.io().items()}
+    L.step()
+    ref_out, ref_dx = L.out.cpu(), L.dx.cpu()
+    host_in = {n: inp[n].pin_memory() for n in ("x", "topk", "w_comb", "dout")}
+    host_out = {n: torch.zeros_like(getattr(L, n), device="cpu").pin_memory() for n in ("out", "dx")}
+    host_stream_steps(L, host_in, host_out, 3)
+    torch.cuda.synchronize()
+    api.sync_status()
+    assert torch.equal(host_out["out"], ref_out) and torch.equal(host_out["dx"], ref_dx)
+    assert {n: t.data_ptr() for n, t in L.io().items()} == own
