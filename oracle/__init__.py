@@ -255,6 +255,21 @@ def mxfp8_requant_transpose_sr(codes, sf, outer, group_rows: int, seed: int, str
     return oc, oe
 
 
+def mxfp8_requant_entry(codes32, sf32, outer32, col: int, t: int, rows: int, row0: int, seed: int, stream: int,
+                        R: int):
+    """One entry of mxfp8_requant_transpose_sr, computed alone: output [col, row0 + t]
+    of a call on a tensor with `rows` rows, from the 32 input rows row0..row0+31
+    (codes32 [32, cols/2], row-major sf32 [32, cols/16], per-row outer32 [32]).
+    Returns (E4M3 code, E8M0 byte) following the same steps as the full call:
+    dequantise, block amax, E8M0 exponent, exact scaling, SR with the bits of
+    linear index col * rows + row0 + t."""
+    xh = nvfp4_dequantize(codes32, sf32, outer32, 1)[:, col].astype(np.float64)
+    e = e8m0_exponent(float(np.max(np.abs(xh))))
+    y = float(np.ldexp(xh[t], -e))
+    L = col * rows + row0 + t
+    return e4m3_sr(y, sr_bits(seed, stream, R, L), R), e + 127
+
+
 def mxfp8_quantize_rows(x_bf16, sr: bool = False, seed: int = 0, stream: int = 0, R: int = 8):
     x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
     rows, cols = x.shape

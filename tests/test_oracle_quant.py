@@ -251,3 +251,21 @@ def test_requant_per_expert_outer_for_weights(orc):
     # |back - xh| is below one quantum of the element's block
     q = 2.0 ** (oe.astype(np.int64) - 127 + 5).repeat(32, axis=1)
     assert np.all(np.abs(back - xh.T) <= q)
+
+
+def test_requant_entry_matches_the_full_call(orc):
+    # the single-entry form used for sampled checks at full size equals the
+    # full requantisation, per-token and per-expert outer scales, R = 8 and 16
+    for group_rows, R in ((1, 16), (128, 8)):
+        rows, cols = 256, 96
+        x = _rand_rows(orc, rows, cols, seed=11 + R)
+        codes, sf, outer = orc.nvfp4_quantize(x, group_rows=group_rows)
+        full_c, full_e = orc.mxfp8_requant_transpose_sr(codes, sf, outer, group_rows, seed=5, stream=9, R=R)
+        per_row = np.repeat(outer, group_rows).astype(np.float32)
+        rng = np.random.default_rng(R)
+        for _ in range(200):
+            col, r = int(rng.integers(cols)), int(rng.integers(rows))
+            row0, t = r - r % 32, r % 32
+            code, e8 = orc.mxfp8_requant_entry(codes[row0:row0 + 32], sf[row0:row0 + 32], per_row[row0:row0 + 32],
+                                               col, t, rows, row0, 5, 9, R)
+            assert code == full_c[col, r] and e8 == full_e[col, r // 32]
