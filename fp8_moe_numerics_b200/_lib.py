@@ -31,6 +31,7 @@ SIGNATURES = {
     "mx_last_cuda_error": (I32, []),
     "mx_kernel_launches": (ctypes.c_ulonglong, []),
     "mx_sync_status": (I32, [P]),
+    "mx_wait_selftest": (I32, [I64, P]),
     "mx_sf_bytes": (SZ, [I64, I64, I32, I32]),
     "nvfp4_quantize": (I32, [P, I64, I64, I64, P, P, P, I32, P]),
     "mxfp8_requant_transpose_sr": (I32, [P, P, P, I64, I64, I64, I32, P, U64, U64, I32, P, P, I32, P]),

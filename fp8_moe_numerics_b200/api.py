@@ -17,7 +17,7 @@ from ._lib import (MX_GEMM_DGRAD, MX_GEMM_WGRAD, MX_OUT_BF16, MX_OUT_F32, MX_ROU
 
 __all__ = [
     "MX_SF_ROWMAJOR", "MX_SF_MMA", "MX_ROUND_RNE", "MX_ROUND_SR", "MX_GEMM_DGRAD", "MX_GEMM_WGRAD", "MxError",
-    "sf_bytes", "sync_status", "nvfp4_quantize", "mxfp8_requant_transpose_sr", "mxfp8_quantize",
+    "sf_bytes", "sync_status", "wait_selftest", "nvfp4_quantize", "mxfp8_requant_transpose_sr", "mxfp8_quantize",
     "grouped_gemm_nvfp4", "grouped_gemm_mxfp8", "moe_route", "nvfp4_gather_rows", "swiglu_fwd", "swiglu_bwd",
     "moe_combine", "moe_dispatch_grad",
 ]
@@ -53,6 +53,12 @@ def sync_status(stream=None) -> None:
     st = L.lib().mx_sync_status(s)
     if st != L.MX_OK:
         raise MxError("mx_sync_status", st, L.lib().mx_last_cuda_error())
+
+
+def wait_selftest(limit_us: int) -> None:
+    """Run the bounded-wait expiry path once; the next sync_status() raises
+    MxError with status MX_ETIMEOUT."""
+    L.call("mx_wait_selftest", int(limit_us), _s())
 
 
 def nvfp4_quantize(x: torch.Tensor, group_rows: int = 1, sf_layout: int = MX_SF_MMA, out=None):

@@ -91,13 +91,14 @@ __device__ __forceinline__ unsigned long long globaltimer() {
 
 // Bounded wait: false (and the abort flag / status word set) on expiry or when
 // another role of this CTA has already aborted.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort_flag) return false;
-        if (globaltimer() - t0 > kWaitLimitNs) {
+        if (globaltimer() - t0 > limit_ns) {
             *abort_flag = 1;
             atomicOr(&g_mx_status_word, 1u);
             return false;
@@ -790,6 +791,20 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     }
 }
 
+// The bounded wait on a barrier that nothing completes: exercises the expiry
+// path (status word set, kernel returns) without a fault or a hang.
+__global__ void wait_selftest_kernel(unsigned long long limit_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) (void)mbar_wait(&bar, 0, &abort_flag, limit_ns);
+}
+
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
@@ -924,11 +939,19 @@ extern "C" int mx_sync_status(cudaStream_t stream) {
     return word ? MX_ETIMEOUT : MX_OK;
 }
 
+extern "C" int mx_wait_selftest(int64_t limit_us, cudaStream_t stream) {
+    if (limit_us <= 0 || limit_us > 10 * 1000 * 1000) return MX_EINVAL;
+    if (int st = mx_check_device()) return st;
+    wait_selftest_kernel<<<1, 32, 0, stream>>>((unsigned long long)limit_us * 1000ull);
+    mx_count_launch();
+    return mx_launch_status();
+}
+
 extern "C" int grouped_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_outer,
                                   const uint8_t* b_codes, const uint8_t* b_sf, const float* b_outer,
                                   const int64_t* seg_offsets, int64_t E, int64_t M_cap, int64_t N, int64_t K,
                                   void* out, int out_dtype, cudaStream_t stream) {
-    if (!a_codes || !a_sf || !a_outer || !b_codes || !b_sf || !b_outer || !seg_offsets || !out || E < 1 ||
+    if (((!a_codes || !a_sf || !a_outer || !b_codes || !b_sf || !b_outer || !seg_offsets || !out) && M_cap > 0) || E < 1 ||
         M_cap < 0 || M_cap % 128 || N <= 0 || N % 128 || K <= 0 || K % 256)
         return MX_EINVAL;
     if (out_dtype != MX_OUT_F32 && out_dtype != MX_OUT_BF16) return MX_EINVAL;
@@ -952,7 +975,8 @@ extern "C" int grouped_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_sf, c
 extern "C" int grouped_gemm_mxfp8(int mode, const uint8_t* a_codes, const uint8_t* a_e8m0, const uint8_t* b_codes,
                                   const uint8_t* b_e8m0, const int64_t* seg_offsets, int64_t E, int64_t M_cap,
                                   int64_t N, int64_t K, void* out, int out_dtype, cudaStream_t stream) {
-    if (!a_codes || !a_e8m0 || !b_codes || !b_e8m0 || !seg_offsets || !out || E < 1 || M_cap < 0 || M_cap % 128 ||
+    if (((!a_codes || !a_e8m0 || !b_codes || !b_e8m0 || !seg_offsets) && M_cap > 0) || !out || E < 1 || M_cap < 0 ||
+        M_cap % 128 ||
         N <= 0 || N % 128 || K <= 0 || K % 128)
         return MX_EINVAL;
     if (mode != MX_GEMM_DGRAD && mode != MX_GEMM_WGRAD) return MX_EINVAL;
@@ -963,6 +987,10 @@ extern "C" int grouped_gemm_mxfp8(int mode, const uint8_t* a_codes, const uint8_
     if (M_cap >= (int64_t)1 << 31 || E * K >= (int64_t)1 << 31 || N >= (int64_t)1 << 31) return MX_EINVAL;
     if (int st = mx_check_device()) return st;
     if (M_cap == 0 && mode == MX_GEMM_DGRAD) return MX_OK;
+    if (M_cap == 0) {                                   // WGRAD without routed rows: every dW_e is zero
+        const cudaError_t e = cudaMemsetAsync(out, 0, (size_t)(E * N * K) * (out_dtype == MX_OUT_BF16 ? 2 : 4), stream);
+        return e == cudaSuccess ? MX_OK : mx_set_cuda_error(e);
+    }
     CUtensorMap ma, mb;
     GemmArgs a{};
     a.sfa = a_e8m0; a.sfb = b_e8m0; a.seg = seg_offsets; a.out = out;
@@ -976,7 +1004,6 @@ extern "C" int grouped_gemm_mxfp8(int mode, const uint8_t* a_codes, const uint8_
                                                (M_cap / kBM) * (N / 256), (M_cap / kBM) * (N / 128), stream);
     }
     // WGRAD: A [N, M_cap], B [K, M_cap]; out [E, N, K]
-    if (M_cap == 0) return MX_EINVAL;
     if (int st = make_map(&ma, a_codes, N, M_cap, kBM)) return st;
     if (int st = make_map(&mb, b_codes, K, M_cap, 128)) return st;
     a.sfa_groups = M_cap / 128; a.sfb_groups = M_cap / 128; a.ldo = K;

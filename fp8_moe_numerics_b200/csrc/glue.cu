@@ -259,7 +259,8 @@ dispatch_grad_kernel(const uint16_t* __restrict__ dout, const int32_t* __restric
 
 extern "C" int moe_route(const int32_t* topk, int64_t T, int64_t k, int64_t E, int64_t M_cap, int64_t* seg_offsets,
                          int32_t* src, int32_t* pos, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
-    if (!topk || !seg_offsets || !src || !pos || T < 0 || k <= 0 || k > 32 || E <= 0 || M_cap < 0 || M_cap % 128)
+    if (((!topk || !pos) && T > 0) || !seg_offsets || !src || T < 0 || k <= 0 || k > 32 || E <= 0 || M_cap < 0 ||
+        M_cap % 128)
         return MX_EINVAL;
     const int64_t need_rows = (T * k + 127 * E + 127) / 128 * 128;
     if (M_cap < need_rows || !workspace || workspace_bytes < mx_route_workspace_bytes(T, E)) return MX_EINVAL;
@@ -286,7 +287,7 @@ extern "C" int moe_route(const int32_t* topk, int64_t T, int64_t k, int64_t E, i
 extern "C" int nvfp4_gather_rows(const uint8_t* codes, const uint8_t* sf, const float* outer, const int32_t* src,
                                  int64_t k, int64_t M_cap, int64_t cols, uint8_t* out_codes, uint8_t* out_sf,
                                  float* out_outer, cudaStream_t stream) {
-    if (!codes || !sf || !outer || !src || !out_codes || !out_sf || !out_outer || k <= 0 || M_cap < 0 ||
+    if (((!codes || !sf || !outer || !src || !out_codes || !out_sf || !out_outer) && M_cap > 0) || k <= 0 || M_cap < 0 ||
         M_cap % 128 || cols <= 0 || cols % 64 || !mx_aligned(codes, 16) || !mx_aligned(out_codes, 16) ||
         !mx_aligned(sf, 4) || !mx_aligned(out_sf, 4))
         return MX_EINVAL;

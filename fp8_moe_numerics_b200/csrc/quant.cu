@@ -422,7 +422,8 @@ int dispatch_layout(int layout, F&& f) {
 
 extern "C" int nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t group_rows, uint8_t* codes,
                               uint8_t* sf, float* outer, int sf_layout, cudaStream_t stream) {
-    if (!x || !codes || !sf || !outer || rows < 0 || cols <= 0 || cols % 16 || group_rows <= 0 ||
+    // an empty problem succeeds without touching memory (its pointers may be null)
+    if (((!x || !codes || !sf || !outer) && rows > 0) || rows < 0 || cols <= 0 || cols % 16 || group_rows <= 0 ||
         rows % group_rows || !mx_aligned(x, 16) || !mx_aligned(codes, 16))
         return MX_EINVAL;
     if (sf_layout != MX_SF_ROWMAJOR && sf_layout != MX_SF_MMA) return MX_EINVAL;
@@ -475,7 +476,8 @@ extern "C" int mxfp8_quantize(const void* x, int64_t rows, int64_t cols, int rou
                               uint8_t* row_codes, uint8_t* row_e8m0, uint8_t* col_codes, uint8_t* col_e8m0,
                               int sf_layout, cudaStream_t stream) {
     const bool do_row = row_codes != nullptr, do_col = col_codes != nullptr;
-    if (!x || rows < 0 || cols <= 0 || rows % kTR || cols % 128 || !mx_aligned(x, 16)) return MX_EINVAL;
+    if ((!x && rows > 0) || rows < 0 || cols <= 0 || rows % kTR || cols % 128 || !mx_aligned(x, 16)) return MX_EINVAL;
+    if (rows == 0) return MX_OK;                        // nothing to compute in either form
     if (!do_row && !do_col) return MX_EINVAL;
     if ((do_row && (!row_e8m0 || !mx_aligned(row_codes, 16))) || (do_col && (!col_e8m0 || !mx_aligned(col_codes, 16))))
         return MX_EINVAL;
@@ -483,7 +485,6 @@ extern "C" int mxfp8_quantize(const void* x, int64_t rows, int64_t cols, int rou
     if (rounding == MX_ROUND_SR && rbits != 8 && rbits != 16 && rbits != 32) return MX_EINVAL;
     if (sf_layout != MX_SF_ROWMAJOR && sf_layout != MX_SF_MMA) return MX_EINVAL;
     if (int st = mx_check_device()) return st;
-    if (rows == 0) return MX_OK;
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const dim3 grid((unsigned)std::min<int64_t>((cols / kTC) * (rows / kTR), (int64_t)sms * 4));
@@ -519,7 +520,8 @@ extern "C" int mxfp8_requant_transpose_sr(const uint8_t* codes, const uint8_t* s
                                           const int64_t* rows_valid, uint64_t seed, uint64_t stream_id, int rbits,
                                           uint8_t* out_codes, uint8_t* out_e8m0, int out_sf_layout,
                                           cudaStream_t stream) {
-    if (!codes || !sf || !outer || !out_codes || !out_e8m0 || rows < 0 || cols <= 0 || rows % kTR || cols % kTC ||
+    if (((!codes || !sf || !outer || !out_codes || !out_e8m0) && rows > 0) || rows < 0 || cols <= 0 || rows % kTR ||
+        cols % kTC ||
         group_rows <= 0 || rows % group_rows || !mx_aligned(codes, 16) || !mx_aligned(out_codes, 16))
         return MX_EINVAL;
     if (rbits != 8 && rbits != 16 && rbits != 32) return MX_EINVAL;

@@ -21,6 +21,9 @@
  *     mx_last_cuda_error() gives the cudaError_t), MX_EUNSUPPORTED (device is
  *     not sm_100 or a mode that is not built).  Device-side bounded waits that
  *     expire are reported later by mx_sync_status() as MX_ETIMEOUT.
+ *   - An empty problem (rows == 0, M_cap == 0, T == 0) succeeds without
+ *     touching memory, and the pointers of its empty arrays may be NULL; a
+ *     weight-gradient GEMM without routed rows writes zeros to its output.
  *   - bf16 tensors are row-major, 2 bytes per element.
  *   - NVFP4 tensor [rows, cols]: codes u8 [rows, cols/2] (E2M1, element 2j in
  *     the low nibble of byte j), E4M3 block scales (one per 16 consecutive
@@ -79,6 +82,14 @@ MX_API unsigned long long mx_kernel_launches(void);
  * expired since the last call (that kernel's output is then undefined),
  * MX_ECUDA if the synchronisation failed, else MX_OK. */
 MX_API int mx_sync_status(cudaStream_t stream);
+
+/* Failure-detection self-test: one kernel waits on a barrier that nothing
+ * completes, gives up after `limit_us` microseconds (1 .. 10^7) the way the
+ * GEMM kernels' bounded waits do, and records MX_ETIMEOUT in the device status
+ * word; the next mx_sync_status() returns MX_ETIMEOUT and clears it.  Nothing
+ * faults and the context stays usable.  MX_EINVAL for a limit out of range.
+ * The pages have no counterpart. */
+MX_API int mx_wait_selftest(int64_t limit_us, cudaStream_t stream);
 
 /* Bytes of a scale array of `rows` x `cols` elements with one scale per
  * `block` (16 or 32) elements in `sf_layout`; 0 if the shape is not allowed

@@ -31,6 +31,11 @@ def test_every_declared_symbol_is_exported(mx):
     assert set(SIGNATURES) == set(names)
 
 
+def test_wait_selftest_limit_checked_on_host(mx):
+    assert mx.mx_wait_selftest(0, None) == 1
+    assert mx.mx_wait_selftest(10 * 1000 * 1000 + 1, None) == 1
+
+
 def test_launch_counter_ignores_rejected_calls(mx):
     before = mx.mx_kernel_launches()
     assert isinstance(before, int) and before >= 0
