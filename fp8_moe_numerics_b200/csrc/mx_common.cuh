@@ -42,12 +42,18 @@ __host__ __device__ __forceinline__ int64_t sf_offset(int64_t r, int64_t s, int6
 // Element conversions (PTX cvt, sm_100a)
 // ---------------------------------------------------------------------------
 // Two fp32 -> one byte of two E2M1 codes; `lo` lands in the low nibble.
-__device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
+// Eight values -> one word of E2M1 codes: byte j holds v[2j] in its low nibble
+// and v[2j+1] in its high nibble (RNE, satfinite); the four code bytes are
+// packed by a vector mov, with byte 0 the least significant.
+__device__ __forceinline__ uint32_t cvt_e2m1x8(const float* v) {
     uint32_t out;
-    asm("{\n\t.reg .b8 b;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b, %2, %1;\n\t"
-        "cvt.u32.u8 %0, b;\n\t}"
-        : "=r"(out) : "f"(lo), "f"(hi));
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(out) : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
     return out;
 }
 

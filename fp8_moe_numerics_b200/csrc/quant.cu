@@ -34,12 +34,13 @@ __device__ __forceinline__ uint32_t nvfp4_block(const uint4& a, const uint4& b, 
     if (sc == 0) { packed = make_uint2(0u, 0u); return 0u; }
     float inv = __frcp_rn(__fmul_rn(e4m3_to_f32(sc), s));
     const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-    uint32_t byte[8];
+    float y[16];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) byte[i] = cvt_e2m1x2(__fmul_rn(bf16_lo(w[i]), inv), __fmul_rn(bf16_hi(w[i]), inv));
-    // bytes -> words with byte permutes (byte 1 of a code byte is zero)
-    packed = make_uint2(__byte_perm(__byte_perm(byte[0], byte[1], 0x1140), __byte_perm(byte[2], byte[3], 0x1140), 0x5410),
-                        __byte_perm(__byte_perm(byte[4], byte[5], 0x1140), __byte_perm(byte[6], byte[7], 0x1140), 0x5410));
+    for (int i = 0; i < 8; ++i) {
+        y[2 * i] = __fmul_rn(bf16_lo(w[i]), inv);
+        y[2 * i + 1] = __fmul_rn(bf16_hi(w[i]), inv);
+    }
+    packed = make_uint2(cvt_e2m1x8(y), cvt_e2m1x8(y + 8));
     return sc;
 }
 
