@@ -64,6 +64,18 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
     return out;
 }
 
+// Four values -> E4M3 codes v0 | v1 << 8 | v2 << 16 | v3 << 24 (RNE, satfinite),
+// the two code pairs packed by a vector mov.
+__device__ __forceinline__ uint32_t cvt_e4m3x4(float v0, float v1, float v2, float v3) {
+    uint32_t out;
+    asm("{\n\t.reg .b16 h0, h1;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 h0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 h1, %4, %3;\n\t"
+        "mov.b32 %0, {h0, h1};\n\t}"
+        : "=r"(out) : "f"(v0), "f"(v1), "f"(v2), "f"(v3));
+    return out;
+}
+
 // One E4M3 code -> fp32 (exact).
 __device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
     uint32_t h2;
@@ -72,14 +84,21 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
     return __half2float(__ushort_as_half((unsigned short)(h2 & 0xffff)));
 }
 
-// Byte of two E2M1 codes -> two halves (exact).
-__device__ __forceinline__ __half2 e2m1x2_to_h2(uint32_t byte) {
-    uint32_t h2;
-    asm("{\n\t.reg .b8 b;\n\t"
-        "cvt.u8.u32 b, %1;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %0, b;\n\t}"
-        : "=r"(h2) : "r"(byte));
-    return *reinterpret_cast<__half2*>(&h2);
+// Word of eight E2M1 codes -> four halves pairs (exact): h[j] holds the codes
+// of byte j (low nibble first); the bytes are unpacked by a vector mov.
+__device__ __forceinline__ void e2m1x8_to_h2x4(uint32_t w, __half2* h) {
+    uint32_t r0, r1, r2, r3;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+        : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(w));
+    h[0] = *reinterpret_cast<__half2*>(&r0);
+    h[1] = *reinterpret_cast<__half2*>(&r1);
+    h[2] = *reinterpret_cast<__half2*>(&r2);
+    h[3] = *reinterpret_cast<__half2*>(&r3);
 }
 
 // E4M3 code -> half (exact: E4M3 is a subset of fp16).

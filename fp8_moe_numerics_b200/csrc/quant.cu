@@ -274,8 +274,8 @@ __device__ __forceinline__ void tile_emit_transposed(const float* T, int64_t row
             const float sc = exp2_neg(e);
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-                w[i] = cvt_e4m3x2(__fmul_rn(v[4 * i], sc), __fmul_rn(v[4 * i + 1], sc)) |
-                       (cvt_e4m3x2(__fmul_rn(v[4 * i + 2], sc), __fmul_rn(v[4 * i + 3], sc)) << 16);
+                w[i] = cvt_e4m3x4(__fmul_rn(v[4 * i], sc), __fmul_rn(v[4 * i + 1], sc), __fmul_rn(v[4 * i + 2], sc),
+                                  __fmul_rn(v[4 * i + 3], sc));
         }
         *reinterpret_cast<uint4*>(out_codes + cg * rows + rr) = make_uint4(w[0], w[1], w[2], w[3]);
         if ((g & 1) == 0) out_e8m0[sf_offset(cg, rr >> 5, S, kLayout)] = (uint8_t)(e + 127);
@@ -354,8 +354,8 @@ mxfp8_tile_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, co
                 const float sc = exp2_neg(e);
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
-                    w[i] = cvt_e4m3x2(__fmul_rn(v[4 * i], sc), __fmul_rn(v[4 * i + 1], sc)) |
-                           (cvt_e4m3x2(__fmul_rn(v[4 * i + 2], sc), __fmul_rn(v[4 * i + 3], sc)) << 16);
+                    w[i] = cvt_e4m3x4(__fmul_rn(v[4 * i], sc), __fmul_rn(v[4 * i + 1], sc),
+                                      __fmul_rn(v[4 * i + 2], sc), __fmul_rn(v[4 * i + 3], sc));
             }
             uint4* dst = reinterpret_cast<uint4*>(row_codes + L0);
             dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
@@ -397,11 +397,12 @@ requant_tile_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict
     const float so = outer[group_rows == 1 ? r : (int64_t)((uint32_t)r0 / (uint32_t)group_rows)];
     const __half2 f0 = __half2half2(e4m3_to_h(sc0)), f1 = __half2half2(e4m3_to_h(sc1));
     const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+    __half2 hv[16];                                    // hv[i]: elements 2i, 2i+1
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {                     // byte i = elements 2i, 2i+1
-        const uint32_t byte = (w[i >> 2] >> (8 * (i & 3))) & 0xffu;
-        const __half2 p = __hmul2(e2m1x2_to_h2(byte), i < 8 ? f0 : f1);   // exact
-        const float2 pf = __half22float2(p);
+    for (int j = 0; j < 4; ++j) e2m1x8_to_h2x4(w[j], hv + 4 * j);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float2 pf = __half22float2(__hmul2(hv[i], i < 8 ? f0 : f1));   // exact products
         T[tsw(32 * h + 2 * i, rl)] = __fmul_rn(pf.x, so);
         T[tsw(32 * h + 2 * i + 1, rl)] = __fmul_rn(pf.y, so);
     }
