@@ -404,7 +404,7 @@ __device__ __forceinline__ Tile make_tile(const GemmArgs& p, int64_t idx, uint32
 // only two scale regions (a ring released by MMA commits, decoupled from the
 // shared-memory stages) to make that overlap small.
 constexpr int kSmemLimit = 227 * 1024;
-template <int kKind, int kBN, bool kPair>
+template <int kKind, int kBN, bool kPair, bool kOutBF16>
 struct Smem {
     static constexpr int kA = kBM * kStageBytesK;                       // 16 KB
     static constexpr int kB = (kPair ? kBN / 2 : kBN) * kStageBytesK;
@@ -415,16 +415,22 @@ struct Smem {
     static constexpr int kAbTx = kA + kB;                               // operand bytes per stage and CTA
     static constexpr int kSfTx = kSfa + kSfb;
     static constexpr int kStage = (kAbTx + kSfTx + 1023) / 1024 * 1024;  // stride keeps every SW128 tile 1024-aligned
-    static constexpr int kStaging = 8 * 4096;                           // epilogue: 4 KB of store boxes per warp
     static constexpr int kSfaCols = 4 * kAtomsA;
     static constexpr int kSfbCols = 4 * kAtomsB;
     static constexpr int kSfRegion = kSfaCols + kSfbCols;
     static constexpr int kPfxBytes = kPair ? 4 * (kMaxPairExperts + 4) : 0;
-    static constexpr int kFixed = kStaging + 512 + kPfxBytes + 1024;    // + barriers + prefix + alignment slack
-    static constexpr int fit(int s) {
-        return s * kStage + kFixed <= kSmemLimit ? s : 0;
+    static constexpr int kFixed = 512 + kPfxBytes + 1024;               // barriers + prefix + alignment slack
+    static constexpr int stages_for(int staging) {
+        for (int s = 6; s > 2; --s)
+            if (s * kStage + staging + kFixed <= kSmemLimit) return s;
+        return 2;
     }
-    static constexpr int kStages = fit(6) ? 6 : fit(5) ? 5 : fit(4) ? 4 : fit(3) ? 3 : 2;
+    // Epilogue staging, 8 warps: fp32 boxes need 4 KB each; bf16 boxes are 2 KB
+    // and get two buffers per warp unless giving up the second buys a
+    // pipeline stage (operands in flight are what bound these kernels).
+    static constexpr bool kOneBox = kOutBF16 && stages_for(8 * 2048) > stages_for(8 * 4096);
+    static constexpr int kStaging = kOneBox ? 8 * 2048 : 8 * 4096;
+    static constexpr int kStages = stages_for(kStaging);
     static constexpr int kStagingOff = kStages * kStage;
     static_assert(kStage % 1024 == 0 && kStagingOff % 1024 == 0, "128-byte swizzle needs 1024-byte aligned tiles");
     static constexpr int kBarOff = kStagingOff + kStaging;
@@ -457,7 +463,7 @@ template <int kKind, int kMode, int kBN, bool kOutBF16, bool kPair>
 __global__ void __launch_bounds__(kThreads, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmOut, const GemmArgs p) {
-    using L = Smem<kKind, kBN, kPair>;
+    using L = Smem<kKind, kBN, kPair, kOutBF16>;
     constexpr int kStages = L::kStages;
     constexpr int kSlots = L::kSfSlots;
     constexpr bool kSfRing = kSlots < kStages;                          // scale regions released by MMA commits
@@ -678,14 +684,15 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         // reports on acc_free, then converts, stages each chunk as one 32x32
         // box in shared memory and writes it with a TMA tensor store.  bf16
         // boxes (64-byte rows, 64-byte swizzle) alternate between two 2 KB
-        // buffers; fp32 boxes (128-byte rows, 128-byte swizzle) use one 4 KB
-        // buffer.  A pair's CTAs each drain their own 128 rows.
+        // buffers, or use one when the second would cost a pipeline stage;
+        // fp32 boxes (128-byte rows, 128-byte swizzle) use one 4 KB buffer.  A
+        // pair's CTAs each drain their own 128 rows.
         constexpr int kChunks = kBN / 32;
         constexpr int kOv = L::kOvChunks;
         const int q = warp & 3;
         const int h = (warp - 8) >> 2;
         const int r = q * 32 + lane;
-        uint8_t* stg = smem + L::kStagingOff + (warp - 8) * 4096;
+        uint8_t* stg = smem + L::kStagingOff + (warp - 8) * (L::kStaging / 8);
         const uint32_t acc_free_lead[2] = {kPair ? map_to_rank(&acc_free[0], 0) : 0u,
                                            kPair ? map_to_rank(&acc_free[1], 0) : 0u};
         uint32_t it = 0, nbox = 0;
@@ -731,8 +738,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     for (int u = 0; u < 2; ++u) {
                         uint8_t* box;
                         if (kOutBF16) {
-                            box = stg + (nbox & 1u) * 2048;
-                            if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+                            if (L::kOneBox) {
+                                box = stg;
+                                if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+                            } else {
+                                box = stg + (nbox & 1u) * 2048;
+                                if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+                            }
                             __syncwarp();
                             const uint32_t row = smem_u32(box) + (uint32_t)lane * 64u;
 #pragma unroll
@@ -882,7 +894,7 @@ int max_pairs(Kern kern, const cudaLaunchConfig_t& cfg) {
 template <int kKind, int kMode, int kBN, bool kOutBF16, bool kPair>
 int launch(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mo, const GemmArgs& args, int64_t items,
            cudaStream_t stream) {
-    using L = Smem<kKind, kBN, kPair>;
+    using L = Smem<kKind, kBN, kPair, kOutBF16>;
     auto kern = grouped_gemm_kernel<kKind, kMode, kBN, kOutBF16, kPair>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes) != cudaSuccess)
         return mx_launch_status();

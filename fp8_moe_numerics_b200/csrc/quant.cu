@@ -34,13 +34,18 @@ __device__ __forceinline__ uint32_t nvfp4_block(const uint4& a, const uint4& b, 
     if (sc == 0) { packed = make_uint2(0u, 0u); return 0u; }
     float inv = __frcp_rn(__fmul_rn(e4m3_to_f32(sc), s));
     const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-    float y[16];
+    uint32_t word[2];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        y[2 * i] = __fmul_rn(bf16_lo(w[i]), inv);
-        y[2 * i + 1] = __fmul_rn(bf16_hi(w[i]), inv);
+    for (int h = 0; h < 2; ++h) {                      // eight products, then their code word
+        float y[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            y[2 * i] = __fmul_rn(bf16_lo(w[4 * h + i]), inv);
+            y[2 * i + 1] = __fmul_rn(bf16_hi(w[4 * h + i]), inv);
+        }
+        word[h] = cvt_e2m1x8(y);
     }
-    packed = make_uint2(cvt_e2m1x8(y), cvt_e2m1x8(y + 8));
+    packed = make_uint2(word[0], word[1]);
     return sc;
 }
 
