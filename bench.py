@@ -440,7 +440,7 @@ def cpu_baseline(inp, layer, seconds: float = 15.0):
 # larger than L2 where DRAM traffic is read off)
 # --------------------------------------------------------------------------
 KERNEL_CASES = ("gemm_nvfp4", "gemm_mxfp8_dgrad", "gemm_mxfp8_wgrad", "requant", "requant_w", "nvfp4_quantize",
-                "mxfp8_quantize")
+                "quant_w", "mxfp8_quantize")
 
 
 def run_kernel(args):
@@ -484,6 +484,12 @@ def run_kernel(args):
         w = workloads.weights(E, N, K, 0.02, 2, dev).view(E * N, K)
         q = api.nvfp4_quantize(w, N)
         run = lambda: api.mxfp8_requant_transpose_sr(*q, E * N, K, N, seed=1, stream_id=3)
+    elif which == "quant_w":
+        # per-expert NVFP4 of 64 experts of 2048 x 4096 bf16 weights (1.07 GB > L2)
+        E, N, K = 64, 2048, 4096
+        w = workloads.weights(E, N, K, 0.02, 2, dev).view(E * N, K)
+        q = api.nvfp4_quantize(w, N, api.MX_SF_MMA)
+        run = lambda: api.nvfp4_quantize(w, N, api.MX_SF_MMA, out=q)
     else:                                               # mxfp8_quantize, row + column forms, RNE
         x = workloads.gradient(65536, 4096, 1.0, 5, dev)
         run = lambda: api.mxfp8_quantize(x)

@@ -113,6 +113,33 @@ def test_nvfp4_quantize_per_expert_unaligned_groups(cuda):
     assert np.array_equal(np_(go).view(np.uint32), outer.view(np.uint32))
 
 
+@pytest.mark.parametrize("E,N,K,layout", [
+    (8, 512, 4096, api.MX_SF_MMA),        # 4 rows per quantiser block
+    (24, 2048, 1024, api.MX_SF_MMA),      # 16 rows per quantiser block
+    (6, 4096, 1024, api.MX_SF_ROWMAJOR),  # the W2 shape of the 384-expert layer, 6 experts
+    (4, 256, 16384, api.MX_SF_MMA),       # one row per quantiser block
+    (3, 128, 20480, api.MX_SF_ROWMAJOR),  # rows of 1280 blocks: each row read twice by its threads
+])
+def test_nvfp4_quantize_per_expert_spread_and_zero_experts(cuda, E, N, K, layout):
+    # experts six decades apart, one all-zero expert and one expert whose amax
+    # is a single element: a per-expert scale taken from the wrong expert, or
+    # an amax missing some of the expert's rows, changes codes
+    w = workloads.weights(E, N, K, 0.02, seed=E + N + K).float()
+    w *= (10.0 ** torch.linspace(-3, 3, E)).view(E, 1, 1)
+    w[1] = 0
+    w[E - 1, N // 2, K // 3] = 1e4
+    w = w.to(torch.bfloat16)
+    wn = w.reshape(E * N, K).view(torch.int16).numpy().view(np.uint16)
+    codes, sf, outer = oracle.nvfp4_quantize(wn, group_rows=N)
+    gc, gsf, go = api.nvfp4_quantize(w.reshape(E * N, K).cuda(), group_rows=N, sf_layout=layout)
+    api.sync_status()
+    assert np.array_equal(np_(gc), codes)
+    got_sf = mma_to_rowmajor(np_(gsf), E * N, K // 16) if layout == api.MX_SF_MMA else np_(gsf).reshape(sf.shape)
+    assert np.array_equal(got_sf, sf)
+    assert np.array_equal(np_(go).view(np.uint32), outer.view(np.uint32))
+    assert outer[1] == 0 and np.all(codes[N:2 * N] == 0)
+
+
 # ---------------------------------------------------------------------------
 # MXFP8 quantiser
 # ---------------------------------------------------------------------------
