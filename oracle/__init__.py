@@ -31,11 +31,16 @@ Parity pins (tests/test_oracle_*.py):
   GEMMs ............. brute-force loops on tiny inputs; plain matmul special
                       cases; empty experts
   glue .............. brute-force permutation; SiLU vs torch; combine loops
+  hadamard / s2f6 ... butterflies vs the Kronecker-built Sylvester matrix on
+                      integer vectors; H32 H32 = 32 I; exponent by search
+                      over all exponents; ties to even; one-hot outlier
+                      closed form; reconstruction error bound; combine loops
 No oracle function is "parity unpinned".
 """
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 import subprocess
 
@@ -467,3 +472,107 @@ def dispatch_grad(dout_bf16: np.ndarray, pos: np.ndarray, w: np.ndarray, M: int)
     for j in range(k):
         dy[pos[:, j]] = w[:, j, None].astype(np.float64) * d
     return f64_to_bf16(dy)
+
+
+# --------------------------------------------------------------------------
+# Combine path: 32-d random Hadamard rotation + block-scaled S2F6
+# [ai-primer §Quantized NVLink and BBBK]: expert outputs are rotated by a
+# 32-dimensional random Hadamard transform and quantised to S2F6 (eight-bit
+# fixed point: two signed integer bits, six fractional bits) with a block
+# scale before the combine.  Readings taken where the pages are silent:
+#   rotation  z = H32 (sigma_j * x) per 32-column block j of a row, H32 the
+#             unnormalised Sylvester matrix, H[a][b] = (-1)^popcount(a & b);
+#             sigma_j in {+1,-1}^32: coordinate i flipped iff bit i of word 0
+#             of Philox4x32-10(counter (j, stream), key seed) is set.  Inverse
+#             x = sigma_j * (H32 z) / 32 (H32 H32 = 32 I), so both directions
+#             scale by powers of two only.
+#   order     z is the fp32 result of the five butterfly stages h = 1, 2, 4,
+#             8, 16: (a, b) -> (a + b, a - b) for every pair (i, i + h) with
+#             i & h == 0, each an fp32 round-to-nearest add.
+#   scale     one E8M0 exponent per 32-value block: e = smallest integer with
+#             amax|z| <= (127/64) 2^e, clamped to [-127, 127] (-127 for a zero
+#             block); code c = RNE(z 2^(6-e)) clamped to [-127, 127] (int8);
+#             value c 2^(e-6).  -128 is never produced (symmetric range).
+# --------------------------------------------------------------------------
+S2F6_MAX = 127.0 / 64.0
+
+
+def hadamard_sign_words(seed: int, stream: int, nblocks: int) -> np.ndarray:
+    """Sign mask of each 32-column block j < nblocks (bit i set: coordinate i
+    is negated before the transform)."""
+    key = [seed & 0xFFFFFFFF, seed >> 32]
+    out = np.empty(nblocks, dtype=np.uint32)
+    for j in range(nblocks):
+        out[j] = philox4x32_10([j & 0xFFFFFFFF, j >> 32, stream & 0xFFFFFFFF, stream >> 32], key)[0]
+    return out
+
+
+def hadamard_signs(seed: int, stream: int, cols: int) -> np.ndarray:
+    """+1/-1 per column (float64), from hadamard_sign_words."""
+    words = hadamard_sign_words(seed, stream, cols // 32)
+    bits = (words[:, None] >> np.arange(32, dtype=np.uint32)[None, :]) & 1
+    return np.where(bits.reshape(-1) == 1, -1.0, 1.0)
+
+
+def fwht32_f32(y: np.ndarray) -> np.ndarray:
+    """Unnormalised Walsh-Hadamard transform of the last axis (length 32) in
+    fp32, stage by stage as stated above."""
+    z = np.array(y, dtype=np.float32, copy=True)
+    lead = z.shape[:-1]
+    h = 1
+    while h < 32:
+        z = z.reshape(lead + (32 // (2 * h), 2, h))
+        a, b = z[..., 0, :], z[..., 1, :]
+        z = np.stack([a + b, a - b], axis=-2).reshape(lead + (32,))
+        h *= 2
+    return z
+
+
+def s2f6_exponent(amax: float) -> int:
+    """Smallest integer e with amax <= (127/64) 2^e, clamped to [-127, 127]."""
+    if amax == 0.0:
+        return -127
+    m, E = math.frexp(float(amax))              # amax = m 2^E, m in [0.5, 1)
+    m2, E1 = 2.0 * m, E - 1                     # amax = m2 2^E1, m2 in [1, 2)
+    e = E1 if m2 <= S2F6_MAX else E1 + 1
+    return max(-127, min(127, e))
+
+
+def s2f6_quantize_hadamard(x_f32: np.ndarray, seed: int, stream: int):
+    """x fp32 [rows, cols] (cols % 32 == 0) -> (codes int8 [rows, cols],
+    e8m0 uint8 [rows, cols/32], biased by 127)."""
+    x = np.ascontiguousarray(x_f32, dtype=np.float32)
+    rows, cols = x.shape
+    sig = hadamard_signs(seed, stream, cols).astype(np.float32)
+    z = fwht32_f32((x * sig[None, :]).reshape(rows, cols // 32, 32))       # sign flips are exact
+    amax = np.abs(z).max(axis=-1).astype(np.float64)
+    e = np.array([s2f6_exponent(a) for a in amax.reshape(-1)], dtype=np.int64).reshape(amax.shape)
+    y = z.astype(np.float64) * np.ldexp(1.0, 6 - e)[..., None]             # exact: power-of-two scaling
+    c = np.clip(np.rint(y), -127, 127).astype(np.int8)                     # np.rint: round half to even
+    return c.reshape(rows, cols), (e + 127).astype(np.uint8)
+
+
+def s2f6_dequantize_hadamard(codes: np.ndarray, e8m0: np.ndarray, seed: int, stream: int) -> np.ndarray:
+    """Inverse of s2f6_quantize_hadamard up to the quantisation: fp64 [rows, cols]."""
+    rows, cols = codes.shape
+    zhat = codes.astype(np.float64).reshape(rows, cols // 32, 32) * np.ldexp(1.0, e8m0.astype(np.int64) - 127 - 6)[..., None]
+    H = sylvester_hadamard(32)
+    x = (zhat @ H.T).reshape(rows, cols) / 32.0
+    return x * hadamard_signs(seed, stream, cols)[None, :]
+
+
+def sylvester_hadamard(n: int) -> np.ndarray:
+    """H_n by Kronecker products of [[1, 1], [1, -1]] (fp64)."""
+    H = np.ones((1, 1))
+    while H.shape[0] < n:
+        H = np.kron(H, np.array([[1.0, 1.0], [1.0, -1.0]]))
+    return H
+
+
+def combine_s2f6(codes: np.ndarray, e8m0: np.ndarray, pos: np.ndarray, w: np.ndarray, seed: int,
+                 stream: int) -> np.ndarray:
+    """out[t] = sum_j w[t, j] * xhat[pos[t, j]], xhat the dequantised, rotated-
+    back rows (fp64, one rounding to bf16)."""
+    xhat = s2f6_dequantize_hadamard(codes, e8m0, seed, stream)
+    out = np.einsum("tj,tjd->td", w.astype(np.float64), xhat[pos])
+    return f64_to_bf16(out)
