@@ -306,6 +306,7 @@ def run_ours(args):
                             "frac_measured": round(tf / (peaks["bf16_sus"] * ratio), 3) if tf else None}
 
     quant = quantiser_stream(dev, peaks) if rank == 0 else None
+    s2f6 = combine_s2f6_leg(layer, c, counts, peaks) if rank == 0 else None
 
     # ---------------------------------------------------------------- e2e
     e2e = e2e_leg(layer, inp, dev, args, gemm_flops / K, pg, world)
@@ -325,6 +326,7 @@ def run_ours(args):
                        "peak_measured_basis": f"{peaks['src']} bf16 sustained {peaks['bf16_sus']} x4"},
         "stages": breakdown,
         "quantiser": quant,
+        "combine_s2f6": s2f6,
         "roofline": roof,
         "clocks": clk.summary(),
         "e2e": e2e,
@@ -374,6 +376,51 @@ def quantiser_stream(dev, peaks, reps: int = 20):
         res[name] = {"us": round(med * 1e3, 2), "GB/s": round(gbs, 1), "frac_hbm_measured": round(gbs / peaks["hbm"], 3),
                      "frac_hbm_8tbs": round(gbs / NOMINAL_HBM_GBS, 3), "bytes": int(nbytes)}
     res["workload"] = "quant_stream: bf16 16384x4096 Student-t(4) x 10^U(-3,3) per row; L2 flushed per launch"
+    return res
+
+
+def combine_s2f6_leg(layer, c, counts, peaks, reps: int = 10):
+    """The combine path in S2F6 beside the bf16 one, on the layer's own
+    operands after the timed steps: GEMM2 with the bf16 epilogue vs the
+    rotate + S2F6 epilogue, and the combine reading bf16 vs S2F6 rows."""
+    import torch
+    from fp8_moe_numerics_b200 import api
+    L = layer
+    E, D, F, T, k, M = L.E, L.D, L.F, L.T, L.k, L.M_cap
+    seed, sid = c["seed"], 101
+    codes = torch.empty(M, D, dtype=torch.int8, device=L.dev)
+    e8 = torch.empty(M, D // 32, dtype=torch.uint8, device=L.dev)
+    rows = int(sum(int(x) for x in counts))
+    flops = 2 * rows * D * F
+    legs = (
+        ("gemm2_bf16", lambda: api.grouped_gemm_nvfp4(L.aq, L.w2q, L.seg, E, D, F, out=L.y2), "flops", flops),
+        ("gemm2_s2f6", lambda: api.grouped_gemm_nvfp4_s2f6(L.aq, L.w2q, L.seg, E, D, F, seed, sid, out=(codes, e8)),
+         "flops", flops),
+        ("combine_bf16", lambda: api.moe_combine(L.y2, L.pos, L.w_comb, D, out=L.out), "bytes",
+         T * k * D * 2 + T * D * 2 + T * k * 8),
+        ("combine_s2f6", lambda: api.moe_combine_s2f6(codes, e8, L.pos, L.w_comb, seed, sid, out=L.out), "bytes",
+         T * k * (D + D // 32) + T * D * 2 + T * k * 8),
+    )
+    res = {}
+    for name, fn, kind, work in legs:
+        for _ in range(3):
+            fn()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / reps
+        if kind == "flops":
+            res[name] = {"ms": round(ms, 4), "TFLOP/s": round(work / (ms * 1e-3) / 1e12, 1)}
+        else:
+            gbs = work / (ms * 1e-3) / 1e9
+            res[name] = {"ms": round(ms, 4), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm"], 3)}
+    api.sync_status()
+    res["bytes_y2"] = {"bf16": M * D * 2, "s2f6": M * D + M * D // 32}
+    res["note"] = ("32-d random Hadamard + block-scaled S2F6 in GEMM2's epilogue and the combine reading it, "
+                   f"on the layer's operands ({reps} back-to-back launches each)")
     return res
 
 
@@ -439,8 +486,8 @@ def cpu_baseline(inp, layer, seconds: float = 15.0):
 # single-kernel cases for ncu captures (small enough to profile, outputs
 # larger than L2 where DRAM traffic is read off)
 # --------------------------------------------------------------------------
-KERNEL_CASES = ("gemm_nvfp4", "gemm_mxfp8_dgrad", "gemm_mxfp8_wgrad", "requant", "requant_w", "nvfp4_quantize",
-                "quant_w", "mxfp8_quantize")
+KERNEL_CASES = ("gemm_nvfp4", "gemm_nvfp4_s2f6", "gemm_mxfp8_dgrad", "gemm_mxfp8_wgrad", "requant", "requant_w",
+                "nvfp4_quantize", "quant_w", "mxfp8_quantize")
 
 
 def run_kernel(args):
@@ -461,6 +508,11 @@ def run_kernel(args):
         w1q = api.nvfp4_quantize(w1, 2 * F, api.MX_SF_MMA)
         if which == "gemm_nvfp4":
             run = lambda: api.grouped_gemm_nvfp4(xp, w1q, seg, E, 2 * F, D)
+        elif which == "gemm_nvfp4_s2f6":
+            # the down projection (N = d_model, K = d_ff) with the rotate + S2F6 epilogue
+            a = api.nvfp4_quantize(workloads.activations(M, F, "t3", 4, dev), 1, api.MX_SF_MMA)
+            w2q = api.nvfp4_quantize(workloads.weights(E, D, F, 0.02, 5, dev).view(E * D, F), D, api.MX_SF_MMA)
+            run = lambda: api.grouped_gemm_nvfp4_s2f6(a, w2q, seg, E, D, F, 1, 101)
         else:
             dh = workloads.gradient(M, 2 * F, 1e-3, 3, dev)
             q = api.mxfp8_quantize(dh)

@@ -19,7 +19,7 @@ __all__ = [
     "MX_SF_ROWMAJOR", "MX_SF_MMA", "MX_ROUND_RNE", "MX_ROUND_SR", "MX_GEMM_DGRAD", "MX_GEMM_WGRAD", "MxError",
     "sf_bytes", "sync_status", "wait_selftest", "nvfp4_quantize", "mxfp8_requant_transpose_sr", "mxfp8_quantize",
     "grouped_gemm_nvfp4", "grouped_gemm_mxfp8", "moe_route", "nvfp4_gather_rows", "swiglu_fwd", "swiglu_bwd",
-    "moe_combine", "moe_dispatch_grad",
+    "moe_combine", "moe_dispatch_grad", "hadamard_s2f6_quantize", "grouped_gemm_nvfp4_s2f6", "moe_combine_s2f6",
 ]
 
 
@@ -203,4 +203,40 @@ def moe_dispatch_grad(dout: torch.Tensor, src: torch.Tensor, pos: torch.Tensor, 
     if out is None:
         out = torch.empty(M_cap, D, dtype=torch.bfloat16, device=dout.device)
     L.call("moe_dispatch_grad", _p(dout), _p(src), _p(pos), _p(w), T, k, M_cap, D, _p(out), _s())
+    return out
+
+
+def hadamard_s2f6_quantize(x: torch.Tensor, seed: int, stream_id: int, out=None):
+    """bf16 [rows, cols] -> (codes int8 [rows, cols], e8m0 u8 [rows, cols/32]):
+    32-d random Hadamard rotation per column block, block-scaled S2F6."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2
+    rows, cols = x.shape
+    if out is None:
+        out = (torch.empty(rows, cols, dtype=torch.int8, device=x.device),
+               torch.empty(rows, cols // 32, dtype=torch.uint8, device=x.device))
+    codes, e8m0 = out
+    L.call("hadamard_s2f6_quantize", _p(x), rows, cols, seed, stream_id, _p(codes), _p(e8m0), _s())
+    return codes, e8m0
+
+
+def grouped_gemm_nvfp4_s2f6(a, b, seg: torch.Tensor, E: int, N: int, K: int, seed: int, stream_id: int, out=None):
+    """grouped_gemm_nvfp4 whose epilogue writes S2F6: (codes int8 [M_cap, N], e8m0 u8 [M_cap, N/32])."""
+    M_cap = a[0].shape[0]
+    if out is None:
+        out = (torch.empty(M_cap, N, dtype=torch.int8, device=a[0].device),
+               torch.empty(M_cap, N // 32, dtype=torch.uint8, device=a[0].device))
+    codes, e8m0 = out
+    L.call("grouped_gemm_nvfp4_s2f6", _p(a[0]), _p(a[1]), _p(a[2]), _p(b[0]), _p(b[1]), _p(b[2]), _p(seg), E, M_cap,
+           N, K, seed, stream_id, _p(codes), _p(e8m0), _s())
+    return codes, e8m0
+
+
+def moe_combine_s2f6(codes: torch.Tensor, e8m0: torch.Tensor, pos: torch.Tensor, w, seed: int, stream_id: int,
+                     out=None):
+    """out[t] = sum_j w[t, j] * rotated-back S2F6 row pos[t, j]; bf16 [T, D]."""
+    T, k = pos.shape
+    D = codes.shape[1]
+    if out is None:
+        out = torch.empty(T, D, dtype=torch.bfloat16, device=codes.device)
+    L.call("moe_combine_s2f6", _p(codes), _p(e8m0), _p(pos), _p(w), T, k, D, seed, stream_id, _p(out), _s())
     return out

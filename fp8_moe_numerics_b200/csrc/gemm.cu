@@ -35,6 +35,7 @@ __device__ unsigned int g_mx_status_word = 0;
 namespace {
 
 constexpr int kKindNVFP4 = 0, kKindMXFP8 = 1;
+constexpr int kOutTypeF32 = 0, kOutTypeBF16 = 1, kOutTypeS2F6 = 2;   // epilogue output
 constexpr int kModeRows = 0, kModeWgrad = 1;
 constexpr int kBM = 128;
 constexpr int kStageBytesK = 128;       // bytes of K per stage (one 128B swizzle atom)
@@ -53,6 +54,8 @@ struct GemmArgs {
     int64_t sfa_groups;       // scale-column groups (of 4) per 128-row group of A
     int64_t sfb_groups;       // same for B
     int64_t ldo;              // output row stride (elements)
+    uint8_t* e8m0_out;        // S2F6 output: one exponent per 32 outputs of a row
+    uint64_t seed, stream_id; // S2F6 output: key and stream of the rotation's signs
 };
 
 // ---------------------------------------------------------------------------
@@ -404,7 +407,7 @@ __device__ __forceinline__ Tile make_tile(const GemmArgs& p, int64_t idx, uint32
 // only two scale regions (a ring released by MMA commits, decoupled from the
 // shared-memory stages) to make that overlap small.
 constexpr int kSmemLimit = 227 * 1024;
-template <int kKind, int kBN, bool kPair, bool kOutBF16>
+template <int kKind, int kBN, bool kPair, int kOut>
 struct Smem {
     static constexpr int kA = kBM * kStageBytesK;                       // 16 KB
     static constexpr int kB = (kPair ? kBN / 2 : kBN) * kStageBytesK;
@@ -419,7 +422,9 @@ struct Smem {
     static constexpr int kSfbCols = 4 * kAtomsB;
     static constexpr int kSfRegion = kSfaCols + kSfbCols;
     static constexpr int kPfxBytes = kPair ? 4 * (kMaxPairExperts + 4) : 0;
-    static constexpr int kFixed = 512 + kPfxBytes + 1024;               // barriers + prefix + alignment slack
+    // S2F6: the rotation's signs (+-1.0f) of every output column, N <= 4096
+    static constexpr int kMaskWords = kOut == kOutTypeS2F6 ? 4096 : 0;
+    static constexpr int kFixed = 512 + kPfxBytes + 4 * kMaskWords + 1024;   // barriers + prefix + masks + slack
     static constexpr int stages_for(int staging) {
         for (int s = 6; s > 2; --s)
             if (s * kStage + staging + kFixed <= kSmemLimit) return s;
@@ -428,14 +433,16 @@ struct Smem {
     // Epilogue staging, 8 warps: fp32 boxes need 4 KB each; bf16 boxes are 2 KB
     // and get two buffers per warp unless giving up the second buys a
     // pipeline stage (operands in flight are what bound these kernels).
-    static constexpr bool kOneBox = kOutBF16 && stages_for(8 * 2048) > stages_for(8 * 4096);
-    static constexpr int kStaging = kOneBox ? 8 * 2048 : 8 * 4096;
+    static constexpr bool kOneBox = kOut == kOutTypeBF16 && stages_for(8 * 2048) > stages_for(8 * 4096);
+    // S2F6 boxes are 32 rows x 32 bytes: two 1 KB buffers per warp.
+    static constexpr int kStaging = kOut == kOutTypeS2F6 ? 8 * 2048 : (kOneBox ? 8 * 2048 : 8 * 4096);
     static constexpr int kStages = stages_for(kStaging);
     static constexpr int kStagingOff = kStages * kStage;
     static_assert(kStage % 1024 == 0 && kStagingOff % 1024 == 0, "128-byte swizzle needs 1024-byte aligned tiles");
     static constexpr int kBarOff = kStagingOff + kStaging;
     static constexpr int kPfxOff = kBarOff + 512;
-    static constexpr int kBytes = kPfxOff + kPfxBytes + 1024;
+    static constexpr int kMaskOff = kPfxOff + kPfxBytes;
+    static constexpr int kBytes = kMaskOff + 4 * kMaskWords + 1024;
     static_assert(kBytes <= kSmemLimit, "shared memory budget");
     // TMEM
     static constexpr int kSfSlots = (kPair && kKind == kKindNVFP4) ? 2 : kStages;
@@ -459,11 +466,11 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, unsig
     while (!mbar_try_wait(bar, parity) && globaltimer() - t0 < kWaitLimitNs) {}
 }
 
-template <int kKind, int kMode, int kBN, bool kOutBF16, bool kPair>
+template <int kKind, int kMode, int kBN, int kOut, bool kPair>
 __global__ void __launch_bounds__(kThreads, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmOut, const GemmArgs p) {
-    using L = Smem<kKind, kBN, kPair, kOutBF16>;
+    using L = Smem<kKind, kBN, kPair, kOut>;
     constexpr int kStages = L::kStages;
     constexpr int kSlots = L::kSfSlots;
     constexpr bool kSfRing = kSlots < kStages;                          // scale regions released by MMA commits
@@ -696,8 +703,36 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         const uint32_t acc_free_lead[2] = {kPair ? map_to_rank(&acc_free[0], 0) : 0u,
                                            kPair ? map_to_rank(&acc_free[1], 0) : 0u};
         uint32_t it = 0, nbox = 0;
+        // S2F6: the rotation's signs of every output column as +-1.0f, once per
+        // CTA (the eight epilogue warps fill the table, then meet on named
+        // barrier 1); wider outputs take each block's mask word instead
+        float* signs = reinterpret_cast<float*>(smem + L::kMaskOff);
+        const bool sign_table = kOut == kOutTypeS2F6 && p.ldo <= L::kMaskWords;
+        if (sign_table) {
+            for (int64_t j = threadIdx.x - 256; j < (p.ldo >> 5); j += 256) {
+                const uint32_t m = hadamard_sign_word(p.seed, p.stream_id, (uint64_t)j);
+#pragma unroll
+                for (int i = 0; i < 32; i += 4)
+                    *reinterpret_cast<float4*>(signs + 32 * j + i) =
+                        make_float4((m >> i) & 1 ? -1.0f : 1.0f, (m >> (i + 1)) & 1 ? -1.0f : 1.0f,
+                                    (m >> (i + 2)) & 1 ? -1.0f : 1.0f, (m >> (i + 3)) & 1 ? -1.0f : 1.0f);
+            }
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+        }
+        // NVFP4: each tile's outer scales (a per-row and a per-expert fp32) are
+        // loaded one tile ahead, so their latency overlaps the previous drain.
+        auto tile_scale = [&](const Tile& tt) -> float {
+            return (kKind == kKindNVFP4 && tt.store) ? __ldg(p.a_outer + tt.row0 + r) * __ldg(p.b_outer + tt.e) : 1.0f;
+        };
+        Tile t_next = make_tile<kKind, kMode, kBN, kPair>(p, first, rank, pfx);
+        float scale_next = tile_scale(t_next);
         for (int64_t idx = first; idx < total; idx += stride) {
-            const Tile t = make_tile<kKind, kMode, kBN, kPair>(p, idx, rank, pfx);
+            const Tile t = t_next;
+            const float scale = scale_next;
+            if (idx + stride < total) {
+                t_next = make_tile<kKind, kMode, kBN, kPair>(p, idx + stride, rank, pfx);
+                scale_next = tile_scale(t_next);
+            }
             const int b = (int)(it & 1);
             if (!mbar_wait(&acc_full[b], (it >> 1) & 1u, abort_flag)) break;
             tc_fence_after();
@@ -712,8 +747,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             if (!t.store) {
                 release();
             } else {
-                float scale = 1.0f;
-                if (kKind == kKindNVFP4) scale = __ldg(p.a_outer + t.row0 + r) * __ldg(p.b_outer + t.e);
                 const uint32_t tbase = tmem + (uint32_t)(b * L::kAccStride) + ((uint32_t)(q * 32) << 16);
                 const int oy = (int)(t.row0 + q * 32);
 #pragma unroll
@@ -734,10 +767,50 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                             for (int i = 0; i < 32; ++i) v[u][i] = 0.0f;
                     }
                     if (g == (kOv > 0 ? 0 : kChunks / 4 - 1)) release();
+                    if constexpr (kOut == kOutTypeS2F6) {
+                        // Each thread holds 32 consecutive outputs of its row: one
+                        // rotation block.  Scale, rotate and quantise it in registers,
+                        // stage the warp's 32 rows x 32 codes as one box (two 1 KB
+                        // buffers per warp) and write it with a TMA tensor store; the
+                        // exponent byte goes straight to global memory.
+                        const int64_t orow = t.row0 + r;
+#pragma unroll
+                        for (int u = 0; u < 2; ++u) {
+                            const int64_t ocol = t.col0 + col[u];
+                            uint32_t w[8];
+                            int e;
+                            if (sign_table) {
+                                e = s2f6_block_scaled(v[u], scale, signs + ocol, w);
+                            } else {
+#pragma unroll
+                                for (int i = 0; i < 32; ++i) v[u][i] = v[u][i] * scale;
+                                e = s2f6_block_mask(v[u], hadamard_sign_word(p.seed, p.stream_id, (uint64_t)(ocol >> 5)), w);
+                            }
+                            uint8_t* box = stg + (nbox & 1u) * 1024;
+                            if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+                            __syncwarp();
+                            const uint32_t row = smem_u32(box) + (uint32_t)lane * 32u;
+                            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                                         :: "r"(row), "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]) : "memory");
+                            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                                         :: "r"(row + 16u), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7]) : "memory");
+                            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                            __syncwarp();
+                            if (lane == 0) {
+                                asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];"
+                                             :: "l"(reinterpret_cast<uint64_t>(&tmOut)), "r"((int)ocol), "r"(oy),
+                                                "r"(smem_u32(box)) : "memory");
+                                asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                            }
+                            ++nbox;
+                            p.e8m0_out[orow * (p.ldo >> 5) + (ocol >> 5)] = (uint8_t)(e + 127);
+                        }
+                        continue;
+                    }
 #pragma unroll
                     for (int u = 0; u < 2; ++u) {
                         uint8_t* box;
-                        if (kOutBF16) {
+                        if (kOut == kOutTypeBF16) {
                             if (L::kOneBox) {
                                 box = stg;
                                 if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
@@ -853,6 +926,19 @@ int make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t inner, int 
 
 // Output [rows, cols] (row stride cols), box 32 x 32: bf16 with 64-byte rows
 // and 64-byte swizzle, fp32 with 128-byte rows and 128-byte swizzle.
+// S2F6 codes [rows, cols] int8, box 32 x 32 (32-byte rows, no swizzle).
+int make_s2f6_map(CUtensorMap* m, void* base, int64_t rows, int64_t cols) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return MX_EUNSUPPORTED;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols};
+    const cuuint32_t box[2] = {32, 32};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MX_OK : MX_EINVAL;
+}
+
 int make_out_map(CUtensorMap* m, void* base, int64_t rows, int64_t cols, bool bf16) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return MX_EUNSUPPORTED;
@@ -891,11 +977,11 @@ int max_pairs(Kern kern, const cudaLaunchConfig_t& cfg) {
     return clusters;
 }
 
-template <int kKind, int kMode, int kBN, bool kOutBF16, bool kPair>
+template <int kKind, int kMode, int kBN, int kOut, bool kPair>
 int launch(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mo, const GemmArgs& args, int64_t items,
            cudaStream_t stream) {
-    using L = Smem<kKind, kBN, kPair, kOutBF16>;
-    auto kern = grouped_gemm_kernel<kKind, kMode, kBN, kOutBF16, kPair>;
+    using L = Smem<kKind, kBN, kPair, kOut>;
+    auto kern = grouped_gemm_kernel<kKind, kMode, kBN, kOut, kPair>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes) != cudaSuccess)
         return mx_launch_status();
     cudaLaunchConfig_t cfg = {};
@@ -921,6 +1007,8 @@ int launch(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mo, 
     return mx_launch_status();
 }
 
+constexpr int kOutS2F6Dtype = -2;                      // internal out_dtype of grouped_gemm_nvfp4_s2f6
+
 // CTA pairs with 256 x 256 output tiles wherever the shape allows (measured
 // on B200: halving each CTA's B traffic per flop and the deeper pipeline it
 // buys lift the tensor pipe's duty cycle); otherwise single CTAs with 128 x
@@ -930,13 +1018,22 @@ int dispatch(bool pair, int64_t out_rows, int64_t out_cols, int out_dtype, const
              const CUtensorMap& mb, const GemmArgs& args, int64_t items_pair, int64_t items_single,
              cudaStream_t stream) {
     CUtensorMap mo;
+    if (out_dtype == kOutS2F6Dtype) {
+        if constexpr (kKind == kKindNVFP4 && kMode == kModeRows) {
+            if (int st = make_s2f6_map(&mo, args.out, out_rows, out_cols)) return st;
+            return pair ? launch<kKind, kMode, 256, kOutTypeS2F6, true>(ma, mb, mo, args, items_pair, stream)
+                        : launch<kKind, kMode, 128, kOutTypeS2F6, false>(ma, mb, mo, args, items_single, stream);
+        } else {
+            return MX_EINVAL;
+        }
+    }
     const bool bf16 = out_dtype == MX_OUT_BF16;
     if (int st = make_out_map(&mo, args.out, out_rows, out_cols, bf16)) return st;
     if (pair)
-        return bf16 ? launch<kKind, kMode, 256, true, true>(ma, mb, mo, args, items_pair, stream)
-                    : launch<kKind, kMode, 256, false, true>(ma, mb, mo, args, items_pair, stream);
-    return bf16 ? launch<kKind, kMode, 128, true, false>(ma, mb, mo, args, items_single, stream)
-                : launch<kKind, kMode, 128, false, false>(ma, mb, mo, args, items_single, stream);
+        return bf16 ? launch<kKind, kMode, 256, kOutTypeBF16, true>(ma, mb, mo, args, items_pair, stream)
+                    : launch<kKind, kMode, 256, kOutTypeF32, true>(ma, mb, mo, args, items_pair, stream);
+    return bf16 ? launch<kKind, kMode, 128, kOutTypeBF16, false>(ma, mb, mo, args, items_single, stream)
+                : launch<kKind, kMode, 128, kOutTypeF32, false>(ma, mb, mo, args, items_single, stream);
 }
 
 }  // namespace
@@ -982,6 +1079,32 @@ extern "C" int grouped_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_sf, c
     a.sfa_groups = K / 64; a.sfb_groups = K / 64; a.ldo = N;
     return dispatch<kKindNVFP4, kModeRows>(N % 256 == 0 && E <= kMaxPairExperts, M_cap, N, out_dtype, ma, mb, a, (M_cap / kBM) * (N / 256),
                                            (M_cap / kBM) * (N / 128), stream);
+}
+
+extern "C" int grouped_gemm_nvfp4_s2f6(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_outer,
+                                       const uint8_t* b_codes, const uint8_t* b_sf, const float* b_outer,
+                                       const int64_t* seg_offsets, int64_t E, int64_t M_cap, int64_t N, int64_t K,
+                                       uint64_t seed, uint64_t stream_id, int8_t* codes, uint8_t* e8m0,
+                                       cudaStream_t stream) {
+    if (((!a_codes || !a_sf || !a_outer || !b_codes || !b_sf || !b_outer || !seg_offsets || !codes || !e8m0) &&
+         M_cap > 0) || E < 1 || M_cap < 0 || M_cap % 128 || N <= 0 || N % 128 || K <= 0 || K % 256)
+        return MX_EINVAL;
+    if (!mx_aligned(a_codes, 16) || !mx_aligned(b_codes, 16) || !mx_aligned(a_sf, 16) || !mx_aligned(b_sf, 16) ||
+        !mx_aligned(codes, 16))
+        return MX_EINVAL;
+    if (M_cap >= (int64_t)1 << 31 || E * N >= (int64_t)1 << 31 || K / 2 >= (int64_t)1 << 31) return MX_EINVAL;
+    if (int st = mx_check_device()) return st;
+    if (M_cap == 0) return MX_OK;
+    CUtensorMap ma, mb;
+    if (int st = make_map(&ma, a_codes, M_cap, K / 2, kBM)) return st;
+    if (int st = make_map(&mb, b_codes, E * N, K / 2, 128)) return st;
+    GemmArgs a{};
+    a.sfa = a_sf; a.sfb = b_sf; a.a_outer = a_outer; a.b_outer = b_outer; a.seg = seg_offsets; a.out = codes;
+    a.E = E; a.M_cap = M_cap; a.N = N; a.K = K;
+    a.sfa_groups = K / 64; a.sfb_groups = K / 64; a.ldo = N;
+    a.e8m0_out = e8m0; a.seed = seed; a.stream_id = stream_id;
+    return dispatch<kKindNVFP4, kModeRows>(N % 256 == 0 && E <= kMaxPairExperts, M_cap, N, kOutS2F6Dtype, ma, mb, a,
+                                           (M_cap / kBM) * (N / 256), (M_cap / kBM) * (N / 128), stream);
 }
 
 extern "C" int grouped_gemm_mxfp8(int mode, const uint8_t* a_codes, const uint8_t* a_e8m0, const uint8_t* b_codes,

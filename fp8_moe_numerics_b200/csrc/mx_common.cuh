@@ -263,3 +263,185 @@ __device__ __forceinline__ int64_t load_rows_valid(const int64_t* rows_valid, in
     int64_t v = *rows_valid;
     return v < rows ? v : rows;
 }
+
+// ---------------------------------------------------------------------------
+// Combine path ([ai-primer §Quantized NVLink and BBBK]): expert outputs are
+// rotated by a 32-dimensional random Hadamard transform and quantised to
+// block-scaled S2F6, eight-bit fixed point with two signed integer bits and
+// six fractional bits.  Per 32-column block j of a row: z = H32 (sigma_j x),
+// H32 the unnormalised Sylvester matrix, sigma_j flipping coordinate i when
+// bit i of hadamard_sign_word(j) is set; one E8M0 exponent e per block (the
+// smallest with amax|z| <= (127/64) 2^e, in [-127, 127]); int8 codes
+// c = RNE(z 2^(6-e)) in [-127, 127].  The inverse is x = sigma_j (H32 z) / 32.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t hadamard_sign_word(uint64_t seed, uint64_t stream, uint64_t j) {
+    return philox4x32_10(j, stream, seed).x;
+}
+
+// Two fp32 lanes in one 64-bit register, for sm_100a's packed f32x2
+// arithmetic: each lane of add/sub/mul/fma .rn.f32x2 is one IEEE
+// round-to-nearest operation, so a packed op gives the two scalar results.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t r, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r));
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+
+// Smallest integer e with amax <= (127/64) 2^e, clamped to [-127, 127]
+// (-127 for amax == 0); amax finite and >= 0.  A subnormal amax is first
+// scaled by 2^64 (exact) so its exponent field is meaningful.
+__device__ __forceinline__ int s2f6_exponent(float amax) {
+    if (amax == 0.0f) return -127;
+    int adj = 0;
+    if (amax < 1.17549435e-38f) {
+        amax = __fmul_rn(amax, 18446744073709551616.0f);
+        adj = 64;
+    }
+    const uint32_t b = __float_as_uint(amax);
+    int e = (int)(b >> 23) - 127 - adj;
+    if ((b & 0x7fffffu) > 0x7e0000u) ++e;               // significand above 127/64 = 1.111111b
+    return e < -127 ? -127 : (e > 127 ? 127 : e);
+}
+
+// Codes of one block from its rotated values in pairs P[q] = (z_2q, z_2q+1):
+// c_i = RNE(z_i 2^(6-e)) clamped to [-127, 127], packed four per word (code i
+// in byte i%4 of word i/4, two's complement).  One fma adds 1.5 * 2^23 to the
+// exactly scaled value, so the sum rounds once to the nearest integer (ties
+// to even) and its low byte is the code.  kClamp: e == 127, where 127.99..
+// can occur; kTiny: 2^(6-e) is not finite in fp32, so 2^64 of it is applied
+// first (exactly).
+template <bool kClamp, bool kTiny>
+__device__ __forceinline__ void s2f6_codes_pairs(const uint64_t* P, float scale, uint32_t* words) {
+    const float magic = 12582912.0f;
+    const uint64_t S2 = f2_pack(scale, scale), M2 = f2_pack(magic, magic);
+    const uint64_t T2 = f2_pack(18446744073709551616.0f, 18446744073709551616.0f);
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+        float y[4];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const uint64_t z = kTiny ? f2_mul(P[2 * w + h], T2) : P[2 * w + h];
+            f2_unpack(f2_fma(z, S2, M2), y[2 * h], y[2 * h + 1]);
+        }
+        uint32_t b[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            if (kClamp) y[i] = fminf(fmaxf(y[i], magic - 127.0f), magic + 127.0f);
+            b[i] = __float_as_uint(y[i]);
+        }
+        words[w] = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
+    }
+}
+
+// Stages 2..16 of the rotation on pairs P[q] = (z_2q, z_2q+1) -- stage h
+// pairs element i with i + h, i.e. pair q with pair q + h/2 -- then the
+// block's exponent and codes.  Returns e.
+__device__ __forceinline__ int s2f6_finish(uint64_t* P, uint32_t* words) {
+#pragma unroll
+    for (int h2 = 1; h2 < 16; h2 <<= 1) {
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+            if ((q & h2) == 0) {
+                const uint64_t a = P[q], b = P[q + h2];
+                P[q] = f2_add(a, b);
+                P[q + h2] = f2_sub(a, b);
+            }
+        }
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+        float a, b;
+        f2_unpack(P[q], a, b);
+        amax = fmaxf(amax, fmaxf(fabsf(a), fabsf(b)));
+    }
+    const int e = s2f6_exponent(amax);
+    const int sh = 6 - e;                               // in [-121, 133]
+    if (sh > 126) s2f6_codes_pairs<false, true>(P, __uint_as_float((uint32_t)(sh - 64 + 127) << 23), words);
+    else if (e == 127) s2f6_codes_pairs<true, false>(P, __uint_as_float((uint32_t)(sh + 127) << 23), words);
+    else s2f6_codes_pairs<false, false>(P, __uint_as_float((uint32_t)(sh + 127) << 23), words);
+    return e;
+}
+
+// One 32-value block v (fp32, unrotated): negated where bit i of `mask` is
+// set, rotated by H32 (stage h = 1 on scalars into pairs, stages 2..16 on
+// pairs -- the same adds in the same order as one scalar butterfly network),
+// then its exponent and codes.  Returns e.
+__device__ __forceinline__ int s2f6_block_mask(const float* v, uint32_t mask, uint32_t* words) {
+    uint64_t P[16];
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+        const float a = __uint_as_float(__float_as_uint(v[2 * q]) ^ ((mask << (31 - 2 * q)) & 0x80000000u));
+        const float b = __uint_as_float(__float_as_uint(v[2 * q + 1]) ^ ((mask << (30 - 2 * q)) & 0x80000000u));
+        P[q] = f2_pack(__fadd_rn(a, b), __fsub_rn(a, b));
+    }
+    return s2f6_finish(P, words);
+}
+
+// The same block with v first multiplied by `scale`, the signs given as a
+// table sig[i] = +-1.0f (16-byte aligned): x_i = v_i (sig_i scale), which is
+// sig_i RN(v_i scale) exactly.
+__device__ __forceinline__ int s2f6_block_scaled(const float* v, float scale, const float* sig, uint32_t* words) {
+    const uint64_t S2 = f2_pack(scale, scale);
+    uint64_t P[16];
+#pragma unroll
+    for (int q4 = 0; q4 < 8; ++q4) {
+        const float4 sg = *reinterpret_cast<const float4*>(sig + 4 * q4);
+        const uint64_t s01 = f2_mul(f2_pack(sg.x, sg.y), S2), s23 = f2_mul(f2_pack(sg.z, sg.w), S2);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int q = 2 * q4 + h;
+            float a, b;
+            f2_unpack(f2_mul(f2_pack(v[2 * q], v[2 * q + 1]), h ? s23 : s01), a, b);
+            P[q] = f2_pack(__fadd_rn(a, b), __fsub_rn(a, b));
+        }
+    }
+    return s2f6_finish(P, words);
+}
+
+// Scalar forms, used where no pairs are at hand (the combine's inverse).
+// Negate v[i] where bit i of `mask` is set (exact).
+__device__ __forceinline__ void apply_signs32(float* v, uint32_t mask) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(__float_as_uint(v[i]) ^ ((mask << (31 - i)) & 0x80000000u));
+}
+
+// Unnormalised Walsh-Hadamard transform of 32 values in registers: stages
+// h = 1, 2, 4, 8, 16, each pair (i, i + h) with i & h == 0 becoming
+// (a + b, a - b), one fp32 round-to-nearest add each.
+__device__ __forceinline__ void fwht32(float* v) {
+#pragma unroll
+    for (int h = 1; h < 32; h <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            if ((i & h) == 0) {
+                const float a = v[i], b = v[i + h];
+                v[i] = __fadd_rn(a, b);
+                v[i + h] = __fsub_rn(a, b);
+            }
+        }
+    }
+}

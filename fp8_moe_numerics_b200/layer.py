@@ -7,7 +7,10 @@ across transposes):
   forward   route -> NVFP4 quantise tokens (per-token outer scale) -> gather
             into expert order -> NVFP4 quantise W1, W2 (per-expert outer
             scale) -> grouped NVFP4 GEMM1 -> SwiGLU -> NVFP4 quantise ->
-            grouped NVFP4 GEMM2 -> combine
+            grouped NVFP4 GEMM2 -> combine (with combine="s2f6", GEMM2's epilogue
+            rotates each 32-column block by a random Hadamard transform and
+            writes block-scaled S2F6, and the combine reads that:
+            [ai-primer §Quantized NVLink and BBBK])
   backward  combine gradient -> MXFP8 quantise dY2 (row- and column-wise) ->
             requantise W2 and the saved activations (dequantise, transpose,
             MXFP8 with stochastic rounding) -> MXFP8 dgrad / wgrad GEMMs ->
@@ -35,11 +38,17 @@ class ExpertLayer:
 
     x [T, D] bf16, topk [T, k] int32, w_comb [T, k] f32, w1 [E, 2F or F, D]
     bf16, w2 [E, D, F] bf16, dout [T, D] bf16, all on one CUDA device.
-    `wgrad_dtype` is the dtype of dW1 / dW2 (bf16 or fp32).
+    `wgrad_dtype` is the dtype of dW1 / dW2 (bf16 or fp32).  `combine` is
+    "bf16" (GEMM2 writes bf16 rows) or "s2f6" (GEMM2 writes rotated S2F6 rows,
+    one byte per value plus one exponent per 32).
     """
 
+    S2F6_STREAM = 101                                   # Philox stream of the rotation's signs
+
     def __init__(self, x, topk, w_comb, w1, w2, dout, gated: bool = True, seed: int = 0,
-                 wgrad_dtype=torch.bfloat16, out_dtype=torch.bfloat16, rbits: int = 16):
+                 wgrad_dtype=torch.bfloat16, out_dtype=torch.bfloat16, rbits: int = 16, combine: str = "bf16"):
+        assert combine in ("bf16", "s2f6")
+        self.combine = combine
         dev = x.device
         self.dev = dev
         self.T, self.D = x.shape
@@ -68,7 +77,10 @@ class ExpertLayer:
         self.h1 = e(M, N1, dt=out_dtype)
         self.a = e(M, F, dt=torch.bfloat16)
         self.aq = (e(M, F // 2), e(sfb(M, F, 16, MX_SF_MMA)), e(M, dt=torch.float32))
-        self.y2 = e(M, D, dt=out_dtype)
+        if combine == "s2f6":
+            self.y2s = (e(M, D, dt=torch.int8), e(M, D // 32))
+        else:
+            self.y2 = e(M, D, dt=out_dtype)
         self.out = e(T, D, dt=torch.bfloat16)
         # backward
         self.dy2 = e(M, D, dt=torch.bfloat16)
@@ -130,9 +142,15 @@ class ExpertLayer:
         self._mark("swiglu", record)
         api.nvfp4_quantize(self.a, 1, MX_SF_MMA, out=self.aq)
         self._mark("quant_a", record)
-        api.grouped_gemm_nvfp4(self.aq, self.w2q, self.seg, E, D, F, out=self.y2)
-        self._mark("gemm2", record)
-        api.moe_combine(self.y2, self.pos, self.w_comb, D, out=self.out)
+        if self.combine == "s2f6":
+            api.grouped_gemm_nvfp4_s2f6(self.aq, self.w2q, self.seg, E, D, F, self.seed, self.S2F6_STREAM,
+                                        out=self.y2s)
+            self._mark("gemm2", record)
+            api.moe_combine_s2f6(*self.y2s, self.pos, self.w_comb, self.seed, self.S2F6_STREAM, out=self.out)
+        else:
+            api.grouped_gemm_nvfp4(self.aq, self.w2q, self.seg, E, D, F, out=self.y2)
+            self._mark("gemm2", record)
+            api.moe_combine(self.y2, self.pos, self.w_comb, D, out=self.out)
         self._mark("combine", record)
         return self.out
 

@@ -276,6 +276,59 @@ MX_API int moe_combine(const void* y, const int32_t* pos, const float* w, int64_
 MX_API int moe_dispatch_grad(const void* dout, const int32_t* src, const int32_t* pos, const float* w, int64_t T,
                              int64_t k, int64_t M_cap, int64_t D, void* dy, cudaStream_t stream);
 
+/* --------------------------------------------------------------------------
+ * Combine path in S2F6.  [ai-primer §Quantized NVLink and BBBK]: expert
+ * outputs are rotated by a 32-dimensional random Hadamard transform and
+ * quantised into block-scaled S2F6 (eight-bit fixed point, two signed integer
+ * bits and six fractional bits) for the combine, the transform and the
+ * quantisation folded into the output GEMM's epilogue.  The pages give the
+ * format's bit split only; the readings taken here:
+ *   rotation  per 32-column block j of a row, z = H32 (sigma_j * x): H32 the
+ *             unnormalised Sylvester-Hadamard matrix (H[a][b] =
+ *             (-1)^popcount(a & b)), evaluated as five butterfly stages
+ *             h = 1, 2, 4, 8, 16 of fp32 adds (a, b) -> (a + b, a - b) on the
+ *             pairs (i, i + h), i & h == 0; sigma_j negates coordinate i when
+ *             bit i of word 0 of Philox4x32-10(counter (j lo, j hi, stream_id
+ *             lo, stream_id hi), key (seed lo, seed hi)) is set.  The inverse
+ *             is x = sigma_j * (H32 z) / 32.
+ *   scale     one E8M0 byte per block, e + 127 with e the smallest integer
+ *             such that max|z| <= (127/64) * 2^e, clamped to [-127, 127]
+ *             (-127 for a zero block).
+ *   codes     int8 c = round-half-even(z * 2^(6-e)) clamped to [-127, 127];
+ *             value c * 2^(e-6).
+ * Layout: codes int8 [rows, cols] row-major, exponents u8 [rows, cols/32]
+ * row-major.  Inputs finite.
+ * ------------------------------------------------------------------------ */
+
+/* hadamard_s2f6_quantize -- bf16 x [rows, cols] -> S2F6 codes and exponents
+ * (the unfused form: x holds bf16 expert outputs).  cols % 32 == 0, x and
+ * codes 16-byte aligned; else MX_EINVAL.  rows == 0 succeeds without touching
+ * memory. */
+MX_API int hadamard_s2f6_quantize(const void* x, int64_t rows, int64_t cols, uint64_t seed, uint64_t stream_id,
+                                  int8_t* codes, uint8_t* e8m0, cudaStream_t stream);
+
+/* grouped_gemm_nvfp4_s2f6 -- grouped_gemm_nvfp4 with the S2F6 epilogue: each
+ * output row's fp32 values (those the MX_OUT_F32 form would store) are rotated
+ * and quantised per 32-column block as above, in the registers that drain
+ * the accumulator.  Arguments and requirements as grouped_gemm_nvfp4, the
+ * output being codes int8 [M_cap, N] and e8m0 u8 [M_cap, N/32] (rows of
+ * padding hold codes of zero sums).  codes 16-byte aligned. */
+MX_API int grouped_gemm_nvfp4_s2f6(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_outer,
+                                   const uint8_t* b_codes, const uint8_t* b_sf, const float* b_outer,
+                                   const int64_t* seg_offsets, int64_t E, int64_t M_cap, int64_t N, int64_t K,
+                                   uint64_t seed, uint64_t stream_id, int8_t* codes, uint8_t* e8m0,
+                                   cudaStream_t stream);
+
+/* moe_combine_s2f6 -- moe_combine reading S2F6 rows: out[t] =
+ * sum_j w[t,j] * xhat(pos[t,j]), xhat the rotated-back dequantised row.  The
+ * sum is taken in the rotated domain (u = sum_j w_j 2^(e_j - 6) c_j, fp32,
+ * j in order) and rotated back once per token block; bf16 round-to-nearest
+ * output [T, D].  w NULL: all weights 1.  D % 32 == 0, codes and out 16-byte
+ * aligned; else MX_EINVAL. */
+MX_API int moe_combine_s2f6(const int8_t* codes, const uint8_t* e8m0, const int32_t* pos, const float* w,
+                            int64_t T, int64_t k, int64_t D, uint64_t seed, uint64_t stream_id, void* out,
+                            cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

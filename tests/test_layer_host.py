@@ -48,3 +48,18 @@ def test_layer_sequence_passes_host_validation(host_calls, name):
     assert names.count("mxfp8_requant_transpose_sr") == 4
     assert len(names) == 23
     assert all(st == _lib.MX_ECUDA for _, st in host_calls)   # valid, and no device here
+
+
+def test_s2f6_combine_sequence_passes_host_validation(host_calls):
+    inp = workloads.layer_inputs("tiny_layer", device="cpu")
+    c = inp["cfg"]
+    L = ExpertLayer(inp["x"], inp["topk"], inp["w_comb"], inp["w1"], inp["w2"], inp["dout"], gated=c["gated"],
+                    combine="s2f6")
+    L.step()
+    names = [n for n, _ in host_calls]
+    assert names.count("grouped_gemm_nvfp4") == 1 and names.count("grouped_gemm_nvfp4_s2f6") == 1
+    # the forward combine reads S2F6; the backward's un-permute of dX stays a bf16 combine
+    assert names.count("moe_combine_s2f6") == 1 and names.count("moe_combine") == 1
+    assert names.index("moe_combine_s2f6") == names.index("grouped_gemm_nvfp4_s2f6") + 1
+    assert len(names) == 23
+    assert all(st == _lib.MX_ECUDA for _, st in host_calls)

@@ -9,14 +9,15 @@ Sylvester matrix, H32 H32 = 32 I, a search over every exponent, hand-written
 tie cases, the closed form of a one-hot block, the quantisation error bound
 and a per-element loop over the combine.
 """
-
 import numpy as np
 import pytest
 
 import oracle
 
+
 def _popcount_hadamard(n):
     return np.array([[(-1.0) ** bin(a & b).count("1") for b in range(n)] for a in range(n)])
+
 
 def test_butterflies_equal_the_sylvester_matrix_on_integers():
     rng = np.random.default_rng(0)
@@ -25,10 +26,12 @@ def test_butterflies_equal_the_sylvester_matrix_on_integers():
     assert np.array_equal(oracle.sylvester_hadamard(32), H)
     assert np.array_equal(oracle.fwht32_f32(x).astype(np.float64), x.astype(np.float64) @ H.T)
 
+
 def test_transform_applied_twice_is_32_times_identity():
     rng = np.random.default_rng(1)
     x = rng.integers(-300, 301, size=(20, 32)).astype(np.float32)
     assert np.array_equal(oracle.fwht32_f32(oracle.fwht32_f32(x)), 32.0 * x)
+
 
 def test_sign_masks_are_balanced_and_keyed():
     w = oracle.hadamard_sign_words(7, 3, 512)
@@ -41,6 +44,7 @@ def test_sign_masks_are_balanced_and_keyed():
     assert set(np.unique(s)) <= {-1.0, 1.0} and s.shape == (64,)
     assert s[0] == (-1.0 if w[0] & 1 else 1.0) and s[33] == (-1.0 if (w[1] >> 1) & 1 else 1.0)
 
+
 def _exponent_by_search(amax):
     if amax == 0.0:
         return -127
@@ -49,16 +53,21 @@ def _exponent_by_search(amax):
             return e
     return 127
 
+
 @pytest.mark.parametrize("amax", [0.0, 1.0, 127 / 64, np.nextafter(np.float32(127 / 64), np.float32(2)), 2.0, 1.9,
                                   3.0, 127 / 32, 0.75, 1e-30, 1e-40, 2.0 ** -149, 2.0 ** -126, 1e20, 3.0e38,
                                   float(np.finfo(np.float32).max)])
+
+
 def test_exponent_is_the_smallest_that_fits(amax):
     assert oracle.s2f6_exponent(float(np.float32(amax))) == _exponent_by_search(float(np.float32(amax)))
+
 
 def test_exponent_on_random_magnitudes():
     rng = np.random.default_rng(2)
     for a in (rng.standard_normal(2000) * 10.0 ** rng.uniform(-40, 38, 2000)).astype(np.float32):
         assert oracle.s2f6_exponent(abs(float(a))) == _exponent_by_search(abs(float(a)))
+
 
 def _block_with_rotated_values(z, seed, stream):
     """fp32 x (one block) whose rotation is exactly z (z dyadic, small)."""
@@ -66,6 +75,7 @@ def _block_with_rotated_values(z, seed, stream):
     x = (oracle.sylvester_hadamard(32) @ np.asarray(z, np.float64)) / 32.0 * sig
     assert np.array_equal(x.astype(np.float32).astype(np.float64), x)
     return x.astype(np.float32)[None, :]
+
 
 def test_codes_round_half_to_even():
     # amax 127/64 gives e = 0, so a code is z * 64; half codes are ties
@@ -82,6 +92,7 @@ def test_codes_round_half_to_even():
     assert c[0, 1:1 + len(halves)].tolist() == expect
     assert np.all(c[0, 1 + len(halves):] == 0)
 
+
 def test_one_hot_outlier_spreads_to_every_coordinate():
     # a single value A in a block rotates to +-A in all 32 coordinates
     for A in (1.0, 3.0, 1000.0, 7.3e-5):
@@ -94,6 +105,7 @@ def test_one_hot_outlier_spreads_to_every_coordinate():
         assert np.all(np.abs(c[0, 32:].astype(np.float64)) == mag)
         assert np.all(c[0, :32] == 0)
 
+
 def test_top_exponent_saturates_codes():
     # a one-hot block of the largest fp32 value rotates to |z| = (2 - 2^-23) 2^127
     # in every coordinate: e would be 128, clamps to 127, and 127.99... -> 127
@@ -102,6 +114,7 @@ def test_top_exponent_saturates_codes():
     c, e = oracle.s2f6_quantize_hadamard(x, 0, 0)
     assert e[0, 0] == 127 + 127
     assert np.all(np.abs(c.astype(np.int64)) == 127)
+
 
 def test_reconstruction_error_bound():
     rng = np.random.default_rng(3)
@@ -118,6 +131,7 @@ def test_reconstruction_error_bound():
     # the inverse divides the 2-norm by sqrt(32); fp32 butterflies add < 1e-6
     assert np.all(err <= step_half + 1e-6 * nrm)
     assert np.all(xh[9] == 0)
+
 
 def test_combine_matches_element_loops():
     rng = np.random.default_rng(4)
