@@ -61,37 +61,6 @@ struct GemmArgs {
 // ---------------------------------------------------------------------------
 // PTX wrappers
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(smem_u32(bar)), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(smem_u32(bar)), "r"(bytes) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(smem_u32(bar)) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile("{\n\t.reg .pred p;\n\t"
-                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-                 "selp.u32 %0, 1, 0, p;\n\t}"
-                 : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
-    return ok != 0;
-}
-
-__device__ __forceinline__ unsigned long long globaltimer() {
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-    return t;
-}
-
 // Bounded wait: false (and the abort flag / status word set) on expiry or when
 // another role of this CTA has already aborted.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
@@ -1046,6 +1015,42 @@ extern "C" int mx_sync_status(cudaStream_t stream) {
     if (word && (e = cudaMemcpyToSymbol(g_mx_status_word, &zero, sizeof(zero))) != cudaSuccess)
         return mx_set_cuda_error(e);
     return word ? MX_ETIMEOUT : MX_OK;
+}
+
+// Device address of the status word on the current device, looked up once per
+// device; kernels in other translation units take it as an argument.
+static std::mutex g_status_addr_mutex;
+static unsigned int* g_status_addr[64] = {nullptr};
+
+int mx_status_word_address(unsigned int** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return mx_set_cuda_error(e);
+    if (dev < 0 || dev >= 64) return MX_EUNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_status_addr_mutex);
+    if (!g_status_addr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_mx_status_word);
+        if (e != cudaSuccess || !p) return mx_set_cuda_error(e != cudaSuccess ? e : cudaErrorInvalidSymbol);
+        g_status_addr[dev] = static_cast<unsigned int*>(p);
+    }
+    *out = g_status_addr[dev];
+    return MX_OK;
+}
+
+// bf16 [rows, cols] (row stride cols), box box_rows x box_cols, 128-byte swizzle
+// (box_cols * 2 == 128).
+int mx_make_bf16_tile_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_cols, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return MX_EUNSUPPORTED;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MX_OK : MX_EINVAL;
 }
 
 extern "C" int mx_wait_selftest(int64_t limit_us, cudaStream_t stream) {

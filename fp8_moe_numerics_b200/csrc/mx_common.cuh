@@ -23,8 +23,53 @@ int mx_set_cuda_error(cudaError_t e);   // records e, returns MX_ECUDA
 int mx_check_device(void);              // MX_OK on sm_100, else MX_EUNSUPPORTED / MX_ECUDA
 int mx_launch_status(void);             // cudaGetLastError -> MX_OK / MX_ECUDA
 void mx_count_launch(void);             // one more kernel launched by this library (mx_kernel_launches)
+int mx_status_word_address(unsigned int** out);   // device address of the bounded-wait status word
+struct CUtensorMap_st;
+int mx_make_bf16_tile_map(struct CUtensorMap_st* m, const void* base, int64_t rows, int64_t cols, int box_cols,
+                          int box_rows);             // bf16 [rows, cols] TMA map, 128-byte swizzle
 
 static inline bool mx_aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// ---------------------------------------------------------------------------
+// Shared-memory addresses, mbarriers and the GPU clock
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ unsigned long long globaltimer() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Nanosecond wall clock of the GPU (bounded waits measure their limit on it).
+__device__ __forceinline__ unsigned long long mx_globaltimer() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
 
 // ---------------------------------------------------------------------------
 // Scale-factor layouts

@@ -6,6 +6,8 @@
 // cvt or by exact integer arithmetic (see mx_common.cuh).
 #include "mx_common.cuh"
 
+#include <cuda.h>
+
 namespace {
 
 // Max of |bf16| over the 8 elements of a uint4, as the bf16 magnitude bits
@@ -381,6 +383,187 @@ mxfp8_tile_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, co
 }
 
 
+// ---------------------------------------------------------------------------
+// MXFP8 quantiser (RNE), fed by TMA.  A persistent block of 8 consumer warps
+// and one producer warp walks the same 128 x 64 tiles as mxfp8_tile_kernel.
+// The producer's lane 0 keeps kQStages bf16 tiles in flight with 2-D TMA
+// loads (128-byte swizzle) into a ring of shared-memory stages, so the
+// consumers never wait on a global load of their own.  Per tile:
+//   phase 1  thread (row t/2, half t%2) reads its 64 bytes of the row from the
+//            stage, releases the stage, quantises them row-wise, and stores the
+//            16 words (pairs of columns) into the transposed tile T2.
+//   phase 2  after one barrier of the consumer warps, thread (column pair
+//            t/8, row group t%8) reads 16 rows x 2 columns of T2 and emits two
+//            16-row halves of column-wise MXFP8 blocks (lanes g, g^1 form one
+//            32-row block).
+// T2 is double-buffered, so the next tile's phase 1 needs no second barrier:
+// a warp still in phase 2 of tile i reads the other buffer, and phase 1 of
+// tile i+2 comes after every warp has passed tile i+1's barrier.  T2 holds
+// word (cp, r) = columns 2cp, 2cp+1 of row r; column pairs 16..31 flip row
+// bit 4 and every 4-word chunk index is XOR-ed with row/32, which keeps the
+// phase-1 stores and the phase-2 16-byte loads free of bank conflicts.
+// Waits are bounded (2 s): on expiry the status word records a timeout and
+// the block stops.
+// ---------------------------------------------------------------------------
+#ifndef MX_Q_STAGES
+#define MX_Q_STAGES 4          // bf16 tiles in flight per block
+#endif
+#ifndef MX_Q_MIN_BLOCKS
+#define MX_Q_MIN_BLOCKS 2      // co-resident blocks per SM (bounds the registers)
+#endif
+constexpr int kQStages = MX_Q_STAGES;
+constexpr int kQTileBytes = kTR * kTC * 2;                  // 16 KB of bf16
+constexpr int kQThreads = kTileThreads + 32;
+constexpr int kQSmemBytes = kQStages * kQTileBytes + 2 * kQTileBytes + 256 + 1024;
+constexpr unsigned long long kQWaitLimitNs = 2ull * 1000ull * 1000ull * 1000ull;
+
+__device__ __forceinline__ int t2_word(int cp, int r) {
+    int rr = r ^ ((cp >> 4) << 4);
+    rr ^= ((rr >> 5) & 3) << 2;
+    return cp * kTR + rr;
+}
+
+__device__ __forceinline__ bool q_wait(uint64_t* bar, uint32_t parity, volatile int* abort, unsigned int* status) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = mx_globaltimer();
+    while (!mbar_try_wait(bar, parity)) {
+        if (*abort) return false;
+        if (mx_globaltimer() - t0 > kQWaitLimitNs) {
+            *abort = 1;
+            atomicOr(status, 1u);
+            return false;
+        }
+    }
+    return true;
+}
+
+template <bool kRow, bool kCol, int kLayout>
+__global__ void __launch_bounds__(kQThreads, MX_Q_MIN_BLOCKS)
+mxfp8_tile_tma_kernel(const __grid_constant__ CUtensorMap tmX, int64_t rows, int64_t cols, const int64_t* rows_valid,
+                      uint8_t* __restrict__ row_codes, uint8_t* __restrict__ row_e8m0, uint8_t* __restrict__ col_codes,
+                      uint8_t* __restrict__ col_e8m0, unsigned int* status) {
+    extern __shared__ uint8_t q_smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(q_smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* stages = smem;                                              // SW128 tiles: 1024-byte aligned
+    uint32_t* T2 = reinterpret_cast<uint32_t*>(smem + kQStages * kQTileBytes);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kQStages * kQTileBytes + 2 * kQTileBytes);
+    uint64_t* empty = full + kQStages;
+    volatile int* abort = reinterpret_cast<volatile int*>(empty + kQStages);
+    volatile int* stop = abort + 1;                                      // [2], by tile parity
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t tiles_c = cols / kTC;
+    const int64_t ntiles = tiles_c * ((load_rows_valid(rows_valid, rows) + kTR - 1) / kTR);
+    if ((int64_t)blockIdx.x >= ntiles) return;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kQStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], kTileThreads / 32); }
+        *abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(&tmX)) : "memory");
+    }
+    __syncthreads();
+
+    if (warp == kTileThreads / 32) {                                     // producer
+        if (lane == 0) {
+            uint32_t it = 0;
+            for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+                const int s = (int)(it % kQStages);
+                if (!q_wait(&empty[s], ((it / kQStages) & 1) ^ 1, abort, status)) break;
+                mbar_expect_tx(&full[s], kQTileBytes);
+                const int c0 = (int)((tile % tiles_c) * kTC), r0 = (int)((tile / tiles_c) * kTR);
+                asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+                             " [%0], [%1, {%2, %3}], [%4];"
+                             :: "r"(smem_u32(stages + s * kQTileBytes)), "l"(reinterpret_cast<uint64_t>(&tmX)),
+                                "r"(c0), "r"(r0), "r"(smem_u32(&full[s])) : "memory");
+            }
+            // every issued copy lands before the block exits
+            const unsigned long long t0 = mx_globaltimer();
+            for (uint32_t k = it > kQStages ? it - kQStages : 0; k < it; ++k)
+                while (!mbar_try_wait(&full[k % kQStages], (k / kQStages) & 1) &&
+                       mx_globaltimer() - t0 < kQWaitLimitNs) {}
+        }
+        return;
+    }
+
+    const int t = threadIdx.x;
+    const int rl = t >> 1, h = t & 1;
+    const int cp = t >> 3, g = t & 7;
+    uint32_t it = 0;
+    int buf = 0;
+    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+        const int s = (int)(it % kQStages);
+        // on a failed wait the warps still meet at this tile's barrier (a warp
+        // leaving early would strand the others there) and stop after it
+        const bool ok = q_wait(&full[s], (it / kQStages) & 1, abort, status);
+        if (!kCol && !ok) break;
+        const int64_t c0 = (tile % tiles_c) * kTC, r0 = (tile / tiles_c) * kTR;
+        const uint8_t* st = stages + s * kQTileBytes + rl * 128;
+        uint4 q[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) q[i] = *reinterpret_cast<const uint4*>(st + (((4 * h + i) ^ (rl & 7)) << 4));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+        if (kRow) {
+            const int64_t r = r0 + rl;
+            uint32_t m = 0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) m = max(m, absmax8_bf16(q[i]));
+            const int e = e8m0_exponent(__uint_as_float(m << 16));
+            const float sc = exp2_neg(e);
+            uint32_t w[8];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                w[2 * i] = cvt_e4m3x4(__fmul_rn(bf16_lo(q[i].x), sc), __fmul_rn(bf16_hi(q[i].x), sc),
+                                      __fmul_rn(bf16_lo(q[i].y), sc), __fmul_rn(bf16_hi(q[i].y), sc));
+                w[2 * i + 1] = cvt_e4m3x4(__fmul_rn(bf16_lo(q[i].z), sc), __fmul_rn(bf16_hi(q[i].z), sc),
+                                          __fmul_rn(bf16_lo(q[i].w), sc), __fmul_rn(bf16_hi(q[i].w), sc));
+            }
+            uint4* dst = reinterpret_cast<uint4*>(row_codes + r * cols + c0 + 32 * h);
+            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+            dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+            row_e8m0[sf_offset(r, (c0 >> 5) + h, cols >> 5, kLayout)] = (uint8_t)(e + 127);
+        }
+        if (kCol) {
+            uint32_t* Tb = T2 + buf * (kTC / 2) * kTR;
+            const uint32_t wq[16] = {q[0].x, q[0].y, q[0].z, q[0].w, q[1].x, q[1].y, q[1].z, q[1].w,
+                                     q[2].x, q[2].y, q[2].z, q[2].w, q[3].x, q[3].y, q[3].z, q[3].w};
+#pragma unroll
+            for (int j = 0; j < 16; ++j) Tb[t2_word(16 * h + j, rl)] = wq[j];
+            if (t == 0) stop[it & 1] = *abort;                             // one reading of the flag for all warps
+            asm volatile("bar.sync 1, %0;" :: "n"(kTileThreads) : "memory");
+            uint32_t a[16];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint4 v = *reinterpret_cast<const uint4*>(Tb + t2_word(cp, 16 * g + 4 * k));
+                a[4 * k] = v.x; a[4 * k + 1] = v.y; a[4 * k + 2] = v.z; a[4 * k + 3] = v.w;
+            }
+            const int64_t rr = r0 + 16 * g;
+            const int64_t S = rows >> 5;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {                        // column 2cp + half
+                float v[16];
+#pragma unroll
+                for (int m = 0; m < 16; ++m) v[m] = half ? bf16_hi(a[m]) : bf16_lo(a[m]);
+                float mf = 0.0f;
+#pragma unroll
+                for (int m = 0; m < 16; ++m) mf = fmaxf(mf, fabsf(v[m]));
+                mf = fmaxf(mf, __shfl_xor_sync(0xffffffffu, mf, 1));
+                const int e = e8m0_exponent(mf);
+                const float sc = exp2_neg(e);
+                uint32_t w[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    w[i] = cvt_e4m3x4(__fmul_rn(v[4 * i], sc), __fmul_rn(v[4 * i + 1], sc), __fmul_rn(v[4 * i + 2], sc),
+                                      __fmul_rn(v[4 * i + 3], sc));
+                const int64_t cg = c0 + 2 * cp + half;
+                *reinterpret_cast<uint4*>(col_codes + cg * rows + rr) = make_uint4(w[0], w[1], w[2], w[3]);
+                if ((g & 1) == 0) col_e8m0[sf_offset(cg, rr >> 5, S, kLayout)] = (uint8_t)(e + 127);
+            }
+            buf ^= 1;
+            if (stop[it & 1]) break;                                     // the same decision in every warp
+        }
+    }
+}
+
 // NVFP4 [rows, cols] -> dequantise -> transpose -> MXFP8 with SR.
 template <int kR, int kInLayout, int kOutLayout>
 __global__ void __launch_bounds__(kTileThreads, 4)
@@ -501,6 +684,24 @@ extern "C" int mxfp8_quantize(const void* x, int64_t rows, int64_t cols, int rou
         constexpr int kL = decltype(L)::value;
         auto launch = [&](auto kRowC, auto kColC) {
             constexpr bool kRow = decltype(kRowC)::value, kCol = decltype(kColC)::value;
+            if (rounding == MX_ROUND_RNE) {                 // TMA-fed form
+                auto kern = mxfp8_tile_tma_kernel<kRow, kCol, kL>;
+                CUtensorMap tm;
+                unsigned int* status = nullptr;
+                int occ = 0;
+                if (mx_make_bf16_tile_map(&tm, x, rows, cols, kTC, kTR) == MX_OK &&
+                    mx_status_word_address(&status) == MX_OK &&
+                    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmemBytes) == cudaSuccess &&
+                    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kQThreads, kQSmemBytes) == cudaSuccess &&
+                    occ > 0) {
+                    const dim3 qgrid((unsigned)std::min<int64_t>((cols / kTC) * (rows / kTR), (int64_t)sms * occ));
+                    kern<<<qgrid, kQThreads, kQSmemBytes, stream>>>(tm, rows, cols, rows_valid, row_codes, row_e8m0,
+                                                                    col_codes, col_e8m0, status);
+                    mx_count_launch();
+                    return;
+                }
+                cudaGetLastError();
+            }
             if (rounding == MX_ROUND_RNE)
                 mxfp8_tile_kernel<kRow, kCol, false, 8, kL><<<grid, kTileThreads, 0, stream>>>(
                     xb, rows, cols, rows_valid, seed, s_row, s_col, row_codes, row_e8m0, col_codes, col_e8m0);
