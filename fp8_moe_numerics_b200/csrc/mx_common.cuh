@@ -349,6 +349,10 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
     asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
     return r;
 }
+// (a * s, b * s) with s2 = (s, s): two round-to-nearest products, one instruction.
+__device__ __forceinline__ void mul2_rn(float& a, float& b, uint64_t s2) {
+    f2_unpack(f2_mul(f2_pack(a, b), s2), a, b);
+}
 __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
     uint64_t r;
     asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));

@@ -36,14 +36,16 @@ __device__ __forceinline__ uint32_t nvfp4_block(const uint4& a, const uint4& b, 
     if (sc == 0) { packed = make_uint2(0u, 0u); return 0u; }
     float inv = __frcp_rn(__fmul_rn(e4m3_to_f32(sc), s));
     const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    const uint64_t inv2 = f2_pack(inv, inv);
     uint32_t word[2];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {                      // eight products, then their code word
+    for (int h = 0; h < 2; ++h) {                      // eight products (in pairs), then their code word
         float y[8];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            y[2 * i] = __fmul_rn(bf16_lo(w[4 * h + i]), inv);
-            y[2 * i + 1] = __fmul_rn(bf16_hi(w[4 * h + i]), inv);
+            y[2 * i] = bf16_lo(w[4 * h + i]);
+            y[2 * i + 1] = bf16_hi(w[4 * h + i]);
+            mul2_rn(y[2 * i], y[2 * i + 1], inv2);
         }
         word[h] = cvt_e2m1x8(y);
     }
@@ -252,6 +254,7 @@ __device__ __forceinline__ void tile_emit_transposed(const float* T, int64_t row
             // hardware stochastic rounding, two elements per instruction
             const int64_t L0 = cg * rows + rr;          // output element index
             const float sc = exp2_neg(e);
+            const uint64_t sc2 = f2_pack(sc, sc);
 #pragma unroll
             for (int blk = 0; blk < 2; ++blk) {
                 const uint4 rnd = philox4x32_10((uint64_t)(L0 / 8) + blk, stream_id, seed);
@@ -259,9 +262,10 @@ __device__ __forceinline__ void tile_emit_transposed(const float* T, int64_t row
 #pragma unroll
                 for (int q = 0; q < 4; q += 2) {       // elements i..i+3 use words q, q+1
                     const int i = blk * 8 + 2 * q;
-                    w[blk * 2 + (q >> 1)] = cvt_rs16_e4m3_quad(__fmul_rn(v[i], sc), __fmul_rn(v[i + 1], sc),
-                                                               __fmul_rn(v[i + 2], sc), __fmul_rn(v[i + 3], sc),
-                                                               wd[q], wd[q + 1]);
+                    float a0 = v[i], a1 = v[i + 1], a2 = v[i + 2], a3 = v[i + 3];
+                    mul2_rn(a0, a1, sc2);
+                    mul2_rn(a2, a3, sc2);
+                    w[blk * 2 + (q >> 1)] = cvt_rs16_e4m3_quad(a0, a1, a2, a3, wd[q], wd[q + 1]);
                 }
             }
         } else if (kSR) {
@@ -279,10 +283,15 @@ __device__ __forceinline__ void tile_emit_transposed(const float* T, int64_t row
             }
         } else {
             const float sc = exp2_neg(e);
+            const uint64_t sc2 = f2_pack(sc, sc);
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-                w[i] = cvt_e4m3x4(__fmul_rn(v[4 * i], sc), __fmul_rn(v[4 * i + 1], sc), __fmul_rn(v[4 * i + 2], sc),
-                                  __fmul_rn(v[4 * i + 3], sc));
+            {
+                float a0 = v[4 * i], a1 = v[4 * i + 1], a2 = v[4 * i + 2], a3 = v[4 * i + 3];
+                mul2_rn(a0, a1, sc2);
+                mul2_rn(a2, a3, sc2);
+                w[i] = cvt_e4m3x4(a0, a1, a2, a3);
+            }
         }
         *reinterpret_cast<uint4*>(out_codes + cg * rows + rr) = make_uint4(w[0], w[1], w[2], w[3]);
         if ((g & 1) == 0) out_e8m0[sf_offset(cg, rr >> 5, S, kLayout)] = (uint8_t)(e + 127);
@@ -333,6 +342,7 @@ mxfp8_tile_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, co
             const int64_t L0 = r * cols + c0 + 32 * h;
             if (kSR && kR == 16) {
                 const float sc = exp2_neg(e);
+                const uint64_t sc2 = f2_pack(sc, sc);
 #pragma unroll
                 for (int blk = 0; blk < 4; ++blk) {
                     const uint4 rnd = philox4x32_10((uint64_t)(L0 / 8) + blk, stream_row, seed);
@@ -340,9 +350,10 @@ mxfp8_tile_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, co
 #pragma unroll
                     for (int q = 0; q < 4; q += 2) {
                         const int i = blk * 8 + 2 * q;
-                        w[blk * 2 + (q >> 1)] = cvt_rs16_e4m3_quad(__fmul_rn(v[i], sc), __fmul_rn(v[i + 1], sc),
-                                                                   __fmul_rn(v[i + 2], sc), __fmul_rn(v[i + 3], sc),
-                                                                   wd[q], wd[q + 1]);
+                        float a0 = v[i], a1 = v[i + 1], a2 = v[i + 2], a3 = v[i + 3];
+                        mul2_rn(a0, a1, sc2);
+                        mul2_rn(a2, a3, sc2);
+                        w[blk * 2 + (q >> 1)] = cvt_rs16_e4m3_quad(a0, a1, a2, a3, wd[q], wd[q + 1]);
                     }
                 }
             } else if (kSR) {
@@ -359,10 +370,15 @@ mxfp8_tile_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, co
                 }
             } else {
                 const float sc = exp2_neg(e);
+                const uint64_t sc2 = f2_pack(sc, sc);
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
-                    w[i] = cvt_e4m3x4(__fmul_rn(v[4 * i], sc), __fmul_rn(v[4 * i + 1], sc),
-                                      __fmul_rn(v[4 * i + 2], sc), __fmul_rn(v[4 * i + 3], sc));
+                {
+                    float a0 = v[4 * i], a1 = v[4 * i + 1], a2 = v[4 * i + 2], a3 = v[4 * i + 3];
+                    mul2_rn(a0, a1, sc2);
+                    mul2_rn(a2, a3, sc2);
+                    w[i] = cvt_e4m3x4(a0, a1, a2, a3);
+                }
             }
             uint4* dst = reinterpret_cast<uint4*>(row_codes + L0);
             dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
@@ -509,13 +525,20 @@ mxfp8_tile_tma_kernel(const __grid_constant__ CUtensorMap tmX, int64_t rows, int
             for (int i = 0; i < 4; ++i) m = max(m, absmax8_bf16(q[i]));
             const int e = e8m0_exponent(__uint_as_float(m << 16));
             const float sc = exp2_neg(e);
+            const uint64_t sc2 = f2_pack(sc, sc);
             uint32_t w[8];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                w[2 * i] = cvt_e4m3x4(__fmul_rn(bf16_lo(q[i].x), sc), __fmul_rn(bf16_hi(q[i].x), sc),
-                                      __fmul_rn(bf16_lo(q[i].y), sc), __fmul_rn(bf16_hi(q[i].y), sc));
-                w[2 * i + 1] = cvt_e4m3x4(__fmul_rn(bf16_lo(q[i].z), sc), __fmul_rn(bf16_hi(q[i].z), sc),
-                                          __fmul_rn(bf16_lo(q[i].w), sc), __fmul_rn(bf16_hi(q[i].w), sc));
+                const uint32_t qw[4] = {q[i].x, q[i].y, q[i].z, q[i].w};
+                float y[8];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    y[2 * j] = bf16_lo(qw[j]);
+                    y[2 * j + 1] = bf16_hi(qw[j]);
+                    mul2_rn(y[2 * j], y[2 * j + 1], sc2);
+                }
+                w[2 * i] = cvt_e4m3x4(y[0], y[1], y[2], y[3]);
+                w[2 * i + 1] = cvt_e4m3x4(y[4], y[5], y[6], y[7]);
             }
             uint4* dst = reinterpret_cast<uint4*>(row_codes + r * cols + c0 + 32 * h);
             dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
@@ -549,11 +572,16 @@ mxfp8_tile_tma_kernel(const __grid_constant__ CUtensorMap tmX, int64_t rows, int
                 mf = fmaxf(mf, __shfl_xor_sync(0xffffffffu, mf, 1));
                 const int e = e8m0_exponent(mf);
                 const float sc = exp2_neg(e);
+                const uint64_t sc2 = f2_pack(sc, sc);
                 uint32_t w[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
-                    w[i] = cvt_e4m3x4(__fmul_rn(v[4 * i], sc), __fmul_rn(v[4 * i + 1], sc), __fmul_rn(v[4 * i + 2], sc),
-                                      __fmul_rn(v[4 * i + 3], sc));
+                {
+                    float a0 = v[4 * i], a1 = v[4 * i + 1], a2 = v[4 * i + 2], a3 = v[4 * i + 3];
+                    mul2_rn(a0, a1, sc2);
+                    mul2_rn(a2, a3, sc2);
+                    w[i] = cvt_e4m3x4(a0, a1, a2, a3);
+                }
                 const int64_t cg = c0 + 2 * cp + half;
                 *reinterpret_cast<uint4*>(col_codes + cg * rows + rr) = make_uint4(w[0], w[1], w[2], w[3]);
                 if ((g & 1) == 0) col_e8m0[sf_offset(cg, rr >> 5, S, kLayout)] = (uint8_t)(e + 127);
@@ -584,6 +612,7 @@ requant_tile_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict
     // group_rows is 1 or a multiple of 128, so a tile's rows share one group
     const float so = outer[group_rows == 1 ? r : (int64_t)((uint32_t)r0 / (uint32_t)group_rows)];
     const __half2 f0 = __half2half2(e4m3_to_h(sc0)), f1 = __half2half2(e4m3_to_h(sc1));
+    const uint64_t so2 = f2_pack(so, so);
     const uint32_t w[4] = {q.x, q.y, q.z, q.w};
     __half2 hv[16];                                    // hv[i]: elements 2i, 2i+1
 #pragma unroll
@@ -591,8 +620,10 @@ requant_tile_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
         const float2 pf = __half22float2(__hmul2(hv[i], i < 8 ? f0 : f1));   // exact products
-        T[tsw(32 * h + 2 * i, rl)] = __fmul_rn(pf.x, so);
-        T[tsw(32 * h + 2 * i + 1, rl)] = __fmul_rn(pf.y, so);
+        float a = pf.x, b = pf.y;
+        mul2_rn(a, b, so2);
+        T[tsw(32 * h + 2 * i, rl)] = a;
+        T[tsw(32 * h + 2 * i + 1, rl)] = b;
     }
     __syncthreads();
     tile_emit_transposed<true, kR, kOutLayout>(T, rows, cols, r0, c0, seed, stream_id, out_codes, out_e8m0);
