@@ -307,6 +307,7 @@ def run_ours(args):
 
     quant = quantiser_stream(dev, peaks) if rank == 0 else None
     s2f6 = combine_s2f6_leg(layer, c, counts, peaks) if rank == 0 else None
+    mx_fwd = mxfp8_forward_leg(layer, counts, peaks, breakdown) if rank == 0 else None
 
     # ---------------------------------------------------------------- e2e
     e2e = e2e_leg(layer, inp, dev, args, gemm_flops / K, pg, world)
@@ -327,6 +328,7 @@ def run_ours(args):
         "stages": breakdown,
         "quantiser": quant,
         "combine_s2f6": s2f6,
+        "mxfp8_forward": mx_fwd,
         "roofline": roof,
         "clocks": clk.summary(),
         "e2e": e2e,
@@ -421,6 +423,46 @@ def combine_s2f6_leg(layer, c, counts, peaks, reps: int = 10):
     res["bytes_y2"] = {"bf16": M * D * 2, "s2f6": M * D + M * D // 32}
     res["note"] = ("32-d random Hadamard + block-scaled S2F6 in GEMM2's epilogue and the combine reading it, "
                    f"on the layer's operands ({reps} back-to-back launches each)")
+    return res
+
+
+def mxfp8_forward_leg(layer, counts, peaks, breakdown, reps: int = 10):
+    """The pages' comparison on this GPU: the two forward expert GEMMs with
+    MXFP8 operands (E8M0 per 32, RNE) instead of NVFP4, on the layer's own
+    activations and weights, through the MXFP8 row GEMM (weights laid out
+    [N, E*K]); against the NVFP4 GEMM times of the timed steps."""
+    import torch
+    from fp8_moe_numerics_b200 import api
+    L = layer
+    E, D, F, N1, k, M = L.E, L.D, L.F, L.N1, L.k, L.M_cap
+    rows = int(sum(int(x) for x in counts))
+    idx = (L.src.clamp(min=0) // k).long()
+    res = {}
+    for name, a_bf16, w, N, K in (("gemm1", None, L.w1, N1, D), ("gemm2", L.a, L.w2, D, F)):
+        if a_bf16 is None:
+            a_bf16 = L.x[idx]
+            a_bf16[L.src < 0] = 0
+        aq = api.mxfp8_quantize(a_bf16, col=False)
+        wq = api.mxfp8_quantize(w.permute(1, 0, 2).reshape(N, E * K).contiguous(), col=False)
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=L.dev)
+        fn = lambda: api.grouped_gemm_mxfp8(api.MX_GEMM_DGRAD, aq[0], aq[1], wq[0], wq[1], L.seg, E, M, N, K, out=out)
+        for _ in range(3):
+            fn()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / reps
+        tf = 2 * rows * N * K / (ms * 1e-3) / 1e12
+        nv = breakdown[name]
+        res[name] = {"mxfp8_ms": round(ms, 4), "mxfp8_TFLOP/s": round(tf, 1), "nvfp4_ms": nv["ms"],
+                     "nvfp4_TFLOP/s": nv["TFLOP/s"], "nvfp4_speedup": round(ms / nv["ms"], 3)}
+        del aq, wq, out
+    api.sync_status()
+    res["note"] = ("forward expert GEMMs with MXFP8 operands on the same layer, 10 back-to-back launches each, "
+                   "vs the NVFP4 GEMMs of the timed steps (quantisation not included on either side)")
     return res
 
 

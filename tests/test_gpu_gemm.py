@@ -138,6 +138,27 @@ def test_grouped_gemm_mxfp8_dgrad(cuda, E, Nout, Kc, counts):
     assert np.all(np.abs(gb - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-4 * np.abs(ref).max())
 
 
+@pytest.mark.parametrize("E,N,K,counts", [(3, 256, 512, [100, 0, 300]), (2, 512, 256, [130, 50])])
+def test_mxfp8_forward_gemm_with_weights_as_rows(cuda, E, N, K, counts):
+    # the MXFP8 forward baseline: X [M, K] and W [E, N, K] both row-wise MXFP8
+    # (RNE, quantised on the GPU), W laid out [N, E*K] for the row GEMM
+    x, seg = routed_rows(counts, K, seed=3 * E + N + K, nu=4)
+    M_pad = int(seg[-1])
+    M_cap = M_pad + 128
+    w = workloads.weights(E, N, K, 0.02, seed=N + 2 * K)
+    wp = w.permute(1, 0, 2).reshape(N, E * K).contiguous()
+    ac, ae = oracle.mxfp8_quantize_rows(pad_rows(x, M_cap))
+    bc, be = oracle.mxfp8_quantize_rows(wp.view(torch.int16).numpy().view(np.uint16))
+    ref = oracle.grouped_gemm_mxfp8_dgrad(ac[:M_pad], ae[:M_pad], bc, be, seg)
+    ga = api.mxfp8_quantize(dev(pad_rows(x, M_cap).view(np.int16)).view(torch.bfloat16), col=False)
+    gb = api.mxfp8_quantize(wp.cuda(), col=False)
+    assert np.array_equal(ga[0].cpu().numpy(), ac) and np.array_equal(gb[0].cpu().numpy(), bc)
+    out = api.grouped_gemm_mxfp8(api.MX_GEMM_DGRAD, ga[0], ga[1], gb[0], gb[1], dev(seg), E, M_cap, N, K,
+                                 out_dtype=torch.float32)
+    api.sync_status()
+    assert rel_fro(out.cpu().numpy()[:M_pad].astype(np.float64), ref) <= TOL_FRO
+
+
 @pytest.mark.parametrize("E,Nw,Kw,counts", [(3, 256, 256, [128, 0, 300]), (2, 128, 384, [60, 200]),
                                             (4, 256, 512, [0, 129, 1, 256])])
 def test_grouped_gemm_mxfp8_wgrad(cuda, E, Nw, Kw, counts):
