@@ -44,6 +44,7 @@ SIGNATURES = {
     "nvfp4_gather_rows": (I32, [P, P, P, P, I64, I64, I64, P, P, P, P]),
     "swiglu_fwd": (I32, [P, I64, I64, I32, P, P, P]),
     "swiglu_bwd": (I32, [P, P, I64, I64, I32, P, P, P]),
+    "swiglu_nvfp4_quantize": (I32, [P, I64, I64, I32, P, P, P, P, I32, P]),
     "moe_combine": (I32, [P, P, P, I64, I64, I64, P, P]),
     "moe_dispatch_grad": (I32, [P, P, P, P, I64, I64, I64, I64, P, P]),
     "hadamard_s2f6_quantize": (I32, [P, I64, I64, U64, U64, P, P, P]),

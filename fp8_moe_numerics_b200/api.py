@@ -19,7 +19,7 @@ __all__ = [
     "MX_SF_ROWMAJOR", "MX_SF_MMA", "MX_ROUND_RNE", "MX_ROUND_SR", "MX_GEMM_DGRAD", "MX_GEMM_WGRAD", "MxError",
     "sf_bytes", "sync_status", "wait_selftest", "nvfp4_quantize", "mxfp8_requant_transpose_sr", "mxfp8_quantize",
     "grouped_gemm_nvfp4", "grouped_gemm_mxfp8", "moe_route", "nvfp4_gather_rows", "swiglu_fwd", "swiglu_bwd",
-    "moe_combine", "moe_dispatch_grad", "hadamard_s2f6_quantize", "grouped_gemm_nvfp4_s2f6", "moe_combine_s2f6",
+    "moe_combine", "moe_dispatch_grad", "swiglu_nvfp4_quantize", "hadamard_s2f6_quantize", "grouped_gemm_nvfp4_s2f6", "moe_combine_s2f6",
 ]
 
 
@@ -240,3 +240,19 @@ def moe_combine_s2f6(codes: torch.Tensor, e8m0: torch.Tensor, pos: torch.Tensor,
         out = torch.empty(T, D, dtype=torch.bfloat16, device=codes.device)
     L.call("moe_combine_s2f6", _p(codes), _p(e8m0), _p(pos), _p(w), T, k, D, seed, stream_id, _p(out), _s())
     return out
+
+
+def swiglu_nvfp4_quantize(h: torch.Tensor, F: int, gated: bool = True, rows_valid=None, sf_layout: int = MX_SF_MMA,
+                          out=None):
+    """SwiGLU of h (bf16 [rows, 2F] or [rows, F]) quantised to NVFP4 per token:
+    (codes u8 [rows, F/2], sf u8, outer f32 [rows])."""
+    assert h.dtype == torch.bfloat16 and h.dim() == 2
+    rows = h.shape[0]
+    if out is None:
+        out = (torch.empty(rows, F // 2, dtype=torch.uint8, device=h.device),
+               _u8(sf_bytes(rows, F, 16, sf_layout), h.device),
+               torch.empty(rows, dtype=torch.float32, device=h.device))
+    codes, sf, outer = out
+    L.call("swiglu_nvfp4_quantize", _p(h), rows, F, int(gated), _p(rows_valid), _p(codes), _p(sf), _p(outer),
+           sf_layout, _s())
+    return codes, sf, outer

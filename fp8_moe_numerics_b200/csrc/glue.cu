@@ -123,20 +123,11 @@ __global__ void gather_rows_kernel(const uint8_t* __restrict__ codes, const uint
     if (lane == 0) out_outer[p] = t < 0 ? 0.0f : outer[t];
 }
 
-// sigmoid with the fast exponential and division intrinsics: a few fp32 ulp,
-// far below the bf16 rounding that follows (results stay within one bf16
-// rounding of the exact value); exp overflow gives sigmoid 0, as it should.
-__device__ __forceinline__ float sigmoid_f(float g) { return __fdividef(1.0f, 1.0f + __expf(-g)); }
-__device__ __forceinline__ float silu_f(float g) { return g * sigmoid_f(g); }
 __device__ __forceinline__ float dsilu_f(float g) {
     const float s = sigmoid_f(g);
     return s * (1.0f + g * (1.0f - s));
 }
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t*>(&v);
-}
 
 // 8 outputs per thread.
 __global__ void swiglu_fwd_kernel(const uint16_t* __restrict__ h, int64_t rows, int64_t F, int gated,
@@ -158,7 +149,7 @@ __global__ void swiglu_fwd_kernel(const uint16_t* __restrict__ h, int64_t rows, 
         uint32_t ow[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-            ow[j] = pack_bf16x2(silu_f(bf16_lo(gw[j])) * bf16_lo(uw[j]), silu_f(bf16_hi(gw[j])) * bf16_hi(uw[j]));
+            ow[j] = swiglu_word(gw[j], uw[j]);
         o = make_uint4(ow[0], ow[1], ow[2], ow[3]);
     }
     *reinterpret_cast<uint4*>(a + r * F + c) = o;

@@ -157,6 +157,23 @@ __device__ __forceinline__ __half e4m3_to_h(uint32_t code) {
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// sigmoid with the fast exponential and division intrinsics: a few fp32 ulp,
+// far below the bf16 rounding that follows (results stay within one bf16
+// rounding of the exact value); exp overflow gives sigmoid 0, as it should.
+__device__ __forceinline__ float sigmoid_f(float g) { return __fdividef(1.0f, 1.0f + __expf(-g)); }
+__device__ __forceinline__ float silu_f(float g) { return g * sigmoid_f(g); }
+
+// Two SwiGLU outputs silu(g) * u, each rounded to bf16, from two bf16 pairs
+// (the one definition the standalone and the fused-quantiser kernels share).
+__device__ __forceinline__ uint32_t swiglu_word(uint32_t g, uint32_t u) {
+    return pack_bf16x2(silu_f(bf16_lo(g)) * bf16_lo(u), silu_f(bf16_hi(g)) * bf16_hi(u));
+}
+
 // ---------------------------------------------------------------------------
 // MXFP8 block exponent: smallest e with amax <= 448 * 2^e, clamped to
 // [-127, 127]; -127 for amax == 0.  448 = 1.75 * 2^8, so for a normal

@@ -53,6 +53,29 @@ __device__ __forceinline__ uint32_t nvfp4_block(const uint4& a, const uint4& b, 
     return sc;
 }
 
+// Codes and scale of block `blk` of `row` (outer scale s); every lane of the
+// warp calls it, live or not, because the scale bytes of four consecutive
+// blocks (in lanes 4m..4m+3) are merged by shuffles into one 32-bit store
+// when `word_sf`.
+template <int kLayout>
+__device__ __forceinline__ void emit_nvfp4_block(int64_t row, int64_t blk, int64_t nblk, bool active, float s,
+                                                 const uint4& a, const uint4& b, uint8_t* __restrict__ crow,
+                                                 uint8_t* __restrict__ sf, bool word_sf, int lane) {
+    uint2 packed = make_uint2(0u, 0u);
+    uint32_t sc = 0;
+    const bool live = active && blk < nblk;
+    if (live && s > 0.0f) sc = nvfp4_block(a, b, s, packed);
+    if (live) *reinterpret_cast<uint2*>(crow + blk * 8) = packed;
+    if (word_sf) {
+        uint32_t w = sc << (8 * (lane & 3));
+        w |= __shfl_xor_sync(0xffffffffu, w, 1);
+        w |= __shfl_xor_sync(0xffffffffu, w, 2);
+        if (live && (lane & 3) == 0) *reinterpret_cast<uint32_t*>(sf + sf_offset(row, blk, nblk, kLayout)) = w;
+    } else if (live) {
+        sf[sf_offset(row, blk, nblk, kLayout)] = (uint8_t)sc;
+    }
+}
+
 // kTPR threads per row (a power of two, 16..256), 256 / kTPR rows per block.
 // Thread j of a row handles the 16-element blocks j, j + kTPR, ... (kNB of
 // them held in registers when the row fits, so each warp's loads cover
@@ -122,19 +145,7 @@ __device__ __forceinline__ void quant_rows_block(const uint16_t* __restrict__ x,
 
     uint8_t* crow = codes + (active ? row : 0) * (cols >> 1);
     auto emit = [&](int64_t blk, const uint4& a, const uint4& b) {
-        uint2 packed = make_uint2(0u, 0u);
-        uint32_t sc = 0;
-        const bool live = active && blk < nblk;
-        if (live && s > 0.0f) sc = nvfp4_block(a, b, s, packed);
-        if (live) *reinterpret_cast<uint2*>(crow + blk * 8) = packed;
-        if (word_sf) {                                   // blocks 4m..4m+3 sit in lanes 4m'..4m'+3
-            uint32_t w = sc << (8 * (lane & 3));
-            w |= __shfl_xor_sync(0xffffffffu, w, 1);
-            w |= __shfl_xor_sync(0xffffffffu, w, 2);
-            if (live && (lane & 3) == 0) *reinterpret_cast<uint32_t*>(sf + sf_offset(row, blk, nblk, kLayout)) = w;
-        } else if (live) {
-            sf[sf_offset(row, blk, nblk, kLayout)] = (uint8_t)sc;
-        }
+        emit_nvfp4_block<kLayout>(row, blk, nblk, active, s, a, b, crow, sf, word_sf, lane);
     };
     if (resident) {
 #pragma unroll
@@ -155,6 +166,70 @@ nvfp4_quant_rows_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t co
     __shared__ uint32_t wmax[kRowThreads / 32];
     quant_rows_block<kTPR, kNB, kGroup, kLayout>(x, rows, rows, cols, group_rows, word_sf, codes, sf, outer,
                                                  (int64_t)blockIdx.x, wmax);
+}
+
+// SwiGLU fused into the per-token NVFP4 quantiser: the activation a =
+// silu(g) * u of each element is formed in registers exactly as swiglu_fwd
+// writes it (swiglu_word, bf16 round-to-nearest) and quantised as
+// nvfp4_quant_rows_kernel quantises a bf16 row, so the result equals the two
+// kernels run one after the other, without a's round trip through HBM.
+// h = [g | u] (gated, [rows, 2F]) or [g] ([rows, F], u = 1).  Rows at or past
+// *rows_valid are zero rows (codes 0, scales 0, outer 0).  Rows must fit in
+// registers: F/16 <= 4 kTPR.
+template <int kTPR, int kLayout>
+__global__ void __launch_bounds__(kRowThreads, 4)
+swiglu_nvfp4_rows_kernel(const uint16_t* __restrict__ h, int64_t rows, int64_t F, int gated, const int64_t* rows_valid,
+                         bool word_sf, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
+                         float* __restrict__ outer) {
+    constexpr int kNB = 4;
+    constexpr int kRPB = kRowThreads / kTPR;
+    __shared__ uint32_t wmax[kRowThreads / 32];
+    const int lane = threadIdx.x & 31;
+    const int j = threadIdx.x % kTPR;
+    const int64_t row = (int64_t)blockIdx.x * kRPB + threadIdx.x / kTPR;
+    const bool active = row < rows;
+    const bool live = active && row < load_rows_valid(rows_valid, rows);
+    const int64_t nblk = F >> 4;
+    const int64_t hw = gated ? 2 * F : F;
+    const uint4* gr = reinterpret_cast<const uint4*>(h + (live ? row : 0) * hw);
+    const uint4* ur = reinterpret_cast<const uint4*>(h + (live ? row : 0) * hw + F);
+    const uint4 one = make_uint4(0x3f803f80u, 0x3f803f80u, 0x3f803f80u, 0x3f803f80u);   // bf16 1.0
+    uint4 va[kNB], vb[kNB];
+    uint32_t amax_bits = 0;
+#pragma unroll
+    for (int i = 0; i < kNB; ++i) {
+        const int64_t blk = j + (int64_t)kTPR * i;
+        va[i] = make_uint4(0, 0, 0, 0);
+        vb[i] = va[i];
+        if (live && blk < nblk) {
+            const uint4 g0 = __ldcs(gr + 2 * blk), g1 = __ldcs(gr + 2 * blk + 1);
+            const uint4 u0 = gated ? __ldcs(ur + 2 * blk) : one, u1 = gated ? __ldcs(ur + 2 * blk + 1) : one;
+            va[i] = make_uint4(swiglu_word(g0.x, u0.x), swiglu_word(g0.y, u0.y), swiglu_word(g0.z, u0.z),
+                               swiglu_word(g0.w, u0.w));
+            vb[i] = make_uint4(swiglu_word(g1.x, u1.x), swiglu_word(g1.y, u1.y), swiglu_word(g1.z, u1.z),
+                               swiglu_word(g1.w, u1.w));
+        }
+        amax_bits = max(amax_bits, max(absmax8_bf16(va[i]), absmax8_bf16(vb[i])));
+    }
+    if (kTPR >= 32) {
+        amax_bits = warp_max_u32(amax_bits);
+    } else {
+#pragma unroll
+        for (int o = kTPR / 2; o > 0; o >>= 1) amax_bits = max(amax_bits, __shfl_xor_sync(0xffffffffu, amax_bits, o));
+    }
+    if (kTPR > 32) {
+        if (lane == 0) wmax[threadIdx.x >> 5] = amax_bits;
+        __syncthreads();
+        const int w0 = (threadIdx.x / kTPR) * (kTPR / 32);
+#pragma unroll
+        for (int w = 0; w < kTPR / 32; ++w) amax_bits = max(amax_bits, wmax[w0 + w]);
+    }
+    const float s = __fdiv_rn(__uint_as_float(amax_bits << 16), 2688.0f);
+    if (active && j == 0) outer[row] = s;
+    uint8_t* crow = codes + (active ? row : 0) * (F >> 1);
+#pragma unroll
+    for (int i = 0; i < kNB; ++i)
+        emit_nvfp4_block<kLayout>(row, j + (int64_t)kTPR * i, nblk, active, s, va[i], vb[i], crow, sf, word_sf, lane);
 }
 
 // amax over each group of rows, as fp32 bits, atomically max-ed into outer[g]
@@ -688,6 +763,35 @@ extern "C" int nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t
             nvfp4_group_finish_kernel<<<(unsigned)((ngroups + 255) / 256), 256, 0, stream>>>(outer, ngroups);
             mx_count_launch();
         }
+        return mx_launch_status();
+    });
+}
+
+extern "C" int swiglu_nvfp4_quantize(const void* h, int64_t rows, int64_t F, int gated, const int64_t* rows_valid,
+                                     uint8_t* codes, uint8_t* sf, float* outer, int sf_layout, cudaStream_t stream) {
+    if (((!h || !codes || !sf || !outer) && rows > 0) || rows < 0 || F <= 0 || F % 16 || F / 16 > 1024 ||
+        !mx_aligned(h, 16) || !mx_aligned(codes, 16))
+        return MX_EINVAL;
+    if (sf_layout != MX_SF_ROWMAJOR && sf_layout != MX_SF_MMA) return MX_EINVAL;
+    if (sf_layout == MX_SF_MMA && (rows % 128 || F % 64)) return MX_EINVAL;
+    if (int st = mx_check_device()) return st;
+    if (rows == 0) return MX_OK;
+    const int64_t nblk = F / 16;
+    const bool word_sf = nblk % 4 == 0 && mx_aligned(sf, 4);
+    const uint16_t* hb = static_cast<const uint16_t*>(h);
+    return dispatch_layout(sf_layout, [&](auto L) {
+        constexpr int kL = decltype(L)::value;
+        auto go = [&](auto kern, int tpr) {
+            const int64_t rpb = kRowThreads / tpr;
+            kern<<<(unsigned)((rows + rpb - 1) / rpb), kRowThreads, 0, stream>>>(hb, rows, F, gated, rows_valid, word_sf,
+                                                                                   codes, sf, outer);
+            mx_count_launch();
+        };
+        if (nblk <= 64) go(swiglu_nvfp4_rows_kernel<16, kL>, 16);
+        else if (nblk <= 128) go(swiglu_nvfp4_rows_kernel<32, kL>, 32);
+        else if (nblk <= 256) go(swiglu_nvfp4_rows_kernel<64, kL>, 64);
+        else if (nblk <= 512) go(swiglu_nvfp4_rows_kernel<128, kL>, 128);
+        else go(swiglu_nvfp4_rows_kernel<256, kL>, 256);
         return mx_launch_status();
     });
 }

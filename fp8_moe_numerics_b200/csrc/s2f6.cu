@@ -24,11 +24,6 @@ __device__ __forceinline__ float pow2_int(int n) {
     return n >= -126 ? __uint_as_float((uint32_t)(n + 127) << 23) : __uint_as_float(1u << (n + 149));
 }
 
-__device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
-    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t*>(&v);
-}
-
 __global__ void __launch_bounds__(kThreads)
 hadamard_s2f6_quantize_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t nbc, uint64_t seed,
                               uint64_t stream_id, uint8_t* __restrict__ codes, uint8_t* __restrict__ e8m0) {
@@ -88,7 +83,7 @@ moe_combine_s2f6_kernel(const uint8_t* __restrict__ codes, const uint8_t* __rest
     apply_signs32(u, hadamard_sign_word(seed, stream_id, (uint64_t)jb));
     uint32_t o[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) o[i] = bf16x2_rn(__fmul_rn(u[2 * i], 0.03125f), __fmul_rn(u[2 * i + 1], 0.03125f));
+    for (int i = 0; i < 16; ++i) o[i] = pack_bf16x2(__fmul_rn(u[2 * i], 0.03125f), __fmul_rn(u[2 * i + 1], 0.03125f));
     uint4* dst = reinterpret_cast<uint4*>(out + item * 32);
 #pragma unroll
     for (int q = 0; q < 4; ++q) dst[q] = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);

@@ -6,7 +6,7 @@ across transposes):
 
   forward   route -> NVFP4 quantise tokens (per-token outer scale) -> gather
             into expert order -> NVFP4 quantise W1, W2 (per-expert outer
-            scale) -> grouped NVFP4 GEMM1 -> SwiGLU -> NVFP4 quantise ->
+            scale) -> grouped NVFP4 GEMM1 -> SwiGLU + NVFP4 quantise (one kernel) ->
             grouped NVFP4 GEMM2 -> combine (with combine="s2f6", GEMM2's epilogue
             rotates each 32-column block by a random Hadamard transform and
             writes block-scaled S2F6, and the combine reads that:
@@ -38,7 +38,9 @@ class ExpertLayer:
 
     x [T, D] bf16, topk [T, k] int32, w_comb [T, k] f32, w1 [E, 2F or F, D]
     bf16, w2 [E, D, F] bf16, dout [T, D] bf16, all on one CUDA device.
-    `wgrad_dtype` is the dtype of dW1 / dW2 (bf16 or fp32).  `combine` is
+    `wgrad_dtype` is the dtype of dW1 / dW2 (bf16 or fp32).  `fuse_swiglu`
+    quantises SwiGLU's output in the same kernel (the bf16 activation is then
+    never written; `a` holds it only with fuse_swiglu=False).  `combine` is
     "bf16" (GEMM2 writes bf16 rows) or "s2f6" (GEMM2 writes rotated S2F6 rows,
     one byte per value plus one exponent per 32).
     """
@@ -46,9 +48,11 @@ class ExpertLayer:
     S2F6_STREAM = 101                                   # Philox stream of the rotation's signs
 
     def __init__(self, x, topk, w_comb, w1, w2, dout, gated: bool = True, seed: int = 0,
-                 wgrad_dtype=torch.bfloat16, out_dtype=torch.bfloat16, rbits: int = 16, combine: str = "bf16"):
+                 wgrad_dtype=torch.bfloat16, out_dtype=torch.bfloat16, rbits: int = 16, combine: str = "bf16",
+                 fuse_swiglu: bool = True):
         assert combine in ("bf16", "s2f6")
         self.combine = combine
+        self.fuse_swiglu = fuse_swiglu
         dev = x.device
         self.dev = dev
         self.T, self.D = x.shape
@@ -138,10 +142,14 @@ class ExpertLayer:
         self._mark("quant_w", record)
         api.grouped_gemm_nvfp4(self.xp, self.w1q, self.seg, E, N1, D, out=self.h1)
         self._mark("gemm1", record)
-        api.swiglu_fwd(self.h1, F, self.gated, self.rows_valid, out=self.a)
-        self._mark("swiglu", record)
-        api.nvfp4_quantize(self.a, 1, MX_SF_MMA, out=self.aq)
-        self._mark("quant_a", record)
+        if self.fuse_swiglu:
+            api.swiglu_nvfp4_quantize(self.h1, F, self.gated, self.rows_valid, MX_SF_MMA, out=self.aq)
+            self._mark("swiglu_quant", record)
+        else:
+            api.swiglu_fwd(self.h1, F, self.gated, self.rows_valid, out=self.a)
+            self._mark("swiglu", record)
+            api.nvfp4_quantize(self.a, 1, MX_SF_MMA, out=self.aq)
+            self._mark("quant_a", record)
         if self.combine == "s2f6":
             api.grouped_gemm_nvfp4_s2f6(self.aq, self.w2q, self.seg, E, D, F, self.seed, self.S2F6_STREAM,
                                         out=self.y2s)

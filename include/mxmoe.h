@@ -260,6 +260,19 @@ MX_API int swiglu_fwd(const void* h, int64_t rows, int64_t F, int gated, const i
 MX_API int swiglu_bwd(const void* h, const void* da, int64_t rows, int64_t F, int gated,
                const int64_t* rows_valid, void* dh, cudaStream_t stream);
 
+/* swiglu_nvfp4_quantize -- swiglu_fwd fused into nvfp4_quantize (per-token
+ * outer scale, group_rows = 1): each a = silu(g)*u is rounded to bf16 exactly
+ * as swiglu_fwd rounds it and quantised exactly as nvfp4_quantize quantises a
+ * bf16 row, so the outputs equal those two calls in sequence while a never
+ * reaches HBM ([ai-primer §NVFP4 forward, MXFP8 backward]: both expert GEMMs
+ * of the forward pass take NVFP4 operands).  h bf16 [rows, 2F] (gated, g then
+ * u) or [rows, F]; rows at or past *rows_valid (when rows_valid != NULL)
+ * quantise as zero rows.  Outputs as nvfp4_quantize of [rows, F].  F % 16 ==
+ * 0 and F <= 16384 (F % 64 == 0 and rows % 128 == 0 for MX_SF_MMA); h and
+ * codes 16-byte aligned; else MX_EINVAL. */
+MX_API int swiglu_nvfp4_quantize(const void* h, int64_t rows, int64_t F, int gated, const int64_t* rows_valid,
+                                 uint8_t* codes, uint8_t* sf, float* outer, int sf_layout, cudaStream_t stream);
+
 /* moe_combine -- out[t] = sum_j w[t,j] * y[pos[t,j]], fp32 accumulation,
  * bf16 output.  y device bf16 [*, D], pos int32 [T, k], w f32 [T, k] (NULL:
  * all weights 1). */

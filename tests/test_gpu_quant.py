@@ -140,6 +140,33 @@ def test_nvfp4_quantize_per_expert_spread_and_zero_experts(cuda, E, N, K, layout
     assert outer[1] == 0 and np.all(codes[N:2 * N] == 0)
 
 
+@pytest.mark.parametrize("rows,F,gated,valid,layout", [(384, 1024, True, 300, api.MX_SF_MMA),
+                                                        (256, 512, False, None, api.MX_SF_MMA),
+                                                        (128, 4096, True, None, api.MX_SF_MMA),
+                                                        (130, 96, False, 77, api.MX_SF_ROWMAJOR)])
+def test_swiglu_nvfp4_quantize_fuses_the_two_kernels(cuda, rows, F, gated, valid, layout):
+    rng = np.random.default_rng(rows + F)
+    h = oracle.f32_to_bf16((rng.standard_normal((rows, 2 * F if gated else F)) * 3).astype(np.float32))
+    hd = to_dev_bf16(h)
+    rv = torch.tensor([valid], dtype=torch.int64, device="cuda") if valid is not None else None
+    fused = api.swiglu_nvfp4_quantize(hd, F, gated, rv, layout)
+    a = api.swiglu_fwd(hd, F, gated, rv)
+    two = api.nvfp4_quantize(a, 1, layout)
+    api.sync_status()
+    for got, want in zip(fused, two):                          # the same bytes as the two kernels in sequence
+        assert torch.equal(got, want)
+    # against the oracle's SwiGLU (fp64, one bf16 rounding) and quantiser: the
+    # GPU's fast sigmoid can move a value by one bf16 unit, so rare codes differ
+    n = rows if valid is None else valid
+    ref_a = oracle.swiglu_fwd(h[:n], gated=gated)
+    rc, rs, ro = oracle.nvfp4_quantize(ref_a)
+    gc = np_(fused[0])
+    assert np.mean(gc[:n] == rc) >= 0.99
+    go = np_(fused[2])
+    assert np.all(np.abs(go[:n] - ro) <= 2.0 ** -7 * np.abs(ro))
+    assert np.all(gc[n:] == 0) and np.all(go[n:] == 0)
+
+
 # ---------------------------------------------------------------------------
 # MXFP8 quantiser
 # ---------------------------------------------------------------------------

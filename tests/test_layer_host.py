@@ -46,7 +46,8 @@ def test_layer_sequence_passes_host_validation(host_calls, name):
     assert names[0] == "moe_route" and names[-1] == "moe_combine"
     assert names.count("grouped_gemm_nvfp4") == 2 and names.count("grouped_gemm_mxfp8") == 4
     assert names.count("mxfp8_requant_transpose_sr") == 4
-    assert len(names) == 23
+    assert names.count("swiglu_nvfp4_quantize") == 1 and "swiglu_fwd" not in names   # fused by default
+    assert len(names) == 22
     assert all(st == _lib.MX_ECUDA for _, st in host_calls)   # valid, and no device here
 
 
@@ -61,5 +62,18 @@ def test_s2f6_combine_sequence_passes_host_validation(host_calls):
     # the forward combine reads S2F6; the backward's un-permute of dX stays a bf16 combine
     assert names.count("moe_combine_s2f6") == 1 and names.count("moe_combine") == 1
     assert names.index("moe_combine_s2f6") == names.index("grouped_gemm_nvfp4_s2f6") + 1
+    assert len(names) == 22
+    assert all(st == _lib.MX_ECUDA for _, st in host_calls)
+
+
+def test_unfused_swiglu_sequence_passes_host_validation(host_calls):
+    inp = workloads.layer_inputs("tiny_layer", device="cpu")
+    c = inp["cfg"]
+    L = ExpertLayer(inp["x"], inp["topk"], inp["w_comb"], inp["w1"], inp["w2"], inp["dout"], gated=c["gated"],
+                    fuse_swiglu=False)
+    L.step()
+    names = [n for n, _ in host_calls]
+    assert "swiglu_nvfp4_quantize" not in names and names.count("swiglu_fwd") == 1
+    assert names.count("nvfp4_quantize") == 4                   # tokens, W1, W2, activations
     assert len(names) == 23
     assert all(st == _lib.MX_ECUDA for _, st in host_calls)
