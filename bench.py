@@ -66,15 +66,57 @@ def load_peaks():
 # clocks sampled during the timed region
 # --------------------------------------------------------------------------
 class ClockSampler:
+    """SM clock, power and clock-event reasons during the timed region: read
+    through NVML every 20 ms on a host thread (read-only queries), or, where
+    NVML is unavailable, from `nvidia-smi -lms 200`."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    REASON_BITS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown"}
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
+        self.thread = None
+        self.rows = []
+
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        try:                                              # the CUDA device's own GPU, whatever the visible set
+            uuid = str(torch.cuda.get_device_properties(self.gpu).uuid)
+            return pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+            idx = int(vis.split(",")[self.gpu]) if vis and vis.split(",")[self.gpu].isdigit() else self.gpu
+            return pynvml.nvmlDeviceGetHandleByIndex(idx)
 
     def __enter__(self):
+        import threading
+        try:
+            import pynvml
+            h = self._nvml_handle()
+            smax = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self.stop = threading.Event()
+
+            def loop():
+                while not self.stop.is_set():
+                    try:
+                        r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    except Exception:
+                        r = pynvml.nvmlDeviceGetCurrentClocksThrottleReasons(h)
+                    self.rows.append(dict(sm=float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)),
+                                          smax=float(smax), power=pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0,
+                                          reasons={n for b, n in self.REASON_BITS.items() if r & b}))
+                    self.stop.wait(0.02)
+
+            self.thread = threading.Thread(target=loop, daemon=True)
+            self.thread.start()
+            return self
+        except Exception:
+            self.thread = None
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
                                           "--format=csv,noheader,nounits", "-lms", "200"],
@@ -84,37 +126,41 @@ class ClockSampler:
         return self
 
     def __exit__(self, *a):
-        self.out = ""
+        if self.thread is not None:
+            self.stop.set()
+            self.thread.join(timeout=5)
+            return
+        out = ""
         if self.proc is not None:
             self.proc.terminate()
             try:
-                self.out, _ = self.proc.communicate(timeout=5)
+                out, _ = self.proc.communicate(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-                self.out, _ = self.proc.communicate()
-
-    def summary(self):
-        rows = []
-        for line in (self.out or "").strip().splitlines():
+                out, _ = self.proc.communicate()
+        for line in (out or "").strip().splitlines():
             f = [x.strip() for x in line.split(",")]
             if len(f) < 9:
                 continue
             try:
-                rows.append(dict(sm=float(f[1]), smax=float(f[2]), power=float(f[3]),
-                                 hw=f[5], hwt=f[6], swt=f[7], pcap=f[8]))
+                self.rows.append(dict(sm=float(f[1]), smax=float(f[2]), power=float(f[3]),
+                                      reasons={n for n, v in zip(("hw_slowdown", "hw_thermal_slowdown",
+                                                                  "sw_thermal_slowdown", "sw_power_cap"), f[5:9])
+                                               if v.lower().startswith("active")}))
             except ValueError:
                 continue
+
+    def summary(self):
+        rows = self.rows
         if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no nvidia-smi samples"], "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no clock samples"], "samples": 0}
         loaded = [r for r in rows if r["power"] > 300] or rows
         reasons = set()
         for r in loaded:
-            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"), ("swt", "sw_thermal_slowdown"),
-                              ("pcap", "sw_power_cap")):
-                if r[key].lower().startswith("active"):
-                    reasons.add(name)
+            reasons |= r["reasons"]
         return {"sm_mhz": statistics.median(r["sm"] for r in loaded), "sm_max_mhz": max(r["smax"] for r in rows),
-                "reasons": sorted(reasons), "samples": len(loaded)}
+                "reasons": sorted(reasons), "samples": len(loaded),
+                "source": "nvml, 20 ms" if self.thread is not None else "nvidia-smi, 200 ms"}
 
 
 # --------------------------------------------------------------------------

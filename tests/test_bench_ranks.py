@@ -1,4 +1,5 @@
-"""bench.py's multi-process plumbing on CPU ranks (gloo, world size 2).
+"""bench.py's host plumbing on CPU: its multi-process reductions on gloo ranks
+(world size 2) and its clock sampler against a fake NVML.
 
 The expert layer runs as independent replicas, one per GPU, with no
 collective on the data path; bench.py only reduces its timings (max over
@@ -63,3 +64,33 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
 
     bench.run_reference(Args())                  # returns before touching the oracle
     assert capsys.readouterr().out == ""
+
+
+def test_clock_sampler_reads_nvml_on_a_thread(monkeypatch):
+    # a fake NVML (read-only queries): 1700 MHz under a 700 W load with the
+    # power-cap reason set, and an idle sample that the summary ignores
+    import time
+    import types
+    sys.path.insert(0, ROOT)
+    import bench
+    calls = {"n": 0}
+    fake = types.SimpleNamespace(
+        NVML_CLOCK_SM=1,
+        nvmlInit=lambda: None,
+        nvmlDeviceGetHandleByUUID=lambda u: "h",
+        nvmlDeviceGetHandleByIndex=lambda i: "h",
+        nvmlDeviceGetMaxClockInfo=lambda h, c: 1965,
+        nvmlDeviceGetClockInfo=lambda h, c: 1700,
+        nvmlDeviceGetCurrentClocksEventReasons=lambda h: 0x4,
+    )
+
+    def power(h):
+        calls["n"] += 1
+        return 100_000 if calls["n"] == 1 else 700_000          # milliwatts
+    fake.nvmlDeviceGetPowerUsage = power
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    with bench.ClockSampler(0) as clk:
+        time.sleep(0.15)
+    s = clk.summary()
+    assert s["source"].startswith("nvml") and s["samples"] >= 3
+    assert s["sm_mhz"] == 1700 and s["sm_max_mhz"] == 1965 and s["reasons"] == ["sw_power_cap"]
