@@ -307,7 +307,7 @@ __device__ __forceinline__ void tile_emit_transposed(const float* T, int64_t row
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane & 7;
     const int64_t S = rows >> 5;                        // output scales per output row
-#pragma unroll 1
+#pragma unroll
     for (int it = 0; it < 2; ++it) {
         const int c = it * 32 + warp * 4 + (lane >> 3);
         float v[16];
