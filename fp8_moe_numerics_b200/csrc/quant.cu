@@ -671,7 +671,7 @@ mxfp8_tile_tma_kernel(const __grid_constant__ CUtensorMap tmX, int64_t rows, int
 template <int kR, int kInLayout, int kOutLayout>
 __global__ void __launch_bounds__(kTileThreads, 4)
 requant_tile_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sf, const float* __restrict__ outer,
-                    int64_t rows, int64_t cols, int64_t group_rows, const int64_t* rows_valid,
+                    int64_t rows, int64_t cols, int64_t group_rows, int group_shift, const int64_t* rows_valid,
                     uint64_t seed, uint64_t stream_id, uint8_t* __restrict__ out_codes, uint8_t* __restrict__ out_e8m0) {
     __shared__ __align__(16) float T[kTC * kTR];
     const int64_t c0 = (int64_t)blockIdx.x * kTC, r0 = (int64_t)blockIdx.y * kTR;
@@ -685,7 +685,9 @@ requant_tile_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict
     const uint32_t sc0 = sf[sf_offset(r, s0, S, kInLayout)];
     const uint32_t sc1 = sf[sf_offset(r, s0 + 1, S, kInLayout)];
     // group_rows is 1 or a multiple of 128, so a tile's rows share one group
-    const float so = outer[group_rows == 1 ? r : (int64_t)((uint32_t)r0 / (uint32_t)group_rows)];
+    const int64_t gi = group_rows == 1 ? r
+                     : (group_shift >= 0 ? (r0 >> group_shift) : (int64_t)((uint32_t)r0 / (uint32_t)group_rows));
+    const float so = outer[gi];
     const __half2 f0 = __half2half2(e4m3_to_h(sc0)), f1 = __half2half2(e4m3_to_h(sc1));
     const uint64_t so2 = f2_pack(so, so);
     const uint32_t w[4] = {q.x, q.y, q.z, q.w};
@@ -879,18 +881,22 @@ extern "C" int mxfp8_requant_transpose_sr(const uint8_t* codes, const uint8_t* s
     // block's loads overlap another's rounding arithmetic (measured faster on
     // B200 than persistent blocks, which move through the phases in step)
     const dim3 grid((unsigned)(cols / kTC), (unsigned)(rows / kTR));
+    // expert groups of a power-of-two size index their outer scale by a shift
+    int gshift = -1;
+    if (group_rows > 1 && (group_rows & (group_rows - 1)) == 0)
+        for (gshift = 0; ((int64_t)1 << gshift) < group_rows; ++gshift) {}
     return dispatch_layout(in_sf_layout, [&](auto Li) {
         return dispatch_layout(out_sf_layout, [&](auto Lo) {
             constexpr int kLi = decltype(Li)::value, kLo = decltype(Lo)::value;
             if (rbits == 8)
                 requant_tile_kernel<8, kLi, kLo><<<grid, kTileThreads, 0, stream>>>(
-                    codes, sf, outer, rows, cols, group_rows, rows_valid, seed, stream_id, out_codes, out_e8m0);
+                    codes, sf, outer, rows, cols, group_rows, gshift, rows_valid, seed, stream_id, out_codes, out_e8m0);
             else if (rbits == 16)
                 requant_tile_kernel<16, kLi, kLo><<<grid, kTileThreads, 0, stream>>>(
-                    codes, sf, outer, rows, cols, group_rows, rows_valid, seed, stream_id, out_codes, out_e8m0);
+                    codes, sf, outer, rows, cols, group_rows, gshift, rows_valid, seed, stream_id, out_codes, out_e8m0);
             else
                 requant_tile_kernel<32, kLi, kLo><<<grid, kTileThreads, 0, stream>>>(
-                    codes, sf, outer, rows, cols, group_rows, rows_valid, seed, stream_id, out_codes, out_e8m0);
+                    codes, sf, outer, rows, cols, group_rows, gshift, rows_valid, seed, stream_id, out_codes, out_e8m0);
             mx_count_launch();
             return mx_launch_status();
         });

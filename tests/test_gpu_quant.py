@@ -249,13 +249,17 @@ def test_requant_extreme_dynamic_range(cuda, R):
     assert np.array_equal(np_(ge).reshape(oe.shape), oe)
 
 
-def test_requant_weights_per_expert_outer(cuda):
-    E, N, K = 3, 128, 256
-    w = workloads.weights(E, N, K, 0.02, seed=5).reshape(E * N, K).view(torch.int16).numpy().view(np.uint16)
+@pytest.mark.parametrize("E,N,K,R", [(3, 128, 256, 8), (3, 384, 256, 16), (2, 1024, 128, 16)])
+def test_requant_weights_per_expert_outer(cuda, E, N, K, R):
+    # expert sizes a power of two (outer scale found by a shift) and not (by a division);
+    # experts six decades apart, so a scale taken from the wrong expert changes codes
+    w = workloads.weights(E, N, K, 0.02, seed=5 + N).float()
+    w *= (10.0 ** torch.linspace(-3, 3, E)).view(E, 1, 1)
+    w = w.to(torch.bfloat16).reshape(E * N, K).view(torch.int16).numpy().view(np.uint16)
     codes, sf, outer = oracle.nvfp4_quantize(w, group_rows=N)
-    oc, oe = oracle.mxfp8_requant_transpose_sr(codes, sf, outer, N, 3, 4, 8)
+    oc, oe = oracle.mxfp8_requant_transpose_sr(codes, sf, outer, N, 3, 4, R)
     gc, ge = api.mxfp8_requant_transpose_sr(torch.from_numpy(codes).cuda(), torch.from_numpy(rowmajor_to_mma(sf)).cuda(),
-                                            torch.from_numpy(outer).cuda(), E * N, K, N, api.MX_SF_MMA, None, 3, 4, 8,
+                                            torch.from_numpy(outer).cuda(), E * N, K, N, api.MX_SF_MMA, None, 3, 4, R,
                                             api.MX_SF_MMA)
     assert np.array_equal(np_(gc), oc)
     assert np.array_equal(mma_to_rowmajor(np_(ge), K, E * N // 32), oe)
