@@ -391,8 +391,9 @@ def run_ours(args):
 
 
 def quantiser_stream(dev, peaks, reps: int = 20):
-    """NVFP4 quantise + MXFP8 stochastic requantise-transpose of the
-    16384x4096 Student-t(4) stream; L2 flushed before every launch."""
+    """NVFP4 quantise, Hadamard + S2F6 quantise and MXFP8 stochastic
+    requantise-transpose of the 16384x4096 Student-t(4) stream; L2 flushed
+    before every launch."""
     import torch
     from fp8_moe_numerics_b200 import api, workloads
     c = workloads.CONFIGS[QUANT_WORKLOAD]
@@ -401,10 +402,13 @@ def quantiser_stream(dev, peaks, reps: int = 20):
     q = api.nvfp4_quantize(x, 1, api.MX_SF_MMA)
     t = api.mxfp8_requant_transpose_sr(*q, rows, cols, 1, api.MX_SF_MMA, None, c["sr_seed"], 0, 16, api.MX_SF_MMA)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    hs = api.hadamard_s2f6_quantize(x, c["sr_seed"], 101)
     res = {}
     for name, fn, nbytes in (
             ("nvfp4_quantize", lambda: api.nvfp4_quantize(x, 1, api.MX_SF_MMA, out=q),
              rows * cols * 2 + rows * cols * (0.5 + 1 / 16) + rows * 4),
+            ("hadamard_s2f6_quantize", lambda: api.hadamard_s2f6_quantize(x, c["sr_seed"], 101, out=hs),
+             rows * cols * 2 + rows * cols * (1 + 1 / 32)),
             ("mxfp8_requant_transpose_sr", lambda: api.mxfp8_requant_transpose_sr(
                 *q, rows, cols, 1, api.MX_SF_MMA, None, c["sr_seed"], 0, 16, api.MX_SF_MMA, out=t),
              rows * cols * (0.5 + 1 / 16) + rows * 4 + rows * cols * (1 + 1 / 32))):
