@@ -474,6 +474,19 @@ __device__ __forceinline__ int s2f6_block_mask(const float* v, uint32_t mask, ui
     return s2f6_finish(P, words);
 }
 
+// The same block read straight from 16 words of bf16 pairs (word q holds
+// values 2q and 2q+1), without first widening all 32 values.
+__device__ __forceinline__ int s2f6_block_mask_bf16(const uint32_t* wq, uint32_t mask, uint32_t* words) {
+    uint64_t P[16];
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+        const float a = __uint_as_float((wq[q] << 16) ^ ((mask << (31 - 2 * q)) & 0x80000000u));
+        const float b = __uint_as_float((wq[q] & 0xffff0000u) ^ ((mask << (30 - 2 * q)) & 0x80000000u));
+        P[q] = f2_pack(__fadd_rn(a, b), __fsub_rn(a, b));
+    }
+    return s2f6_finish(P, words);
+}
+
 // The same block with v first multiplied by `scale`, the signs given as a
 // table sig[i] = +-1.0f (16-byte aligned): x_i = v_i (sig_i scale), which is
 // sig_i RN(v_i scale) exactly.
