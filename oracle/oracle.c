@@ -144,7 +144,7 @@ ORC_API double orc_round_nearest_on_grid(double x, const double* grid, int n) {
 /* 0 and 2 by the two round constants, crosses the high halves with words    */
 /* 1 and 3 and the key, and the key is advanced by the two Weyl constants    */
 /* between rounds.  The pages only say "stochastic rounding"; the generator  */
-/* is this build's reading (a counter-based stream the GPU can reproduce).   */
+/* is a reading taken here (a counter-based stream the GPU can reproduce).   */
 /* ------------------------------------------------------------------------ */
 
 #define PHILOX_M0 0xD2511F53u
