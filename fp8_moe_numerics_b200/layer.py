@@ -218,10 +218,13 @@ def host_stream_steps(layer: ExpertLayer, host_in: dict, host_out: dict, steps: 
     whose outputs go back to it, every step copying its own inputs and results.
 
     host_in holds pinned x, topk, w_comb, dout; host_out pinned out, dx.  Two
-    device buffer sets alternate between steps; a host-to-device stream fills
-    step i+1's inputs and a device-to-host stream drains step i-1's outputs
-    while step i's kernels run on the current stream (the copy engines work
-    beside the SMs).  Everything is enqueued; the caller synchronises.
+    device buffer sets alternate between steps.  A host-to-device stream fills
+    a step's forward inputs (x, topk, w_comb) and then its upstream gradient
+    (dout), so the forward starts before dout has arrived; a device-to-host
+    stream drains the forward output as soon as the forward ends (beside the
+    backward) and dx after the backward.  The copy engines work beside the
+    SMs, so only the first step's forward inputs and the last step's dx are
+    not hidden behind kernels.  Everything is enqueued; the caller synchronises.
     """
     cs = torch.cuda.current_stream()
     up, down = torch.cuda.Stream(), torch.cuda.Stream()
@@ -231,31 +234,40 @@ def host_stream_steps(layer: ExpertLayer, host_in: dict, host_out: dict, steps: 
     for t in list(own.values()) + list(sets[1].values()):
         t.record_stream(up)                                # used beside the allocating stream
         t.record_stream(down)
-    in_ready = [torch.cuda.Event() for _ in range(2)]
-    in_free = [torch.cuda.Event() for _ in range(2)]
-    out_ready = [torch.cuda.Event() for _ in range(2)]
-    out_free = [torch.cuda.Event() for _ in range(2)]
+    ev = lambda: [torch.cuda.Event() for _ in range(2)]
+    fwd_ready, bwd_ready, in_free = ev(), ev(), ev()
+    out_ready, out_free, dx_ready, dx_free = ev(), ev(), ev(), ev()
     for i in range(steps):
         b = i % 2
         buf = sets[b]
         with torch.cuda.stream(up):
             if i >= 2:
                 up.wait_event(in_free[b])                  # step i-2 has read this set
-            for n in ("x", "topk", "w_comb", "dout"):
+            for n in ("x", "topk", "w_comb"):
                 buf[n].copy_(host_in[n], non_blocking=True)
-            in_ready[b].record(up)
-        cs.wait_event(in_ready[b])
-        if i >= 2:
-            cs.wait_event(out_free[b])                     # step i-2's results are on the host
+            fwd_ready[b].record(up)
+            buf["dout"].copy_(host_in["dout"], non_blocking=True)
+            bwd_ready[b].record(up)
         layer.bind_io(buf)
-        layer.step()
-        in_free[b].record(cs)
+        cs.wait_event(fwd_ready[b])
+        if i >= 2:
+            cs.wait_event(out_free[b])                     # step i-2's output is on the host
+        layer.forward()
         out_ready[b].record(cs)
         with torch.cuda.stream(down):
             down.wait_event(out_ready[b])
-            for n in ("out", "dx"):
-                host_out[n].copy_(buf[n], non_blocking=True)
+            host_out["out"].copy_(buf["out"], non_blocking=True)
             out_free[b].record(down)
+        cs.wait_event(bwd_ready[b])
+        if i >= 2:
+            cs.wait_event(dx_free[b])                      # step i-2's dx is on the host
+        layer.backward()
+        in_free[b].record(cs)
+        dx_ready[b].record(cs)
+        with torch.cuda.stream(down):
+            down.wait_event(dx_ready[b])
+            host_out["dx"].copy_(buf["dx"], non_blocking=True)
+            dx_free[b].record(down)
     cs.wait_stream(down)
     layer.bind_io(own)
 
