@@ -106,6 +106,50 @@ def test_grouped_gemm_nvfp4_full_layer_shape(cuda, N, K):
     assert _close_bf16(got, ref)
 
 
+def test_grouped_gemm_nvfp4_s2f6_epilogue_full_layer_shape(cuda):
+    # GEMM2 of the 384-expert layer with the rotate + S2F6 epilogue: sampled
+    # 32-column blocks against the oracle's rotation and quantisation of the
+    # fp64 product (rounded to fp32); codes within one, exponents equal away
+    # from a boundary
+    seg, M_cap = _moe_routing()
+    E, N, K = MOE["E"], MOE["D"], MOE["F"]
+    seed, stream = 5, 101
+    g = torch.Generator(device="cuda")
+    g.manual_seed(77)
+    a = (_rand_u8((M_cap, K // 2), 0, 256, g), _rand_u8((M_cap * K // 16,), 0x28, 0x49, g),
+         torch.rand(M_cap, device="cuda", generator=g) + 0.5)
+    b = (_rand_u8((E * N, K // 2), 0, 256, g), _rand_u8((E * N * K // 16,), 0x28, 0x49, g),
+         torch.rand(E, device="cuda", generator=g) + 0.5)
+    codes, e8 = api.grouped_gemm_nvfp4_s2f6(a, b, torch.from_numpy(seg).cuda(), E, N, K, seed, stream)
+    api.sync_status()
+    rng = np.random.default_rng(3)
+    rows = rng.integers(0, int(seg[E]), 48)
+    blocks = rng.integers(0, N // 32, 48)
+    ex = np.searchsorted(seg, rows, side="right") - 1
+    a_sf, b_sf = np_(a[1]), np_(b[1])
+    a_val = oracle.nvfp4_block_values(np_(a[0][torch.from_numpy(rows).cuda()]), mma_rows(a_sf, rows, K // 16))
+    flips = 0
+    for i, (r, jb, e) in enumerate(zip(rows, blocks, ex)):
+        brow = e * N + 32 * jb + np.arange(32)
+        b_val = oracle.nvfp4_block_values(np_(b[0][torch.from_numpy(brow).cuda()]), mma_rows(b_sf, brow, K // 16))
+        ref = (b_val @ a_val[i]) * float(np_(a[2])[r]) * float(np_(b[2])[e])
+        xrow = np.zeros((1, 32 * (jb + 1)), np.float32)
+        xrow[0, 32 * jb:] = ref.astype(np.float32)
+        rc, re = oracle.s2f6_quantize_hadamard(xrow, seed, stream)
+        gc = np_(codes[int(r), 32 * jb:32 * (jb + 1)]).astype(np.int64)
+        ge = int(np_(e8[int(r), jb]))
+        if ge != int(re[0, jb]):                      # only where the block amax sits on a boundary
+            z = oracle.fwht32_f32(xrow[:, 32 * jb:] * oracle.hadamard_signs(seed, stream, 32 * (jb + 1))[32 * jb:]
+                                  .astype(np.float32))
+            ratio = np.abs(z).max() / np.ldexp(127 / 64, int(re[0, jb]) - 127)
+            assert min(abs(ratio - 1.0), abs(2 * ratio - 1.0)) < 1e-5
+            continue
+        d = np.abs(gc - rc[0, 32 * jb:].astype(np.int64))
+        assert d.max() <= 1
+        flips += int(np.count_nonzero(d))
+    assert flips <= 0.01 * 48 * 32
+
+
 def _rand_e4m3(shape, g):
     """Random E4M3 code bytes without the two NaN codes."""
     c = torch.randint(0, 254, shape, dtype=torch.int32, device="cuda", generator=g)

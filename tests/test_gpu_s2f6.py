@@ -39,6 +39,9 @@ def heavy_rows(rows, cols, seed):
     if rows > 4:
         x[3, :32] = 1e-39                                          # a block of subnormal-range values
         x[4, 32:64] = 5e36                                         # large: the rotation's sums stay finite
+    if rows > 4 and cols >= 96:
+        x[4, 64:96] = 0
+        x[4, 70] = 3.3895e38                                       # one-hot near the bf16 top: e clamps at 127
     return oracle.f32_to_bf16(x.astype(np.float32))
 
 
