@@ -25,10 +25,11 @@ __device__ __forceinline__ uint32_t warp_max_u32(uint32_t v) {
     return v;
 }
 
-// Quantise one 16-element block (two uint4 of bf16) with outer scale s > 0.
-// Returns the E4M3 scale code; writes 8 bytes of packed E2M1 codes.
-__device__ __forceinline__ uint32_t nvfp4_block(const uint4& a, const uint4& b, float s, uint2& packed) {
-    uint32_t ab_bits = max(absmax8_bf16(a), absmax8_bf16(b));
+// Quantise one 16-element block (two uint4 of bf16) with outer scale s > 0;
+// ab_bits = the block's max |x| as bf16 magnitude bits (callers have it from
+// the row amax).  Returns the E4M3 scale code; writes 8 bytes of E2M1 codes.
+__device__ __forceinline__ uint32_t nvfp4_block(const uint4& a, const uint4& b, uint32_t ab_bits, float s,
+                                                uint2& packed) {
     float ab = __uint_as_float(ab_bits << 16);
     float t = __fmul_rn(6.0f, s);
     float d = __fdiv_rn(ab, t);
@@ -59,12 +60,13 @@ __device__ __forceinline__ uint32_t nvfp4_block(const uint4& a, const uint4& b, 
 // when `word_sf`.
 template <int kLayout>
 __device__ __forceinline__ void emit_nvfp4_block(int64_t row, int64_t blk, int64_t nblk, bool active, float s,
-                                                 const uint4& a, const uint4& b, uint8_t* __restrict__ crow,
-                                                 uint8_t* __restrict__ sf, bool word_sf, int lane) {
+                                                 const uint4& a, const uint4& b, uint32_t ab_bits,
+                                                 uint8_t* __restrict__ crow, uint8_t* __restrict__ sf, bool word_sf,
+                                                 int lane) {
     uint2 packed = make_uint2(0u, 0u);
     uint32_t sc = 0;
     const bool live = active && blk < nblk;
-    if (live && s > 0.0f) sc = nvfp4_block(a, b, s, packed);
+    if (live && s > 0.0f) sc = nvfp4_block(a, b, ab_bits, s, packed);
     if (live) *reinterpret_cast<uint2*>(crow + blk * 8) = packed;
     if (word_sf) {
         uint32_t w = sc << (8 * (lane & 3));
@@ -102,6 +104,7 @@ __device__ __forceinline__ void quant_rows_block(const uint16_t* __restrict__ x,
     const uint4* xr = reinterpret_cast<const uint4*>(x + (active ? row : 0) * cols);
 
     uint4 va[kNB], vb[kNB];
+    uint32_t bmax[kNB];                                 // each block's max |x| (bf16 magnitude bits)
     uint32_t amax_bits = 0;
     const bool resident = nblk <= (int64_t)kTPR * kNB;
 #pragma unroll
@@ -115,7 +118,10 @@ __device__ __forceinline__ void quant_rows_block(const uint16_t* __restrict__ x,
         }
     }
 #pragma unroll
-    for (int i = 0; i < kNB; ++i) amax_bits = max(amax_bits, max(absmax8_bf16(va[i]), absmax8_bf16(vb[i])));
+    for (int i = 0; i < kNB; ++i) {
+        bmax[i] = max(absmax8_bf16(va[i]), absmax8_bf16(vb[i]));
+        amax_bits = max(amax_bits, bmax[i]);
+    }
     if (active && !resident) {
         for (int64_t blk = j; blk < nblk; blk += kTPR)
             amax_bits = max(amax_bits, max(absmax8_bf16(xr[2 * blk]), absmax8_bf16(xr[2 * blk + 1])));
@@ -144,17 +150,18 @@ __device__ __forceinline__ void quant_rows_block(const uint16_t* __restrict__ x,
     }
 
     uint8_t* crow = codes + (active ? row : 0) * (cols >> 1);
-    auto emit = [&](int64_t blk, const uint4& a, const uint4& b) {
-        emit_nvfp4_block<kLayout>(row, blk, nblk, active, s, a, b, crow, sf, word_sf, lane);
+    auto emit = [&](int64_t blk, const uint4& a, const uint4& b, uint32_t ab_bits) {
+        emit_nvfp4_block<kLayout>(row, blk, nblk, active, s, a, b, ab_bits, crow, sf, word_sf, lane);
     };
     if (resident) {
 #pragma unroll
-        for (int i = 0; i < kNB; ++i) emit(j + (int64_t)kTPR * i, va[i], vb[i]);
+        for (int i = 0; i < kNB; ++i) emit(j + (int64_t)kTPR * i, va[i], vb[i], bmax[i]);
     } else {
         const int64_t nb_pad = (nblk + kTPR - 1) / kTPR * kTPR;   // every lane runs every shuffle
         for (int64_t blk = j; blk < nb_pad; blk += kTPR) {
             const bool in = active && blk < nblk;
-            emit(blk, in ? xr[2 * blk] : make_uint4(0, 0, 0, 0), in ? xr[2 * blk + 1] : make_uint4(0, 0, 0, 0));
+            const uint4 a = in ? xr[2 * blk] : make_uint4(0, 0, 0, 0), b = in ? xr[2 * blk + 1] : make_uint4(0, 0, 0, 0);
+            emit(blk, a, b, max(absmax8_bf16(a), absmax8_bf16(b)));
         }
     }
 }
@@ -195,6 +202,7 @@ swiglu_nvfp4_rows_kernel(const uint16_t* __restrict__ h, int64_t rows, int64_t F
     const uint4* ur = reinterpret_cast<const uint4*>(h + (live ? row : 0) * hw + F);
     const uint4 one = make_uint4(0x3f803f80u, 0x3f803f80u, 0x3f803f80u, 0x3f803f80u);   // bf16 1.0
     uint4 va[kNB], vb[kNB];
+    uint32_t bmax[kNB];
     uint32_t amax_bits = 0;
 #pragma unroll
     for (int i = 0; i < kNB; ++i) {
@@ -209,7 +217,8 @@ swiglu_nvfp4_rows_kernel(const uint16_t* __restrict__ h, int64_t rows, int64_t F
             vb[i] = make_uint4(swiglu_word(g1.x, u1.x), swiglu_word(g1.y, u1.y), swiglu_word(g1.z, u1.z),
                                swiglu_word(g1.w, u1.w));
         }
-        amax_bits = max(amax_bits, max(absmax8_bf16(va[i]), absmax8_bf16(vb[i])));
+        bmax[i] = max(absmax8_bf16(va[i]), absmax8_bf16(vb[i]));
+        amax_bits = max(amax_bits, bmax[i]);
     }
     if (kTPR >= 32) {
         amax_bits = warp_max_u32(amax_bits);
@@ -229,7 +238,8 @@ swiglu_nvfp4_rows_kernel(const uint16_t* __restrict__ h, int64_t rows, int64_t F
     uint8_t* crow = codes + (active ? row : 0) * (F >> 1);
 #pragma unroll
     for (int i = 0; i < kNB; ++i)
-        emit_nvfp4_block<kLayout>(row, j + (int64_t)kTPR * i, nblk, active, s, va[i], vb[i], crow, sf, word_sf, lane);
+        emit_nvfp4_block<kLayout>(row, j + (int64_t)kTPR * i, nblk, active, s, va[i], vb[i], bmax[i], crow, sf, word_sf,
+                                  lane);
 }
 
 // amax over each group of rows, as fp32 bits, atomically max-ed into outer[g]
