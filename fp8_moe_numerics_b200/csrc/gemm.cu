@@ -1054,6 +1054,7 @@ int mx_make_bf16_tile_map(CUtensorMap* m, const void* base, int64_t rows, int64_
 }
 
 extern "C" int mx_wait_selftest(int64_t limit_us, cudaStream_t stream) {
+    MX_NVTX_RANGE("mx_wait_selftest");
     if (limit_us <= 0 || limit_us > 10 * 1000 * 1000) return MX_EINVAL;
     if (int st = mx_check_device()) return st;
     wait_selftest_kernel<<<1, 32, 0, stream>>>((unsigned long long)limit_us * 1000ull);
@@ -1065,6 +1066,7 @@ extern "C" int grouped_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_sf, c
                                   const uint8_t* b_codes, const uint8_t* b_sf, const float* b_outer,
                                   const int64_t* seg_offsets, int64_t E, int64_t M_cap, int64_t N, int64_t K,
                                   void* out, int out_dtype, cudaStream_t stream) {
+    MX_NVTX_RANGE("grouped_gemm_nvfp4");
     if (((!a_codes || !a_sf || !a_outer || !b_codes || !b_sf || !b_outer || !seg_offsets || !out) && M_cap > 0) || E < 1 ||
         M_cap < 0 || M_cap % 128 || N <= 0 || N % 128 || K <= 0 || K % 256)
         return MX_EINVAL;
@@ -1091,6 +1093,7 @@ extern "C" int grouped_gemm_nvfp4_s2f6(const uint8_t* a_codes, const uint8_t* a_
                                        const int64_t* seg_offsets, int64_t E, int64_t M_cap, int64_t N, int64_t K,
                                        uint64_t seed, uint64_t stream_id, int8_t* codes, uint8_t* e8m0,
                                        cudaStream_t stream) {
+    MX_NVTX_RANGE("grouped_gemm_nvfp4_s2f6");
     if (((!a_codes || !a_sf || !a_outer || !b_codes || !b_sf || !b_outer || !seg_offsets || !codes || !e8m0) &&
          M_cap > 0) || E < 1 || M_cap < 0 || M_cap % 128 || N <= 0 || N % 128 || K <= 0 || K % 256)
         return MX_EINVAL;
@@ -1115,6 +1118,7 @@ extern "C" int grouped_gemm_nvfp4_s2f6(const uint8_t* a_codes, const uint8_t* a_
 extern "C" int grouped_gemm_mxfp8(int mode, const uint8_t* a_codes, const uint8_t* a_e8m0, const uint8_t* b_codes,
                                   const uint8_t* b_e8m0, const int64_t* seg_offsets, int64_t E, int64_t M_cap,
                                   int64_t N, int64_t K, void* out, int out_dtype, cudaStream_t stream) {
+    MX_NVTX_RANGE("grouped_gemm_mxfp8");
     if (((!a_codes || !a_e8m0 || !b_codes || !b_e8m0 || !seg_offsets) && M_cap > 0) || !out || E < 1 || M_cap < 0 ||
         M_cap % 128 ||
         N <= 0 || N % 128 || K <= 0 || K % 128)

@@ -254,6 +254,7 @@ dispatch_grad_kernel(const uint16_t* __restrict__ dout, const int32_t* __restric
 
 extern "C" int moe_route(const int32_t* topk, int64_t T, int64_t k, int64_t E, int64_t M_cap, int64_t* seg_offsets,
                          int32_t* src, int32_t* pos, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+    MX_NVTX_RANGE("moe_route");
     if (((!topk || !pos) && T > 0) || !seg_offsets || !src || T < 0 || k <= 0 || k > 32 || E <= 0 || M_cap < 0 ||
         M_cap % 128)
         return MX_EINVAL;
@@ -282,6 +283,7 @@ extern "C" int moe_route(const int32_t* topk, int64_t T, int64_t k, int64_t E, i
 extern "C" int nvfp4_gather_rows(const uint8_t* codes, const uint8_t* sf, const float* outer, const int32_t* src,
                                  int64_t k, int64_t M_cap, int64_t cols, uint8_t* out_codes, uint8_t* out_sf,
                                  float* out_outer, cudaStream_t stream) {
+    MX_NVTX_RANGE("nvfp4_gather_rows");
     if (((!codes || !sf || !outer || !src || !out_codes || !out_sf || !out_outer) && M_cap > 0) || k <= 0 || M_cap < 0 ||
         M_cap % 128 || cols <= 0 || cols % 64 || !mx_aligned(codes, 16) || !mx_aligned(out_codes, 16) ||
         !mx_aligned(sf, 4) || !mx_aligned(out_sf, 4))
@@ -296,6 +298,7 @@ extern "C" int nvfp4_gather_rows(const uint8_t* codes, const uint8_t* sf, const 
 
 extern "C" int swiglu_fwd(const void* h, int64_t rows, int64_t F, int gated, const int64_t* rows_valid, void* a,
                           cudaStream_t stream) {
+    MX_NVTX_RANGE("swiglu_fwd");
     if (!h || !a || rows < 0 || F <= 0 || F % 8 || !mx_aligned(h, 16) || !mx_aligned(a, 16)) return MX_EINVAL;
     if (int st = mx_check_device()) return st;
     const int64_t n = rows * (F / 8);
@@ -308,6 +311,7 @@ extern "C" int swiglu_fwd(const void* h, int64_t rows, int64_t F, int gated, con
 
 extern "C" int swiglu_bwd(const void* h, const void* da, int64_t rows, int64_t F, int gated, const int64_t* rows_valid,
                           void* dh, cudaStream_t stream) {
+    MX_NVTX_RANGE("swiglu_bwd");
     if (!h || !da || !dh || rows < 0 || F <= 0 || F % 8 || !mx_aligned(h, 16) || !mx_aligned(da, 16) ||
         !mx_aligned(dh, 16))
         return MX_EINVAL;
@@ -323,6 +327,7 @@ extern "C" int swiglu_bwd(const void* h, const void* da, int64_t rows, int64_t F
 
 extern "C" int moe_combine(const void* y, const int32_t* pos, const float* w, int64_t T, int64_t k, int64_t D,
                            void* out, cudaStream_t stream) {
+    MX_NVTX_RANGE("moe_combine");
     if (!y || !pos || !out || T < 0 || k <= 0 || D <= 0 || D % 8 || !mx_aligned(y, 16) || !mx_aligned(out, 16))
         return MX_EINVAL;
     if (int st = mx_check_device()) return st;
@@ -335,6 +340,7 @@ extern "C" int moe_combine(const void* y, const int32_t* pos, const float* w, in
 
 extern "C" int moe_dispatch_grad(const void* dout, const int32_t* src, const int32_t* pos, const float* w, int64_t T,
                                  int64_t k, int64_t M_cap, int64_t D, void* dy, cudaStream_t stream) {
+    MX_NVTX_RANGE("moe_dispatch_grad");
     if (!dout || !src || !pos || !dy || T < 0 || k <= 0 || k > 32 || M_cap < 0 || D <= 0 || D % 8 ||
         !mx_aligned(dout, 16) || !mx_aligned(dy, 16))
         return MX_EINVAL;
@@ -392,6 +398,7 @@ int route_scratch_address(void** out) {
 
 extern "C" int moe_route_static(const int32_t* topk, int64_t T, int64_t k, int64_t E, int64_t M_cap,
                                 int64_t* seg_offsets, int32_t* src, int32_t* pos, cudaStream_t stream) {
+    MX_NVTX_RANGE("moe_route_static");
     if (!topk || !seg_offsets || !src || !pos || T < 0 || k <= 0 || k > 32 || E <= 0 || M_cap < 0 || M_cap % 128)
         return MX_EINVAL;
     if (mx_route_workspace_bytes(T, E) > kRouteStaticScratchBytes) return MX_EINVAL;   // beyond the fixed scratch

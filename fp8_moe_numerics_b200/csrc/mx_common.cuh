@@ -16,6 +16,19 @@
 
 #include "../../include/mxmoe.h"
 
+#include <nvtx3/nvToolsExt.h>
+
+// One NVTX range per C-ABI call, named after the entry point: it marks the
+// call's host side (validation and launches) in profiler timelines and costs
+// a few nanoseconds when no profiling tool is attached (header-only NVTX3).
+struct MxNvtxRange {
+    explicit MxNvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~MxNvtxRange() { nvtxRangePop(); }
+    MxNvtxRange(const MxNvtxRange&) = delete;
+    MxNvtxRange& operator=(const MxNvtxRange&) = delete;
+};
+#define MX_NVTX_RANGE(name) MxNvtxRange mx_nvtx_range_(name)
+
 // ---------------------------------------------------------------------------
 // Host-side status helpers (defined in abi.cu)
 // ---------------------------------------------------------------------------

@@ -730,6 +730,7 @@ int dispatch_layout(int layout, F&& f) {
 
 extern "C" int nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t group_rows, uint8_t* codes,
                               uint8_t* sf, float* outer, int sf_layout, cudaStream_t stream) {
+    MX_NVTX_RANGE("nvfp4_quantize");
     // an empty problem succeeds without touching memory (its pointers may be null)
     if (((!x || !codes || !sf || !outer) && rows > 0) || rows < 0 || cols <= 0 || cols % 16 || group_rows <= 0 ||
         rows % group_rows || !mx_aligned(x, 16) || !mx_aligned(codes, 16))
@@ -781,6 +782,7 @@ extern "C" int nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t
 
 extern "C" int swiglu_nvfp4_quantize(const void* h, int64_t rows, int64_t F, int gated, const int64_t* rows_valid,
                                      uint8_t* codes, uint8_t* sf, float* outer, int sf_layout, cudaStream_t stream) {
+    MX_NVTX_RANGE("swiglu_nvfp4_quantize");
     if (((!h || !codes || !sf || !outer) && rows > 0) || rows < 0 || F <= 0 || F % 16 || F / 16 > 1024 ||
         !mx_aligned(h, 16) || !mx_aligned(codes, 16))
         return MX_EINVAL;
@@ -812,6 +814,7 @@ extern "C" int mxfp8_quantize(const void* x, int64_t rows, int64_t cols, int rou
                               uint64_t stream_id, int rbits, const int64_t* rows_valid,
                               uint8_t* row_codes, uint8_t* row_e8m0, uint8_t* col_codes, uint8_t* col_e8m0,
                               int sf_layout, cudaStream_t stream) {
+    MX_NVTX_RANGE("mxfp8_quantize");
     const bool do_row = row_codes != nullptr, do_col = col_codes != nullptr;
     if ((!x && rows > 0) || rows < 0 || cols <= 0 || rows % kTR || cols % 128 || !mx_aligned(x, 16)) return MX_EINVAL;
     if (rows == 0) return MX_OK;                        // nothing to compute in either form
@@ -875,6 +878,7 @@ extern "C" int mxfp8_requant_transpose_sr(const uint8_t* codes, const uint8_t* s
                                           const int64_t* rows_valid, uint64_t seed, uint64_t stream_id, int rbits,
                                           uint8_t* out_codes, uint8_t* out_e8m0, int out_sf_layout,
                                           cudaStream_t stream) {
+    MX_NVTX_RANGE("mxfp8_requant_transpose_sr");
     if (((!codes || !sf || !outer || !out_codes || !out_e8m0) && rows > 0) || rows < 0 || cols <= 0 || rows % kTR ||
         cols % kTC ||
         group_rows <= 0 || rows % group_rows || !mx_aligned(codes, 16) || !mx_aligned(out_codes, 16))

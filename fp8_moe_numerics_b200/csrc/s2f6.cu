@@ -117,6 +117,7 @@ moe_combine_s2f6_kernel(const uint8_t* __restrict__ codes, const uint8_t* __rest
 
 extern "C" int hadamard_s2f6_quantize(const void* x, int64_t rows, int64_t cols, uint64_t seed, uint64_t stream_id,
                                       int8_t* codes, uint8_t* e8m0, cudaStream_t stream) {
+    MX_NVTX_RANGE("hadamard_s2f6_quantize");
     if (((!x || !codes || !e8m0) && rows > 0) || rows < 0 || cols <= 0 || cols % 32 || !mx_aligned(x, 16) ||
         !mx_aligned(codes, 16))
         return MX_EINVAL;
@@ -132,6 +133,7 @@ extern "C" int hadamard_s2f6_quantize(const void* x, int64_t rows, int64_t cols,
 extern "C" int moe_combine_s2f6(const int8_t* codes, const uint8_t* e8m0, const int32_t* pos, const float* w,
                                 int64_t T, int64_t k, int64_t D, uint64_t seed, uint64_t stream_id, void* out,
                                 cudaStream_t stream) {
+    MX_NVTX_RANGE("moe_combine_s2f6");
     if (((!codes || !e8m0 || !pos || !out) && T > 0) || T < 0 || k < 1 || D <= 0 || D % 32 ||
         !mx_aligned(codes, 16) || !mx_aligned(out, 16))
         return MX_EINVAL;
