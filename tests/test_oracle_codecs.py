@@ -3,8 +3,10 @@
 Each check compares the oracle with something other than itself: closed
 forms, the ml_dtypes package's independent float4/float8 conversions, Triton's
 independent Philox4x32-10 (run on the CPU by its interpreter), exhaustive
-enumeration, and the numbers the pages print.
+enumeration, and the numbers the pages print (tests/golden/pages_worked_examples.json,
+each with its page and section).
 """
+import json
 import os
 import subprocess
 import sys
@@ -87,27 +89,36 @@ def test_negative_values_that_round_to_zero_keep_sign(orc):
     assert orc.e4m3_encode(np.array([0.0], np.float32))[0] == 0x00
 
 
+def _pages(name):
+    """A worked example as the pages print it (tests/golden, with its citation)."""
+    with open(os.path.join(os.path.dirname(__file__), "golden", "pages_worked_examples.json")) as f:
+        return json.load(f)[name]
+
+
 def test_toy_round_to_nearest_example(orc):
     # aibuzzwire "Why Fewer Bits Means Faster Training": a format holding only
     # 3 and 4 stores 3.2 as 3, an error of 0.2.
-    r = orc.round_nearest_on_grid(3.2, [3.0, 4.0])
-    assert r == 3.0
-    assert abs((3.2 - r) - 0.2) < 1e-12
+    ex = _pages("round_to_nearest_toy")
+    r = orc.round_nearest_on_grid(ex["value"], ex["grid"])
+    assert r == ex["stored"]
+    assert abs((ex["value"] - r) - ex["error"]) < 1e-12
 
 
 def test_bits_per_value_of_the_formats(orc):
     # ai-primer "Block scales and per-token activations" table:
     # BF16 16, MXFP8 8.25, NVFP4 4.5 bits per value including block scales;
     # aibuzzwire "Three Formats": NVFP4 stores 3.6x fewer bits than BF16.
+    bits = _pages("bits_per_value")
     rows, cols = 8, 256
     x = orc.f32_to_bf16(np.random.default_rng(0).standard_normal((rows, cols)).astype(np.float32))
     codes, sf, outer = orc.nvfp4_quantize(x)
+    assert sf.shape[1] * _pages("nvfp4_block")["values_per_scale"] == cols
     nvfp4_bits = 8 * (codes.nbytes + sf.nbytes) / x.size
-    assert nvfp4_bits == 4.5
+    assert nvfp4_bits == bits["nvfp4"]
     c8, e8 = orc.mxfp8_quantize_rows(x)
-    assert 8 * (c8.nbytes + e8.nbytes) / x.size == 8.25
-    assert 8 * x.nbytes / x.size == 16
-    assert round(16 / nvfp4_bits, 1) == 3.6
+    assert 8 * (c8.nbytes + e8.nbytes) / x.size == bits["mxfp8"]
+    assert 8 * x.nbytes / x.size == bits["bf16"]
+    assert round(bits["bf16"] / nvfp4_bits, 1) == bits["bf16_over_nvfp4"]
 
 
 # --------------------------------------------------------------------------
@@ -119,11 +130,12 @@ def test_worked_example_4_5_on_fp4_grid(orc, R):
     # ai-primer "Stochastic rounding across transposes": a represented 4.5
     # becomes 4 with probability 0.75 and 6 with probability 0.25, so its
     # expectation stays 4.5.  Enumerate every R-bit random value.
-    vals = np.array([orc.sr_value(4.5, u, R, 1, -1) for u in range(1 << R)])
-    assert set(np.unique(vals)) == {4.0, 6.0}
-    assert np.count_nonzero(vals == 6.0) == (1 << R) // 4
-    assert np.count_nonzero(vals == 4.0) == 3 * (1 << R) // 4
-    assert vals.mean() == 4.5
+    ex = _pages("stochastic_rounding_example")
+    vals = np.array([orc.sr_value(ex["value"], u, R, 1, -1) for u in range(1 << R)])
+    assert set(np.unique(vals)) == {v for v, _ in ex["outcomes"]}
+    for v, p in ex["outcomes"]:
+        assert np.count_nonzero(vals == v) == p * (1 << R)
+    assert vals.mean() == ex["expectation"]
     codes = {orc.e2m1_sr(4.5, u, R) for u in range(1 << R)}
     assert codes == {0x6, 0x7}                   # E2M1 codes of 4 and 6
     neg = np.array([orc.sr_value(-4.5, u, R, 1, -1) for u in range(0, 1 << R, 7)])
