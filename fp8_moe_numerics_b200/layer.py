@@ -207,7 +207,7 @@ class ExpertLayer:
         mark's name (call after synchronising)."""
         out = {}
         for (_, a), (name, b) in zip(self.marks, self.marks[1:]):
-            if name in ("start",):
+            if name in ("start", "bwd_start"):                 # boundaries, not stages
                 continue
             out[name] = out.get(name, 0.0) + a.elapsed_time(b)
         return out

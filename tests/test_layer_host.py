@@ -77,3 +77,33 @@ def test_unfused_swiglu_sequence_passes_host_validation(host_calls):
     assert names.count("nvfp4_quantize") == 4                   # tokens, W1, W2, activations
     assert len(names) == 23
     assert all(st == _lib.MX_ECUDA for _, st in host_calls)
+
+
+@pytest.mark.parametrize("opts", [{}, {"fuse_swiglu": False}, {"combine": "s2f6"}])
+def test_every_marked_stage_has_work_in_bench(host_calls, monkeypatch, opts):
+    # bench.py turns the layer's stage marks into GB/s and TFLOP/s; a stage
+    # without an entry in its work table would be reported without a rate
+    import os
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+
+    class FakeEvent:
+        def __init__(self, **kw):
+            pass
+
+        def record(self, *a):
+            pass
+
+        def elapsed_time(self, other):
+            return 1.0
+    monkeypatch.setattr(torch.cuda, "Event", FakeEvent)
+    inp = workloads.layer_inputs("tiny_layer", device="cpu")
+    c = inp["cfg"]
+    L = ExpertLayer(inp["x"], inp["topk"], inp["w_comb"], inp["w1"], inp["w2"], inp["dout"], gated=c["gated"],
+                    **opts)
+    L.step(record=True)
+    stages = L.stage_times_ms()
+    work = bench.stage_work(c, [c["T"] * c["k"] // c["E"]] * c["E"], L.M_cap)
+    assert set(stages) <= set(work), set(stages) - set(work)
+    assert {"gemm1", "gemm2", "requant_w1", "wgrad1"} <= set(stages)
