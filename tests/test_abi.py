@@ -74,3 +74,35 @@ def test_invalid_arguments_are_rejected_before_launch(mx):
     assert mx.grouped_gemm_mxfp8(5, p, p, p, p, p, 1, 128, 128, 128, p, 0, null) == EINVAL
     # routing capacity too small
     assert mx.moe_route(p, 16, 2, 4, 128, p, p, p, p, 4096, null) == EINVAL
+
+
+def test_c_program_compiles_links_and_calls_the_library(mx, tmp_path):
+    # the boundary from C itself: the header as C99, the library linked by
+    # name, host-side calls that need no GPU
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use.c"
+    src.write_text(
+        '#include "mxmoe.h"\n'
+        '#include <stdio.h>\n'
+        'int main(void) {\n'
+        '    unsigned long long n0 = mx_kernel_launches();\n'
+        '    int bad = nvfp4_quantize(0, 128, 100, 1, 0, 0, 0, MX_SF_ROWMAJOR, 0);  /* cols % 16 != 0 */\n'
+        '    size_t sf = mx_sf_bytes(256, 4096, 16, MX_SF_MMA);\n'
+        '    printf("%d %d %zu %llu\\n", mx_version(), bad, sf, mx_kernel_launches() - n0);\n'
+        '    return 0;\n'
+        '}\n')
+    lib_dir = os.path.join(ROOT, "fp8_moe_numerics_b200")
+    exe = tmp_path / "use"
+    cuda_inc = next((d for d in ("/usr/local/cuda/include", os.environ.get("CUDA_HOME", "") + "/include")
+                     if os.path.exists(os.path.join(d, "cuda_runtime.h"))), None)
+    if cuda_inc is None:
+        pytest.skip("no CUDA headers")
+    subprocess.run([cc, "-std=c99", "-I", os.path.join(ROOT, "include"), "-I", cuda_inc, str(src), "-o", str(exe),
+                    "-L", lib_dir, "-lmxmoe", "-Wl,-rpath," + lib_dir], check=True, capture_output=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    assert int(out[0]) == mx.mx_version() and int(out[1]) == 1          # MX_EINVAL
+    assert int(out[2]) == 256 * 4096 // 16 and int(out[3]) == 0          # nothing launched
