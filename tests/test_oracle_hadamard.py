@@ -57,8 +57,6 @@ def _exponent_by_search(amax):
 @pytest.mark.parametrize("amax", [0.0, 1.0, 127 / 64, np.nextafter(np.float32(127 / 64), np.float32(2)), 2.0, 1.9,
                                   3.0, 127 / 32, 0.75, 1e-30, 1e-40, 2.0 ** -149, 2.0 ** -126, 1e20, 3.0e38,
                                   float(np.finfo(np.float32).max)])
-
-
 def test_exponent_is_the_smallest_that_fits(amax):
     assert oracle.s2f6_exponent(float(np.float32(amax))) == _exponent_by_search(float(np.float32(amax)))
 
