@@ -4,6 +4,12 @@ Argument marshalling only: each function allocates its outputs with torch on
 the inputs' CUDA device, passes raw device pointers and the current CUDA
 stream to the library, and raises MxError on a non-MX_OK status.  Every
 computation happens in the library's sm_100a kernels.
+
+Since the library sees bare pointers, the binding checks what only it can:
+every tensor is contiguous, on the current CUDA device, and holds at least
+the bytes include/mxmoe.h gives for its role (ValueError otherwise, before
+anything is launched).  Index contents (routing rows, segment offsets) are
+not read on the host.
 """
 from __future__ import annotations
 
@@ -19,7 +25,8 @@ __all__ = [
     "MX_SF_ROWMAJOR", "MX_SF_MMA", "MX_ROUND_RNE", "MX_ROUND_SR", "MX_GEMM_DGRAD", "MX_GEMM_WGRAD", "MxError",
     "sf_bytes", "sync_status", "wait_selftest", "nvfp4_quantize", "mxfp8_requant_transpose_sr", "mxfp8_quantize",
     "grouped_gemm_nvfp4", "grouped_gemm_mxfp8", "moe_route", "nvfp4_gather_rows", "swiglu_fwd", "swiglu_bwd",
-    "moe_combine", "moe_dispatch_grad", "swiglu_nvfp4_quantize", "hadamard_s2f6_quantize", "grouped_gemm_nvfp4_s2f6", "moe_combine_s2f6",
+    "moe_combine", "moe_dispatch_grad", "swiglu_nvfp4_quantize", "hadamard_s2f6_quantize", "grouped_gemm_nvfp4_s2f6",
+    "moe_combine_s2f6",
 ]
 
 
@@ -30,7 +37,23 @@ def _p(t) -> ctypes.c_void_p:
         raise ValueError("mxmoe operates on CUDA tensors")
     if not t.is_contiguous():
         raise ValueError("mxmoe expects contiguous tensors")
+    if t.get_device() != torch.cuda.current_device():
+        raise ValueError(f"mxmoe launches on the current device (cuda:{torch.cuda.current_device()}); "
+                         f"a tensor is on cuda:{t.get_device()}")
     return ctypes.c_void_p(t.data_ptr())
+
+
+def _fits(what: str, t, need: int) -> None:
+    """The library receives bare pointers and cannot see a buffer's extent:
+    raise unless tensor `t` (when given) holds the `need` bytes the call
+    reads or writes through it, as include/mxmoe.h sizes them."""
+    if t is not None and t.numel() * t.element_size() < need:
+        raise ValueError(f"{what}: {t.numel() * t.element_size()} bytes, the call needs {need}")
+
+
+def _bf16_2d(what: str, t) -> None:
+    if t.dtype != torch.bfloat16 or t.dim() != 2:
+        raise ValueError(f"{what} must be a 2-D bf16 tensor, got {t.dtype} of {t.dim()} dims")
 
 
 def _s() -> ctypes.c_void_p:
@@ -63,7 +86,7 @@ def wait_selftest(limit_us: int) -> None:
 
 def nvfp4_quantize(x: torch.Tensor, group_rows: int = 1, sf_layout: int = MX_SF_MMA, out=None):
     """bf16 [rows, cols] -> (codes u8 [rows, cols/2], sf u8, outer f32 [rows/group_rows])."""
-    assert x.dtype == torch.bfloat16 and x.dim() == 2
+    _bf16_2d("x", x)
     rows, cols = x.shape
     dev = x.device
     if out is None:
@@ -71,6 +94,9 @@ def nvfp4_quantize(x: torch.Tensor, group_rows: int = 1, sf_layout: int = MX_SF_
                _u8(sf_bytes(rows, cols, 16, sf_layout), dev),
                torch.empty(rows // group_rows, dtype=torch.float32, device=dev))
     codes, sf, outer = out
+    _fits("codes", codes, rows * cols // 2)
+    _fits("sf", sf, rows * (cols // 16))
+    _fits("outer", outer, 4 * (rows // max(group_rows, 1)))
     L.call("nvfp4_quantize", _p(x), rows, cols, group_rows, _p(codes), _p(sf), _p(outer), sf_layout, _s())
     return codes, sf, outer
 
@@ -83,6 +109,12 @@ def mxfp8_requant_transpose_sr(codes, sf, outer, rows: int, cols: int, group_row
     if out is None:
         out = (torch.empty(cols, rows, dtype=torch.uint8, device=dev), _u8(sf_bytes(cols, rows, 32, out_sf_layout), dev))
     oc, oe = out
+    _fits("codes", codes, rows * cols // 2)
+    _fits("sf", sf, rows * (cols // 16))
+    _fits("outer", outer, 4 * (rows // max(group_rows, 1)))
+    _fits("rows_valid", rows_valid, 8)
+    _fits("out codes", oc, rows * cols)
+    _fits("out e8m0", oe, cols * (rows // 32))
     L.call("mxfp8_requant_transpose_sr", _p(codes), _p(sf), _p(outer), rows, cols, group_rows, in_sf_layout,
            _p(rows_valid), ctypes.c_uint64(seed), ctypes.c_uint64(stream_id), rbits, _p(oc), _p(oe),
            out_sf_layout, _s())
@@ -94,7 +126,7 @@ def mxfp8_quantize(x: torch.Tensor, row: bool = True, col: bool = True, rounding
                    sf_layout: int = MX_SF_MMA, out=None):
     """bf16 [rows, cols] -> (row codes [rows, cols], row E8M0, col codes [cols, rows], col E8M0);
     the forms not requested are None."""
-    assert x.dtype == torch.bfloat16 and x.dim() == 2
+    _bf16_2d("x", x)
     rows, cols = x.shape
     dev = x.device
     if out is None:
@@ -103,6 +135,11 @@ def mxfp8_quantize(x: torch.Tensor, row: bool = True, col: bool = True, rounding
                torch.empty(cols, rows, dtype=torch.uint8, device=dev) if col else None,
                _u8(sf_bytes(cols, rows, 32, sf_layout), dev) if col else None)
     rc, re, cc, ce = out
+    _fits("row codes", rc, rows * cols)
+    _fits("row e8m0", re, rows * (cols // 32))
+    _fits("col codes", cc, rows * cols)
+    _fits("col e8m0", ce, cols * (rows // 32))
+    _fits("rows_valid", rows_valid, 8)
     L.call("mxfp8_quantize", _p(x), rows, cols, rounding, ctypes.c_uint64(seed), ctypes.c_uint64(stream_id), rbits,
            _p(rows_valid), _p(rc), _p(re), _p(cc), _p(ce), sf_layout, _s())
     return rc, re, cc, ce
@@ -116,12 +153,24 @@ def _out_code(dtype) -> int:
     raise ValueError(dtype)
 
 
+def _nvfp4_operands_fit(a, b, seg, E: int, M_cap: int, N: int, K: int) -> None:
+    _fits("a codes", a[0], M_cap * K // 2)
+    _fits("a sf", a[1], M_cap * (K // 16))
+    _fits("a outer", a[2], 4 * M_cap)
+    _fits("b codes", b[0], E * N * K // 2)
+    _fits("b sf", b[1], E * N * (K // 16))
+    _fits("b outer", b[2], 4 * E)
+    _fits("seg", seg, 8 * (E + 1))
+
+
 def grouped_gemm_nvfp4(a, b, seg: torch.Tensor, E: int, N: int, K: int, out_dtype=torch.bfloat16, out=None):
     """a = (codes [M_cap, K/2], sf, outer [M_cap]); b = (codes [E*N, K/2], sf, outer [E]).
     Returns out [M_cap, N]; rows >= seg[E] are not written."""
     M_cap = a[0].shape[0]
     if out is None:
         out = torch.empty(M_cap, N, dtype=out_dtype, device=a[0].device)
+    _nvfp4_operands_fit(a, b, seg, E, M_cap, N, K)
+    _fits("out", out, M_cap * N * out.element_size())
     L.call("grouped_gemm_nvfp4", _p(a[0]), _p(a[1]), _p(a[2]), _p(b[0]), _p(b[1]), _p(b[2]), _p(seg), E, M_cap, N,
            K, _p(out), _out_code(out.dtype), _s())
     return out
@@ -134,6 +183,19 @@ def grouped_gemm_mxfp8(mode: int, a_codes, a_e8m0, b_codes, b_e8m0, seg: torch.T
     if out is None:
         shape = (M_cap, N) if mode == MX_GEMM_DGRAD else (E, N, K)
         out = torch.empty(*shape, dtype=out_dtype, device=a_codes.device)
+    if mode == MX_GEMM_DGRAD:
+        _fits("a codes", a_codes, M_cap * K)
+        _fits("a e8m0", a_e8m0, M_cap * (K // 32))
+        _fits("b codes", b_codes, N * E * K)
+        _fits("b e8m0", b_e8m0, N * (E * K // 32))
+        _fits("out", out, M_cap * N * out.element_size())
+    else:
+        _fits("a codes", a_codes, N * M_cap)
+        _fits("a e8m0", a_e8m0, N * (M_cap // 32))
+        _fits("b codes", b_codes, K * M_cap)
+        _fits("b e8m0", b_e8m0, K * (M_cap // 32))
+        _fits("out", out, E * N * K * out.element_size())
+    _fits("seg", seg, 8 * (E + 1))
     L.call("grouped_gemm_mxfp8", mode, _p(a_codes), _p(a_e8m0), _p(b_codes), _p(b_e8m0), _p(seg), E, M_cap, N, K,
            _p(out), _out_code(out.dtype), _s())
     return out
@@ -155,7 +217,11 @@ def moe_route(topk: torch.Tensor, E: int, M_cap: int | None = None, out=None):
         out = (torch.empty(E + 1, dtype=torch.int64, device=dev), torch.empty(M_cap, dtype=torch.int32, device=dev),
                torch.empty(T, k, dtype=torch.int32, device=dev), _u8(max(ws_bytes, 16), dev))
     seg, src, pos, ws = out
-    L.call("moe_route", _p(topk), T, k, E, M_cap, _p(seg), _p(src), _p(pos), _p(ws), ws.numel(), _s())
+    _fits("seg", seg, 8 * (E + 1))
+    _fits("src", src, 4 * M_cap)
+    _fits("pos", pos, 4 * T * k)
+    L.call("moe_route", _p(topk), T, k, E, M_cap, _p(seg), _p(src), _p(pos), _p(ws), ws.numel() * ws.element_size(),
+           _s())
     return seg, src, pos
 
 
@@ -166,6 +232,9 @@ def nvfp4_gather_rows(codes, sf_rowmajor, outer, src: torch.Tensor, k: int, cols
         out = (torch.empty(M_cap, cols // 2, dtype=torch.uint8, device=dev), _u8(sf_bytes(M_cap, cols, 16, MX_SF_MMA), dev),
                torch.empty(M_cap, dtype=torch.float32, device=dev))
     oc, osf, oo = out
+    _fits("out codes", oc, M_cap * cols // 2)
+    _fits("out sf", osf, M_cap * (cols // 16))
+    _fits("out outer", oo, 4 * M_cap)
     L.call("nvfp4_gather_rows", _p(codes), _p(sf_rowmajor), _p(outer), _p(src), k, M_cap, cols, _p(oc), _p(osf),
            _p(oo), _s())
     return oc, osf, oo
@@ -175,6 +244,9 @@ def swiglu_fwd(h: torch.Tensor, F: int, gated: bool = True, rows_valid=None, out
     rows = h.shape[0]
     if out is None:
         out = torch.empty(rows, F, dtype=torch.bfloat16, device=h.device)
+    _fits("h", h, rows * (2 * F if gated else F) * 2)
+    _fits("a", out, rows * F * 2)
+    _fits("rows_valid", rows_valid, 8)
     L.call("swiglu_fwd", _p(h), rows, F, int(gated), _p(rows_valid), _p(out), _s())
     return out
 
@@ -183,6 +255,10 @@ def swiglu_bwd(h: torch.Tensor, da: torch.Tensor, F: int, gated: bool = True, ro
     rows = h.shape[0]
     if out is None:
         out = torch.empty_like(h)
+    _fits("h", h, rows * (2 * F if gated else F) * 2)
+    _fits("da", da, rows * F * 2)
+    _fits("dh", out, rows * (2 * F if gated else F) * 2)
+    _fits("rows_valid", rows_valid, 8)
     L.call("swiglu_bwd", _p(h), _p(da), rows, F, int(gated), _p(rows_valid), _p(out), _s())
     return out
 
@@ -191,6 +267,8 @@ def moe_combine(y: torch.Tensor, pos: torch.Tensor, w, D: int, out=None):
     T, k = pos.shape
     if out is None:
         out = torch.empty(T, D, dtype=torch.bfloat16, device=y.device)
+    _fits("w", w, 4 * T * k)
+    _fits("out", out, T * D * 2)
     L.call("moe_combine", _p(y), _p(pos), _p(w), T, k, D, _p(out), _s())
     return out
 
@@ -202,6 +280,9 @@ def moe_dispatch_grad(dout: torch.Tensor, src: torch.Tensor, pos: torch.Tensor, 
     D = dout.shape[1]
     if out is None:
         out = torch.empty(M_cap, D, dtype=torch.bfloat16, device=dout.device)
+    _fits("dout", dout, T * D * 2)
+    _fits("w", w, 4 * T * k)
+    _fits("dy", out, M_cap * D * 2)
     L.call("moe_dispatch_grad", _p(dout), _p(src), _p(pos), _p(w), T, k, M_cap, D, _p(out), _s())
     return out
 
@@ -209,12 +290,14 @@ def moe_dispatch_grad(dout: torch.Tensor, src: torch.Tensor, pos: torch.Tensor, 
 def hadamard_s2f6_quantize(x: torch.Tensor, seed: int, stream_id: int, out=None):
     """bf16 [rows, cols] -> (codes int8 [rows, cols], e8m0 u8 [rows, cols/32]):
     32-d random Hadamard rotation per column block, block-scaled S2F6."""
-    assert x.dtype == torch.bfloat16 and x.dim() == 2
+    _bf16_2d("x", x)
     rows, cols = x.shape
     if out is None:
         out = (torch.empty(rows, cols, dtype=torch.int8, device=x.device),
                torch.empty(rows, cols // 32, dtype=torch.uint8, device=x.device))
     codes, e8m0 = out
+    _fits("codes", codes, rows * cols)
+    _fits("e8m0", e8m0, rows * (cols // 32))
     L.call("hadamard_s2f6_quantize", _p(x), rows, cols, seed, stream_id, _p(codes), _p(e8m0), _s())
     return codes, e8m0
 
@@ -226,6 +309,9 @@ def grouped_gemm_nvfp4_s2f6(a, b, seg: torch.Tensor, E: int, N: int, K: int, see
         out = (torch.empty(M_cap, N, dtype=torch.int8, device=a[0].device),
                torch.empty(M_cap, N // 32, dtype=torch.uint8, device=a[0].device))
     codes, e8m0 = out
+    _nvfp4_operands_fit(a, b, seg, E, M_cap, N, K)
+    _fits("codes", codes, M_cap * N)
+    _fits("e8m0", e8m0, M_cap * (N // 32))
     L.call("grouped_gemm_nvfp4_s2f6", _p(a[0]), _p(a[1]), _p(a[2]), _p(b[0]), _p(b[1]), _p(b[2]), _p(seg), E, M_cap,
            N, K, seed, stream_id, _p(codes), _p(e8m0), _s())
     return codes, e8m0
@@ -238,6 +324,9 @@ def moe_combine_s2f6(codes: torch.Tensor, e8m0: torch.Tensor, pos: torch.Tensor,
     D = codes.shape[1]
     if out is None:
         out = torch.empty(T, D, dtype=torch.bfloat16, device=codes.device)
+    _fits("e8m0", e8m0, codes.shape[0] * (D // 32))
+    _fits("w", w, 4 * T * k)
+    _fits("out", out, T * D * 2)
     L.call("moe_combine_s2f6", _p(codes), _p(e8m0), _p(pos), _p(w), T, k, D, seed, stream_id, _p(out), _s())
     return out
 
@@ -246,13 +335,18 @@ def swiglu_nvfp4_quantize(h: torch.Tensor, F: int, gated: bool = True, rows_vali
                           out=None):
     """SwiGLU of h (bf16 [rows, 2F] or [rows, F]) quantised to NVFP4 per token:
     (codes u8 [rows, F/2], sf u8, outer f32 [rows])."""
-    assert h.dtype == torch.bfloat16 and h.dim() == 2
+    _bf16_2d("h", h)
     rows = h.shape[0]
     if out is None:
         out = (torch.empty(rows, F // 2, dtype=torch.uint8, device=h.device),
                _u8(sf_bytes(rows, F, 16, sf_layout), h.device),
                torch.empty(rows, dtype=torch.float32, device=h.device))
     codes, sf, outer = out
+    _fits("h", h, rows * (2 * F if gated else F) * 2)
+    _fits("codes", codes, rows * F // 2)
+    _fits("sf", sf, rows * (F // 16))
+    _fits("outer", outer, 4 * rows)
+    _fits("rows_valid", rows_valid, 8)
     L.call("swiglu_nvfp4_quantize", _p(h), rows, F, int(gated), _p(rows_valid), _p(codes), _p(sf), _p(outer),
            sf_layout, _s())
     return codes, sf, outer

@@ -50,7 +50,8 @@ class ExpertLayer:
     def __init__(self, x, topk, w_comb, w1, w2, dout, gated: bool = True, seed: int = 0,
                  wgrad_dtype=torch.bfloat16, out_dtype=torch.bfloat16, rbits: int = 16, combine: str = "bf16",
                  fuse_swiglu: bool = True):
-        assert combine in ("bf16", "s2f6")
+        if combine not in ("bf16", "s2f6"):
+            raise ValueError(f"combine must be 'bf16' or 's2f6', got {combine!r}")
         self.combine = combine
         self.fuse_swiglu = fuse_swiglu
         dev = x.device
@@ -60,7 +61,9 @@ class ExpertLayer:
         self.E, self.N1, _ = w1.shape
         self.F = w2.shape[2]
         self.gated = gated
-        assert self.N1 == (2 * self.F if gated else self.F)
+        if self.N1 != (2 * self.F if gated else self.F):
+            raise ValueError(f"w1 has {self.N1} rows per expert; {'2F' if gated else 'F'} = "
+                             f"{2 * self.F if gated else self.F} expected")
         self.seed, self.rbits = seed, rbits
         self.x, self.topk, self.w_comb, self.w1, self.w2, self.dout = x, topk, w_comb, w1, w2, dout
         T, D, k, E, F, N1 = self.T, self.D, self.k, self.E, self.F, self.N1
@@ -124,7 +127,9 @@ class ExpertLayer:
         the per-step inputs and outputs (weights and intermediates stay)."""
         for n in self.IO:
             t = bufs[n]
-            assert t.shape == getattr(self, n).shape and t.dtype == getattr(self, n).dtype, n
+            if t.shape != getattr(self, n).shape or t.dtype != getattr(self, n).dtype:
+                raise ValueError(f"{n}: {tuple(t.shape)} {t.dtype}, the layer was built for "
+                                 f"{tuple(getattr(self, n).shape)} {getattr(self, n).dtype}")
             setattr(self, n, t)
 
     # ----------------------------------------------------------------- forward
