@@ -90,6 +90,36 @@ def test_grouped_gemm_mxfp8_dgrad_and_wgrad_brute_force(orc):
             assert abs(W[1, n, k] - ref) <= 1e-12 * max(1, abs(ref))
 
 
+def test_grouped_gemm_mxfp8_experts_past_the_first_segment(orc):
+    # two non-empty experts around an empty one, the later one 1000x larger:
+    # each expert's operands and scales sit at its own token or column offset
+    rng = np.random.default_rng(15)
+    E, Kc, Nout, Nw, Kw = 3, 64, 8, 4, 6
+    seg = np.array([0, 64, 64, 160], dtype=np.int64)
+    M = 160
+    mag = np.where(np.arange(M) >= 64, 1000.0, 1.0)[:, None]
+    a_c, a_e = orc.mxfp8_quantize_rows(orc.f32_to_bf16((rng.standard_normal((M, Kc)) * mag).astype(np.float32)))
+    bw = rng.standard_normal((Nout, E * Kc)) * np.repeat([1.0, 7.0, 1000.0], Kc)[None, :]
+    b_c, b_e = orc.mxfp8_quantize_rows(orc.f32_to_bf16(bw.astype(np.float32)))
+    C = orc.grouped_gemm_mxfp8_dgrad(a_c, a_e, b_c, b_e, seg)
+    A, B = _decode_mxfp8_ml(a_c, a_e), _decode_mxfp8_ml(b_c, b_e)
+    for r in range(M):
+        e = 0 if r < 64 else 2
+        for n in range(Nout):
+            ref = sum(A[r, k] * B[n, e * Kc + k] for k in range(Kc))
+            assert abs(C[r, n] - ref) <= 1e-12 * max(1, abs(ref))
+    wa_c, wa_e = orc.mxfp8_quantize_cols(orc.f32_to_bf16((rng.standard_normal((M, Nw)) * mag).astype(np.float32)))
+    wb_c, wb_e = orc.mxfp8_quantize_cols(orc.f32_to_bf16(rng.standard_normal((M, Kw)).astype(np.float32)))
+    W = orc.grouped_gemm_mxfp8_wgrad(wa_c, wa_e, wb_c, wb_e, seg)
+    assert np.all(W[1] == 0)
+    WA, WB = _decode_mxfp8_ml(wa_c, wa_e), _decode_mxfp8_ml(wb_c, wb_e)
+    for e, (t0, t1) in ((0, (0, 64)), (2, (64, 160))):
+        for n in range(Nw):
+            for k in range(Kw):
+                ref = sum(WA[n, t] * WB[k, t] for t in range(t0, t1))
+                assert abs(W[e, n, k] - ref) <= 1e-12 * max(1, abs(ref))
+
+
 def test_integer_exact_gemm_case(orc):
     # Power-of-two scales and small integer products: the fp64 sum is exact.
     E, N, K, M = 1, 4, 64, 4
