@@ -35,7 +35,9 @@ Parity pins (tests/test_oracle_*.py):
                       integer vectors; H32 H32 = 32 I; exponent by search
                       over all exponents; ties to even; one-hot outlier
                       closed form; reconstruction error bound; combine loops
-No oracle function is "parity unpinned".
+No oracle function is "parity unpinned".  tests/test_oracle_mutants.py plants
+plausible mistakes in a copy of this package and checks that a pin fails on
+each.
 """
 from __future__ import annotations
 
