@@ -17,6 +17,26 @@ import numpy as np
 import pytest
 
 
+def test_f32_to_bf16_matches_ml_dtypes_on_ties(orc):
+    # exact ties (dropped half 0x8000) above even and odd kept bits, their
+    # neighbours, values that overflow to infinity, and random finite patterns;
+    # ml_dtypes' bfloat16 conversion rounds to nearest even independently
+    rng = np.random.default_rng(31)
+    hi = rng.integers(0, 0x7F7F, 4000, dtype=np.uint32)
+    sign = rng.integers(0, 2, 4000, dtype=np.uint32) << 31
+    pats = [(hi << 16) | d | sign for d in (0x8000, 0x7FFF, 0x8001, 0x0000, 0xFFFF)]
+    pats.append(np.array([0x7F7FFFFF, 0x7F7F8000, 0x7F7F7FFF, 0xFF7FFFFF, 0x00008000, 0x00018000,
+                          0x80008000], dtype=np.uint32))
+    finite = rng.integers(0, 0xFFFFFFFF, 20000, dtype=np.uint64, endpoint=True).astype(np.uint32)
+    pats.append(finite[(finite & 0x7F800000) != 0x7F800000])
+    x = np.concatenate(pats).view(np.float32)
+    want = x.astype(ml_dtypes.bfloat16).view(np.uint16)
+    assert np.array_equal(orc.f32_to_bf16(x), want)
+    lib = orc.lib()
+    got_c = np.array([lib.orc_f32_to_bf16(float(v)) for v in x], dtype=np.uint16)
+    assert np.array_equal(got_c, want)
+
+
 def test_e2m1_decode_table_closed_form_and_ml_dtypes(orc):
     t = orc.e2m1_decode_table()
     expect = np.array([0, .5, 1, 1.5, 2, 3, 4, 6], dtype=np.float32)

@@ -45,6 +45,29 @@ MUTANTS = [
     ("dequantisation drops the outer scale", "oracle.c",
      "return nvfp4_block_product(codes, sf, cols, r, c) * outer[r / group_rows];",
      "return nvfp4_block_product(codes, sf, cols, r, c);", [QUANT]),
+    ("E4M3 stochastic rounding with two mantissa bits", "oracle.c",
+     "double v = orc_sr_value(y, u, R, 3, -9);", "double v = orc_sr_value(y, u, R, 2, -9);", [CODECS]),
+    ("E4M3 stochastic rounding with the subnormal step one binade high", "oracle.c",
+     "double v = orc_sr_value(y, u, R, 3, -9);", "double v = orc_sr_value(y, u, R, 3, -8);", [CODECS, QUANT]),
+    ("Philox multiplies the wrong counter word", "oracle.c",
+     "uint64_t p1 = (uint64_t)PHILOX_M1 * c2;", "uint64_t p1 = (uint64_t)PHILOX_M1 * c1;", [CODECS]),
+    ("E8M0 decode with bias 128", "oracle.c",
+     "return ldexp(1.0, (int)c - 127);", "return ldexp(1.0, (int)c - 128);", [CODECS]),
+    ("fp32 -> bf16 rounds ties up", "oracle.c",
+     "u += 0x7fffu + lsb;", "u += 0x7fffu;", [CODECS, QUANT]),
+    ("NVFP4 packs element 2j in the high nibble", "oracle.c",
+     "cb[i / 2] = (uint8_t)(orc_e2m1_encode(v0) | (orc_e2m1_encode(v1) << 4));",
+     "cb[i / 2] = (uint8_t)(orc_e2m1_encode(v1) | (orc_e2m1_encode(v0) << 4));", [QUANT]),
+    ("NVFP4 block values read the scale of block c/32", "oracle.c",
+     "(double)orc_e4m3_decode(sf[r * (cols / 16) + c / 16]);",
+     "(double)orc_e4m3_decode(sf[r * (cols / 16) + c / 32]);", [GEMM]),
+    ("MXFP8 dequantisation uses each row's first scale", "oracle.c",
+     "orc_e8m0_decode(e8m0[r * nb + c / 32]);", "orc_e8m0_decode(e8m0[r * nb]);", [GEMM, QUANT]),
+    ("column-wise MXFP8 takes amax over the transposed index", "oracle.c",
+     "double a = fabs((double)bf16_to_f32(x[(b * 32 + t) * cols + c]));",
+     "double a = fabs((double)bf16_to_f32(x[c * rows + b * 32 + t]));", [QUANT]),
+    ("requantisation writes E8M0 with bias 126", "oracle.c",
+     "out_e8m0[c * nb + b] = (uint8_t)(e + 127);", "out_e8m0[c * nb + b] = (uint8_t)(e + 126);", [QUANT]),
     # __init__.py: GEMM references and glue
     ("NVFP4 GEMM drops the expert's outer scale", "__init__.py",
      "* a_outer[r0:r1, None].astype(np.float64) * float(b_outer[e])",
@@ -66,6 +89,15 @@ MUTANTS = [
      'out = np.einsum("tj,tjd->td", w.astype(np.float64), y[pos])', "out = y[pos].sum(axis=1)", [GEMM]),
     ("combine gradient drops the routing weights", "__init__.py",
      "dy[pos[:, j]] = w[:, j, None].astype(np.float64) * d", "dy[pos[:, j]] = d", [GEMM]),
+    ("numpy fp32 -> bf16 rounds ties up", "__init__.py",
+     "u = u + 0x7FFF + ((u >> 16) & 1)", "u = u + 0x7FFF", [CODECS, QUANT, GEMM]),
+    ("fp64 -> bf16 rounds ties away from zero", "__init__.py",
+     "r = np.ldexp(np.rint(np.ldexp(m, 8)), e - 8)",
+     "r = np.ldexp(np.trunc(np.ldexp(m, 8) + np.copysign(0.5, m)), e - 8)", [GEMM]),
+    ("expert segments not padded to 128 rows", "__init__.py",
+     "padded = (counts + align - 1) // align * align", "padded = counts", [GEMM]),
+    ("S2F6 codes may reach -128", "__init__.py",
+     "c = np.clip(np.rint(y), -127, 127).astype(np.int8)", "c = np.clip(np.rint(y), -128, 127).astype(np.int8)", [HAD]),
     # __init__.py: Hadamard rotation and S2F6
     ("butterfly difference with the wrong sign", "__init__.py",
      "z = np.stack([a + b, a - b], axis=-2)", "z = np.stack([a + b, b - a], axis=-2)", [HAD]),
