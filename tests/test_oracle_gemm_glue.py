@@ -120,6 +120,28 @@ def test_grouped_gemm_mxfp8_experts_past_the_first_segment(orc):
                 assert abs(W[e, n, k] - ref) <= 1e-12 * max(1, abs(ref))
 
 
+def test_gather_puts_each_token_at_its_routed_rows(orc):
+    # after routing, row pos[t, j] of the gathered tensor is token t's
+    # quantised row, bit for bit (codes, block scales, outer scale) and so
+    # decodes to the same values; every other row is a zero padding row
+    rng = np.random.default_rng(17)
+    T, k, E, cols = 40, 3, 5, 64
+    topk = np.stack([rng.choice(E, k, replace=False) for _ in range(T)]).astype(np.int32)
+    seg, src, pos = orc.route(topk, E)
+    codes, sf, outer = _q_nvfp4(orc, T, cols, 18)
+    gc, gsf, go = orc.gather_nvfp4_rows(codes, sf, outer, src)
+    assert gc.shape == (int(seg[-1]), cols // 2) and gsf.shape == (int(seg[-1]), cols // 16)
+    used = np.zeros(int(seg[-1]), bool)
+    for t in range(T):
+        for j in range(k):
+            p = int(pos[t, j])
+            used[p] = True
+            assert np.array_equal(gc[p], codes[t]) and np.array_equal(gsf[p], sf[t]) and go[p] == outer[t]
+    assert np.all(gc[~used] == 0) and np.all(gsf[~used] == 0) and np.all(go[~used] == 0)
+    deq = orc.nvfp4_dequantize(gc, gsf, go)
+    assert np.array_equal(deq[pos.reshape(-1)], orc.nvfp4_dequantize(codes, sf, outer)[np.repeat(np.arange(T), k)])
+
+
 def test_integer_exact_gemm_case(orc):
     # Power-of-two scales and small integer products: the fp64 sum is exact.
     E, N, K, M = 1, 4, 64, 4

@@ -98,6 +98,15 @@ MUTANTS = [
      "padded = (counts + align - 1) // align * align", "padded = counts", [GEMM]),
     ("S2F6 codes may reach -128", "__init__.py",
      "c = np.clip(np.rint(y), -127, 127).astype(np.int8)", "c = np.clip(np.rint(y), -128, 127).astype(np.int8)", [HAD]),
+    ("gather takes the block scales of the previous token", "__init__.py",
+     "osf[ok] = sf[src[ok]]", "osf[ok] = sf[np.maximum(src[ok] - 1, 0)]", [GEMM]),
+    ("gather drops the outer scale", "__init__.py",
+     "oo[ok] = outer[src[ok]]", "oo[ok] = 1.0", [GEMM]),
+    ("sampled NVFP4 GEMM reads expert 0's weight rows", "__init__.py",
+     "b = nvfp4_block_values(b_codes[e * N + n:e * N + n + 1], b_sf[e * N + n:e * N + n + 1])[0]",
+     "b = nvfp4_block_values(b_codes[n:n + 1], b_sf[n:n + 1])[0]", [GEMM]),
+    ("single requantised entry draws the bits of the wrong index", "__init__.py",
+     "L = col * rows + row0 + t", "L = col * rows + t", [QUANT]),
     # __init__.py: Hadamard rotation and S2F6
     ("butterfly difference with the wrong sign", "__init__.py",
      "z = np.stack([a + b, a - b], axis=-2)", "z = np.stack([a + b, b - a], axis=-2)", [HAD]),
