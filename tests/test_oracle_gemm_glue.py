@@ -191,6 +191,12 @@ def test_silu_swiglu_against_torch(orc):
     (torch.nn.functional.silu(hv[:, :8]) * hv[:, 8:] * daf).sum().backward()
     dh = orc.bf16_to_f32(orc.swiglu_bwd(h, da, gated=True)).astype(np.float64)
     assert np.allclose(dh, hv.grad.numpy(), rtol=2 ** -8, atol=1e-30)
+    # ungated backward: autograd of silu(h)
+    da1 = orc.f32_to_bf16(rng.standard_normal((5, 16)).astype(np.float32))
+    hv1 = hf.clone().requires_grad_(True)
+    (torch.nn.functional.silu(hv1) * torch.from_numpy(orc.bf16_to_f32(da1).astype(np.float64))).sum().backward()
+    dh1 = orc.bf16_to_f32(orc.swiglu_bwd(h, da1, gated=False)).astype(np.float64)
+    assert np.allclose(dh1, hv1.grad.numpy(), rtol=2 ** -8, atol=1e-30)
     assert orc.bf16_to_f32(orc.swiglu_fwd(orc.f32_to_bf16(np.zeros((1, 2), np.float32)), True))[0, 0] == 0
 
 

@@ -85,6 +85,10 @@ MUTANTS = [
      "a = _silu(h[:, :F]) * h[:, F:]", "a = _silu(h[:, F:]) * h[:, :F]", [GEMM]),
     ("SiLU derivative with a wrong sign", "__init__.py",
      "return s * (1.0 + g * (1.0 - s))", "return s * (1.0 - g * (1.0 - s))", [GEMM]),
+    ("ungated activation squares the SiLU input", "__init__.py",
+     "        a = _silu(h)\n", "        a = h * _silu(h)\n", [GEMM]),
+    ("ungated backward uses SiLU instead of its derivative", "__init__.py",
+     "dh = da * _dsilu(h)", "dh = da * _silu(h)", [GEMM]),
     ("combine drops the routing weights", "__init__.py",
      'out = np.einsum("tj,tjd->td", w.astype(np.float64), y[pos])', "out = y[pos].sum(axis=1)", [GEMM]),
     ("combine gradient drops the routing weights", "__init__.py",
