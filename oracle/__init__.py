@@ -31,6 +31,11 @@ Parity pins (tests/test_oracle_*.py):
   GEMMs ............. brute-force loops on tiny inputs; plain matmul special
                       cases; empty experts
   glue .............. brute-force permutation; SiLU vs torch; combine loops
+  nvfp4 backward .... equal to the forward quantiser without SR; grid
+                      neighbours and the 4.5 example with SR; the regrouping
+                      example across the transpose; unbiasedness over
+                      streams; brute-force dgrad/wgrad; the 16x16 tile's
+                      outlier statement and orientation invariance
   hadamard / s2f6 ... butterflies vs the Kronecker-built Sylvester matrix on
                       integer vectors; H32 H32 = 32 I; exponent by search
                       over all exponents; ties to even; one-hot outlier
@@ -104,6 +109,8 @@ def _declare(L: ctypes.CDLL) -> None:
         "orc_mxfp8_quantize_rows": (None, [P, I64, I64, I32, U64, U64, I32, P, P]),
         "orc_mxfp8_quantize_cols": (None, [P, I64, I64, I32, U64, U64, I32, P, P]),
         "orc_mxfp8_dequantize": (None, [P, P, I64, I64, P]),
+        "orc_nvfp4_quantize_f32": (None, [P, I64, I64, I64, I32, U64, U64, I32, P, P, P]),
+        "orc_nvfp4_quantize_tile16": (None, [P, I64, I64, I64, P, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -381,6 +388,108 @@ def grouped_gemm_mxfp8_wgrad(a_codes, a_e8, b_codes, b_e8, seg) -> np.ndarray:
         Bv = mxfp8_dequantize(np.ascontiguousarray(b_codes[:, t0:t1]), np.ascontiguousarray(b_e8[:, t0 // 32:t1 // 32]))
         C[e] = Av @ Bv.T
     return C
+
+
+# --------------------------------------------------------------------------
+# NVFP4 in the backward pass (the pages' stated future work) and the rejected
+# 16x16 shared-scale alternative.  [ai-primer §NVFP4 forward, MXFP8 backward]:
+# the lab is exploring four-bit arithmetic in the backward pass; [ai-primer
+# §Stochastic rounding across transposes]: a scale shared by each 16x16 tile
+# proved too sensitive to outliers.  Readings taken (pages silent):
+#   quantiser   the NVFP4 scale rules of the forward quantiser on fp32 input,
+#               element codes rounded stochastically (E2M1, random integer of
+#               the linear output index), see orc_nvfp4_quantize_f32;
+#   requant     dequantise ((q sf) s in fp32), transpose, re-quantise to NVFP4
+#               with SR; the transposed tensor takes one outer scale per row
+#               (per feature) for activations and gradients, one per expert
+#               for an expert weight stack, so that in every backward GEMM
+#               both outer scales factor out of the contraction;
+#   dgrad       dX = dY W_e per expert is the forward grouped GEMM with B the
+#               stack of W_e^T [E*K, N] (grouped_gemm_nvfp4);
+#   wgrad       dW_e = dY_e^T X_e with both operands NVFP4 along the tokens
+#               (grouped_gemm_nvfp4_wgrad);
+#   tile16      one E4M3 scale per 16x16 tile, one outer scale per group of
+#               rows (a multiple of 16), codes to nearest even.
+# --------------------------------------------------------------------------
+
+def nvfp4_quantize_f32(x_f32: np.ndarray, group_rows: int = 1, sr: bool = False, seed: int = 0, stream: int = 0,
+                       R: int = 8):
+    """fp32 [rows, cols] -> NVFP4 (codes [rows, cols/2], sf [rows, cols/16] row-major, outer
+    [rows/group_rows]); element codes stochastically rounded when sr."""
+    x = np.ascontiguousarray(x_f32, dtype=np.float32)
+    rows, cols = x.shape
+    assert cols % 16 == 0 and rows % group_rows == 0 and R in (8, 16, 32)
+    codes = np.empty((rows, cols // 2), dtype=np.uint8)
+    sf = np.empty((rows, cols // 16), dtype=np.uint8)
+    outer = np.empty(rows // group_rows, dtype=np.float32)
+    lib().orc_nvfp4_quantize_f32(_p(x), rows, cols, group_rows, int(sr), seed, stream, R, _p(codes), _p(sf),
+                                 _p(outer))
+    return codes, sf, outer
+
+
+def nvfp4_requant_transpose_sr(codes, sf, outer, group_rows: int, seed: int, stream: int, R: int = 8,
+                               sr: bool = True):
+    """Saved NVFP4 [rows, cols] (outer per group_rows rows) -> NVFP4 of its transpose
+    [cols, rows], one outer scale per output row, blocks of 16 along the old rows."""
+    xh = nvfp4_dequantize(codes, sf, outer, group_rows)
+    return nvfp4_quantize_f32(np.ascontiguousarray(xh.T), 1, sr, seed, stream, R)
+
+
+def nvfp4_requant_transpose_experts_sr(codes, sf, outer, E: int, seed: int, stream: int, R: int = 8,
+                                       sr: bool = True):
+    """Saved expert weight stack [E*N, K] (outer per expert) -> NVFP4 stack of the
+    per-expert transposes W_e^T, [E*K, N], outer per expert; the B operand of
+    the NVFP4 dgrad (grouped_gemm_nvfp4 with output width K)."""
+    rows, K = codes.shape[0], codes.shape[1] * 2
+    N = rows // E
+    xh = nvfp4_dequantize(codes, sf, outer, N).reshape(E, N, K)
+    return nvfp4_quantize_f32(np.ascontiguousarray(xh.transpose(0, 2, 1).reshape(E * K, N)), K, sr, seed, stream, R)
+
+
+def grouped_gemm_nvfp4_wgrad(a_codes, a_sf, a_outer, b_codes, b_sf, b_outer, seg) -> np.ndarray:
+    """WGRAD in NVFP4: A [Nw, M] and B [Kw, M] (blocks of 16 along M, the tokens;
+    one outer scale per row).  C [E, Nw, Kw] fp64:
+    C[e, n, k] = a_outer[n] b_outer[k] sum_{t in segment e} (qa sfa)[n, t] (qb sfb)[k, t];
+    empty experts give 0."""
+    Nw, Kw = a_codes.shape[0], b_codes.shape[0]
+    E = len(seg) - 1
+    Av = nvfp4_block_values(a_codes, a_sf) * np.asarray(a_outer, np.float64)[:, None]
+    Bv = nvfp4_block_values(b_codes, b_sf) * np.asarray(b_outer, np.float64)[:, None]
+    C = np.zeros((E, Nw, Kw), dtype=np.float64)
+    for e in range(E):
+        t0, t1 = int(seg[e]), int(seg[e + 1])
+        if t1 > t0:
+            C[e] = Av[:, t0:t1] @ Bv[:, t0:t1].T
+    return C
+
+
+def nvfp4_quantize_tile16(x_f32: np.ndarray, group_rows: int = 16):
+    """fp32 [rows, cols] -> (codes [rows, cols/2], sf_tile [rows/16, cols/16], outer
+    [rows/group_rows]) with one E4M3 scale per 16x16 tile."""
+    x = np.ascontiguousarray(x_f32, dtype=np.float32)
+    rows, cols = x.shape
+    assert rows % 16 == 0 and cols % 16 == 0 and group_rows % 16 == 0 and rows % group_rows == 0
+    codes = np.empty((rows, cols // 2), dtype=np.uint8)
+    sf = np.empty((rows // 16, cols // 16), dtype=np.uint8)
+    outer = np.empty(rows // group_rows, dtype=np.float32)
+    lib().orc_nvfp4_quantize_tile16(_p(x), rows, cols, group_rows, _p(codes), _p(sf), _p(outer))
+    return codes, sf, outer
+
+
+def nvfp4_tile16_dequantize(codes, sf_tile, outer, group_rows: int = 16) -> np.ndarray:
+    """fp32 (q sf_tile) s of each element (one rounding, as nvfp4_dequantize)."""
+    sf_rows = np.repeat(np.asarray(sf_tile, np.uint8), 16, axis=0)           # each 1x16 block's tile scale
+    outer_rows = np.repeat(np.asarray(outer, np.float32), group_rows)         # each row's outer scale
+    return nvfp4_dequantize(codes, np.ascontiguousarray(sf_rows), outer_rows, 1)
+
+
+def nvfp4_tile16_transpose(codes, sf_tile):
+    """The same tile-scaled tensor in the other orientation: element codes moved
+    to [cols, rows] (two per byte, element 2j in the low nibble), tile scales
+    transposed.  No value changes."""
+    q = np.stack([codes & 15, codes >> 4], axis=-1).reshape(codes.shape[0], -1).T
+    q = np.ascontiguousarray(q)
+    return (q[:, 0::2] | (q[:, 1::2] << 4)).astype(np.uint8), np.ascontiguousarray(np.asarray(sf_tile).T)
 
 
 # --------------------------------------------------------------------------

@@ -451,3 +451,94 @@ ORC_API void orc_nvfp4_block_values(const uint8_t* codes, const uint8_t* sf, int
             out[r * cols + c] = (double)orc_e2m1_decode(q) * (double)orc_e4m3_decode(sf[r * (cols / 16) + c / 16]);
         }
 }
+
+/* ------------------------------------------------------------------------ */
+/* NVFP4 in the backward pass: the pages' stated future work ([P2 §NVFP4     */
+/* forward, MXFP8 backward]: four-bit arithmetic in the backward pass is     */
+/* being explored; a first NVFP4 forward+backward attempt cost too much).    */
+/* Readings taken (pages silent): the scale rules of orc_nvfp4_quantize      */
+/* (outer s = amax / (6*448) per group of rows, one E4M3 scale of            */
+/* amax_b / (6s) per 16 consecutive values of a row, both round-to-nearest); */
+/* the element code is E2M1 of x / (sf*s), rounded stochastically with the   */
+/* random integer of linear element index L = r*cols + c (orc_sr_bits,       */
+/* orc_e2m1_sr; values past 6 saturate) when sr != 0, to nearest even       */
+/* otherwise.  The input is fp32, so that a dequantised, transposed tensor   */
+/* is re-quantised without an intermediate bf16 rounding.                    */
+/* ------------------------------------------------------------------------ */
+ORC_API void orc_nvfp4_quantize_f32(const float* x, int64_t rows, int64_t cols, int64_t group_rows, int sr,
+                                    uint64_t seed, uint64_t stream, int R,
+                                    uint8_t* codes, uint8_t* sf, float* outer) {
+    const int64_t nblk = cols / 16;
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t g = 0; g < rows / group_rows; ++g) {
+        float gmax = 0.0f;
+        for (int64_t i = g * group_rows * cols; i < (g + 1) * group_rows * cols; ++i)
+            if (fabsf(x[i]) > gmax) gmax = fabsf(x[i]);
+        const float s = gmax / (6.0f * 448.0f);
+        outer[g] = s;
+        for (int64_t r = g * group_rows; r < (g + 1) * group_rows; ++r) {
+            for (int64_t b = 0; b < nblk; ++b) {
+                const float* xb = x + r * cols + b * 16;
+                uint8_t* cb = codes + (r * cols + b * 16) / 2;
+                float bmax = 0.0f;
+                for (int i = 0; i < 16; ++i)
+                    if (fabsf(xb[i]) > bmax) bmax = fabsf(xb[i]);
+                const uint8_t scode = (s > 0.0f) ? orc_e4m3_encode(bmax / (6.0f * s)) : 0;
+                sf[r * nblk + b] = scode;
+                memset(cb, 0, 8);
+                if (scode == 0) continue;
+                const float inv = 1.0f / (orc_e4m3_decode(scode) * s);
+                for (int i = 0; i < 16; ++i) {
+                    const float y = xb[i] * inv;
+                    const uint64_t L = (uint64_t)(r * cols + b * 16 + i);
+                    const uint8_t q = sr ? orc_e2m1_sr((double)y, orc_sr_bits(seed, stream, R, L), R)
+                                         : orc_e2m1_encode(y);
+                    cb[i / 2] |= (uint8_t)((i & 1) ? (q << 4) : q);
+                }
+            }
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* The rejected alternative ([P2 §Stochastic rounding across transposes]):   */
+/* one scale shared by each 16x16 tile, so that both orientations of the     */
+/* tensor hold the same codes, at the price of outlier sensitivity (one      */
+/* large value can force the tile's other values to round to zero).          */
+/* Readings taken: the tile scale is E4M3 of tile_amax / (6s) with the outer */
+/* scale s of orc_nvfp4_quantize_f32, one per group_rows rows (a multiple of */
+/* 16, so that no tile straddles two outer scales); codes round to nearest   */
+/* even.  sf_tile is row-major [rows/16][cols/16].                           */
+/* ------------------------------------------------------------------------ */
+ORC_API void orc_nvfp4_quantize_tile16(const float* x, int64_t rows, int64_t cols, int64_t group_rows,
+                                       uint8_t* codes, uint8_t* sf_tile, float* outer) {
+    const int64_t ntc = cols / 16;
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t g = 0; g < rows / group_rows; ++g) {
+        float gmax = 0.0f;
+        for (int64_t i = g * group_rows * cols; i < (g + 1) * group_rows * cols; ++i)
+            if (fabsf(x[i]) > gmax) gmax = fabsf(x[i]);
+        const float s = gmax / (6.0f * 448.0f);
+        outer[g] = s;
+        for (int64_t tr = g * group_rows / 16; tr < (g + 1) * group_rows / 16; ++tr) {
+            for (int64_t tc = 0; tc < ntc; ++tc) {
+                float tmax = 0.0f;
+                for (int64_t r = tr * 16; r < tr * 16 + 16; ++r)
+                    for (int64_t c = tc * 16; c < tc * 16 + 16; ++c)
+                        if (fabsf(x[r * cols + c]) > tmax) tmax = fabsf(x[r * cols + c]);
+                const uint8_t scode = (s > 0.0f) ? orc_e4m3_encode(tmax / (6.0f * s)) : 0;
+                sf_tile[tr * ntc + tc] = scode;
+                const float inv = scode ? 1.0f / (orc_e4m3_decode(scode) * s) : 0.0f;
+                for (int64_t r = tr * 16; r < tr * 16 + 16; ++r) {
+                    uint8_t* cb = codes + (r * cols + tc * 16) / 2;
+                    memset(cb, 0, 8);
+                    if (scode == 0) continue;
+                    for (int i = 0; i < 16; ++i) {
+                        const uint8_t q = orc_e2m1_encode(x[r * cols + tc * 16 + i] * inv);
+                        cb[i / 2] |= (uint8_t)((i & 1) ? (q << 4) : q);
+                    }
+                }
+            }
+        }
+    }
+}

@@ -18,8 +18,8 @@ import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 TESTS = os.path.join(ROOT, "tests")
-CODECS, QUANT, GEMM, HAD = ("test_oracle_codecs.py", "test_oracle_quant.py", "test_oracle_gemm_glue.py",
-                            "test_oracle_hadamard.py")
+CODECS, QUANT, GEMM, HAD, BWD = ("test_oracle_codecs.py", "test_oracle_quant.py", "test_oracle_gemm_glue.py",
+                                 "test_oracle_hadamard.py", "test_oracle_nvfp4_backward.py")
 
 # (what the slip is, file, text, replacement, pin files expected to catch it)
 MUTANTS = [
@@ -68,6 +68,15 @@ MUTANTS = [
      "double a = fabs((double)bf16_to_f32(x[c * rows + b * 32 + t]));", [QUANT]),
     ("requantisation writes E8M0 with bias 126", "oracle.c",
      "out_e8m0[c * nb + b] = (uint8_t)(e + 127);", "out_e8m0[c * nb + b] = (uint8_t)(e + 126);", [QUANT]),
+    ("NVFP4 backward quantiser: block scale of amax / (4s)", "oracle.c",
+     "orc_e4m3_encode(bmax / (6.0f * s))", "orc_e4m3_encode(bmax / (4.0f * s))", [BWD]),
+    ("NVFP4 backward quantiser ignores the stochastic-rounding flag", "oracle.c",
+     "const uint8_t q = sr ? orc_e2m1_sr((double)y, orc_sr_bits(seed, stream, R, L), R)",
+     "const uint8_t q = 0 ? orc_e2m1_sr((double)y, orc_sr_bits(seed, stream, R, L), R)", [BWD]),
+    ("16x16 tile scale of amax / (3s)", "oracle.c",
+     "orc_e4m3_encode(tmax / (6.0f * s))", "orc_e4m3_encode(tmax / (3.0f * s))", [BWD]),
+    ("16x16 tile amax over half the tile's columns", "oracle.c",
+     "for (int64_t c = tc * 16; c < tc * 16 + 16; ++c)", "for (int64_t c = tc * 16; c < tc * 16 + 8; ++c)", [BWD]),
     # __init__.py: GEMM references and glue
     ("NVFP4 GEMM drops the expert's outer scale", "__init__.py",
      "* a_outer[r0:r1, None].astype(np.float64) * float(b_outer[e])",
@@ -111,6 +120,19 @@ MUTANTS = [
      "b = nvfp4_block_values(b_codes[n:n + 1], b_sf[n:n + 1])[0]", [GEMM]),
     ("single requantised entry draws the bits of the wrong index", "__init__.py",
      "L = col * rows + row0 + t", "L = col * rows + t", [QUANT]),
+    ("NVFP4 requantisation without the transpose", "__init__.py",
+     "return nvfp4_quantize_f32(np.ascontiguousarray(xh.T), 1, sr, seed, stream, R)",
+     "return nvfp4_quantize_f32(np.ascontiguousarray(xh.reshape(xh.shape[1], xh.shape[0])), 1, sr, seed, stream, R)",
+     [BWD]),
+    ("expert weight requantisation stacks untransposed experts", "__init__.py",
+     "np.ascontiguousarray(xh.transpose(0, 2, 1).reshape(E * K, N))", "np.ascontiguousarray(xh.reshape(E * K, N))",
+     [BWD]),
+    ("NVFP4 wgrad drops the second operand's outer scales", "__init__.py",
+     "Bv = nvfp4_block_values(b_codes, b_sf) * np.asarray(b_outer, np.float64)[:, None]",
+     "Bv = nvfp4_block_values(b_codes, b_sf)", [BWD]),
+    ("tile-scaled transpose swaps the nibbles", "__init__.py",
+     "return (q[:, 0::2] | (q[:, 1::2] << 4)).astype(np.uint8)", "return (q[:, 1::2] | (q[:, 0::2] << 4)).astype(np.uint8)",
+     [BWD]),
     # __init__.py: Hadamard rotation and S2F6
     ("butterfly difference with the wrong sign", "__init__.py",
      "z = np.stack([a + b, a - b], axis=-2)", "z = np.stack([a + b, b - a], axis=-2)", [HAD]),
@@ -155,7 +177,7 @@ def results(tmp_path_factory):
     if shutil.which("gcc") is None:
         pytest.skip("no C compiler for the oracle")
     base = tmp_path_factory.mktemp("mutants")
-    jobs = {"control": (None, [CODECS, QUANT, GEMM, HAD])}
+    jobs = {"control": (None, [CODECS, QUANT, GEMM, HAD, BWD])}
     for i, m in enumerate(MUTANTS):
         jobs[i] = (m, m[4])
     dirs = {}
