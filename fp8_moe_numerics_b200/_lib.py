@@ -50,6 +50,10 @@ SIGNATURES = {
     "hadamard_s2f6_quantize": (I32, [P, I64, I64, U64, U64, P, P, P]),
     "grouped_gemm_nvfp4_s2f6": (I32, [P, P, P, P, P, P, P, I64, I64, I64, I64, U64, U64, P, P, P]),
     "moe_combine_s2f6": (I32, [P, P, P, P, I64, I64, I64, U64, U64, P, P]),
+    "nvfp4_quantize_sr": (I32, [P, I64, I64, I64, I32, U64, U64, I32, P, P, P, I32, P]),
+    "nvfp4_requant_transpose_sr": (I32, [P, P, P, I64, I64, I64, I32, I64, I32, I32, U64, U64, I32, P, P, P, I32,
+                                         P]),
+    "nvfp4_quantize_tile16": (I32, [P, I64, I64, I64, P, P, P, P]),
 }
 
 _lib = None

@@ -26,7 +26,7 @@ __all__ = [
     "sf_bytes", "sync_status", "wait_selftest", "nvfp4_quantize", "mxfp8_requant_transpose_sr", "mxfp8_quantize",
     "grouped_gemm_nvfp4", "grouped_gemm_mxfp8", "moe_route", "nvfp4_gather_rows", "swiglu_fwd", "swiglu_bwd",
     "moe_combine", "moe_dispatch_grad", "swiglu_nvfp4_quantize", "hadamard_s2f6_quantize", "grouped_gemm_nvfp4_s2f6",
-    "moe_combine_s2f6",
+    "moe_combine_s2f6", "nvfp4_quantize_sr", "nvfp4_requant_transpose_sr", "nvfp4_quantize_tile16",
 ]
 
 
@@ -350,3 +350,70 @@ def swiglu_nvfp4_quantize(h: torch.Tensor, F: int, gated: bool = True, rows_vali
     L.call("swiglu_nvfp4_quantize", _p(h), rows, F, int(gated), _p(rows_valid), _p(codes), _p(sf), _p(outer),
            sf_layout, _s())
     return codes, sf, outer
+
+
+# NVFP4 in the backward pass and the 16x16 shared-scale format (not yet run
+# against the oracle on a GPU; include/mxmoe.h gives the readings).
+
+def nvfp4_quantize_sr(x: torch.Tensor, group_rows: int = 1, rounding: int = MX_ROUND_SR, seed: int = 0,
+                      stream_id: int = 0, rbits: int = 16, sf_layout: int = MX_SF_MMA, out=None):
+    """bf16 [rows, cols] -> NVFP4 (codes u8 [rows, cols/2], sf u8, outer f32 [rows/group_rows]) with
+    stochastically rounded E2M1 codes (MX_ROUND_SR) or to nearest (MX_ROUND_RNE)."""
+    _bf16_2d("x", x)
+    rows, cols = x.shape
+    dev = x.device
+    if out is None:
+        out = (torch.empty(rows, cols // 2, dtype=torch.uint8, device=dev),
+               _u8(sf_bytes(rows, cols, 16, sf_layout), dev),
+               torch.empty(rows // group_rows, dtype=torch.float32, device=dev))
+    codes, sf, outer = out
+    _fits("codes", codes, rows * cols // 2)
+    _fits("sf", sf, rows * (cols // 16))
+    _fits("outer", outer, 4 * (rows // max(group_rows, 1)))
+    L.call("nvfp4_quantize_sr", _p(x), rows, cols, group_rows, rounding, ctypes.c_uint64(seed),
+           ctypes.c_uint64(stream_id), rbits, _p(codes), _p(sf), _p(outer), sf_layout, _s())
+    return codes, sf, outer
+
+
+def nvfp4_requant_transpose_sr(codes, sf, outer, rows: int, cols: int, group_rows: int = 1,
+                               in_sf_layout: int = MX_SF_MMA, experts: int = 1, out_outer_per_expert: bool = False,
+                               rounding: int = MX_ROUND_SR, seed: int = 0, stream_id: int = 0, rbits: int = 16,
+                               out_sf_layout: int = MX_SF_MMA, out=None):
+    """Saved NVFP4 [rows, cols] (`experts` stacked row blocks) -> NVFP4 of each block's transpose,
+    stacked: (codes u8 [experts*cols, rows/experts/2], sf u8, outer f32 [experts*cols or experts])."""
+    dev = codes.device
+    orows, ocols = experts * cols, rows // max(experts, 1)
+    n_outer = experts if out_outer_per_expert else orows
+    if out is None:
+        out = (torch.empty(orows, ocols // 2, dtype=torch.uint8, device=dev),
+               _u8(sf_bytes(orows, ocols, 16, out_sf_layout), dev),
+               torch.empty(n_outer, dtype=torch.float32, device=dev))
+    oc, osf, oo = out
+    _fits("codes", codes, rows * cols // 2)
+    _fits("sf", sf, rows * (cols // 16))
+    _fits("outer", outer, 4 * (rows // max(group_rows, 1)))
+    _fits("out codes", oc, orows * ocols // 2)
+    _fits("out sf", osf, orows * (ocols // 16))
+    _fits("out outer", oo, 4 * n_outer)
+    L.call("nvfp4_requant_transpose_sr", _p(codes), _p(sf), _p(outer), rows, cols, group_rows, in_sf_layout, experts,
+           int(out_outer_per_expert), rounding, ctypes.c_uint64(seed), ctypes.c_uint64(stream_id), rbits, _p(oc),
+           _p(osf), _p(oo), out_sf_layout, _s())
+    return oc, osf, oo
+
+
+def nvfp4_quantize_tile16(x: torch.Tensor, group_rows: int = 16, out=None):
+    """bf16 [rows, cols] -> NVFP4 with one E4M3 scale per 16x16 tile: (codes u8 [rows, cols/2],
+    sf_tile u8 [rows/16, cols/16], outer f32 [rows/group_rows])."""
+    _bf16_2d("x", x)
+    rows, cols = x.shape
+    dev = x.device
+    if out is None:
+        out = (torch.empty(rows, cols // 2, dtype=torch.uint8, device=dev),
+               torch.empty(rows // 16, cols // 16, dtype=torch.uint8, device=dev),
+               torch.empty(rows // max(group_rows, 1), dtype=torch.float32, device=dev))
+    codes, sf_tile, outer = out
+    _fits("codes", codes, rows * cols // 2)
+    _fits("sf_tile", sf_tile, (rows // 16) * (cols // 16))
+    _fits("outer", outer, 4 * (rows // max(group_rows, 1)))
+    L.call("nvfp4_quantize_tile16", _p(x), rows, cols, group_rows, _p(codes), _p(sf_tile), _p(outer), _s())
+    return codes, sf_tile, outer

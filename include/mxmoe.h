@@ -342,6 +342,70 @@ MX_API int moe_combine_s2f6(const int8_t* codes, const uint8_t* e8m0, const int3
                             int64_t T, int64_t k, int64_t D, uint64_t seed, uint64_t stream_id, void* out,
                             cudaStream_t stream);
 
+/* --------------------------------------------------------------------------
+ * NVFP4 in the backward pass, and the 16x16 shared-scale format.
+ * [ai-primer §NVFP4 forward, MXFP8 backward]: four-bit arithmetic in the
+ * backward pass is the lab's stated future work.  [ai-primer §Stochastic
+ * rounding across transposes]: a scale shared by each 16x16 tile keeps both
+ * orientations' codes equal but was rejected as outlier-sensitive.  The pages
+ * give no rule; the readings taken here:
+ *   scales    those of nvfp4_quantize: outer s = amax / 2688 per group of
+ *             rows, E4M3 block scale RNE(amax_b / (6 s)) per 16 values;
+ *   rounding  MX_ROUND_RNE: E2M1 of y = x * (1 / (sf s)) to nearest even, as
+ *             nvfp4_quantize; MX_ROUND_SR: with q the E2M1 step at |y|
+ *             (2^max(floor(log2|y|) - 1, -1)), lo = floor(|y| / q) q, round
+ *             up to lo + q iff u < floor(((|y| - lo) / q) 2^rbits), u the
+ *             rbits-bit random integer of the output element (the Philox
+ *             stream of mxfp8_requant_transpose_sr, L = the element's linear
+ *             index in the output); magnitudes past 6 saturate; the sign of y
+ *             is kept, also on a zero.
+ * These entry points have not yet been run against the oracle on a GPU.
+ * ------------------------------------------------------------------------ */
+
+/* nvfp4_quantize_sr -- bf16 [rows, cols] -> NVFP4 with the rounding above
+ * (the gradient operands of an NVFP4 backward).  Arguments, layouts and
+ * requirements as nvfp4_quantize, plus rounding, seed, stream_id and rbits
+ * (8, 16 or 32 for MX_ROUND_SR).  With MX_ROUND_RNE the outputs equal those
+ * of nvfp4_quantize. */
+MX_API int nvfp4_quantize_sr(const void* x, int64_t rows, int64_t cols, int64_t group_rows, int rounding,
+                             uint64_t seed, uint64_t stream_id, int rbits, uint8_t* codes, uint8_t* sf,
+                             float* outer, int sf_layout, cudaStream_t stream);
+
+/* nvfp4_requant_transpose_sr -- saved NVFP4 -> NVFP4 of its transpose.
+ * The input [rows, cols] (codes, sf in in_sf_layout, outer per group_rows
+ * rows) holds `experts` stacked blocks of rows / experts rows each (1 for an
+ * activation tensor, E for an expert weight stack [E*N, K]).  Each value is
+ * dequantised ((q * sf) * outer, fp32), each block is transposed, and the
+ * result [experts * cols, rows / experts] (block e's transpose in rows
+ * e*cols ..) is quantised with the rounding above, blocks of 16 along the old
+ * rows.  Outer scales: one per output row (out_outer_per_expert = 0; out_outer
+ * [experts * cols]) or one per expert (1; out_outer [experts]).  With
+ * experts = E this gives the stack of W_e^T that grouped_gemm_nvfp4 takes as
+ * B for the NVFP4 input gradient (output width K).
+ *   out_codes device u8 [experts*cols, rows/experts/2]; out_sf device u8
+ *   mx_sf_bytes(experts*cols, rows/experts, 16, out_sf_layout)
+ * Requires cols % 64 == 0, rows / experts % 128 == 0, rows % group_rows == 0
+ * (rows % 128 == 0 for an MX_SF_MMA input; experts*cols % 128 == 0 for an
+ * MX_SF_MMA output), 16-byte aligned codes and out_codes.  out_outer is
+ * written twice (the per-target maxima, then the scales) by the calls this
+ * entry point enqueues. */
+MX_API int nvfp4_requant_transpose_sr(const uint8_t* codes, const uint8_t* sf, const float* outer, int64_t rows,
+                                      int64_t cols, int64_t group_rows, int in_sf_layout, int64_t experts,
+                                      int out_outer_per_expert, int rounding, uint64_t seed, uint64_t stream_id,
+                                      int rbits, uint8_t* out_codes, uint8_t* out_sf, float* out_outer,
+                                      int out_sf_layout, cudaStream_t stream);
+
+/* nvfp4_quantize_tile16 -- bf16 [rows, cols] -> NVFP4 with one E4M3 scale per
+ * 16x16 tile: scale RNE(tile_amax / (6 s)), codes RNE; outer s = amax / 2688
+ * per group_rows rows (a multiple of 16).  Both orientations of the tensor
+ * hold the same codes.
+ *   codes device u8 [rows, cols/2]; sf_tile device u8 [rows/16, cols/16]
+ *   row-major; outer device f32 [rows/group_rows]
+ * Requires rows % 16 == 0, cols % 16 == 0, group_rows % 16 == 0, 16-byte
+ * aligned x and codes. */
+MX_API int nvfp4_quantize_tile16(const void* x, int64_t rows, int64_t cols, int64_t group_rows, uint8_t* codes,
+                                 uint8_t* sf_tile, float* outer, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -85,6 +85,21 @@ CASES = {
     "moe_combine_s2f6": ((A, A, A, None, 16, 2, 64, 1, 2, A, None), [
         ("D % 32", {6: 48}), ("k 0", {5: 0}), ("out misaligned", {9: A8}), ("null codes", {0: None}),
     ]),
+    "nvfp4_quantize_sr": ((A, 128, 64, 1, 1, 1, 2, 16, A, A, A, 0, None), [
+        ("cols % 16", {2: 40}), ("unknown rounding", {4: 3}), ("SR with rbits 12", {7: 12}),
+        ("group_rows 0", {3: 0}), ("MMA layout rows % 128", {1: 64, 11: 1}), ("x misaligned", {0: A8}),
+        ("null outer", {10: None}),
+    ]),
+    "nvfp4_requant_transpose_sr": ((A, A, A, 256, 64, 1, 0, 2, 0, 1, 1, 2, 16, A, A, A, 0, None), [
+        ("cols % 64", {4: 32}), ("rows per expert % 128", {7: 4}), ("rows % experts", {7: 3}),
+        ("no experts", {7: 0}), ("unknown rounding", {9: 2}), ("SR with rbits 4", {12: 4}),
+        ("unknown out layout", {16: 3}), ("outer-per-expert flag 2", {8: 2}), ("out codes misaligned", {13: A8}),
+        ("null out outer", {15: None}), ("out outer misaligned", {15: A1}),
+    ]),
+    "nvfp4_quantize_tile16": ((A, 64, 48, 32, A, A, A, None), [
+        ("rows % 16", {1: 40}), ("cols % 16", {2: 40}), ("group_rows % 16", {3: 8}), ("rows % group_rows", {3: 48}),
+        ("codes misaligned", {4: A8}), ("null sf_tile", {5: None}),
+    ]),
 }
 
 

@@ -165,3 +165,24 @@ def test_layer_rejects_mismatched_configuration():
         ExpertLayer(*args, combine="fp8")
     with pytest.raises(ValueError, match="rows per expert"):
         ExpertLayer(*args, gated=True)                  # w1 holds F rows per expert: an ungated layer
+
+
+def test_nvfp4_backward_buffers():
+    x = bf16(256, 128)
+    good = (u8(256, 64), u8(256 * 8), f32(256))
+    _passes_size_checks(lambda: api.nvfp4_quantize_sr(x, out=good))
+    _size_error(lambda: api.nvfp4_quantize_sr(x, out=(good[0], u8(256 * 8 - 1), good[2])), "sf")
+    # requantisation of a [256, 128] tensor: one expert, outer per output row
+    q = (u8(256, 64), u8(256 * 8), f32(256))
+    out = (u8(128, 128), u8(128 * 16), f32(128))
+    _passes_size_checks(lambda: api.nvfp4_requant_transpose_sr(*q, 256, 128, out=out))
+    _size_error(lambda: api.nvfp4_requant_transpose_sr(*q, 256, 128, out=(out[0], out[1], f32(127))), "out outer")
+    # two experts of 128 rows with a per-expert outer scale: [2*128, 64] out, outer [2]
+    out2 = (u8(256, 64), u8(256 * 8), f32(2))
+    _passes_size_checks(lambda: api.nvfp4_requant_transpose_sr(*q, 256, 128, 128, experts=2,
+                                                               out_outer_per_expert=True, out=out2))
+    _size_error(lambda: api.nvfp4_requant_transpose_sr(*q, 256, 128, 128, experts=2, out_outer_per_expert=True,
+                                                       out=(u8(256, 63), out2[1], out2[2])), "out codes")
+    t = bf16(64, 48)
+    _passes_size_checks(lambda: api.nvfp4_quantize_tile16(t, 32, out=(u8(64, 24), u8(4, 3), f32(2))))
+    _size_error(lambda: api.nvfp4_quantize_tile16(t, 32, out=(u8(64, 24), u8(4, 2), f32(2))), "sf_tile")

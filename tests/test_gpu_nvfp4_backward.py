@@ -1,0 +1,125 @@
+"""GPU parity of the NVFP4-backward entry points and the 16x16 shared-scale
+quantiser (csrc/nvfp4_bwd.cu) against the oracle.
+
+Bar: bit-exact codes, scales and outer scales; both sides take every
+rounding decision in fp32 in the same order, and the stochastic rounding
+draws the same Philox integers.  The NVFP4 dgrad (the forward grouped GEMM
+with the requantised W_e^T stack as B) within the forward GEMM's relative
+Frobenius bound of the oracle's fp64 product.
+
+The kernels have not yet run on a GPU: their index arithmetic is checked on
+the CPU (tests/test_nvfp4_bwd_indexing.py) and the module stays skipped until
+a first run on a B200 has passed it.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from fp8_moe_numerics_b200 import api
+from tests.layouts import mma_to_rowmajor
+from tests.test_gpu_gemm import dev, rel_fro
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skip(reason="not yet run on a GPU; enable after a first run of this module on a B200")]
+
+
+def to_dev_bf16(u16):
+    return torch.from_numpy(np.ascontiguousarray(u16).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def bf16_input(rows, cols, seed):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_t(3, (rows, cols)) * 10.0 ** rng.uniform(-3, 3, (rows, 1))
+    x[rows // 2] = 0.0                                           # a zero row
+    x[1, 5] = -0.0
+    return oracle.f32_to_bf16(x.astype(np.float32))
+
+
+def host(t):
+    return t.cpu().numpy()
+
+
+@pytest.mark.parametrize("rows,cols,group_rows,layout", [(128, 256, 1, api.MX_SF_MMA), (256, 512, 128, api.MX_SF_MMA),
+                                                         (48, 96, 16, api.MX_SF_ROWMAJOR)])
+@pytest.mark.parametrize("rbits", [8, 16, 32])
+def test_nvfp4_quantize_sr_bit_exact(cuda, rows, cols, group_rows, layout, rbits):
+    x = bf16_input(rows, cols, rows + cols + rbits)
+    seed, stream = 1234, 5
+    c, sf, o = api.nvfp4_quantize_sr(to_dev_bf16(x), group_rows, api.MX_ROUND_SR, seed, stream, rbits, layout)
+    api.sync_status()
+    rc, rsf, ro = oracle.nvfp4_quantize_f32(oracle.bf16_to_f32(x), group_rows, True, seed, stream, rbits)
+    sf_h = mma_to_rowmajor(host(sf), rows, cols // 16) if layout == api.MX_SF_MMA else host(sf).reshape(rows, -1)
+    assert np.array_equal(host(o), ro)
+    assert np.array_equal(sf_h, rsf)
+    assert np.array_equal(host(c), rc)
+
+
+def test_nvfp4_quantize_sr_rne_equals_the_forward_quantiser(cuda):
+    x = to_dev_bf16(bf16_input(256, 256, 3))
+    a = api.nvfp4_quantize_sr(x, 1, api.MX_ROUND_RNE)
+    b = api.nvfp4_quantize(x, 1, api.MX_SF_MMA)
+    api.sync_status()
+    for u, v in zip(a, b):
+        assert torch.equal(u, v)
+
+
+@pytest.mark.parametrize("rows,cols,rbits", [(256, 128, 16), (384, 256, 8), (128, 128, 32)])
+def test_requant_transpose_activations_bit_exact(cuda, rows, cols, rbits):
+    q = oracle.nvfp4_quantize(bf16_input(rows, cols, rows * cols))
+    from tests.layouts import rowmajor_to_mma
+    seed, stream = 77, 9
+    oc, osf, oo = api.nvfp4_requant_transpose_sr(dev(q[0]), dev(rowmajor_to_mma(q[1])), dev(q[2]), rows, cols, 1,
+                                                 api.MX_SF_MMA, 1, False, api.MX_ROUND_SR, seed, stream, rbits,
+                                                 api.MX_SF_MMA)
+    api.sync_status()
+    rc, rsf, ro = oracle.nvfp4_requant_transpose_sr(*q, 1, seed, stream, rbits)
+    assert np.array_equal(host(oo), ro)
+    assert np.array_equal(mma_to_rowmajor(host(osf), cols, rows // 16), rsf)
+    assert np.array_equal(host(oc), rc)
+
+
+def test_requant_transpose_expert_weights_bit_exact(cuda):
+    E, N, K = 3, 128, 256
+    rng = np.random.default_rng(4)
+    w = (rng.standard_normal((E * N, K)) * np.repeat([1.0, 30.0, 0.01], N)[:, None]).astype(np.float32)
+    q = oracle.nvfp4_quantize(oracle.f32_to_bf16(w), group_rows=N)
+    from tests.layouts import rowmajor_to_mma
+    seed, stream = 5, 6
+    oc, osf, oo = api.nvfp4_requant_transpose_sr(dev(q[0]), dev(rowmajor_to_mma(q[1])), dev(q[2]), E * N, K, N,
+                                                 api.MX_SF_MMA, E, True, api.MX_ROUND_SR, seed, stream, 16,
+                                                 api.MX_SF_MMA)
+    api.sync_status()
+    rc, rsf, ro = oracle.nvfp4_requant_transpose_experts_sr(*q, E, seed, stream, 16)
+    assert np.array_equal(host(oo), ro)
+    assert np.array_equal(mma_to_rowmajor(host(osf), E * K, N // 16), rsf)
+    assert np.array_equal(host(oc), rc)
+
+
+@pytest.mark.parametrize("rows,cols,group_rows", [(64, 48, 32), (256, 512, 256), (16, 16, 16)])
+def test_tile16_bit_exact(cuda, rows, cols, group_rows):
+    x = bf16_input(rows, cols, 11 + rows)
+    c, sf, o = api.nvfp4_quantize_tile16(to_dev_bf16(x), group_rows)
+    api.sync_status()
+    rc, rsf, ro = oracle.nvfp4_quantize_tile16(oracle.bf16_to_f32(x), group_rows)
+    assert np.array_equal(host(o), ro) and np.array_equal(host(sf), rsf) and np.array_equal(host(c), rc)
+
+
+def test_nvfp4_dgrad_through_the_forward_gemm(cuda):
+    # dX = dY W_e per expert, with dY quantised by SR and B the requantised
+    # stack of W_e^T: the forward grouped GEMM with output width K
+    from tests.layouts import rowmajor_to_mma
+    E, N, K, M = 2, 256, 256, 256
+    seg = np.array([0, 128, 256], dtype=np.int64)
+    rng = np.random.default_rng(12)
+    w = oracle.nvfp4_quantize(oracle.f32_to_bf16((rng.standard_normal((E * N, K)) * 0.02).astype(np.float32)), N)
+    dy = oracle.f32_to_bf16(rng.standard_normal((M, N)).astype(np.float32))
+    wt = api.nvfp4_requant_transpose_sr(dev(w[0]), dev(rowmajor_to_mma(w[1])), dev(w[2]), E * N, K, N,
+                                        api.MX_SF_MMA, E, True, api.MX_ROUND_SR, 2, 5, 16, api.MX_SF_MMA)
+    dq = api.nvfp4_quantize_sr(to_dev_bf16(dy), 1, api.MX_ROUND_SR, 3, 6, 16, api.MX_SF_MMA)
+    dx = api.grouped_gemm_nvfp4(dq, wt, dev(seg), E, K, N, out_dtype=torch.float32)
+    api.sync_status()
+    rwt = oracle.nvfp4_requant_transpose_experts_sr(*w, E, 2, 5, 16)
+    rdq = oracle.nvfp4_quantize_f32(oracle.bf16_to_f32(dy), 1, True, 3, 6, 16)
+    ref = oracle.grouped_gemm_nvfp4(*rdq, *rwt, seg, K)
+    assert rel_fro(host(dx).astype(np.float64), ref) <= 1e-4

@@ -1,0 +1,120 @@
+"""Index arithmetic of the NVFP4-backward kernels (csrc/nvfp4_bwd.cu), checked
+on the CPU before they run on a GPU.
+
+Each kernel's launch grid and thread-to-element mapping is replayed here (the
+formulas restated from the kernel source) over several shapes, scale layouts
+and expert splits: every global read stays inside its buffer, every output
+byte is written by exactly one thread, and every atomic target lies inside
+the scale array.
+"""
+import numpy as np
+import pytest
+
+T = 256                                   # threads per block
+
+
+def sf_offset(r, s, S, mma):
+    """Scale byte of row r, block column s of an [R, S] scale array (MMA: 512-byte
+    atoms of 128 rows x 4 columns)."""
+    if not mma:
+        return r * S + s
+    return (((r >> 7) * (S >> 2) + (s >> 2)) << 9) + ((r & 31) << 4) + (((r >> 5) & 3) << 2) + (s & 3)
+
+
+def _threads(items):
+    grid = (items + T - 1) // T
+    g = np.arange(grid * T, dtype=np.int64)
+    return g[g < items]
+
+
+def _exactly_once(starts, width, size):
+    """Byte ranges [start, start + width) tile [0, size) with no overlap."""
+    starts = np.sort(np.asarray(starts, np.int64))
+    assert starts.min() >= 0 and starts.max() + width <= size
+    assert len(starts) * width == size and np.all(np.diff(starts) == width)
+
+
+@pytest.mark.parametrize("rows,cols,group_rows,mma", [(128, 64, 1, True), (256, 128, 128, True), (48, 32, 16, False),
+                                                      (16, 16, 1, False)])
+def test_quantize_sr_kernel_indexing(rows, cols, group_rows, mma):
+    assert cols % 16 == 0 and rows % group_rows == 0 and (not mma or (rows % 128 == 0 and cols % 64 == 0))
+    # group_outer_kernel: block g reads uint4 words i < group_rows * cols / 8 of its group
+    n = group_rows * cols // 8
+    last = (rows // group_rows - 1) * group_rows * cols * 2 + (n - 1) * 16 + 16
+    assert last <= rows * cols * 2 and (group_rows * cols) % 8 == 0
+    # nvfp4_quantize_sr_kernel: one thread per 16-value block
+    S = cols // 16
+    item = _threads(rows * S)
+    r, b = item // S, item % S
+    x_start = (r * cols + b * 16) * 2
+    assert x_start.min() >= 0 and x_start.max() + 32 <= rows * cols * 2 and np.all(x_start % 16 == 0)
+    assert np.all(r // group_rows < rows // group_rows)
+    _exactly_once((r * cols + b * 16) // 2, 8, rows * cols // 2)
+    _exactly_once([sf_offset(int(a), int(c), S, mma) for a, c in zip(r, b)], 1, rows * S)
+
+
+@pytest.mark.parametrize("rows,cols,group_rows,experts,per_expert,in_mma,out_mma", [
+    (256, 128, 1, 1, 0, True, True),            # activations: one outer scale per output row
+    (512, 128, 128, 4, 1, True, True),          # weight stack [E*N, K]: per-expert outer scale
+    (384, 64, 1, 3, 0, False, False),
+    (256, 192, 256, 1, 1, True, False),
+])
+def test_requant_kernels_indexing(rows, cols, group_rows, experts, per_expert, in_mma, out_mma):
+    rpe = rows // experts
+    # the shapes the entry point accepts
+    assert rpe % 128 == 0 and cols % 64 == 0 and rows % group_rows == 0
+    assert not in_mma or rows % 128 == 0
+    assert not out_mma or ((experts * cols) % 128 == 0 and rpe % 64 == 0)
+    S_in = cols // 16
+    # pass 1: grid (cols / 64, rows / 128); thread (cl = t % 64, rg = t / 64) reads 32 rows of one column
+    n_outer = experts if per_expert else experts * cols
+    for by in range(rows // 128):
+        r0 = by * 128
+        e = r0 // rpe
+        assert (r0 + 127) // rpe == e                         # a block never straddles two experts
+        for bx in range(cols // 64):
+            t = np.arange(T)
+            cl, rg = t & 63, t >> 6
+            c = bx * 64 + cl
+            rr = r0 + rg[:, None] * 32 + np.arange(32)[None, :]
+            assert rr.max() < rows and c.max() < cols
+            assert ((rr * cols + c[:, None]) // 2).max() < rows * cols // 2
+            offs = [sf_offset(int(a), int(cc) // 16, S_in, in_mma) for a, cc in zip(rr.reshape(-1),
+                                                                                    np.repeat(c, 32))]
+            assert min(offs) >= 0 and max(offs) < rows * S_in
+            targets = np.full(1, e) if per_expert else e * cols + c[:64]
+            assert targets.min() >= 0 and targets.max() < n_outer
+    # pass 2: one thread per output block of 16; item -> (c fastest, then block b, then expert e)
+    nb = rpe // 16
+    item = _threads(experts * nb * cols)
+    c = item % cols
+    b = (item // cols) % nb
+    e = item // cols // nb
+    o = e * cols + c
+    rr = e[:, None] * rpe + b[:, None] * 16 + np.arange(16)[None, :]
+    assert rr.max() < rows
+    assert np.all((per_expert and e.max() < experts) or o.max() < experts * cols)
+    _exactly_once((o * rpe + b * 16) // 2, 8, experts * cols * rpe // 2)
+    _exactly_once([sf_offset(int(a), int(bb), nb, out_mma) for a, bb in zip(o, b)], 1, experts * cols * nb)
+    # the random index of each element is its linear output index, each used once
+    L = (o * rpe + b * 16)[:, None] + np.arange(16)[None, :]
+    assert np.array_equal(np.sort(L.reshape(-1)), np.arange(experts * cols * rpe))
+
+
+@pytest.mark.parametrize("rows,cols,group_rows", [(64, 48, 32), (16, 16, 16), (128, 256, 128)])
+def test_tile16_kernel_indexing(rows, cols, group_rows):
+    ntc = cols // 16
+    warps = rows // 16 * ntc
+    gid = _threads(warps * 32)
+    tile, lane = gid >> 5, gid & 31
+    assert np.all(tile < warps)
+    tr, tc = tile // ntc, tile % ntc
+    r, c0 = tr * 16 + (lane >> 1), tc * 16 + 8 * (lane & 1)
+    x_start = (r * cols + c0) * 2
+    assert x_start.max() + 16 <= rows * cols * 2 and np.all(x_start % 16 == 0)
+    assert np.all((tr * 16) // group_rows < rows // group_rows)
+    _exactly_once((r * cols + c0) // 2, 4, rows * cols // 2)
+    lead = lane == 0
+    _exactly_once(tr[lead] * ntc + tc[lead], 1, rows // 16 * ntc)
+    # every warp's lanes belong to one tile (the warp leaves or stays whole)
+    assert np.all(np.diff(tile.reshape(-1, 32), axis=1) == 0)
