@@ -581,7 +581,7 @@ def cpu_baseline(inp, layer, seconds: float = 15.0):
 # larger than L2 where DRAM traffic is read off)
 # --------------------------------------------------------------------------
 KERNEL_CASES = ("gemm_nvfp4", "gemm_nvfp4_s2f6", "gemm_mxfp8_dgrad", "gemm_mxfp8_wgrad", "requant", "requant_w",
-                "nvfp4_quantize", "quant_w", "mxfp8_quantize")
+                "nvfp4_quantize", "quant_w", "mxfp8_quantize", "nvfp4_quantize_sr", "requant_nvfp4")
 
 
 def run_kernel(args):
@@ -616,14 +616,19 @@ def run_kernel(args):
             else:
                 xt = api.mxfp8_requant_transpose_sr(*xp, M, D, 1, rows_valid=seg[E:E + 1], seed=1, stream_id=2)
                 run = lambda: api.grouped_gemm_mxfp8(api.MX_GEMM_WGRAD, q[2], q[3], *xt, seg, E, M, 2 * F, D)
-    elif which in ("requant", "nvfp4_quantize"):
+    elif which in ("requant", "nvfp4_quantize", "nvfp4_quantize_sr", "requant_nvfp4"):
         c = workloads.CONFIGS[QUANT_WORKLOAD]
         x = workloads.activations(c["rows"], c["cols"], c["x_dist"], c["seed"], dev)
         q = api.nvfp4_quantize(x)
         if which == "requant":
             run = lambda: api.mxfp8_requant_transpose_sr(*q, c["rows"], c["cols"], seed=c["sr_seed"])
-        else:
+        elif which == "nvfp4_quantize":
             run = lambda: api.nvfp4_quantize(x, out=q)
+        elif which == "nvfp4_quantize_sr":            # NVFP4 backward: E2M1 codes rounded stochastically, R = 16
+            run = lambda: api.nvfp4_quantize_sr(x, seed=c["sr_seed"], out=q)
+        else:                                           # NVFP4 backward: requantisation across the transpose
+            t = api.nvfp4_requant_transpose_sr(*q, c["rows"], c["cols"], seed=c["sr_seed"])
+            run = lambda: api.nvfp4_requant_transpose_sr(*q, c["rows"], c["cols"], seed=c["sr_seed"], out=t)
     elif which == "requant_w":
         # 64 experts of 2048 x 4096 weights, per-expert outer scales (output 0.55 GB > L2)
         E, N, K = 64, 2048, 4096
