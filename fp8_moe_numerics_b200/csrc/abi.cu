@@ -6,7 +6,10 @@
 namespace {
 thread_local int g_last_cuda_error = 0;
 constexpr int kMaxDevices = 64;
-int g_device_ok[kMaxDevices] = {0};   // 0 unknown, 1 sm_100, -1 other
+// 0 unknown, 1 sm_100, -1 other; read and written by every host thread that
+// calls an entry point (relaxed: each thread that finds 0 computes the same
+// value and stores it)
+std::atomic<int> g_device_ok[kMaxDevices] = {};
 }  // namespace
 
 int mx_set_cuda_error(cudaError_t e) {
@@ -31,13 +34,16 @@ int mx_check_device(void) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return mx_set_cuda_error(e);
-    if (dev >= 0 && dev < kMaxDevices && g_device_ok[dev]) return g_device_ok[dev] > 0 ? MX_OK : MX_EUNSUPPORTED;
+    if (dev >= 0 && dev < kMaxDevices) {
+        const int known = g_device_ok[dev].load(std::memory_order_relaxed);
+        if (known) return known > 0 ? MX_OK : MX_EUNSUPPORTED;
+    }
     int major = 0, minor = 0;
     if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
         (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess)
         return mx_set_cuda_error(e);
     const bool ok = major == 10 && minor == 0;
-    if (dev >= 0 && dev < kMaxDevices) g_device_ok[dev] = ok ? 1 : -1;
+    if (dev >= 0 && dev < kMaxDevices) g_device_ok[dev].store(ok ? 1 : -1, std::memory_order_relaxed);
     return ok ? MX_OK : MX_EUNSUPPORTED;
 }
 
