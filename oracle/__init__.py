@@ -111,6 +111,7 @@ def _declare(L: ctypes.CDLL) -> None:
         "orc_mxfp8_dequantize": (None, [P, P, I64, I64, P]),
         "orc_nvfp4_quantize_f32": (None, [P, I64, I64, I64, I32, U64, U64, I32, P, P, P]),
         "orc_nvfp4_quantize_tile16": (None, [P, I64, I64, I64, P, P, P]),
+        "orc_nvfp4_quantize_f32_block_outer": (None, [P, I64, I64, P, I32, U64, U64, I32, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -406,8 +407,11 @@ def grouped_gemm_mxfp8_wgrad(a_codes, a_e8, b_codes, b_e8, seg) -> np.ndarray:
 #               both outer scales factor out of the contraction;
 #   dgrad       dX = dY W_e per expert is the forward grouped GEMM with B the
 #               stack of W_e^T [E*K, N] (grouped_gemm_nvfp4);
-#   wgrad       dW_e = dY_e^T X_e with both operands NVFP4 along the tokens
-#               (grouped_gemm_nvfp4_wgrad);
+#   wgrad       dW_e = dY_e^T X_e with both operands NVFP4 along the tokens,
+#               outer scales per expert segment of the tokens: per (segment,
+#               row) for dY^T, per segment for X^T, so that the GEMM applies a
+#               per-row times a per-expert factor as in the forward
+#               (nvfp4_quantize_transpose_segments, grouped_gemm_nvfp4_wgrad);
 #   tile16      one E4M3 scale per 16x16 tile, one outer scale per group of
 #               rows (a multiple of 16), codes to nearest even.
 # --------------------------------------------------------------------------
@@ -446,20 +450,56 @@ def nvfp4_requant_transpose_experts_sr(codes, sf, outer, E: int, seed: int, stre
     return nvfp4_quantize_f32(np.ascontiguousarray(xh.transpose(0, 2, 1).reshape(E * K, N)), K, sr, seed, stream, R)
 
 
+def nvfp4_quantize_transpose_segments(x_f32: np.ndarray, seg, per_row: bool, sr: bool = True, seed: int = 0,
+                                      stream: int = 0, R: int = 8):
+    """x fp32 [M, C] -> NVFP4 of its transpose [C, M] (blocks of 16 along M, the
+    tokens) with outer scales per expert segment of M (seg [E+1], starts at
+    multiples of 16): one per (segment, row), outer [E, C], when per_row; one
+    per segment, outer [E], otherwise.  Each scale is the segment's amax / 2688
+    (fp32); columns past seg[E] (padding rows of the expert-major layout)
+    quantise to zero.  The wgrad operands: dY^T per (segment, row), X^T per
+    segment, so that the GEMM's outer factors are a per-row and a per-expert
+    value, as in the forward GEMM."""
+    x = np.ascontiguousarray(x_f32, dtype=np.float32)
+    M, C = x.shape
+    seg = np.asarray(seg, dtype=np.int64)
+    E = len(seg) - 1
+    assert M % 16 == 0 and np.all(seg % 16 == 0) and seg[-1] <= M and R in (8, 16, 32)
+    xt = np.ascontiguousarray(x.T)
+    s_blk = np.zeros((C, M // 16), dtype=np.float32)
+    outer = np.zeros((E, C) if per_row else E, dtype=np.float32)
+    for e in range(E):
+        t0, t1 = int(seg[e]), int(seg[e + 1])
+        if t1 <= t0:
+            continue
+        amax = np.abs(xt[:, t0:t1]).max(axis=1) if per_row else np.abs(xt[:, t0:t1]).max()
+        s = np.asarray(amax, dtype=np.float32) / np.float32(2688.0)              # one fp32 division
+        outer[e] = s
+        s_blk[:, t0 // 16:t1 // 16] = s[:, None] if per_row else s
+    codes = np.empty((C, M // 2), dtype=np.uint8)
+    sf = np.empty((C, M // 16), dtype=np.uint8)
+    lib().orc_nvfp4_quantize_f32_block_outer(_p(xt), C, M, _p(s_blk), int(sr), seed, stream, R, _p(codes), _p(sf))
+    return codes, sf, outer
+
+
 def grouped_gemm_nvfp4_wgrad(a_codes, a_sf, a_outer, b_codes, b_sf, b_outer, seg) -> np.ndarray:
-    """WGRAD in NVFP4: A [Nw, M] and B [Kw, M] (blocks of 16 along M, the tokens;
-    one outer scale per row).  C [E, Nw, Kw] fp64:
-    C[e, n, k] = a_outer[n] b_outer[k] sum_{t in segment e} (qa sfa)[n, t] (qb sfb)[k, t];
+    """WGRAD in NVFP4: A [Nw, M] and B [Kw, M] (blocks of 16 along M, the tokens)
+    with outer scales per expert segment: a_outer [E, Nw], b_outer [E] (or
+    [E, Kw]).  C [E, Nw, Kw] fp64:
+    C[e, n, k] = a_outer[e, n] b_outer[e(, k)] sum_{t in segment e} (qa sfa)[n, t] (qb sfb)[k, t];
     empty experts give 0."""
     Nw, Kw = a_codes.shape[0], b_codes.shape[0]
     E = len(seg) - 1
-    Av = nvfp4_block_values(a_codes, a_sf) * np.asarray(a_outer, np.float64)[:, None]
-    Bv = nvfp4_block_values(b_codes, b_sf) * np.asarray(b_outer, np.float64)[:, None]
+    Av = nvfp4_block_values(a_codes, a_sf)
+    Bv = nvfp4_block_values(b_codes, b_sf)
+    ao = np.asarray(a_outer, np.float64).reshape(E, Nw)
+    bo = np.asarray(b_outer, np.float64)
+    bo = bo.reshape(E, 1) if bo.ndim == 1 else bo.reshape(E, Kw)
     C = np.zeros((E, Nw, Kw), dtype=np.float64)
     for e in range(E):
         t0, t1 = int(seg[e]), int(seg[e + 1])
         if t1 > t0:
-            C[e] = Av[:, t0:t1] @ Bv[:, t0:t1].T
+            C[e] = (Av[:, t0:t1] @ Bv[:, t0:t1].T) * ao[e][:, None] * bo[e][None, :]
     return C
 
 

@@ -465,6 +465,28 @@ ORC_API void orc_nvfp4_block_values(const uint8_t* codes, const uint8_t* sf, int
 /* otherwise.  The input is fp32, so that a dequantised, transposed tensor   */
 /* is re-quantised without an intermediate bf16 rounding.                    */
 /* ------------------------------------------------------------------------ */
+/* One block of 16 fp32 values under outer scale s: E4M3 scale code (0 when  */
+/* s == 0 or the block is zero) and eight code bytes, element 2j in the low  */
+/* nibble of byte j; L0 is the linear output index of element 0.             */
+static uint8_t nvfp4_block_f32(const float* xb, float s, int sr, uint64_t seed, uint64_t stream, int R,
+                               uint64_t L0, uint8_t* cb) {
+    float bmax = 0.0f;
+    for (int i = 0; i < 16; ++i)
+        if (fabsf(xb[i]) > bmax) bmax = fabsf(xb[i]);
+    const uint8_t scode = (s > 0.0f) ? orc_e4m3_encode(bmax / (6.0f * s)) : 0;
+    memset(cb, 0, 8);
+    if (scode == 0) return 0;
+    const float inv = 1.0f / (orc_e4m3_decode(scode) * s);
+    for (int i = 0; i < 16; ++i) {
+        const float y = xb[i] * inv;
+        const uint64_t L = L0 + (uint64_t)i;
+        const uint8_t q = sr ? orc_e2m1_sr((double)y, orc_sr_bits(seed, stream, R, L), R)
+                             : orc_e2m1_encode(y);
+        cb[i / 2] |= (uint8_t)((i & 1) ? (q << 4) : q);
+    }
+    return scode;
+}
+
 ORC_API void orc_nvfp4_quantize_f32(const float* x, int64_t rows, int64_t cols, int64_t group_rows, int sr,
                                     uint64_t seed, uint64_t stream, int R,
                                     uint8_t* codes, uint8_t* sf, float* outer) {
@@ -476,28 +498,25 @@ ORC_API void orc_nvfp4_quantize_f32(const float* x, int64_t rows, int64_t cols, 
             if (fabsf(x[i]) > gmax) gmax = fabsf(x[i]);
         const float s = gmax / (6.0f * 448.0f);
         outer[g] = s;
-        for (int64_t r = g * group_rows; r < (g + 1) * group_rows; ++r) {
-            for (int64_t b = 0; b < nblk; ++b) {
-                const float* xb = x + r * cols + b * 16;
-                uint8_t* cb = codes + (r * cols + b * 16) / 2;
-                float bmax = 0.0f;
-                for (int i = 0; i < 16; ++i)
-                    if (fabsf(xb[i]) > bmax) bmax = fabsf(xb[i]);
-                const uint8_t scode = (s > 0.0f) ? orc_e4m3_encode(bmax / (6.0f * s)) : 0;
-                sf[r * nblk + b] = scode;
-                memset(cb, 0, 8);
-                if (scode == 0) continue;
-                const float inv = 1.0f / (orc_e4m3_decode(scode) * s);
-                for (int i = 0; i < 16; ++i) {
-                    const float y = xb[i] * inv;
-                    const uint64_t L = (uint64_t)(r * cols + b * 16 + i);
-                    const uint8_t q = sr ? orc_e2m1_sr((double)y, orc_sr_bits(seed, stream, R, L), R)
-                                         : orc_e2m1_encode(y);
-                    cb[i / 2] |= (uint8_t)((i & 1) ? (q << 4) : q);
-                }
-            }
-        }
+        for (int64_t r = g * group_rows; r < (g + 1) * group_rows; ++r)
+            for (int64_t b = 0; b < nblk; ++b)
+                sf[r * nblk + b] = nvfp4_block_f32(x + r * cols + b * 16, s, sr, seed, stream, R,
+                                                   (uint64_t)(r * cols + b * 16), codes + (r * cols + b * 16) / 2);
     }
+}
+
+/* The same blocks with the outer scale of each block given (s_blk, row-major */
+/* [rows][cols/16]): for outer scales that change along a row, as those of a */
+/* transposed tensor taken per expert segment of its columns.                */
+ORC_API void orc_nvfp4_quantize_f32_block_outer(const float* x, int64_t rows, int64_t cols, const float* s_blk,
+                                                int sr, uint64_t seed, uint64_t stream, int R,
+                                                uint8_t* codes, uint8_t* sf) {
+    const int64_t nblk = cols / 16;
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t b = 0; b < nblk; ++b)
+            sf[r * nblk + b] = nvfp4_block_f32(x + r * cols + b * 16, s_blk[r * nblk + b], sr, seed, stream, R,
+                                               (uint64_t)(r * cols + b * 16), codes + (r * cols + b * 16) / 2);
 }
 
 /* ------------------------------------------------------------------------ */

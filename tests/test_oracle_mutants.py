@@ -128,8 +128,14 @@ MUTANTS = [
      "np.ascontiguousarray(xh.transpose(0, 2, 1).reshape(E * K, N))", "np.ascontiguousarray(xh.reshape(E * K, N))",
      [BWD]),
     ("NVFP4 wgrad drops the second operand's outer scales", "__init__.py",
-     "Bv = nvfp4_block_values(b_codes, b_sf) * np.asarray(b_outer, np.float64)[:, None]",
-     "Bv = nvfp4_block_values(b_codes, b_sf)", [BWD]),
+     "C[e] = (Av[:, t0:t1] @ Bv[:, t0:t1].T) * ao[e][:, None] * bo[e][None, :]",
+     "C[e] = (Av[:, t0:t1] @ Bv[:, t0:t1].T) * ao[e][:, None]", [BWD]),
+    ("segment outer scales taken over the whole row", "__init__.py",
+     "amax = np.abs(xt[:, t0:t1]).max(axis=1) if per_row else np.abs(xt[:, t0:t1]).max()",
+     "amax = np.abs(xt).max(axis=1) if per_row else np.abs(xt[:, t0:t1]).max()", [BWD]),
+    ("segment blocks take the next segment's scale", "__init__.py",
+     "s_blk[:, t0 // 16:t1 // 16] = s[:, None] if per_row else s",
+     "s_blk[:, t0 // 16 + 1:t1 // 16 + 1] = s[:, None] if per_row else s", [BWD]),
     ("tile-scaled transpose swaps the nibbles", "__init__.py",
      "return (q[:, 0::2] | (q[:, 1::2] << 4)).astype(np.uint8)", "return (q[:, 1::2] | (q[:, 0::2] << 4)).astype(np.uint8)",
      [BWD]),

@@ -161,14 +161,51 @@ def test_expert_weight_requant_is_per_expert(orc):
         assert np.all(np.abs(back[e] - ref).reshape(K, N // 16, 16) <= blk / 4 + 1e-30)
 
 
+def test_segment_transpose_with_one_segment_is_the_row_quantiser(orc):
+    # one segment over all tokens: per (segment, row) is the per-row quantiser
+    # of the transpose, per segment the per-tensor one, random indices included
+    x = _rand_bf16_values(orc, 64, 48, 13)
+    seg = np.array([0, 64])
+    for per_row, g in ((True, 1), (False, 48)):
+        c, sf, o = orc.nvfp4_quantize_transpose_segments(x, seg, per_row, True, 4, 7, 16)
+        rc, rsf, ro = orc.nvfp4_quantize_f32(np.ascontiguousarray(x.T), g, True, 4, 7, 16)
+        assert np.array_equal(c, rc) and np.array_equal(sf, rsf) and np.array_equal(o.reshape(-1), ro)
+
+
+def test_segment_outer_scales_closed_form_and_padding(orc):
+    rng = np.random.default_rng(14)
+    M, C = 160, 32
+    seg = np.array([0, 64, 64, 128])                             # expert 1 empty; rows 128.. are padding
+    x = (rng.standard_normal((M, C)) * np.where(np.arange(M) < 64, 1.0, 40.0)[:, None]).astype(np.float32)
+    a, sa, oa = orc.nvfp4_quantize_transpose_segments(x, seg, True, sr=False)
+    b, sb, ob = orc.nvfp4_quantize_transpose_segments(x, seg, False, sr=False)
+    assert oa.shape == (3, C) and ob.shape == (3,)
+    for e, (t0, t1) in ((0, (0, 64)), (2, (64, 128))):
+        assert np.array_equal(oa[e], np.abs(x[t0:t1]).max(axis=0).astype(np.float32) / np.float32(2688.0))
+        assert ob[e] == np.float32(np.abs(x[t0:t1]).max()) / np.float32(2688.0)
+    assert np.all(oa[1] == 0) and ob[1] == 0
+    for codes, sf in ((a, sa), (b, sb)):
+        assert np.all(codes[:, 128 // 2:] == 0) and np.all(sf[:, 128 // 16:] == 0)
+    # decoded values within NVFP4's block error of the transposed input
+    for codes, sf, outer_of in ((a, sa, lambda e: oa[e][:, None]), (b, sb, lambda e: ob[e])):
+        v = _e2m1_values(codes) * np.repeat(_e4m3(sf), 16, axis=1)
+        for e, (t0, t1) in ((0, (0, 64)), (2, (64, 128))):
+            got = v[:, t0:t1] * outer_of(e)
+            ref = x[t0:t1].T.astype(np.float64)
+            blk = np.abs(ref).reshape(C, -1, 16).max(-1, keepdims=True)
+            assert np.all(np.abs(got - ref).reshape(C, -1, 16) <= blk / 4 + 1e-30)
+
+
 def test_nvfp4_wgrad_brute_force(orc):
     rng = np.random.default_rng(8)
     E, Nw, Kw = 3, 4, 5
     seg = np.array([0, 64, 64, 160], dtype=np.int64)            # expert 1 empty
     M = 160
-    mag = np.where(np.arange(M) >= 64, 300.0, 1.0)
-    a = orc.nvfp4_quantize_f32((rng.standard_normal((Nw, M)) * mag).astype(np.float32))
-    b = orc.nvfp4_quantize_f32((rng.standard_normal((Kw, M)) * mag[::-1]).astype(np.float32))
+    mag = np.where(np.arange(M) >= 64, 300.0, 1.0)[:, None]
+    dy = (rng.standard_normal((M, Nw)) * mag).astype(np.float32)
+    x = (rng.standard_normal((M, Kw)) * mag[::-1]).astype(np.float32)
+    a = orc.nvfp4_quantize_transpose_segments(dy, seg, True, True, 1, 2, 16)     # dY^T, per (segment, row)
+    b = orc.nvfp4_quantize_transpose_segments(x, seg, False, True, 1, 3, 16)     # X^T, per segment
     C = orc.grouped_gemm_nvfp4_wgrad(*a, *b, seg)
     A = _e2m1_values(a[0]) * np.repeat(_e4m3(a[1]), 16, axis=1)
     B = _e2m1_values(b[0]) * np.repeat(_e4m3(b[1]), 16, axis=1)
@@ -176,8 +213,12 @@ def test_nvfp4_wgrad_brute_force(orc):
     for e, (t0, t1) in ((0, (0, 64)), (2, (64, 160))):
         for n in range(Nw):
             for k in range(Kw):
-                ref = float(a[2][n]) * float(b[2][k]) * sum(A[n, t] * B[k, t] for t in range(t0, t1))
+                ref = float(a[2][e, n]) * float(b[2][e]) * sum(A[n, t] * B[k, t] for t in range(t0, t1))
                 assert abs(C[e, n, k] - ref) <= 1e-12 * max(1e-30, abs(ref))
+    # and close to the unquantised product (SR noise over 64-96 tokens)
+    for e, (t0, t1) in ((0, (0, 64)), (2, (64, 160))):
+        exact = dy[t0:t1].T.astype(np.float64) @ x[t0:t1].astype(np.float64)
+        assert np.linalg.norm(C[e] - exact) <= 0.2 * np.linalg.norm(exact)
 
 
 def test_nvfp4_dgrad_is_the_forward_gemm_with_transposed_weights(orc):
