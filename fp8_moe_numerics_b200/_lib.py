@@ -54,6 +54,9 @@ SIGNATURES = {
     "nvfp4_requant_transpose_sr": (I32, [P, P, P, I64, I64, I64, I32, I64, I32, I32, U64, U64, I32, P, P, P, I32,
                                          P]),
     "nvfp4_quantize_tile16": (I32, [P, I64, I64, I64, P, P, P, P]),
+    "nvfp4_quantize_transpose_segments": (I32, [P, I64, I64, P, I64, I32, I32, U64, U64, I32, P, P, P, I32, P]),
+    "nvfp4_requant_transpose_segments": (I32, [P, P, P, I32, I64, I64, I64, P, I64, I32, I32, U64, U64, I32, P, P,
+                                               P, I32, P]),
 }
 
 _lib = None

@@ -27,6 +27,7 @@ __all__ = [
     "grouped_gemm_nvfp4", "grouped_gemm_mxfp8", "moe_route", "nvfp4_gather_rows", "swiglu_fwd", "swiglu_bwd",
     "moe_combine", "moe_dispatch_grad", "swiglu_nvfp4_quantize", "hadamard_s2f6_quantize", "grouped_gemm_nvfp4_s2f6",
     "moe_combine_s2f6", "nvfp4_quantize_sr", "nvfp4_requant_transpose_sr", "nvfp4_quantize_tile16",
+    "nvfp4_quantize_transpose_segments", "nvfp4_requant_transpose_segments",
 ]
 
 
@@ -417,3 +418,45 @@ def nvfp4_quantize_tile16(x: torch.Tensor, group_rows: int = 16, out=None):
     _fits("outer", outer, 4 * (rows // max(group_rows, 1)))
     L.call("nvfp4_quantize_tile16", _p(x), rows, cols, group_rows, _p(codes), _p(sf_tile), _p(outer), _s())
     return codes, sf_tile, outer
+
+
+def _segment_outputs(M: int, C: int, E: int, per_row: bool, out_sf_layout: int, dev, out):
+    n_outer = E * C if per_row else E
+    if out is None:
+        out = (torch.empty(C, M // 2, dtype=torch.uint8, device=dev), _u8(sf_bytes(C, M, 16, out_sf_layout), dev),
+               torch.empty(n_outer, dtype=torch.float32, device=dev))
+    oc, osf, oo = out
+    _fits("out codes", oc, C * M // 2)
+    _fits("out sf", osf, C * (M // 16))
+    _fits("out outer", oo, 4 * n_outer)
+    return oc, osf, oo
+
+
+def nvfp4_quantize_transpose_segments(x: torch.Tensor, seg: torch.Tensor, E: int, per_row: bool = True,
+                                      rounding: int = MX_ROUND_SR, seed: int = 0, stream_id: int = 0, rbits: int = 16,
+                                      out_sf_layout: int = MX_SF_MMA, out=None):
+    """bf16 [M, C] token-major -> NVFP4 of its transpose [C, M] with outer scales per expert
+    segment (per (segment, row) when per_row): (codes u8 [C, M/2], sf u8, outer f32)."""
+    _bf16_2d("x", x)
+    M, C = x.shape
+    _fits("seg", seg, 8 * (E + 1))
+    oc, osf, oo = _segment_outputs(M, C, E, per_row, out_sf_layout, x.device, out)
+    L.call("nvfp4_quantize_transpose_segments", _p(x), M, C, _p(seg), E, int(per_row), rounding, ctypes.c_uint64(seed),
+           ctypes.c_uint64(stream_id), rbits, _p(oc), _p(osf), _p(oo), out_sf_layout, _s())
+    return oc, osf, oo
+
+
+def nvfp4_requant_transpose_segments(codes, sf, outer, M: int, C: int, seg: torch.Tensor, E: int,
+                                     per_row: bool = False, group_rows: int = 1, in_sf_layout: int = MX_SF_MMA,
+                                     rounding: int = MX_ROUND_SR, seed: int = 0, stream_id: int = 0, rbits: int = 16,
+                                     out_sf_layout: int = MX_SF_MMA, out=None):
+    """Saved NVFP4 [M, C] -> NVFP4 of its transpose [C, M] with outer scales per expert segment."""
+    _fits("codes", codes, M * C // 2)
+    _fits("sf", sf, M * (C // 16))
+    _fits("outer", outer, 4 * (M // max(group_rows, 1)))
+    _fits("seg", seg, 8 * (E + 1))
+    oc, osf, oo = _segment_outputs(M, C, E, per_row, out_sf_layout, codes.device, out)
+    L.call("nvfp4_requant_transpose_segments", _p(codes), _p(sf), _p(outer), in_sf_layout, group_rows, M, C, _p(seg),
+           E, int(per_row), rounding, ctypes.c_uint64(seed), ctypes.c_uint64(stream_id), rbits, _p(oc), _p(osf),
+           _p(oo), out_sf_layout, _s())
+    return oc, osf, oo

@@ -268,6 +268,94 @@ nvfp4_tile16_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, 
     if (lane == 0) sf_tile[tr * ntc + tc] = (uint8_t)scode;
 }
 
+// ---------------------------------------------------------------------------
+// The wgrad operands: the transpose [C, M] of a token-major [M, C] tensor
+// with outer scales per expert segment of the tokens (seg [E+1], starts and
+// lengths multiples of 128): per (segment, row) for dY^T, per segment for
+// X^T.  Tokens past seg[E] (padding rows) quantise to zero.  The input is
+// bf16 (the gradient) or the saved NVFP4 tensor (dequantised on load).
+// ---------------------------------------------------------------------------
+struct Bf16Src {
+    const uint16_t* x;
+    int64_t C;
+    __device__ __forceinline__ float operator()(int64_t t, int64_t c) const {
+        return __uint_as_float((uint32_t)__ldg(x + t * C + c) << 16);
+    }
+};
+struct Nvfp4Src {
+    const uint8_t* codes;
+    const uint8_t* sf;
+    const float* outer;
+    int64_t C, group_rows;
+    int layout;
+    __device__ __forceinline__ float operator()(int64_t t, int64_t c) const {
+        return nvfp4_value(codes, sf, outer, C, group_rows, layout, t, c);
+    }
+};
+
+// Pass 1: block = 128 tokens x 64 columns of one segment (tiles at or past
+// seg[E] do nothing); per-target maxima merged by atomicMax on the float bits.
+template <typename Src>
+__global__ void __launch_bounds__(kThreads)
+segment_amax_kernel(Src src, const int64_t* __restrict__ seg, int64_t E, int64_t C, int per_row,
+                    uint32_t* __restrict__ amax_bits) {
+    __shared__ float part[4][64];
+    __shared__ float red[kThreads / 32];
+    const int64_t r0 = (int64_t)blockIdx.y * 128, c0 = (int64_t)blockIdx.x * 64;
+    const int64_t end = __ldg(seg + E);
+    if (r0 >= end) return;                                 // the whole block leaves together
+    const int cl = threadIdx.x & 63, rg = threadIdx.x >> 6;
+    const int64_t c = c0 + cl;
+    float m = 0.0f;
+    for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(src(r0 + rg * 32 + i, c)));
+    part[rg][cl] = m;
+    __syncthreads();
+    int64_t lo = 0, hi = E;                                // seg[lo] <= r0 < seg[hi]
+    while (hi - lo > 1) {
+        const int64_t mid = (lo + hi) >> 1;
+        if (__ldg(seg + mid) <= r0) lo = mid; else hi = mid;
+    }
+    if (per_row) {
+        if (threadIdx.x < 64) {
+            const float v = fmaxf(fmaxf(part[0][cl], part[1][cl]), fmaxf(part[2][cl], part[3][cl]));
+            atomicMax(amax_bits + lo * C + c, __float_as_uint(v));
+        }
+    } else {
+        const float v = block_reduce_max(part[rg][cl], red);
+        if (threadIdx.x == 0) atomicMax(amax_bits + lo, __float_as_uint(v));
+    }
+}
+
+// Pass 2: one thread per output block of 16 tokens; consecutive threads take
+// consecutive columns c (output rows).
+template <int R, bool kSR, typename Src>
+__global__ void __launch_bounds__(kThreads)
+segment_quantize_kernel(Src src, const int64_t* __restrict__ seg, int64_t E, int64_t M, int64_t C, int per_row,
+                        const float* __restrict__ out_outer, uint64_t seed, uint64_t stream_id, int out_layout,
+                        uint8_t* __restrict__ out_codes, uint8_t* __restrict__ out_sf) {
+    const int64_t nb = M / 16;
+    const int64_t item = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+    if (item >= nb * C) return;
+    const int64_t c = item % C, b = item / C;
+    const int64_t t0 = b * 16;
+    uint32_t scode = 0;
+    uint2 packed = make_uint2(0u, 0u);
+    if (t0 < __ldg(seg + E)) {
+        int64_t lo = 0, hi = E;
+        while (hi - lo > 1) {
+            const int64_t mid = (lo + hi) >> 1;
+            if (__ldg(seg + mid) <= t0) lo = mid; else hi = mid;
+        }
+        float v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = src(t0 + i, c);
+        const float s = __ldg(out_outer + (per_row ? lo * C + c : lo));
+        quantize_block16<R, kSR>(v, s, seed, stream_id, (uint64_t)(c * M + t0), scode, packed);
+    }
+    *reinterpret_cast<uint2*>(out_codes + (c * M + t0) / 2) = packed;
+    out_sf[sf_offset(c, b, nb, out_layout)] = (uint8_t)scode;
+}
+
 template <bool kSR, typename F>
 int dispatch_rbits(int rbits, F&& f) {
     if (!kSR) return f(std::integral_constant<int, 16>{});
@@ -375,4 +463,80 @@ extern "C" int nvfp4_quantize_tile16(const void* x, int64_t rows, int64_t cols, 
         static_cast<const uint16_t*>(x), rows, cols, group_rows, outer, codes, sf_tile);
     mx_count_launch();
     return mx_launch_status();
+}
+
+namespace {
+
+template <typename Src>
+int segments_common(Src src, int64_t M, int64_t C, const int64_t* seg, int64_t E, int per_row, int rounding,
+                    uint64_t seed, uint64_t stream_id, int rbits, uint8_t* out_codes, uint8_t* out_sf,
+                    float* out_outer, int out_sf_layout, cudaStream_t stream) {
+    const int64_t n_outer = per_row ? E * C : E;
+    cudaError_t ce = cudaMemsetAsync(out_outer, 0, (size_t)n_outer * sizeof(float), stream);
+    if (ce != cudaSuccess) return mx_set_cuda_error(ce);
+    segment_amax_kernel<Src><<<dim3((unsigned)(C / 64), (unsigned)(M / 128)), kThreads, 0, stream>>>(
+        src, seg, E, C, per_row, reinterpret_cast<uint32_t*>(out_outer));
+    mx_count_launch();
+    amax_to_outer_kernel<<<(unsigned)((n_outer + kThreads - 1) / kThreads), kThreads, 0, stream>>>(out_outer,
+                                                                                                   n_outer);
+    mx_count_launch();
+    const int64_t items = (M / 16) * C;
+    const unsigned grid = (unsigned)((items + kThreads - 1) / kThreads);
+    auto launch = [&](auto kSRc) {
+        constexpr bool kSR = decltype(kSRc)::value;
+        return dispatch_rbits<kSR>(rbits, [&](auto Rc) {
+            segment_quantize_kernel<decltype(Rc)::value, kSR, Src><<<grid, kThreads, 0, stream>>>(
+                src, seg, E, M, C, per_row, out_outer, seed, stream_id, out_sf_layout, out_codes, out_sf);
+            mx_count_launch();
+            return mx_launch_status();
+        });
+    };
+    return rounding == MX_ROUND_SR ? launch(std::true_type{}) : launch(std::false_type{});
+}
+
+int segments_check(int64_t M, int64_t C, const int64_t* seg, int64_t E, int per_row, int rounding, int rbits,
+                   const uint8_t* out_codes, const uint8_t* out_sf, const float* out_outer, int out_sf_layout) {
+    if (((!seg || !out_codes || !out_sf || !out_outer) && M > 0) || M < 0 || M % 128 || C <= 0 || C % 64 || E < 1 ||
+        !mx_aligned(out_codes, 16) || !mx_aligned(out_outer, 4))
+        return MX_EINVAL;
+    if (per_row != 0 && per_row != 1) return MX_EINVAL;
+    if (rounding != MX_ROUND_RNE && rounding != MX_ROUND_SR) return MX_EINVAL;
+    if (rounding == MX_ROUND_SR && rbits != 8 && rbits != 16 && rbits != 32) return MX_EINVAL;
+    if (out_sf_layout != MX_SF_ROWMAJOR && out_sf_layout != MX_SF_MMA) return MX_EINVAL;
+    if (out_sf_layout == MX_SF_MMA && C % 128) return MX_EINVAL;
+    return MX_OK;
+}
+
+}  // namespace
+
+extern "C" int nvfp4_quantize_transpose_segments(const void* x, int64_t M, int64_t C, const int64_t* seg, int64_t E,
+                                                 int per_row, int rounding, uint64_t seed, uint64_t stream_id,
+                                                 int rbits, uint8_t* out_codes, uint8_t* out_sf, float* out_outer,
+                                                 int out_sf_layout, cudaStream_t stream) {
+    MX_NVTX_RANGE("nvfp4_quantize_transpose_segments");
+    if ((!x && M > 0) || !mx_aligned(x, 16)) return MX_EINVAL;
+    if (int st = segments_check(M, C, seg, E, per_row, rounding, rbits, out_codes, out_sf, out_outer, out_sf_layout))
+        return st;
+    if (int st = mx_check_device()) return st;
+    if (M == 0) return MX_OK;
+    return segments_common(Bf16Src{static_cast<const uint16_t*>(x), C}, M, C, seg, E, per_row, rounding, seed,
+                           stream_id, rbits, out_codes, out_sf, out_outer, out_sf_layout, stream);
+}
+
+extern "C" int nvfp4_requant_transpose_segments(const uint8_t* codes, const uint8_t* sf, const float* outer,
+                                                int in_sf_layout, int64_t group_rows, int64_t M, int64_t C,
+                                                const int64_t* seg, int64_t E, int per_row, int rounding,
+                                                uint64_t seed, uint64_t stream_id, int rbits, uint8_t* out_codes,
+                                                uint8_t* out_sf, float* out_outer, int out_sf_layout,
+                                                cudaStream_t stream) {
+    MX_NVTX_RANGE("nvfp4_requant_transpose_segments");
+    if (((!codes || !sf || !outer) && M > 0) || group_rows <= 0 || M % group_rows || !mx_aligned(codes, 16))
+        return MX_EINVAL;
+    if (in_sf_layout != MX_SF_ROWMAJOR && in_sf_layout != MX_SF_MMA) return MX_EINVAL;
+    if (int st = segments_check(M, C, seg, E, per_row, rounding, rbits, out_codes, out_sf, out_outer, out_sf_layout))
+        return st;
+    if (int st = mx_check_device()) return st;
+    if (M == 0) return MX_OK;
+    return segments_common(Nvfp4Src{codes, sf, outer, C, group_rows, in_sf_layout}, M, C, seg, E, per_row, rounding,
+                           seed, stream_id, rbits, out_codes, out_sf, out_outer, out_sf_layout, stream);
 }

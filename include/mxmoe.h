@@ -406,6 +406,33 @@ MX_API int nvfp4_requant_transpose_sr(const uint8_t* codes, const uint8_t* sf, c
 MX_API int nvfp4_quantize_tile16(const void* x, int64_t rows, int64_t cols, int64_t group_rows, uint8_t* codes,
                                  uint8_t* sf_tile, float* outer, cudaStream_t stream);
 
+/* The wgrad operands of an NVFP4 backward: NVFP4 of the transpose [C, M] of a
+ * token-major [M, C] tensor in expert-major row order (seg [E+1] from
+ * moe_route: segment starts and lengths multiples of 128), blocks of 16 along
+ * the tokens, with outer scales per expert segment so that the wgrad GEMM
+ * applies a per-row times a per-expert factor: per (segment, row) when
+ * per_row = 1 (out_outer [E, C], for dY^T), per segment when per_row = 0
+ * (out_outer [E], for X^T).  Each scale is the segment's amax / 2688; rounding
+ * as above with L = c*M + t; tokens at or past seg[E] quantise to zero.
+ *   out_codes device u8 [C, M/2]; out_sf device u8 mx_sf_bytes(C, M, 16,
+ *   out_sf_layout); out_outer written twice (maxima, then scales).
+ * Requires M % 128 == 0, C % 64 == 0 (C % 128 == 0 for an MX_SF_MMA output),
+ * 16-byte aligned inputs and out_codes.  Segment boundaries off multiples of
+ * 128 give wrong scales (no out-of-bounds access). */
+MX_API int nvfp4_quantize_transpose_segments(const void* x, int64_t M, int64_t C, const int64_t* seg, int64_t E,
+                                             int per_row, int rounding, uint64_t seed, uint64_t stream_id,
+                                             int rbits, uint8_t* out_codes, uint8_t* out_sf, float* out_outer,
+                                             int out_sf_layout, cudaStream_t stream);
+
+/* The same from a saved NVFP4 tensor [M, C] (codes, sf in in_sf_layout, outer
+ * per group_rows rows), each value dequantised ((q * sf) * outer, fp32). */
+MX_API int nvfp4_requant_transpose_segments(const uint8_t* codes, const uint8_t* sf, const float* outer,
+                                            int in_sf_layout, int64_t group_rows, int64_t M, int64_t C,
+                                            const int64_t* seg, int64_t E, int per_row, int rounding,
+                                            uint64_t seed, uint64_t stream_id, int rbits, uint8_t* out_codes,
+                                            uint8_t* out_sf, float* out_outer, int out_sf_layout,
+                                            cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -96,6 +96,16 @@ CASES = {
         ("unknown out layout", {16: 3}), ("outer-per-expert flag 2", {8: 2}), ("out codes misaligned", {13: A8}),
         ("null out outer", {15: None}), ("out outer misaligned", {15: A1}),
     ]),
+    "nvfp4_quantize_transpose_segments": ((A, 256, 128, A, 2, 1, 1, 1, 2, 16, A, A, A, 1, None), [
+        ("M % 128", {1: 192}), ("C % 64", {2: 96}), ("no experts", {4: 0}), ("per_row 2", {5: 2}),
+        ("MMA output C % 128", {2: 64}), ("null seg", {3: None}), ("x misaligned", {0: A8}),
+        ("SR with rbits 4", {9: 4}),
+    ]),
+    "nvfp4_requant_transpose_segments": ((A, A, A, 1, 1, 256, 128, A, 2, 0, 1, 1, 2, 16, A, A, A, 1, None), [
+        ("unknown input layout", {3: 4}), ("group_rows 0", {4: 0}), ("M % group_rows", {4: 3}),
+        ("codes misaligned", {0: A8}), ("M % 128", {5: 64}), ("out outer misaligned", {16: A1}),
+        ("unknown rounding", {10: 5}),
+    ]),
     "nvfp4_quantize_tile16": ((A, 64, 48, 32, A, A, A, None), [
         ("rows % 16", {1: 40}), ("cols % 16", {2: 40}), ("group_rows % 16", {3: 8}), ("rows % group_rows", {3: 48}),
         ("codes misaligned", {4: A8}), ("null sf_tile", {5: None}),

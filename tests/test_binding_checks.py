@@ -186,3 +186,17 @@ def test_nvfp4_backward_buffers():
     t = bf16(64, 48)
     _passes_size_checks(lambda: api.nvfp4_quantize_tile16(t, 32, out=(u8(64, 24), u8(4, 3), f32(2))))
     _size_error(lambda: api.nvfp4_quantize_tile16(t, 32, out=(u8(64, 24), u8(4, 2), f32(2))), "sf_tile")
+
+
+def test_segment_transpose_buffers():
+    M, C, E = 256, 128, 2
+    seg = torch.zeros(E + 1, dtype=torch.int64)
+    x = bf16(M, C)
+    out = (u8(C, M // 2), u8(C * M // 16), f32(E * C))
+    _passes_size_checks(lambda: api.nvfp4_quantize_transpose_segments(x, seg, E, True, out=out))
+    _size_error(lambda: api.nvfp4_quantize_transpose_segments(x, seg, E, True, out=(out[0], out[1], f32(E))),
+                "out outer")                                   # per (segment, row) needs E * C scales
+    _size_error(lambda: api.nvfp4_quantize_transpose_segments(x, seg[:-1], E, True, out=out), "seg")
+    q = (u8(M, C // 2), u8(M * C // 16), f32(M))
+    _passes_size_checks(lambda: api.nvfp4_requant_transpose_segments(*q, M, C, seg, E, out=(out[0], out[1], f32(E))))
+    _size_error(lambda: api.nvfp4_requant_transpose_segments(q[0][:-1], q[1], q[2], M, C, seg, E), "codes")

@@ -123,3 +123,39 @@ def test_nvfp4_dgrad_through_the_forward_gemm(cuda):
     rdq = oracle.nvfp4_quantize_f32(oracle.bf16_to_f32(dy), 1, True, 3, 6, 16)
     ref = oracle.grouped_gemm_nvfp4(*rdq, *rwt, seg, K)
     assert rel_fro(host(dx).astype(np.float64), ref) <= 1e-4
+
+
+def _segments(counts):
+    seg = np.zeros(len(counts) + 1, dtype=np.int64)
+    seg[1:] = np.cumsum([(c + 127) // 128 * 128 for c in counts])
+    return seg
+
+
+@pytest.mark.parametrize("per_row", [True, False])
+def test_transpose_segments_from_bf16_bit_exact(cuda, per_row):
+    seg = _segments([200, 0, 90, 300])
+    M, C = int(seg[-1]) + 128, 128                                # one block of padding rows
+    x = bf16_input(M, C, 21)
+    oc, osf, oo = api.nvfp4_quantize_transpose_segments(to_dev_bf16(x), dev(seg), len(seg) - 1, per_row,
+                                                        api.MX_ROUND_SR, 8, 9, 16, api.MX_SF_MMA)
+    api.sync_status()
+    rc, rsf, ro = oracle.nvfp4_quantize_transpose_segments(oracle.bf16_to_f32(x), seg, per_row, True, 8, 9, 16)
+    assert np.array_equal(host(oo), ro.reshape(-1))
+    assert np.array_equal(mma_to_rowmajor(host(osf), C, M // 16), rsf)
+    assert np.array_equal(host(oc), rc)
+
+
+def test_requant_transpose_segments_bit_exact(cuda):
+    from tests.layouts import rowmajor_to_mma
+    seg = _segments([130, 60, 0, 250])
+    M, C = int(seg[-1]), 256
+    q = oracle.nvfp4_quantize(bf16_input(M, C, 22))
+    oc, osf, oo = api.nvfp4_requant_transpose_segments(dev(q[0]), dev(rowmajor_to_mma(q[1])), dev(q[2]), M, C,
+                                                       dev(seg), len(seg) - 1, False, 1, api.MX_SF_MMA,
+                                                       api.MX_ROUND_SR, 10, 11, 8, api.MX_SF_MMA)
+    api.sync_status()
+    xh = oracle.nvfp4_dequantize(*q)
+    rc, rsf, ro = oracle.nvfp4_quantize_transpose_segments(xh, seg, False, True, 10, 11, 8)
+    assert np.array_equal(host(oo), ro)
+    assert np.array_equal(mma_to_rowmajor(host(osf), C, M // 16), rsf)
+    assert np.array_equal(host(oc), rc)

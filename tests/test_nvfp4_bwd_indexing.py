@@ -118,3 +118,59 @@ def test_tile16_kernel_indexing(rows, cols, group_rows):
     _exactly_once(tr[lead] * ntc + tc[lead], 1, rows // 16 * ntc)
     # every warp's lanes belong to one tile (the warp leaves or stays whole)
     assert np.all(np.diff(tile.reshape(-1, 32), axis=1) == 0)
+
+
+def _find_expert(seg, E, t):
+    lo, hi = 0, E                                # seg[lo] <= t < seg[hi]
+    while hi - lo > 1:
+        mid = (lo + hi) >> 1
+        if seg[mid] <= t:
+            lo = mid
+        else:
+            hi = mid
+    return lo
+
+
+@pytest.mark.parametrize("M,C,seg,per_row,out_mma,in_mma,group_rows", [
+    (512, 128, [0, 128, 128, 384], True, True, True, 1),          # an empty expert, 128 padding rows
+    (384, 64, [0, 384], False, False, False, 1),
+    (640, 256, [0, 0, 256, 256, 512, 512], True, True, True, 128),
+])
+def test_segment_kernels_indexing(M, C, seg, per_row, out_mma, in_mma, group_rows):
+    seg = np.array(seg)
+    E = len(seg) - 1
+    # the shapes the entry points accept; segments as moe_route writes them
+    assert M % 128 == 0 and C % 64 == 0 and (not out_mma or C % 128 == 0) and M % group_rows == 0
+    assert np.all(seg % 128 == 0) and seg[-1] <= M and np.all(np.diff(seg) >= 0)
+    end = seg[E]
+    n_outer = E * C if per_row else E
+    # pass 1: grid (C / 64, M / 128); blocks at or past seg[E] leave before any barrier
+    for by in range(M // 128):
+        r0 = by * 128
+        if r0 >= end:
+            continue
+        lo = _find_expert(seg, E, r0)
+        assert seg[lo] <= r0 and r0 + 127 < seg[lo + 1]              # the tile lies in one segment
+        for bx in range(C // 64):
+            c = bx * 64 + np.arange(64)
+            rows = r0 + np.arange(128)
+            assert rows.max() < M and c.max() < C
+            assert ((rows[:, None] * C + c[None, :]) // 2).max() < M * C // 2       # NVFP4 source bytes
+            assert (rows[:, None] * C + c[None, :]).max() < M * C                    # bf16 source elements
+            offs = [sf_offset(int(r), int(cc) // 16, C // 16, in_mma) for r in rows[::31] for cc in c[::15]]
+            assert max(offs) < M * (C // 16) and (rows // group_rows).max() < M // group_rows
+            tg = lo * C + c if per_row else np.array([lo])
+            assert tg.min() >= 0 and tg.max() < n_outer
+    # pass 2: one thread per output block of 16 tokens, c fastest
+    nb = M // 16
+    item = _threads(nb * C)
+    c, b = item % C, item // C
+    t0 = b * 16
+    assert (t0 + 15).max() < M
+    for tt in np.unique(t0[t0 < end]):
+        lo = _find_expert(seg, E, int(tt))
+        assert seg[lo] <= tt < seg[lo + 1]
+    _exactly_once((c * M + t0) // 2, 8, C * M // 2)
+    _exactly_once([sf_offset(int(a), int(bb), nb, out_mma) for a, bb in zip(c, b)], 1, C * nb)
+    L = (c * M + t0)[:, None] + np.arange(16)[None, :]
+    assert np.array_equal(np.sort(L.reshape(-1)), np.arange(C * M))
