@@ -57,6 +57,7 @@ SIGNATURES = {
     "nvfp4_quantize_transpose_segments": (I32, [P, I64, I64, P, I64, I32, I32, U64, U64, I32, P, P, P, I32, P]),
     "nvfp4_requant_transpose_segments": (I32, [P, P, P, I32, I64, I64, I64, P, I64, I32, I32, U64, U64, I32, P, P,
                                                P, I32, P]),
+    "grouped_gemm_nvfp4_wgrad": (I32, [P, P, P, P, P, P, P, I64, I64, I64, I64, P, I32, P]),
 }
 
 _lib = None

@@ -27,7 +27,7 @@ __all__ = [
     "grouped_gemm_nvfp4", "grouped_gemm_mxfp8", "moe_route", "nvfp4_gather_rows", "swiglu_fwd", "swiglu_bwd",
     "moe_combine", "moe_dispatch_grad", "swiglu_nvfp4_quantize", "hadamard_s2f6_quantize", "grouped_gemm_nvfp4_s2f6",
     "moe_combine_s2f6", "nvfp4_quantize_sr", "nvfp4_requant_transpose_sr", "nvfp4_quantize_tile16",
-    "nvfp4_quantize_transpose_segments", "nvfp4_requant_transpose_segments",
+    "nvfp4_quantize_transpose_segments", "nvfp4_requant_transpose_segments", "grouped_gemm_nvfp4_wgrad",
 ]
 
 
@@ -460,3 +460,22 @@ def nvfp4_requant_transpose_segments(codes, sf, outer, M: int, C: int, seg: torc
            E, int(per_row), rounding, ctypes.c_uint64(seed), ctypes.c_uint64(stream_id), rbits, _p(oc), _p(osf),
            _p(oo), out_sf_layout, _s())
     return oc, osf, oo
+
+
+def grouped_gemm_nvfp4_wgrad(a, b, seg: torch.Tensor, E: int, N: int, K: int, out_dtype=torch.float32, out=None):
+    """a = (codes [N, M_cap/2], sf, outer [E*N]); b = (codes [K, M_cap/2], sf, outer [E]).
+    Returns out [E, N, K] = per-expert sums over the segment's tokens (segments at multiples of 256)."""
+    M_cap = a[0].shape[1] * 2
+    if out is None:
+        out = torch.empty(E, N, K, dtype=out_dtype, device=a[0].device)
+    _fits("a codes", a[0], N * M_cap // 2)
+    _fits("a sf", a[1], N * (M_cap // 16))
+    _fits("a outer", a[2], 4 * E * N)
+    _fits("b codes", b[0], K * M_cap // 2)
+    _fits("b sf", b[1], K * (M_cap // 16))
+    _fits("b outer", b[2], 4 * E)
+    _fits("seg", seg, 8 * (E + 1))
+    _fits("out", out, E * N * K * out.element_size())
+    L.call("grouped_gemm_nvfp4_wgrad", _p(a[0]), _p(a[1]), _p(a[2]), _p(b[0]), _p(b[1]), _p(b[2]), _p(seg), E, M_cap,
+           N, K, _p(out), _out_code(out.dtype), _s())
+    return out

@@ -353,12 +353,21 @@ __device__ __forceinline__ Tile make_tile(const GemmArgs& p, int64_t idx, uint32
         t.a_y = tn * rows + half;
         t.row0 = t.e * p.N + t.a_y;
         t.col0 = tk * kBN;
-        t.k_tiles = (s1 - s0) / kStageBytesK;
-        t.k0_bytes = s0;
         t.b_x0 = 0;
         t.b_y = t.col0 + b_half;
-        t.sfa_atom0 = t.a_y / kBM * p.sfa_groups + s0 / 128;
-        t.sfb_atom0 = t.col0 / kBM * p.sfb_groups + s0 / 128;
+        if constexpr (kKind == kKindNVFP4) {
+            // two tokens per K-byte: a stage holds 256 tokens, a scale atom
+            // 64 (segments are multiples of 256 tokens)
+            t.k_tiles = (s1 - s0) / (2 * kStageBytesK);
+            t.k0_bytes = s0 / 2;
+            t.sfa_atom0 = t.a_y / kBM * p.sfa_groups + s0 / 64;
+            t.sfb_atom0 = t.col0 / kBM * p.sfb_groups + s0 / 64;
+        } else {
+            t.k_tiles = (s1 - s0) / kStageBytesK;
+            t.k0_bytes = s0;
+            t.sfa_atom0 = t.a_y / kBM * p.sfa_groups + s0 / 128;
+            t.sfb_atom0 = t.col0 / kBM * p.sfb_groups + s0 / 128;
+        }
     }
     return t;
 }
@@ -1153,5 +1162,42 @@ extern "C" int grouped_gemm_mxfp8(int mode, const uint8_t* a_codes, const uint8_
     a.sfa_groups = M_cap / 128; a.sfb_groups = M_cap / 128; a.ldo = K;
     const bool pair = N % 256 == 0 && K % 256 == 0;
     return dispatch<kKindMXFP8, kModeWgrad>(pair, E * N, K, out_dtype, ma, mb, a, E * (N / 256) * (K / 256),
+                                            E * (N / 128) * (K / 128), stream);
+}
+
+// NVFP4 weight gradient (the NVFP4 backward's wgrad): A [N, M_cap] and B
+// [K, M_cap] in NVFP4 along the tokens (codes [rows, M_cap/2], scales in the
+// MMA layout), outer scales per expert segment: a_outer [E*N] (segment,
+// row), b_outer [E].  out[e, n, k] = a_outer[e*N + n] * b_outer[e] * sum over
+// the tokens of segment e.  Segments must be multiples of 256 tokens (a
+// K-stage of NVFP4 holds 256); other boundaries give wrong sums, no
+// out-of-bounds access.  Not yet run on a GPU.
+extern "C" int grouped_gemm_nvfp4_wgrad(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_outer,
+                                        const uint8_t* b_codes, const uint8_t* b_sf, const float* b_outer,
+                                        const int64_t* seg_offsets, int64_t E, int64_t M_cap, int64_t N, int64_t K,
+                                        void* out, int out_dtype, cudaStream_t stream) {
+    MX_NVTX_RANGE("grouped_gemm_nvfp4_wgrad");
+    if (((!a_codes || !a_sf || !a_outer || !b_codes || !b_sf || !b_outer || !seg_offsets) && M_cap > 0) || !out ||
+        E < 1 || M_cap < 0 || M_cap % 256 || N <= 0 || N % 128 || K <= 0 || K % 128)
+        return MX_EINVAL;
+    if (out_dtype != MX_OUT_F32 && out_dtype != MX_OUT_BF16) return MX_EINVAL;
+    if (!mx_aligned(a_codes, 16) || !mx_aligned(b_codes, 16) || !mx_aligned(a_sf, 16) || !mx_aligned(b_sf, 16) ||
+        !mx_aligned(out, 16))
+        return MX_EINVAL;
+    if (M_cap >= (int64_t)1 << 31 || E * N >= (int64_t)1 << 31 || K >= (int64_t)1 << 31) return MX_EINVAL;
+    if (int st = mx_check_device()) return st;
+    if (M_cap == 0) {                                   // no routed rows: every dW_e is zero
+        const cudaError_t e = cudaMemsetAsync(out, 0, (size_t)(E * N * K) * (out_dtype == MX_OUT_BF16 ? 2 : 4), stream);
+        return e == cudaSuccess ? MX_OK : mx_set_cuda_error(e);
+    }
+    CUtensorMap ma, mb;
+    if (int st = make_map(&ma, a_codes, N, M_cap / 2, kBM)) return st;
+    if (int st = make_map(&mb, b_codes, K, M_cap / 2, 128)) return st;
+    GemmArgs a{};
+    a.sfa = a_sf; a.sfb = b_sf; a.a_outer = a_outer; a.b_outer = b_outer; a.seg = seg_offsets; a.out = out;
+    a.E = E; a.M_cap = M_cap; a.N = N; a.K = K;
+    a.sfa_groups = M_cap / 64; a.sfb_groups = M_cap / 64; a.ldo = K;
+    const bool pair = N % 256 == 0 && K % 256 == 0;
+    return dispatch<kKindNVFP4, kModeWgrad>(pair, E * N, K, out_dtype, ma, mb, a, E * (N / 256) * (K / 256),
                                             E * (N / 128) * (K / 128), stream);
 }

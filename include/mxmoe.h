@@ -433,6 +433,23 @@ MX_API int nvfp4_requant_transpose_segments(const uint8_t* codes, const uint8_t*
                                             uint8_t* out_sf, float* out_outer, int out_sf_layout,
                                             cudaStream_t stream);
 
+/* grouped_gemm_nvfp4_wgrad -- the NVFP4 weight gradient on tcgen05
+ * block-scaled MMA (kind::mxf4nvf4, the MXFP8 WGRAD tile schedule).
+ *   A: NVFP4 [N, M_cap] (dY^T, codes [N, M_cap/2], sf MX_SF_MMA), a_outer
+ *      [E*N] per (segment, row); B: NVFP4 [K, M_cap] (X^T), b_outer [E] per
+ *      segment -- as nvfp4_quantize_transpose_segments /
+ *      nvfp4_requant_transpose_segments write them;
+ *   out[e, n, k] = a_outer[e*N + n] * b_outer[e] * sum over the tokens t of
+ *      segment e of (qa*sfa)[n, t] * (qb*sfb)[k, t], fp32 accumulate; out
+ *      [E, N, K] f32 or bf16; an empty expert gets zeros.
+ * Requires segments at multiples of 256 tokens (a K-stage of NVFP4 holds 256
+ * tokens; other boundaries give wrong sums, no out-of-bounds access),
+ * M_cap % 256 == 0, N % 128 == 0, K % 128 == 0, 16-byte aligned operands. */
+MX_API int grouped_gemm_nvfp4_wgrad(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_outer,
+                                    const uint8_t* b_codes, const uint8_t* b_sf, const float* b_outer,
+                                    const int64_t* seg_offsets, int64_t E, int64_t M_cap, int64_t N, int64_t K,
+                                    void* out, int out_dtype, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -106,6 +106,11 @@ CASES = {
         ("codes misaligned", {0: A8}), ("M % 128", {5: 64}), ("out outer misaligned", {16: A1}),
         ("unknown rounding", {10: 5}),
     ]),
+    "grouped_gemm_nvfp4_wgrad": ((A, A, A, A, A, A, A, 2, 512, 128, 256, A, 0, None), [
+        ("M_cap % 256", {8: 384}), ("N % 128", {9: 64}), ("K % 128", {10: 64}), ("no experts", {7: 0}),
+        ("unknown out_dtype", {12: 2}), ("a_sf misaligned", {1: A4}), ("null out", {11: None}),
+        ("null seg", {6: None}),
+    ]),
     "nvfp4_quantize_tile16": ((A, 64, 48, 32, A, A, A, None), [
         ("rows % 16", {1: 40}), ("cols % 16", {2: 40}), ("group_rows % 16", {3: 8}), ("rows % group_rows", {3: 48}),
         ("codes misaligned", {4: A8}), ("null sf_tile", {5: None}),

@@ -200,3 +200,14 @@ def test_segment_transpose_buffers():
     q = (u8(M, C // 2), u8(M * C // 16), f32(M))
     _passes_size_checks(lambda: api.nvfp4_requant_transpose_segments(*q, M, C, seg, E, out=(out[0], out[1], f32(E))))
     _size_error(lambda: api.nvfp4_requant_transpose_segments(q[0][:-1], q[1], q[2], M, C, seg, E), "codes")
+
+
+def test_nvfp4_wgrad_buffers():
+    E, M, N, K = 2, 512, 128, 256
+    seg = torch.zeros(E + 1, dtype=torch.int64)
+    a = (u8(N, M // 2), u8(N * M // 16), f32(E * N))
+    b = (u8(K, M // 2), u8(K * M // 16), f32(E))
+    _passes_size_checks(lambda: api.grouped_gemm_nvfp4_wgrad(a, b, seg, E, N, K, out=f32(E, N, K)))
+    _size_error(lambda: api.grouped_gemm_nvfp4_wgrad((a[0], a[1], f32(N)), b, seg, E, N, K, out=f32(E, N, K)),
+                "a outer")                                     # one scale per (segment, row)
+    _size_error(lambda: api.grouped_gemm_nvfp4_wgrad(a, b, seg, E, N, K, out=f32(E, N, K - 1)), "out")

@@ -159,3 +159,28 @@ def test_requant_transpose_segments_bit_exact(cuda):
     assert np.array_equal(host(oo), ro)
     assert np.array_equal(mma_to_rowmajor(host(osf), C, M // 16), rsf)
     assert np.array_equal(host(oc), rc)
+
+
+@pytest.mark.parametrize("Nw,Kw,counts", [(256, 256, [300, 0, 200, 512]), (128, 384, [100, 40])])
+def test_nvfp4_wgrad_gemm(cuda, Nw, Kw, counts):
+    # operands from the oracle (segments at multiples of 256 tokens), the GEMM on the GPU
+    from tests.layouts import rowmajor_to_mma
+    seg = np.zeros(len(counts) + 1, dtype=np.int64)
+    seg[1:] = np.cumsum([(c + 255) // 256 * 256 for c in counts])
+    E, M = len(counts), int(seg[-1])
+    rng = np.random.default_rng(Nw + Kw)
+    dy = (rng.standard_normal((M, Nw)) * 10.0 ** rng.uniform(-2, 2, (M, 1))).astype(np.float32)
+    x = rng.standard_t(3, (M, Kw)).astype(np.float32)
+    a = oracle.nvfp4_quantize_transpose_segments(dy, seg, True, True, 3, 4, 16)
+    b = oracle.nvfp4_quantize_transpose_segments(x, seg, False, True, 3, 5, 16)
+    A = (dev(a[0]), dev(rowmajor_to_mma(a[1])), dev(a[2].reshape(-1)))
+    B = (dev(b[0]), dev(rowmajor_to_mma(b[1])), dev(b[2]))
+    out = api.grouped_gemm_nvfp4_wgrad(A, B, dev(seg), E, Nw, Kw, out_dtype=torch.float32)
+    api.sync_status()
+    ref = oracle.grouped_gemm_nvfp4_wgrad(*a, *b, seg)
+    got = host(out).astype(np.float64)
+    for e in range(E):
+        if seg[e + 1] == seg[e]:
+            assert np.all(got[e] == 0)
+        else:
+            assert rel_fro(got[e], ref[e]) <= 1e-4

@@ -174,3 +174,41 @@ def test_segment_kernels_indexing(M, C, seg, per_row, out_mma, in_mma, group_row
     _exactly_once([sf_offset(int(a), int(bb), nb, out_mma) for a, bb in zip(c, b)], 1, C * nb)
     L = (c * M + t0)[:, None] + np.arange(16)[None, :]
     assert np.array_equal(np.sort(L.reshape(-1)), np.arange(C * M))
+
+
+@pytest.mark.parametrize("M,N,K,seg,pair", [
+    (1280, 256, 256, [0, 512, 512, 768, 1280], True),
+    (512, 128, 384, [0, 256, 512], False),
+])
+def test_nvfp4_wgrad_tile_mapping(M, N, K, seg, pair):
+    # csrc/gemm.cu make_tile, WGRAD branch with NVFP4 operands: A [N, M] and B
+    # [K, M] codes (M/2 bytes per row), scale atoms of 128 rows x 64 tokens
+    seg = np.array(seg)
+    assert np.all(seg % 256 == 0) and seg[-1] <= M and M % 256 == 0
+    kBM, kStage = 128, 128
+    kBN = 256 if pair else 128
+    rows = 2 * kBM if pair else kBM
+    groups = M // 64                                             # sfa_groups = sfb_groups
+    atoms_a, atoms_b = (N // 128) * groups, (K // 128) * groups
+    E = len(seg) - 1
+    for idx in range(E * (N // rows) * (K // kBN)):
+        e = idx // ((N // rows) * (K // kBN))
+        rem = idx % ((N // rows) * (K // kBN))
+        tn, tk = rem // (K // kBN), rem % (K // kBN)
+        s0, s1 = seg[e], seg[e + 1]
+        for rank in ((0, 1) if pair else (0,)):
+            a_y = tn * rows + rank * kBM
+            col0 = tk * kBN
+            b_y = col0 + (rank * kBN // 2 if pair else 0)
+            k_tiles, k0 = (s1 - s0) // (2 * kStage), s0 // 2
+            sfa0 = a_y // kBM * groups + s0 // 64
+            sfb0 = col0 // kBM * groups + s0 // 64
+            assert a_y + kBM <= N and b_y + (kBN // 2 if pair else kBN) <= K
+            for kt in range(k_tiles):
+                kx = k0 + kt * kStage
+                assert kx % 16 == 0 and kx + kStage <= M // 2          # TMA x aligned and inside the row
+                assert sfa0 + kt * 4 + 4 <= atoms_a
+                for h in range(kBN // 128):
+                    assert sfb0 + h * groups + kt * 4 + 4 <= atoms_b
+            # the stages cover the segment's tokens exactly
+            assert k_tiles * 256 == s1 - s0
