@@ -581,7 +581,7 @@ def cpu_baseline(inp, layer, seconds: float = 15.0):
 # larger than L2 where DRAM traffic is read off)
 # --------------------------------------------------------------------------
 KERNEL_CASES = ("gemm_nvfp4", "gemm_nvfp4_s2f6", "gemm_mxfp8_dgrad", "gemm_mxfp8_wgrad", "requant", "requant_w",
-                "nvfp4_quantize", "quant_w", "mxfp8_quantize", "nvfp4_quantize_sr", "requant_nvfp4")
+                "nvfp4_quantize", "quant_w", "mxfp8_quantize", "nvfp4_quantize_sr", "requant_nvfp4", "gemm_nvfp4_wgrad")
 
 
 def run_kernel(args):
@@ -607,6 +607,24 @@ def run_kernel(args):
             a = api.nvfp4_quantize(workloads.activations(M, F, "t3", 4, dev), 1, api.MX_SF_MMA)
             w2q = api.nvfp4_quantize(workloads.weights(E, D, F, 0.02, 5, dev).view(E * D, F), D, api.MX_SF_MMA)
             run = lambda: api.grouped_gemm_nvfp4_s2f6(a, w2q, seg, E, D, F, 1, 101)
+        elif which == "gemm_nvfp4_wgrad":
+            # dW1 in NVFP4 on the same routing with segments padded to 256 tokens: A = dH^T [2F, M256],
+            # B = X^T [D, M256]; valid random codes and scales (the kernel's time does not depend on them)
+            cnt = (seg[1:] - seg[:-1]).cpu()
+            s256 = torch.zeros(E + 1, dtype=torch.int64)
+            s256[1:] = torch.cumsum((cnt + 255) // 256 * 256, 0)
+            M2 = int(s256[-1])
+            g = torch.Generator(device=dev)
+            g.manual_seed(8)
+            ops = []
+            for rows in (2 * F, D):
+                codes = torch.randint(0, 256, (rows, M2 // 2), dtype=torch.uint8, device=dev, generator=g)
+                sf = torch.randint(0x30, 0x48, (rows * M2 // 16,), dtype=torch.uint8, device=dev, generator=g)
+                ops.append((codes, sf))
+            A = (*ops[0], torch.full((E * 2 * F,), 1e-3, device=dev))
+            B = (*ops[1], torch.full((E,), 1e-3, device=dev))
+            s256 = s256.to(dev)
+            run = lambda: api.grouped_gemm_nvfp4_wgrad(A, B, s256, E, 2 * F, D, out_dtype=torch.bfloat16)
         else:
             dh = workloads.gradient(M, 2 * F, 1e-3, 3, dev)
             q = api.mxfp8_quantize(dh)
