@@ -41,6 +41,7 @@ SIGNATURES = {
     "mx_route_workspace_bytes": (SZ, [I64, I64]),
     "moe_route": (I32, [P, I64, I64, I64, I64, P, P, P, P, SZ, P]),
     "moe_route_static": (I32, [P, I64, I64, I64, I64, P, P, P, P]),
+    "moe_route_aligned": (I32, [P, I64, I64, I64, I64, I64, P, P, P, P, SZ, P]),
     "nvfp4_gather_rows": (I32, [P, P, P, P, I64, I64, I64, P, P, P, P]),
     "swiglu_fwd": (I32, [P, I64, I64, I32, P, P, P]),
     "swiglu_bwd": (I32, [P, P, I64, I64, I32, P, P, P]),

@@ -28,6 +28,7 @@ __all__ = [
     "moe_combine", "moe_dispatch_grad", "swiglu_nvfp4_quantize", "hadamard_s2f6_quantize", "grouped_gemm_nvfp4_s2f6",
     "moe_combine_s2f6", "nvfp4_quantize_sr", "nvfp4_requant_transpose_sr", "nvfp4_quantize_tile16",
     "nvfp4_quantize_transpose_segments", "nvfp4_requant_transpose_segments", "grouped_gemm_nvfp4_wgrad",
+    "max_routed_rows",
 ]
 
 
@@ -202,17 +203,18 @@ def grouped_gemm_mxfp8(mode: int, a_codes, a_e8m0, b_codes, b_e8m0, seg: torch.T
     return out
 
 
-def max_routed_rows(T: int, k: int, E: int) -> int:
-    cap = T * k + 127 * E
-    return (cap + 127) // 128 * 128
+def max_routed_rows(T: int, k: int, E: int, align: int = 128) -> int:
+    cap = T * k + (align - 1) * E
+    return (cap + align - 1) // align * align
 
 
-def moe_route(topk: torch.Tensor, E: int, M_cap: int | None = None, out=None):
-    """topk int32 [T, k] -> (seg int64 [E+1], src int32 [M_cap], pos int32 [T, k])."""
+def moe_route(topk: torch.Tensor, E: int, M_cap: int | None = None, out=None, align: int = 128):
+    """topk int32 [T, k] -> (seg int64 [E+1], src int32 [M_cap], pos int32 [T, k]); segments
+    padded to a multiple of `align` rows (128, or 256 for the NVFP4 wgrad)."""
     T, k = topk.shape
     dev = topk.device
     if M_cap is None:
-        M_cap = max_routed_rows(T, k, E)
+        M_cap = max_routed_rows(T, k, E, align)
     ws_bytes = L.lib().mx_route_workspace_bytes(T, E)
     if out is None:
         out = (torch.empty(E + 1, dtype=torch.int64, device=dev), torch.empty(M_cap, dtype=torch.int32, device=dev),
@@ -221,8 +223,12 @@ def moe_route(topk: torch.Tensor, E: int, M_cap: int | None = None, out=None):
     _fits("seg", seg, 8 * (E + 1))
     _fits("src", src, 4 * M_cap)
     _fits("pos", pos, 4 * T * k)
-    L.call("moe_route", _p(topk), T, k, E, M_cap, _p(seg), _p(src), _p(pos), _p(ws), ws.numel() * ws.element_size(),
-           _s())
+    if align == 128:
+        L.call("moe_route", _p(topk), T, k, E, M_cap, _p(seg), _p(src), _p(pos), _p(ws),
+               ws.numel() * ws.element_size(), _s())
+    else:
+        L.call("moe_route_aligned", _p(topk), T, k, E, align, M_cap, _p(seg), _p(src), _p(pos), _p(ws),
+               ws.numel() * ws.element_size(), _s())
     return seg, src, pos
 
 

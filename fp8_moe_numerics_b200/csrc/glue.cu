@@ -26,8 +26,9 @@ __global__ void route_count_kernel(const int32_t* __restrict__ topk, int64_t T, 
     for (int64_t e = threadIdx.x; e < E; e += blockDim.x) hist[(int64_t)blockIdx.x * E + e] = h[e];
 }
 
-// Totals, 128-padded exclusive scan into seg_offsets, and per-(chunk, expert)
-// base rows written back over hist.
+// Totals, kAlign-padded exclusive scan into seg_offsets, and per-(chunk,
+// expert) base rows written back over hist.
+template <int kAlign>
 __global__ void route_scan_kernel(int32_t* __restrict__ hist, int32_t* __restrict__ counts, int64_t nchunks,
                                   int64_t E, int64_t* __restrict__ seg) {
     extern __shared__ int64_t start[];   // [E + 1]
@@ -35,7 +36,7 @@ __global__ void route_scan_kernel(int32_t* __restrict__ hist, int32_t* __restric
         int64_t c = 0;
         for (int64_t ch = 0; ch < nchunks; ++ch) c += hist[ch * E + e];
         counts[e] = (int32_t)c;
-        start[e + 1] = (c + 127) / 128 * 128;
+        start[e + 1] = (c + kAlign - 1) / kAlign * kAlign;
     }
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -252,16 +253,13 @@ dispatch_grad_kernel(const uint16_t* __restrict__ dout, const int32_t* __restric
 
 }  // namespace
 
-extern "C" int moe_route(const int32_t* topk, int64_t T, int64_t k, int64_t E, int64_t M_cap, int64_t* seg_offsets,
-                         int32_t* src, int32_t* pos, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
-    MX_NVTX_RANGE("moe_route");
-    if (((!topk || !pos) && T > 0) || !seg_offsets || !src || T < 0 || k <= 0 || k > 32 || E <= 0 || M_cap < 0 ||
-        M_cap % 128)
-        return MX_EINVAL;
-    const int64_t need_rows = (T * k + 127 * E + 127) / 128 * 128;
-    if (M_cap < need_rows || !workspace || workspace_bytes < mx_route_workspace_bytes(T, E)) return MX_EINVAL;
-    if (T * k >= (int64_t)1 << 31 || E * 8 > 48 * 1024) return MX_EINVAL;
-    if (int st = mx_check_device()) return st;
+namespace {
+
+// The routing launches (count, kAlign-padded scan, scatter, padding rows)
+// after the entry point's checks.
+template <int kAlign>
+int route_launch(const int32_t* topk, int64_t T, int64_t k, int64_t E, int64_t M_cap, int64_t* seg_offsets,
+                 int32_t* src, int32_t* pos, void* workspace, cudaStream_t stream) {
     const int64_t nchunks = (T + kChunk - 1) / kChunk;
     int32_t* hist = static_cast<int32_t*>(workspace);
     int32_t* counts = hist + nchunks * E;
@@ -269,7 +267,7 @@ extern "C" int moe_route(const int32_t* topk, int64_t T, int64_t k, int64_t E, i
         route_count_kernel<<<(unsigned)nchunks, kChunk, E * sizeof(int32_t), stream>>>(topk, T, k, E, hist);
         mx_count_launch();
     }
-    route_scan_kernel<<<1, 1024, (E + 1) * sizeof(int64_t), stream>>>(hist, counts, nchunks, E, seg_offsets);
+    route_scan_kernel<kAlign><<<1, 1024, (E + 1) * sizeof(int64_t), stream>>>(hist, counts, nchunks, E, seg_offsets);
     mx_count_launch();
     if (nchunks > 0) {
         route_scatter_kernel<<<(unsigned)nchunks, 32, 2 * E * sizeof(uint32_t), stream>>>(topk, T, k, E, hist, src, pos);
@@ -278,6 +276,40 @@ extern "C" int moe_route(const int32_t* topk, int64_t T, int64_t k, int64_t E, i
     route_pad_kernel<<<(unsigned)(E + 1), 256, 0, stream>>>(seg_offsets, counts, E, M_cap, src);
     mx_count_launch();
     return mx_launch_status();
+}
+
+int route_check(const int32_t* topk, int64_t T, int64_t k, int64_t E, int64_t align, int64_t M_cap,
+                const int64_t* seg_offsets, const int32_t* src, const int32_t* pos, const void* workspace,
+                size_t workspace_bytes) {
+    if (((!topk || !pos) && T > 0) || !seg_offsets || !src || T < 0 || k <= 0 || k > 32 || E <= 0 || M_cap < 0 ||
+        M_cap % align)
+        return MX_EINVAL;
+    const int64_t need_rows = (T * k + (align - 1) * E + align - 1) / align * align;
+    if (M_cap < need_rows || !workspace || workspace_bytes < mx_route_workspace_bytes(T, E)) return MX_EINVAL;
+    if (T * k >= (int64_t)1 << 31 || E * 8 > 48 * 1024) return MX_EINVAL;
+    return MX_OK;
+}
+
+}  // namespace
+
+extern "C" int moe_route(const int32_t* topk, int64_t T, int64_t k, int64_t E, int64_t M_cap, int64_t* seg_offsets,
+                         int32_t* src, int32_t* pos, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+    MX_NVTX_RANGE("moe_route");
+    if (int st = route_check(topk, T, k, E, 128, M_cap, seg_offsets, src, pos, workspace, workspace_bytes)) return st;
+    if (int st = mx_check_device()) return st;
+    return route_launch<128>(topk, T, k, E, M_cap, seg_offsets, src, pos, workspace, stream);
+}
+
+extern "C" int moe_route_aligned(const int32_t* topk, int64_t T, int64_t k, int64_t E, int64_t align, int64_t M_cap,
+                                 int64_t* seg_offsets, int32_t* src, int32_t* pos, void* workspace,
+                                 size_t workspace_bytes, cudaStream_t stream) {
+    MX_NVTX_RANGE("moe_route_aligned");
+    if (align != 128 && align != 256) return MX_EINVAL;
+    if (int st = route_check(topk, T, k, E, align, M_cap, seg_offsets, src, pos, workspace, workspace_bytes))
+        return st;
+    if (int st = mx_check_device()) return st;
+    return align == 128 ? route_launch<128>(topk, T, k, E, M_cap, seg_offsets, src, pos, workspace, stream)
+                        : route_launch<256>(topk, T, k, E, M_cap, seg_offsets, src, pos, workspace, stream);
 }
 
 extern "C" int nvfp4_gather_rows(const uint8_t* codes, const uint8_t* sf, const float* outer, const int32_t* src,

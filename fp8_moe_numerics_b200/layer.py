@@ -25,7 +25,7 @@ from __future__ import annotations
 import torch
 
 from . import api
-from .api import MX_GEMM_DGRAD, MX_GEMM_WGRAD, MX_ROUND_RNE, MX_SF_MMA, MX_SF_ROWMAJOR
+from .api import MX_GEMM_DGRAD, MX_GEMM_WGRAD, MX_ROUND_RNE, MX_ROUND_SR, MX_SF_MMA, MX_SF_ROWMAJOR
 
 
 def nvfp4_gemm_flops(counts, N: int, K: int) -> int:
@@ -42,16 +42,24 @@ class ExpertLayer:
     quantises SwiGLU's output in the same kernel (the bf16 activation is then
     never written; `a` holds it only with fuse_swiglu=False).  `combine` is
     "bf16" (GEMM2 writes bf16 rows) or "s2f6" (GEMM2 writes rotated S2F6 rows,
-    one byte per value plus one exponent per 32).
+    one byte per value plus one exponent per 32).  `backward` is "mxfp8" (the
+    pages' recipe) or "nvfp4": the four backward GEMMs in NVFP4 with
+    stochastically rounded operands (the pages' stated future work; routing
+    then pads experts to 256 rows for the NVFP4 wgrad's K-stage; its kernels
+    have not yet run on a GPU).
     """
 
     S2F6_STREAM = 101                                   # Philox stream of the rotation's signs
 
     def __init__(self, x, topk, w_comb, w1, w2, dout, gated: bool = True, seed: int = 0,
                  wgrad_dtype=torch.bfloat16, out_dtype=torch.bfloat16, rbits: int = 16, combine: str = "bf16",
-                 fuse_swiglu: bool = True):
+                 fuse_swiglu: bool = True, backward: str = "mxfp8"):
         if combine not in ("bf16", "s2f6"):
             raise ValueError(f"combine must be 'bf16' or 's2f6', got {combine!r}")
+        if backward not in ("mxfp8", "nvfp4"):
+            raise ValueError(f"backward must be 'mxfp8' or 'nvfp4', got {backward!r}")
+        self.backward_format = backward
+        self.align = 256 if backward == "nvfp4" else 128
         self.combine = combine
         self.fuse_swiglu = fuse_swiglu
         dev = x.device
@@ -67,7 +75,7 @@ class ExpertLayer:
         self.seed, self.rbits = seed, rbits
         self.x, self.topk, self.w_comb, self.w1, self.w2, self.dout = x, topk, w_comb, w1, w2, dout
         T, D, k, E, F, N1 = self.T, self.D, self.k, self.E, self.F, self.N1
-        self.M_cap = M = api.max_routed_rows(T, k, E)
+        self.M_cap = M = api.max_routed_rows(T, k, E, self.align)
         e = lambda *s, dt=torch.uint8: torch.empty(*s, dtype=dt, device=dev)
         sfb = api.sf_bytes
         # routing
@@ -103,6 +111,16 @@ class ExpertLayer:
         self.xt = (e(D, M), e(sfb(D, M, 32, MX_SF_MMA)))
         self.dw1 = e(E, N1, D, dt=wgrad_dtype)
         self.dx = e(T, D, dt=torch.bfloat16)
+        if backward == "nvfp4":
+            q4 = lambda r, c, n_outer: (e(r, c // 2), e(sfb(r, c, 16, MX_SF_MMA)), e(n_outer, dt=torch.float32))
+            self.dy2n = q4(M, D, M)                     # dgrad2 A: dY2, per-token outer
+            self.w2tn = q4(E * F, D, E)                 # dgrad2 B: stack of W2_e^T, per-expert outer
+            self.dy2tn = q4(D, M, E * D)                # wgrad2 A: dY2^T, per (segment, row)
+            self.atn = q4(F, M, E)                      # wgrad2 B: a^T, per segment
+            self.dh1n = q4(M, N1, M)
+            self.w1tn = q4(E * D, N1, E)
+            self.dh1tn = q4(N1, M, E * N1)
+            self.xtn = q4(D, M, E)
         self.marks = []
 
     # ------------------------------------------------------------------ timing
@@ -136,7 +154,7 @@ class ExpertLayer:
     def forward(self, record: bool = False):
         T, D, k, E, F, N1, M = self.T, self.D, self.k, self.E, self.F, self.N1, self.M_cap
         self._mark("start", record)
-        api.moe_route(self.topk, E, M, out=(self.seg, self.src, self.pos, self.route_ws))
+        api.moe_route(self.topk, E, M, out=(self.seg, self.src, self.pos, self.route_ws), align=self.align)
         self._mark("route", record)
         api.nvfp4_quantize(self.x, 1, MX_SF_ROWMAJOR, out=self.xq)
         self._mark("quant_x", record)
@@ -169,6 +187,8 @@ class ExpertLayer:
 
     # ---------------------------------------------------------------- backward
     def backward(self, record: bool = False):
+        if self.backward_format == "nvfp4":
+            return self._backward_nvfp4(record)
         T, D, k, E, F, N1, M = self.T, self.D, self.k, self.E, self.F, self.N1, self.M_cap
         s, R = self.seed, self.rbits
         self._mark("bwd_start", record)
@@ -197,6 +217,48 @@ class ExpertLayer:
         self._mark("requant_x", record)
         api.grouped_gemm_mxfp8(MX_GEMM_WGRAD, self.dh1q[2], self.dh1q[3], *self.xt, self.seg, E, M, N1, D,
                                out=self.dw1)
+        self._mark("wgrad1", record)
+        api.moe_combine(self.dxp, self.pos, None, D, out=self.dx)
+        self._mark("unpermute", record)
+        return self.dx, self.dw1, self.dw2
+
+    def _backward_nvfp4(self, record: bool):
+        """The four backward GEMMs in NVFP4: dgrad as the forward grouped GEMM
+        with B the requantised stack of W_e^T; wgrad on the transposes with
+        outer scales per expert segment.  Every operand is rounded
+        stochastically (its own Philox stream)."""
+        D, E, F, N1, M = self.D, self.E, self.F, self.N1, self.M_cap
+        s, R, SR = self.seed, self.rbits, MX_ROUND_SR
+        self._mark("bwd_start", record)
+        api.moe_dispatch_grad(self.dout, self.src, self.pos, self.w_comb, out=self.dy2)
+        self._mark("dispatch_grad", record)
+        api.nvfp4_quantize_sr(self.dy2, 1, SR, s, 11, R, MX_SF_MMA, out=self.dy2n)
+        self._mark("quant_dy2", record)
+        api.nvfp4_requant_transpose_sr(*self.w2q, E * D, F, D, MX_SF_MMA, E, True, SR, s, 12, R, MX_SF_MMA,
+                                       out=self.w2tn)
+        self._mark("requant_w2", record)
+        api.grouped_gemm_nvfp4(self.dy2n, self.w2tn, self.seg, E, F, D, out=self.da)
+        self._mark("dgrad2", record)
+        api.nvfp4_quantize_transpose_segments(self.dy2, self.seg, E, True, SR, s, 13, R, MX_SF_MMA, out=self.dy2tn)
+        api.nvfp4_requant_transpose_segments(*self.aq, M, F, self.seg, E, False, 1, MX_SF_MMA, SR, s, 14, R,
+                                             MX_SF_MMA, out=self.atn)
+        self._mark("requant_a", record)
+        api.grouped_gemm_nvfp4_wgrad(self.dy2tn, self.atn, self.seg, E, D, F, out=self.dw2)
+        self._mark("wgrad2", record)
+        api.swiglu_bwd(self.h1, self.da, F, self.gated, self.rows_valid, out=self.dh1)
+        self._mark("swiglu_bwd", record)
+        api.nvfp4_quantize_sr(self.dh1, 1, SR, s, 15, R, MX_SF_MMA, out=self.dh1n)
+        self._mark("quant_dh1", record)
+        api.nvfp4_requant_transpose_sr(*self.w1q, E * N1, D, N1, MX_SF_MMA, E, True, SR, s, 16, R, MX_SF_MMA,
+                                       out=self.w1tn)
+        self._mark("requant_w1", record)
+        api.grouped_gemm_nvfp4(self.dh1n, self.w1tn, self.seg, E, D, N1, out=self.dxp)
+        self._mark("dgrad1", record)
+        api.nvfp4_quantize_transpose_segments(self.dh1, self.seg, E, True, SR, s, 17, R, MX_SF_MMA, out=self.dh1tn)
+        api.nvfp4_requant_transpose_segments(*self.xp, M, D, self.seg, E, False, 1, MX_SF_MMA, SR, s, 18, R,
+                                             MX_SF_MMA, out=self.xtn)
+        self._mark("requant_x", record)
+        api.grouped_gemm_nvfp4_wgrad(self.dh1tn, self.xtn, self.seg, E, N1, D, out=self.dw1)
         self._mark("wgrad1", record)
         api.moe_combine(self.dxp, self.pos, None, D, out=self.dx)
         self._mark("unpermute", record)

@@ -225,6 +225,14 @@ MX_API int moe_route(const int32_t* topk, int64_t T, int64_t k, int64_t E, int64
               int64_t* seg_offsets, int32_t* src, int32_t* pos,
               void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* moe_route_aligned -- moe_route with each segment padded to a multiple of
+ * `align` rows (128 or 256; 256 for the NVFP4 wgrad GEMM, whose K-stage holds
+ * 256 tokens).  M_cap must be a multiple of align and at least T*k +
+ * (align-1)*E rounded up to align.  With align = 128 it is moe_route. */
+MX_API int moe_route_aligned(const int32_t* topk, int64_t T, int64_t k, int64_t E, int64_t align, int64_t M_cap,
+                             int64_t* seg_offsets, int32_t* src, int32_t* pos,
+                             void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
 /* moe_route_static -- moe_route without a caller-provided workspace.
  * The pages describe nothing like this; it exists for callers that cannot
  * allocate device memory for scratch (for example code running inside an

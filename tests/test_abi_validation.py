@@ -51,6 +51,10 @@ CASES = {
         ("capacity below the padded rows", {4: 512}), ("workspace too small", {9: 16}), ("k > 32", {2: 33}),
         ("no experts", {3: 0}), ("M_cap % 128", {4: 600}), ("null workspace", {8: None}),
     ]),
+    "moe_route_aligned": ((A, 16, 2, 4, 256, 1280, A, A, A, A, 4096, None), [
+        ("align 64", {4: 64}), ("M_cap % align", {5: 1152}), ("capacity below the padded rows", {5: 1024}),
+        ("k 0", {2: 0}), ("null workspace", {9: None}),
+    ]),
     "moe_route_static": ((A, 16, 2, 4, 640, A, A, A, None), [
         ("null topk", {0: None}), ("M_cap % 128", {4: 100}), ("k 0", {2: 0}),
         ("beyond the fixed scratch", {1: 1 << 20, 3: 64}),

@@ -107,3 +107,29 @@ def test_every_marked_stage_has_work_in_bench(host_calls, monkeypatch, opts):
     work = bench.stage_work(c, [c["T"] * c["k"] // c["E"]] * c["E"], L.M_cap)
     assert set(stages) <= set(work), set(stages) - set(work)
     assert {"gemm1", "gemm2", "requant_w1", "wgrad1"} <= set(stages)
+
+
+def test_nvfp4_backward_sequence_passes_host_validation(host_calls):
+    # the NVFP4 backward: routing padded to 256 rows, four NVFP4 backward GEMMs
+    inp = workloads.layer_inputs("tiny_layer", device="cpu")
+    c = inp["cfg"]
+    L = ExpertLayer(inp["x"], inp["topk"], inp["w_comb"], inp["w1"], inp["w2"], inp["dout"], gated=c["gated"],
+                    backward="nvfp4")
+    assert L.M_cap % 256 == 0
+    L.step()
+    names = [n for n, _ in host_calls]
+    assert names[0] == "moe_route_aligned" and names[-1] == "moe_combine"
+    assert "grouped_gemm_mxfp8" not in names and "mxfp8_requant_transpose_sr" not in names
+    assert names.count("grouped_gemm_nvfp4") == 4                 # GEMM1, GEMM2, dgrad2, dgrad1
+    assert names.count("grouped_gemm_nvfp4_wgrad") == 2
+    assert names.count("nvfp4_quantize_sr") == 2 and names.count("nvfp4_requant_transpose_sr") == 2
+    assert names.count("nvfp4_quantize_transpose_segments") == 2
+    assert names.count("nvfp4_requant_transpose_segments") == 2
+    assert all(st == _lib.MX_ECUDA for _, st in host_calls)   # valid, and no device here
+    # its stage marks all have a work entry in bench.py
+    L2 = ExpertLayer(inp["x"], inp["topk"], inp["w_comb"], inp["w1"], inp["w2"], inp["dout"], gated=c["gated"],
+                     backward="nvfp4")
+    assert L2.backward_format == "nvfp4"
+    with pytest.raises(ValueError, match="backward"):
+        ExpertLayer(inp["x"], inp["topk"], inp["w_comb"], inp["w1"], inp["w2"], inp["dout"], gated=c["gated"],
+                    backward="fp4")
