@@ -116,9 +116,9 @@ def fake_gpu(monkeypatch):
     monkeypatch.setattr(api, "_s", lambda: ctypes.c_void_p(0))
     route = api.moe_route
 
-    def routed(topk, E, M_cap=None, out=None):
-        seg, src, pos = route(topk, E, M_cap, out)
-        s, _, p = oracle.route(topk.numpy(), E)
+    def routed(topk, E, M_cap=None, out=None, align=128):
+        seg, src, pos = route(topk, E, M_cap, out, align)
+        s, _, p = oracle.route(topk.numpy(), E, align)
         seg.copy_(torch.from_numpy(np.asarray(s, np.int64)))
         T, k = p.shape
         flat = np.full(src.numel(), -1, np.int32)
