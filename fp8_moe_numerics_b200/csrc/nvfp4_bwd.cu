@@ -420,6 +420,7 @@ extern "C" int nvfp4_requant_transpose_sr(const uint8_t* codes, const uint8_t* s
     if (in_sf_layout == MX_SF_MMA && rows % 128) return MX_EINVAL;
     if (out_sf_layout == MX_SF_MMA && ((experts * cols) % 128 || rpe % 64)) return MX_EINVAL;
     if (out_outer_per_expert != 0 && out_outer_per_expert != 1) return MX_EINVAL;
+    if (!out_outer_per_expert && experts != 1) return MX_EINVAL;   // per-row scales: one block (activations)
     if (int st = mx_check_device()) return st;
     if (rows == 0) return MX_OK;
     const int64_t n_outer = out_outer_per_expert ? experts : experts * cols;

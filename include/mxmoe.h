@@ -382,7 +382,8 @@ MX_API int nvfp4_quantize_sr(const void* x, int64_t rows, int64_t cols, int64_t 
 /* nvfp4_requant_transpose_sr -- saved NVFP4 -> NVFP4 of its transpose.
  * The input [rows, cols] (codes, sf in in_sf_layout, outer per group_rows
  * rows) holds `experts` stacked blocks of rows / experts rows each (1 for an
- * activation tensor, E for an expert weight stack [E*N, K]).  Each value is
+ * activation tensor, E for an expert weight stack [E*N, K]; per-row outer
+ * scales take experts = 1).  Each value is
  * dequantised ((q * sf) * outer, fp32), each block is transposed, and the
  * result [experts * cols, rows / experts] (block e's transpose in rows
  * e*cols ..) is quantised with the rounding above, blocks of 16 along the old

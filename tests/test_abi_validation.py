@@ -94,11 +94,12 @@ CASES = {
         ("group_rows 0", {3: 0}), ("MMA layout rows % 128", {1: 64, 11: 1}), ("x misaligned", {0: A8}),
         ("null outer", {10: None}),
     ]),
-    "nvfp4_requant_transpose_sr": ((A, A, A, 256, 64, 1, 0, 2, 0, 1, 1, 2, 16, A, A, A, 0, None), [
+    "nvfp4_requant_transpose_sr": ((A, A, A, 256, 64, 1, 0, 2, 1, 1, 1, 2, 16, A, A, A, 0, None), [
         ("cols % 64", {4: 32}), ("rows per expert % 128", {7: 4}), ("rows % experts", {7: 3}),
         ("no experts", {7: 0}), ("unknown rounding", {9: 2}), ("SR with rbits 4", {12: 4}),
         ("unknown out layout", {16: 3}), ("outer-per-expert flag 2", {8: 2}), ("out codes misaligned", {13: A8}),
         ("null out outer", {15: None}), ("out outer misaligned", {15: A1}),
+        ("per-row outer scales over two experts", {8: 0}),
     ]),
     "nvfp4_quantize_transpose_segments": ((A, 256, 128, A, 2, 1, 1, 1, 2, 16, A, A, A, 1, None), [
         ("M % 128", {1: 192}), ("C % 64", {2: 96}), ("no experts", {4: 0}), ("per_row 2", {5: 2}),

@@ -56,7 +56,7 @@ def test_quantize_sr_kernel_indexing(rows, cols, group_rows, mma):
 @pytest.mark.parametrize("rows,cols,group_rows,experts,per_expert,in_mma,out_mma", [
     (256, 128, 1, 1, 0, True, True),            # activations: one outer scale per output row
     (512, 128, 128, 4, 1, True, True),          # weight stack [E*N, K]: per-expert outer scale
-    (384, 64, 1, 3, 0, False, False),
+    (384, 64, 1, 3, 1, False, False),
     (256, 192, 256, 1, 1, True, False),
 ])
 def test_requant_kernels_indexing(rows, cols, group_rows, experts, per_expert, in_mma, out_mma):
@@ -65,6 +65,7 @@ def test_requant_kernels_indexing(rows, cols, group_rows, experts, per_expert, i
     assert rpe % 128 == 0 and cols % 64 == 0 and rows % group_rows == 0
     assert not in_mma or rows % 128 == 0
     assert not out_mma or ((experts * cols) % 128 == 0 and rpe % 64 == 0)
+    assert per_expert or experts == 1
     S_in = cols // 16
     # pass 1: grid (cols / 64, rows / 128); thread (cl = t % 64, rg = t / 64) reads 32 rows of one column
     n_outer = experts if per_expert else experts * cols
