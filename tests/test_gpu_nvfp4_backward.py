@@ -184,3 +184,62 @@ def test_nvfp4_wgrad_gemm(cuda, Nw, Kw, counts):
             assert np.all(got[e] == 0)
         else:
             assert rel_fro(got[e], ref[e]) <= 1e-4
+
+
+def test_tiny_layer_nvfp4_backward_against_oracle(cuda):
+    # the tiny layer with backward="nvfp4" against the oracle's own chain:
+    # routing padded to 256 rows, Philox streams 11-18 as the layer uses them
+    from fp8_moe_numerics_b200 import workloads
+    from fp8_moe_numerics_b200.layer import ExpertLayer
+    from tests.test_gpu_layer import f64, pad, rel, u16
+    inp = workloads.layer_inputs("tiny_layer", device="cpu")
+    c = inp["cfg"]
+    E, D, F = c["E"], c["D"], c["F"]
+    seed, R = 99, 16
+    L = ExpertLayer(inp["x"].cuda(), inp["topk"].cuda(), inp["w_comb"].cuda(), inp["w1"].cuda(), inp["w2"].cuda(),
+                    inp["dout"].cuda(), gated=False, seed=seed, wgrad_dtype=torch.float32, backward="nvfp4")
+    L.step()
+    api.sync_status()
+    M = L.M_cap
+    g = lambda t: t.cpu().numpy()
+
+    x, dout = u16(inp["x"]), u16(inp["dout"])
+    w1, w2 = u16(inp["w1"]).reshape(E * F, D), u16(inp["w2"]).reshape(E * D, F)
+    w = inp["w_comb"].numpy()
+    seg, src, pos = oracle.route(inp["topk"].numpy(), E, 256)
+    Mp = int(seg[-1])
+    xp = oracle.gather_nvfp4_rows(*oracle.nvfp4_quantize(x), src)
+    w1q = oracle.nvfp4_quantize(w1, group_rows=F)
+    w2q = oracle.nvfp4_quantize(w2, group_rows=D)
+    h1 = oracle.f64_to_bf16(oracle.grouped_gemm_nvfp4(*xp, *w1q, seg, F))
+    aq = oracle.nvfp4_quantize(oracle.swiglu_fwd(h1, gated=False))
+    dy2 = oracle.dispatch_grad(dout, pos, w, Mp)
+    f32 = lambda u, rows: oracle.bf16_to_f32(pad(u, rows))
+    deq = lambda q: oracle.nvfp4_dequantize(pad(q[0], M), pad(q[1], M), pad(q[2], M))
+    dy2n = oracle.nvfp4_quantize_f32(f32(dy2, M), 1, True, seed, 11, R)
+    w2tn = oracle.nvfp4_requant_transpose_experts_sr(*w2q, E, seed, 12, R)
+    da = oracle.f64_to_bf16(oracle.grouped_gemm_nvfp4(*dy2n, *w2tn, seg, F)[:Mp])
+    dy2tn = oracle.nvfp4_quantize_transpose_segments(f32(dy2, M), seg, True, True, seed, 13, R)
+    atn = oracle.nvfp4_quantize_transpose_segments(deq(aq), seg, False, True, seed, 14, R)
+    dw2 = oracle.grouped_gemm_nvfp4_wgrad(*dy2tn, *atn, seg)
+    dh1 = oracle.swiglu_bwd(h1, da, gated=False)
+    dh1n = oracle.nvfp4_quantize_f32(f32(dh1, M), 1, True, seed, 15, R)
+    w1tn = oracle.nvfp4_requant_transpose_experts_sr(*w1q, E, seed, 16, R)
+    dxp = oracle.f64_to_bf16(oracle.grouped_gemm_nvfp4(*dh1n, *w1tn, seg, D)[:Mp])
+    dh1tn = oracle.nvfp4_quantize_transpose_segments(f32(dh1, M), seg, True, True, seed, 17, R)
+    xtn = oracle.nvfp4_quantize_transpose_segments(deq(xp), seg, False, True, seed, 18, R)
+    dw1 = oracle.grouped_gemm_nvfp4_wgrad(*dh1tn, *xtn, seg)
+    dx = oracle.combine(dxp, pos, np.ones_like(w))
+
+    # operands built from bit-exact inputs: bit for bit
+    assert np.array_equal(g(L.seg), seg)
+    for got, ref, rows, cols in ((L.w2tn, w2tn, E * F, D), (L.w1tn, w1tn, E * D, F), (L.dy2n, dy2n, M, D),
+                                 (L.dy2tn, dy2tn, D, M)):
+        assert np.array_equal(g(got[0]), ref[0])
+        assert np.array_equal(mma_to_rowmajor(g(got[1]), rows, cols // 16), ref[1])
+        assert np.array_equal(g(got[2]), ref[2].reshape(-1))
+    # after a GEMM output (fp32 vs fp64 sums, one bf16 rounding): rare code flips only
+    assert np.mean(g(L.atn[0]) == atn[0]) >= 0.99 and np.mean(g(L.dh1n[0]) == dh1n[0]) >= 0.99
+    for got, ref in ((f64(u16(L.da)[:Mp]), f64(da)), (g(L.dw2).astype(np.float64), dw2),
+                     (f64(u16(L.dxp)[:Mp]), f64(dxp)), (g(L.dw1).astype(np.float64), dw1), (f64(u16(L.dx)), f64(dx))):
+        assert rel(got, ref) < 2e-2
