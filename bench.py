@@ -581,7 +581,8 @@ def cpu_baseline(inp, layer, seconds: float = 15.0):
 # larger than L2 where DRAM traffic is read off)
 # --------------------------------------------------------------------------
 KERNEL_CASES = ("gemm_nvfp4", "gemm_nvfp4_s2f6", "gemm_mxfp8_dgrad", "gemm_mxfp8_wgrad", "requant", "requant_w",
-                "nvfp4_quantize", "quant_w", "mxfp8_quantize", "nvfp4_quantize_sr", "requant_nvfp4", "gemm_nvfp4_wgrad")
+                "nvfp4_quantize", "quant_w", "mxfp8_quantize", "nvfp4_quantize_sr", "requant_nvfp4", "gemm_nvfp4_wgrad",
+                "step_nvfp4_backward")
 
 
 def run_kernel(args):
@@ -589,7 +590,15 @@ def run_kernel(args):
     from fp8_moe_numerics_b200 import api, workloads
     dev = torch.device("cuda")
     which = args.kernel
-    if which.startswith("gemm"):
+    if which == "step_nvfp4_backward":
+        # one forward + backward step of the benchmark layer with the four backward GEMMs in NVFP4
+        from fp8_moe_numerics_b200.layer import ExpertLayer
+        c = workloads.CONFIGS[WORKLOAD]
+        inp = workloads.layer_inputs(WORKLOAD, device=dev)
+        layer = ExpertLayer(inp["x"], inp["topk"], inp["w_comb"], inp["w1"], inp["w2"], inp["dout"],
+                            gated=c["gated"], seed=c["seed"], backward="nvfp4")
+        run = layer.step
+    elif which.startswith("gemm"):
         # 64 experts, top-8 of 4096 tokens (Zipf 1.2), d_model 4096, d_ff 1024 (gated)
         E, T, k, D, F = 64, 4096, 8, 4096, 1024
         ids = workloads.routing(T, k, E, "zipf", 1.2, 0, 7).to(dev)

@@ -58,7 +58,7 @@ def test_default_line_has_every_contract_key(small_bench, monkeypatch, capsys):
 
 
 def test_kernel_cases_run(small_bench, monkeypatch, capsys):
-    for case in ("nvfp4_quantize", "requant", "nvfp4_quantize_sr", "requant_nvfp4"):
+    for case in ("nvfp4_quantize", "requant", "nvfp4_quantize_sr", "requant_nvfp4", "step_nvfp4_backward"):
         with fake_gpu(monkeypatch) as calls:
             monkeypatch.setattr(sys, "argv", ["bench.py", "--kernel", case])
             small_bench.main()
