@@ -213,3 +213,46 @@ def test_nvfp4_wgrad_tile_mapping(M, N, K, seg, pair):
                     assert sfb0 + h * groups + kt * 4 + 4 <= atoms_b
             # the stages cover the segment's tokens exactly
             assert k_tiles * 256 == s1 - s0
+
+
+# The same replays over shapes drawn at random within what the entry points
+# accept: expert counts, empty experts, padding rows, layouts, group sizes.
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@settings(max_examples=30, deadline=None)
+@given(st.data())
+def test_segment_kernels_indexing_random_shapes(data):
+    E = data.draw(st.integers(1, 5))
+    seg = np.concatenate([[0], np.cumsum([data.draw(st.integers(0, 3)) * 128 for _ in range(E)])])
+    M = max(128, int(seg[-1]) + data.draw(st.integers(0, 2)) * 128)
+    C = data.draw(st.sampled_from([64, 128, 192, 256]))
+    out_mma = C % 128 == 0 and data.draw(st.booleans())
+    group_rows = data.draw(st.sampled_from([g for g in (1, 64, 128) if M % g == 0]))
+    test_segment_kernels_indexing(M, C, list(seg), data.draw(st.booleans()), out_mma,
+                                  data.draw(st.booleans()), group_rows)
+
+
+@settings(max_examples=30, deadline=None)
+@given(st.data())
+def test_requant_kernels_indexing_random_shapes(data):
+    per_expert = data.draw(st.booleans())
+    experts = data.draw(st.integers(1, 4)) if per_expert else 1
+    rpe = data.draw(st.integers(1, 3)) * 128
+    rows = experts * rpe
+    cols = data.draw(st.sampled_from([64, 128, 192, 256]))
+    out_mma = (experts * cols) % 128 == 0 and data.draw(st.booleans())
+    group_rows = data.draw(st.sampled_from([g for g in (1, 128, rpe) if rows % g == 0]))
+    test_requant_kernels_indexing(rows, cols, group_rows, experts, int(per_expert), data.draw(st.booleans()),
+                                  out_mma)
+
+
+@settings(max_examples=30, deadline=None)
+@given(st.data())
+def test_quantize_and_tile_indexing_random_shapes(data):
+    rows = data.draw(st.integers(1, 6)) * 128
+    cols = data.draw(st.sampled_from([64, 128, 192, 320]))
+    test_quantize_sr_kernel_indexing(rows, cols, data.draw(st.sampled_from([1, 16, 128])), cols % 64 == 0)
+    trows, tcols = data.draw(st.integers(1, 8)) * 16, data.draw(st.integers(1, 8)) * 16
+    test_tile16_kernel_indexing(trows, tcols, data.draw(st.sampled_from([g for g in (16, 32, trows)
+                                                                          if trows % g == 0 and g % 16 == 0])))
