@@ -11,13 +11,13 @@ import os
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmxmoe.so")
 
-MX_OK, MX_EINVAL, MX_ECUDA, MX_ETIMEOUT, MX_EUNSUPPORTED = 0, 1, 2, 3, 4
+MX_OK, MX_EINVAL, MX_ECUDA, MX_ETIMEOUT, MX_EUNSUPPORTED, MX_EDATA = 0, 1, 2, 3, 4, 5
 MX_SF_ROWMAJOR, MX_SF_MMA = 0, 1
 MX_OUT_F32, MX_OUT_BF16 = 0, 1
 MX_ROUND_RNE, MX_ROUND_SR = 0, 1
 MX_GEMM_DGRAD, MX_GEMM_WGRAD = 0, 1
 
-STATUS_NAMES = {0: "MX_OK", 1: "MX_EINVAL", 2: "MX_ECUDA", 3: "MX_ETIMEOUT", 4: "MX_EUNSUPPORTED"}
+STATUS_NAMES = {0: "MX_OK", 1: "MX_EINVAL", 2: "MX_ECUDA", 3: "MX_ETIMEOUT", 4: "MX_EUNSUPPORTED", 5: "MX_EDATA"}
 
 P = ctypes.c_void_p
 I64 = ctypes.c_int64

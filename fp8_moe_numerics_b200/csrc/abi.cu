@@ -64,6 +64,7 @@ extern "C" size_t mx_sf_bytes(int64_t rows, int64_t cols, int block, int sf_layo
 
 extern "C" size_t mx_route_workspace_bytes(int64_t T, int64_t E) {
     if (T < 0 || E <= 0) return 0;
-    const int64_t chunks = (T + 255) / 256;
+    const int64_t chunks = T / 256 + (T % 256 != 0);
+    if (chunks > (INT64_MAX / (int64_t)sizeof(int32_t) - E) / E) return SIZE_MAX;   // would overflow int64
     return (size_t)((chunks * E + E) * sizeof(int32_t));
 }

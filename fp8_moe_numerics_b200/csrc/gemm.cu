@@ -72,7 +72,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
         if (*abort_flag) return false;
         if (globaltimer() - t0 > limit_ns) {
             *abort_flag = 1;
-            atomicOr(&g_mx_status_word, 1u);
+            atomicOr(&g_mx_status_word, kStatusTimeout);
             return false;
         }
     }
@@ -1023,7 +1023,8 @@ extern "C" int mx_sync_status(cudaStream_t stream) {
     if ((e = cudaMemcpyFromSymbol(&word, g_mx_status_word, sizeof(word))) != cudaSuccess) return mx_set_cuda_error(e);
     if (word && (e = cudaMemcpyToSymbol(g_mx_status_word, &zero, sizeof(zero))) != cudaSuccess)
         return mx_set_cuda_error(e);
-    return word ? MX_ETIMEOUT : MX_OK;
+    if (word & kStatusTimeout) return MX_ETIMEOUT;
+    return word ? MX_EDATA : MX_OK;
 }
 
 // Device address of the status word on the current device, looked up once per

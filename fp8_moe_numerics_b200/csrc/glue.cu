@@ -13,15 +13,30 @@ namespace {
 
 constexpr int kChunk = 256;   // tokens per routing chunk
 
+// Whether entry j of token t names an expert: an id in [0, E) that no earlier
+// entry of the same token names.  Other entries are left out of the routing
+// (their pos is -1) and flag the device status word.
+__device__ __forceinline__ bool route_entry_valid(const int32_t* __restrict__ topk, int64_t t, int64_t k, int64_t j,
+                                                  int64_t E) {
+    const int32_t id = topk[t * k + j];
+    if ((uint64_t)(uint32_t)id >= (uint64_t)E || id < 0) return false;
+    for (int64_t i = 0; i < j; ++i)
+        if (topk[t * k + i] == id) return false;
+    return true;
+}
+
 // Per-chunk expert histogram: hist[c][e].
 __global__ void route_count_kernel(const int32_t* __restrict__ topk, int64_t T, int64_t k, int64_t E,
-                                   int32_t* __restrict__ hist) {
+                                   int32_t* __restrict__ hist, unsigned int* __restrict__ status) {
     extern __shared__ int32_t h[];
     for (int64_t e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
     __syncthreads();
     const int64_t t = (int64_t)blockIdx.x * kChunk + threadIdx.x;
     if (t < T)
-        for (int64_t j = 0; j < k; ++j) atomicAdd(&h[topk[t * k + j]], 1);
+        for (int64_t j = 0; j < k; ++j) {
+            if (route_entry_valid(topk, t, k, j, E)) atomicAdd(&h[topk[t * k + j]], 1);
+            else atomicOr(status, kStatusBadRoute);
+        }
     __syncthreads();
     for (int64_t e = threadIdx.x; e < E; e += blockDim.x) hist[(int64_t)blockIdx.x * E + e] = h[e];
 }
@@ -71,11 +86,17 @@ __global__ void route_scatter_kernel(const int32_t* __restrict__ topk, int64_t T
     for (int gi = 0; gi < kChunk / 32; ++gi) {
         const int64_t t = (int64_t)blockIdx.x * kChunk + gi * 32 + lane;
         const bool act = t < T;
+        uint32_t valid = 0;   // bit j: entry j of this lane's token names an expert
         if (act)
-            for (int64_t j = 0; j < k; ++j) atomicOr(&mask[topk[t * k + j]], 1u << lane);
+            for (int64_t j = 0; j < k; ++j)
+                if (route_entry_valid(topk, t, k, j, E)) {
+                    valid |= 1u << j;
+                    atomicOr(&mask[topk[t * k + j]], 1u << lane);
+                }
         __syncwarp();
         if (act)
             for (int64_t j = 0; j < k; ++j) {
+                if (!(valid >> j & 1u)) { pos[t * k + j] = -1; continue; }
                 const int32_t e = topk[t * k + j];
                 const int32_t p = run[e] + __popc(mask[e] & below);
                 pos[t * k + j] = p;
@@ -84,6 +105,7 @@ __global__ void route_scatter_kernel(const int32_t* __restrict__ topk, int64_t T
         __syncwarp();
         if (act)
             for (int64_t j = 0; j < k; ++j) {
+                if (!(valid >> j & 1u)) continue;
                 const int32_t e = topk[t * k + j];
                 const uint32_t m = mask[e];
                 if ((m & below) == 0) { run[e] += __popc(m); mask[e] = 0; }
@@ -196,8 +218,10 @@ __global__ void combine_kernel(const uint16_t* __restrict__ y, const int32_t* __
     for (int64_t c = threadIdx.x * 8; c < D; c += blockDim.x * 8) {
         float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
         for (int64_t j = 0; j < k; ++j) {
+            const int32_t p = pos[t * k + j];
+            if (p < 0) continue;                           // entry left out by the routing
             const float wj = w ? w[t * k + j] : 1.0f;
-            const uint4 v = __ldg(reinterpret_cast<const uint4*>(y + (int64_t)pos[t * k + j] * D + c));
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(y + (int64_t)p * D + c));
             const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -232,6 +256,7 @@ dispatch_grad_kernel(const uint16_t* __restrict__ dout, const int32_t* __restric
         for (int64_t c = threadIdx.x * 8; c < D; c += kDispatchThreads * 8) {
             const uint4 v = __ldcs(reinterpret_cast<const uint4*>(dout + b * D + c));
             for (int64_t j = 0; j < k; ++j) {
+                if (sp[j] < 0) continue;                   // entry left out by the routing
                 const float wj = sw[j];
                 const uint4 o = make_uint4(pack_bf16x2(wj * bf16_lo(v.x), wj * bf16_hi(v.x)),
                                            pack_bf16x2(wj * bf16_lo(v.y), wj * bf16_hi(v.y)),
@@ -263,30 +288,47 @@ int route_launch(const int32_t* topk, int64_t T, int64_t k, int64_t E, int64_t M
     const int64_t nchunks = (T + kChunk - 1) / kChunk;
     int32_t* hist = static_cast<int32_t*>(workspace);
     int32_t* counts = hist + nchunks * E;
+    unsigned int* status = nullptr;
+    if (int st = mx_status_word_address(&status)) return st;
+    // Each launch reads what the previous one wrote: stop at the first failure.
     if (nchunks > 0) {
-        route_count_kernel<<<(unsigned)nchunks, kChunk, E * sizeof(int32_t), stream>>>(topk, T, k, E, hist);
+        route_count_kernel<<<(unsigned)nchunks, kChunk, E * sizeof(int32_t), stream>>>(topk, T, k, E, hist, status);
         mx_count_launch();
+        if (int st = mx_launch_status()) return st;
     }
     route_scan_kernel<kAlign><<<1, 1024, (E + 1) * sizeof(int64_t), stream>>>(hist, counts, nchunks, E, seg_offsets);
     mx_count_launch();
+    if (int st = mx_launch_status()) return st;
     if (nchunks > 0) {
         route_scatter_kernel<<<(unsigned)nchunks, 32, 2 * E * sizeof(uint32_t), stream>>>(topk, T, k, E, hist, src, pos);
         mx_count_launch();
+        if (int st = mx_launch_status()) return st;
     }
     route_pad_kernel<<<(unsigned)(E + 1), 256, 0, stream>>>(seg_offsets, counts, E, M_cap, src);
     mx_count_launch();
     return mx_launch_status();
 }
 
-int route_check(const int32_t* topk, int64_t T, int64_t k, int64_t E, int64_t align, int64_t M_cap,
-                const int64_t* seg_offsets, const int32_t* src, const int32_t* pos, const void* workspace,
-                size_t workspace_bytes) {
+// Largest dynamic shared memory of the routing launches: the scan's
+// (E + 1) int64 starts (the count needs 4E bytes, the scatter 8E).
+constexpr int64_t kRouteSmemLimit = 48 * 1024;
+
+// Arguments of a routing call apart from its workspace.
+int route_check_args(const int32_t* topk, int64_t T, int64_t k, int64_t E, int64_t align, int64_t M_cap,
+                     const int64_t* seg_offsets, const int32_t* src, const int32_t* pos) {
     if (((!topk || !pos) && T > 0) || !seg_offsets || !src || T < 0 || k <= 0 || k > 32 || E <= 0 || M_cap < 0 ||
         M_cap % align)
         return MX_EINVAL;
+    if ((E + 1) * (int64_t)sizeof(int64_t) > kRouteSmemLimit || T >= ((int64_t)1 << 31) / k) return MX_EINVAL;
     const int64_t need_rows = (T * k + (align - 1) * E + align - 1) / align * align;
-    if (M_cap < need_rows || !workspace || workspace_bytes < mx_route_workspace_bytes(T, E)) return MX_EINVAL;
-    if (T * k >= (int64_t)1 << 31 || E * 8 > 48 * 1024) return MX_EINVAL;
+    return M_cap < need_rows ? MX_EINVAL : MX_OK;
+}
+
+int route_check(const int32_t* topk, int64_t T, int64_t k, int64_t E, int64_t align, int64_t M_cap,
+                const int64_t* seg_offsets, const int32_t* src, const int32_t* pos, const void* workspace,
+                size_t workspace_bytes) {
+    if (int st = route_check_args(topk, T, k, E, align, M_cap, seg_offsets, src, pos)) return st;
+    if (!workspace || workspace_bytes < mx_route_workspace_bytes(T, E)) return MX_EINVAL;
     return MX_OK;
 }
 
@@ -431,8 +473,7 @@ int route_scratch_address(void** out) {
 extern "C" int moe_route_static(const int32_t* topk, int64_t T, int64_t k, int64_t E, int64_t M_cap,
                                 int64_t* seg_offsets, int32_t* src, int32_t* pos, cudaStream_t stream) {
     MX_NVTX_RANGE("moe_route_static");
-    if (!topk || !seg_offsets || !src || !pos || T < 0 || k <= 0 || k > 32 || E <= 0 || M_cap < 0 || M_cap % 128)
-        return MX_EINVAL;
+    if (int st = route_check_args(topk, T, k, E, 128, M_cap, seg_offsets, src, pos)) return st;
     if (mx_route_workspace_bytes(T, E) > kRouteStaticScratchBytes) return MX_EINVAL;   // beyond the fixed scratch
     if (int st = mx_check_device()) return st;
     void* scratch = nullptr;

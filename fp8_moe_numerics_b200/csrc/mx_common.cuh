@@ -37,6 +37,9 @@ int mx_check_device(void);              // MX_OK on sm_100, else MX_EUNSUPPORTED
 int mx_launch_status(void);             // cudaGetLastError -> MX_OK / MX_ECUDA
 void mx_count_launch(void);             // one more kernel launched by this library (mx_kernel_launches)
 int mx_status_word_address(unsigned int** out);   // device address of the bounded-wait status word
+// Bits of the device status word: a bounded wait expired; a routing entry was
+// out of range or repeated within its token.
+constexpr unsigned int kStatusTimeout = 1u, kStatusBadRoute = 2u;
 struct CUtensorMap_st;
 int mx_make_bf16_tile_map(struct CUtensorMap_st* m, const void* base, int64_t rows, int64_t cols, int box_cols,
                           int box_rows);             // bf16 [rows, cols] TMA map, 128-byte swizzle

@@ -90,6 +90,7 @@ moe_combine_s2f6_kernel(const uint8_t* __restrict__ codes, const uint8_t* __rest
     for (int i = 0; i < 32; ++i) u[i] = 0.0f;
     for (int64_t j = 0; j < k; ++j) {
         const int64_t r = __ldg(pos + t * k + j);
+        if (r < 0) continue;                               // entry left out by the routing
         const float wj = wts ? __ldg(wts + t * k + j) : 1.0f;
         const int e = (int)__ldg(e8m0 + r * nbc + jb) - 127;
         const float sc = __fmul_rn(wj, pow2_int(e - 6));

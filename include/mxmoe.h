@@ -61,7 +61,7 @@
 extern "C" {
 #endif
 
-enum { MX_OK = 0, MX_EINVAL = 1, MX_ECUDA = 2, MX_ETIMEOUT = 3, MX_EUNSUPPORTED = 4 };
+enum { MX_OK = 0, MX_EINVAL = 1, MX_ECUDA = 2, MX_ETIMEOUT = 3, MX_EUNSUPPORTED = 4, MX_EDATA = 5 };
 enum { MX_SF_ROWMAJOR = 0, MX_SF_MMA = 1 };
 enum { MX_OUT_F32 = 0, MX_OUT_BF16 = 1 };
 enum { MX_ROUND_RNE = 0, MX_ROUND_SR = 1 };
@@ -79,8 +79,10 @@ MX_API unsigned long long mx_kernel_launches(void);
 
 /* Synchronises `stream`, then returns and clears the device status word of
  * the current device: MX_ETIMEOUT if a bounded wait inside a GEMM kernel
- * expired since the last call (that kernel's output is then undefined),
- * MX_ECUDA if the synchronisation failed, else MX_OK. */
+ * expired since the last call (that kernel's output is then undefined);
+ * otherwise MX_EDATA if a routing call since the last call met an expert id
+ * outside [0, E) or the same id twice in one token (those entries were left
+ * out, see moe_route); MX_ECUDA if the synchronisation failed; else MX_OK. */
 MX_API int mx_sync_status(cudaStream_t stream);
 
 /* Failure-detection self-test: one kernel waits on a barrier that nothing
@@ -220,7 +222,12 @@ MX_API size_t mx_route_workspace_bytes(int64_t T, int64_t E);
  *   pos        device int32 [T, k] out: row of assignment (t, j)
  *   workspace  device, mx_route_workspace_bytes(T, E) bytes of scratch
  * Rows of one expert are in increasing token order.  M_cap must be at least
- * T*k + 127*E rounded up to 128. */
+ * T*k + 127*E rounded up to 128; (E+1)*8 <= 48 KiB; T*k < 2^31.
+ * An entry whose id is outside [0, E), or repeats an id of an earlier entry of
+ * the same token, is left out: it takes no row, its pos is -1 (moe_combine,
+ * moe_combine_s2f6 and moe_dispatch_grad skip such entries), and the next
+ * mx_sync_status() returns MX_EDATA.  Nothing is read or written outside the
+ * buffers above.  The launches stop at the first launch failure (MX_ECUDA). */
 MX_API int moe_route(const int32_t* topk, int64_t T, int64_t k, int64_t E, int64_t M_cap,
               int64_t* seg_offsets, int32_t* src, int32_t* pos,
               void* workspace, size_t workspace_bytes, cudaStream_t stream);

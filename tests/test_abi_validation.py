@@ -50,6 +50,8 @@ CASES = {
     "moe_route": ((A, 16, 2, 4, 640, A, A, A, A, 4096, None), [
         ("capacity below the padded rows", {4: 512}), ("workspace too small", {9: 16}), ("k > 32", {2: 33}),
         ("no experts", {3: 0}), ("M_cap % 128", {4: 600}), ("null workspace", {8: None}),
+        # the scan's (E + 1) int64 starts exceed 48 KiB of shared memory at E = 6144 (E * 8 alone does not)
+        ("scan shared memory, E = 6144", {3: 6144, 4: 128 * 6144 + 128, 9: 1 << 20}),
     ]),
     "moe_route_aligned": ((A, 16, 2, 4, 256, 1280, A, A, A, A, 4096, None), [
         ("align 64", {4: 64}), ("M_cap % align", {5: 1152}), ("capacity below the padded rows", {5: 1024}),
@@ -57,7 +59,8 @@ CASES = {
     ]),
     "moe_route_static": ((A, 16, 2, 4, 640, A, A, A, None), [
         ("null topk", {0: None}), ("M_cap % 128", {4: 100}), ("k 0", {2: 0}),
-        ("beyond the fixed scratch", {1: 1 << 20, 3: 64}),
+        ("beyond the fixed scratch", {1: 1 << 20, 3: 64}), ("null pos", {7: None}),
+        ("scan shared memory, E = 6144", {1: 0, 3: 6144, 4: 128 * 6144 + 128}),
     ]),
     "nvfp4_gather_rows": ((A, A, A, A, 2, 128, 64, A, A, A, None), [
         ("cols % 64", {6: 32}), ("M_cap % 128", {5: 100}), ("k 0", {4: 0}), ("sf misaligned", {1: A1}),
@@ -152,3 +155,22 @@ def test_each_broken_requirement_is_rejected_on_the_host(mx, name):
             args[i] = v
         assert fn(*args) == MX_EINVAL, (name, what)
     assert mx.mx_kernel_launches() == before
+
+
+@pytest.mark.parametrize("name", ["moe_route", "moe_route_static"])
+def test_empty_routing_accepts_null_token_arrays(mx, name):
+    """An empty problem (T = 0) may pass NULL topk and pos, as the header's
+    convention says; the call then fails only at the device check here."""
+    if torch.cuda.is_available():
+        pytest.skip("the host-valid call would reach a launch on a GPU machine")
+    args = {"moe_route": (None, 0, 2, 4, 512, A, A, None, A, 4096, None),
+            "moe_route_static": (None, 0, 2, 4, 512, A, A, None, None)}[name]
+    assert getattr(mx, name)(*args) == MX_ECUDA
+
+
+def test_route_workspace_size_saturates_instead_of_wrapping(mx):
+    size_max = (1 << 64) - 1
+    assert mx.mx_route_workspace_bytes(16, 4) == (1 * 4 + 4) * 4      # one chunk histogram + counts
+    assert mx.mx_route_workspace_bytes(1 << 62, 1 << 20) == size_max
+    assert mx.mx_route_workspace_bytes((1 << 63) - 1, 2) == ((1 << 55) * 2 + 2) * 4   # largest T, no overflow
+    assert mx.mx_route_workspace_bytes((1 << 63) - 1, 1 << 10) == size_max

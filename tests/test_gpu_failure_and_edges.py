@@ -71,3 +71,60 @@ def test_gemms_with_no_routed_rows(cuda):
     api.grouped_gemm_mxfp8(api.MX_GEMM_WGRAD, ac, ae, bc, be, seg, E, M_cap, N, K, out=dw)
     api.sync_status()
     assert torch.all(dw == 0)
+
+
+def test_routing_leaves_out_bad_ids_and_reports_them(cuda):
+    """Expert ids outside [0, E) and an id repeated within a token are left
+    out of the routing (pos = -1, no row), flagged as MX_EDATA by the next
+    status query, and skipped by the combine; nothing is written outside the
+    buffers and the context stays usable."""
+    from fp8_moe_numerics_b200._lib import MX_EDATA
+    rng = np.random.default_rng(3)
+    T, k, E, D = 300, 4, 8, 64
+    topk = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+    topk[5, 1] = -3
+    topk[17, 0] = E
+    topk[40, 3] = 1 << 30
+    topk[41, 2] = topk[41, 0]                            # repeat within one token
+    topk[299, 1] = -(1 << 31)
+    valid = np.ones((T, k), bool)
+    valid[5, 1] = valid[17, 0] = valid[40, 3] = valid[41, 2] = valid[299, 1] = False
+    api.sync_status()
+    seg, src, pos = api.moe_route(torch.from_numpy(topk).cuda(), E)
+    with pytest.raises(MxError) as err:
+        api.sync_status()
+    assert err.value.status == MX_EDATA
+    api.sync_status()                                   # cleared by the previous query
+    # expected routing of the valid entries: per expert in token order, segments padded to 128
+    counts = np.bincount(topk[valid], minlength=E)
+    seg_ref = np.concatenate([[0], np.cumsum((counts + 127) // 128 * 128)])
+    assert np.array_equal(seg.cpu().numpy(), seg_ref)
+    pos_ref = np.full((T, k), -1, np.int64)
+    fill = seg_ref[:-1].copy()
+    for t in range(T):
+        for j in range(k):
+            if valid[t, j]:
+                pos_ref[t, j] = fill[topk[t, j]]
+                fill[topk[t, j]] += 1
+    assert np.array_equal(pos.cpu().numpy(), pos_ref)
+    src_np = src.cpu().numpy()
+    src_ref = np.full(src_np.shape, -1, np.int64)
+    src_ref[pos_ref[valid]] = np.flatnonzero(valid.ravel())
+    assert np.array_equal(src_np, src_ref)
+    # the combine skips the left-out entries
+    y = torch.randn(src.shape[0], D, device="cuda").to(torch.bfloat16)
+    w = torch.rand(T, k, device="cuda")
+    out = api.moe_combine(y, pos, w, D).float().cpu()
+    yh, wh = y.float().cpu(), w.cpu()
+    ref = torch.zeros(T, D)
+    for j in range(k):
+        p = torch.from_numpy(pos_ref[:, j])
+        ok = p >= 0
+        ref[ok] += wh[ok, j:j + 1] * yh[p[ok]]
+    assert torch.allclose(out, ref, rtol=2 ** -7, atol=1e-6)
+    # a valid routing afterwards matches the oracle
+    good = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+    seg, src, pos = api.moe_route(torch.from_numpy(good).cuda(), E)
+    api.sync_status()
+    seg_o, src_o, pos_o = oracle.route(good, E)
+    assert np.array_equal(seg.cpu().numpy(), seg_o) and np.array_equal(pos.cpu().numpy(), pos_o)
