@@ -310,26 +310,29 @@ def run_ours(args):
     kind, wk = work[dom]
     per_launch_ms = stage_ms[dom] / K
     if kind == "alu":
+        # the requantisation: algorithmic bytes against HBM (the roofline), with the kernel's issue rate
+        # (warp-instructions per element from one ncu capture) beside it as a diagnostic
         nbytes, elems = wk
-        achieved = REQUANT_WARP_INST_PER_ELEM * elems / (per_launch_ms * 1e-3) / 1e9
-        roof = {"bound": "alu", "achieved": round(achieved, 1), "peak": round(issue_peak, 1), "unit": "Ginst/s",
-                "frac": round(achieved / issue_peak, 4),
+        achieved = nbytes / (per_launch_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm"], 4),
                 "traffic": round(REQUANT_DRAM_BYTES_PER_ELEM * elems) if REQUANT_DRAM_BYTES_PER_ELEM else None,
-                "kernel": dom,
-                "peak_source": f"{sms} SMs x 4 warp schedulers x {SM_MAX_MHZ} MHz (one warp-instruction each per "
-                               "clock); instructions per element from ncu smsp__inst_executed",
-                "hbm_frac": round(nbytes / (per_launch_ms * 1e-3) / 1e9 / peaks["hbm"], 4)}
+                "kernel": dom, "algorithmic_bytes": int(nbytes),
+                "peak_source": peaks["src"] + " copy bandwidth",
+                "issue_frac": round(REQUANT_WARP_INST_PER_ELEM * elems / (per_launch_ms * 1e-3) / 1e9 / issue_peak, 4),
+                "issue_note": f"warp-instructions per element {REQUANT_WARP_INST_PER_ELEM} (ncu) x elements / time, "
+                              f"against {sms} SMs x 4 schedulers x {SM_MAX_MHZ} MHz"}
     elif kind == "hbm":
         achieved = wk / (per_launch_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm"], "unit": "GB/s",
-                "frac": round(achieved / peaks["hbm"], 4), "traffic": None, "kernel": dom,
+                "frac": round(achieved / peaks["hbm"], 4), "traffic": None, "kernel": dom, "algorithmic_bytes": int(wk),
                 "peak_source": peaks["src"] + " copy bandwidth"}
     else:
         ratio = 4 if kind == "tensor4" else 2
         peak = peaks["bf16_sus"] * ratio
         achieved = wk / (per_launch_ms * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
-                "frac": round(achieved / peak, 4), "traffic": None, "kernel": dom,
+                "frac": round(achieved / peak, 4), "traffic": None, "kernel": dom, "algorithmic_flops": int(wk),
                 "peak_source": f"{peaks['src']} sustained bf16 x {ratio} (nominal dense ratio)"}
     breakdown = {}
     for n in names:
@@ -358,6 +361,13 @@ def run_ours(args):
 
     # ---------------------------------------------------------------- e2e
     e2e = e2e_leg(layer, inp, dev, args, gemm_flops / K, pg, world)
+    cpu_sample = {"x": inp["x"][:256].cpu(), "w1": inp["w1"][0:1, :256].cpu()}
+
+    # the 64-expert layer's forward GEMMs and backward, after the 384-expert layer's buffers are released
+    del layer, inp, topk
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    cfg_legs = gemm_config_legs(dev, peaks) if rank == 0 else None
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": K,
@@ -376,6 +386,8 @@ def run_ours(args):
         "quantiser": quant,
         "combine_s2f6": s2f6,
         "mxfp8_forward": mx_fwd,
+        "fwd_gemm": cfg_legs["fwd_gemm"] if cfg_legs else None,
+        "bwd_gemm": cfg_legs["bwd_gemm"] if cfg_legs else None,
         "roofline": roof,
         "clocks": clk.summary(),
         "e2e": e2e,
@@ -383,7 +395,7 @@ def run_ours(args):
         "impl": "ours",
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(inp, layer, seconds=args.cpu_seconds)
+        line["cpu_baseline"] = cpu_baseline(cpu_sample, seconds=args.cpu_seconds)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if pg is not None:
@@ -401,7 +413,9 @@ def quantiser_stream(dev, peaks, reps: int = 20):
     x = workloads.activations(rows, cols, c["x_dist"], c["seed"], dev)
     q = api.nvfp4_quantize(x, 1, api.MX_SF_MMA)
     t = api.mxfp8_requant_transpose_sr(*q, rows, cols, 1, api.MX_SF_MMA, None, c["sr_seed"], 0, 16, api.MX_SF_MMA)
-    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    # L2 is flushed by READING a 512 MB buffer (a reduction): zeroing it instead would leave up to
+    # 126 MB of dirty lines that the next, timed launch writes back
+    flush = torch.ones(64 << 20, dtype=torch.int64, device=dev)
     hs = api.hadamard_s2f6_quantize(x, c["sr_seed"], 101)
     res = {}
     for name, fn, nbytes in (
@@ -416,7 +430,7 @@ def quantiser_stream(dev, peaks, reps: int = 20):
             fn()
         ms = []
         for _ in range(reps):
-            flush.zero_()
+            flush.sum()
             a = torch.cuda.Event(enable_timing=True)
             b = torch.cuda.Event(enable_timing=True)
             a.record()
@@ -428,7 +442,8 @@ def quantiser_stream(dev, peaks, reps: int = 20):
         gbs = nbytes / (med * 1e-3) / 1e9
         res[name] = {"us": round(med * 1e3, 2), "GB/s": round(gbs, 1), "frac_hbm_measured": round(gbs / peaks["hbm"], 3),
                      "frac_hbm_8tbs": round(gbs / NOMINAL_HBM_GBS, 3), "bytes": int(nbytes)}
-    res["workload"] = "quant_stream: bf16 16384x4096 Student-t(4) x 10^U(-3,3) per row; L2 flushed per launch"
+    res["workload"] = ("quant_stream: bf16 16384x4096 Student-t(4) x 10^U(-3,3) per row; L2 flushed before every "
+                       "launch by a read-only pass over 512 MB; median of 20")
     return res
 
 
@@ -518,6 +533,81 @@ def mxfp8_forward_leg(layer, counts, peaks, breakdown, reps: int = 10):
     return res
 
 
+def gemm_config_legs(dev, peaks, steps: int = 3, warmup: int = 2):
+    """The 64-expert layer (top-8 of 16384 tokens, Zipf(1.1), d_model 4096,
+    d_ff 1536 SwiGLU, N(0,1) tokens): its two NVFP4 forward GEMMs, and its
+    backward (requantisation of the saved NVFP4 operands, MXFP8 dgrad and wgrad)
+    on an upstream gradient N(0, 1e-3).  Whole layer steps, each stage timed by
+    CUDA events as in the main step."""
+    import torch
+    from fp8_moe_numerics_b200 import api, workloads
+    from fp8_moe_numerics_b200.layer import ExpertLayer
+    c, cb = workloads.CONFIGS["fwd_gemm"], workloads.CONFIGS["bwd_gemm"]
+    inp = workloads.layer_inputs("fwd_gemm", device=dev)
+    T, k, E, D, F = c["T"], c["k"], c["E"], c["D"], c["F"]
+    dout = workloads.gradient(T, D, cb["grad_std"], cb["seed"] + 4, dev)
+    layer = ExpertLayer(inp["x"], inp["topk"].to(dev), inp["w_comb"].to(dev), inp["w1"], inp["w2"], dout,
+                        gated=c["gated"], seed=c["seed"])
+    counts = torch.bincount(inp["topk"].reshape(-1).long(), minlength=E).tolist()
+    M_pad = sum((x + 127) // 128 * 128 for x in counts)
+    for _ in range(warmup):
+        layer.step()
+    torch.cuda.synchronize()
+    layer.reset_marks()
+    for _ in range(steps):
+        layer.step(record=True)
+    torch.cuda.synchronize()
+    api.sync_status()
+    st = layer.stage_times_ms()
+    work = stage_work(c, counts, M_pad)
+    out = {}
+    for n, (kind, wk) in work.items():
+        if n not in st:
+            continue
+        t = st[n] / steps
+        if kind in ("tensor4", "tensor8"):
+            ratio = 4 if kind == "tensor4" else 2
+            tf = wk / (t * 1e-3) / 1e12
+            out[n] = {"ms": round(t, 4), "TFLOP/s": round(tf, 1),
+                      "frac_nominal": round(tf / (NOMINAL_NVFP4_TFLOPS if ratio == 4 else NOMINAL_MXFP8_TFLOPS), 4),
+                      "frac_measured": round(tf / (peaks["bf16_sus"] * ratio), 4)}
+        else:
+            nbytes = wk[0] if kind == "alu" else wk
+            gbs = nbytes / (t * 1e-3) / 1e9
+            out[n] = {"ms": round(t, 4), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm"], 4)}
+
+    def total(names, kind):
+        ms = sum(out[n]["ms"] for n in names)
+        if kind == "flops":
+            tf = sum(work[n][1] for n in names) / (ms * 1e-3) / 1e12
+            return {"ms": round(ms, 4), "TFLOP/s": round(tf, 1)}
+        gbs = sum(work[n][1][0] for n in names) / (ms * 1e-3) / 1e9
+        return {"ms": round(ms, 4), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm"], 4)}
+
+    fwd = total(("gemm1", "gemm2"), "flops")
+    fwd["frac_of_9pf_nominal"] = round(fwd["TFLOP/s"] / NOMINAL_NVFP4_TFLOPS, 4)
+    fwd["frac_measured"] = round(fwd["TFLOP/s"] / (peaks["bf16_sus"] * 4), 4)
+    bwd = total(("dgrad2", "wgrad2", "dgrad1", "wgrad1"), "flops")
+    bwd["frac_of_4p5pf_nominal"] = round(bwd["TFLOP/s"] / NOMINAL_MXFP8_TFLOPS, 4)
+    bwd["frac_measured"] = round(bwd["TFLOP/s"] / (peaks["bf16_sus"] * 2), 4)
+    req = total(("requant_w2", "requant_a", "requant_w1", "requant_x"), "bytes")
+    res = {
+        "fwd_gemm": {"workload": f"64 experts, top-8 of {T} tokens ({T * k} routed rows, {M_pad} padded), Zipf(1.1), "
+                                 "d_model 4096, W1 4096->3072 (SwiGLU), W2 1536->4096, N(0,1) tokens",
+                     "nvfp4_gemms": fwd, "gemm1": out["gemm1"], "gemm2": out["gemm2"]},
+        "bwd_gemm": {"workload": "the same layer's backward on an upstream gradient N(0,1e-3): requantisation of "
+                                 "the saved NVFP4 W1, W2, tokens and activations to MXFP8 with stochastic rounding "
+                                 "(R = 16), MXFP8 dgrad and wgrad of both GEMMs (dH1 is the SwiGLU backward of "
+                                 "dgrad2's output)",
+                     "mxfp8_gemms": bwd, "requant": req,
+                     **{n: out[n] for n in ("requant_w2", "dgrad2", "requant_a", "wgrad2", "requant_w1", "dgrad1",
+                                            "requant_x", "wgrad1")}},
+        "steps": steps,
+    }
+    del layer, inp, dout
+    return res
+
+
 def e2e_leg(layer, inp, dev, args, flops_per_step, pg, world):
     """Same metric through the public API with host buffers: every step copies
     its inputs (tokens, routing, combine weights, upstream gradient) from
@@ -549,7 +639,7 @@ def e2e_leg(layer, inp, dev, args, flops_per_step, pg, world):
                                 "(copies of neighbouring steps overlap each step's kernels)"}
 
 
-def cpu_baseline(inp, layer, seconds: float = 15.0):
+def cpu_baseline(inp, seconds: float = 15.0):
     """The oracle, as it stands, on the host cores: NVFP4-quantise a sample of
     token rows and expert-weight rows and run the fp64 grouped GEMM of those
     rows against one expert's W1 tile, until ~`seconds` of CPU work."""

@@ -359,8 +359,8 @@ def swiglu_nvfp4_quantize(h: torch.Tensor, F: int, gated: bool = True, rows_vali
     return codes, sf, outer
 
 
-# NVFP4 in the backward pass and the 16x16 shared-scale format (not yet run
-# against the oracle on a GPU; include/mxmoe.h gives the readings).
+# NVFP4 in the backward pass and the 16x16 shared-scale format
+# (include/mxmoe.h gives the readings).
 
 def nvfp4_quantize_sr(x: torch.Tensor, group_rows: int = 1, rounding: int = MX_ROUND_SR, seed: int = 0,
                       stream_id: int = 0, rbits: int = 16, sf_layout: int = MX_SF_MMA, out=None):

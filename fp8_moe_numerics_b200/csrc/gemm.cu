@@ -1172,7 +1172,7 @@ extern "C" int grouped_gemm_mxfp8(int mode, const uint8_t* a_codes, const uint8_
 // row), b_outer [E].  out[e, n, k] = a_outer[e*N + n] * b_outer[e] * sum over
 // the tokens of segment e.  Segments must be multiples of 256 tokens (a
 // K-stage of NVFP4 holds 256); other boundaries give wrong sums, no
-// out-of-bounds access.  Not yet run on a GPU.
+// out-of-bounds access.
 extern "C" int grouped_gemm_nvfp4_wgrad(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_outer,
                                         const uint8_t* b_codes, const uint8_t* b_sf, const float* b_outer,
                                         const int64_t* seg_offsets, int64_t E, int64_t M_cap, int64_t N, int64_t K,

@@ -45,8 +45,7 @@ class ExpertLayer:
     one byte per value plus one exponent per 32).  `backward` is "mxfp8" (the
     pages' recipe) or "nvfp4": the four backward GEMMs in NVFP4 with
     stochastically rounded operands (the pages' stated future work; routing
-    then pads experts to 256 rows for the NVFP4 wgrad's K-stage; its kernels
-    have not yet run on a GPU).
+    then pads experts to 256 rows for the NVFP4 wgrad's K-stage).
     """
 
     S2F6_STREAM = 101                                   # Philox stream of the rotation's signs

@@ -374,7 +374,6 @@ MX_API int moe_combine_s2f6(const int8_t* codes, const uint8_t* e8m0, const int3
  *             stream of mxfp8_requant_transpose_sr, L = the element's linear
  *             index in the output); magnitudes past 6 saturate; the sign of y
  *             is kept, also on a zero.
- * These entry points have not yet been run against the oracle on a GPU.
  * ------------------------------------------------------------------------ */
 
 /* nvfp4_quantize_sr -- bf16 [rows, cols] -> NVFP4 with the rounding above

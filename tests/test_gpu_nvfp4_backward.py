@@ -7,9 +7,8 @@ draws the same Philox integers.  The NVFP4 dgrad (the forward grouped GEMM
 with the requantised W_e^T stack as B) within the forward GEMM's relative
 Frobenius bound of the oracle's fp64 product.
 
-The kernels have not yet run on a GPU: their index arithmetic is checked on
-the CPU (tests/test_nvfp4_bwd_indexing.py) and the module stays skipped until
-a first run on a B200 has passed it.
+Their index arithmetic is also replayed on the CPU
+(tests/test_nvfp4_bwd_indexing.py).
 """
 import numpy as np
 import pytest
@@ -20,8 +19,7 @@ from fp8_moe_numerics_b200 import api
 from tests.layouts import mma_to_rowmajor
 from tests.test_gpu_gemm import dev, rel_fro
 
-pytestmark = [pytest.mark.gpu,
-              pytest.mark.skip(reason="not yet run on a GPU; enable after a first run of this module on a B200")]
+pytestmark = pytest.mark.gpu
 
 
 def to_dev_bf16(u16):
