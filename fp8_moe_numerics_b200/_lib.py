@@ -43,6 +43,7 @@ SIGNATURES = {
     "moe_route_static": (I32, [P, I64, I64, I64, I64, P, P, P, P]),
     "moe_route_aligned": (I32, [P, I64, I64, I64, I64, I64, P, P, P, P, SZ, P]),
     "nvfp4_gather_rows": (I32, [P, P, P, P, I64, I64, I64, P, P, P, P]),
+    "moe_permute_row_groups": (I32, [P, I64, P, I64, I64, P, P]),
     "swiglu_fwd": (I32, [P, I64, I64, I32, P, P, P]),
     "swiglu_bwd": (I32, [P, P, I64, I64, I32, P, P, P]),
     "swiglu_nvfp4_quantize": (I32, [P, I64, I64, I32, P, P, P, P, I32, P]),

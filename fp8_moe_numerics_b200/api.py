@@ -28,7 +28,7 @@ __all__ = [
     "moe_combine", "moe_dispatch_grad", "swiglu_nvfp4_quantize", "hadamard_s2f6_quantize", "grouped_gemm_nvfp4_s2f6",
     "moe_combine_s2f6", "nvfp4_quantize_sr", "nvfp4_requant_transpose_sr", "nvfp4_quantize_tile16",
     "nvfp4_quantize_transpose_segments", "nvfp4_requant_transpose_segments", "grouped_gemm_nvfp4_wgrad",
-    "max_routed_rows",
+    "max_routed_rows", "moe_permute_row_groups",
 ]
 
 
@@ -245,6 +245,24 @@ def nvfp4_gather_rows(codes, sf_rowmajor, outer, src: torch.Tensor, k: int, cols
     L.call("nvfp4_gather_rows", _p(codes), _p(sf_rowmajor), _p(outer), _p(src), k, M_cap, cols, _p(oc), _p(osf),
            _p(oo), _s())
     return oc, osf, oo
+
+
+def moe_permute_row_groups(x: torch.Tensor, group_src: torch.Tensor, group_bytes: int, out=None):
+    """Regroup a row buffer array by whole groups of `group_bytes` bytes (128
+    rows' worth): out group g = x group group_src[g] (int32 on the device), or
+    zeros where group_src[g] < 0."""
+    nin = x.numel() * x.element_size() // group_bytes
+    nout = group_src.numel()
+    if out is None:
+        out = torch.empty(nout * group_bytes // x.element_size(), dtype=x.dtype, device=x.device)
+    if group_src.dtype != torch.int32:
+        raise ValueError("group_src must be int32")
+    _fits("out", out, nout * group_bytes)
+    if out.data_ptr() < x.data_ptr() + x.numel() * x.element_size() and \
+            x.data_ptr() < out.data_ptr() + out.numel() * out.element_size():
+        raise ValueError("moe_permute_row_groups: in and out overlap")
+    L.call("moe_permute_row_groups", _p(x), nin, _p(out), nout, group_bytes, _p(group_src), _s())
+    return out
 
 
 def swiglu_fwd(h: torch.Tensor, F: int, gated: bool = True, rows_valid=None, out=None):

@@ -7,6 +7,7 @@
 // quantised once and gathered into expert-major order.
 #include "mx_common.cuh"
 
+#include <algorithm>
 #include <mutex>
 
 namespace {
@@ -423,6 +424,56 @@ extern "C" int moe_dispatch_grad(const void* dout, const int32_t* src, const int
     const int64_t blocks = T + (M_cap + 31) / 32;
     dispatch_grad_kernel<<<(unsigned)blocks, kDispatchThreads, 0, stream>>>(
         static_cast<const uint16_t*>(dout), src, pos, w, T, k, M_cap, D, static_cast<uint16_t*>(dy));
+    mx_count_launch();
+    return mx_launch_status();
+}
+
+// ===========================================================================
+// moe_permute_row_groups -- moves whole 128-row groups of an expert-major
+// buffer (the unit every expert segment is padded to) from one order into
+// another: the reordering of the expert-parallel exchange, where rows arrive
+// grouped by source rank and the expert GEMMs want them grouped by expert.
+// ===========================================================================
+namespace {
+
+constexpr int kPermuteThreads = 256;
+
+// Output group g = input group group_src[g] (group_vec 16-byte vectors each),
+// or zeros where group_src[g] < 0; an index past the input is written as zeros
+// and flags the device status word.
+__global__ void __launch_bounds__(kPermuteThreads)
+permute_row_groups_kernel(const uint4* __restrict__ in, int64_t ngroups_in, uint4* __restrict__ out,
+                          int64_t ngroups_out, int64_t group_vec, const int32_t* __restrict__ group_src,
+                          unsigned int* __restrict__ status) {
+    const int64_t total = ngroups_out * group_vec;
+    for (int64_t v = (int64_t)blockIdx.x * kPermuteThreads + threadIdx.x; v < total;
+         v += (int64_t)gridDim.x * kPermuteThreads) {
+        const int64_t g = v / group_vec, i = v - g * group_vec;
+        const int32_t sg = __ldg(group_src + g);
+        uint4 val = make_uint4(0u, 0u, 0u, 0u);
+        if (sg >= 0 && sg < ngroups_in) val = __ldcs(in + sg * group_vec + i);
+        else if (sg >= 0 && i == 0) atomicOr(status, kStatusBadRoute);
+        out[v] = val;
+    }
+}
+
+}  // namespace
+
+extern "C" int moe_permute_row_groups(const void* in, int64_t ngroups_in, void* out, int64_t ngroups_out,
+                                      int64_t group_bytes, const int32_t* group_src, cudaStream_t stream) {
+    MX_NVTX_RANGE("moe_permute_row_groups");
+    if (((!out || !group_src) && ngroups_out > 0) || (!in && ngroups_in > 0) || ngroups_in < 0 || ngroups_out < 0 ||
+        group_bytes <= 0 || group_bytes % 16 || !mx_aligned(in, 16) || !mx_aligned(out, 16))
+        return MX_EINVAL;
+    if (int st = mx_check_device()) return st;
+    if (ngroups_out == 0) return MX_OK;
+    unsigned int* status = nullptr;
+    if (int st = mx_status_word_address(&status)) return st;
+    const int64_t total = ngroups_out * (group_bytes / 16);
+    const int64_t blocks = std::min<int64_t>((total + kPermuteThreads - 1) / kPermuteThreads, 148 * 16);
+    permute_row_groups_kernel<<<(unsigned)blocks, kPermuteThreads, 0, stream>>>(
+        static_cast<const uint4*>(in), ngroups_in, static_cast<uint4*>(out), ngroups_out, group_bytes / 16, group_src,
+        status);
     mx_count_launch();
     return mx_launch_status();
 }

@@ -82,7 +82,8 @@ MX_API unsigned long long mx_kernel_launches(void);
  * expired since the last call (that kernel's output is then undefined);
  * otherwise MX_EDATA if a routing call since the last call met an expert id
  * outside [0, E) or the same id twice in one token (those entries were left
- * out, see moe_route); MX_ECUDA if the synchronisation failed; else MX_OK. */
+ * out, see moe_route) or a row-group permutation met a group index past its
+ * input; MX_ECUDA if the synchronisation failed; else MX_OK. */
 MX_API int mx_sync_status(cudaStream_t stream);
 
 /* Failure-detection self-test: one kernel waits on a barrier that nothing
@@ -255,6 +256,23 @@ MX_API int moe_route_aligned(const int32_t* topk, int64_t T, int64_t k, int64_t 
  * streams, other host threads) race on the array and give undefined results. */
 MX_API int moe_route_static(const int32_t* topk, int64_t T, int64_t k, int64_t E, int64_t M_cap,
                             int64_t* seg_offsets, int32_t* src, int32_t* pos, cudaStream_t stream);
+
+/* moe_permute_row_groups -- reorder an expert-major row buffer by whole
+ * groups of 128 rows (the unit every expert segment is padded to).
+ * [ai-primer §Quantized NVLink and BBBK]: tokens travel to the GPU holding
+ * their expert in NVFP4 and come back through the combine; in that exchange
+ * rows arrive grouped by source rank, and this call regroups them by expert
+ * (and back) without touching their bytes.
+ *   in         device, ngroups_in groups of group_bytes bytes (one array of a
+ *              row buffer: codes, MMA-layout scales, outer scales, bf16 rows...)
+ *   out        device, ngroups_out groups of group_bytes bytes
+ *   group_src  device int32 [ngroups_out]: input group of output group g, or
+ *              -1 for a group of zeros
+ * An index >= ngroups_in is written as zeros and the next mx_sync_status()
+ * returns MX_EDATA.  Requires group_bytes % 16 == 0 and 16-byte aligned
+ * in/out; in and out must not overlap. */
+MX_API int moe_permute_row_groups(const void* in, int64_t ngroups_in, void* out, int64_t ngroups_out,
+                                  int64_t group_bytes, const int32_t* group_src, cudaStream_t stream);
 
 /* nvfp4_gather_rows -- dispatch per-token NVFP4 rows into expert-major order:
  * row p of the output is row src[p]/k of the input (zeros when src[p] < 0).

@@ -66,6 +66,10 @@ CASES = {
         ("cols % 64", {6: 32}), ("M_cap % 128", {5: 100}), ("k 0", {4: 0}), ("sf misaligned", {1: A1}),
         ("out_codes misaligned", {7: A8}), ("null src", {3: None}),
     ]),
+    "moe_permute_row_groups": ((A, 4, A, 6, 512, A, None), [
+        ("group_bytes % 16", {4: 520}), ("group_bytes 0", {4: 0}), ("null out", {2: None}), ("null table", {5: None}),
+        ("in misaligned", {0: A8}), ("out misaligned", {2: A4}), ("negative ngroups_in", {1: -1}),
+    ]),
     "swiglu_fwd": ((A, 128, 64, 1, None, A, None), [
         ("F % 8", {2: 12}), ("null h", {0: None}), ("negative rows", {1: -1}), ("a misaligned", {5: A8}),
     ]),

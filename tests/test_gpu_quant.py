@@ -356,3 +356,29 @@ def test_combine_and_dispatch_grad(cuda):
         gdy = to_np_u16(api.moe_dispatch_grad(to_dev_bf16(dout), gsrc, gpos, wd))
         assert np.array_equal(gdy[:M], ref_dy)
         assert np.all(gdy[M:] == 0)
+
+
+def test_permute_row_groups_against_indexing(cuda):
+    """moe_permute_row_groups moves whole 128-row groups (the expert-parallel
+    regrouping): equal to indexing by the table, zeros for -1; an index past
+    the input gives zeros and MX_EDATA, not a fault."""
+    from fp8_moe_numerics_b200._lib import MX_EDATA, MxError
+    g = torch.Generator(device="cuda")
+    g.manual_seed(3)
+    for group_bytes, n_in in ((128 * 2048, 9), (128 * 128, 5), (512, 40)):
+        x = torch.randint(0, 256, (n_in * group_bytes,), dtype=torch.uint8, device="cuda", generator=g)
+        table = torch.tensor([3, -1, 0, n_in - 1, 1, 1, 2, -1], dtype=torch.int32, device="cuda")
+        out = api.moe_permute_row_groups(x, table, group_bytes)
+        api.sync_status()
+        xg = x.view(-1, group_bytes)
+        want = torch.zeros(table.numel(), group_bytes, dtype=torch.uint8, device="cuda")
+        ok = (table >= 0) & (table < n_in)
+        want[ok] = xg[table[ok].long()]
+        assert torch.equal(out.view(-1, group_bytes), want)
+    bad = torch.tensor([0, 7], dtype=torch.int32, device="cuda")
+    out = api.moe_permute_row_groups(torch.ones(2 * 512, dtype=torch.uint8, device="cuda"), bad, 512)
+    with pytest.raises(MxError) as err:
+        api.sync_status()
+    assert err.value.status == MX_EDATA
+    assert torch.all(out[:512] == 1) and torch.all(out[512:] == 0)
+    api.sync_status()
