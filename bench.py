@@ -685,7 +685,7 @@ def run_kernel(args):
         from fp8_moe_numerics_b200.layer import ExpertLayer
         c = workloads.CONFIGS[WORKLOAD]
         inp = workloads.layer_inputs(WORKLOAD, device=dev)
-        layer = ExpertLayer(inp["x"], inp["topk"], inp["w_comb"], inp["w1"], inp["w2"], inp["dout"],
+        layer = ExpertLayer(inp["x"], inp["topk"].to(dev), inp["w_comb"].to(dev), inp["w1"], inp["w2"], inp["dout"],
                             gated=c["gated"], seed=c["seed"], backward="nvfp4")
         run = layer.step
     elif which.startswith("gemm"):

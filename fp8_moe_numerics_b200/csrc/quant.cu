@@ -716,6 +716,179 @@ requant_tile_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict
     tile_emit_transposed<true, kR, kOutLayout>(T, rows, cols, r0, c0, seed, stream_id, out_codes, out_e8m0);
 }
 
+// ---------------------------------------------------------------------------
+// The R = 16 requantisation (the hardware stochastic rounding, the layer's
+// default): a 128 x 64 input tile per block, as in requant_tile_kernel, with
+// the work per element cut down.
+//   Phase 1: each thread decodes 2 rows x 16 columns (one scale block per
+//   row) to the exact f16 products q*sf (cvt e2m1x2 -> f16x2, one f16x2
+//   multiply per pair) and the warp stores its 16 x 64 products transposed
+//   with four stmatrix.trans (8 x 8 blocks of 16-bit values, 8 values per
+//   thread each).  The tile lives in shared memory as f16 [64 cols][128 rows],
+//   16-byte chunks XOR-swizzled by swz() so that both phases are free of bank
+//   conflicts.
+//   Phase 2: each thread takes 16 consecutive rows of one output row, twice:
+//   two 16-byte loads, f16 -> fp32, the outer scale, the 32-row amax (the
+//   block's other half is in lane ^ 8), the E8M0 exponent, y = x * 2^-e and
+//   cvt.rs.  With one outer scale for the whole tile (expert weights) the amax
+//   is taken on the f16 products (s > 0 is monotone) and the two products
+//   fold into one: RN(RN(p s) 2^-e) = RN(p (s 2^-e)) whenever p s stays in
+//   fp32's normal range, which s >= 2^-100 guarantees (|p| >= 2^-10); smaller
+//   s takes the two products.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int rq_swz(int c) { return ((c >> 4) & 3) | ((c & 1) << 2); }
+
+__device__ __forceinline__ uint32_t h2_of_e4m3(uint32_t code) {
+    uint32_t h2;
+    const uint16_t in = (uint16_t)(code * 0x0101u);
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
+    return h2;
+}
+__device__ __forceinline__ uint32_t h2_of_e2m1(uint32_t byte_in_low) {
+    uint32_t h2;
+    asm("{\n\t.reg .b8 b;\n\tcvt.u8.u32 b, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, b;\n\t}" : "=r"(h2) : "r"(byte_in_low));
+    return h2;
+}
+__device__ __forceinline__ uint32_t h2_mul(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+// max(|a|, |b|) per lane; the sign bit is not meaningful (callers drop it).
+__device__ __forceinline__ uint32_t h2_maxabs(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.xorsign.abs.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ void h2_to_f32x2(uint32_t h, float& lo, float& hi) {
+    asm("{\n\t.reg .f16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, h;\n\t}"
+        : "=f"(lo), "=f"(hi) : "r"(h));
+}
+__device__ __forceinline__ void stmatrix_x4_trans(uint32_t addr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1, %2, %3, %4};"
+                 :: "r"(addr), "r"(r0), "r"(r1), "r"(r2), "r"(r3) : "memory");
+}
+__device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
+
+constexpr float kFoldMinScale = 7.888609052210118e-31f;          // 2^-100
+
+template <int kInLayout, int kOutLayout, bool kPerRow>
+__global__ void __launch_bounds__(kTileThreads, 4)
+requant16_tile_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sf,
+                      const float* __restrict__ outer, int64_t rows, int64_t cols, int64_t group_rows, int group_shift,
+                      const int64_t* rows_valid, uint64_t seed, uint64_t stream_id, uint8_t* __restrict__ out_codes,
+                      uint8_t* __restrict__ out_e8m0) {
+    __shared__ __align__(1024) uint16_t T[kTC * kTR];
+    __shared__ __align__(16) float so[kPerRow ? kTR : 4];
+    const int64_t c0 = (int64_t)blockIdx.x * kTC, r0 = (int64_t)blockIdx.y * kTR;
+    if (r0 >= load_rows_valid(rows_valid, rows)) return;
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const uint32_t tbase = smem_u32(T);
+    float s_uni = 0.0f;
+    if (!kPerRow)                     // group_rows is a multiple of 128: one outer scale per tile
+        s_uni = __ldg(outer + (group_shift >= 0 ? (r0 >> group_shift) : (int64_t)((uint32_t)r0 / (uint32_t)group_rows)));
+    // ---------------- phase 1: lane (rho = lane / 4, b = lane % 4): rows 16w + rho and 16w + 8 + rho,
+    // code bytes 8b..8b+7 of the tile row = columns 16b..16b+15 (scale block b of the tile)
+    {
+        const int rho = lane >> 2, b = lane & 3;
+        const int64_t S = cols >> 4;
+        uint32_t pr[2][8];
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+            const int64_t r = r0 + 16 * w + 8 * g + rho;
+            const uint2 cw = __ldcs(reinterpret_cast<const uint2*>(codes + r * (cols >> 1) + (c0 >> 1) + 8 * b));
+            const uint32_t sw = __ldg(reinterpret_cast<const uint32_t*>(sf + sf_offset(r, c0 >> 4, S, kInLayout)));
+            const uint32_t f = h2_of_e4m3((sw >> (8 * b)) & 0xffu);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) pr[g][kk] = h2_mul(h2_of_e2m1((kk < 4 ? cw.x : cw.y) >> (8 * (kk & 3))), f);
+            if (kPerRow && b == 0) so[16 * w + 8 * g + rho] = __ldg(outer + r);
+        }
+        // stmatrix call n: 8-row group g = n / 2 of the warp's rows, column groups kappa = 4 (n % 2) + j for its
+        // matrices j = 0..3.  Thread (rho, b) holds fragment row rho, fragment columns 2b, 2b+1 = tile columns
+        // 16b + 2 kappa + {0, 1}; stored row m of matrix j (address from lane 8j + m) is tile column
+        // 16 (m / 2) + 2 kappa + m % 2, its 8 values the 8 rows of chunk 2w + g.
+        const int j = lane >> 3, m = lane & 7;
+#pragma unroll
+        for (int n = 0; n < 4; ++n) {
+            const int g = n >> 1, kap = 4 * (n & 1) + j;
+            const int c = 16 * (m >> 1) + 2 * kap + (m & 1);
+            const int kb = 4 * (n & 1);
+            stmatrix_x4_trans(tbase + c * 256 + (((2 * w + g) ^ rq_swz(c)) << 4), pr[g][kb], pr[g][kb + 1],
+                              pr[g][kb + 2], pr[g][kb + 3]);
+        }
+    }
+    __syncthreads();
+    // ---------------- phase 2: lane (m = lane % 8, jj = (lane / 8) % 2, q = lane / 16) of warp w: output row
+    // c = 16 (m / 2) + 2w + m % 2 of the tile, input rows 16j..16j+15 with j = 2 (2 it + q) + jj
+    const int m = lane & 7, jj = (lane >> 3) & 1, q = lane >> 4;
+    const int c = 16 * (m >> 1) + 2 * w + (m & 1);
+    const int64_t cg = c0 + c;
+    const int64_t Se = rows >> 5;
+#pragma unroll
+    for (int it = 0; it < 2; ++it) {
+        const int j = 2 * (2 * it + q) + jj;
+        const uint4 v0 = lds_v4(tbase + c * 256 + (((2 * j) ^ rq_swz(c)) << 4));
+        const uint4 v1 = lds_v4(tbase + c * 256 + (((2 * j + 1) ^ rq_swz(c)) << 4));
+        const uint32_t hw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        float y[16];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) h2_to_f32x2(hw[i], y[2 * i], y[2 * i + 1]);
+        int e;
+        if (kPerRow) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float4 s4 = *reinterpret_cast<const float4*>(so + 16 * j + 4 * i);
+                mul2_rn(y[4 * i], y[4 * i + 1], f2_pack(s4.x, s4.y));
+                mul2_rn(y[4 * i + 2], y[4 * i + 3], f2_pack(s4.z, s4.w));
+            }
+            float mf = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) mf = fmaxf(mf, fabsf(y[i]));
+            mf = fmaxf(mf, __shfl_xor_sync(0xffffffffu, mf, 8));
+            e = e8m0_exponent(mf);
+            const float sc = exp2_neg(e);
+            const uint64_t sc2 = f2_pack(sc, sc);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) mul2_rn(y[2 * i], y[2 * i + 1], sc2);
+        } else {
+            const uint32_t hm = h2_maxabs(h2_maxabs(h2_maxabs(hw[0], hw[1]), h2_maxabs(hw[2], hw[3])),
+                                          h2_maxabs(h2_maxabs(hw[4], hw[5]), h2_maxabs(hw[6], hw[7])));
+            float ml, mh;
+            h2_to_f32x2(hm, ml, mh);
+            float pm = fmaxf(fabsf(ml), fabsf(mh));
+            pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, 8));
+            e = e8m0_exponent(__fmul_rn(pm, s_uni));
+            const bool fold = s_uni >= kFoldMinScale;
+            const float s2 = fold ? __fmul_rn(s_uni, exp2_neg(e)) : s_uni;
+            const uint64_t s22 = f2_pack(s2, s2);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) mul2_rn(y[2 * i], y[2 * i + 1], s22);
+            if (!fold) {
+                const float sc = exp2_neg(e);
+                const uint64_t sc2 = f2_pack(sc, sc);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) mul2_rn(y[2 * i], y[2 * i + 1], sc2);
+            }
+        }
+        const int64_t rr = r0 + 16 * j;
+        const int64_t L0 = cg * rows + rr;              // linear index of the first output element
+        uint32_t wo[4];
+#pragma unroll
+        for (int blk = 0; blk < 2; ++blk) {
+            const uint4 rnd = philox4x32_10((uint64_t)(L0 / 8) + blk, stream_id, seed);
+            wo[2 * blk] = cvt_rs16_e4m3_quad(y[8 * blk], y[8 * blk + 1], y[8 * blk + 2], y[8 * blk + 3], rnd.x, rnd.y);
+            wo[2 * blk + 1] = cvt_rs16_e4m3_quad(y[8 * blk + 4], y[8 * blk + 5], y[8 * blk + 6], y[8 * blk + 7], rnd.z,
+                                                 rnd.w);
+        }
+        *reinterpret_cast<uint4*>(out_codes + cg * rows + rr) = make_uint4(wo[0], wo[1], wo[2], wo[3]);
+        if (jj == 0) out_e8m0[sf_offset(cg, rr >> 5, Se, kOutLayout)] = (uint8_t)(e + 127);
+    }
+}
+
 template <typename F>
 int dispatch_layout(int layout, F&& f) {
     if (layout == MX_SF_MMA) return f(std::integral_constant<int, MX_SF_MMA>());
@@ -899,14 +1072,18 @@ extern "C" int mxfp8_requant_transpose_sr(const uint8_t* codes, const uint8_t* s
     int gshift = -1;
     if (group_rows > 1 && (group_rows & (group_rows - 1)) == 0)
         for (gshift = 0; ((int64_t)1 << gshift) < group_rows; ++gshift) {}
+    const bool sf_words = mx_aligned(sf, 4);            // the R = 16 kernel reads a row's 4 scale bytes as a word
     return dispatch_layout(in_sf_layout, [&](auto Li) {
         return dispatch_layout(out_sf_layout, [&](auto Lo) {
             constexpr int kLi = decltype(Li)::value, kLo = decltype(Lo)::value;
             if (rbits == 8)
                 requant_tile_kernel<8, kLi, kLo><<<grid, kTileThreads, 0, stream>>>(
                     codes, sf, outer, rows, cols, group_rows, gshift, rows_valid, seed, stream_id, out_codes, out_e8m0);
-            else if (rbits == 16)
-                requant_tile_kernel<16, kLi, kLo><<<grid, kTileThreads, 0, stream>>>(
+            else if (rbits == 16 && group_rows == 1 && sf_words)
+                requant16_tile_kernel<kLi, kLo, true><<<grid, kTileThreads, 0, stream>>>(
+                    codes, sf, outer, rows, cols, group_rows, gshift, rows_valid, seed, stream_id, out_codes, out_e8m0);
+            else if (rbits == 16 && sf_words)
+                requant16_tile_kernel<kLi, kLo, false><<<grid, kTileThreads, 0, stream>>>(
                     codes, sf, outer, rows, cols, group_rows, gshift, rows_valid, seed, stream_id, out_codes, out_e8m0);
             else
                 requant_tile_kernel<32, kLi, kLo><<<grid, kTileThreads, 0, stream>>>(

@@ -27,6 +27,37 @@ def test_butterflies_equal_the_sylvester_matrix_on_integers():
     assert np.array_equal(oracle.fwht32_f32(x).astype(np.float64), x.astype(np.float64) @ H.T)
 
 
+def _sylvester_recursive_f32(x):
+    """H_n x from the recursion H_2n = [[H_n, H_n], [H_n, -H_n]], each sum one
+    fp32 rounding: H_2n [u; v] = [H_n u + H_n v; H_n u - H_n v]."""
+    n = x.shape[-1]
+    if n == 1:
+        return x.astype(np.float32)
+    u = _sylvester_recursive_f32(x[..., : n // 2])
+    v = _sylvester_recursive_f32(x[..., n // 2:])
+    return np.concatenate([np.float32(u + v), np.float32(u - v)], axis=-1)
+
+
+def test_fp32_order_is_the_sylvester_recursion():
+    """Reading R20 (evaluation order): on general fp32 inputs, where the order
+    of the roundings shows, the butterflies give bit for bit the fp32
+    evaluation of the Sylvester recursion that defines H32, and stay within
+    the five-rounding error bound of the exact product."""
+    rng = np.random.default_rng(11)
+    x = (rng.standard_normal((400, 32)) * 10.0 ** rng.uniform(-3, 3, (400, 1))).astype(np.float32)
+    got = oracle.fwht32_f32(x)
+    assert np.array_equal(got.view(np.uint32), _sylvester_recursive_f32(x).view(np.uint32))
+    exact = x.astype(np.float64) @ _popcount_hadamard(32).T
+    bound = 5 * 2.0 ** -24 * np.abs(x).astype(np.float64).sum(axis=-1, keepdims=True) * 1.0001
+    assert np.all(np.abs(got - exact) <= bound)
+    # a different order (h = 16 first) differs somewhere on these inputs: the pin has teeth
+    z = x.copy()
+    for h in (16, 8, 4, 2, 1):
+        z = z.reshape(400, 32 // (2 * h), 2, h)
+        z = np.stack([z[:, :, 0] + z[:, :, 1], z[:, :, 0] - z[:, :, 1]], axis=2).reshape(400, 32)
+    assert not np.array_equal(z.view(np.uint32), got.view(np.uint32))
+
+
 def test_transform_applied_twice_is_32_times_identity():
     rng = np.random.default_rng(1)
     x = rng.integers(-300, 301, size=(20, 32)).astype(np.float32)

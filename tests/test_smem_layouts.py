@@ -112,3 +112,84 @@ def test_pair_tile_holds_each_row_pair_once():
         for j in range(16):
             seen[t2_word(16 * (t & 1) + j, t >> 1)] += 1
     assert np.all(seen == 1)
+
+
+# ---------------------------------------------------------------------------
+# The R = 16 requantisation's f16 tile (requant16_tile_kernel): f16 [64 cols][128 rows],
+# 256 bytes per column, 16-byte chunks (8 rows) XOR-swizzled by rq_swz(c).
+# ---------------------------------------------------------------------------
+
+def rq_swz(c):
+    return ((c >> 4) & 3) | ((c & 1) << 2)
+
+
+def rq_chunk_addr(c, k):            # byte address of chunk k (rows 8k..8k+7) of column c
+    return c * 256 + ((k ^ rq_swz(c)) << 4)
+
+
+def test_f16_tile_chunks_are_a_bijection():
+    addrs = sorted(rq_chunk_addr(c, k) for c in range(TC) for k in range(TR // 8))
+    assert addrs == list(range(0, TC * TR * 2, 16))
+
+
+def _stmatrix_rows(warp, n):
+    """Stored rows of stmatrix call n of `warp`: for lane 8j + m, (matrix j, tile column, chunk)."""
+    out = []
+    for lane in range(32):
+        j, m = lane >> 3, lane & 7
+        g, kap = n >> 1, 4 * (n & 1) + j
+        out.append((j, 16 * (m >> 1) + 2 * kap + (m & 1), 2 * warp + g))
+    return out
+
+
+def test_f16_tile_stmatrix_writes_every_value_once_in_its_place():
+    # fragment: lane (rho, b) holds, for matrix (g, kappa), tile row 16 warp + 8 g + rho and tile columns
+    # 2 beta, 2 beta + 1 with beta = 8 b + kappa (its code byte); stored row m of the transposed matrix is
+    # fragment column m = 2b + delta, i.e. tile column 16 b + 2 kappa + delta, values = the 8 fragment rows
+    seen = {}
+    for warp in range(8):
+        for n in range(4):
+            g = n >> 1
+            for j, c, k in _stmatrix_rows(warp, n):
+                kap = 4 * (n & 1) + j
+                b, delta = (c - 2 * kap) // 16, (c - 2 * kap) % 16
+                assert delta in (0, 1) and 0 <= b < 4          # column c is in lane b's code bytes
+                assert 2 * (8 * b + kap) + delta == c
+                rows = [16 * warp + 8 * g + rho for rho in range(8)]
+                for i, r in enumerate(rows):
+                    a = rq_chunk_addr(c, k) + 2 * i
+                    assert r // 8 == k and r % 8 == i              # row r sits at position r % 8 of chunk r / 8
+                    assert a not in seen
+                    seen[a] = (c, r)
+    assert len(seen) == TC * TR
+
+
+def test_f16_tile_stmatrix_conflict_free():
+    # each 8x8 matrix is 8 stored rows of 16 bytes; its 8 row addresses must hit 8 distinct bank groups
+    for warp in range(8):
+        for n in range(4):
+            rows = _stmatrix_rows(warp, n)
+            for j in range(4):
+                addrs = [rq_chunk_addr(c, k) for jj, c, k in rows if jj == j]
+                assert len({(a // 16) % 8 for a in addrs}) == 8, (warp, n, j)
+
+
+def test_f16_tile_phase2_loads_conflict_free_and_cover_the_tile():
+    # lane (m = lane % 8, jj = lane / 8 % 2, q = lane / 16) of warp w, pass it: column c = 16 (m / 2) + 2 w + m % 2,
+    # rows 16 j .. 16 j + 15 with j = 2 (2 it + q) + jj, read as chunks 2j and 2j + 1
+    covered = set()
+    for warp in range(8):
+        for it in range(2):
+            for half in range(2):
+                addrs = []
+                for lane in range(32):
+                    m, jj, q = lane & 7, (lane >> 3) & 1, lane >> 4
+                    c = 16 * (m >> 1) + 2 * warp + (m & 1)
+                    j = 2 * (2 * it + q) + jj
+                    addrs.append(rq_chunk_addr(c, 2 * j + half))
+                    covered.add((c, 2 * j + half))
+                    # the 32-row E8M0 block of this lane is completed by lane ^ 8
+                    m2, jj2, q2 = (lane ^ 8) & 7, ((lane ^ 8) >> 3) & 1, (lane ^ 8) >> 4
+                    assert (m2, q2) == (m, q) and jj2 != jj
+                assert _quads_conflict_free(addrs), (warp, it, half)
+    assert len(covered) == TC * TR // 8
