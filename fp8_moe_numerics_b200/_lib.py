@@ -9,7 +9,8 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libmxmoe.so")
+# MX_DEBUG=1 loads the bounds-checked build (python -m fp8_moe_numerics_b200.build --debug-bounds)
+LIB_PATH = os.path.join(_HERE, "libmxmoe_debug.so" if os.environ.get("MX_DEBUG") == "1" else "libmxmoe.so")
 
 MX_OK, MX_EINVAL, MX_ECUDA, MX_ETIMEOUT, MX_EUNSUPPORTED, MX_EDATA = 0, 1, 2, 3, 4, 5
 MX_SF_ROWMAJOR, MX_SF_MMA = 0, 1
@@ -33,6 +34,8 @@ SIGNATURES = {
     "mx_sync_status": (I32, [P]),
     "mx_wait_selftest": (I32, [I64, P]),
     "mx_sf_bytes": (SZ, [I64, I64, I32, I32]),
+    "mx_debug_bounds_build": (I32, []),
+    "mx_debug_bounds_violations": (ctypes.c_ulonglong, [I32]),
     "nvfp4_quantize": (I32, [P, I64, I64, I64, P, P, P, I32, P]),
     "mxfp8_requant_transpose_sr": (I32, [P, P, P, I64, I64, I64, I32, P, U64, U64, I32, P, P, I32, P]),
     "mxfp8_quantize": (I32, [P, I64, I64, I32, U64, U64, I32, P, P, P, P, P, I32, P]),
@@ -78,7 +81,8 @@ def lib() -> ctypes.CDLL:
     global _lib
     if _lib is None:
         if not os.path.exists(LIB_PATH):
-            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m fp8_moe_numerics_b200.build` "
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m fp8_moe_numerics_b200.build`"
+                               f"{' --debug-bounds' if LIB_PATH.endswith('_debug.so') else ''} "
                                "(there is no non-CUDA implementation of this library)")
         L = ctypes.CDLL(LIB_PATH)
         for name, (res, args) in SIGNATURES.items():

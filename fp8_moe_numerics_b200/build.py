@@ -1,11 +1,13 @@
 """Build libmxmoe.so (the C-ABI CUDA library) in-tree for sm_100a.
 
-    python -m fp8_moe_numerics_b200.build [--force] [--verbose]
+    python -m fp8_moe_numerics_b200.build [--force] [--verbose] [--debug-bounds]
 
 Each csrc/*.cu is compiled separately with nvcc
 (-gencode arch=compute_100a,code=sm_100a, -O3, -lineinfo, no fast-math) and
 linked into fp8_moe_numerics_b200/libmxmoe.so with the CUDA runtime linked
-statically.  Objects go to fp8_moe_numerics_b200/_build/.
+statically.  Objects go to fp8_moe_numerics_b200/_build/.  --debug-bounds
+builds the bounds-checked variant (-DMX_DEBUG_BOUNDS) as libmxmoe_debug.so
+from objects in _build_debug/; the package loads it when MX_DEBUG=1.
 """
 from __future__ import annotations
 
@@ -21,6 +23,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libmxmoe.so")
+BUILD_DEBUG = os.path.join(PKG, "_build_debug")
+LIB_DEBUG = os.path.join(PKG, "libmxmoe_debug.so")
 INCLUDE = os.path.join(os.path.dirname(PKG), "include")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -50,8 +54,8 @@ def _stale(target: str, deps) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def _compile(src: str, verbose: bool, extra) -> str:
-    obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+def _compile(src: str, verbose: bool, extra, build_dir: str = BUILD) -> str:
+    obj = os.path.join(build_dir, os.path.basename(src)[:-3] + ".o")
     if _stale(obj, [src, *_headers(), __file__]):
         cmd = [nvcc(), *ARCH, *NVCC_FLAGS, *extra, "-I", INCLUDE, "-c", src, "-o", obj]
         if verbose:
@@ -64,24 +68,26 @@ def _compile(src: str, verbose: bool, extra) -> str:
     return obj
 
 
-def build(force: bool = False, verbose: bool = False, extra=()) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, extra=(), debug_bounds: bool = False) -> str:
+    build_dir, lib_path = (BUILD_DEBUG, LIB_DEBUG) if debug_bounds else (BUILD, LIB)
+    extra = list(extra) + (["-DMX_DEBUG_BOUNDS"] if debug_bounds else [])
+    os.makedirs(build_dir, exist_ok=True)
     if force:
-        for o in glob.glob(os.path.join(BUILD, "*.o")):
+        for o in glob.glob(os.path.join(build_dir, "*.o")):
             os.remove(o)
     srcs = _sources()
     with cf.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
-        objs = list(ex.map(lambda s: _compile(s, verbose, list(extra)), srcs))
-    if force or _stale(LIB, objs):
-        tmp = LIB + f".tmp{os.getpid()}"
+        objs = list(ex.map(lambda s: _compile(s, verbose, extra, build_dir), srcs))
+    if force or _stale(lib_path, objs):
+        tmp = lib_path + f".tmp{os.getpid()}"
         cmd = [nvcc(), *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs]
         if verbose:
             print(" ".join(cmd), flush=True)
         res = subprocess.run(cmd, capture_output=True, text=True)
         if res.returncode != 0:
             raise RuntimeError(f"link failed:\n{res.stdout}\n{res.stderr}")
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib_path)
+    return lib_path
 
 
 def main(argv=None) -> int:
@@ -89,9 +95,11 @@ def main(argv=None) -> int:
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
     ap.add_argument("--ptxas-info", action="store_true", help="print registers / spills per kernel")
+    ap.add_argument("--debug-bounds", action="store_true", help="build the bounds-checked libmxmoe_debug.so")
     a = ap.parse_args(argv)
     extra = ["-Xptxas", "-v"] if a.ptxas_info else []
-    print(build(force=a.force or a.ptxas_info, verbose=a.verbose or a.ptxas_info, extra=extra))
+    print(build(force=a.force or a.ptxas_info, verbose=a.verbose or a.ptxas_info, extra=extra,
+                debug_bounds=a.debug_bounds))
     return 0
 
 

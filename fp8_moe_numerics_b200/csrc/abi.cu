@@ -68,3 +68,19 @@ extern "C" size_t mx_route_workspace_bytes(int64_t T, int64_t E) {
     if (chunks > (INT64_MAX / (int64_t)sizeof(int32_t) - E) / E) return SIZE_MAX;   // would overflow int64
     return (size_t)((chunks * E + E) * sizeof(int32_t));
 }
+
+MX_BOUNDS_READER(mx_bounds_word_abi)
+
+extern "C" int mx_debug_bounds_build(void) {
+#ifdef MX_DEBUG_BOUNDS
+    return 1;
+#else
+    return 0;
+#endif
+}
+
+extern "C" unsigned long long mx_debug_bounds_violations(int clear) {
+    const bool c = clear != 0;
+    return (unsigned long long)mx_bounds_word_abi(c) + mx_bounds_word_quant(c) + mx_bounds_word_glue(c) +
+           mx_bounds_word_gemm(c) + mx_bounds_word_s2f6(c) + mx_bounds_word_nvfp4_bwd(c);
+}

@@ -56,6 +56,7 @@ struct GemmArgs {
     int64_t ldo;              // output row stride (elements)
     uint8_t* e8m0_out;        // S2F6 output: one exponent per 32 outputs of a row
     uint64_t seed, stream_id; // S2F6 output: key and stream of the rotation's signs
+    int64_t sfa_atoms, sfb_atoms, a_outer_n;   // extents of the scale arrays (512-byte atoms) and of a_outer
 };
 
 // ---------------------------------------------------------------------------
@@ -530,11 +531,17 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                         tma_load_2d(sa, &tmA, &full[stage], kx, (int)t.a_y);
                         tma_load_2d(sb, &tmB, &full[stage], (int)t.b_x0 + kx, (int)t.b_y);
                     }
-                    bulk_load(ssfa, p.sfa + (t.sfa_atom0 + kt * L::kAtomsA) * 512, L::kSfa, sf_bar);
+                    // (in the bounds-checked build an atom range past its array is read from atom 0
+                    // instead, so that the barrier still completes; the violation is counted)
+                    const int64_t fa = t.sfa_atom0 + kt * L::kAtomsA;
+                    bulk_load(ssfa, p.sfa + (mx_in_range(fa, L::kAtomsA, p.sfa_atoms) ? fa : 0) * 512, L::kSfa, sf_bar);
 #pragma unroll
-                    for (int h = 0; h < kBN / 128; ++h)
-                        bulk_load(ssfb + h * L::kAtomsA * 512, p.sfb + (t.sfb_atom0 + h * p.sfb_groups + kt * L::kAtomsA) * 512,
-                                  L::kAtomsA * 512, sf_bar);
+                    for (int h = 0; h < kBN / 128; ++h) {
+                        const int64_t fb = t.sfb_atom0 + h * p.sfb_groups + kt * L::kAtomsA;
+                        bulk_load(ssfb + h * L::kAtomsA * 512,
+                                  p.sfb + (mx_in_range(fb, L::kAtomsA, p.sfb_atoms) ? fb : 0) * 512, L::kAtomsA * 512,
+                                  sf_bar);
+                    }
                     issued[stage] = true;
                     issued_phase[stage] = phase;
                     if (++stage == kStages) { stage = 0; phase ^= 1u; }
@@ -700,7 +707,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         // NVFP4: each tile's outer scales (a per-row and a per-expert fp32) are
         // loaded one tile ahead, so their latency overlaps the previous drain.
         auto tile_scale = [&](const Tile& tt) -> float {
-            return (kKind == kKindNVFP4 && tt.store) ? __ldg(p.a_outer + tt.row0 + r) * __ldg(p.b_outer + tt.e) : 1.0f;
+            return (kKind == kKindNVFP4 && tt.store && mx_in_range(tt.row0 + r, 1, p.a_outer_n))
+                       ? __ldg(p.a_outer + tt.row0 + r) * __ldg(p.b_outer + tt.e) : 1.0f;
         };
         Tile t_next = make_tile<kKind, kMode, kBN, kPair>(p, first, rank, pfx);
         float scale_next = tile_scale(t_next);
@@ -1094,6 +1102,7 @@ extern "C" int grouped_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_sf, c
     a.sfa = a_sf; a.sfb = b_sf; a.a_outer = a_outer; a.b_outer = b_outer; a.seg = seg_offsets; a.out = out;
     a.E = E; a.M_cap = M_cap; a.N = N; a.K = K;
     a.sfa_groups = K / 64; a.sfb_groups = K / 64; a.ldo = N;
+    a.sfa_atoms = M_cap / 128 * a.sfa_groups; a.sfb_atoms = E * N / 128 * a.sfb_groups; a.a_outer_n = M_cap;
     return dispatch<kKindNVFP4, kModeRows>(N % 256 == 0 && E <= kMaxPairExperts, M_cap, N, out_dtype, ma, mb, a, (M_cap / kBM) * (N / 256),
                                            (M_cap / kBM) * (N / 128), stream);
 }
@@ -1120,6 +1129,7 @@ extern "C" int grouped_gemm_nvfp4_s2f6(const uint8_t* a_codes, const uint8_t* a_
     a.sfa = a_sf; a.sfb = b_sf; a.a_outer = a_outer; a.b_outer = b_outer; a.seg = seg_offsets; a.out = codes;
     a.E = E; a.M_cap = M_cap; a.N = N; a.K = K;
     a.sfa_groups = K / 64; a.sfb_groups = K / 64; a.ldo = N;
+    a.sfa_atoms = M_cap / 128 * a.sfa_groups; a.sfb_atoms = E * N / 128 * a.sfb_groups; a.a_outer_n = M_cap;
     a.e8m0_out = e8m0; a.seed = seed; a.stream_id = stream_id;
     return dispatch<kKindNVFP4, kModeRows>(N % 256 == 0 && E <= kMaxPairExperts, M_cap, N, kOutS2F6Dtype, ma, mb, a,
                                            (M_cap / kBM) * (N / 256), (M_cap / kBM) * (N / 128), stream);
@@ -1154,6 +1164,7 @@ extern "C" int grouped_gemm_mxfp8(int mode, const uint8_t* a_codes, const uint8_
         if (int st = make_map(&ma, a_codes, M_cap, K, kBM)) return st;
         if (int st = make_map(&mb, b_codes, N, E * K, 128)) return st;
         a.sfa_groups = K / 128; a.sfb_groups = E * K / 128; a.ldo = N;
+        a.sfa_atoms = M_cap / 128 * a.sfa_groups; a.sfb_atoms = N / 128 * a.sfb_groups; a.a_outer_n = M_cap;
         return dispatch<kKindMXFP8, kModeRows>(N % 256 == 0 && E <= kMaxPairExperts, M_cap, N, out_dtype, ma, mb, a,
                                                (M_cap / kBM) * (N / 256), (M_cap / kBM) * (N / 128), stream);
     }
@@ -1161,6 +1172,7 @@ extern "C" int grouped_gemm_mxfp8(int mode, const uint8_t* a_codes, const uint8_
     if (int st = make_map(&ma, a_codes, N, M_cap, kBM)) return st;
     if (int st = make_map(&mb, b_codes, K, M_cap, 128)) return st;
     a.sfa_groups = M_cap / 128; a.sfb_groups = M_cap / 128; a.ldo = K;
+    a.sfa_atoms = N / 128 * a.sfa_groups; a.sfb_atoms = K / 128 * a.sfb_groups; a.a_outer_n = E * N;
     const bool pair = N % 256 == 0 && K % 256 == 0;
     return dispatch<kKindMXFP8, kModeWgrad>(pair, E * N, K, out_dtype, ma, mb, a, E * (N / 256) * (K / 256),
                                             E * (N / 128) * (K / 128), stream);
@@ -1198,7 +1210,10 @@ extern "C" int grouped_gemm_nvfp4_wgrad(const uint8_t* a_codes, const uint8_t* a
     a.sfa = a_sf; a.sfb = b_sf; a.a_outer = a_outer; a.b_outer = b_outer; a.seg = seg_offsets; a.out = out;
     a.E = E; a.M_cap = M_cap; a.N = N; a.K = K;
     a.sfa_groups = M_cap / 64; a.sfb_groups = M_cap / 64; a.ldo = K;
+    a.sfa_atoms = N / 128 * a.sfa_groups; a.sfb_atoms = K / 128 * a.sfb_groups; a.a_outer_n = E * N;
     const bool pair = N % 256 == 0 && K % 256 == 0;
     return dispatch<kKindNVFP4, kModeWgrad>(pair, E * N, K, out_dtype, ma, mb, a, E * (N / 256) * (K / 256),
                                             E * (N / 128) * (K / 128), stream);
 }
+
+MX_BOUNDS_READER(mx_bounds_word_gemm)

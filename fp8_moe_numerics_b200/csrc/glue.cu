@@ -39,7 +39,8 @@ __global__ void route_count_kernel(const int32_t* __restrict__ topk, int64_t T, 
             else atomicOr(status, kStatusBadRoute);
         }
     __syncthreads();
-    for (int64_t e = threadIdx.x; e < E; e += blockDim.x) hist[(int64_t)blockIdx.x * E + e] = h[e];
+    for (int64_t e = threadIdx.x; e < E; e += blockDim.x)
+        if (mx_in_range((int64_t)blockIdx.x * E + e, 1, (int64_t)gridDim.x * E)) hist[(int64_t)blockIdx.x * E + e] = h[e];
 }
 
 // Totals, kAlign-padded exclusive scan into seg_offsets, and per-(chunk,
@@ -75,7 +76,7 @@ __global__ void route_scan_kernel(int32_t* __restrict__ hist, int32_t* __restric
 // tokens a shared bitmask per expert marks the lanes that chose it; a lane's
 // rank is the number of lower lanes in that mask.
 __global__ void route_scatter_kernel(const int32_t* __restrict__ topk, int64_t T, int64_t k, int64_t E,
-                                     const int32_t* __restrict__ base, int32_t* __restrict__ src,
+                                     int64_t M_cap, const int32_t* __restrict__ base, int32_t* __restrict__ src,
                                      int32_t* __restrict__ pos) {
     extern __shared__ uint32_t sm[];
     uint32_t* mask = sm;                                   // [E]
@@ -101,7 +102,7 @@ __global__ void route_scatter_kernel(const int32_t* __restrict__ topk, int64_t T
                 const int32_t e = topk[t * k + j];
                 const int32_t p = run[e] + __popc(mask[e] & below);
                 pos[t * k + j] = p;
-                src[p] = (int32_t)(t * k + j);
+                if (mx_in_range(p, 1, M_cap)) src[p] = (int32_t)(t * k + j);
             }
         __syncwarp();
         if (act)
@@ -122,7 +123,8 @@ __global__ void route_pad_kernel(const int64_t* __restrict__ seg, const int32_t*
     int64_t a, b;
     if (e < E) { a = seg[e] + counts[e]; b = seg[e + 1]; }
     else { a = seg[E]; b = M_cap; }
-    for (int64_t p = a + threadIdx.x; p < b; p += blockDim.x) src[p] = -1;
+    for (int64_t p = a + threadIdx.x; p < b; p += blockDim.x)
+        if (mx_in_range(p, 1, M_cap)) src[p] = -1;
 }
 
 // One warp per output row.
@@ -257,7 +259,7 @@ dispatch_grad_kernel(const uint16_t* __restrict__ dout, const int32_t* __restric
         for (int64_t c = threadIdx.x * 8; c < D; c += kDispatchThreads * 8) {
             const uint4 v = __ldcs(reinterpret_cast<const uint4*>(dout + b * D + c));
             for (int64_t j = 0; j < k; ++j) {
-                if (sp[j] < 0) continue;                   // entry left out by the routing
+                if (sp[j] < 0 || !mx_in_range((int64_t)sp[j] * D + c, 8, M_cap * D)) continue;   // left out
                 const float wj = sw[j];
                 const uint4 o = make_uint4(pack_bf16x2(wj * bf16_lo(v.x), wj * bf16_hi(v.x)),
                                            pack_bf16x2(wj * bf16_lo(v.y), wj * bf16_hi(v.y)),
@@ -301,7 +303,8 @@ int route_launch(const int32_t* topk, int64_t T, int64_t k, int64_t E, int64_t M
     mx_count_launch();
     if (int st = mx_launch_status()) return st;
     if (nchunks > 0) {
-        route_scatter_kernel<<<(unsigned)nchunks, 32, 2 * E * sizeof(uint32_t), stream>>>(topk, T, k, E, hist, src, pos);
+        route_scatter_kernel<<<(unsigned)nchunks, 32, 2 * E * sizeof(uint32_t), stream>>>(topk, T, k, E, M_cap, hist,
+                                                                                          src, pos);
         mx_count_launch();
         if (int st = mx_launch_status()) return st;
     }
@@ -531,3 +534,5 @@ extern "C" int moe_route_static(const int32_t* topk, int64_t T, int64_t k, int64
     if (int st = route_scratch_address(&scratch)) return st;
     return moe_route(topk, T, k, E, M_cap, seg_offsets, src, pos, scratch, kRouteStaticScratchBytes, stream);
 }
+
+MX_BOUNDS_READER(mx_bounds_word_glue)

@@ -47,6 +47,44 @@ int mx_make_bf16_tile_map(struct CUtensorMap_st* m, const void* base, int64_t ro
 static inline bool mx_aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 // ---------------------------------------------------------------------------
+// Bounds-checked build.  Compiled with -DMX_DEBUG_BOUNDS (libmxmoe_debug.so,
+// `python -m fp8_moe_numerics_b200.build --debug-bounds`), the kernels check
+// the global indices they compute against the extent of the buffer the call's
+// arguments give it: an access out of range is skipped and counted in a
+// device word of its translation unit, which mx_debug_bounds_violations()
+// reads and clears.  This replaces a memory checker that cannot run here.  In
+// the normal build mx_in_range() is the constant true and the checks compile
+// away.
+// ---------------------------------------------------------------------------
+#ifdef MX_DEBUG_BOUNDS
+static __device__ unsigned int g_mx_bounds_word;           // one per translation unit
+// [first, first + count) inside [0, extent)?  Counts a violation when not.
+__device__ __forceinline__ bool mx_in_range(int64_t first, int64_t count, int64_t extent) {
+    if (first >= 0 && count >= 0 && first + count <= extent) return true;
+    atomicAdd(&g_mx_bounds_word, 1u);
+    return false;
+}
+#define MX_BOUNDS_READER(name)                                                              \
+    unsigned int name(bool clear) {                                                         \
+        unsigned int v = 0, zero = 0;                                                       \
+        if (cudaMemcpyFromSymbol(&v, g_mx_bounds_word, sizeof(v)) != cudaSuccess) return 0; \
+        if (clear && v) cudaMemcpyToSymbol(g_mx_bounds_word, &zero, sizeof(zero));          \
+        return v;                                                                           \
+    }
+#else
+__device__ __forceinline__ constexpr bool mx_in_range(int64_t, int64_t, int64_t) { return true; }
+#define MX_BOUNDS_READER(name) \
+    unsigned int name(bool) { return 0u; }
+#endif
+// Per translation unit readers of the bounds word (defined in each .cu).
+unsigned int mx_bounds_word_abi(bool clear);
+unsigned int mx_bounds_word_quant(bool clear);
+unsigned int mx_bounds_word_glue(bool clear);
+unsigned int mx_bounds_word_gemm(bool clear);
+unsigned int mx_bounds_word_s2f6(bool clear);
+unsigned int mx_bounds_word_nvfp4_bwd(bool clear);
+
+// ---------------------------------------------------------------------------
 // Shared-memory addresses, mbarriers and the GPU clock
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

@@ -155,12 +155,16 @@ nvfp4_quantize_sr_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t c
 // Dequantised NVFP4 element (r, c): (q * sf) * outer[r / group_rows], one
 // fp32 rounding after the exact block product.
 __device__ __forceinline__ float nvfp4_value(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sf,
-                                             const float* __restrict__ outer, int64_t cols, int64_t group_rows,
-                                             int in_layout, int64_t r, int64_t c) {
-    const uint32_t byte = __ldg(codes + (r * cols + c) / 2);
+                                             const float* __restrict__ outer, int64_t rows, int64_t cols,
+                                             int64_t group_rows, int in_layout, int64_t r, int64_t c) {
+    const int64_t ci = (r * cols + c) / 2, si = sf_offset(r, c / 16, cols / 16, in_layout);
+    if (!mx_in_range(ci, 1, rows * cols / 2) || !mx_in_range(si, 1, rows * (cols / 16)) ||
+        !mx_in_range(r / group_rows, 1, rows / group_rows))
+        return 0.0f;
+    const uint32_t byte = __ldg(codes + ci);
     const uint32_t q = (c & 1) ? (byte >> 4) : (byte & 15u);
     const float qv = (q & 8) ? -e2m1_mag(q & 7) : e2m1_mag(q & 7);
-    const float bp = __fmul_rn(qv, e4m3_to_f32(__ldg(sf + sf_offset(r, c / 16, cols / 16, in_layout))));
+    const float bp = __fmul_rn(qv, e4m3_to_f32(__ldg(sf + si)));
     return __fmul_rn(bp, __ldg(outer + r / group_rows));
 }
 
@@ -180,7 +184,7 @@ requant_amax_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict
     const int64_t c = c0 + cl;
     float m = 0.0f;
     for (int i = 0; i < 32; ++i)
-        m = fmaxf(m, fabsf(nvfp4_value(codes, sf, outer, cols, group_rows, in_layout, r0 + rg * 32 + i, c)));
+        m = fmaxf(m, fabsf(nvfp4_value(codes, sf, outer, rows, cols, group_rows, in_layout, r0 + rg * 32 + i, c)));
     part[rg][cl] = m;
     __syncthreads();
     const int64_t e = r0 / rows_per_expert;
@@ -223,13 +227,14 @@ requant_nvfp4_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restric
     float v[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i)
-        v[i] = nvfp4_value(codes, sf, outer, cols, group_rows, in_layout, e * rows_per_expert + b * 16 + i, c);
+        v[i] = nvfp4_value(codes, sf, outer, rows, cols, group_rows, in_layout, e * rows_per_expert + b * 16 + i, c);
     uint32_t scode;
     uint2 packed;
     const float s = __ldg(out_outer + (per_expert ? e : o));
     quantize_block16<R, kSR>(v, s, seed, stream_id, (uint64_t)(o * rows_per_expert + b * 16), scode, packed);
-    *reinterpret_cast<uint2*>(out_codes + (o * rows_per_expert + b * 16) / 2) = packed;
-    out_sf[sf_offset(o, b, nb, out_layout)] = (uint8_t)scode;
+    if (mx_in_range((o * rows_per_expert + b * 16) / 2, 8, rows * cols / 2))
+        *reinterpret_cast<uint2*>(out_codes + (o * rows_per_expert + b * 16) / 2) = packed;
+    if (mx_in_range(sf_offset(o, b, nb, out_layout), 1, rows * cols / 16)) out_sf[sf_offset(o, b, nb, out_layout)] = (uint8_t)scode;
 }
 
 // 16x16 tiles: one warp per tile, lane l takes row l / 2 of the tile and its
@@ -286,10 +291,10 @@ struct Nvfp4Src {
     const uint8_t* codes;
     const uint8_t* sf;
     const float* outer;
-    int64_t C, group_rows;
+    int64_t M, C, group_rows;
     int layout;
     __device__ __forceinline__ float operator()(int64_t t, int64_t c) const {
-        return nvfp4_value(codes, sf, outer, C, group_rows, layout, t, c);
+        return nvfp4_value(codes, sf, outer, M, C, group_rows, layout, t, c);
     }
 };
 
@@ -352,8 +357,8 @@ segment_quantize_kernel(Src src, const int64_t* __restrict__ seg, int64_t E, int
         const float s = __ldg(out_outer + (per_row ? lo * C + c : lo));
         quantize_block16<R, kSR>(v, s, seed, stream_id, (uint64_t)(c * M + t0), scode, packed);
     }
-    *reinterpret_cast<uint2*>(out_codes + (c * M + t0) / 2) = packed;
-    out_sf[sf_offset(c, b, nb, out_layout)] = (uint8_t)scode;
+    if (mx_in_range((c * M + t0) / 2, 8, C * M / 2)) *reinterpret_cast<uint2*>(out_codes + (c * M + t0) / 2) = packed;
+    if (mx_in_range(sf_offset(c, b, nb, out_layout), 1, C * M / 16)) out_sf[sf_offset(c, b, nb, out_layout)] = (uint8_t)scode;
 }
 
 template <bool kSR, typename F>
@@ -538,6 +543,8 @@ extern "C" int nvfp4_requant_transpose_segments(const uint8_t* codes, const uint
         return st;
     if (int st = mx_check_device()) return st;
     if (M == 0) return MX_OK;
-    return segments_common(Nvfp4Src{codes, sf, outer, C, group_rows, in_sf_layout}, M, C, seg, E, per_row, rounding,
+    return segments_common(Nvfp4Src{codes, sf, outer, M, C, group_rows, in_sf_layout}, M, C, seg, E, per_row, rounding,
                            seed, stream_id, rbits, out_codes, out_sf, out_outer, out_sf_layout, stream);
 }
+
+MX_BOUNDS_READER(mx_bounds_word_nvfp4_bwd)

@@ -677,64 +677,26 @@ mxfp8_tile_tma_kernel(const __grid_constant__ CUtensorMap tmX, int64_t rows, int
     }
 }
 
-// NVFP4 [rows, cols] -> dequantise -> transpose -> MXFP8 with SR.
-template <int kR, int kInLayout, int kOutLayout>
-__global__ void __launch_bounds__(kTileThreads, 4)
-requant_tile_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sf, const float* __restrict__ outer,
-                    int64_t rows, int64_t cols, int64_t group_rows, int group_shift, const int64_t* rows_valid,
-                    uint64_t seed, uint64_t stream_id, uint8_t* __restrict__ out_codes, uint8_t* __restrict__ out_e8m0) {
-    __shared__ __align__(16) float T[kTC * kTR];
-    const int64_t c0 = (int64_t)blockIdx.x * kTC, r0 = (int64_t)blockIdx.y * kTR;
-    if (r0 >= load_rows_valid(rows_valid, rows)) return;
-    const int t = threadIdx.x;
-    const int rl = t >> 1, h = t & 1;
-    const int64_t r = r0 + rl;
-    const uint4 q = __ldcs(reinterpret_cast<const uint4*>(codes + r * (cols >> 1) + (c0 >> 1) + 16 * h));
-    const int64_t S = cols >> 4;
-    const int64_t s0 = (c0 >> 4) + 2 * h;
-    const uint32_t sc0 = sf[sf_offset(r, s0, S, kInLayout)];
-    const uint32_t sc1 = sf[sf_offset(r, s0 + 1, S, kInLayout)];
-    // group_rows is 1 or a multiple of 128, so a tile's rows share one group
-    const int64_t gi = group_rows == 1 ? r
-                     : (group_shift >= 0 ? (r0 >> group_shift) : (int64_t)((uint32_t)r0 / (uint32_t)group_rows));
-    const float so = outer[gi];
-    const __half2 f0 = __half2half2(e4m3_to_h(sc0)), f1 = __half2half2(e4m3_to_h(sc1));
-    const uint64_t so2 = f2_pack(so, so);
-    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-    __half2 hv[16];                                    // hv[i]: elements 2i, 2i+1
-#pragma unroll
-    for (int j = 0; j < 4; ++j) e2m1x8_to_h2x4(w[j], hv + 4 * j);
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const float2 pf = __half22float2(__hmul2(hv[i], i < 8 ? f0 : f1));   // exact products
-        float a = pf.x, b = pf.y;
-        mul2_rn(a, b, so2);
-        T[tsw(32 * h + 2 * i, rl)] = a;
-        T[tsw(32 * h + 2 * i + 1, rl)] = b;
-    }
-    __syncthreads();
-    tile_emit_transposed<true, kR, kOutLayout>(T, rows, cols, r0, c0, seed, stream_id, out_codes, out_e8m0);
-}
-
 // ---------------------------------------------------------------------------
-// The R = 16 requantisation (the hardware stochastic rounding, the layer's
-// default): a 128 x 64 input tile per block, as in requant_tile_kernel, with
-// the work per element cut down.
+// NVFP4 [rows, cols] -> dequantise -> transpose -> MXFP8 with stochastic
+// rounding: one 128 x 64 input tile per block, 256 threads.
 //   Phase 1: each thread decodes 2 rows x 16 columns (one scale block per
 //   row) to the exact f16 products q*sf (cvt e2m1x2 -> f16x2, one f16x2
-//   multiply per pair) and the warp stores its 16 x 64 products transposed
-//   with four stmatrix.trans (8 x 8 blocks of 16-bit values, 8 values per
-//   thread each).  The tile lives in shared memory as f16 [64 cols][128 rows],
-//   16-byte chunks XOR-swizzled by swz() so that both phases are free of bank
-//   conflicts.
+//   multiply per pair; |q sf| <= 2688 and >= 2^-10 when nonzero, so f16 holds
+//   it exactly) and the warp stores its 16 x 64 products transposed with four
+//   stmatrix.trans (8 x 8 blocks of 16-bit values).  The tile lives in shared
+//   memory as f16 [64 cols][128 rows], 16-byte chunks XOR-swizzled by
+//   rq_swz() so that both phases are free of bank conflicts.
 //   Phase 2: each thread takes 16 consecutive rows of one output row, twice:
-//   two 16-byte loads, f16 -> fp32, the outer scale, the 32-row amax (the
-//   block's other half is in lane ^ 8), the E8M0 exponent, y = x * 2^-e and
-//   cvt.rs.  With one outer scale for the whole tile (expert weights) the amax
-//   is taken on the f16 products (s > 0 is monotone) and the two products
-//   fold into one: RN(RN(p s) 2^-e) = RN(p (s 2^-e)) whenever p s stays in
-//   fp32's normal range, which s >= 2^-100 guarantees (|p| >= 2^-10); smaller
-//   s takes the two products.
+//   two 16-byte loads, f16 -> fp32, the outer scale (x = RN(p s)), the
+//   32-row amax (the block's other half is in lane ^ 8), the E8M0 exponent e,
+//   y = x 2^-e, and the rounding: R = 16 and R = 8 by cvt.rs (two values per
+//   instruction), R = 32 by exact integer arithmetic on y.  With one
+//   outer scale for the whole tile (expert weights) the amax is taken on the
+//   f16 products (s > 0 is monotone) and the two products fold into one:
+//   RN(RN(p s) 2^-e) = RN(p (s 2^-e)) whenever p s stays in fp32's normal
+//   range, which s >= 2^-100 guarantees (|p| >= 2^-10); smaller s takes the
+//   two products.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ int rq_swz(int c) { return ((c >> 4) & 3) | ((c & 1) << 2); }
 
@@ -774,14 +736,25 @@ __device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
     return v;
 }
 
+// cvt.rs on four values with their 16-bit random fields given as cvt.rs takes
+// them (y0 in bits 15:0 of f01, y1 in bits 31:16, likewise y2, y3 in f23);
+// codes packed y0 | y1 << 8 | y2 << 16 | y3 << 24.
+__device__ __forceinline__ uint32_t cvt_rs_quad_fields(float y0, float y1, float y2, float y3, uint32_t f01,
+                                                       uint32_t f23) {
+    uint32_t d0, d1;
+    asm("cvt.rs.satfinite.e4m3x4.f32 %0, {%1, %2, %3, %4}, %5;" : "=r"(d0) : "f"(0.0f), "f"(y1), "f"(0.0f), "f"(y0), "r"(f01));
+    asm("cvt.rs.satfinite.e4m3x4.f32 %0, {%1, %2, %3, %4}, %5;" : "=r"(d1) : "f"(0.0f), "f"(y3), "f"(0.0f), "f"(y2), "r"(f23));
+    return __byte_perm(d0, d1, 0x6420);
+}
+
 constexpr float kFoldMinScale = 7.888609052210118e-31f;          // 2^-100
 
-template <int kInLayout, int kOutLayout, bool kPerRow>
+template <int kR, int kInLayout, int kOutLayout, bool kPerRow>
 __global__ void __launch_bounds__(kTileThreads, 4)
-requant16_tile_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sf,
-                      const float* __restrict__ outer, int64_t rows, int64_t cols, int64_t group_rows, int group_shift,
-                      const int64_t* rows_valid, uint64_t seed, uint64_t stream_id, uint8_t* __restrict__ out_codes,
-                      uint8_t* __restrict__ out_e8m0) {
+requant_tile_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sf, bool sf_words, bool e8_words,
+                    const float* __restrict__ outer, int64_t rows, int64_t cols, int64_t group_rows, int group_shift,
+                    const int64_t* rows_valid, uint64_t seed, uint64_t stream_id, uint8_t* __restrict__ out_codes,
+                    uint8_t* __restrict__ out_e8m0) {
     __shared__ __align__(1024) uint16_t T[kTC * kTR];
     __shared__ __align__(16) float so[kPerRow ? kTR : 4];
     const int64_t c0 = (int64_t)blockIdx.x * kTC, r0 = (int64_t)blockIdx.y * kTR;
@@ -789,8 +762,10 @@ requant16_tile_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restri
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     const uint32_t tbase = smem_u32(T);
     float s_uni = 0.0f;
-    if (!kPerRow)                     // group_rows is a multiple of 128: one outer scale per tile
-        s_uni = __ldg(outer + (group_shift >= 0 ? (r0 >> group_shift) : (int64_t)((uint32_t)r0 / (uint32_t)group_rows)));
+    if (!kPerRow) {                   // group_rows is a multiple of 128: one outer scale per tile
+        const int64_t gi = group_shift >= 0 ? (r0 >> group_shift) : (int64_t)((uint32_t)r0 / (uint32_t)group_rows);
+        if (mx_in_range(gi, 1, rows / group_rows)) s_uni = __ldg(outer + gi);
+    }
     // ---------------- phase 1: lane (rho = lane / 4, b = lane % 4): rows 16w + rho and 16w + 8 + rho,
     // code bytes 8b..8b+7 of the tile row = columns 16b..16b+15 (scale block b of the tile)
     {
@@ -800,12 +775,21 @@ requant16_tile_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restri
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
             const int64_t r = r0 + 16 * w + 8 * g + rho;
-            const uint2 cw = __ldcs(reinterpret_cast<const uint2*>(codes + r * (cols >> 1) + (c0 >> 1) + 8 * b));
-            const uint32_t sw = __ldg(reinterpret_cast<const uint32_t*>(sf + sf_offset(r, c0 >> 4, S, kInLayout)));
+            const int64_t co = r * (cols >> 1) + (c0 >> 1) + 8 * b, so_ = sf_offset(r, c0 >> 4, S, kInLayout);
+            uint2 cw = make_uint2(0u, 0u);
+            uint32_t sw = 0;
+            if (mx_in_range(co, 8, rows * (cols >> 1)))
+                cw = __ldcs(reinterpret_cast<const uint2*>(codes + co));
+            if (mx_in_range(so_, 4, rows * S)) {
+                const uint8_t* sr = sf + so_;                            // the row's 4 scale bytes, consecutive
+                sw = sf_words ? __ldg(reinterpret_cast<const uint32_t*>(sr))
+                              : (uint32_t)__ldg(sr) | (uint32_t)__ldg(sr + 1) << 8 | (uint32_t)__ldg(sr + 2) << 16 |
+                                    (uint32_t)__ldg(sr + 3) << 24;
+            }
             const uint32_t f = h2_of_e4m3((sw >> (8 * b)) & 0xffu);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) pr[g][kk] = h2_mul(h2_of_e2m1((kk < 4 ? cw.x : cw.y) >> (8 * (kk & 3))), f);
-            if (kPerRow && b == 0) so[16 * w + 8 * g + rho] = __ldg(outer + r);
+            if (kPerRow && b == 0) so[16 * w + 8 * g + rho] = mx_in_range(r, 1, rows) ? __ldg(outer + r) : 0.0f;
         }
         // stmatrix call n: 8-row group g = n / 2 of the warp's rows, column groups kappa = 4 (n % 2) + j for its
         // matrices j = 0..3.  Thread (rho, b) holds fragment row rho, fragment columns 2b, 2b+1 = tile columns
@@ -828,6 +812,7 @@ requant16_tile_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restri
     const int c = 16 * (m >> 1) + 2 * w + (m & 1);
     const int64_t cg = c0 + c;
     const int64_t Se = rows >> 5;
+    uint32_t e_bytes = 0;                               // E8M0 bytes of blocks q and 2 + q of this output row
 #pragma unroll
     for (int it = 0; it < 2; ++it) {
         const int j = 2 * (2 * it + q) + jj;
@@ -877,15 +862,52 @@ requant16_tile_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restri
         const int64_t rr = r0 + 16 * j;
         const int64_t L0 = cg * rows + rr;              // linear index of the first output element
         uint32_t wo[4];
+        if constexpr (kR == 16) {                       // the hardware stochastic rounding, two values per cvt
 #pragma unroll
-        for (int blk = 0; blk < 2; ++blk) {
-            const uint4 rnd = philox4x32_10((uint64_t)(L0 / 8) + blk, stream_id, seed);
-            wo[2 * blk] = cvt_rs16_e4m3_quad(y[8 * blk], y[8 * blk + 1], y[8 * blk + 2], y[8 * blk + 3], rnd.x, rnd.y);
-            wo[2 * blk + 1] = cvt_rs16_e4m3_quad(y[8 * blk + 4], y[8 * blk + 5], y[8 * blk + 6], y[8 * blk + 7], rnd.z,
-                                                 rnd.w);
+            for (int blk = 0; blk < 2; ++blk) {
+                const uint4 rnd = philox4x32_10((uint64_t)(L0 / 8) + blk, stream_id, seed);
+                wo[2 * blk] = cvt_rs16_e4m3_quad(y[8 * blk], y[8 * blk + 1], y[8 * blk + 2], y[8 * blk + 3], rnd.x,
+                                                 rnd.y);
+                wo[2 * blk + 1] = cvt_rs16_e4m3_quad(y[8 * blk + 4], y[8 * blk + 5], y[8 * blk + 6], y[8 * blk + 7],
+                                                     rnd.z, rnd.w);
+            }
+        } else if constexpr (kR == 8) {
+            // The same instruction with R = 8: element j's 8-bit integer u (byte j % 4 of word j / 4 of the
+            // block) enters as the 16-bit field (255 - u) << 8.  cvt.rs rounds up iff 0xFFFF - field <
+            // F16 = floor(frac 2^16), i.e. iff 256 u + 255 < F16, i.e. iff u < floor(F16 / 256) =
+            // floor(frac 2^8): the R = 8 rule exactly.
+            const uint4 rnd = philox4x32_10((uint64_t)(L0 / 16), stream_id, seed);
+            const uint32_t nw[4] = {~rnd.x, ~rnd.y, ~rnd.z, ~rnd.w};
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4)
+                wo[k4] = cvt_rs_quad_fields(y[4 * k4], y[4 * k4 + 1], y[4 * k4 + 2], y[4 * k4 + 3],
+                                            __byte_perm(nw[k4], 0u, 0x1404), __byte_perm(nw[k4], 0u, 0x3424));
+        } else {                                        // exact integer rounding of y = x 2^-e (block exponent 0)
+            const SrBlock sb = sr_block(0);
+            constexpr int kPer = 128 / kR;              // values per Philox block
+#pragma unroll
+            for (int blk = 0; blk < (16 + kPer - 1) / kPer; ++blk) {
+                const uint4 rnd = philox4x32_10((uint64_t)(L0 / kPer) + blk, stream_id, seed);
+#pragma unroll
+                for (int f = 0; f < kPer && blk * kPer + f < 16; ++f) {
+                    const int i = blk * kPer + f;
+                    const uint32_t code = e4m3_sr_code<kR>(y[i], sb, philox_field<kR>(rnd, f));
+                    if ((i & 3) == 0) wo[i >> 2] = code; else wo[i >> 2] |= code << (8 * (i & 3));
+                }
+            }
         }
-        *reinterpret_cast<uint4*>(out_codes + cg * rows + rr) = make_uint4(wo[0], wo[1], wo[2], wo[3]);
-        if (jj == 0) out_e8m0[sf_offset(cg, rr >> 5, Se, kOutLayout)] = (uint8_t)(e + 127);
+        if (mx_in_range(cg * rows + rr, 16, cols * rows))
+            *reinterpret_cast<uint4*>(out_codes + cg * rows + rr) = make_uint4(wo[0], wo[1], wo[2], wo[3]);
+        e_bytes |= (uint32_t)(e + 127) << (16 * it);
+    }
+    // The tile's four E8M0 blocks of output row cg are 4 consecutive bytes in either layout (r0 / 32 is a
+    // multiple of 4): lane q = 0 holds blocks 0 and 2, lane ^ 16 blocks 1 and 3; one 32-bit store.
+    const uint32_t other = __shfl_xor_sync(0xffffffffu, e_bytes, 16);
+    if (jj == 0 && q == 0 && mx_in_range(sf_offset(cg, r0 >> 5, Se, kOutLayout), 4, cols * Se)) {
+        uint8_t* dst = out_e8m0 + sf_offset(cg, r0 >> 5, Se, kOutLayout);
+        const uint32_t word = e_bytes | (other << 8);
+        if (e8_words) *reinterpret_cast<uint32_t*>(dst) = word;
+        else { dst[0] = (uint8_t)word; dst[1] = (uint8_t)(word >> 8); dst[2] = (uint8_t)(word >> 16); dst[3] = (uint8_t)(word >> 24); }
     }
 }
 
@@ -1072,24 +1094,27 @@ extern "C" int mxfp8_requant_transpose_sr(const uint8_t* codes, const uint8_t* s
     int gshift = -1;
     if (group_rows > 1 && (group_rows & (group_rows - 1)) == 0)
         for (gshift = 0; ((int64_t)1 << gshift) < group_rows; ++gshift) {}
-    const bool sf_words = mx_aligned(sf, 4);            // the R = 16 kernel reads a row's 4 scale bytes as a word
+    const bool sf_words = mx_aligned(sf, 4);            // a row's 4 scale bytes read as one word
+    const bool e8_words = mx_aligned(out_e8m0, 4);      // an output row's 4 E8M0 bytes of a tile stored as one word
     return dispatch_layout(in_sf_layout, [&](auto Li) {
         return dispatch_layout(out_sf_layout, [&](auto Lo) {
             constexpr int kLi = decltype(Li)::value, kLo = decltype(Lo)::value;
-            if (rbits == 8)
-                requant_tile_kernel<8, kLi, kLo><<<grid, kTileThreads, 0, stream>>>(
-                    codes, sf, outer, rows, cols, group_rows, gshift, rows_valid, seed, stream_id, out_codes, out_e8m0);
-            else if (rbits == 16 && group_rows == 1 && sf_words)
-                requant16_tile_kernel<kLi, kLo, true><<<grid, kTileThreads, 0, stream>>>(
-                    codes, sf, outer, rows, cols, group_rows, gshift, rows_valid, seed, stream_id, out_codes, out_e8m0);
-            else if (rbits == 16 && sf_words)
-                requant16_tile_kernel<kLi, kLo, false><<<grid, kTileThreads, 0, stream>>>(
-                    codes, sf, outer, rows, cols, group_rows, gshift, rows_valid, seed, stream_id, out_codes, out_e8m0);
-            else
-                requant_tile_kernel<32, kLi, kLo><<<grid, kTileThreads, 0, stream>>>(
-                    codes, sf, outer, rows, cols, group_rows, gshift, rows_valid, seed, stream_id, out_codes, out_e8m0);
+            auto go = [&](auto Rc, auto per_row) {
+                requant_tile_kernel<decltype(Rc)::value, kLi, kLo, decltype(per_row)::value>
+                    <<<grid, kTileThreads, 0, stream>>>(codes, sf, sf_words, e8_words, outer, rows, cols, group_rows, gshift,
+                                                         rows_valid, seed, stream_id, out_codes, out_e8m0);
+            };
+            auto by_r = [&](auto per_row) {
+                if (rbits == 8) go(std::integral_constant<int, 8>(), per_row);
+                else if (rbits == 16) go(std::integral_constant<int, 16>(), per_row);
+                else go(std::integral_constant<int, 32>(), per_row);
+            };
+            if (group_rows == 1) by_r(std::true_type());
+            else by_r(std::false_type());
             mx_count_launch();
             return mx_launch_status();
         });
     });
 }
+
+MX_BOUNDS_READER(mx_bounds_word_quant)

@@ -147,3 +147,5 @@ extern "C" int moe_combine_s2f6(const int8_t* codes, const uint8_t* e8m0, const 
     mx_count_launch();
     return mx_launch_status();
 }
+
+MX_BOUNDS_READER(mx_bounds_word_s2f6)

@@ -94,6 +94,17 @@ MX_API int mx_sync_status(cudaStream_t stream);
  * The pages have no counterpart. */
 MX_API int mx_wait_selftest(int64_t limit_us, cudaStream_t stream);
 
+/* Bounds-checked build (libmxmoe_debug.so, built with -DMX_DEBUG_BOUNDS): the
+ * kernels check the global indices they compute against the extents their
+ * call's arguments give the buffers, skip an access out of range and count
+ * it.  mx_debug_bounds_build() is 1 in that library and 0 in libmxmoe.so;
+ * mx_debug_bounds_violations() synchronises nothing, reads the counts of
+ * everything that has completed (the caller synchronises first), clears them
+ * when `clear` is nonzero, and is always 0 in libmxmoe.so.  The pages have no
+ * counterpart: it stands in for a memory checker. */
+MX_API int mx_debug_bounds_build(void);
+MX_API unsigned long long mx_debug_bounds_violations(int clear);
+
 /* Bytes of a scale array of `rows` x `cols` elements with one scale per
  * `block` (16 or 32) elements in `sf_layout`; 0 if the shape is not allowed
  * for that layout. */

@@ -106,3 +106,21 @@ def test_c_program_compiles_links_and_calls_the_library(mx, tmp_path):
     out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
     assert int(out[0]) == mx.mx_version() and int(out[1]) == 1          # MX_EINVAL
     assert int(out[2]) == 256 * 4096 // 16 and int(out[3]) == 0          # nothing launched
+
+
+def test_bounds_checked_build_exports_the_same_symbols(mx):
+    """libmxmoe_debug.so (-DMX_DEBUG_BOUNDS) builds from the same sources, exports
+    every declared symbol, reports itself as the bounds-checked build, and the
+    normal library reports 0 and never counts anything."""
+    import ctypes
+    from fp8_moe_numerics_b200 import build
+    path = build.build(debug_bounds=True)
+    dbg = ctypes.CDLL(path)
+    for n in _declared():
+        assert hasattr(dbg, n), n
+    dbg.mx_debug_bounds_build.restype = ctypes.c_int
+    dbg.mx_debug_bounds_violations.restype = ctypes.c_ulonglong
+    dbg.mx_debug_bounds_violations.argtypes = [ctypes.c_int]
+    assert dbg.mx_debug_bounds_build() == 1
+    assert mx.mx_debug_bounds_build() == 0
+    assert mx.mx_debug_bounds_violations(1) == 0

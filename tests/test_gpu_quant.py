@@ -265,9 +265,10 @@ def test_requant_weights_per_expert_outer(cuda, E, N, K, R):
     assert np.array_equal(mma_to_rowmajor(np_(ge), K, E * N // 32), oe)
 
 
+@pytest.mark.parametrize("R", [8, 16, 32])
 @pytest.mark.parametrize("scale_exp", [-40, -36, -30, 0, 30])
-def test_requant_weights_fold_boundary(cuda, scale_exp):
-    """R = 16 with one outer scale per expert: the kernel folds the outer scale
+def test_requant_weights_fold_boundary(cuda, scale_exp, R):
+    """One outer scale per expert: the kernel folds the outer scale
     and 2^-e into one product while p*s stays in fp32's normal range (outer
     scale >= 2^-100) and takes the two products below it.  Experts scaled by
     10^scale_exp (outer scales around the 2^-100 switch, fp32 subnormal
@@ -279,14 +280,14 @@ def test_requant_weights_fold_boundary(cuda, scale_exp):
     wf = w.reshape(E * N, K).to(torch.float32).numpy()
     w16 = oracle.f32_to_bf16(wf)
     codes, sf, outer = oracle.nvfp4_quantize(w16, group_rows=N)
-    oc, oe = oracle.mxfp8_requant_transpose_sr(codes, sf, outer, N, 21, 22, 16)
+    oc, oe = oracle.mxfp8_requant_transpose_sr(codes, sf, outer, N, 21, 22, R)
     sf_mma = rowmajor_to_mma(sf)
     for off in (0, 1):                                   # scales at an aligned and a misaligned address
         buf = torch.zeros(sf_mma.size + 16, dtype=torch.uint8, device="cuda")
         buf[off:off + sf_mma.size] = torch.from_numpy(sf_mma).cuda()
         gc, ge = api.mxfp8_requant_transpose_sr(torch.from_numpy(codes).cuda(), buf[off:off + sf_mma.size],
                                                 torch.from_numpy(outer).cuda(), E * N, K, N, api.MX_SF_MMA, None, 21,
-                                                22, 16, api.MX_SF_MMA)
+                                                22, R, api.MX_SF_MMA)
         assert np.array_equal(np_(gc), oc), off
         assert np.array_equal(mma_to_rowmajor(np_(ge), K, E * N // 32), oe), off
 
