@@ -672,7 +672,7 @@ def cpu_baseline(inp, seconds: float = 15.0):
 # --------------------------------------------------------------------------
 KERNEL_CASES = ("gemm_nvfp4", "gemm_nvfp4_s2f6", "gemm_mxfp8_dgrad", "gemm_mxfp8_wgrad", "requant", "requant_w",
                 "nvfp4_quantize", "quant_w", "mxfp8_quantize", "nvfp4_quantize_sr", "requant_nvfp4", "gemm_nvfp4_wgrad",
-                "step_nvfp4_backward")
+                "step_nvfp4_backward", "gemm1_moe_layer", "gemm2_moe_layer")
 
 
 def run_kernel(args):
@@ -688,6 +688,26 @@ def run_kernel(args):
         layer = ExpertLayer(inp["x"], inp["topk"].to(dev), inp["w_comb"].to(dev), inp["w1"], inp["w2"], inp["dout"],
                             gated=c["gated"], seed=c["seed"], backward="nvfp4")
         run = layer.step
+    elif which in ("gemm1_moe_layer", "gemm2_moe_layer"):
+        # the 384-expert layer's forward GEMMs at their own shapes and routing (262144 routed rows, Zipf 1.2 with
+        # 8 empty experts): seeded valid codes and scales (the kernel's time does not depend on their values);
+        # about 4 GB on the device
+        c = workloads.CONFIGS[WORKLOAD]
+        E, T, k, D, F = c["E"], c["T"], c["k"], c["D"], c["F"]
+        ids = workloads.routing(T, k, E, c["routing"], c["zipf"], c["n_empty"], c["seed"]).to(dev)
+        seg, src, pos = api.moe_route(ids, E)
+        M = src.shape[0]
+        N, K = (2 * F, D) if which == "gemm1_moe_layer" else (D, F)
+        g = torch.Generator(device=dev)
+        g.manual_seed(9)
+        a = (torch.randint(0, 256, (M, K // 2), dtype=torch.uint8, device=dev, generator=g),
+             torch.randint(0x30, 0x48, (M * K // 16,), dtype=torch.uint8, device=dev, generator=g),
+             torch.full((M,), 1e-3, device=dev))
+        b = (torch.randint(0, 256, (E * N, K // 2), dtype=torch.uint8, device=dev, generator=g),
+             torch.randint(0x30, 0x48, (E * N * K // 16,), dtype=torch.uint8, device=dev, generator=g),
+             torch.full((E,), 1e-3, device=dev))
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        run = lambda: api.grouped_gemm_nvfp4(a, b, seg, E, N, K, out=out)
     elif which.startswith("gemm"):
         # 64 experts, top-8 of 4096 tokens (Zipf 1.2), d_model 4096, d_ff 1024 (gated)
         E, T, k, D, F = 64, 4096, 8, 4096, 1024
