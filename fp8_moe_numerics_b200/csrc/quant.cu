@@ -290,8 +290,8 @@ __global__ void nvfp4_group_finish_kernel(float* outer, int64_t ngroups) {
 }
 
 // ---------------------------------------------------------------------------
-// Transpose tile: 128 rows x 64 columns of the input.  Phase 1 loads the tile
-// (bf16, or NVFP4 dequantised to fp32) -- thread t owns row t/2, columns
+// Transpose tile of the register-prefetch MXFP8 quantiser: 128 rows x 64
+// columns of the bf16 input.  Phase 1 loads the tile -- thread t owns row t/2, columns
 // 32*(t%2) .. +31 -- and stores fp32 values transposed into shared memory
 // T[c][r] (128 words per row c).  Phase 2: thread (c, g) takes output row c,
 // elements r = 16g .. 16g+15 as four 16-byte chunks (8 threads cover the

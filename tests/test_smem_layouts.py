@@ -2,7 +2,7 @@
 
 The requantisation and the MXFP8 quantiser transpose their tiles through
 shared memory with XOR swizzles (csrc/quant.cu: tsw for the fp32 tile of the
-requantisation and the register-prefetch MXFP8 kernel, t2_word for the bf16
+register-prefetch MXFP8 kernel, rq_swz for the f16 tile of the requantisation, t2_word for the bf16
 pair tile of the TMA-fed MXFP8 kernel; the TMA tiles use the hardware's
 128-byte swizzle).  The swizzle functions are restated here and every warp
 access pattern of the kernels is replayed to check that each layout is a
