@@ -368,6 +368,8 @@ def run_ours(args):
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
     cfg_legs = gemm_config_legs(dev, peaks) if rank == 0 else None
+    torch.cuda.empty_cache()
+    nv_bwd = nvfp4_backward_leg(dev, peaks) if rank == 0 else None
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": K,
@@ -388,6 +390,7 @@ def run_ours(args):
         "mxfp8_forward": mx_fwd,
         "fwd_gemm": cfg_legs["fwd_gemm"] if cfg_legs else None,
         "bwd_gemm": cfg_legs["bwd_gemm"] if cfg_legs else None,
+        "nvfp4_backward": nv_bwd,
         "roofline": roof,
         "clocks": clk.summary(),
         "e2e": e2e,
@@ -605,6 +608,65 @@ def gemm_config_legs(dev, peaks, steps: int = 3, warmup: int = 2):
         "steps": steps,
     }
     del layer, inp, dout
+    return res
+
+
+def nvfp4_backward_leg(dev, peaks, steps: int = 2, warmup: int = 1):
+    """The 384-expert layer with the four backward GEMMs in NVFP4 (stochastically
+    rounded E2M1 operands, the pages' stated future work) beside the MXFP8
+    backward of the timed steps: step time and per-stage times."""
+    import torch
+    from fp8_moe_numerics_b200 import api, workloads
+    from fp8_moe_numerics_b200.layer import ExpertLayer
+    c = workloads.CONFIGS[WORKLOAD]
+    inp = workloads.layer_inputs(WORKLOAD, device=dev)
+    layer = ExpertLayer(inp["x"], inp["topk"].to(dev), inp["w_comb"].to(dev), inp["w1"], inp["w2"], inp["dout"],
+                        gated=c["gated"], seed=c["seed"], backward="nvfp4")
+    counts = torch.bincount(inp["topk"].reshape(-1).long(), minlength=c["E"]).tolist()
+    for _ in range(warmup):
+        layer.step()
+    torch.cuda.synchronize()
+    layer.reset_marks()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        layer.step(record=True)
+    b.record()
+    torch.cuda.synchronize()
+    api.sync_status()
+    st = layer.stage_times_ms()
+    T, k, D, F, E = c["T"], c["k"], c["D"], c["F"], c["E"]
+    R, N1 = T * k, 2 * F
+    M = layer.M_cap
+    nv = lambda rows, cols: rows * cols * (0.5 + 1 / 16) + rows * 4
+    work = {   # algorithmic bytes (requantisations, quantisers) or flops over true rows (GEMMs)
+        "quant_dy2": ("hbm", R * D * 2 + nv(R, D)),
+        "requant_w2": ("hbm", 2 * nv(E * D, F)),
+        "dgrad2": ("tensor4", 2 * R * F * D),
+        "requant_a": ("hbm", R * D * 2 + nv(D, R) + 2 * nv(R, F)),
+        "wgrad2": ("tensor4", 2 * R * D * F),
+        "quant_dh1": ("hbm", R * N1 * 2 + nv(R, N1)),
+        "requant_w1": ("hbm", 2 * nv(E * N1, D)),
+        "dgrad1": ("tensor4", 2 * R * D * N1),
+        "requant_x": ("hbm", R * N1 * 2 + nv(N1, R) + 2 * nv(R, D)),
+        "wgrad1": ("tensor4", 2 * R * N1 * D),
+    }
+    res = {"ms_per_step": round(a.elapsed_time(b) / steps, 3), "steps": steps,
+           "padded_rows": M, "note": "segments padded to 256 rows for the NVFP4 wgrad's K-stage; requant_a and "
+           "requant_x are the two transposed wgrad operands of that GEMM (dY^T from bf16, the saved NVFP4 "
+           "activations^T); bytes of each stage read once and written once"}
+    for n, (kind, wk) in work.items():
+        if n not in st:
+            continue
+        t = st[n] / steps
+        if kind == "hbm":
+            gbs = wk / (t * 1e-3) / 1e9
+            res[n] = {"ms": round(t, 4), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm"], 4)}
+        else:
+            tf = wk / (t * 1e-3) / 1e12
+            res[n] = {"ms": round(t, 4), "TFLOP/s": round(tf, 1), "frac_nominal": round(tf / NOMINAL_NVFP4_TFLOPS, 4),
+                      "frac_measured": round(tf / (peaks["bf16_sus"] * 4), 4)}
+    del layer, inp
     return res
 
 
