@@ -5,6 +5,7 @@
 // packed-integer max and warp shuffles, every rounding decision taken by a PTX
 // cvt or by exact integer arithmetic (see mx_common.cuh).
 #include "mx_common.cuh"
+#include "requant_tile.cuh"
 
 #include <cuda.h>
 
@@ -302,6 +303,7 @@ __global__ void nvfp4_group_finish_kernel(float* outer, int64_t ngroups) {
 // quarter warp) are both free of bank conflicts.
 // ---------------------------------------------------------------------------
 constexpr int kTR = 128, kTC = 64, kTileThreads = 256;
+static_assert(kTR == kRqRows && kTC == kRqCols && kTileThreads == kRqThreads, "one tile shape");
 
 __device__ __forceinline__ int tsw(int c, int r) {
     const int rs = (r & ~12) | ((((r >> 2) & 3) ^ ((r >> 5) & 3)) << 2);
@@ -680,13 +682,8 @@ mxfp8_tile_tma_kernel(const __grid_constant__ CUtensorMap tmX, int64_t rows, int
 // ---------------------------------------------------------------------------
 // NVFP4 [rows, cols] -> dequantise -> transpose -> MXFP8 with stochastic
 // rounding: one 128 x 64 input tile per block, 256 threads.
-//   Phase 1: each thread decodes 2 rows x 16 columns (one scale block per
-//   row) to the exact f16 products q*sf (cvt e2m1x2 -> f16x2, one f16x2
-//   multiply per pair; |q sf| <= 2688 and >= 2^-10 when nonzero, so f16 holds
-//   it exactly) and the warp stores its 16 x 64 products transposed with four
-//   stmatrix.trans (8 x 8 blocks of 16-bit values).  The tile lives in shared
-//   memory as f16 [64 cols][128 rows], 16-byte chunks XOR-swizzled by
-//   rq_swz() so that both phases are free of bank conflicts.
+//   Phase 1 (rq_load_tile): the tile's exact f16 products q*sf, transposed
+//   into shared memory.
 //   Phase 2: each thread takes 16 consecutive rows of one output row, twice:
 //   two 16-byte loads, f16 -> fp32, the outer scale (x = RN(p s)), the
 //   32-row amax (the block's other half is in lane ^ 8), the E8M0 exponent e,
@@ -698,44 +695,6 @@ mxfp8_tile_tma_kernel(const __grid_constant__ CUtensorMap tmX, int64_t rows, int
 //   range, which s >= 2^-100 guarantees (|p| >= 2^-10); smaller s takes the
 //   two products.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ int rq_swz(int c) { return ((c >> 4) & 3) | ((c & 1) << 2); }
-
-__device__ __forceinline__ uint32_t h2_of_e4m3(uint32_t code) {
-    uint32_t h2;
-    const uint16_t in = (uint16_t)(code * 0x0101u);
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
-    return h2;
-}
-__device__ __forceinline__ uint32_t h2_of_e2m1(uint32_t byte_in_low) {
-    uint32_t h2;
-    asm("{\n\t.reg .b8 b;\n\tcvt.u8.u32 b, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, b;\n\t}" : "=r"(h2) : "r"(byte_in_low));
-    return h2;
-}
-__device__ __forceinline__ uint32_t h2_mul(uint32_t a, uint32_t b) {
-    uint32_t d;
-    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
-}
-// max(|a|, |b|) per lane; the sign bit is not meaningful (callers drop it).
-__device__ __forceinline__ uint32_t h2_maxabs(uint32_t a, uint32_t b) {
-    uint32_t d;
-    asm("max.xorsign.abs.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
-}
-__device__ __forceinline__ void h2_to_f32x2(uint32_t h, float& lo, float& hi) {
-    asm("{\n\t.reg .f16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, h;\n\t}"
-        : "=f"(lo), "=f"(hi) : "r"(h));
-}
-__device__ __forceinline__ void stmatrix_x4_trans(uint32_t addr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
-    asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1, %2, %3, %4};"
-                 :: "r"(addr), "r"(r0), "r"(r1), "r"(r2), "r"(r3) : "memory");
-}
-__device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
-    uint4 v;
-    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
-    return v;
-}
-
 // cvt.rs on four values with their 16-bit random fields given as cvt.rs takes
 // them (y0 in bits 15:0 of f01, y1 in bits 31:16, likewise y2, y3 in f23);
 // codes packed y0 | y1 << 8 | y2 << 16 | y3 << 24.
@@ -759,66 +718,26 @@ requant_tile_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict
     __shared__ __align__(16) float so[kPerRow ? kTR : 4];
     const int64_t c0 = (int64_t)blockIdx.x * kTC, r0 = (int64_t)blockIdx.y * kTR;
     if (r0 >= load_rows_valid(rows_valid, rows)) return;
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     const uint32_t tbase = smem_u32(T);
     float s_uni = 0.0f;
     if (!kPerRow) {                   // group_rows is a multiple of 128: one outer scale per tile
         const int64_t gi = group_shift >= 0 ? (r0 >> group_shift) : (int64_t)((uint32_t)r0 / (uint32_t)group_rows);
         if (mx_in_range(gi, 1, rows / group_rows)) s_uni = __ldg(outer + gi);
     }
-    // ---------------- phase 1: lane (rho = lane / 4, b = lane % 4): rows 16w + rho and 16w + 8 + rho,
-    // code bytes 8b..8b+7 of the tile row = columns 16b..16b+15 (scale block b of the tile)
-    {
-        const int rho = lane >> 2, b = lane & 3;
-        const int64_t S = cols >> 4;
-        uint32_t pr[2][8];
-#pragma unroll
-        for (int g = 0; g < 2; ++g) {
-            const int64_t r = r0 + 16 * w + 8 * g + rho;
-            const int64_t co = r * (cols >> 1) + (c0 >> 1) + 8 * b, so_ = sf_offset(r, c0 >> 4, S, kInLayout);
-            uint2 cw = make_uint2(0u, 0u);
-            uint32_t sw = 0;
-            if (mx_in_range(co, 8, rows * (cols >> 1)))
-                cw = __ldcs(reinterpret_cast<const uint2*>(codes + co));
-            if (mx_in_range(so_, 4, rows * S)) {
-                const uint8_t* sr = sf + so_;                            // the row's 4 scale bytes, consecutive
-                sw = sf_words ? __ldg(reinterpret_cast<const uint32_t*>(sr))
-                              : (uint32_t)__ldg(sr) | (uint32_t)__ldg(sr + 1) << 8 | (uint32_t)__ldg(sr + 2) << 16 |
-                                    (uint32_t)__ldg(sr + 3) << 24;
-            }
-            const uint32_t f = h2_of_e4m3((sw >> (8 * b)) & 0xffu);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) pr[g][kk] = h2_mul(h2_of_e2m1((kk < 4 ? cw.x : cw.y) >> (8 * (kk & 3))), f);
-            if (kPerRow && b == 0) so[16 * w + 8 * g + rho] = mx_in_range(r, 1, rows) ? __ldg(outer + r) : 0.0f;
-        }
-        // stmatrix call n: 8-row group g = n / 2 of the warp's rows, column groups kappa = 4 (n % 2) + j for its
-        // matrices j = 0..3.  Thread (rho, b) holds fragment row rho, fragment columns 2b, 2b+1 = tile columns
-        // 16b + 2 kappa + {0, 1}; stored row m of matrix j (address from lane 8j + m) is tile column
-        // 16 (m / 2) + 2 kappa + m % 2, its 8 values the 8 rows of chunk 2w + g.
-        const int j = lane >> 3, m = lane & 7;
-#pragma unroll
-        for (int n = 0; n < 4; ++n) {
-            const int g = n >> 1, kap = 4 * (n & 1) + j;
-            const int c = 16 * (m >> 1) + 2 * kap + (m & 1);
-            const int kb = 4 * (n & 1);
-            stmatrix_x4_trans(tbase + c * 256 + (((2 * w + g) ^ rq_swz(c)) << 4), pr[g][kb], pr[g][kb + 1],
-                              pr[g][kb + 2], pr[g][kb + 3]);
-        }
-    }
+    rq_load_tile<kInLayout, kPerRow>(codes, sf, sf_words, outer, rows, cols, 1, r0, c0, tbase, so);
     __syncthreads();
     // ---------------- phase 2: lane (m = lane % 8, jj = (lane / 8) % 2, q = lane / 16) of warp w: output row
     // c = 16 (m / 2) + 2w + m % 2 of the tile, input rows 16j..16j+15 with j = 2 (2 it + q) + jj
-    const int m = lane & 7, jj = (lane >> 3) & 1, q = lane >> 4;
-    const int c = 16 * (m >> 1) + 2 * w + (m & 1);
+    const RqLane ln;
+    const int jj = ln.jj, q = ln.q, c = ln.c;
     const int64_t cg = c0 + c;
     const int64_t Se = rows >> 5;
     uint32_t e_bytes = 0;                               // E8M0 bytes of blocks q and 2 + q of this output row
 #pragma unroll
     for (int it = 0; it < 2; ++it) {
-        const int j = 2 * (2 * it + q) + jj;
-        const uint4 v0 = lds_v4(tbase + c * 256 + (((2 * j) ^ rq_swz(c)) << 4));
-        const uint4 v1 = lds_v4(tbase + c * 256 + (((2 * j + 1) ^ rq_swz(c)) << 4));
-        const uint32_t hw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        const int j = ln.chunk(it);
+        uint32_t hw[8];
+        rq_read16(tbase, c, j, hw);
         float y[16];
 #pragma unroll
         for (int i = 0; i < 8; ++i) h2_to_f32x2(hw[i], y[2 * i], y[2 * i + 1]);
@@ -840,11 +759,7 @@ requant_tile_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict
 #pragma unroll
             for (int i = 0; i < 8; ++i) mul2_rn(y[2 * i], y[2 * i + 1], sc2);
         } else {
-            const uint32_t hm = h2_maxabs(h2_maxabs(h2_maxabs(hw[0], hw[1]), h2_maxabs(hw[2], hw[3])),
-                                          h2_maxabs(h2_maxabs(hw[4], hw[5]), h2_maxabs(hw[6], hw[7])));
-            float ml, mh;
-            h2_to_f32x2(hm, ml, mh);
-            float pm = fmaxf(fabsf(ml), fabsf(mh));
+            float pm = rq_maxabs16(hw);
             pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, 8));
             e = e8m0_exponent(__fmul_rn(pm, s_uni));
             const bool fold = s_uni >= kFoldMinScale;

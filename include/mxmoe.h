@@ -428,9 +428,10 @@ MX_API int nvfp4_quantize_sr(const void* x, int64_t rows, int64_t cols, int64_t 
  * B for the NVFP4 input gradient (output width K).
  *   out_codes device u8 [experts*cols, rows/experts/2]; out_sf device u8
  *   mx_sf_bytes(experts*cols, rows/experts, 16, out_sf_layout)
- * Requires cols % 64 == 0, rows / experts % 128 == 0, rows % group_rows == 0
- * (rows % 128 == 0 for an MX_SF_MMA input; experts*cols % 128 == 0 for an
- * MX_SF_MMA output), 16-byte aligned codes and out_codes.  out_outer is
+ * Requires cols % 64 == 0, rows / experts % 128 == 0, rows % group_rows == 0,
+ * rows <= 65535 * 128 (rows % 128 == 0 for an MX_SF_MMA input;
+ * experts*cols % 128 == 0 for an MX_SF_MMA output), 16-byte aligned codes
+ * and out_codes.  out_outer is
  * written twice (the per-target maxima, then the scales) by the calls this
  * entry point enqueues. */
 MX_API int nvfp4_requant_transpose_sr(const uint8_t* codes, const uint8_t* sf, const float* outer, int64_t rows,
@@ -469,7 +470,8 @@ MX_API int nvfp4_quantize_transpose_segments(const void* x, int64_t M, int64_t C
                                              int out_sf_layout, cudaStream_t stream);
 
 /* The same from a saved NVFP4 tensor [M, C] (codes, sf in in_sf_layout, outer
- * per group_rows rows), each value dequantised ((q * sf) * outer, fp32). */
+ * per group_rows rows), each value dequantised ((q * sf) * outer, fp32).
+ * Also requires M <= 65535 * 128 and 16-byte aligned codes. */
 MX_API int nvfp4_requant_transpose_segments(const uint8_t* codes, const uint8_t* sf, const float* outer,
                                             int in_sf_layout, int64_t group_rows, int64_t M, int64_t C,
                                             const int64_t* seg, int64_t E, int per_row, int rounding,

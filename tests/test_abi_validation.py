@@ -107,6 +107,7 @@ CASES = {
         ("unknown out layout", {16: 3}), ("outer-per-expert flag 2", {8: 2}), ("out codes misaligned", {13: A8}),
         ("null out outer", {15: None}), ("out outer misaligned", {15: A1}),
         ("per-row outer scales over two experts", {8: 0}),
+        ("more tile rows than the grid's y axis", {3: 65536 * 128, 5: 128, 7: 1}),
     ]),
     "nvfp4_quantize_transpose_segments": ((A, 256, 128, A, 2, 1, 1, 1, 2, 16, A, A, A, 1, None), [
         ("M % 128", {1: 192}), ("C % 64", {2: 96}), ("no experts", {4: 0}), ("per_row 2", {5: 2}),
@@ -116,7 +117,7 @@ CASES = {
     "nvfp4_requant_transpose_segments": ((A, A, A, 1, 1, 256, 128, A, 2, 0, 1, 1, 2, 16, A, A, A, 1, None), [
         ("unknown input layout", {3: 4}), ("group_rows 0", {4: 0}), ("M % group_rows", {4: 3}),
         ("codes misaligned", {0: A8}), ("M % 128", {5: 64}), ("out outer misaligned", {16: A1}),
-        ("unknown rounding", {10: 5}),
+        ("unknown rounding", {10: 5}), ("more tile rows than the grid's y axis", {5: 65536 * 128}),
     ]),
     "grouped_gemm_nvfp4_wgrad": ((A, A, A, A, A, A, A, 2, 512, 128, 256, A, 0, None), [
         ("M_cap % 256", {8: 384}), ("N % 128", {9: 64}), ("K % 128", {10: 64}), ("no experts", {7: 0}),

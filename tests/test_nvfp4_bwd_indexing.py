@@ -34,6 +34,102 @@ def _exactly_once(starts, width, size):
     assert len(starts) * width == size and np.all(np.diff(starts) == width)
 
 
+def _group_amax_replay(rows, cols, group_rows, in_mma, block_rows, target_of_block, n_targets):
+    """group_amax_nvfp4_kernel: block = 128 rows (skipped when target_of_block
+    gives None), thread t = row r0 + t % 128, 64-value chunks k = t / 128,
+    t / 128 + 2, ...: 32 code bytes and the 4 scale bytes of blocks 4k .. 4k + 3."""
+    S = cols // 16
+    t = np.arange(T)
+    for r0 in block_rows:
+        tg = target_of_block(r0)
+        if tg is None:
+            continue
+        assert 0 <= tg < n_targets
+        r = r0 + (t & 127)
+        assert r.max() < rows and (r // group_rows).max() < rows // group_rows
+        for k in range(cols // 64):
+            rr = r[(t >> 7) == (k & 1)]
+            co = rr * (cols // 2) + 32 * k
+            assert co.min() >= 0 and (co + 32).max() <= rows * cols // 2 and np.all(co % 16 == 0)
+            so = np.array([sf_offset(int(a), 4 * k, S, in_mma) for a in rr])
+            assert so.min() >= 0 and (so + 4).max() <= rows * S and np.all(so % 4 == 0)
+            # the 4 scale bytes of a chunk are blocks 4k .. 4k + 3 of the row, in order
+            for a in rr[::37]:
+                base = sf_offset(int(a), 4 * k, S, in_mma)
+                assert [sf_offset(int(a), 4 * k + i, S, in_mma) for i in range(4)] == [base + i for i in range(4)]
+
+
+def _requant_tile_replay(rows, cols, group_rows, in_mma, out_mma, live_of_tile, out_row_base, out_cols, n_out_rows,
+                         bf16=False):
+    """requant_nvfp4_tile_kernel: grid (cols / 64, rows / 128), 8 warps.
+    Phase 1: lane (rho, b) of warp w loads rows r0 + 16w + 8g + rho (g = 0, 1):
+    8 code bytes at column c0 + 16b, the row's 4 scale bytes of the tile.
+    Phase 2: lane (m, jj, q) of warp w takes tile column c = 16 (m / 2) + 2w + m % 2
+    and, for it = 0, 1, input rows 16j .. with j = 4 it + 2q + jj: 8 output code
+    bytes at L0 / 2 (L0 = o * out_cols + n0 + 16j), and lane jj = q = 0 one scale
+    word at block n0 / 16 + 4 it of output row o.  A bf16 source (bf16=True)
+    loads in phase 1 16 bytes per lane instead: unit n of warp w is row
+    r0 + 16w + 8 (n / 2) + rho, columns c0 + 16b + 8 (n % 2) .. + 7."""
+    S = cols // 16
+    codes_out, sf_words, L_all = [], [], []
+    lane = np.arange(32)
+    for by in range(rows // 128):
+        r0 = by * 128
+        live = live_of_tile(r0)
+        n0, o_base = out_row_base(r0)
+        for bx in range(cols // 64):
+            c0 = bx * 64
+            for w in range(8):
+                if live and bf16:
+                    rho, b = lane >> 2, lane & 3
+                    seen = []
+                    for n in range(4):
+                        r = r0 + 16 * w + 8 * (n >> 1) + rho
+                        xi = r * cols + c0 + 16 * b + 8 * (n & 1)
+                        assert xi.min() >= 0 and (xi + 8).max() <= rows * cols and np.all(xi % 8 == 0)
+                        seen.extend(xi.tolist())
+                    # the warp's 16 rows x 64 columns, each element loaded once
+                    rel = np.array(seen) - (r0 + 16 * w) * cols - c0
+                    _exactly_once(rel // cols * 64 + rel % cols, 8, 16 * 64)
+                elif live:
+                    rho, b = lane >> 2, lane & 3
+                    for g in range(2):
+                        r = r0 + 16 * w + 8 * g + rho
+                        co = r * (cols // 2) + c0 // 2 + 8 * b
+                        assert co.min() >= 0 and (co + 8).max() <= rows * cols // 2 and np.all(co % 8 == 0)
+                        so = np.array([sf_offset(int(a), c0 // 16, S, in_mma) for a in r])
+                        assert so.min() >= 0 and (so + 4).max() <= rows * S
+                        # the row's four scale bytes of the tile are consecutive
+                        assert all(sf_offset(int(a), c0 // 16 + i, S, in_mma) == sf_offset(int(a), c0 // 16, S, in_mma)
+                                   + i for a in r[:4] for i in range(4))
+                        assert (r // group_rows).max() < rows // group_rows
+                m, jj, q = lane & 7, (lane >> 3) & 1, lane >> 4
+                c = 16 * (m >> 1) + 2 * w + (m & 1)
+                o = o_base + c0 + c
+                assert o.max() < n_out_rows
+                for it in range(2):
+                    j = 4 * it + 2 * q + jj
+                    L0 = o * out_cols + n0 + 16 * j
+                    codes_out.extend((L0 // 2).tolist())
+                    L_all.append(L0)
+                    lead = (jj == 0) & (q == 0)
+                    nb = out_cols // 16
+                    for a in o[lead]:
+                        base = sf_offset(int(a), n0 // 16 + 4 * it, nb, out_mma)
+                        assert base % 4 == 0
+                        assert [sf_offset(int(a), n0 // 16 + 4 * it + i, nb, out_mma) for i in range(4)] == \
+                            [base + i for i in range(4)]
+                        sf_words.append(base)
+                    # the word's bytes come from lanes ^ 8 and ^ 16 of the same output row, byte 2q + jj
+                    for l in range(32):
+                        assert c[l ^ 8] == c[l] and c[l ^ 16] == c[l]
+    n_out = n_out_rows * out_cols
+    _exactly_once(codes_out, 8, n_out // 2)
+    _exactly_once(sf_words, 4, n_out // 16)
+    L = np.concatenate(L_all)[:, None] + np.arange(16)[None, :]
+    assert np.array_equal(np.sort(L.reshape(-1)), np.arange(n_out))
+
+
 @pytest.mark.parametrize("rows,cols,group_rows,mma", [(128, 64, 1, True), (256, 128, 128, True), (48, 32, 16, False),
                                                       (16, 16, 1, False)])
 def test_quantize_sr_kernel_indexing(rows, cols, group_rows, mma):
@@ -67,39 +163,31 @@ def test_requant_kernels_indexing(rows, cols, group_rows, experts, per_expert, i
     assert not out_mma or ((experts * cols) % 128 == 0 and rpe % 64 == 0)
     assert per_expert or experts == 1
     S_in = cols // 16
-    # pass 1: grid (cols / 64, rows / 128); thread (cl = t % 64, rg = t / 64) reads 32 rows of one column
     n_outer = experts if per_expert else experts * cols
-    for by in range(rows // 128):
-        r0 = by * 128
-        e = r0 // rpe
-        assert (r0 + 127) // rpe == e                         # a block never straddles two experts
-        for bx in range(cols // 64):
-            t = np.arange(T)
-            cl, rg = t & 63, t >> 6
-            c = bx * 64 + cl
-            rr = r0 + rg[:, None] * 32 + np.arange(32)[None, :]
-            assert rr.max() < rows and c.max() < cols
-            assert ((rr * cols + c[:, None]) // 2).max() < rows * cols // 2
-            offs = [sf_offset(int(a), int(cc) // 16, S_in, in_mma) for a, cc in zip(rr.reshape(-1),
-                                                                                    np.repeat(c, 32))]
-            assert min(offs) >= 0 and max(offs) < rows * S_in
-            targets = np.full(1, e) if per_expert else e * cols + c[:64]
-            assert targets.min() >= 0 and targets.max() < n_outer
-    # pass 2: one thread per output block of 16; item -> (c fastest, then block b, then expert e)
-    nb = rpe // 16
-    item = _threads(experts * nb * cols)
-    c = item % cols
-    b = (item // cols) % nb
-    e = item // cols // nb
-    o = e * cols + c
-    rr = e[:, None] * rpe + b[:, None] * 16 + np.arange(16)[None, :]
-    assert rr.max() < rows
-    assert np.all((per_expert and e.max() < experts) or o.max() < experts * cols)
-    _exactly_once((o * rpe + b * 16) // 2, 8, experts * cols * rpe // 2)
-    _exactly_once([sf_offset(int(a), int(bb), nb, out_mma) for a, bb in zip(o, b)], 1, experts * cols * nb)
-    # the random index of each element is its linear output index, each used once
-    L = (o * rpe + b * 16)[:, None] + np.arange(16)[None, :]
-    assert np.array_equal(np.sort(L.reshape(-1)), np.arange(experts * cols * rpe))
+    assert rows // 128 <= 65535
+    for r0 in range(0, rows, 128):
+        assert (r0 + 127) // rpe == r0 // rpe                 # a block never straddles two experts
+    if per_expert:
+        # pass 1, one outer scale per expert: group_amax_nvfp4_kernel, grid rows / 128
+        _group_amax_replay(rows, cols, group_rows, in_mma, range(0, rows, 128), lambda r0: r0 // rpe, n_outer)
+    else:
+        # pass 1, one outer scale per output row (experts == 1): requant_amax_kernel, grid (cols / 64, rows / 128);
+        # thread (cl = t % 64, rg = t / 64) reads 32 rows of one column, target the column
+        for r0 in range(0, rows, 128):
+            for bx in range(cols // 64):
+                t = np.arange(T)
+                cl, rg = t & 63, t >> 6
+                c = bx * 64 + cl
+                rr = r0 + rg[:, None] * 32 + np.arange(32)[None, :]
+                assert rr.max() < rows and c.max() < cols
+                assert ((rr * cols + c[:, None]) // 2).max() < rows * cols // 2
+                offs = [sf_offset(int(a), int(cc) // 16, S_in, in_mma) for a, cc in zip(rr.reshape(-1),
+                                                                                        np.repeat(c, 32))]
+                assert min(offs) >= 0 and max(offs) < rows * S_in
+                assert c.max() < n_outer
+    # pass 2: the tile kernel; output row o = e * cols + c, its rpe columns the expert's rows
+    _requant_tile_replay(rows, cols, group_rows, in_mma, out_mma, lambda r0: True,
+                         lambda r0: (r0 - (r0 // rpe) * rpe, (r0 // rpe) * cols), rpe, experts * cols)
 
 
 @pytest.mark.parametrize("rows,cols,group_rows", [(64, 48, 32), (16, 16, 16), (128, 256, 128)])
@@ -145,7 +233,21 @@ def test_segment_kernels_indexing(M, C, seg, per_row, out_mma, in_mma, group_row
     assert np.all(seg % 128 == 0) and seg[-1] <= M and np.all(np.diff(seg) >= 0)
     end = seg[E]
     n_outer = E * C if per_row else E
-    # pass 1: grid (C / 64, M / 128); blocks at or past seg[E] leave before any barrier
+    # pass 1 of the bf16 source: segment_amax_bf16_kernel, grid (C / 64, M / 128); thread (k = t % 8,
+    # g = t / 8) loads 16 bytes of rows r0 + 4g .. r0 + 4g + 3 at column c0 + 8k
+    t = np.arange(T)
+    k8, g8 = t & 7, t >> 3
+    assert np.all(k8 == (t ^ 8) & 7) and np.all(k8 == (t ^ 16) & 7)   # the lanes a shuffle combines
+    for r0 in range(0, min(M, end), 128):
+        lo = _find_expert(seg, E, r0)
+        for bx in range(C // 64):
+            xi = ((r0 + 4 * g8[:, None] + np.arange(4)[None, :]) * C + bx * 64 + 8 * k8[:, None]).reshape(-1)
+            assert xi.min() >= 0 and (xi + 8).max() <= M * C and np.all(xi % 8 == 0)
+            _exactly_once(np.sort((xi // C - r0) * 64 + xi % C - bx * 64), 8, 128 * 64)
+            tg = lo * C + bx * 64 + np.arange(64) if per_row else np.array([lo])
+            assert tg.min() >= 0 and tg.max() < n_outer
+    # pass 1 of the NVFP4 source with per-row outer scales: segment_amax_kernel, grid (C / 64, M / 128);
+    # blocks at or past seg[E] leave before any barrier
     for by in range(M // 128):
         r0 = by * 128
         if r0 >= end:
@@ -162,19 +264,18 @@ def test_segment_kernels_indexing(M, C, seg, per_row, out_mma, in_mma, group_row
             assert max(offs) < M * (C // 16) and (rows // group_rows).max() < M // group_rows
             tg = lo * C + c if per_row else np.array([lo])
             assert tg.min() >= 0 and tg.max() < n_outer
-    # pass 2: one thread per output block of 16 tokens, c fastest
-    nb = M // 16
-    item = _threads(nb * C)
-    c, b = item % C, item // C
-    t0 = b * 16
-    assert (t0 + 15).max() < M
-    for tt in np.unique(t0[t0 < end]):
-        lo = _find_expert(seg, E, int(tt))
-        assert seg[lo] <= tt < seg[lo + 1]
-    _exactly_once((c * M + t0) // 2, 8, C * M // 2)
-    _exactly_once([sf_offset(int(a), int(bb), nb, out_mma) for a, bb in zip(c, b)], 1, C * nb)
-    L = (c * M + t0)[:, None] + np.arange(16)[None, :]
-    assert np.array_equal(np.sort(L.reshape(-1)), np.arange(C * M))
+    # pass 1 of the NVFP4 source with per-segment outer scales: group_amax_nvfp4_kernel over the live blocks
+    if not per_row:
+        _group_amax_replay(M, C, group_rows, in_mma, range(0, M, 128),
+                           lambda r0: None if r0 >= end else _find_expert(seg, E, r0), n_outer)
+    # pass 2: the tile kernel, output row c, its M columns the tokens; tiles past seg[E] only write zeros
+    for r0 in range(0, M, 128):
+        if r0 < end:
+            lo = _find_expert(seg, E, r0)
+            assert (lo * C + C - 1 if per_row else lo) < n_outer
+    _requant_tile_replay(M, C, group_rows, in_mma, out_mma, lambda r0: r0 < end, lambda r0: (r0, 0), M, C)
+    # pass 2 of the bf16 source: the same tile kernel with bf16 loads
+    _requant_tile_replay(M, C, 1, in_mma, out_mma, lambda r0: r0 < end, lambda r0: (r0, 0), M, C, bf16=True)
 
 
 @pytest.mark.parametrize("M,N,K,seg,pair", [
