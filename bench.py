@@ -732,7 +732,7 @@ def cpu_baseline(inp, seconds: float = 15.0):
 # single-kernel cases for ncu captures (small enough to profile, outputs
 # larger than L2 where DRAM traffic is read off)
 # --------------------------------------------------------------------------
-KERNEL_CASES = ("gemm_nvfp4", "gemm_nvfp4_s2f6", "gemm_mxfp8_dgrad", "gemm_mxfp8_wgrad", "requant", "requant_w",
+KERNEL_CASES = ("gemm_nvfp4", "gemm_nvfp4_s2f6", "gemm_nvfp4_down", "gemm_mxfp8_dgrad", "gemm_mxfp8_wgrad", "requant", "requant_w",
                 "nvfp4_quantize", "quant_w", "mxfp8_quantize", "nvfp4_quantize_sr", "requant_nvfp4", "gemm_nvfp4_wgrad",
                 "step_nvfp4_backward", "gemm1_moe_layer", "gemm2_moe_layer")
 
@@ -783,11 +783,15 @@ def run_kernel(args):
         w1q = api.nvfp4_quantize(w1, 2 * F, api.MX_SF_MMA)
         if which == "gemm_nvfp4":
             run = lambda: api.grouped_gemm_nvfp4(xp, w1q, seg, E, 2 * F, D)
-        elif which == "gemm_nvfp4_s2f6":
-            # the down projection (N = d_model, K = d_ff) with the rotate + S2F6 epilogue
+        elif which in ("gemm_nvfp4_s2f6", "gemm_nvfp4_down"):
+            # the down projection (N = d_model, K = d_ff) with the rotate + S2F6 epilogue, or with the bf16
+            # epilogue on the same operands
             a = api.nvfp4_quantize(workloads.activations(M, F, "t3", 4, dev), 1, api.MX_SF_MMA)
             w2q = api.nvfp4_quantize(workloads.weights(E, D, F, 0.02, 5, dev).view(E * D, F), D, api.MX_SF_MMA)
-            run = lambda: api.grouped_gemm_nvfp4_s2f6(a, w2q, seg, E, D, F, 1, 101)
+            if which == "gemm_nvfp4_s2f6":
+                run = lambda: api.grouped_gemm_nvfp4_s2f6(a, w2q, seg, E, D, F, 1, 101)
+            else:
+                run = lambda: api.grouped_gemm_nvfp4(a, w2q, seg, E, D, F)
         elif which == "gemm_nvfp4_wgrad":
             # dW1 in NVFP4 on the same routing with segments padded to 256 tokens: A = dH^T [2F, M256],
             # B = X^T [D, M256]; valid random codes and scales (the kernel's time does not depend on them)

@@ -413,8 +413,11 @@ struct Smem {
     // and get two buffers per warp unless giving up the second buys a
     // pipeline stage (operands in flight are what bound these kernels).
     static constexpr bool kOneBox = kOut == kOutTypeBF16 && stages_for(8 * 2048) > stages_for(8 * 4096);
-    // S2F6 boxes are 32 rows x 32 bytes: two 1 KB buffers per warp.
-    static constexpr int kStaging = kOut == kOutTypeS2F6 ? 8 * 2048 : (kOneBox ? 8 * 2048 : 8 * 4096);
+    // S2F6 boxes are 32 rows x 32 bytes: two 1 KB buffers per warp, then the
+    // tile's E8M0 bytes (128 rows x 8 bytes, two buffers).
+    static constexpr int kWarpStaging = kOut == kOutTypeS2F6 ? 2048 : (kOneBox ? 2048 : 4096);
+    static constexpr int kE8Bytes = kOut == kOutTypeS2F6 ? 2 * kBM * (kBN / 32) : 0;
+    static constexpr int kStaging = 8 * kWarpStaging + kE8Bytes;
     static constexpr int kStages = stages_for(kStaging);
     static constexpr int kStagingOff = kStages * kStage;
     static_assert(kStage % 1024 == 0 && kStagingOff % 1024 == 0, "128-byte swizzle needs 1024-byte aligned tiles");
@@ -464,6 +467,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     uint64_t* acc_free = acc_full + 2;           // [2]: see the epilogue (pair: both CTAs report)
     uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(acc_free + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
+    uint64_t* e8_ready = acc_free + 3;           // [4][2] S2F6: warp 12 + q wrote its E8M0 bytes into buffer b
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = kPair ? cluster_ctarank() : 0u;
@@ -485,6 +489,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             mbar_init(&sf_free[s], 1);
         }
         for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_free[b], kPair ? 16 : 8); }
+        for (int qq = 0; qq < 8; ++qq) mbar_init(&e8_ready[qq], 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
@@ -684,7 +689,16 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         const int q = warp & 3;
         const int h = (warp - 8) >> 2;
         const int r = q * 32 + lane;
-        uint8_t* stg = smem + L::kStagingOff + (warp - 8) * (L::kStaging / 8);
+        uint8_t* stg = smem + L::kStagingOff + (warp - 8) * L::kWarpStaging;
+        // S2F6: the E8M0 bytes of the tile's rows, [128][kBN / 32] per buffer;
+        // warp 8 + q stores each row's group of kBN / 32 bytes once warp 12 + q
+        // reported its half on e8_ready[q][buffer], one store per row instead
+        // of one per byte.  Buffers (and their barriers) alternate by stored
+        // tile: warp 12 + q reaches the next use of a buffer only after warp
+        // 8 + q released the tile that follows it, which it does after the
+        // store, so a barrier never runs a phase ahead of its waiter.
+        uint8_t* e8s = smem + L::kStagingOff + 8 * L::kWarpStaging;
+        uint32_t n_stored = 0;
         const uint32_t acc_free_lead[2] = {kPair ? map_to_rank(&acc_free[0], 0) : 0u,
                                            kPair ? map_to_rank(&acc_free[1], 0) : 0u};
         uint32_t it = 0, nbox = 0;
@@ -759,7 +773,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                         // stage the warp's 32 rows x 32 codes as one box (two 1 KB
                         // buffers per warp) and write it with a TMA tensor store; the
                         // exponent byte goes straight to global memory.
-                        const int64_t orow = t.row0 + r;
 #pragma unroll
                         for (int u = 0; u < 2; ++u) {
                             const int64_t ocol = t.col0 + col[u];
@@ -789,7 +802,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                                 asm volatile("cp.async.bulk.commit_group;" ::: "memory");
                             }
                             ++nbox;
-                            p.e8m0_out[orow * (p.ldo >> 5) + (ocol >> 5)] = (uint8_t)(e + 127);
+                            e8s[(n_stored & 1u) * (L::kE8Bytes / 2) + r * (kBN / 32) + (col[u] >> 5)] = (uint8_t)(e + 127);
                         }
                         continue;
                     }
@@ -843,6 +856,21 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                         ++nbox;
                     }
                 }
+            }
+            if (kOut == kOutTypeS2F6 && t.store) {
+                const uint8_t* src = e8s + (n_stored & 1u) * (L::kE8Bytes / 2) + r * (kBN / 32);
+                uint64_t* ready = &e8_ready[2 * q + (n_stored & 1u)];
+                if (h == 1) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(ready);
+                } else {
+                    if (!mbar_wait(ready, (n_stored >> 1) & 1u, abort_flag)) break;
+                    static_assert(kBN / 32 == 8 || kBN / 32 == 4, "E8M0 group of a tile row: one 8- or 4-byte store");
+                    uint8_t* dst = p.e8m0_out + (t.row0 + r) * (p.ldo >> 5) + (t.col0 >> 5);
+                    if (kBN / 32 == 8) *reinterpret_cast<uint2*>(dst) = *reinterpret_cast<const uint2*>(src);
+                    else *reinterpret_cast<uint32_t*>(dst) = *reinterpret_cast<const uint32_t*>(src);
+                }
+                ++n_stored;
             }
             ++it;
         }
@@ -1117,7 +1145,7 @@ extern "C" int grouped_gemm_nvfp4_s2f6(const uint8_t* a_codes, const uint8_t* a_
          M_cap > 0) || E < 1 || M_cap < 0 || M_cap % 128 || N <= 0 || N % 128 || K <= 0 || K % 256)
         return MX_EINVAL;
     if (!mx_aligned(a_codes, 16) || !mx_aligned(b_codes, 16) || !mx_aligned(a_sf, 16) || !mx_aligned(b_sf, 16) ||
-        !mx_aligned(codes, 16))
+        !mx_aligned(codes, 16) || !mx_aligned(e8m0, 8))
         return MX_EINVAL;
     if (M_cap >= (int64_t)1 << 31 || E * N >= (int64_t)1 << 31 || K / 2 >= (int64_t)1 << 31) return MX_EINVAL;
     if (int st = mx_check_device()) return st;

@@ -17,7 +17,9 @@
 //     outer scales of every backward GEMM factor out of its contraction.
 //
 // Every step is one IEEE fp32 round-to-nearest operation in the order the
-// oracle takes them; the stochastic rounding is done in software, exactly.
+// oracle takes them.  The stochastic rounding runs on the hardware cvt.rs
+// instruction for R = 16 and R = 8 (it computes the rule above exactly) and
+// in exact software arithmetic for R = 32.
 #include <type_traits>
 
 #include "mx_common.cuh"
@@ -55,6 +57,43 @@ __device__ __forceinline__ float e2m1_sr_magnitude(float y, uint32_t u) {
     return ((unsigned long long)u < __float2ull_rz(thr)) ? __fadd_rn(lo, q) : lo;
 }
 
+// Hardware stochastic rounding onto E2M1: sm_100a cvt.rs.satfinite.e2m1x4.f32
+// d, {a, b, c, f}, rbits puts f's code in bits 3:0 of d and b's in bits 11:8.
+// f adds the 16-bit random value rbits[23:16]:rbits[7:0], b the value
+// rbits[31:24]:rbits[15:8], just below the kept E2M1 bit, and truncates (the
+// carry rounds up).  With u the element's 16-bit integer, feeding 0xFFFF - u
+// rounds up exactly when u < floor(frac * 2^16): the rule of
+// e2m1_sr_magnitude<16>, signs and saturation included (established by
+// comparing the instruction with the oracle on a B200).  a and c share b's and
+// f's random bits and are not used.
+// Two elements: y_even in f, y_odd in b; codes y_even | y_odd << 8.
+__device__ __forceinline__ uint32_t cvt_rs_e2m1_pair(float y_even, float y_odd, uint32_t rbits) {
+    uint16_t d;
+    asm("cvt.rs.satfinite.e2m1x4.f32 %0, {%1, %2, %3, %4}, %5;"
+        : "=h"(d) : "f"(0.0f), "f"(y_odd), "f"(0.0f), "f"(y_even), "r"(rbits));
+    return d;
+}
+// rbits for elements 2k, 2k+1 whose 16-bit integers are the low and high
+// halves of word w (R = 16).
+__device__ __forceinline__ uint32_t rbits16_pair(uint32_t w) { return __byte_perm(~w, 0u, 0x3120); }
+// R = 8: element j's 8-bit integer u enters as the 16-bit value (255 - u) << 8,
+// which rounds up iff 256 u + 255 < floor(frac 2^16), i.e. iff u < floor(frac
+// 2^8): the R = 8 rule.  Elements 4k .. 4k + 3 are the bytes of word w; h = 0
+// takes the pair 4k, 4k + 1, h = 1 the pair 4k + 2, 4k + 3.
+__device__ __forceinline__ uint32_t rbits8_pair(uint32_t w, int h) {
+    return __byte_perm(~w, 0u, h ? 0x3244 : 0x1044);
+}
+// Eight code bytes from eight pair results (element 2j in the low nibble of byte j).
+__device__ __forceinline__ uint2 pack_e2m1_pairs(const uint32_t d[8]) {
+    uint32_t t[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const uint32_t w = d[2 * k] | (d[2 * k + 1] << 16);     // codes in the low nibbles of bytes 0 .. 3
+        t[k] = (w | (w >> 4)) & 0x00ff00ffu;                     // code bytes of the two pairs in bytes 0 and 2
+    }
+    return make_uint2(__byte_perm(t[0], t[1], 0x6420), __byte_perm(t[2], t[3], 0x6420));
+}
+
 // One 16-value block: E4M3 scale of bmax / (6 s) (0 when s == 0) and the
 // eight code bytes, element 2j in the low nibble of byte j.  L0 is the linear
 // output index of element 0 (for the random integers), a multiple of 16.
@@ -74,6 +113,30 @@ __device__ __forceinline__ void quantize_block16(const float* v, float s, uint64
     if constexpr (!kSR) {
         packed.x = cvt_e2m1x8(y);
         packed.y = cvt_e2m1x8(y + 8);
+    } else if constexpr (R == 16) {
+        // L0 is a multiple of 16: the block's random integers are the 16-bit halves of two Philox blocks,
+        // elements 2k and 2k + 1 in word k % 4 of block k / 4
+        uint32_t d[8];
+#pragma unroll
+        for (int blk = 0; blk < 2; ++blk) {
+            const uint4 rnd = philox4x32_10(L0 / 8 + blk, stream_id, seed);
+            const uint32_t w[4] = {rnd.x, rnd.y, rnd.z, rnd.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                d[4 * blk + k] = cvt_rs_e2m1_pair(y[8 * blk + 2 * k], y[8 * blk + 2 * k + 1], rbits16_pair(w[k]));
+        }
+        packed = pack_e2m1_pairs(d);
+    } else if constexpr (R == 8) {
+        // one Philox block: elements 4k .. 4k + 3 are the bytes of word k
+        const uint4 rnd = philox4x32_10(L0 / 16, stream_id, seed);
+        const uint32_t w[4] = {rnd.x, rnd.y, rnd.z, rnd.w};
+        uint32_t d[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            d[2 * k] = cvt_rs_e2m1_pair(y[4 * k], y[4 * k + 1], rbits8_pair(w[k], 0));
+            d[2 * k + 1] = cvt_rs_e2m1_pair(y[4 * k + 2], y[4 * k + 3], rbits8_pair(w[k], 1));
+        }
+        packed = pack_e2m1_pairs(d);
     } else {
         // magnitudes on the grid are encoded exactly; the sign of y is kept,
         // also where the magnitude is zero

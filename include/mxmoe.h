@@ -369,7 +369,8 @@ MX_API int hadamard_s2f6_quantize(const void* x, int64_t rows, int64_t cols, uin
  * and quantised per 32-column block as above, in the registers that drain
  * the accumulator.  Arguments and requirements as grouped_gemm_nvfp4, the
  * output being codes int8 [M_cap, N] and e8m0 u8 [M_cap, N/32] (rows of
- * padding hold codes of zero sums).  codes 16-byte aligned. */
+ * padding hold codes of zero sums).  codes 16-byte and e8m0 8-byte aligned;
+ * else MX_EINVAL. */
 MX_API int grouped_gemm_nvfp4_s2f6(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_outer,
                                    const uint8_t* b_codes, const uint8_t* b_sf, const float* b_outer,
                                    const int64_t* seg_offsets, int64_t E, int64_t M_cap, int64_t N, int64_t K,

@@ -91,7 +91,7 @@ CASES = {
     ]),
     "grouped_gemm_nvfp4_s2f6": ((A, A, A, A, A, A, A, 1, 128, 128, 256, 1, 2, A, A, None), [
         ("K % 256", {10: 128}), ("N % 128", {9: 64}), ("codes misaligned", {13: A8}), ("null e8m0", {14: None}),
-        ("M_cap % 128", {8: 64}),
+        ("M_cap % 128", {8: 64}), ("e8m0 misaligned", {14: A4}),
     ]),
     "moe_combine_s2f6": ((A, A, A, None, 16, 2, 64, 1, 2, A, None), [
         ("D % 32", {6: 48}), ("k 0", {5: 0}), ("out misaligned", {9: A8}), ("null codes", {0: None}),

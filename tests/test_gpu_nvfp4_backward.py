@@ -53,6 +53,47 @@ def test_nvfp4_quantize_sr_bit_exact(cuda, rows, cols, group_rows, layout, rbits
     assert np.array_equal(host(c), rc)
 
 
+def edge_input(rows, cols, seed):
+    """Blocks that reach the rounding's special cases: the block maximum and
+    values down to bf16 subnormals (scaled values below fp32's normal range),
+    signed zeros, values on the E2M1 grid of their block (k/6 of the maximum),
+    values just above 6 after scaling (the block scale rounded down), and
+    saturating blocks."""
+    rng = np.random.default_rng(seed)
+    x = np.zeros((rows, cols), np.float64)
+    for r in range(rows):
+        for b in range(cols // 16):
+            kind = (r + b) % 5
+            big = 10.0 ** rng.uniform(-2, 3)
+            v = rng.standard_normal(16) * big
+            if kind == 0:                                        # tiny neighbours of a large maximum
+                v[1:] = np.ldexp(rng.uniform(1, 2, 15), rng.integers(-133, -110, 15))
+            elif kind == 1:                                      # grid points of the block
+                v = big * np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6] * 2) / 6 * rng.choice([-1, 1], 16)
+            elif kind == 2:                                      # signed zeros with one nonzero
+                v[:] = -0.0
+                v[7] = big
+            elif kind == 3:                                      # a maximum whose scale rounds down
+                v[0] = big * 1.0624
+                v[1:] = big * rng.uniform(0.9, 1.0, 15)
+            v[0] = abs(v[0]) if kind != 2 else v[0]
+            x[r, 16 * b:16 * b + 16] = v
+    return oracle.f32_to_bf16(x.astype(np.float32))
+
+
+@pytest.mark.parametrize("rbits", [8, 16, 32])
+def test_nvfp4_quantize_sr_edge_values_bit_exact(cuda, rbits):
+    rows, cols = 256, 256
+    x = edge_input(rows, cols, 40 + rbits)
+    seed, stream = 77, 3
+    c, sf, o = api.nvfp4_quantize_sr(to_dev_bf16(x), 1, api.MX_ROUND_SR, seed, stream, rbits, api.MX_SF_MMA)
+    api.sync_status()
+    rc, rsf, ro = oracle.nvfp4_quantize_f32(oracle.bf16_to_f32(x), 1, True, seed, stream, rbits)
+    assert np.array_equal(host(o), ro)
+    assert np.array_equal(mma_to_rowmajor(host(sf), rows, cols // 16), rsf)
+    assert np.array_equal(host(c), rc)
+
+
 def test_nvfp4_quantize_sr_rne_equals_the_forward_quantiser(cuda):
     x = to_dev_bf16(bf16_input(256, 256, 3))
     a = api.nvfp4_quantize_sr(x, 1, api.MX_ROUND_RNE)
