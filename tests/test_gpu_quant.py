@@ -100,6 +100,22 @@ def test_nvfp4_quantize_per_expert_bit_exact(cuda, E, N, K):
     assert np.array_equal(np_(go).view(np.uint32), outer.view(np.uint32))
 
 
+@pytest.mark.parametrize("E,N,K", [(2, 16, 64), (64, 128, 256), (5, 2048, 4096)])
+def test_nvfp4_quantize_per_expert_group_sizes(cuda, E, N, K):
+    # two tiny groups, 64 small groups, five 16.8 MB groups; experts decades
+    # apart so that a scale from another group changes codes
+    w = workloads.weights(E, N, K, 0.02, seed=E * 7 + N + K).float()
+    w *= (10.0 ** torch.linspace(-2, 2, E)).view(E, 1, 1)
+    w = w.to(torch.bfloat16)
+    wn = w.reshape(E * N, K).view(torch.int16).numpy().view(np.uint16)
+    codes, sf, outer = oracle.nvfp4_quantize(wn, group_rows=N)
+    gc, gsf, go = api.nvfp4_quantize(w.reshape(E * N, K).cuda(), group_rows=N, sf_layout=api.MX_SF_ROWMAJOR)
+    api.sync_status()
+    assert np.array_equal(np_(go).view(np.uint32), outer.view(np.uint32))
+    assert np.array_equal(np_(gsf).reshape(sf.shape), sf)
+    assert np.array_equal(np_(gc), codes)
+
+
 def test_nvfp4_quantize_per_expert_unaligned_groups(cuda):
     # 3 experts of 2046 x 4096 (16.8 MB each): expert boundaries fall inside a
     # block of rows of the quantiser, with row-major scales
