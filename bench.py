@@ -234,6 +234,7 @@ def stage_work(c, counts, M_pad):
         "combine": ("hbm", R * D * 2 + T * D * 2),
         "dispatch_grad": ("hbm", T * D * 2 + R * D * 2),
         "quant_dy2": ("hbm", R * D * 2 + 2 * mx(R, D)),
+        "dispatch_grad_quant": ("hbm", T * D * 2 + 2 * mx(R, D)),  # dispatch gradient + MXFP8 in one kernel
         "requant_w2": ("alu", (nv(E * D, F) + mx(E * D, F), (E * D) * (F))),
         "dgrad2": ("tensor8", 2 * R * F * D),
         "requant_a": ("alu", (nv(R, F) + mx(R, F), (R) * (F))),

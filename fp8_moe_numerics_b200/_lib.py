@@ -52,6 +52,7 @@ SIGNATURES = {
     "swiglu_nvfp4_quantize": (I32, [P, I64, I64, I32, P, P, P, P, I32, P]),
     "moe_combine": (I32, [P, P, P, I64, I64, I64, P, P]),
     "moe_dispatch_grad": (I32, [P, P, P, P, I64, I64, I64, I64, P, P]),
+    "moe_dispatch_grad_mxfp8_quantize": (I32, [P, P, P, I64, I64, I64, I64, P, P, P, P, P, I32, P]),
     "hadamard_s2f6_quantize": (I32, [P, I64, I64, U64, U64, P, P, P]),
     "grouped_gemm_nvfp4_s2f6": (I32, [P, P, P, P, P, P, P, I64, I64, I64, I64, U64, U64, P, P, P]),
     "moe_combine_s2f6": (I32, [P, P, P, P, I64, I64, I64, U64, U64, P, P]),

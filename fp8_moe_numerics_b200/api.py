@@ -312,6 +312,33 @@ def moe_dispatch_grad(dout: torch.Tensor, src: torch.Tensor, pos: torch.Tensor, 
     return out
 
 
+def _mxfp8_pair_out(rows: int, cols: int, sf_layout: int, dev, out):
+    """The four outputs of an MXFP8 quantisation of [rows, cols] (both forms)."""
+    if out is None:
+        out = (torch.empty(rows, cols, dtype=torch.uint8, device=dev), _u8(sf_bytes(rows, cols, 32, sf_layout), dev),
+               torch.empty(cols, rows, dtype=torch.uint8, device=dev), _u8(sf_bytes(cols, rows, 32, sf_layout), dev))
+    rc, re, cc, ce = out
+    _fits("row codes", rc, rows * cols)
+    _fits("row e8m0", re, rows * (cols // 32))
+    _fits("col codes", cc, rows * cols)
+    _fits("col e8m0", ce, cols * (rows // 32))
+    return out
+
+
+def moe_dispatch_grad_mxfp8_quantize(dout: torch.Tensor, src: torch.Tensor, w, k: int, rows_valid=None,
+                                     sf_layout: int = MX_SF_MMA, out=None):
+    """mxfp8_quantize(moe_dispatch_grad(dout, src, pos, w), RNE, both forms, rows_valid) without the bf16 dy:
+    (row codes, row E8M0, col codes, col E8M0) of dy [M_cap, D]."""
+    M_cap = src.shape[0]
+    T, D = dout.shape
+    _fits("w", w, 4 * T * k)
+    _fits("rows_valid", rows_valid, 8)
+    rc, re, cc, ce = _mxfp8_pair_out(M_cap, D, sf_layout, dout.device, out)
+    L.call("moe_dispatch_grad_mxfp8_quantize", _p(dout), _p(src), _p(w), T, k, M_cap, D, _p(rows_valid), _p(rc),
+           _p(re), _p(cc), _p(ce), sf_layout, _s())
+    return rc, re, cc, ce
+
+
 def hadamard_s2f6_quantize(x: torch.Tensor, seed: int, stream_id: int, out=None):
     """bf16 [rows, cols] -> (codes int8 [rows, cols], e8m0 u8 [rows, cols/32]):
     32-d random Hadamard rotation per column block, block-scaled S2F6."""

@@ -149,11 +149,6 @@ __global__ void gather_rows_kernel(const uint8_t* __restrict__ codes, const uint
     if (lane == 0) out_outer[p] = t < 0 ? 0.0f : outer[t];
 }
 
-__device__ __forceinline__ float dsilu_f(float g) {
-    const float s = sigmoid_f(g);
-    return s * (1.0f + g * (1.0f - s));
-}
-
 
 // 8 outputs per thread.
 __global__ void swiglu_fwd_kernel(const uint16_t* __restrict__ h, int64_t rows, int64_t F, int gated,
@@ -201,11 +196,8 @@ __global__ void swiglu_bwd_kernel(const uint16_t* __restrict__ h, const uint16_t
         uint32_t wg[4], wu[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const float g0 = bf16_lo(gw[j]), g1 = bf16_hi(gw[j]);
-            const float d0 = bf16_lo(dw[j]), d1 = bf16_hi(dw[j]);
-            const float u0 = bf16_lo(uw[j]), u1 = bf16_hi(uw[j]);
-            wg[j] = pack_bf16x2(d0 * u0 * dsilu_f(g0), d1 * u1 * dsilu_f(g1));
-            wu[j] = pack_bf16x2(d0 * silu_f(g0), d1 * silu_f(g1));
+            wg[j] = swiglu_bwd_gate_word(gw[j], uw[j], dw[j]);
+            wu[j] = swiglu_bwd_up_word(gw[j], dw[j]);
         }
         og = make_uint4(wg[0], wg[1], wg[2], wg[3]);
         ou = make_uint4(wu[0], wu[1], wu[2], wu[3]);
@@ -261,10 +253,8 @@ dispatch_grad_kernel(const uint16_t* __restrict__ dout, const int32_t* __restric
             for (int64_t j = 0; j < k; ++j) {
                 if (sp[j] < 0 || !mx_in_range((int64_t)sp[j] * D + c, 8, M_cap * D)) continue;   // left out
                 const float wj = sw[j];
-                const uint4 o = make_uint4(pack_bf16x2(wj * bf16_lo(v.x), wj * bf16_hi(v.x)),
-                                           pack_bf16x2(wj * bf16_lo(v.y), wj * bf16_hi(v.y)),
-                                           pack_bf16x2(wj * bf16_lo(v.z), wj * bf16_hi(v.z)),
-                                           pack_bf16x2(wj * bf16_lo(v.w), wj * bf16_hi(v.w)));
+                const uint4 o = make_uint4(scaled_bf16_word(wj, v.x), scaled_bf16_word(wj, v.y),
+                                           scaled_bf16_word(wj, v.z), scaled_bf16_word(wj, v.w));
                 *reinterpret_cast<uint4*>(dy + (int64_t)sp[j] * D + c) = o;
             }
         }

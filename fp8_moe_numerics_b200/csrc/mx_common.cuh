@@ -228,6 +228,27 @@ __device__ __forceinline__ uint32_t swiglu_word(uint32_t g, uint32_t u) {
     return pack_bf16x2(silu_f(bf16_lo(g)) * bf16_lo(u), silu_f(bf16_hi(g)) * bf16_hi(u));
 }
 
+__device__ __forceinline__ float dsilu_f(float g) {
+    const float s = sigmoid_f(g);
+    return s * (1.0f + g * (1.0f - s));
+}
+
+// The SwiGLU backward of two elements from bf16 pairs of the gate g, the up
+// projection u and the upstream gradient d: dg = d u silu'(g) and du =
+// d silu(g), each rounded to bf16 (the one definition the standalone kernel
+// and the fused MXFP8 quantiser share).
+__device__ __forceinline__ uint32_t swiglu_bwd_gate_word(uint32_t g, uint32_t u, uint32_t d) {
+    return pack_bf16x2(bf16_lo(d) * bf16_lo(u) * dsilu_f(bf16_lo(g)), bf16_hi(d) * bf16_hi(u) * dsilu_f(bf16_hi(g)));
+}
+__device__ __forceinline__ uint32_t swiglu_bwd_up_word(uint32_t g, uint32_t d) {
+    return pack_bf16x2(bf16_lo(d) * silu_f(bf16_lo(g)), bf16_hi(d) * silu_f(bf16_hi(g)));
+}
+
+// The dispatch gradient of two elements: w * dout, rounded to bf16.
+__device__ __forceinline__ uint32_t scaled_bf16_word(float w, uint32_t v) {
+    return pack_bf16x2(w * bf16_lo(v), w * bf16_hi(v));
+}
+
 // ---------------------------------------------------------------------------
 // MXFP8 block exponent: smallest e with amax <= 448 * 2^e, clamped to
 // [-127, 127]; -127 for amax == 0.  448 = 1.75 * 2^8, so for a normal

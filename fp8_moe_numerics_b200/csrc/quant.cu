@@ -487,6 +487,106 @@ mxfp8_tile_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, co
 
 
 // ---------------------------------------------------------------------------
+// MXFP8 (RNE) row and column forms of the dispatch gradient, formed on the fly
+// from the upstream gradient and the routing so that dY itself never goes
+// through HBM.  The tile walk and both forms are mxfp8_tile_kernel's; each
+// thread's row is gathered from its token's row of dout (the next tile's
+// loads issued before the current tile's transposed phase, their scaling at
+// the top of the next iteration).  Every value is w * dout rounded to bf16 by
+// the definition moe_dispatch_grad uses (scaled_bf16_word), so the codes equal
+// those of moe_dispatch_grad and mxfp8_quantize run one after the other.
+// Row p holds w[s] * dout[s / k] for s = src[p] >= 0, else zeros; a token's
+// row is read by its k rows (kept in L2).
+// ---------------------------------------------------------------------------
+struct DispatchGradRows {
+    const uint16_t* dout;
+    const int32_t* src;
+    const float* w;
+    int64_t Tk, k, D;
+    struct Raw {
+        uint4 v[4];
+        float wt;
+        bool live;
+    };
+    // the thread's 32 columns c .. c + 31 of row r
+    __device__ __forceinline__ void issue(int64_t r, int64_t c, int64_t valid, Raw& q) const {
+        q.live = false;
+        if (r >= valid) return;
+        const int64_t s = __ldg(src + r);
+        if (s < 0 || s >= Tk) return;
+        q.live = true;
+        q.wt = w ? __ldg(w + s) : 1.0f;
+        const uint4* vp = reinterpret_cast<const uint4*>(dout + (s / k) * D + c);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) q.v[i] = __ldg(vp + i);
+    }
+    __device__ __forceinline__ void finish(const Raw& q, uint4* out) const {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            out[i] = q.live ? make_uint4(scaled_bf16_word(q.wt, q.v[i].x), scaled_bf16_word(q.wt, q.v[i].y),
+                                         scaled_bf16_word(q.wt, q.v[i].z), scaled_bf16_word(q.wt, q.v[i].w))
+                            : make_uint4(0u, 0u, 0u, 0u);
+    }
+};
+
+template <int kLayout>
+__global__ void __launch_bounds__(kTileThreads, 2)
+dispatch_grad_mxfp8_kernel(DispatchGradRows src, int64_t rows, int64_t cols, const int64_t* rows_valid,
+                           uint8_t* __restrict__ row_codes, uint8_t* __restrict__ row_e8m0,
+                           uint8_t* __restrict__ col_codes, uint8_t* __restrict__ col_e8m0) {
+    __shared__ __align__(16) float T[kTC * kTR];
+    const int64_t valid = load_rows_valid(rows_valid, rows);
+    const int64_t tiles_c = cols / kTC;
+    const int64_t ntiles = tiles_c * ((valid + kTR - 1) / kTR);
+    int64_t tile = blockIdx.x;
+    if (tile >= ntiles) return;
+    const int t = threadIdx.x;
+    const int rl = t >> 1, h = t & 1;
+    DispatchGradRows::Raw raw;
+    auto issue = [&](int64_t tl) { src.issue((tl / tiles_c) * kTR + rl, (tl % tiles_c) * kTC + 32 * h, valid, raw); };
+    issue(tile);
+    for (; tile < ntiles; tile += gridDim.x) {
+        const int64_t c0 = (tile % tiles_c) * kTC, r0 = (tile / tiles_c) * kTR;
+        const int64_t r = r0 + rl, c = c0 + 32 * h;
+        uint4 q[4];
+        src.finish(raw, q);
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t w[4] = {q[i].x, q[i].y, q[i].z, q[i].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) { v[8 * i + 2 * j] = bf16_lo(w[j]); v[8 * i + 2 * j + 1] = bf16_hi(w[j]); }
+        }
+        {                                                  // row-wise block, RNE (as mxfp8_tile_kernel)
+            uint32_t m = 0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) m = max(m, absmax8_bf16(q[i]));
+            const int e = e8m0_exponent(__uint_as_float(m << 16));
+            const float sc = exp2_neg(e);
+            const uint64_t sc2 = f2_pack(sc, sc);
+            uint32_t w[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                float a0 = v[4 * i], a1 = v[4 * i + 1], a2 = v[4 * i + 2], a3 = v[4 * i + 3];
+                mul2_rn(a0, a1, sc2);
+                mul2_rn(a2, a3, sc2);
+                w[i] = cvt_e4m3x4(a0, a1, a2, a3);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(row_codes + r * cols + c);
+            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+            dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+            row_e8m0[sf_offset(r, c >> 5, cols >> 5, kLayout)] = (uint8_t)(e + 127);
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) T[tsw(32 * h + i, rl)] = v[i];
+        __syncthreads();
+        if (tile + gridDim.x < ntiles) issue(tile + gridDim.x);
+        tile_emit_transposed<false, 8, kLayout>(T, rows, cols, r0, c0, 0, 0, col_codes, col_e8m0);
+        __syncthreads();                                   // T is rewritten by the next tile
+    }
+}
+
+// ---------------------------------------------------------------------------
 // MXFP8 quantiser (RNE), fed by TMA.  A persistent block of 8 consumer warps
 // and one producer warp walks the same 128 x 64 tiles as mxfp8_tile_kernel.
 // The producer's lane 0 keeps kQStages bf16 tiles in flight with 2-D TMA
@@ -1029,6 +1129,36 @@ extern "C" int mxfp8_requant_transpose_sr(const uint8_t* codes, const uint8_t* s
             mx_count_launch();
             return mx_launch_status();
         });
+    });
+}
+
+extern "C" int moe_dispatch_grad_mxfp8_quantize(const void* dout, const int32_t* src, const float* w, int64_t T,
+                                                int64_t k, int64_t M_cap, int64_t D, const int64_t* rows_valid,
+                                                uint8_t* row_codes, uint8_t* row_e8m0, uint8_t* col_codes,
+                                                uint8_t* col_e8m0, int sf_layout, cudaStream_t stream) {
+    MX_NVTX_RANGE("moe_dispatch_grad_mxfp8_quantize");
+    if (((!dout || !src || !row_codes || !row_e8m0 || !col_codes || !col_e8m0) && M_cap > 0) || T < 0 || k <= 0 ||
+        M_cap < 0 || M_cap % kTR || D <= 0 || D % 128 || !mx_aligned(dout, 16) || !mx_aligned(row_codes, 16) ||
+        !mx_aligned(col_codes, 16))
+        return MX_EINVAL;
+    if (sf_layout != MX_SF_ROWMAJOR && sf_layout != MX_SF_MMA) return MX_EINVAL;
+    if (T > ((int64_t)1 << 40) / k) return MX_EINVAL;
+    if (int st = mx_check_device()) return st;
+    if (M_cap == 0) return MX_OK;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const DispatchGradRows rows_src{static_cast<const uint16_t*>(dout), src, w, T * k, k, D};
+    return dispatch_layout(sf_layout, [&](auto L) {
+        constexpr int kL = decltype(L)::value;
+        auto kern = dispatch_grad_mxfp8_kernel<kL>;
+        int occ = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kTileThreads, 0) != cudaSuccess || occ <= 0)
+            occ = 2;
+        const dim3 grid((unsigned)std::min<int64_t>((D / kTC) * (M_cap / kTR), (int64_t)sms * occ));
+        kern<<<grid, kTileThreads, 0, stream>>>(rows_src, M_cap, D, rows_valid, row_codes, row_e8m0, col_codes,
+                                                col_e8m0);
+        mx_count_launch();
+        return mx_launch_status();
     });
 }
 

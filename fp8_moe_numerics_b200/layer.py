@@ -46,13 +46,16 @@ class ExpertLayer:
     pages' recipe) or "nvfp4": the four backward GEMMs in NVFP4 with
     stochastically rounded operands (the pages' stated future work; routing
     then pads experts to 256 rows for the NVFP4 wgrad's K-stage).
+    `fuse_backward` (MXFP8 backward) forms the dispatch gradient inside the
+    gradient quantiser's kernel: the same codes, without the bf16 dy2
+    (allocated only with fuse_backward=False or the NVFP4 backward).
     """
 
     S2F6_STREAM = 101                                   # Philox stream of the rotation's signs
 
     def __init__(self, x, topk, w_comb, w1, w2, dout, gated: bool = True, seed: int = 0,
                  wgrad_dtype=torch.bfloat16, out_dtype=torch.bfloat16, rbits: int = 16, combine: str = "bf16",
-                 fuse_swiglu: bool = True, backward: str = "mxfp8"):
+                 fuse_swiglu: bool = True, backward: str = "mxfp8", fuse_backward: bool = True):
         if combine not in ("bf16", "s2f6"):
             raise ValueError(f"combine must be 'bf16' or 's2f6', got {combine!r}")
         if backward not in ("mxfp8", "nvfp4"):
@@ -61,6 +64,7 @@ class ExpertLayer:
         self.align = 256 if backward == "nvfp4" else 128
         self.combine = combine
         self.fuse_swiglu = fuse_swiglu
+        self.fuse_backward = fuse_backward and backward == "mxfp8"
         dev = x.device
         self.dev = dev
         self.T, self.D = x.shape
@@ -97,7 +101,7 @@ class ExpertLayer:
             self.y2 = e(M, D, dt=out_dtype)
         self.out = e(T, D, dt=torch.bfloat16)
         # backward
-        self.dy2 = e(M, D, dt=torch.bfloat16)
+        self.dy2 = None if self.fuse_backward else e(M, D, dt=torch.bfloat16)
         self.dy2q = (e(M, D), e(sfb(M, D, 32, MX_SF_MMA)), e(D, M), e(sfb(D, M, 32, MX_SF_MMA)))
         self.w2t = (e(F, E * D), e(sfb(F, E * D, 32, MX_SF_MMA)))
         self.da = e(M, F, dt=torch.bfloat16)
@@ -191,10 +195,14 @@ class ExpertLayer:
         T, D, k, E, F, N1, M = self.T, self.D, self.k, self.E, self.F, self.N1, self.M_cap
         s, R = self.seed, self.rbits
         self._mark("bwd_start", record)
-        api.moe_dispatch_grad(self.dout, self.src, self.pos, self.w_comb, out=self.dy2)
-        self._mark("dispatch_grad", record)
-        api.mxfp8_quantize(self.dy2, rows_valid=self.rows_valid, rounding=MX_ROUND_RNE, out=self.dy2q)
-        self._mark("quant_dy2", record)
+        if self.fuse_backward:
+            api.moe_dispatch_grad_mxfp8_quantize(self.dout, self.src, self.w_comb, k, self.rows_valid, out=self.dy2q)
+            self._mark("dispatch_grad_quant", record)
+        else:
+            api.moe_dispatch_grad(self.dout, self.src, self.pos, self.w_comb, out=self.dy2)
+            self._mark("dispatch_grad", record)
+            api.mxfp8_quantize(self.dy2, rows_valid=self.rows_valid, rounding=MX_ROUND_RNE, out=self.dy2q)
+            self._mark("quant_dy2", record)
         api.mxfp8_requant_transpose_sr(*self.w2q, E * D, F, D, MX_SF_MMA, None, s, 1, R, out=self.w2t)
         self._mark("requant_w2", record)
         api.grouped_gemm_mxfp8(MX_GEMM_DGRAD, self.dy2q[0], self.dy2q[1], *self.w2t, self.seg, E, M, F, D, out=self.da)

@@ -333,6 +333,22 @@ MX_API int moe_combine(const void* y, const int32_t* pos, const float* w, int64_
 MX_API int moe_dispatch_grad(const void* dout, const int32_t* src, const int32_t* pos, const float* w, int64_t T,
                              int64_t k, int64_t M_cap, int64_t D, void* dy, cudaStream_t stream);
 
+/* moe_dispatch_grad_mxfp8_quantize -- moe_dispatch_grad fused into the
+ * gradient quantiser that follows it ([ai-primer §NVFP4 forward, MXFP8
+ * backward]: the gradients enter the backward GEMMs as MXFP8).  Writes what
+ * moe_dispatch_grad(dout, src, ., w) followed by mxfp8_quantize (MX_ROUND_RNE,
+ * both forms, the same rows_valid) of dy [M_cap, D] writes, byte for byte,
+ * without dy reaching HBM: each row is gathered from its token's row of dout
+ * and scaled as moe_dispatch_grad scales it.  Outputs as mxfp8_quantize:
+ * row_codes [M_cap, D], row_e8m0, col_codes [D, M_cap], col_e8m0
+ * (sf_layout); row tiles at or past *rows_valid are not written.  Requires
+ * M_cap % 128 == 0, D % 128 == 0, k >= 1, all four outputs, dout and codes
+ * 16-byte aligned; else MX_EINVAL. */
+MX_API int moe_dispatch_grad_mxfp8_quantize(const void* dout, const int32_t* src, const float* w, int64_t T,
+                                            int64_t k, int64_t M_cap, int64_t D, const int64_t* rows_valid,
+                                            uint8_t* row_codes, uint8_t* row_e8m0, uint8_t* col_codes,
+                                            uint8_t* col_e8m0, int sf_layout, cudaStream_t stream);
+
 /* --------------------------------------------------------------------------
  * Combine path in S2F6.  [ai-primer §Quantized NVLink and BBBK]: expert
  * outputs are rotated by a 32-dimensional random Hadamard transform and

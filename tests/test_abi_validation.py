@@ -83,6 +83,10 @@ CASES = {
     "moe_combine": ((A, A, None, 16, 2, 64, A, None), [
         ("D % 8", {5: 12}), ("k 0", {4: 0}), ("null y", {0: None}), ("out misaligned", {6: A8}),
     ]),
+    "moe_dispatch_grad_mxfp8_quantize": ((A, A, None, 16, 2, 128, 128, None, A, A, A, A, 1, None), [
+        ("M_cap % 128", {5: 64}), ("D % 128", {6: 64}), ("k 0", {4: 0}), ("dout misaligned", {0: A8}),
+        ("null src", {1: None}), ("row codes misaligned", {8: A8}), ("unknown layout", {12: 5}),
+    ]),
     "moe_dispatch_grad": ((A, A, A, None, 16, 2, 128, 64, A, None), [
         ("k > 32", {5: 33}), ("D % 8", {7: 4}), ("dy misaligned", {8: A8}), ("negative M_cap", {6: -1}),
     ]),

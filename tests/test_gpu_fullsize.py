@@ -266,13 +266,12 @@ def test_moe_layer_step_full_size(cuda):
 
     # combine gradient and its row-wise MXFP8 form, sampled rows of true tokens and padding
     dout, w = u16(inp["dout"]), np_(inp["w_comb"])
-    dy2, dy2c, dy2e = u16(L.dy2), np_(L.dy2q[0]), mma_rows(np_(L.dy2q[1]), p, D // 32)
+    dy2c, dy2e = np_(L.dy2q[0]), mma_rows(np_(L.dy2q[1]), p, D // 32)
     for i, row in enumerate(p):
         s = int(copy_of[row])                                          # t*k + j, or -1 on padding
         if s >= 0:
             ref = oracle.dispatch_grad(dout[s // k][None], np.zeros((1, 1), np.int32), w[s // k, s % k].reshape(1, 1), 1)
         else:
             ref = np.zeros((1, D), np.uint16)
-        assert np.array_equal(dy2[row], ref[0])
         rc, re = oracle.mxfp8_quantize_rows(ref)
         assert np.array_equal(dy2c[row], rc[0]) and np.array_equal(dy2e[i], re[0])

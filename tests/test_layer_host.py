@@ -36,6 +36,18 @@ def host_calls(monkeypatch):
     return calls
 
 
+def test_unfused_backward_sequence_passes_host_validation(host_calls):
+    inp = workloads.layer_inputs("tiny_layer", device="cpu")
+    c = inp["cfg"]
+    L = ExpertLayer(inp["x"], inp["topk"], inp["w_comb"], inp["w1"], inp["w2"], inp["dout"], gated=c["gated"],
+                    fuse_backward=False)
+    L.step()
+    names = [n for n, _ in host_calls]
+    assert names.count("moe_dispatch_grad") == 1 and names.count("swiglu_bwd") == 1
+    assert names.count("mxfp8_quantize") == 2 and len(names) == 22
+    assert all(st == _lib.MX_ECUDA for _, st in host_calls)
+
+
 @pytest.mark.parametrize("name", ["tiny_layer"])
 def test_layer_sequence_passes_host_validation(host_calls, name):
     inp = workloads.layer_inputs(name, device="cpu")
@@ -47,7 +59,10 @@ def test_layer_sequence_passes_host_validation(host_calls, name):
     assert names.count("grouped_gemm_nvfp4") == 2 and names.count("grouped_gemm_mxfp8") == 4
     assert names.count("mxfp8_requant_transpose_sr") == 4
     assert names.count("swiglu_nvfp4_quantize") == 1 and "swiglu_fwd" not in names   # fused by default
-    assert len(names) == 22
+    # the dispatch gradient fused into its quantiser by default
+    assert names.count("moe_dispatch_grad_mxfp8_quantize") == 1 and "moe_dispatch_grad" not in names
+    assert names.count("swiglu_bwd") == 1 and names.count("mxfp8_quantize") == 1
+    assert len(names) == 21
     assert all(st == _lib.MX_ECUDA for _, st in host_calls)   # valid, and no device here
 
 
@@ -62,7 +77,7 @@ def test_s2f6_combine_sequence_passes_host_validation(host_calls):
     # the forward combine reads S2F6; the backward's un-permute of dX stays a bf16 combine
     assert names.count("moe_combine_s2f6") == 1 and names.count("moe_combine") == 1
     assert names.index("moe_combine_s2f6") == names.index("grouped_gemm_nvfp4_s2f6") + 1
-    assert len(names) == 22
+    assert len(names) == 21
     assert all(st == _lib.MX_ECUDA for _, st in host_calls)
 
 
@@ -75,11 +90,11 @@ def test_unfused_swiglu_sequence_passes_host_validation(host_calls):
     names = [n for n, _ in host_calls]
     assert "swiglu_nvfp4_quantize" not in names and names.count("swiglu_fwd") == 1
     assert names.count("nvfp4_quantize") == 4                   # tokens, W1, W2, activations
-    assert len(names) == 23
+    assert len(names) == 22
     assert all(st == _lib.MX_ECUDA for _, st in host_calls)
 
 
-@pytest.mark.parametrize("opts", [{}, {"fuse_swiglu": False}, {"combine": "s2f6"}])
+@pytest.mark.parametrize("opts", [{}, {"fuse_swiglu": False}, {"combine": "s2f6"}, {"fuse_backward": False}])
 def test_every_marked_stage_has_work_in_bench(host_calls, monkeypatch, opts):
     # bench.py turns the layer's stage marks into GB/s and TFLOP/s; a stage
     # without an entry in its work table would be reported without a rate
