@@ -734,7 +734,8 @@ def cpu_baseline(inp, seconds: float = 15.0):
 # larger than L2 where DRAM traffic is read off)
 # --------------------------------------------------------------------------
 KERNEL_CASES = ("gemm_nvfp4", "gemm_nvfp4_s2f6", "gemm_nvfp4_down", "gemm_mxfp8_dgrad", "gemm_mxfp8_wgrad", "requant", "requant_w",
-                "nvfp4_quantize", "quant_w", "mxfp8_quantize", "nvfp4_quantize_sr", "requant_nvfp4", "gemm_nvfp4_wgrad",
+                "nvfp4_quantize", "quant_w", "mxfp8_quantize", "nvfp4_quantize_sr", "requant_nvfp4", "requant_nvfp4_w",
+                "dispatch_grad_quant", "gemm_nvfp4_wgrad",
                 "step_nvfp4_backward", "gemm1_moe_layer", "gemm2_moe_layer")
 
 
@@ -833,6 +834,25 @@ def run_kernel(args):
         else:                                           # NVFP4 backward: requantisation across the transpose
             t = api.nvfp4_requant_transpose_sr(*q, c["rows"], c["cols"], seed=c["sr_seed"])
             run = lambda: api.nvfp4_requant_transpose_sr(*q, c["rows"], c["cols"], seed=c["sr_seed"], out=t)
+    elif which == "requant_nvfp4_w":
+        # NVFP4 backward: 64 experts of 2048 x 4096 weights requantised to the NVFP4 stack of W_e^T,
+        # per-expert outer scales
+        E, N, K = 64, 2048, 4096
+        w = workloads.weights(E, N, K, 0.02, 2, dev).view(E * N, K)
+        q = api.nvfp4_quantize(w, N, api.MX_SF_MMA)
+        t = api.nvfp4_requant_transpose_sr(*q, E * N, K, N, api.MX_SF_MMA, E, True, seed=1, stream_id=16)
+        run = lambda: api.nvfp4_requant_transpose_sr(*q, E * N, K, N, api.MX_SF_MMA, E, True, seed=1, stream_id=16,
+                                                     out=t)
+    elif which == "dispatch_grad_quant":
+        # the dispatch gradient formed inside its MXFP8 quantiser: 64 experts, top-8 of 16384 tokens (Zipf 1.1),
+        # d_model 4096 (dout 134 MB, outputs 1.1 GB, both > L2)
+        E, T, k, D = 64, 16384, 8, 4096
+        ids = workloads.routing(T, k, E, "zipf", 1.1, 0, 7).to(dev)
+        seg, src, pos = api.moe_route(ids, E)
+        dout = workloads.gradient(T, D, 1.0, 3, dev)
+        w = torch.full((T, k), 1.0 / k, device=dev)
+        q = api.moe_dispatch_grad_mxfp8_quantize(dout, src, w, k, seg[E:E + 1])
+        run = lambda: api.moe_dispatch_grad_mxfp8_quantize(dout, src, w, k, seg[E:E + 1], out=q)
     elif which == "requant_w":
         # 64 experts of 2048 x 4096 weights, per-expert outer scales (output 0.55 GB > L2)
         E, N, K = 64, 2048, 4096
