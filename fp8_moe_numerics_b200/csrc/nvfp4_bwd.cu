@@ -24,75 +24,12 @@
 
 #include "mx_common.cuh"
 #include "requant_tile.cuh"
+#include "e2m1_sr.cuh"
 
 namespace {
 
 constexpr int kThreads = 256;
 constexpr float kOuterDiv = 2688.0f;              // 6 * 448
-
-// |E2M1 code| -> value (exact): 0, 0.5, 1, 1.5, 2, 3, 4, 6.
-__device__ __forceinline__ float e2m1_mag(uint32_t m) {
-    const uint32_t e = (m >> 1) & 3, f = m & 1;
-    return e == 0 ? 0.5f * (float)f : __uint_as_float(((e + 126) << 23) | (f << 22));
-}
-
-// 2^n for -126 <= n <= 127 (exact).
-__device__ __forceinline__ float pow2f(int n) { return __uint_as_float((uint32_t)(n + 127) << 23); }
-
-// |y| rounded stochastically onto the E2M1 magnitudes with the R-bit random
-// integer u: the grid step at |y| is q = 2^max(floor(log2 |y|) - 1, -1); |y|
-// goes to lo = floor(|y| / q) q or lo + q, up iff u < floor(frac * 2^R) with
-// frac = (|y| - lo) / q.  Every step is exact in fp32; the result is a grid
-// magnitude, or 8 and above (saturated to 6 by the encoding).
-template <int R>
-__device__ __forceinline__ float e2m1_sr_magnitude(float y, uint32_t u) {
-    const float ay = fabsf(y);
-    if (ay == 0.0f) return 0.0f;
-    const int fl = (int)((__float_as_uint(ay) >> 23) & 0xff) - 127;        // floor(log2 ay); -127 if subnormal
-    const int Q = max(fl - 1, -1);
-    const float inv_q = pow2f(-Q), q = pow2f(Q);
-    const float lo = __fmul_rn(floorf(__fmul_rn(ay, inv_q)), q);
-    const float frac = __fmul_rn(__fsub_rn(ay, lo), inv_q);
-    const float thr = floorf(__fmul_rn(frac, (float)(1ull << R)));         // integer in [0, 2^R)
-    return ((unsigned long long)u < __float2ull_rz(thr)) ? __fadd_rn(lo, q) : lo;
-}
-
-// Hardware stochastic rounding onto E2M1: sm_100a cvt.rs.satfinite.e2m1x4.f32
-// d, {a, b, c, f}, rbits puts f's code in bits 3:0 of d and b's in bits 11:8.
-// f adds the 16-bit random value rbits[23:16]:rbits[7:0], b the value
-// rbits[31:24]:rbits[15:8], just below the kept E2M1 bit, and truncates (the
-// carry rounds up).  With u the element's 16-bit integer, feeding 0xFFFF - u
-// rounds up exactly when u < floor(frac * 2^16): the rule of
-// e2m1_sr_magnitude<16>, signs and saturation included (established by
-// comparing the instruction with the oracle on a B200).  a and c share b's and
-// f's random bits and are not used.
-// Two elements: y_even in f, y_odd in b; codes y_even | y_odd << 8.
-__device__ __forceinline__ uint32_t cvt_rs_e2m1_pair(float y_even, float y_odd, uint32_t rbits) {
-    uint16_t d;
-    asm("cvt.rs.satfinite.e2m1x4.f32 %0, {%1, %2, %3, %4}, %5;"
-        : "=h"(d) : "f"(0.0f), "f"(y_odd), "f"(0.0f), "f"(y_even), "r"(rbits));
-    return d;
-}
-// rbits for elements 2k, 2k+1 whose 16-bit integers are the low and high
-// halves of word w (R = 16).
-__device__ __forceinline__ uint32_t rbits16_pair(uint32_t w) { return __byte_perm(~w, 0u, 0x3120); }
-// R = 8: element j's 8-bit integer u enters as the 16-bit value (255 - u) << 8,
-// which rounds up iff 256 u + 255 < floor(frac 2^16), i.e. iff u < floor(frac
-// 2^8): the R = 8 rule.  Elements 4k .. 4k + 3 are the bytes of word w; h = 0
-// takes the pair 4k, 4k + 1, h = 1 the pair 4k + 2, 4k + 3.
-__device__ __forceinline__ uint32_t rbits8_pair(uint32_t w, int h) {
-    return __byte_perm(~w, 0u, h ? 0x3244 : 0x1044);
-}
-// Eight code bytes from eight pair results (element 2j in the low nibble of byte j).
-__device__ __forceinline__ uint2 pack_e2m1_pairs(const uint32_t d[8]) {
-    uint32_t t[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const uint32_t w = d[2 * k] | (d[2 * k + 1] << 16);     // codes in the low nibbles of bytes 0 .. 3
-        t[k] = (w | (w >> 4)) & 0x00ff00ffu;                     // code bytes of the two pairs in bytes 0 and 2
-    }
-    return make_uint2(__byte_perm(t[0], t[1], 0x6420), __byte_perm(t[2], t[3], 0x6420));
-}
 
 // One 16-value block: E4M3 scale of bmax / (6 s) (0 when s == 0) and the
 // eight code bytes, element 2j in the low nibble of byte j.  L0 is the linear
@@ -113,51 +50,8 @@ __device__ __forceinline__ void quantize_block16(const float* v, float s, uint64
     if constexpr (!kSR) {
         packed.x = cvt_e2m1x8(y);
         packed.y = cvt_e2m1x8(y + 8);
-    } else if constexpr (R == 16) {
-        // L0 is a multiple of 16: the block's random integers are the 16-bit halves of two Philox blocks,
-        // elements 2k and 2k + 1 in word k % 4 of block k / 4
-        uint32_t d[8];
-#pragma unroll
-        for (int blk = 0; blk < 2; ++blk) {
-            const uint4 rnd = philox4x32_10(L0 / 8 + blk, stream_id, seed);
-            const uint32_t w[4] = {rnd.x, rnd.y, rnd.z, rnd.w};
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-                d[4 * blk + k] = cvt_rs_e2m1_pair(y[8 * blk + 2 * k], y[8 * blk + 2 * k + 1], rbits16_pair(w[k]));
-        }
-        packed = pack_e2m1_pairs(d);
-    } else if constexpr (R == 8) {
-        // one Philox block: elements 4k .. 4k + 3 are the bytes of word k
-        const uint4 rnd = philox4x32_10(L0 / 16, stream_id, seed);
-        const uint32_t w[4] = {rnd.x, rnd.y, rnd.z, rnd.w};
-        uint32_t d[8];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            d[2 * k] = cvt_rs_e2m1_pair(y[4 * k], y[4 * k + 1], rbits8_pair(w[k], 0));
-            d[2 * k + 1] = cvt_rs_e2m1_pair(y[4 * k + 2], y[4 * k + 3], rbits8_pair(w[k], 1));
-        }
-        packed = pack_e2m1_pairs(d);
     } else {
-        // magnitudes on the grid are encoded exactly; the sign of y is kept,
-        // also where the magnitude is zero
-        // L0 is a multiple of 16, so the block's 16 random integers are the fields of
-        // 16 / (128 / R) whole Philox blocks (one generator call per 128 bits)
-        constexpr int kPer = 128 / R;
-        uint32_t u[16];
-#pragma unroll
-        for (int blk = 0; blk < 16 / kPer; ++blk) {
-            const uint4 rnd = philox4x32_10(L0 / kPer + blk, stream_id, seed);
-#pragma unroll
-            for (int f = 0; f < kPer; ++f) u[blk * kPer + f] = philox_field<R>(rnd, f);
-        }
-        float m[16];
-        uint32_t sgn[2] = {0u, 0u};
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            m[i] = e2m1_sr_magnitude<R>(y[i], u[i]);
-            sgn[i >> 3] |= (__float_as_uint(y[i]) >> 31) << (4 * (i & 7) + 3);
-        }
-        packed = make_uint2(cvt_e2m1x8(m) | sgn[0], cvt_e2m1x8(m + 8) | sgn[1]);
+        packed = e2m1_sr_codes<R>(y, seed, stream_id, L0);
     }
 }
 
@@ -192,30 +86,6 @@ group_outer_kernel(const uint16_t* __restrict__ x, int64_t cols, int64_t group_r
     }
     m = block_reduce_max(m, red);
     if (threadIdx.x == 0) outer[g] = __fdiv_rn(m, kOuterDiv);
-}
-
-// One thread per 16-value block of a bf16 [rows, cols]: codes, scale byte.
-template <int R, bool kSR>
-__global__ void __launch_bounds__(kThreads)
-nvfp4_quantize_sr_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t group_rows,
-                         const float* __restrict__ outer, uint64_t seed, uint64_t stream_id, int sf_layout,
-                         uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
-    const int64_t S = cols / 16;
-    const int64_t item = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-    if (item >= rows * S) return;
-    const int64_t r = item / S, b = item - r * S;
-    const uint4* src = reinterpret_cast<const uint4*>(x + r * cols + b * 16);
-    const uint4 u0 = __ldg(src), u1 = __ldg(src + 1);
-    const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-    float v[16];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) { v[2 * k] = bf16_lo(w[k]); v[2 * k + 1] = bf16_hi(w[k]); }
-    uint32_t scode;
-    uint2 packed;
-    quantize_block16<R, kSR>(v, __ldg(outer + (group_rows == 1 ? r : r / group_rows)), seed, stream_id,
-                             (uint64_t)(r * cols + b * 16), scode, packed);
-    *reinterpret_cast<uint2*>(codes + (r * cols + b * 16) / 2) = packed;
-    sf[sf_offset(r, b, S, sf_layout)] = (uint8_t)scode;
 }
 
 // Dequantised NVFP4 values (q * sf) * outer[r / group_rows], one fp32
@@ -669,37 +539,6 @@ int launch_requant_nvfp4_tiles(const uint8_t* codes, const uint8_t* sf, int in_l
 // ===========================================================================
 // C ABI
 // ===========================================================================
-
-extern "C" int nvfp4_quantize_sr(const void* x, int64_t rows, int64_t cols, int64_t group_rows, int rounding,
-                                 uint64_t seed, uint64_t stream_id, int rbits, uint8_t* codes, uint8_t* sf,
-                                 float* outer, int sf_layout, cudaStream_t stream) {
-    MX_NVTX_RANGE("nvfp4_quantize_sr");
-    if (((!x || !codes || !sf || !outer) && rows > 0) || rows < 0 || cols <= 0 || cols % 16 || group_rows <= 0 ||
-        rows % group_rows || !mx_aligned(x, 16) || !mx_aligned(codes, 16))
-        return MX_EINVAL;
-    if (rounding != MX_ROUND_RNE && rounding != MX_ROUND_SR) return MX_EINVAL;
-    if (rounding == MX_ROUND_SR && rbits != 8 && rbits != 16 && rbits != 32) return MX_EINVAL;
-    if (sf_layout != MX_SF_ROWMAJOR && sf_layout != MX_SF_MMA) return MX_EINVAL;
-    if (sf_layout == MX_SF_MMA && (rows % 128 || cols % 64)) return MX_EINVAL;
-    if (int st = mx_check_device()) return st;
-    if (rows == 0) return MX_OK;
-    group_outer_kernel<<<(unsigned)(rows / group_rows), kThreads, 0, stream>>>(static_cast<const uint16_t*>(x), cols,
-                                                                               group_rows, outer);
-    mx_count_launch();
-    const int64_t items = rows * (cols / 16);
-    const unsigned grid = (unsigned)((items + kThreads - 1) / kThreads);
-    auto launch = [&](auto kSRc) {
-        constexpr bool kSR = decltype(kSRc)::value;
-        return dispatch_rbits<kSR>(rbits, [&](auto Rc) {
-            nvfp4_quantize_sr_kernel<decltype(Rc)::value, kSR><<<grid, kThreads, 0, stream>>>(
-                static_cast<const uint16_t*>(x), rows, cols, group_rows, outer, seed, stream_id, sf_layout, codes,
-                sf);
-            mx_count_launch();
-            return mx_launch_status();
-        });
-    };
-    return rounding == MX_ROUND_SR ? launch(std::true_type{}) : launch(std::false_type{});
-}
 
 extern "C" int nvfp4_requant_transpose_sr(const uint8_t* codes, const uint8_t* sf, const float* outer, int64_t rows,
                                           int64_t cols, int64_t group_rows, int in_sf_layout, int64_t experts,

@@ -6,6 +6,7 @@
 // cvt or by exact integer arithmetic (see mx_common.cuh).
 #include "mx_common.cuh"
 #include "requant_tile.cuh"
+#include "e2m1_sr.cuh"
 
 #include <cuda.h>
 
@@ -26,11 +27,20 @@ __device__ __forceinline__ uint32_t warp_max_u32(uint32_t v) {
     return v;
 }
 
+// Random bits of the stochastically rounded form (nvfp4_quantize_sr): key,
+// Philox stream and the linear index of the block's first element.
+struct SrKey {
+    uint64_t seed, stream;
+};
+
 // Quantise one 16-element block (two uint4 of bf16) with outer scale s > 0;
 // ab_bits = the block's max |x| as bf16 magnitude bits (callers have it from
-// the row amax).  Returns the E4M3 scale code; writes 8 bytes of E2M1 codes.
+// the row amax).  Returns the E4M3 scale code; writes 8 bytes of E2M1 codes,
+// to nearest or (kR > 0) rounded stochastically with kR random bits of the
+// elements' linear indices L0 ...
+template <int kR = 0>
 __device__ __forceinline__ uint32_t nvfp4_block(const uint4& a, const uint4& b, uint32_t ab_bits, float s,
-                                                uint2& packed) {
+                                                uint2& packed, SrKey key = {}, uint64_t L0 = 0) {
     float ab = __uint_as_float(ab_bits << 16);
     float t = __fmul_rn(6.0f, s);
     float d = __fdiv_rn(ab, t);
@@ -39,6 +49,17 @@ __device__ __forceinline__ uint32_t nvfp4_block(const uint4& a, const uint4& b, 
     float inv = __frcp_rn(__fmul_rn(e4m3_to_f32(sc), s));
     const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
     const uint64_t inv2 = f2_pack(inv, inv);
+    if constexpr (kR > 0) {
+        float y[16];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            y[2 * i] = bf16_lo(w[i]);
+            y[2 * i + 1] = bf16_hi(w[i]);
+            mul2_rn(y[2 * i], y[2 * i + 1], inv2);
+        }
+        packed = e2m1_sr_codes<kR>(y, key.seed, key.stream, L0);
+        return sc;
+    }
     uint32_t word[2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {                      // eight products (in pairs), then their code word
@@ -59,15 +80,15 @@ __device__ __forceinline__ uint32_t nvfp4_block(const uint4& a, const uint4& b, 
 // warp calls it, live or not, because the scale bytes of four consecutive
 // blocks (in lanes 4m..4m+3) are merged by shuffles into one 32-bit store
 // when `word_sf`.
-template <int kLayout>
+template <int kLayout, int kR = 0>
 __device__ __forceinline__ void emit_nvfp4_block(int64_t row, int64_t blk, int64_t nblk, bool active, float s,
                                                  const uint4& a, const uint4& b, uint32_t ab_bits,
                                                  uint8_t* __restrict__ crow, uint8_t* __restrict__ sf, bool word_sf,
-                                                 int lane) {
+                                                 int lane, SrKey key = {}) {
     uint2 packed = make_uint2(0u, 0u);
     uint32_t sc = 0;
     const bool live = active && blk < nblk;
-    if (live && s > 0.0f) sc = nvfp4_block(a, b, ab_bits, s, packed);
+    if (live && s > 0.0f) sc = nvfp4_block<kR>(a, b, ab_bits, s, packed, key, (uint64_t)((row * nblk + blk) * 16));
     if (live) *reinterpret_cast<uint2*>(crow + blk * 8) = packed;
     if (word_sf) {
         uint32_t w = sc << (8 * (lane & 3));
@@ -91,11 +112,12 @@ __device__ __forceinline__ void emit_nvfp4_block(int64_t row, int64_t blk, int64
 constexpr int kRowThreads = 256;
 
 // Rows [block * 256/kTPR, +256/kTPR) of x, those below row_end.
-template <int kTPR, int kNB, bool kGroup, int kLayout>
+template <int kTPR, int kNB, bool kGroup, int kLayout, int kR = 0>
 __device__ __forceinline__ void quant_rows_block(const uint16_t* __restrict__ x, int64_t rows, int64_t row_end,
                                                  int64_t cols, int64_t group_rows, bool word_sf,
                                                  uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
-                                                 float* __restrict__ outer, int64_t block, uint32_t* wmax) {
+                                                 float* __restrict__ outer, int64_t block, uint32_t* wmax,
+                                                 SrKey key = {}) {
     constexpr int kRPB = kRowThreads / kTPR;
     const int lane = threadIdx.x & 31;
     const int j = threadIdx.x % kTPR;
@@ -152,7 +174,7 @@ __device__ __forceinline__ void quant_rows_block(const uint16_t* __restrict__ x,
 
     uint8_t* crow = codes + (active ? row : 0) * (cols >> 1);
     auto emit = [&](int64_t blk, const uint4& a, const uint4& b, uint32_t ab_bits) {
-        emit_nvfp4_block<kLayout>(row, blk, nblk, active, s, a, b, ab_bits, crow, sf, word_sf, lane);
+        emit_nvfp4_block<kLayout, kR>(row, blk, nblk, active, s, a, b, ab_bits, crow, sf, word_sf, lane, key);
     };
     if (resident) {
 #pragma unroll
@@ -167,13 +189,14 @@ __device__ __forceinline__ void quant_rows_block(const uint16_t* __restrict__ x,
     }
 }
 
-template <int kTPR, int kNB, bool kGroup, int kLayout>
+template <int kTPR, int kNB, bool kGroup, int kLayout, int kR = 0>
 __global__ void __launch_bounds__(kRowThreads, kNB <= 4 ? 4 : 2)
 nvfp4_quant_rows_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t group_rows,
-                        bool word_sf, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, float* __restrict__ outer) {
+                        bool word_sf, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, float* __restrict__ outer,
+                        SrKey key) {
     __shared__ uint32_t wmax[kRowThreads / 32];
-    quant_rows_block<kTPR, kNB, kGroup, kLayout>(x, rows, rows, cols, group_rows, word_sf, codes, sf, outer,
-                                                 (int64_t)blockIdx.x, wmax);
+    quant_rows_block<kTPR, kNB, kGroup, kLayout, kR>(x, rows, rows, cols, group_rows, word_sf, codes, sf, outer,
+                                                     (int64_t)blockIdx.x, wmax, key);
 }
 
 // SwiGLU fused into the per-token NVFP4 quantiser: the activation a =
@@ -938,17 +961,15 @@ int dispatch_layout(int layout, F&& f) {
 // C ABI
 // ===========================================================================
 
-extern "C" int nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t group_rows, uint8_t* codes,
-                              uint8_t* sf, float* outer, int sf_layout, cudaStream_t stream) {
-    MX_NVTX_RANGE("nvfp4_quantize");
-    // an empty problem succeeds without touching memory (its pointers may be null)
-    if (((!x || !codes || !sf || !outer) && rows > 0) || rows < 0 || cols <= 0 || cols % 16 || group_rows <= 0 ||
-        rows % group_rows || !mx_aligned(x, 16) || !mx_aligned(codes, 16))
-        return MX_EINVAL;
-    if (sf_layout != MX_SF_ROWMAJOR && sf_layout != MX_SF_MMA) return MX_EINVAL;
-    if (sf_layout == MX_SF_MMA && (rows % 128 || cols % 64)) return MX_EINVAL;
-    if (int st = mx_check_device()) return st;
-    if (rows == 0) return MX_OK;
+namespace {
+
+// The launches of nvfp4_quantize (kR = 0, codes to nearest) and of
+// nvfp4_quantize_sr (kR random bits): one pass of the row kernel for per-row
+// outer scales, else the group amax pass, the row kernel and the conversion
+// of the group maxima to scales.  Arguments already validated.
+template <int kR>
+int nvfp4_quantize_launch(const void* x, int64_t rows, int64_t cols, int64_t group_rows, uint8_t* codes, uint8_t* sf,
+                          float* outer, int sf_layout, SrKey key, cudaStream_t stream) {
     const uint16_t* xb = static_cast<const uint16_t*>(x);
     const int64_t ngroups = rows / group_rows;
     const int64_t nblk_row = cols / 16;
@@ -961,17 +982,17 @@ extern "C" int nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t
             auto go = [&](auto kern, int tpr) {
                 const int64_t rpb = kRowThreads / tpr;
                 kern<<<(unsigned)((rows + rpb - 1) / rpb), kRowThreads, 0, stream>>>(xb, rows, cols, group_rows, word_sf,
-                                                                                       codes, sf, outer);
+                                                                                       codes, sf, outer, key);
                 mx_count_launch();
             };
             // four 16-element blocks (128 bytes) per thread in flight, 4 CTAs per SM:
             // 128 KB of loads outstanding per SM covers HBM latency under load
-            if (nblk_row <= 64) go(nvfp4_quant_rows_kernel<16, 4, kG, kL>, 16);
-            else if (nblk_row <= 128) go(nvfp4_quant_rows_kernel<32, 4, kG, kL>, 32);
-            else if (nblk_row <= 256) go(nvfp4_quant_rows_kernel<64, 4, kG, kL>, 64);
-            else if (nblk_row <= 512) go(nvfp4_quant_rows_kernel<128, 4, kG, kL>, 128);
-            else if (nblk_row <= 1024) go(nvfp4_quant_rows_kernel<256, 4, kG, kL>, 256);
-            else go(nvfp4_quant_rows_kernel<256, 8, kG, kL>, 256);
+            if (nblk_row <= 64) go(nvfp4_quant_rows_kernel<16, 4, kG, kL, kR>, 16);
+            else if (nblk_row <= 128) go(nvfp4_quant_rows_kernel<32, 4, kG, kL, kR>, 32);
+            else if (nblk_row <= 256) go(nvfp4_quant_rows_kernel<64, 4, kG, kL, kR>, 64);
+            else if (nblk_row <= 512) go(nvfp4_quant_rows_kernel<128, 4, kG, kL, kR>, 128);
+            else if (nblk_row <= 1024) go(nvfp4_quant_rows_kernel<256, 4, kG, kL, kR>, 256);
+            else go(nvfp4_quant_rows_kernel<256, 8, kG, kL, kR>, 256);
         };
         if (group_rows == 1) {
             run(std::false_type());
@@ -988,6 +1009,48 @@ extern "C" int nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t
         }
         return mx_launch_status();
     });
+}
+
+int nvfp4_quantize_check(const void* x, int64_t rows, int64_t cols, int64_t group_rows, const uint8_t* codes,
+                         const uint8_t* sf, const float* outer, int sf_layout) {
+    // an empty problem succeeds without touching memory (its pointers may be null)
+    if (((!x || !codes || !sf || !outer) && rows > 0) || rows < 0 || cols <= 0 || cols % 16 || group_rows <= 0 ||
+        rows % group_rows || !mx_aligned(x, 16) || !mx_aligned(codes, 16))
+        return MX_EINVAL;
+    if (sf_layout != MX_SF_ROWMAJOR && sf_layout != MX_SF_MMA) return MX_EINVAL;
+    if (sf_layout == MX_SF_MMA && (rows % 128 || cols % 64)) return MX_EINVAL;
+    return MX_OK;
+}
+
+}  // namespace
+
+extern "C" int nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t group_rows, uint8_t* codes,
+                              uint8_t* sf, float* outer, int sf_layout, cudaStream_t stream) {
+    MX_NVTX_RANGE("nvfp4_quantize");
+    if (int st = nvfp4_quantize_check(x, rows, cols, group_rows, codes, sf, outer, sf_layout)) return st;
+    if (int st = mx_check_device()) return st;
+    if (rows == 0) return MX_OK;
+    return nvfp4_quantize_launch<0>(x, rows, cols, group_rows, codes, sf, outer, sf_layout, SrKey{}, stream);
+}
+
+// The four-bit backward's quantiser: the same scales, codes rounded
+// stochastically (e2m1_sr.cuh) or to nearest.
+extern "C" int nvfp4_quantize_sr(const void* x, int64_t rows, int64_t cols, int64_t group_rows, int rounding,
+                                 uint64_t seed, uint64_t stream_id, int rbits, uint8_t* codes, uint8_t* sf,
+                                 float* outer, int sf_layout, cudaStream_t stream) {
+    MX_NVTX_RANGE("nvfp4_quantize_sr");
+    if (int st = nvfp4_quantize_check(x, rows, cols, group_rows, codes, sf, outer, sf_layout)) return st;
+    if (rounding != MX_ROUND_RNE && rounding != MX_ROUND_SR) return MX_EINVAL;
+    if (rounding == MX_ROUND_SR && rbits != 8 && rbits != 16 && rbits != 32) return MX_EINVAL;
+    if (int st = mx_check_device()) return st;
+    if (rows == 0) return MX_OK;
+    const SrKey key{seed, stream_id};
+    if (rounding == MX_ROUND_RNE)
+        return nvfp4_quantize_launch<0>(x, rows, cols, group_rows, codes, sf, outer, sf_layout, key, stream);
+    if (rbits == 8) return nvfp4_quantize_launch<8>(x, rows, cols, group_rows, codes, sf, outer, sf_layout, key, stream);
+    if (rbits == 16)
+        return nvfp4_quantize_launch<16>(x, rows, cols, group_rows, codes, sf, outer, sf_layout, key, stream);
+    return nvfp4_quantize_launch<32>(x, rows, cols, group_rows, codes, sf, outer, sf_layout, key, stream);
 }
 
 extern "C" int swiglu_nvfp4_quantize(const void* h, int64_t rows, int64_t F, int gated, const int64_t* rows_valid,
