@@ -403,8 +403,10 @@ __device__ __forceinline__ void tile_emit_transposed(const float* T, int64_t row
                 w[i] = cvt_e4m3x4(a0, a1, a2, a3);
             }
         }
-        *reinterpret_cast<uint4*>(out_codes + cg * rows + rr) = make_uint4(w[0], w[1], w[2], w[3]);
-        if ((g & 1) == 0) out_e8m0[sf_offset(cg, rr >> 5, S, kLayout)] = (uint8_t)(e + 127);
+        if (mx_in_range(cg * rows + rr, 16, cols * rows))
+            *reinterpret_cast<uint4*>(out_codes + cg * rows + rr) = make_uint4(w[0], w[1], w[2], w[3]);
+        if ((g & 1) == 0 && mx_in_range(sf_offset(cg, rr >> 5, S, kLayout), 1, cols * S))
+            out_e8m0[sf_offset(cg, rr >> 5, S, kLayout)] = (uint8_t)(e + 127);
     }
 }
 
@@ -536,7 +538,7 @@ struct DispatchGradRows {
         q.live = false;
         if (r >= valid) return;
         const int64_t s = __ldg(src + r);
-        if (s < 0 || s >= Tk) return;
+        if (s < 0 || s >= Tk || !mx_in_range((s / k) * D + c, 32, (Tk / k) * D)) return;
         q.live = true;
         q.wt = w ? __ldg(w + s) : 1.0f;
         const uint4* vp = reinterpret_cast<const uint4*>(dout + (s / k) * D + c);
@@ -595,10 +597,13 @@ dispatch_grad_mxfp8_kernel(DispatchGradRows src, int64_t rows, int64_t cols, con
                 mul2_rn(a2, a3, sc2);
                 w[i] = cvt_e4m3x4(a0, a1, a2, a3);
             }
-            uint4* dst = reinterpret_cast<uint4*>(row_codes + r * cols + c);
-            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-            dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-            row_e8m0[sf_offset(r, c >> 5, cols >> 5, kLayout)] = (uint8_t)(e + 127);
+            if (mx_in_range(r * cols + c, 32, rows * cols)) {
+                uint4* dst = reinterpret_cast<uint4*>(row_codes + r * cols + c);
+                dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+            }
+            if (mx_in_range(sf_offset(r, c >> 5, cols >> 5, kLayout), 1, rows * (cols >> 5)))
+                row_e8m0[sf_offset(r, c >> 5, cols >> 5, kLayout)] = (uint8_t)(e + 127);
         }
 #pragma unroll
         for (int i = 0; i < 32; ++i) T[tsw(32 * h + i, rl)] = v[i];
