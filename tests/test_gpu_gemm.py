@@ -56,6 +56,10 @@ NVFP4_CASES = [
     (2, 384, 256, [130, 50]),                 # N % 256 != 0: 128-wide tiles
     (5, 256, 1024, [1, 129, 0, 0, 260]),
     (2, 256, 4096, [200, 70]),                # long K
+    (3, 256, 256, [1, 7, 100]),               # one row tile per expert: half pairs only
+    (3, 512, 256, [256, 0, 512]),             # even tile counts
+    # 1 or 3 row tiles per expert, 4 column tiles: 800 leftover tiles, enough for the tail kernel on 148 SMs
+    (200, 1024, 256, [60 + 200 * (i % 2) for i in range(200)]),
 ]
 
 
@@ -110,6 +114,9 @@ MX_CASES = [
     (3, 256, 256, [128, 0, 300]),
     (2, 384, 128, [50, 260]),                 # N % 256 != 0
     (4, 512, 512, [1, 0, 129, 256]),
+    (3, 256, 256, [1, 7, 100]),               # half pairs only
+    (3, 256, 256, [256, 0, 512]),             # full pairs only
+    (200, 1024, 128, [60 + 200 * (i % 2) for i in range(200)]),  # the tail kernel (800 leftover tiles)
 ]
 
 
