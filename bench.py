@@ -44,8 +44,9 @@ NOMINAL_NVFP4_TFLOPS = 9000.0
 NOMINAL_MXFP8_TFLOPS = 4500.0
 NOMINAL_HBM_GBS = 8000.0
 SM_MAX_MHZ = 1965.0                   # clocks.max.sm of this machine's B200s
-# stages that issue more than one kernel (routing: 4; per-expert NVFP4 weights: amax, quantise, finish)
-MULTI_LAUNCH_STAGES = ("route", "quant_w")
+# stages that issue more than one kernel (routing: 4; per-expert NVFP4 weights: amax, quantise, finish;
+# the row-mode grouped GEMMs: the CTA-pair kernel and the tail kernel for the experts' leftover row tiles)
+MULTI_LAUNCH_STAGES = ("route", "quant_w", "gemm1", "gemm2", "dgrad1", "dgrad2")
 # mxfp8_requant_transpose_sr (R = 16) per element, from one ncu capture of `bench.py --kernel requant_w`
 # (64 experts x 2048 x 4096, output 0.55 GB > L2): warp-instructions executed and DRAM bytes (read + write)
 REQUANT_WARP_INST_PER_ELEM = 0.5996
