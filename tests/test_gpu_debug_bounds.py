@@ -6,8 +6,9 @@ GEMMs' scale-atom loads and outer scales, the NVFP4-backward loads and stores)
 is compared with the extent the call's arguments give its buffer; an access
 out of range is skipped and counted.  A child process with MX_DEBUG=1 runs the
 tiny layer's forward and backward in both backward formats plus ragged
-requantisations and routing with empty experts; it must count no violation and
-produce the same bytes as the normal build in this process.
+requantisations, routing with empty experts, and grouped GEMMs with 200 experts
+of one or three row tiles (enough leftover tiles for the row-mode tail kernel);
+it must count no violation and produce the same bytes as the normal build.
 """
 import json
 import os
@@ -49,6 +50,27 @@ def run():
         oc, oe = api.mxfp8_requant_transpose_sr(*q, 384, 192, 1, api.MX_SF_MMA, None, 1, 2, R, api.MX_SF_ROWMAJOR)
         out[f"rq{R}"] = oc.cpu().numpy()
         out[f"rq{R}_e"] = oe.cpu().numpy()
+    # grouped GEMMs whose leftover row tiles go to the tail kernel: 200 experts of 1 or 3 row tiles,
+    # 4 column tiles of 256 (800 leftover tiles); valid random codes and scales
+    counts = [60 + 200 * (i % 2) for i in range(200)]
+    seg2 = torch.tensor(np.concatenate([[0], np.cumsum([(c + 127) // 128 * 128 for c in counts])]),
+                        dtype=torch.int64).cuda()
+    E2, N2, K2, valid = 200, 1024, 256, int(seg2[-1])
+    M2 = valid + 128
+    g = torch.Generator(device="cuda")
+    g.manual_seed(11)
+    u8 = lambda n, lo=0, hi=256: torch.randint(lo, hi, (n,), dtype=torch.uint8, device="cuda", generator=g)
+    a = (u8(M2 * K2 // 2).view(M2, K2 // 2), u8(api.sf_bytes(M2, K2, 16, api.MX_SF_MMA), 0x30, 0x48),
+         torch.full((M2,), 1e-2, device="cuda"))
+    b = (u8(E2 * N2 * K2 // 2).view(E2 * N2, K2 // 2), u8(api.sf_bytes(E2 * N2, K2, 16, api.MX_SF_MMA), 0x30, 0x48),
+         torch.full((E2,), 1e-2, device="cuda"))
+    out["gemm_nvfp4_tail"] = api.grouped_gemm_nvfp4(a, b, seg2, E2, N2, K2).float().cpu().numpy()[:valid]
+    ac = u8(M2 * K2).view(M2, K2) & 0x77
+    bc = u8(N2 * E2 * K2).view(N2, E2 * K2) & 0x77
+    ae = u8(api.sf_bytes(M2, K2, 32, api.MX_SF_MMA), 120, 134)
+    be = u8(api.sf_bytes(N2, E2 * K2, 32, api.MX_SF_MMA), 120, 134)
+    out["gemm_mxfp8_tail"] = api.grouped_gemm_mxfp8(api.MX_GEMM_DGRAD, ac, ae, bc, be, seg2, E2, M2, N2,
+                                                     K2).float().cpu().numpy()[:valid]
     api.sync_status()
     torch.cuda.synchronize()
     return out
