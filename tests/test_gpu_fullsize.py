@@ -71,9 +71,15 @@ def _rand_u8(shape, lo, hi, g):
 
 
 def _sample_rows_cols(seg, E, N, n, seed):
-    """n (row, col, expert) samples over the routed rows (padding rows included)."""
+    """n (row, col, expert) samples over the routed rows (padding rows included), a quarter of
+    them in the last row tile of experts with an odd tile count (at this layer those tiles run in
+    the grouped GEMMs' tail kernel, the rest in the CTA-pair kernel)."""
     rng = np.random.default_rng(seed)
-    rows = rng.integers(0, int(seg[E]), n)
+    tiles = np.diff(seg[:E + 1]) // 128
+    odd = np.flatnonzero(tiles % 2 == 1)
+    n_tail = n // 4
+    tail_rows = seg[odd[rng.integers(0, len(odd), n_tail)] + 1] - 128 + rng.integers(0, 128, n_tail)
+    rows = np.concatenate([rng.integers(0, int(seg[E]), n - n_tail), tail_rows])
     cols = rng.integers(0, N, n)
     experts = np.searchsorted(seg, rows, side="right") - 1
     return rows, cols, experts
@@ -122,10 +128,8 @@ def test_grouped_gemm_nvfp4_s2f6_epilogue_full_layer_shape(cuda):
          torch.rand(E, device="cuda", generator=g) + 0.5)
     codes, e8 = api.grouped_gemm_nvfp4_s2f6(a, b, torch.from_numpy(seg).cuda(), E, N, K, seed, stream)
     api.sync_status()
-    rng = np.random.default_rng(3)
-    rows = rng.integers(0, int(seg[E]), 48)
-    blocks = rng.integers(0, N // 32, 48)
-    ex = np.searchsorted(seg, rows, side="right") - 1
+    rows, _, ex = _sample_rows_cols(seg, E, N, 48, seed=3)
+    blocks = np.random.default_rng(4).integers(0, N // 32, 48)
     a_sf, b_sf = np_(a[1]), np_(b[1])
     a_val = oracle.nvfp4_block_values(np_(a[0][torch.from_numpy(rows).cuda()]), mma_rows(a_sf, rows, K // 16))
     flips = 0
