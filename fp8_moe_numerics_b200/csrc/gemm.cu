@@ -6,22 +6,30 @@
 // transposes).  One persistent, warp-specialised kernel template serves both:
 //
 //   warp 0      TMA producer: operand tiles by cp.async.bulk.tensor (128-byte
-//               swizzle) into a ring of 4 shared-memory stages (mbarriers)
+//               swizzle) and the stage's scale atoms by cp.async.bulk into a
+//               ring of 3-6 shared-memory stages (as many as fit beside the
+//               epilogue staging), completion on mbarriers
 //   warp 1      MMA issuer: allocates TMEM, issues block-scaled tcgen05.mma
 //               (kind::mxf4nvf4 block16 for NVFP4, kind::mxf8f6f4 block32 for
 //               MXFP8), commits stage release / accumulator-ready
-//   warps 4-7   scale loaders: each stage's scale atoms from global memory
-//               into a ring of 4 TMEM scale regions with tcgen05.st (measured
+//   warps 4-7   scale movers: each stage's scale atoms from shared memory
+//               into a ring of TMEM scale regions with tcgen05.st (measured
 //               on B200: tcgen05.cp of scales stalls the MMA pipe ~24 cycles
 //               per atom, tcgen05.st from registers runs beside it)
 //   warps 8-15  epilogue: tcgen05.ld of the fp32 accumulator into registers,
-//               early accumulator release, outer scales (NVFP4), conversion,
-//               128-bit stores overlapping the next tile's main loop
+//               early release of the chunks the next tile's accumulator
+//               shares, outer scales (NVFP4), conversion, 32 x 32 boxes
+//               staged in shared memory and written by TMA tensor stores
+//               while the next tile's main loop runs
 //
-// Tile: 128 rows (MMA M) x kBN columns (MMA N), 128 bytes of K per stage
-// (256 FP4 or 128 FP8 values = 4 MMAs of 32 bytes each).  Every mbarrier wait
-// is bounded: on expiry the kernel records MX_ETIMEOUT in a device status
-// word, stops issuing work, drains its own copies and frees its TMEM.
+// Tile: 128 rows (MMA M) x kBN columns (MMA N) per CTA, 128 bytes of K per
+// stage (256 FP4 or 128 FP8 values = 4 MMAs of 32 bytes each).  Where the
+// shape allows, CTA pairs (cta_group::2) compute 256 x 256 tiles, each CTA
+// loading its 128 rows of A and half of B; row-mode calls add a single-CTA
+// tail kernel with 128 x 256 tiles for the experts' leftover row tiles (see
+// the tile scheduling below).  Every mbarrier wait is bounded: on expiry the
+// kernel records MX_ETIMEOUT in a device status word, stops issuing work,
+// drains its own copies and frees its TMEM.
 #include "mx_common.cuh"
 
 #include <cuda.h>
