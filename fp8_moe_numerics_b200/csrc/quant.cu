@@ -1,7 +1,9 @@
-// quant.cu -- NVFP4 quantiser, MXFP8 quantiser and the NVFP4 -> MXFP8
+// quant.cu -- the NVFP4 quantiser (round-to-nearest and stochastic forms,
+// SwiGLU fused in front for the activations), the MXFP8 quantiser (and its form
+// that builds the combine's gradient rows itself), and the NVFP4 -> MXFP8
 // stochastic requantisation across a transpose (sm_100a).
 //
-// All three are HBM streams: 128-bit coalesced loads and stores, amax by
+// All are written as HBM streams: 128-bit coalesced loads and stores, amax by
 // packed-integer max and warp shuffles, every rounding decision taken by a PTX
 // cvt or by exact integer arithmetic (see mx_common.cuh).
 #include "mx_common.cuh"
