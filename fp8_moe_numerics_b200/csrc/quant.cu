@@ -562,18 +562,23 @@ dispatch_grad_mxfp8_kernel(DispatchGradRows src, int64_t rows, int64_t cols, con
                            uint8_t* __restrict__ row_codes, uint8_t* __restrict__ row_e8m0,
                            uint8_t* __restrict__ col_codes, uint8_t* __restrict__ col_e8m0) {
     __shared__ __align__(16) float T[kTC * kTR];
+    // Row tiles vary fastest: the blocks in flight gather the same 64-column
+    // slice of dout for rows of every expert, so that slice of all tokens (T x
+    // 128 B, a few MB) stays in L2 while each token's k routed rows read it.
+    // (Column tiles fastest, the blocks in flight read whole 8 KB token rows
+    // and a token's other routed rows come back after they left L2.)
     const int64_t valid = load_rows_valid(rows_valid, rows);
-    const int64_t tiles_c = cols / kTC;
-    const int64_t ntiles = tiles_c * ((valid + kTR - 1) / kTR);
+    const int64_t tiles_r = (valid + kTR - 1) / kTR;
+    const int64_t ntiles = (cols / kTC) * tiles_r;
     int64_t tile = blockIdx.x;
     if (tile >= ntiles) return;
     const int t = threadIdx.x;
     const int rl = t >> 1, h = t & 1;
     DispatchGradRows::Raw raw;
-    auto issue = [&](int64_t tl) { src.issue((tl / tiles_c) * kTR + rl, (tl % tiles_c) * kTC + 32 * h, valid, raw); };
+    auto issue = [&](int64_t tl) { src.issue((tl % tiles_r) * kTR + rl, (tl / tiles_r) * kTC + 32 * h, valid, raw); };
     issue(tile);
     for (; tile < ntiles; tile += gridDim.x) {
-        const int64_t c0 = (tile % tiles_c) * kTC, r0 = (tile / tiles_c) * kTR;
+        const int64_t c0 = (tile / tiles_r) * kTC, r0 = (tile % tiles_r) * kTR;
         const int64_t r = r0 + rl, c = c0 + 32 * h;
         uint4 q[4];
         src.finish(raw, q);
