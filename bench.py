@@ -49,8 +49,8 @@ SM_MAX_MHZ = 1965.0                   # clocks.max.sm of this machine's B200s
 MULTI_LAUNCH_STAGES = ("route", "quant_w", "gemm1", "gemm2", "dgrad1", "dgrad2")
 # mxfp8_requant_transpose_sr (R = 16) per element, from one ncu capture of `bench.py --kernel requant_w`
 # (64 experts x 2048 x 4096, output 0.55 GB > L2): warp-instructions executed and DRAM bytes (read + write)
-REQUANT_WARP_INST_PER_ELEM = 0.5996
-REQUANT_DRAM_BYTES_PER_ELEM = 1.5673
+REQUANT_WARP_INST_PER_ELEM = 0.5966
+REQUANT_DRAM_BYTES_PER_ELEM = 1.5817
 
 
 def load_peaks():

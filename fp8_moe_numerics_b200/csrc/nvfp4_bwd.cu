@@ -242,8 +242,10 @@ group_amax_nvfp4_kernel(const uint8_t* __restrict__ codes, const uint8_t* __rest
 // word's other bytes.
 constexpr int kInNvfp4Tile = 0, kInNvfp4Rows = 1, kInBf16 = 2;
 
+// Five blocks per SM where that needs no spills (all but the software R = 32 rounding),
+// as for the MXFP8 requantisation's tile kernel.
 template <int R, bool kSR, int kIn, bool kSeg>
-__global__ void __launch_bounds__(kRqThreads, 4)
+__global__ void __launch_bounds__(kRqThreads, R == 32 ? 4 : 5)
 requant_nvfp4_tile_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sf, int in_layout, bool sf_words,
                           const float* __restrict__ outer, int64_t rows, int64_t cols, int64_t group_rows,
                           int64_t rpe, const int64_t* __restrict__ seg, int64_t E, int out_per_group,

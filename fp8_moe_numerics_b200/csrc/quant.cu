@@ -845,8 +845,14 @@ __device__ __forceinline__ uint32_t cvt_rs_quad_fields(float y0, float y1, float
 
 constexpr float kFoldMinScale = 7.888609052210118e-31f;          // 2^-100
 
+// Five blocks per SM (48 registers, no spills): measured on B200 14% faster than four (62
+// registers) on per-expert weights and 4% on per-row tensors; six spill.  The forms that
+// would spill at five (R = 8, per-row scales into a row-major output) keep four.
+template <int kR, int kOutLayout, bool kPerRow>
+constexpr int rq_min_blocks() { return (kR == 8 || (kPerRow && kOutLayout == MX_SF_ROWMAJOR)) ? 4 : 5; }
+
 template <int kR, int kInLayout, int kOutLayout, bool kPerRow>
-__global__ void __launch_bounds__(kTileThreads, 4)
+__global__ void __launch_bounds__(kTileThreads, rq_min_blocks<kR, kOutLayout, kPerRow>())
 requant_tile_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sf, bool sf_words, bool e8_words,
                     const float* __restrict__ outer, int64_t rows, int64_t cols, int64_t group_rows, int group_shift,
                     const int64_t* rows_valid, uint64_t seed, uint64_t stream_id, uint8_t* __restrict__ out_codes,
