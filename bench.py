@@ -51,6 +51,10 @@ MULTI_LAUNCH_STAGES = ("route", "quant_w", "gemm1", "gemm2", "dgrad1", "dgrad2")
 # (64 experts x 2048 x 4096, output 0.55 GB > L2): warp-instructions executed and DRAM bytes (read + write)
 REQUANT_WARP_INST_PER_ELEM = 0.5966
 REQUANT_DRAM_BYTES_PER_ELEM = 1.5817
+# DRAM bytes (read + write) of one launch of the step's kernels that are not per-element streams, from one
+# ncu capture of `bench.py --steps 1 --warmup 1` (dram__bytes_read.sum + dram__bytes_write.sum, one pass, the
+# timed step's launch): wgrad1 reads 3.56 GB and writes the 6.40 GB weight gradient
+STAGE_DRAM_BYTES = {"wgrad1": 3558820352 + 6397490944}
 
 
 def load_peaks():
@@ -334,7 +338,8 @@ def run_ours(args):
         peak = peaks["bf16_sus"] * ratio
         achieved = wk / (per_launch_ms * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
-                "frac": round(achieved / peak, 4), "traffic": None, "kernel": dom, "algorithmic_flops": int(wk),
+                "frac": round(achieved / peak, 4), "traffic": STAGE_DRAM_BYTES.get(dom), "kernel": dom,
+                "algorithmic_flops": int(wk),
                 "peak_source": f"{peaks['src']} sustained bf16 x {ratio} (nominal dense ratio)"}
     breakdown = {}
     for n in names:

@@ -387,7 +387,10 @@ __device__ __forceinline__ Tile make_tile(const GemmArgs& p, int64_t idx, uint32
         const int64_t nt_n = p.N / rows, nt_k = p.K / kBN;
         t.e = idx / (nt_n * nt_k);
         const int64_t rem = idx % (nt_n * nt_k);
-        const int64_t tn = rem / nt_k, tk = rem % nt_k;
+        // the dimension with fewer tiles varies fastest: a wave of items then
+        // re-streams the smaller set of operand row blocks
+        const bool k_outer = nt_k >= nt_n;
+        const int64_t tn = k_outer ? rem % nt_n : rem / nt_k, tk = k_outer ? rem / nt_n : rem % nt_k;
         const int64_t s0 = __ldg(p.seg + t.e), s1 = __ldg(p.seg + t.e + 1);
         t.a_y = tn * rows + half;
         t.row0 = t.e * p.N + t.a_y;

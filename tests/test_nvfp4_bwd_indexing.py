@@ -281,6 +281,8 @@ def test_segment_kernels_indexing(M, C, seg, per_row, out_mma, in_mma, group_row
 @pytest.mark.parametrize("M,N,K,seg,pair", [
     (1280, 256, 256, [0, 512, 512, 768, 1280], True),
     (512, 128, 384, [0, 256, 512], False),
+    (1280, 512, 1024, [0, 512, 512, 768, 1280], True),    # more k-tiles than n-tiles: n varies fastest
+    (1280, 1024, 256, [0, 256, 1280], True),              # more n-tiles: k varies fastest
 ])
 def test_nvfp4_wgrad_tile_mapping(M, N, K, seg, pair):
     # csrc/gemm.cu make_tile, WGRAD branch with NVFP4 operands: A [N, M] and B
@@ -293,10 +295,15 @@ def test_nvfp4_wgrad_tile_mapping(M, N, K, seg, pair):
     groups = M // 64                                             # sfa_groups = sfb_groups
     atoms_a, atoms_b = (N // 128) * groups, (K // 128) * groups
     E = len(seg) - 1
-    for idx in range(E * (N // rows) * (K // kBN)):
-        e = idx // ((N // rows) * (K // kBN))
-        rem = idx % ((N // rows) * (K // kBN))
-        tn, tk = rem // (K // kBN), rem % (K // kBN)
+    nt_n, nt_k = N // rows, K // kBN
+    seen = set()
+    for idx in range(E * nt_n * nt_k):
+        e = idx // (nt_n * nt_k)
+        rem = idx % (nt_n * nt_k)
+        # the dimension with fewer tiles varies fastest
+        tn, tk = (rem % nt_n, rem // nt_n) if nt_k >= nt_n else (rem // nt_k, rem % nt_k)
+        assert (e, tn, tk) not in seen and 0 <= tn < nt_n and 0 <= tk < nt_k
+        seen.add((e, tn, tk))
         s0, s1 = seg[e], seg[e + 1]
         for rank in ((0, 1) if pair else (0,)):
             a_y = tn * rows + rank * kBM
