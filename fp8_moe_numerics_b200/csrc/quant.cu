@@ -556,9 +556,9 @@ struct DispatchGradRows {
     }
 };
 
-template <int kLayout>
 // Three blocks per SM (78-80 registers, no spills): measured on B200 10% faster than two (the
 // gathers' latency is what bounds it) and than four (which spills).
+template <int kLayout>
 __global__ void __launch_bounds__(kTileThreads, 3)
 dispatch_grad_mxfp8_kernel(DispatchGradRows src, int64_t rows, int64_t cols, const int64_t* rows_valid,
                            uint8_t* __restrict__ row_codes, uint8_t* __restrict__ row_e8m0,
