@@ -853,56 +853,56 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                         ++nbox;
                         e8s[(n_stored & 1u) * (L::kE8Bytes / 2) + r * (kBN / 32) + (col[u] >> 5)] = (uint8_t)(e + 127);
                     }
-                    continue;
-                }
+                } else {
 #pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    uint8_t* box;
-                    if (kOut == kOutTypeBF16) {
-                        if (L::kOneBox) {
+                    for (int u = 0; u < 2; ++u) {
+                        uint8_t* box;
+                        if (kOut == kOutTypeBF16) {
+                            if (L::kOneBox) {
+                                box = stg;
+                                if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+                            } else {
+                                box = stg + (nbox & 1u) * 2048;
+                                if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+                            }
+                            __syncwarp();
+                            const uint32_t row = smem_u32(box) + (uint32_t)lane * 64u;
+#pragma unroll
+                            for (int c = 0; c < 4; ++c) {
+                                uint32_t w[4];
+#pragma unroll
+                                for (int i = 0; i < 4; ++i) {
+                                    __nv_bfloat162 bb = __floats2bfloat162_rn(v[u][8 * c + 2 * i] * scale,
+                                                                              v[u][8 * c + 2 * i + 1] * scale);
+                                    w[i] = *reinterpret_cast<uint32_t*>(&bb);
+                                }
+                                const uint32_t sw = (uint32_t)(c ^ ((lane >> 1) & 3));
+                                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                                             :: "r"(row + sw * 16u), "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]) : "memory");
+                            }
+                        } else {
                             box = stg;
                             if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-                        } else {
-                            box = stg + (nbox & 1u) * 2048;
-                            if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-                        }
-                        __syncwarp();
-                        const uint32_t row = smem_u32(box) + (uint32_t)lane * 64u;
+                            __syncwarp();
+                            const uint32_t row = smem_u32(box) + (uint32_t)lane * 128u;
 #pragma unroll
-                        for (int c = 0; c < 4; ++c) {
-                            uint32_t w[4];
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                __nv_bfloat162 bb = __floats2bfloat162_rn(v[u][8 * c + 2 * i] * scale,
-                                                                          v[u][8 * c + 2 * i + 1] * scale);
-                                w[i] = *reinterpret_cast<uint32_t*>(&bb);
+                            for (int c = 0; c < 8; ++c) {
+                                const uint32_t sw = (uint32_t)(c ^ (lane & 7));
+                                asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};"
+                                             :: "r"(row + sw * 16u), "f"(v[u][4 * c] * scale), "f"(v[u][4 * c + 1] * scale),
+                                                "f"(v[u][4 * c + 2] * scale), "f"(v[u][4 * c + 3] * scale) : "memory");
                             }
-                            const uint32_t sw = (uint32_t)(c ^ ((lane >> 1) & 3));
-                            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
-                                         :: "r"(row + sw * 16u), "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]) : "memory");
                         }
-                    } else {
-                        box = stg;
-                        if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+                        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                         __syncwarp();
-                        const uint32_t row = smem_u32(box) + (uint32_t)lane * 128u;
-#pragma unroll
-                        for (int c = 0; c < 8; ++c) {
-                            const uint32_t sw = (uint32_t)(c ^ (lane & 7));
-                            asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};"
-                                         :: "r"(row + sw * 16u), "f"(v[u][4 * c] * scale), "f"(v[u][4 * c + 1] * scale),
-                                            "f"(v[u][4 * c + 2] * scale), "f"(v[u][4 * c + 3] * scale) : "memory");
+                        if (lane == 0) {
+                            asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];"
+                                         :: "l"(reinterpret_cast<uint64_t>(&tmOut)), "r"((int)t.col0 + col[u]), "r"(oy),
+                                            "r"(smem_u32(box)) : "memory");
+                            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
                         }
+                        ++nbox;
                     }
-                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                    __syncwarp();
-                    if (lane == 0) {
-                        asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];"
-                                     :: "l"(reinterpret_cast<uint64_t>(&tmOut)), "r"((int)t.col0 + col[u]), "r"(oy),
-                                        "r"(smem_u32(box)) : "memory");
-                        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-                    }
-                    ++nbox;
                 }
             }
             if (kOut == kOutTypeS2F6) {

@@ -60,21 +60,21 @@ __device__ __forceinline__ uint32_t nvfp4_block(const uint4& a, const uint4& b, 
             mul2_rn(y[2 * i], y[2 * i + 1], inv2);
         }
         packed = e2m1_sr_codes<kR>(y, key.seed, key.stream, L0);
-        return sc;
-    }
-    uint32_t word[2];
+    } else {
+        uint32_t word[2];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {                      // eight products (in pairs), then their code word
-        float y[8];
+        for (int h = 0; h < 2; ++h) {                  // eight products (in pairs), then their code word
+            float y[8];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            y[2 * i] = bf16_lo(w[4 * h + i]);
-            y[2 * i + 1] = bf16_hi(w[4 * h + i]);
-            mul2_rn(y[2 * i], y[2 * i + 1], inv2);
+            for (int i = 0; i < 4; ++i) {
+                y[2 * i] = bf16_lo(w[4 * h + i]);
+                y[2 * i + 1] = bf16_hi(w[4 * h + i]);
+                mul2_rn(y[2 * i], y[2 * i + 1], inv2);
+            }
+            word[h] = cvt_e2m1x8(y);
         }
-        word[h] = cvt_e2m1x8(y);
+        packed = make_uint2(word[0], word[1]);
     }
-    packed = make_uint2(word[0], word[1]);
     return sc;
 }
 
@@ -516,8 +516,10 @@ mxfp8_tile_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, co
 // ---------------------------------------------------------------------------
 // MXFP8 (RNE) row and column forms of the dispatch gradient, formed on the fly
 // from the upstream gradient and the routing so that dY itself never goes
-// through HBM.  The tile walk and both forms are mxfp8_tile_kernel's; each
-// thread's row is gathered from its token's row of dout (the next tile's
+// through HBM.  The row form is mxfp8_tile_kernel's; the column form is the
+// TMA quantiser's (the tile as bf16 column pairs in two buffers, one barrier
+// per tile; measured on B200 5% faster than an fp32 tile with two barriers).
+// Each thread's row is gathered from its token's row of dout (the next tile's
 // loads issued before the current tile's transposed phase, their scaling at
 // the top of the next iteration).  Every value is w * dout rounded to bf16 by
 // the definition moe_dispatch_grad uses (scaled_bf16_word), so the codes equal
@@ -556,6 +558,13 @@ struct DispatchGradRows {
     }
 };
 
+// word (cp, r) of a transposed bf16 tile: columns 2cp, 2cp + 1 of row r (the TMA quantiser's layout)
+__device__ __forceinline__ int dq_t2_word(int cp, int r) {
+    int rr = r ^ ((cp >> 4) << 4);
+    rr ^= ((rr >> 5) & 3) << 2;
+    return cp * kTR + rr;
+}
+
 // Three blocks per SM (78-80 registers, no spills): measured on B200 10% faster than two (the
 // gathers' latency is what bounds it) and than four (which spills).
 template <int kLayout>
@@ -563,7 +572,7 @@ __global__ void __launch_bounds__(kTileThreads, 3)
 dispatch_grad_mxfp8_kernel(DispatchGradRows src, int64_t rows, int64_t cols, const int64_t* rows_valid,
                            uint8_t* __restrict__ row_codes, uint8_t* __restrict__ row_e8m0,
                            uint8_t* __restrict__ col_codes, uint8_t* __restrict__ col_e8m0) {
-    __shared__ __align__(16) float T[kTC * kTR];
+    __shared__ __align__(16) uint32_t T2d[2 * (kTC / 2) * kTR];      // double-buffered bf16 column pairs
     // Row tiles vary fastest: the blocks in flight gather the same 64-column
     // slice of dout for rows of every expert, so that slice of all tokens (T x
     // 128 B, a few MB) stays in L2 while each token's k routed rows read it.
@@ -576,6 +585,8 @@ dispatch_grad_mxfp8_kernel(DispatchGradRows src, int64_t rows, int64_t cols, con
     if (tile >= ntiles) return;
     const int t = threadIdx.x;
     const int rl = t >> 1, h = t & 1;
+    const int cp = t >> 3, g = t & 7;
+    int buf = 0;
     DispatchGradRows::Raw raw;
     auto issue = [&](int64_t tl) { src.issue((tl % tiles_r) * kTR + rl, (tl / tiles_r) * kTC + 32 * h, valid, raw); };
     issue(tile);
@@ -614,12 +625,52 @@ dispatch_grad_mxfp8_kernel(DispatchGradRows src, int64_t rows, int64_t cols, con
             if (mx_in_range(sf_offset(r, c >> 5, cols >> 5, kLayout), 1, rows * (cols >> 5)))
                 row_e8m0[sf_offset(r, c >> 5, cols >> 5, kLayout)] = (uint8_t)(e + 127);
         }
+        // column form: the tile as bf16 column pairs (the values are bf16 already), one barrier per
+        // tile with two buffers, then thread (cp, g) emits 16 rows of columns 2cp and 2cp + 1
+        uint32_t* Tb = T2d + buf * (kTC / 2) * kTR;
+        {
+            const uint32_t wq[16] = {q[0].x, q[0].y, q[0].z, q[0].w, q[1].x, q[1].y, q[1].z, q[1].w,
+                                     q[2].x, q[2].y, q[2].z, q[2].w, q[3].x, q[3].y, q[3].z, q[3].w};
 #pragma unroll
-        for (int i = 0; i < 32; ++i) T[tsw(32 * h + i, rl)] = v[i];
+            for (int j = 0; j < 16; ++j) Tb[dq_t2_word(16 * h + j, rl)] = wq[j];
+        }
         __syncthreads();
         if (tile + gridDim.x < ntiles) issue(tile + gridDim.x);
-        tile_emit_transposed<false, 8, kLayout>(T, rows, cols, r0, c0, 0, 0, col_codes, col_e8m0);
-        __syncthreads();                                   // T is rewritten by the next tile
+        uint32_t a[16];
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            const uint4 u = *reinterpret_cast<const uint4*>(Tb + dq_t2_word(cp, 16 * g + 4 * kk));
+            a[4 * kk] = u.x; a[4 * kk + 1] = u.y; a[4 * kk + 2] = u.z; a[4 * kk + 3] = u.w;
+        }
+        const int64_t rr = r0 + 16 * g;
+        const int64_t S = rows >> 5;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            float cv[16];
+#pragma unroll
+            for (int m = 0; m < 16; ++m) cv[m] = half ? bf16_hi(a[m]) : bf16_lo(a[m]);
+            float mf = 0.0f;
+#pragma unroll
+            for (int m = 0; m < 16; ++m) mf = fmaxf(mf, fabsf(cv[m]));
+            mf = fmaxf(mf, __shfl_xor_sync(0xffffffffu, mf, 1));
+            const int e = e8m0_exponent(mf);
+            const float sc = exp2_neg(e);
+            const uint64_t sc2 = f2_pack(sc, sc);
+            uint32_t w[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                float a0 = cv[4 * i], a1 = cv[4 * i + 1], a2 = cv[4 * i + 2], a3 = cv[4 * i + 3];
+                mul2_rn(a0, a1, sc2);
+                mul2_rn(a2, a3, sc2);
+                w[i] = cvt_e4m3x4(a0, a1, a2, a3);
+            }
+            const int64_t cg = c0 + 2 * cp + half;
+            if (mx_in_range(cg * rows + rr, 16, cols * rows))
+                *reinterpret_cast<uint4*>(col_codes + cg * rows + rr) = make_uint4(w[0], w[1], w[2], w[3]);
+            if ((g & 1) == 0 && mx_in_range(sf_offset(cg, rr >> 5, S, kLayout), 1, cols * S))
+                col_e8m0[sf_offset(cg, rr >> 5, S, kLayout)] = (uint8_t)(e + 127);
+        }
+        buf ^= 1;
     }
 }
 
