@@ -188,6 +188,10 @@ MX_API int mxfp8_quantize(const void* x, int64_t rows, int64_t cols, int roundin
  *   B: NVFP4 [E*N, K] (expert weight stack), sf MX_SF_MMA, outer per expert
  *   out: [M_cap, N] f32 or bf16 (out_dtype); rows >= seg_offsets[E] untouched
  * Requires K % 256 == 0, N % 128 == 0, M_cap % 128 == 0, 1 <= E.
+ * Enqueues one kernel on `stream`, or two when N % 256 == 0 and E <= 768: CTA
+ * pairs over 256-row tiles, then single CTAs for the experts' leftover
+ * 128-row tiles (the same holds for grouped_gemm_nvfp4_s2f6 and for
+ * grouped_gemm_mxfp8's DGRAD mode).
  * ------------------------------------------------------------------------ */
 MX_API int grouped_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_outer,
                        const uint8_t* b_codes, const uint8_t* b_sf, const float* b_outer,
