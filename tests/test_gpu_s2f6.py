@@ -64,7 +64,10 @@ def test_hadamard_s2f6_quantize_empty(cuda):
 
 @pytest.mark.parametrize("E,N,K,counts", [(4, 256, 256, [128, 0, 256, 300]), (3, 512, 512, [100, 300, 7]),
                                           (2, 384, 256, [130, 50]), (2, 256, 2048, [200, 70]),
-                                          (2, 4352, 256, [130, 50])])      # wider than the sign table
+                                          (2, 4352, 256, [130, 50]),       # wider than the sign table
+                                          # 1 or 3 row tiles per expert, 4 column tiles: 800 leftover tiles,
+                                          # enough for the tail kernel's S2F6 form on 148 SMs
+                                          (200, 1024, 256, [60 + 200 * (i % 2) for i in range(200)])])
 def test_grouped_gemm_nvfp4_s2f6_epilogue(cuda, E, N, K, counts):
     x, seg = routed_rows(counts, K, seed=E * 100 + N + K, nu=4)
     M_pad = int(seg[-1])
